@@ -1,0 +1,388 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix (no GPU).
+
+Each test pins the oracle to something other than its own formulas: a worked example
+printed on a page, a closed form, an invariant, a special case that reduces to a
+textbook routine, or brute force on tiny inputs.
+"""
+import itertools
+
+import numpy as np
+import pytest
+import scipy.linalg
+
+from oracle import gptq_oracle as O
+from post_weight_quantization_16_b200 import synth
+from tests.conftest import read_golden
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _bf16(a):
+    return synth.bf16_bits_to_f32(synth.f32_to_bf16_bits(np.asarray(a, dtype=np.float32)))
+
+
+def _spd(n, seed, cond_boost=0.0):
+    """A random symmetric positive definite matrix shaped like a calibration Hessian."""
+    r = _rng(seed)
+    X = _bf16(r.standard_normal((4 * n + 8, n)).astype(np.float32))
+    if cond_boost:
+        X[:, r.integers(0, n)] *= cond_boost
+    H = O.hessian(X)
+    return H
+
+
+# ----------------------------------------------------------------------------------
+# quantizer
+# ----------------------------------------------------------------------------------
+def test_worked_int8_example_codes_and_scale():
+    g = read_golden("sym_int8_worked_example.txt")
+    bits = int(g["bits"][0])
+    w = np.array([float(x) for x in g["w"]], dtype=np.float32)[None, :]
+    want = np.array([int(x) for x in g["codes"]])
+    r = O.rtn(w.astype(np.float64), bits, -1, True)
+    signed = r["codes"][0] - (1 << (bits - 1))
+    assert signed.tolist() == want.tolist()
+    s_want = np.float32(float(g["scale_numerator"][0])) / np.float32(int(g["scale_denominator"][0]))
+    assert r["scales"][0, 0] == s_want
+    # the same row through the GPTQ sweep with a diagonal H (no compensation) gives the same codes
+    sw = O.gptq_sweep(w.astype(np.float64), np.eye(5), bits, -1, True)
+    assert (sw["codes"][0] - 128).tolist() == want.tolist()
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_asym_grid_endpoints_and_roundtrip(bits):
+    r = _rng(bits)
+    w = r.normal(0, 0.02, size=(64, 128))
+    s, z, _ = O.group_params(w, bits, False)
+    qmax = (1 << bits) - 1
+    w32 = w.astype(np.float32)
+    lo = np.minimum(w32.min(1), 0)
+    hi = np.maximum(w32.max(1), 0)
+    u_lo, _, _ = O.quantize_values(lo, s, z, bits, False)
+    u_hi, _, _ = O.quantize_values(hi, s, z, bits, False)
+    assert (u_lo == 0).all()
+    assert (u_hi == qmax).all()
+    assert (z == np.rint(z)).all() and (z >= 0).all() and (z <= qmax).all()
+    for j in range(w.shape[1]):
+        u, _, wq = O.quantize_values(w[:, j], s, z, bits, False)
+        assert (u >= 0).all() and (u <= qmax).all()
+        # inside the range the round trip is within half a step (plus float32 slack)
+        assert (np.abs(w[:, j] - wq) <= 0.5 * s * (1 + 1e-5) + 1e-12).all()
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_sym_grid(bits):
+    r = _rng(10 + bits)
+    w = r.normal(0, 0.02, size=(32, 64))
+    s, z, _ = O.group_params(w, bits, True)
+    assert (z == (1 << (bits - 1))).all()
+    amax = np.abs(w.astype(np.float32)).max(1)
+    j = np.abs(w.astype(np.float32)).argmax(1)
+    u, _, wq = O.quantize_values(w[np.arange(32), j], s, z, bits, True)
+    # the largest-magnitude value lands on +-(2^(b-1)-1) and round-trips within float32 error
+    assert (np.abs(u - (1 << (bits - 1))) == (1 << (bits - 1)) - 1).all()
+    assert np.allclose(np.abs(wq), amax, rtol=1e-6)
+
+
+def test_zero_group_does_not_divide_by_zero():
+    w = np.zeros((3, 8))
+    for sym in (False, True):
+        r = O.rtn(w, 4, 8, sym)
+        assert np.all(r["what"] == 0)
+        assert np.all(r["scales"] == np.float32(1e-8))
+
+
+# ----------------------------------------------------------------------------------
+# Hessian
+# ----------------------------------------------------------------------------------
+def test_hessian_small_integer_case():
+    X = np.array([[1.0, 2.0], [3.0, 4.0]])
+    # x1 x1^T + x2 x2^T = [[1+9, 2+12], [2+12, 4+16]], times 2
+    assert O.hessian(X).tolist() == [[20.0, 28.0], [28.0, 40.0]]
+
+
+def test_hessian_equals_sum_of_token_outer_products():
+    r = _rng(1)
+    X = _bf16(r.standard_normal((37, 9)).astype(np.float32)).astype(np.float64)
+    acc = np.zeros((9, 9))
+    for t in range(X.shape[0]):
+        for a in range(9):
+            for b in range(9):
+                acc[a, b] += 2.0 * X[t, a] * X[t, b]
+    assert np.array_equal(O.hessian(X), acc)  # bf16 products and these short sums are exact
+
+
+def test_hessian_batches_accumulate():
+    r = _rng(2)
+    X = _bf16(r.standard_normal((100, 16)).astype(np.float32))
+    acc = O.HessianAccumulator(16)
+    for a, b in [(0, 13), (13, 64), (64, 100)]:
+        acc.add(X[a:b])
+    assert acc.n_tok == 100
+    assert np.allclose(acc.H, O.hessian(X), rtol=1e-14, atol=0)
+    assert np.allclose(acc.H, acc.H.T)
+    assert np.linalg.eigvalsh(acc.H).min() > -1e-9
+
+
+# ----------------------------------------------------------------------------------
+# prepare: U
+# ----------------------------------------------------------------------------------
+@pytest.mark.parametrize("n", [1, 5, 16, 130])
+def test_U_is_upper_cholesky_of_inverse(n):
+    H = _spd(n, n, cond_boost=20.0)
+    p = O.prepare(H, 0.01, False)
+    U = p["U"]
+    assert np.allclose(np.tril(U, -1), 0)
+    assert (np.diag(U) > 0).all()
+    # U^T U H = I
+    assert np.allclose(U.T @ U @ p["Hd"], np.eye(n), rtol=0, atol=1e-10)
+    # the textbook route: upper Cholesky factor of the explicit inverse
+    ref = scipy.linalg.cholesky(np.linalg.inv(p["Hd"]), lower=False)
+    assert np.allclose(U, ref, rtol=1e-10, atol=1e-14 * np.abs(ref).max())
+
+
+def test_damping_adds_relative_multiple_of_identity():
+    H = _spd(12, 3)
+    p = O.prepare(H, 0.1, False)
+    d = np.diag(H).mean()
+    assert np.allclose(p["Hd"] - H, 0.1 * d * np.eye(12), rtol=0, atol=1e-12 * d)
+
+
+def test_not_positive_definite_raises():
+    H = np.zeros((4, 4))
+    H[0, 0] = 1.0
+    H[0, 1] = H[1, 0] = 5.0
+    H[1, 1] = 1.0
+    H[2, 2] = H[3, 3] = 1.0
+    with pytest.raises(O.NotPositiveDefinite):
+        O.prepare(H, 0.0, False)
+
+
+def test_dead_columns_fixed_and_zeroed():
+    r = _rng(4)
+    X = _bf16(r.standard_normal((64, 16)).astype(np.float32))
+    X[:, [3, 11]] = 0
+    H = O.hessian(X)
+    W = r.normal(0, 0.02, (8, 16))
+    res = O.quantize_layer(W, H, 4, 8, False, 0.01, True, block=None)
+    assert res["dead"].tolist() == [i in (3, 11) for i in range(16)]
+    assert np.all(res["what_orig"][:, [3, 11]] == 0)
+
+
+# ----------------------------------------------------------------------------------
+# act-order
+# ----------------------------------------------------------------------------------
+def test_act_order_sorts_descending_and_is_stable():
+    H = np.diag([3.0, 7.0, 3.0, 9.0, 1.0, 7.0])
+    assert O.act_order(H).tolist() == [3, 1, 5, 0, 2, 4]
+
+
+@pytest.mark.parametrize("sym", [False, True])
+def test_diagonal_H_with_act_order_equals_rtn_in_permuted_groups(sym):
+    r = _rng(5)
+    n = 64
+    d = r.uniform(1, 10, n)
+    W = r.normal(0, 0.02, (16, n))
+    res = O.quantize_layer(W, np.diag(d), 4, 16, sym, 0.01, True, block=None)
+    perm = np.argsort(-d, kind="stable")
+    assert res["perm"].tolist() == perm.tolist()
+    ref = O.rtn(W[:, perm], 4, 16, sym)
+    assert np.array_equal(res["codes"], ref["codes"])
+    assert np.array_equal(res["scales"], ref["scales"])
+    assert np.array_equal(res["zeros"], ref["zeros"])
+    assert np.array_equal(res["what_orig"], O.unpermute_columns(ref["what"], perm))
+
+
+# ----------------------------------------------------------------------------------
+# sweep
+# ----------------------------------------------------------------------------------
+@pytest.mark.parametrize("sym", [False, True])
+@pytest.mark.parametrize("g", [8, 32, -1])
+def test_diagonal_H_collapses_to_rtn(sym, g):
+    r = _rng(6)
+    W = r.normal(0, 0.02, (24, 32))
+    U = np.diag(1.0 / np.sqrt(r.uniform(0.5, 3.0, 32)))  # diagonal H => diagonal U
+    sw = O.gptq_sweep(W, U, 4, g, sym)
+    ref = O.rtn(W, 4, g, sym)
+    for k in ("codes", "scales", "zeros", "what"):
+        assert np.array_equal(sw[k], ref[k]), k
+
+
+def _obs_sweep(W, Hd, bits, g, sym):
+    """Sequential OBS form: full inverse, error scaled by its diagonal, then the inverse
+    is downdated to remove the quantized column (independent of the Cholesky-row form)."""
+    W = np.array(W, dtype=np.float64)
+    m, n = W.shape
+    g = n if g == -1 else g
+    Hinv = np.linalg.inv(Hd)
+    codes = np.zeros((m, n), dtype=np.int64)
+    what = np.zeros((m, n))
+    for q in range(n):
+        if q % g == 0:
+            s, z, _ = O.group_params(W[:, q:q + g], bits, sym)
+        u, _, wq = O.quantize_values(W[:, q], s, z, bits, sym)
+        codes[:, q], what[:, q] = u, wq
+        err = (W[:, q] - wq) / Hinv[q, q]
+        W[:, q + 1:] -= np.outer(err, Hinv[q, q + 1:])
+        Hinv = Hinv - np.outer(Hinv[:, q], Hinv[q, :]) / Hinv[q, q]
+    return codes, what
+
+
+@pytest.mark.parametrize("n,g,sym,bits", [(8, 4, False, 4), (16, 8, True, 3), (12, -1, False, 2), (16, 16, False, 4)])
+def test_obs_sequential_equals_cholesky_row_form(n, g, sym, bits):
+    for seed in range(5):
+        H = _spd(n, 100 + seed, cond_boost=10.0)
+        p = O.prepare(H, 0.01, False)
+        W = _rng(seed).normal(0, 0.02, (20, n))
+        sw = O.gptq_sweep(W, p["U"], bits, g, sym)
+        codes, what = _obs_sweep(W, p["Hd"], bits, g, sym)
+        assert np.array_equal(sw["codes"], codes)
+        assert np.allclose(sw["what"], what, rtol=1e-12, atol=1e-15)
+
+
+@pytest.mark.parametrize("n,B,g", [(256, 128, 128), (256, 128, 64), (512, 128, 256), (200, 64, -1), (96, 32, 32)])
+def test_blocked_equals_unblocked(n, B, g):
+    H = _spd(n, 7, cond_boost=15.0)
+    p = O.prepare(H, 0.01, True)
+    W = _rng(8).normal(0, 0.02, (16, n))
+    Wp = W[:, p["perm"]]
+    a = O.gptq_sweep(Wp, p["U"], 4, g, False)
+    b = O.gptq_sweep(Wp, p["U"], 4, g, False, block=B)
+    assert np.array_equal(a["codes"], b["codes"])
+    assert np.allclose(a["scales"], b["scales"], rtol=1e-6, atol=0)
+    assert np.allclose(a["what"], b["what"], rtol=1e-12, atol=1e-14)
+
+
+def test_brute_force_optimum_and_gptq_beats_rtn_on_average():
+    bits, n = 4, 4
+    e_gptq, e_rtn = [], []
+    grid = np.array(list(itertools.product(range(16), repeat=n)))  # 65536 code vectors
+    for seed in range(200):
+        r = _rng(1000 + seed)
+        A = r.standard_normal((n, n))
+        H = A @ A.T + 0.05 * np.eye(n) + 0.5 * np.ones((n, n))   # correlated columns
+        w = r.normal(0, 0.02, (1, n))
+        U = O.upper_cholesky_of_inverse(H)
+        sw = O.gptq_sweep(w, U, bits, -1, False)       # per-channel: one static (s, z)
+        s = np.float64(sw["scales"][0, 0])
+        z = np.float64(sw["zeros"][0, 0])
+        d_opt = w - (grid - z) * s
+        opt = np.einsum("ij,jk,ik->i", d_opt, H, d_opt).min()
+        d = w - sw["what"]
+        eg = float((d @ H @ d.T)[0, 0])
+        rt = O.rtn(w, bits, -1, False)
+        dr = w - rt["what"]
+        er = float((dr @ H @ dr.T)[0, 0])
+        assert rt["scales"][0, 0] == sw["scales"][0, 0]
+        assert eg >= opt * (1 - 1e-12)
+        e_gptq.append(eg)
+        e_rtn.append(er)
+    assert np.mean(e_gptq) < np.mean(e_rtn)
+
+
+def test_last_column_keeps_its_own_error():
+    n = 24
+    H = _spd(n, 9, cond_boost=5.0)
+    p = O.prepare(H, 0.01, False)
+    W = _rng(10).normal(0, 0.02, (10, n))
+    sw = O.gptq_sweep(W, p["U"], 4, 8, False)
+    U = p["U"]
+    # the value the last column is quantized from is the original minus every earlier compensation
+    w_last = W[:, -1] - sw["err"][:, :-1] @ U[:-1, -1]
+    s, z = sw["scales"][:, -1], sw["zeros"][:, -1]
+    u, _, wq = O.quantize_values(w_last, s, z, 4, False)
+    assert np.array_equal(u, sw["codes"][:, -1])
+    assert np.allclose(sw["err"][:, -1], (w_last - wq) / U[-1, -1], rtol=1e-12)
+    # and nothing depends on it: changing the last column of W leaves earlier columns alone
+    W2 = W.copy()
+    W2[:, -1] += 0.05
+    sw2 = O.gptq_sweep(W2, p["U"], 4, 8, False)
+    assert np.array_equal(sw2["codes"][:, :16], sw["codes"][:, :16])
+
+
+def test_gptq_layer_error_below_rtn_on_outlier_layer():
+    layer = synth.scaled_layer(synth.WORKLOADS["tiny_256x512"][0], m=64, n=256, n_tok=1024)
+    X = synth.bf16_bits_to_f32(synth.make_x_bf16(layer))
+    W = synth.make_w_fp16(layer).astype(np.float64)
+    H = O.hessian(X)
+    res = O.quantize_layer(W, H, 4, 128, False, 0.01, True)
+    e_gptq = O.layer_error(W, res["what_orig"], H)
+    e_rtn = O.layer_error(W, O.rtn(W, 4, 128, False)["what"], H)
+    assert e_gptq < 0.8 * e_rtn
+
+
+# ----------------------------------------------------------------------------------
+# metrics and outputs
+# ----------------------------------------------------------------------------------
+def test_layer_error_identity_matches_direct_product():
+    r = _rng(11)
+    X = _bf16(r.standard_normal((300, 32)).astype(np.float32)).astype(np.float64)
+    W = r.normal(0, 0.02, (8, 32))
+    What = W + r.normal(0, 0.001, W.shape)
+    direct = np.sum(((W - What) @ X.T) ** 2) / np.sum((W @ X.T) ** 2)
+    assert np.isclose(O.layer_error(W, What, O.hessian(X)), direct, rtol=1e-12)
+
+
+def test_pack_known_words():
+    c = np.array([[1, 2, 3, 4, 5, 6, 7, 8]])
+    assert O.pack_codes(c, 4).tolist() == [[0x87654321]]
+    c2 = np.array([[3, 0, 1, 2] * 4])
+    assert O.pack_codes(c2, 2).tolist() == [[int("10010011" * 4, 2)]]
+    c3 = np.zeros((1, 32), dtype=np.int64)
+    c3[0, 10] = 7          # stream bits 30..32 straddle words 0 and 1
+    assert O.pack_codes(c3, 3).tolist() == [[0xC0000000, 0x1, 0x0]]
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_pack_roundtrip(bits):
+    r = _rng(bits)
+    c = r.integers(0, 1 << bits, (7, 96))
+    assert np.array_equal(O.unpack_codes(O.pack_codes(c, bits), 96, bits), c)
+
+
+def test_g_idx_definition():
+    perm = np.array([2, 0, 3, 1])
+    assert O.g_idx(perm, 2).tolist() == [0, 1, 0, 1]
+
+
+# ----------------------------------------------------------------------------------
+# the parity checker itself (mistakes planted in the oracle's output, on the CPU)
+# ----------------------------------------------------------------------------------
+def test_replay_adopts_in_band_flip_and_flags_out_of_band_flip():
+    n = 64
+    H = _spd(n, 12, cond_boost=5.0)
+    p = O.prepare(H, 0.01, False)
+    W = _rng(13).normal(0, 0.02, (32, n))
+    ref = O.gptq_sweep(W, p["U"], 4, 32, False)
+    dist = O.boundary_distance(ref["pre"], 4, False)
+    # make one column-0 value sit in the band by nudging W there, then plant a flip
+    i = 5
+    codes = ref["codes"].copy()
+    st = O.ReplayStats()
+    O.gptq_sweep(W, p["U"], 4, 32, False, ref_codes=codes, ref_zeros=ref["zeros"], stats=st)
+    assert st.hard_mismatch == 0 and st.adopted == 0 and st.identical == st.total
+    r, c = np.unravel_index(np.argmax(dist > 0.2), dist.shape)
+    codes[r, c] += 1 if codes[r, c] < 15 else -1
+    st = O.ReplayStats()
+    O.gptq_sweep(W, p["U"], 4, 32, False, ref_codes=codes, ref_zeros=ref["zeros"], stats=st)
+    assert st.hard_mismatch >= 1
+    # an in-band flip is adopted: build one at a tiny distance from a boundary
+    W2 = W.copy()
+    s, z = ref["scales"][i, 0], ref["zeros"][i, 0]
+    W2[i, 0] = (np.floor(ref["pre"][i, 0]) + 0.5 - z + 1e-4) * np.float64(s)
+    ref2 = O.gptq_sweep(W2, p["U"], 4, 32, False)
+    assert O.boundary_distance(ref2["pre"][i, 0], 4, False) < 1e-3
+    codes2 = ref2["codes"].copy()
+    codes2[i, 0] -= 1
+    # a reference that took the other side of that one in-band decision and carried on
+    # consistently from there (this is what a correct kernel with a slightly different
+    # rounding of that value produces)
+    planted = O.gptq_sweep(W2, p["U"], 4, 32, False, ref_codes=codes2, ref_zeros=ref2["zeros"])
+    assert planted["codes"][i, 0] == codes2[i, 0]
+    st = O.ReplayStats()
+    out = O.gptq_sweep(W2, p["U"], 4, 32, False, ref_codes=planted["codes"], ref_zeros=planted["zeros"], stats=st)
+    assert st.adopted == 1 and st.hard_mismatch == 0
+    assert st.identical == st.total - 1
+    assert np.array_equal(out["codes"], planted["codes"])
