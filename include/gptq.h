@@ -1,0 +1,156 @@
+/*
+ * gptq.h — C ABI of the B200 (sm_100a) GPTQ per-layer quantization solve.
+ *
+ * The method (quantize one linear layer W [m x n] from calibration activations X [N x n]):
+ *   S1  H += 2 X^T X over calibration batches
+ *       ("模型量化实战：从 INT8 PTQ 到 GPTQ 的精度保持与推理加速全解析", §3.2, accumulate_hessian)
+ *   S2  dead columns (diag H == 0): H_ii = 1 and the weight column is zeroed;
+ *       damping H += damp * mean(diag H) * I  (same page, §3.2 prepare)
+ *   S3  act-order (desc_act): columns sorted by descending diag H
+ *       ("GPTQ量化损失深度解析：原理、影响与优化策略", 减少量化损失的实战策略)
+ *   S4  U = upper Cholesky factor of H^-1 (H^-1 = U^T U)   (§3.2 prepare)
+ *   S5  column sweep in blocks of 128: per-group min-max scale/zero, b-bit code,
+ *       e = (w - q) / U[i,i], W[:, j>i] -= e * U[i, j]
+ *       ("大模型量化：GPTQ/AWQ/GGUF 原理对比，4-bit 量化对推理精度的影响", GPTQ section)
+ *   S6  the later columns of W are updated once per 128-column block by one product
+ *   S7  codes packed per row, scales, zeros, perm and g_idx
+ *
+ * Conventions (all calls):
+ *   - Every tensor pointer is CALLER-OWNED DEVICE memory on the context's device unless the
+ *     argument says otherwise; the context owns only its workspace.
+ *   - All matrices are row-major with the leading dimension stated.
+ *   - Calls are enqueued on the context's CUDA stream and return after launching, except
+ *     gptq_prepare and gptq_synchronize, which wait (with a bounded host wait) for the stream.
+ *   - Arguments are validated on the host before anything is launched; a call that returns
+ *     an error other than GPTQ_ERR_CUDA / GPTQ_ERR_TIMEOUT has enqueued nothing.
+ *   - Device-side failures (a non-positive pivot, a kernel wait that ran out) are recorded
+ *     in a device status word and returned by the next gptq_prepare / gptq_synchronize.
+ *   - There is no CPU fallback: without a CUDA device every compute call fails with
+ *     GPTQ_ERR_CUDA.
+ */
+#ifndef GPTQ_B200_H
+#define GPTQ_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct gptq_ctx gptq_ctx; /* opaque: device H, factor, permutation and workspace */
+
+typedef enum {
+  GPTQ_OK = 0,
+  GPTQ_ERR_ARG = 1,         /* invalid argument (null pointer, size, alignment, range) */
+  GPTQ_ERR_STATE = 2,       /* call not allowed in the context's current state */
+  GPTQ_ERR_NOT_PD = 3,      /* damped Hessian not positive definite (non-positive pivot) */
+  GPTQ_ERR_OOM = 4,         /* workspace does not fit (checked before allocating) */
+  GPTQ_ERR_CUDA = 5,        /* a CUDA runtime/driver call failed (no device, launch error...) */
+  GPTQ_ERR_TIMEOUT = 6,     /* a bounded device or host wait ran out */
+  GPTQ_ERR_UNSUPPORTED = 7  /* valid request that this build does not implement */
+} gptq_status;
+
+/* Quantizer settings ("GPTQ算法原理深度解析" §3.3 quantize_config: bits, group_size; sym from
+ * "GPTQ量化损失深度解析" 调整量化参数).
+ *   bits       : 2, 3, 4 or 8.
+ *   group_size : columns per scale/zero group, in sweep order; -1 = one group per row
+ *                (per-channel).  Must divide n and either divide 128 or be a multiple of
+ *                128; at least 32.
+ *   sym        : 0 = asymmetric min-max (range widened to include 0; zero-point integer in
+ *                [0, 2^b-1]); 1 = symmetric (scale = max|w| / (2^(b-1)-1), signed codes stored
+ *                offset by 2^(b-1), zero = 2^(b-1)).
+ * Dequantization is always (code - zero) * scale. */
+typedef struct {
+  int bits;
+  int group_size;
+  int sym;
+} gptq_qparams;
+
+/* Device bytes a context for n_in input features and at most m_max output rows allocates
+ * (H, damped H, V, U, the inverse temporary, the fp32 working copy of W and small buffers).
+ * Returns 0 for sizes that gptq_create rejects.  Pure host function. */
+size_t gptq_workspace_bytes(int64_t n_in, int64_t m_max);
+
+/* Create a context for layers with n_in input features (n_in % 128 == 0, 128 <= n_in <= 32768)
+ * and up to m_max output rows (1 <= m_max <= 2^24).  `device` is the CUDA ordinal;
+ * `cuda_stream` is a cudaStream_t (NULL = legacy default stream) that every later call of
+ * this context is enqueued on.  Allocates the whole workspace up front: returns GPTQ_ERR_OOM
+ * without allocating when gptq_workspace_bytes() exceeds the device's free memory or the
+ * limit in the environment variable GPTQ_MAX_WORKSPACE_BYTES.  H starts at zero.
+ * On success *out owns the workspace until gptq_destroy. */
+gptq_status gptq_create(gptq_ctx** out, int64_t n_in, int64_t m_max, int device, void* cuda_stream);
+
+/* S1: H += 2 X^T X for one calibration batch and n_tok += batch size (asynchronous).
+ *   X_bf16 : device, bf16, [n_tok x n_in] row-major with leading dimension ld_x elements
+ *            (ld_x >= n_in, ld_x % 8 == 0, 16-byte aligned base).
+ *   n_tok  : tokens in this batch, 0 <= n_tok < 2^31 (0 is a no-op).
+ * Runs the tcgen05 BF16 x BF16 -> FP32 accumulator.  GPTQ_ERR_STATE after gptq_prepare
+ * until gptq_reset. */
+gptq_status gptq_hessian_accumulate(gptq_ctx* ctx, const void* X_bf16, int64_t n_tok, int64_t ld_x);
+
+/* Copy the accumulated H (full symmetric, fp32, [n x n], leading dimension n) to the device
+ * buffer H_out and the token count to the HOST int64 *n_tok_out (either may be NULL).
+ * Waits for the context's stream. */
+gptq_status gptq_get_hessian(gptq_ctx* ctx, float* H_out, int64_t* n_tok_out);
+
+/* Replace H by a caller-provided symmetric fp32 [n x n] device matrix (leading dimension n)
+ * and set the token count (resumes a saved calibration).  Only the upper triangle is read.
+ * GPTQ_ERR_STATE after gptq_prepare until gptq_reset. */
+gptq_status gptq_set_hessian(gptq_ctx* ctx, const float* H_in, int64_t n_tok);
+
+/* S2-S4 (synchronizes once): dead-column fix, optional act-order permutation, damping by
+ * damp * mean(diag H) (0 <= damp <= 1e6), then U = upper-Cholesky(H_perm^-1) by a blocked
+ * reverse Cholesky H_perm = V V^T and U = V^-1.
+ *   desc_act : 0 = identity order; 1 = stable descending diag H (after the dead fix).
+ *   perm_out : device int32 [n] or NULL; perm_out[k] = original column swept at position k.
+ * Returns GPTQ_ERR_NOT_PD when a pivot is not positive (the context stays unprepared).
+ * H itself is left unchanged, so prepare may be repeated with another damp. */
+gptq_status gptq_prepare(gptq_ctx* ctx, double damp, int desc_act, int32_t* perm_out);
+
+/* Copy the factor U (fp32 [n x n], sweep order, zeros below the diagonal) to the device
+ * buffer U_out.  GPTQ_ERR_STATE before gptq_prepare.  Asynchronous. */
+gptq_status gptq_get_factor(gptq_ctx* ctx, float* U_out);
+
+/* S5-S7 (asynchronous): quantize W with the prepared factor.
+ *   W_fp16     : device fp16 [m x n] row-major (ld n), ORIGINAL column order, 1 <= m <= m_max.
+ *   codes_out  : device uint32 [m x n*bits/32]; row r holds its codes in SWEEP order as an
+ *                LSB-first bit stream (code k in stream bits k*bits .. k*bits+bits-1, stream bit
+ *                p = bit p%32 of word p/32).
+ *   scales_out : device fp32 [m x G], G = n / group_size (1 for per-channel), groups in sweep
+ *                order.
+ *   zeros_out  : device fp32 [m x G], integer-valued.
+ *   g_idx_out  : device int32 [n] or NULL; g_idx[perm[k]] = k / group_size.
+ *   W_hat_out  : device fp32 [m x n] or NULL; dequantized weights in ORIGINAL column order.
+ * GPTQ_ERR_STATE before gptq_prepare. */
+gptq_status gptq_quantize_layer(gptq_ctx* ctx, const void* W_fp16, int64_t m, gptq_qparams qp,
+                                uint32_t* codes_out, float* scales_out, float* zeros_out,
+                                int32_t* g_idx_out, float* W_hat_out);
+
+/* Wait (bounded by GPTQ_SYNC_TIMEOUT_MS, default 600000) for the context's stream and return
+ * the first recorded device-side failure, if any. */
+gptq_status gptq_synchronize(gptq_ctx* ctx);
+
+/* Zero H and the token count and return to the accumulate state (asynchronous). */
+gptq_status gptq_reset(gptq_ctx* ctx);
+
+/* Free the workspace (waits for the stream).  NULL is accepted. */
+gptq_status gptq_destroy(gptq_ctx* ctx);
+
+/* Number of kernels this context has launched since gptq_create (instrumentation; -1 for
+ * NULL).  Pure host function. */
+int64_t gptq_launch_count(const gptq_ctx* ctx);
+
+/* Static description of a status code. */
+const char* gptq_status_string(gptq_status s);
+
+/* Tokens per tensor-memory accumulation chunk of S1 (a multiple of 64).  Each chunk is
+ * summed on the tensor cores, then added to H in fp32 by the CUDA cores, which bounds the
+ * accumulation error of long calibration sets.  Default 4096. */
+gptq_status gptq_set_hessian_chunk(gptq_ctx* ctx, int64_t tokens);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GPTQ_B200_H */

@@ -1,0 +1,527 @@
+// gptq_api.cu — the C ABI declared in include/gptq.h: context, argument checks and the
+// launch sequence of the sm_100a kernels on the context's stream.
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <chrono>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <thread>
+
+#include "../../include/gptq.h"
+#include "factor_kernels.cuh"
+#include "hessian_tc.cuh"
+#include "prepare_kernels.cuh"
+#include "sgemm_simt.cuh"
+#include "sweep_kernels.cuh"
+
+using namespace gptq;
+
+namespace {
+
+enum CtxState { ST_ACCUM = 0, ST_PREPARED = 1 };
+
+constexpr int64_t kMaxN = 32768;
+constexpr int64_t kMaxM = int64_t(1) << 24;
+
+}  // namespace
+
+struct gptq_ctx {
+  int device = 0;
+  cudaStream_t stream = nullptr;
+  int64_t n = 0, m_max = 0;
+  float* H = nullptr;    // [n x n] accumulated Hessian (upper triangle valid until mirrored)
+  float* A = nullptr;    // [n x n] damped, permuted H (consumed by the factorization)
+  float* V = nullptr;    // [n x n] reverse Cholesky factor
+  float* U = nullptr;    // [n x n] U = V^-1
+  float* T = nullptr;    // [n/2 x n/2 + slack] temporary of the inverse recursion
+  float* Wq = nullptr;   // [m_max x n] fp32 working weights
+  float* Err = nullptr;  // [m_max x 128]
+  float* keys = nullptr;
+  uint8_t* dead = nullptr;
+  int32_t* perm = nullptr;
+  double* mean = nullptr;
+  int* status = nullptr;      // device status word
+  int* status_host = nullptr; // pinned mirror
+  int64_t n_tok = 0;
+  int state = ST_ACCUM;
+  int mirrored = 0;           // H's lower triangle has been filled
+  int64_t chunk_tokens = 4096;
+  int64_t launches = 0;       // kernels launched by this context (instrumentation)
+  PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+};
+
+namespace {
+
+gptq_status cuda_fail(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return GPTQ_OK;
+  if (std::getenv("GPTQ_VERBOSE")) std::fprintf(stderr, "gptq: %s: %s\n", what, cudaGetErrorString(e));
+  return GPTQ_ERR_CUDA;
+}
+#define CK(call)                                         \
+  do {                                                   \
+    gptq_status _s = cuda_fail((call), #call);           \
+    if (_s != GPTQ_OK) return _s;                        \
+  } while (0)
+#define CKL(what) CK(cudaGetLastError())
+
+size_t t_elems(int64_t n) { return static_cast<size_t>((n / 2 + FB_NB) * (n / 2 + FB_NB)); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+class DeviceGuard {
+ public:
+  explicit DeviceGuard(int dev) {
+    cudaGetDevice(&prev_);
+    cudaSetDevice(dev);
+  }
+  ~DeviceGuard() { cudaSetDevice(prev_); }
+
+ private:
+  int prev_ = 0;
+};
+
+int64_t env_int(const char* name, int64_t dflt) {
+  const char* v = std::getenv(name);
+  if (!v || !*v) return dflt;
+  return std::strtoll(v, nullptr, 10);
+}
+
+// Bounded host wait for everything enqueued so far on the context's stream.
+gptq_status wait_stream(gptq_ctx* c) {
+  cudaEvent_t ev;
+  CK(cudaEventCreateWithFlags(&ev, cudaEventDisableTiming));
+  cudaError_t e = cudaEventRecord(ev, c->stream);
+  if (e != cudaSuccess) {
+    cudaEventDestroy(ev);
+    return cuda_fail(e, "cudaEventRecord");
+  }
+  const int64_t limit_ms = env_int("GPTQ_SYNC_TIMEOUT_MS", 600000);
+  const auto t0 = std::chrono::steady_clock::now();
+  gptq_status st = GPTQ_OK;
+  for (;;) {
+    e = cudaEventQuery(ev);
+    if (e == cudaSuccess) break;
+    if (e != cudaErrorNotReady) {
+      st = cuda_fail(e, "cudaEventQuery");
+      break;
+    }
+    const auto ms =
+        std::chrono::duration_cast<std::chrono::milliseconds>(std::chrono::steady_clock::now() - t0).count();
+    if (ms > limit_ms) {
+      st = GPTQ_ERR_TIMEOUT;
+      break;
+    }
+    std::this_thread::sleep_for(std::chrono::microseconds(50));
+  }
+  cudaEventDestroy(ev);
+  return st;
+}
+
+// Read (and clear) the device status word; waits for the stream.
+gptq_status read_status(gptq_ctx* c, int* flags) {
+  CK(cudaMemcpyAsync(c->status_host, c->status, sizeof(int), cudaMemcpyDeviceToHost, c->stream));
+  gptq_status st = wait_stream(c);
+  if (st != GPTQ_OK) return st;
+  *flags = *c->status_host;
+  if (*flags) CK(cudaMemsetAsync(c->status, 0, sizeof(int), c->stream));
+  return GPTQ_OK;
+}
+
+gptq_status status_from_flags(int f) {
+  if (f & ST_TIMEOUT) return GPTQ_ERR_TIMEOUT;
+  if (f & ST_NOT_PD) return GPTQ_ERR_NOT_PD;
+  if (f & ST_INTERNAL) return GPTQ_ERR_CUDA;
+  return GPTQ_OK;
+}
+
+gptq_status sgemm(gptq_ctx* c, bool transB, int M, int N, int K, float alpha, const float* A, int lda,
+                  const float* B, int ldb, float beta, float* C, int ldc, bool upper_only) {
+  if (M <= 0 || N <= 0) return GPTQ_OK;
+  if (K % SG_BK || N % 4 || lda % 4 || ldb % 4 || ldc % 4 || !aligned16(A) || !aligned16(B) || !aligned16(C))
+    return GPTQ_ERR_ARG;
+  if (K == 0) return GPTQ_OK;
+  dim3 grid((N + SG_BN - 1) / SG_BN, (M + SG_BM - 1) / SG_BM);
+  cudaStream_t st = c->stream;
+  ++c->launches;
+  if (transB)
+    sgemm_kernel<true><<<grid, SG_THREADS, 0, st>>>(M, N, K, alpha, A, lda, B, ldb, beta, C, ldc, upper_only ? 1 : 0);
+  else
+    sgemm_kernel<false><<<grid, SG_THREADS, 0, st>>>(M, N, K, alpha, A, lda, B, ldb, beta, C, ldc, upper_only ? 1 : 0);
+  CKL("sgemm");
+  return GPTQ_OK;
+}
+
+// [V,U] of the diagonal block [o, o+h) of A (h a multiple of FB_NB).
+gptq_status chol_inv(gptq_ctx* c, int o, int h) {
+  const int n = static_cast<int>(c->n);
+  if (h <= FB_NB) {
+    chol_inv_base_kernel<<<1, FB_THREADS, 0, c->stream>>>(c->A, c->V, c->U, n, o, c->status);
+    ++c->launches;
+    CKL("chol_inv_base");
+    return GPTQ_OK;
+  }
+  const int h2 = ((h / FB_NB) / 2) * FB_NB;
+  const int h1 = h - h2;
+  const int o2 = o + h1;
+  gptq_status s;
+  auto at = [n](float* M, int r, int col) { return M + static_cast<size_t>(r) * n + col; };
+  if ((s = chol_inv(c, o2, h2)) != GPTQ_OK) return s;
+  // V12 = A12 U22^T
+  if ((s = sgemm(c, true, h1, h2, h2, 1.f, at(c->A, o, o2), n, at(c->U, o2, o2), n, 0.f, at(c->V, o, o2), n,
+                 false)) != GPTQ_OK)
+    return s;
+  // A11 -= V12 V12^T (upper tiles)
+  if ((s = sgemm(c, true, h1, h1, h2, -1.f, at(c->V, o, o2), n, at(c->V, o, o2), n, 1.f, at(c->A, o, o), n,
+                 true)) != GPTQ_OK)
+    return s;
+  if ((s = chol_inv(c, o, h1)) != GPTQ_OK) return s;
+  // T = V12 U22 ; U12 = -U11 T
+  if ((s = sgemm(c, false, h1, h2, h2, 1.f, at(c->V, o, o2), n, at(c->U, o2, o2), n, 0.f, c->T, h2, false)) !=
+      GPTQ_OK)
+    return s;
+  if ((s = sgemm(c, false, h1, h2, h1, -1.f, at(c->U, o, o), n, c->T, h2, 0.f, at(c->U, o, o2), n, false)) !=
+      GPTQ_OK)
+    return s;
+  return GPTQ_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+}
+
+void free_all(gptq_ctx* c) {
+  float** fs[] = {&c->H, &c->A, &c->V, &c->U, &c->T, &c->Wq, &c->Err, &c->keys};
+  for (float** p : fs)
+    if (*p) {
+      cudaFree(*p);
+      *p = nullptr;
+    }
+  if (c->dead) cudaFree(c->dead);
+  if (c->perm) cudaFree(c->perm);
+  if (c->mean) cudaFree(c->mean);
+  if (c->status) cudaFree(c->status);
+  if (c->status_host) cudaFreeHost(c->status_host);
+  c->dead = nullptr;
+  c->perm = nullptr;
+  c->mean = nullptr;
+  c->status = nullptr;
+  c->status_host = nullptr;
+}
+
+bool valid_qparams(const gptq_qparams& qp, int64_t n) {
+  if (!(qp.bits == 2 || qp.bits == 3 || qp.bits == 4 || qp.bits == 8)) return false;
+  if (!(qp.sym == 0 || qp.sym == 1)) return false;
+  const int64_t g = (qp.group_size == -1) ? n : qp.group_size;
+  if (g < 32 || g > n || n % g) return false;
+  if (!(g % SW_B == 0 || SW_B % g == 0)) return false;
+  return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* gptq_status_string(gptq_status s) {
+  switch (s) {
+    case GPTQ_OK: return "ok";
+    case GPTQ_ERR_ARG: return "invalid argument";
+    case GPTQ_ERR_STATE: return "call not allowed in the current state";
+    case GPTQ_ERR_NOT_PD: return "damped Hessian is not positive definite";
+    case GPTQ_ERR_OOM: return "workspace does not fit in device memory";
+    case GPTQ_ERR_CUDA: return "CUDA error";
+    case GPTQ_ERR_TIMEOUT: return "bounded wait timed out";
+    case GPTQ_ERR_UNSUPPORTED: return "unsupported request";
+  }
+  return "unknown status";
+}
+
+size_t gptq_workspace_bytes(int64_t n, int64_t m_max) {
+  if (n < 128 || n > kMaxN || n % 128 || m_max < 1 || m_max > kMaxM) return 0;
+  const size_t nn = static_cast<size_t>(n) * static_cast<size_t>(n);
+  size_t b = 4 * nn * sizeof(float);                                  // H, A, V, U
+  b += t_elems(n) * sizeof(float);                                    // T
+  b += static_cast<size_t>(m_max) * static_cast<size_t>(n) * sizeof(float);   // Wq
+  b += static_cast<size_t>(m_max) * SW_B * sizeof(float);             // Err
+  b += static_cast<size_t>(n) * (sizeof(float) + 1 + sizeof(int32_t)) + sizeof(double) + sizeof(int);
+  return b;
+}
+
+gptq_status gptq_create(gptq_ctx** out, int64_t n, int64_t m_max, int device, void* stream) {
+  if (!out) return GPTQ_ERR_ARG;
+  *out = nullptr;
+  const size_t need = gptq_workspace_bytes(n, m_max);
+  if (need == 0 || device < 0) return GPTQ_ERR_ARG;
+  const int64_t env_limit = env_int("GPTQ_MAX_WORKSPACE_BYTES", -1);
+  if (env_limit >= 0 && static_cast<int64_t>(need) > env_limit) return GPTQ_ERR_OOM;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || device >= ndev) {
+    cudaGetLastError();
+    return GPTQ_ERR_CUDA;
+  }
+  DeviceGuard dg(device);
+  size_t free_b = 0, total_b = 0;
+  CK(cudaMemGetInfo(&free_b, &total_b));
+  if (need > free_b) return GPTQ_ERR_OOM;
+  int major = 0, minor = 0;
+  CK(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device));
+  CK(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, device));
+  if (major != 10 || minor != 0) return GPTQ_ERR_UNSUPPORTED;  // built for sm_100a only
+
+  gptq_ctx* c = new gptq_ctx();
+  c->device = device;
+  c->stream = static_cast<cudaStream_t>(stream);
+  c->n = n;
+  c->m_max = m_max;
+  c->chunk_tokens = 4096;
+  c->encode = get_encode();
+  const size_t nn = static_cast<size_t>(n) * n;
+  cudaError_t e = cudaSuccess;
+  auto alloc = [&](void** p, size_t bytes) {
+    if (e == cudaSuccess) e = cudaMalloc(p, bytes);
+  };
+  alloc(reinterpret_cast<void**>(&c->H), nn * 4);
+  alloc(reinterpret_cast<void**>(&c->A), nn * 4);
+  alloc(reinterpret_cast<void**>(&c->V), nn * 4);
+  alloc(reinterpret_cast<void**>(&c->U), nn * 4);
+  alloc(reinterpret_cast<void**>(&c->T), t_elems(n) * 4);
+  alloc(reinterpret_cast<void**>(&c->Wq), static_cast<size_t>(m_max) * n * 4);
+  alloc(reinterpret_cast<void**>(&c->Err), static_cast<size_t>(m_max) * SW_B * 4);
+  alloc(reinterpret_cast<void**>(&c->keys), n * 4);
+  alloc(reinterpret_cast<void**>(&c->dead), n);
+  alloc(reinterpret_cast<void**>(&c->perm), n * 4);
+  alloc(reinterpret_cast<void**>(&c->mean), sizeof(double));
+  alloc(reinterpret_cast<void**>(&c->status), sizeof(int));
+  if (e == cudaSuccess) e = cudaMallocHost(reinterpret_cast<void**>(&c->status_host), sizeof(int));
+  if (e != cudaSuccess || !c->encode) {
+    cudaGetLastError();
+    free_all(c);
+    delete c;
+    return (e == cudaErrorMemoryAllocation) ? GPTQ_ERR_OOM : GPTQ_ERR_CUDA;
+  }
+  e = cudaFuncSetAttribute(hessian_syrk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, HS_SMEM);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(sweep_block_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, SW_SMEM);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(sweep_block_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, SW_SMEM);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(sweep_block_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, SW_SMEM);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(gather_damp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kMaxN * 4));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(init_w_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kMaxN * 2));
+  if (e == cudaSuccess) e = cudaMemsetAsync(c->H, 0, nn * 4, c->stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(c->status, 0, sizeof(int), c->stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(c->stream);
+  if (e != cudaSuccess) {
+    cuda_fail(e, "create");
+    free_all(c);
+    delete c;
+    return GPTQ_ERR_CUDA;
+  }
+  *out = c;
+  return GPTQ_OK;
+}
+
+gptq_status gptq_set_hessian_chunk(gptq_ctx* c, int64_t tokens) {
+  if (!c || tokens < HS_BK || tokens % HS_BK || tokens > (int64_t(1) << 30)) return GPTQ_ERR_ARG;
+  c->chunk_tokens = tokens;
+  return GPTQ_OK;
+}
+
+gptq_status gptq_hessian_accumulate(gptq_ctx* c, const void* X, int64_t n_tok, int64_t ld_x) {
+  if (!c) return GPTQ_ERR_ARG;
+  if (c->state != ST_ACCUM) return GPTQ_ERR_STATE;
+  if (n_tok < 0 || n_tok >= (int64_t(1) << 31)) return GPTQ_ERR_ARG;
+  if (n_tok == 0) return GPTQ_OK;
+  if (!X || !aligned16(X) || ld_x < c->n || ld_x % 8) return GPTQ_ERR_ARG;
+  DeviceGuard dg(c->device);
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(c->n), static_cast<cuuint64_t>(n_tok)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_x) * 2};
+  const cuuint32_t box[2] = {64, HS_BK};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = c->encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(X), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return GPTQ_ERR_CUDA;
+  const int chunk_iters = static_cast<int>(c->chunk_tokens / HS_BK);
+  hessian_syrk_kernel<<<hs_num_tiles(static_cast<int>(c->n)), HS_THREADS, HS_SMEM, c->stream>>>(
+      map, c->H, static_cast<int>(c->n), static_cast<int>(n_tok), chunk_iters, c->status);
+  ++c->launches;
+  CKL("hessian");
+  c->n_tok += n_tok;
+  c->mirrored = 0;
+  return GPTQ_OK;
+}
+
+static gptq_status ensure_mirrored(gptq_ctx* c) {
+  if (c->mirrored) return GPTQ_OK;
+  const int n = static_cast<int>(c->n);
+  mirror_upper_kernel<<<dim3(n / 32, n / 32), dim3(32, 8), 0, c->stream>>>(c->H, n);
+  ++c->launches;
+  CKL("mirror");
+  c->mirrored = 1;
+  return GPTQ_OK;
+}
+
+gptq_status gptq_get_hessian(gptq_ctx* c, float* H_out, int64_t* n_tok_out) {
+  if (!c) return GPTQ_ERR_ARG;
+  DeviceGuard dg(c->device);
+  gptq_status s;
+  if ((s = ensure_mirrored(c)) != GPTQ_OK) return s;
+  if (H_out)
+    CK(cudaMemcpyAsync(H_out, c->H, static_cast<size_t>(c->n) * c->n * 4, cudaMemcpyDeviceToDevice, c->stream));
+  if ((s = wait_stream(c)) != GPTQ_OK) return s;
+  if (n_tok_out) *n_tok_out = c->n_tok;
+  return GPTQ_OK;
+}
+
+gptq_status gptq_set_hessian(gptq_ctx* c, const float* H_in, int64_t n_tok) {
+  if (!c || !H_in || n_tok < 0) return GPTQ_ERR_ARG;
+  if (c->state != ST_ACCUM) return GPTQ_ERR_STATE;
+  DeviceGuard dg(c->device);
+  CK(cudaMemcpyAsync(c->H, H_in, static_cast<size_t>(c->n) * c->n * 4, cudaMemcpyDeviceToDevice, c->stream));
+  c->n_tok = n_tok;
+  c->mirrored = 0;  // only the upper triangle is trusted
+  return GPTQ_OK;
+}
+
+gptq_status gptq_prepare(gptq_ctx* c, double damp, int desc_act, int32_t* perm_out) {
+  if (!c) return GPTQ_ERR_ARG;
+  if (!(damp >= 0.0) || damp > 1e6 || !(desc_act == 0 || desc_act == 1)) return GPTQ_ERR_ARG;
+  DeviceGuard dg(c->device);
+  const int n = static_cast<int>(c->n);
+  gptq_status s;
+  c->state = ST_ACCUM;
+  if ((s = ensure_mirrored(c)) != GPTQ_OK) return s;
+  diag_stats_kernel<<<1, 1024, 0, c->stream>>>(c->H, n, c->keys, c->dead, c->mean);
+  ++c->launches;
+  CKL("diag_stats");
+  if (desc_act)
+    rank_perm_kernel<<<(n + 255) / 256, 256, 0, c->stream>>>(c->keys, n, c->perm);
+  else
+    identity_perm_kernel<<<(n + 255) / 256, 256, 0, c->stream>>>(n, c->perm);
+  ++c->launches;
+  CKL("perm");
+  gather_damp_kernel<<<n, 256, static_cast<size_t>(n) * 4, c->stream>>>(c->H, n, c->perm, c->keys, c->mean, damp,
+                                                                        c->A);
+  ++c->launches;
+  CKL("gather");
+  const size_t nn = static_cast<size_t>(n) * n;
+  CK(cudaMemsetAsync(c->U, 0, nn * 4, c->stream));
+  CK(cudaMemsetAsync(c->V, 0, nn * 4, c->stream));
+  if ((s = chol_inv(c, 0, n)) != GPTQ_OK) return s;
+  if (perm_out) CK(cudaMemcpyAsync(perm_out, c->perm, n * 4, cudaMemcpyDeviceToDevice, c->stream));
+  int flags = 0;
+  if ((s = read_status(c, &flags)) != GPTQ_OK) return s;
+  if (flags) return status_from_flags(flags);
+  c->state = ST_PREPARED;
+  return GPTQ_OK;
+}
+
+gptq_status gptq_get_factor(gptq_ctx* c, float* U_out) {
+  if (!c || !U_out) return GPTQ_ERR_ARG;
+  if (c->state != ST_PREPARED) return GPTQ_ERR_STATE;
+  DeviceGuard dg(c->device);
+  CK(cudaMemcpyAsync(U_out, c->U, static_cast<size_t>(c->n) * c->n * 4, cudaMemcpyDeviceToDevice, c->stream));
+  return GPTQ_OK;
+}
+
+gptq_status gptq_quantize_layer(gptq_ctx* c, const void* W, int64_t m, gptq_qparams qp, uint32_t* codes,
+                                float* scales, float* zeros, int32_t* g_idx, float* W_hat) {
+  if (!c) return GPTQ_ERR_ARG;
+  if (c->state != ST_PREPARED) return GPTQ_ERR_STATE;
+  if (!W || !codes || !scales || !zeros || m < 1 || m > c->m_max || !valid_qparams(qp, c->n)) return GPTQ_ERR_ARG;
+  if (!aligned16(codes) || (W_hat && !aligned16(W_hat))) return GPTQ_ERR_ARG;
+  DeviceGuard dg(c->device);
+  const int n = static_cast<int>(c->n);
+  const int mi = static_cast<int>(m);
+  const int g = (qp.group_size == -1) ? n : qp.group_size;
+  init_w_kernel<<<mi, 256, static_cast<size_t>(n) * 2, c->stream>>>(static_cast<const __half*>(W), n, c->perm, c->dead,
+                                                                   c->Wq);
+  ++c->launches;
+  CKL("init_w");
+  SweepArgs a;
+  a.Wq = c->Wq;
+  a.U = c->U;
+  a.Err = c->Err;
+  a.codes = codes;
+  a.scales = scales;
+  a.zeros = zeros;
+  a.W_hat = W_hat;
+  a.perm = c->perm;
+  a.m = mi;
+  a.n = n;
+  a.bits = qp.bits;
+  a.sym = qp.sym;
+  a.g = g;
+  a.G = n / g;
+  const int grid = (mi + SW_THREADS - 1) / SW_THREADS;
+  for (int i1 = 0; i1 < n; i1 += SW_B) {
+    if (g >= SW_B)
+      sweep_block_kernel<0><<<grid, SW_THREADS, SW_SMEM, c->stream>>>(a, i1);
+    else if (g == 64)
+      sweep_block_kernel<64><<<grid, SW_THREADS, SW_SMEM, c->stream>>>(a, i1);
+    else
+      sweep_block_kernel<32><<<grid, SW_THREADS, SW_SMEM, c->stream>>>(a, i1);
+    ++c->launches;
+    CKL("sweep");
+    const int i2 = i1 + SW_B;
+    if (i2 < n) {
+      gptq_status s = sgemm(c, false, mi, n - i2, SW_B, -1.f, c->Err, SW_B,
+                            c->U + static_cast<size_t>(i1) * n + i2, n, 1.f, c->Wq + i2, n, false);
+      if (s != GPTQ_OK) return s;
+    }
+  }
+  if (g_idx) {
+    g_idx_kernel<<<(n + 255) / 256, 256, 0, c->stream>>>(c->perm, n, g, g_idx);
+    ++c->launches;
+    CKL("g_idx");
+  }
+  return GPTQ_OK;
+}
+
+gptq_status gptq_synchronize(gptq_ctx* c) {
+  if (!c) return GPTQ_ERR_ARG;
+  DeviceGuard dg(c->device);
+  int flags = 0;
+  gptq_status s = read_status(c, &flags);
+  if (s != GPTQ_OK) return s;
+  return status_from_flags(flags);
+}
+
+gptq_status gptq_reset(gptq_ctx* c) {
+  if (!c) return GPTQ_ERR_ARG;
+  DeviceGuard dg(c->device);
+  CK(cudaMemsetAsync(c->H, 0, static_cast<size_t>(c->n) * c->n * 4, c->stream));
+  c->n_tok = 0;
+  c->state = ST_ACCUM;
+  c->mirrored = 0;
+  return GPTQ_OK;
+}
+
+int64_t gptq_launch_count(const gptq_ctx* c) { return c ? c->launches : -1; }
+
+gptq_status gptq_destroy(gptq_ctx* c) {
+  if (!c) return GPTQ_OK;
+  gptq_status s;
+  {
+    DeviceGuard dg(c->device);
+    s = wait_stream(c);
+    free_all(c);
+  }
+  delete c;
+  return s;
+}
+
+}  // extern "C"

@@ -1,0 +1,229 @@
+// hessian_tc.cuh — S1: H += 2 X^T X on the sm_100a tensor cores.
+//
+// ("模型量化实战：从 INT8 PTQ 到 GPTQ 的精度保持与推理加速全解析" §3.2, accumulate_hessian:
+//  the calibration Hessian is the running sum of 2 x^T x over the calibration batches.)
+//
+// X is [n_tok x n] bf16, token-major, exactly as a calibration batch arrives.  H[i][j] is a
+// contraction over tokens, so for an output tile H[rows i, cols j] both operands are slices
+// of the same X rows: A = X[:, i-block]^T and B = X[:, j-block], both "MN-major" (the
+// feature index is contiguous).  TMA loads 64-feature x 64-token boxes with the 128-byte
+// swizzle straight into the canonical MN-major layout the tensor core reads, so X is never
+// transposed or copied.
+//
+// Work split: one CTA per 128 x 256 output tile of the upper triangle (tiles wholly below
+// the diagonal are never computed).  Warp roles:
+//   warp 0      TMA producer (one elected lane), 4-stage ring of 48 KB stages
+//   warp 1      tensor-memory allocator + MMA issuer (one lane): tcgen05.mma kind::f16,
+//               M=128, N=256, K=16, bf16 x bf16 -> fp32 in TMEM
+//   warps 2-5   epilogue: TMEM -> registers -> H (fp32, L2-resident) += 2 * partial
+// The 512 TMEM columns hold two 128x256 fp32 accumulators.  Each accumulator sums one chunk
+// of `chunk_iters` x 64 tokens on the tensor cores; the epilogue then adds that partial sum
+// into H with the CUDA cores while the other accumulator takes the next chunk.  Chunking
+// bounds the error of the tensor cores' long fp32 accumulation.
+#pragma once
+
+#include "sm100_ptx.cuh"
+
+namespace gptq {
+
+constexpr int HS_BM = 128;                        // tile rows   (features i)
+constexpr int HS_BN = 256;                        // tile cols   (features j)
+constexpr int HS_BK = 64;                         // tokens per pipeline stage
+constexpr int HS_STAGES = 4;
+constexpr int HS_BOX_BYTES = 64 * HS_BK * 2;      // one TMA box: 64 features x 64 tokens, bf16
+constexpr int HS_A_BYTES = HS_BM * HS_BK * 2;     // 16 KB
+constexpr int HS_B_BYTES = HS_BN * HS_BK * 2;     // 32 KB
+constexpr int HS_STAGE_BYTES = HS_A_BYTES + HS_B_BYTES;
+constexpr int HS_THREADS = 192;
+constexpr int HS_BAR_BYTES = 8 * (2 * HS_STAGES + 5) + 16;
+constexpr int HS_SMEM = HS_STAGES * HS_STAGE_BYTES + HS_BAR_BYTES + 1024;
+
+// Number of tiles for n features: column block bj (256 wide) owns row blocks 0 .. 2*bj+1.
+__host__ __device__ inline int hs_num_tiles(int n) {
+  const int J = (n + HS_BN - 1) / HS_BN;
+  return J * (J + 1);
+}
+
+__device__ __forceinline__ void hs_tile_of(int t, int& bi, int& bj) {
+  int b = static_cast<int>((sqrtf(4.0f * static_cast<float>(t) + 1.0f) - 1.0f) * 0.5f);
+  while (b > 0 && b * (b + 1) > t) --b;
+  while ((b + 1) * (b + 2) <= t) ++b;
+  bj = b;
+  bi = t - b * (b + 1);
+}
+
+// Wait without the abort shortcut (used to drain copies/MMAs still in flight before exit).
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+  }
+  return true;
+}
+
+__global__ void __launch_bounds__(HS_THREADS, 1)
+    hessian_syrk_kernel(const __grid_constant__ CUtensorMap xmap, float* __restrict__ H, int n, int n_tok,
+                        int chunk_iters, int* __restrict__ status) {
+  extern __shared__ uint8_t hs_smem_raw[];
+  const uint32_t raw_s = smem_u32(hs_smem_raw);
+  uint8_t* smem = hs_smem_raw + (((raw_s + 1023u) & ~1023u) - raw_s);
+  const uint32_t sbase = smem_u32(smem);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  int bi, bj;
+  hs_tile_of(blockIdx.x, bi, bj);
+  const int row0 = bi * HS_BM;
+  const int col0 = bj * HS_BN;
+  if (row0 >= n) return;  // uniform over the CTA, before any barrier or TMEM use
+
+  const uint32_t bar_full = sbase + HS_STAGES * HS_STAGE_BYTES;
+  const uint32_t bar_empty = bar_full + 8 * HS_STAGES;
+  const uint32_t bar_tfull = bar_empty + 8 * HS_STAGES;
+  const uint32_t bar_tempty = bar_tfull + 16;
+  const uint32_t bar_drain = bar_tempty + 16;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + HS_STAGES * HS_STAGE_BYTES + 8 * (2 * HS_STAGES + 5));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int k_iters = (n_tok + HS_BK - 1) / HS_BK;
+  const int n_chunks = (k_iters + chunk_iters - 1) / chunk_iters;
+  const int b_boxes = min(4, (n - col0) / 64);  // n % 128 == 0: only whole boxes
+  const uint32_t stage_tx = static_cast<uint32_t>((2 + b_boxes) * HS_BOX_BYTES);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < HS_STAGES; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_tfull + 8 * b, 1);
+      mbar_init(bar_tempty + 8 * b, 4 * 32);
+    }
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) tma_prefetch_desc(&xmap);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      int issued = 0;
+      for (int it = 0; it < k_iters; ++it) {
+        const int s = it % HS_STAGES;
+        const uint32_t ph = static_cast<uint32_t>(it / HS_STAGES) & 1u;
+        if (!mbar_wait_bounded(bar_empty + 8 * s, ph ^ 1u, abort_flag)) break;
+        const uint32_t fb = bar_full + 8 * s;
+        mbar_arrive_expect_tx(fb, stage_tx);
+        const uint32_t a_s = sbase + s * HS_STAGE_BYTES;
+        const uint32_t b_s = a_s + HS_A_BYTES;
+        const int tok = it * HS_BK;
+        tma_load_2d(a_s, &xmap, fb, row0, tok);
+        tma_load_2d(a_s + HS_BOX_BYTES, &xmap, fb, row0 + 64, tok);
+        for (int k = 0; k < b_boxes; ++k) tma_load_2d(b_s + k * HS_BOX_BYTES, &xmap, fb, col0 + 64 * k, tok);
+        issued = it + 1;
+      }
+      // no TMA write may still be in flight when the CTA exits
+      for (int it = max(0, issued - HS_STAGES); it < issued; ++it)
+        mbar_wait_drain(bar_full + 8 * (it % HS_STAGES), static_cast<uint32_t>(it / HS_STAGES) & 1u);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      constexpr uint32_t idesc = idesc_make(1u, 1u, 1u, 1u, HS_BM, HS_BN);  // bf16, MN-major A and B
+      bool ok = true;
+      int it = 0;
+      for (int c = 0; c < n_chunks && ok; ++c) {
+        const int b = c & 1;
+        const uint32_t ph = static_cast<uint32_t>(c >> 1) & 1u;
+        if (!mbar_wait_bounded(bar_tempty + 8 * b, ph ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * HS_BN);
+        const int it0 = c * chunk_iters;
+        const int it_end = min(k_iters, it0 + chunk_iters);
+        for (; it < it_end; ++it) {
+          const int s = it % HS_STAGES;
+          const uint32_t phs = static_cast<uint32_t>(it / HS_STAGES) & 1u;
+          if (!mbar_wait_bounded(bar_full + 8 * s, phs, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_s = sbase + s * HS_STAGE_BYTES;
+          const uint32_t b_s = a_s + HS_A_BYTES;
+#pragma unroll
+          for (int k = 0; k < HS_BK / 16; ++k) {
+            // 16 tokens = two 8-row swizzle atoms of 1024 bytes
+            const uint64_t ad = sdesc_sw128(a_s + k * 2048, HS_BOX_BYTES, 1024);
+            const uint64_t bd = sdesc_sw128(b_s + k * 2048, HS_BOX_BYTES, 1024);
+            umma_f16(d_tmem, ad, bd, idesc, (it > it0 || k > 0) ? 1u : 0u);
+          }
+          umma_commit(bar_empty + 8 * s);
+        }
+        if (!ok) break;
+        umma_commit(bar_tfull + 8 * b);
+      }
+      if (!ok) {
+        // MMAs may still be running: wait for them before the TMEM is released
+        umma_commit(bar_drain);
+        mbar_wait_drain(bar_drain, 0);
+      }
+    }
+  } else {
+    // ---------------- epilogue: TMEM -> H ----------------
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int r = row0 + q * 32 + lane;
+    for (int c = 0; c < n_chunks; ++c) {
+      const int b = c & 1;
+      const uint32_t ph = static_cast<uint32_t>(c >> 1) & 1u;
+      int ok = 0;
+      if (lane == 0) ok = mbar_wait_bounded(bar_tfull + 8 * b, ph, abort_flag) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int cc = 0; cc < HS_BN / 32; ++cc) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * HS_BN + cc * 32),
+                           v);
+        tmem_ld_wait();
+        const int col = col0 + cc * 32;
+        if (r < n && col < n) {
+          float4* dst = reinterpret_cast<float4*>(H + static_cast<size_t>(r) * n + col);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            float4 h = dst[j];
+            h.x = fmaf(2.0f, __uint_as_float(v[4 * j + 0]), h.x);
+            h.y = fmaf(2.0f, __uint_as_float(v[4 * j + 1]), h.y);
+            h.z = fmaf(2.0f, __uint_as_float(v[4 * j + 2]), h.z);
+            h.w = fmaf(2.0f, __uint_as_float(v[4 * j + 3]), h.w);
+            dst[j] = h;
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar_tempty + 8 * b);
+    }
+  }
+
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) atomicOr(status, ST_TIMEOUT);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+}  // namespace gptq

@@ -1,0 +1,122 @@
+// prepare_kernels.cuh — S2/S3 and the data movement around the factorization.
+//
+//   mirror_upper_kernel   H[r][c] = H[c][r] for r > c (the Hessian kernel writes the upper
+//                         triangle only)
+//   diag_stats_kernel     dead columns (diag H == 0 -> treated as 1), sort keys, mean diag
+//                         ("模型量化实战…" §3.2 prepare: damp = 0.01 * mean(diag H))
+//   rank_perm_kernel      desc_act: stable descending order of diag H by rank counting
+//                         ("GPTQ量化损失深度解析…": desc_act=True, 按敏感度排序)
+//   gather_damp_kernel    A = H[perm][:, perm] + damp * mean(diag) * I  (row staged in smem)
+//   init_w_kernel         Wq = fp32(W[:, perm]) with dead columns zeroed
+//   g_idx_kernel          g_idx[perm[k]] = k / group_size
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cstdint>
+
+namespace gptq {
+
+__global__ void mirror_upper_kernel(float* __restrict__ H, int n) {
+  __shared__ float t[32][33];
+  const int tr = blockIdx.y, tc = blockIdx.x;
+  if (tr > tc) return;
+  const int x = threadIdx.x, y = threadIdx.y;  // 32 x 8
+  for (int k = y; k < 32; k += 8) t[k][x] = H[static_cast<size_t>(tr * 32 + k) * n + tc * 32 + x];
+  __syncthreads();
+  // write the transpose into block (tc, tr); on the diagonal block only the strictly lower part
+  for (int k = y; k < 32; k += 8) {
+    const int r = tc * 32 + k, c = tr * 32 + x;
+    if (r > c) H[static_cast<size_t>(r) * n + c] = t[x][k];
+  }
+}
+
+// One CTA of 1024 threads.
+__global__ void diag_stats_kernel(const float* __restrict__ H, int n, float* __restrict__ keys,
+                                  uint8_t* __restrict__ dead, double* __restrict__ mean_out) {
+  __shared__ double red[32];
+  double s = 0.0;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const float d = H[static_cast<size_t>(i) * n + i];
+    const bool z = (d == 0.0f);
+    // a NaN diagonal sorts last (keys must be totally ordered for the rank permutation)
+    const float k = z ? 1.0f : (d == d ? d : -INFINITY);
+    keys[i] = k;
+    dead[i] = z ? 1 : 0;
+    s += static_cast<double>(k);
+  }
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    double v = (threadIdx.x < (blockDim.x >> 5)) ? red[threadIdx.x] : 0.0;
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (threadIdx.x == 0) *mean_out = v / static_cast<double>(n);
+  }
+}
+
+// perm[rank(i)] = i with rank(i) = #{j : key_j > key_i or (key_j == key_i and j < i)}.
+__global__ void rank_perm_kernel(const float* __restrict__ keys, int n, int32_t* __restrict__ perm) {
+  __shared__ float ks[1024];
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  const float ki = (i < n) ? keys[i] : 0.0f;
+  int rank = 0;
+  for (int j0 = 0; j0 < n; j0 += 1024) {
+    __syncthreads();
+    for (int t = threadIdx.x; t < 1024; t += blockDim.x) ks[t] = (j0 + t < n) ? keys[j0 + t] : 0.0f;
+    __syncthreads();
+    const int jn = min(1024, n - j0);
+    for (int t = 0; t < jn; ++t) {
+      const float kj = ks[t];
+      rank += (kj > ki) || (kj == ki && j0 + t < i);
+    }
+  }
+  if (i < n) perm[rank] = i;
+}
+
+__global__ void identity_perm_kernel(int n, int32_t* __restrict__ perm) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) perm[i] = i;
+}
+
+// One CTA per output row a; the source row perm[a] of the (mirrored) H is staged in smem.
+__global__ void gather_damp_kernel(const float* __restrict__ H, int n, const int32_t* __restrict__ perm,
+                                   const float* __restrict__ keys, const double* __restrict__ mean,
+                                   double damp, float* __restrict__ A) {
+  extern __shared__ float row_s[];
+  const int a = blockIdx.x;
+  const int pa = perm[a];
+  const float4* src = reinterpret_cast<const float4*>(H + static_cast<size_t>(pa) * n);
+  for (int k = threadIdx.x; k < n / 4; k += blockDim.x) reinterpret_cast<float4*>(row_s)[k] = src[k];
+  __syncthreads();
+  float* dst = A + static_cast<size_t>(a) * n;
+  for (int b = threadIdx.x; b < n; b += blockDim.x) {
+    float v;
+    if (b == a)
+      v = static_cast<float>(static_cast<double>(keys[pa]) + damp * (*mean));
+    else
+      v = row_s[perm[b]];
+    dst[b] = v;
+  }
+}
+
+// One CTA per row r: Wq[r][k] = dead[perm[k]] ? 0 : float(W[r][perm[k]]).
+__global__ void init_w_kernel(const __half* __restrict__ W, int n, const int32_t* __restrict__ perm,
+                              const uint8_t* __restrict__ dead, float* __restrict__ Wq) {
+  extern __shared__ __half wrow_s[];
+  const int r = blockIdx.x;
+  const __half* src = W + static_cast<size_t>(r) * n;
+  for (int k = threadIdx.x; k < n; k += blockDim.x) wrow_s[k] = src[k];
+  __syncthreads();
+  float* dst = Wq + static_cast<size_t>(r) * n;
+  for (int k = threadIdx.x; k < n; k += blockDim.x) {
+    const int p = perm[k];
+    dst[k] = dead[p] ? 0.0f : __half2float(wrow_s[p]);
+  }
+}
+
+__global__ void g_idx_kernel(const int32_t* __restrict__ perm, int n, int g, int32_t* __restrict__ g_idx) {
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  if (k < n) g_idx[perm[k]] = k / g;
+}
+
+}  // namespace gptq

@@ -1,0 +1,190 @@
+"""Python binding of libgptq (ctypes).  Argument marshalling only: every step of the
+solve runs in the library's CUDA kernels; PyTorch provides device memory and the stream.
+
+The object mirrors the three-call lifecycle of the GPTQ quantizer on the page
+"模型量化实战：从 INT8 PTQ 到 GPTQ 的精度保持与推理加速全解析" (§3.2: accumulate the Hessian
+over calibration batches, prepare the inverse factor, quantize the layer), with the
+quantizer settings named as in AutoGPTQ's quantize_config ("GPTQ算法原理深度解析" §3.3).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libgptq.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "gptq.h")
+
+STATUS = {0: "GPTQ_OK", 1: "GPTQ_ERR_ARG", 2: "GPTQ_ERR_STATE", 3: "GPTQ_ERR_NOT_PD", 4: "GPTQ_ERR_OOM",
+          5: "GPTQ_ERR_CUDA", 6: "GPTQ_ERR_TIMEOUT", 7: "GPTQ_ERR_UNSUPPORTED"}
+OK, ERR_ARG, ERR_STATE, ERR_NOT_PD, ERR_OOM, ERR_CUDA, ERR_TIMEOUT, ERR_UNSUPPORTED = range(8)
+
+
+class GPTQError(RuntimeError):
+    def __init__(self, status: int, call: str):
+        self.status = status
+        self.name = STATUS.get(status, str(status))
+        super().__init__(f"{call}: {self.name} ({lib().gptq_status_string(status).decode()})")
+
+
+class QParams(ctypes.Structure):
+    _fields_ = [("bits", ctypes.c_int), ("group_size", ctypes.c_int), ("sym", ctypes.c_int)]
+
+
+_LIB = None
+_P = ctypes.c_void_p
+_SIGS = {
+    "gptq_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64]),
+    "gptq_create": (ctypes.c_int, [ctypes.POINTER(_P), ctypes.c_int64, ctypes.c_int64, ctypes.c_int, _P]),
+    "gptq_hessian_accumulate": (ctypes.c_int, [_P, _P, ctypes.c_int64, ctypes.c_int64]),
+    "gptq_get_hessian": (ctypes.c_int, [_P, _P, ctypes.POINTER(ctypes.c_int64)]),
+    "gptq_set_hessian": (ctypes.c_int, [_P, _P, ctypes.c_int64]),
+    "gptq_prepare": (ctypes.c_int, [_P, ctypes.c_double, ctypes.c_int, _P]),
+    "gptq_get_factor": (ctypes.c_int, [_P, _P]),
+    "gptq_quantize_layer": (ctypes.c_int, [_P, _P, ctypes.c_int64, QParams, _P, _P, _P, _P, _P]),
+    "gptq_synchronize": (ctypes.c_int, [_P]),
+    "gptq_reset": (ctypes.c_int, [_P]),
+    "gptq_destroy": (ctypes.c_int, [_P]),
+    "gptq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "gptq_set_hessian_chunk": (ctypes.c_int, [_P, ctypes.c_int64]),
+    "gptq_launch_count": (ctypes.c_int64, [_P]),
+}
+
+
+def lib():
+    """Load libgptq.so (built in-tree).  Fails loudly when it is missing: there is no fallback."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libgptq.so is not built ({LIB_PATH}); run "
+                               "`python -m post_weight_quantization_16_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _LIB = L
+    return _LIB
+
+
+def header_functions():
+    """Names of the functions include/gptq.h declares."""
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gptq_[a-z_]+)\s*\(", text)))
+
+
+def _check(status: int, call: str):
+    if status != OK:
+        raise GPTQError(status, call)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+class GPTQContext:
+    """One layer width n: accumulate H over calibration batches, prepare, quantize layers."""
+
+    def __init__(self, n: int, m_max: int, device: int | torch.device = 0, stream: torch.cuda.Stream | None = None):
+        self.device = torch.device("cuda", device if isinstance(device, int) else device.index)
+        self.n, self.m_max = int(n), int(m_max)
+        self.stream = stream if stream is not None else torch.cuda.current_stream(self.device)
+        h = ctypes.c_void_p()
+        _check(lib().gptq_create(ctypes.byref(h), self.n, self.m_max, self.device.index,
+                                 ctypes.c_void_p(self.stream.cuda_stream)), "gptq_create")
+        self._h = h
+
+    # -- lifecycle ---------------------------------------------------------------------------
+    def close(self):
+        if getattr(self, "_h", None):
+            st = lib().gptq_destroy(self._h)
+            self._h = None
+            _check(st, "gptq_destroy")
+
+    def __del__(self):
+        try:
+            if getattr(self, "_h", None):
+                lib().gptq_destroy(self._h)
+                self._h = None
+        except Exception:
+            pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        self.close()
+
+    # -- S1 ----------------------------------------------------------------------------------
+    def set_hessian_chunk(self, tokens: int):
+        _check(lib().gptq_set_hessian_chunk(self._h, int(tokens)), "gptq_set_hessian_chunk")
+
+    def accumulate_hessian(self, X: torch.Tensor):
+        """H += 2 X^T X for a bf16 batch X [tokens, n] on the device (row stride may exceed n)."""
+        if X.dtype != torch.bfloat16 or X.device != self.device or X.dim() != 2 or X.stride(1) != 1:
+            raise ValueError("X must be a bf16 [tokens, n] device tensor with unit column stride")
+        _check(lib().gptq_hessian_accumulate(self._h, _ptr(X), X.shape[0], X.stride(0)), "gptq_hessian_accumulate")
+
+    def get_hessian(self):
+        H = torch.empty((self.n, self.n), dtype=torch.float32, device=self.device)
+        nt = ctypes.c_int64()
+        _check(lib().gptq_get_hessian(self._h, _ptr(H), ctypes.byref(nt)), "gptq_get_hessian")
+        return H, nt.value
+
+    def set_hessian(self, H: torch.Tensor, n_tok: int):
+        if H.dtype != torch.float32 or H.shape != (self.n, self.n) or not H.is_contiguous() or H.device != self.device:
+            raise ValueError("H must be a contiguous fp32 [n, n] device tensor")
+        _check(lib().gptq_set_hessian(self._h, _ptr(H), int(n_tok)), "gptq_set_hessian")
+
+    # -- S2-S4 -------------------------------------------------------------------------------
+    def prepare(self, damp: float = 0.01, desc_act: bool = False) -> torch.Tensor:
+        perm = torch.empty(self.n, dtype=torch.int32, device=self.device)
+        _check(lib().gptq_prepare(self._h, float(damp), int(bool(desc_act)), _ptr(perm)), "gptq_prepare")
+        return perm
+
+    def get_factor(self) -> torch.Tensor:
+        U = torch.empty((self.n, self.n), dtype=torch.float32, device=self.device)
+        _check(lib().gptq_get_factor(self._h, _ptr(U)), "gptq_get_factor")
+        return U
+
+    # -- S5-S7 -------------------------------------------------------------------------------
+    def quantize_layer(self, W: torch.Tensor, bits: int = 4, group_size: int = 128, sym: bool = False,
+                       want_w_hat: bool = True, out: dict | None = None) -> dict:
+        """Quantize fp16 W [m, n] (original column order).  Returns device tensors
+        codes [m, n*bits/32] int32-viewed uint32 words, scales/zeros [m, G], g_idx [n], w_hat [m, n]."""
+        if W.dtype != torch.float16 or W.dim() != 2 or W.shape[1] != self.n or not W.is_contiguous() \
+                or W.device != self.device:
+            raise ValueError("W must be a contiguous fp16 [m, n] device tensor")
+        m = W.shape[0]
+        g = self.n if group_size == -1 else group_size
+        G = self.n // g if g > 0 and self.n % g == 0 else 1
+        if out is None:
+            out = {
+                "codes": torch.empty((m, self.n * bits // 32), dtype=torch.int32, device=self.device),
+                "scales": torch.empty((m, G), dtype=torch.float32, device=self.device),
+                "zeros": torch.empty((m, G), dtype=torch.float32, device=self.device),
+                "g_idx": torch.empty(self.n, dtype=torch.int32, device=self.device),
+                "w_hat": torch.empty((m, self.n), dtype=torch.float32, device=self.device) if want_w_hat else None,
+            }
+        qp = QParams(int(bits), int(group_size), int(bool(sym)))
+        _check(lib().gptq_quantize_layer(self._h, _ptr(W), m, qp, _ptr(out["codes"]), _ptr(out["scales"]),
+                                         _ptr(out["zeros"]), _ptr(out["g_idx"]), _ptr(out.get("w_hat"))),
+               "gptq_quantize_layer")
+        return out
+
+    def synchronize(self):
+        _check(lib().gptq_synchronize(self._h), "gptq_synchronize")
+
+    def launch_count(self) -> int:
+        return int(lib().gptq_launch_count(self._h))
+
+    def reset(self):
+        _check(lib().gptq_reset(self._h), "gptq_reset")
+
+
+def workspace_bytes(n: int, m_max: int) -> int:
+    return int(lib().gptq_workspace_bytes(int(n), int(m_max)))

@@ -1,0 +1,77 @@
+"""Host-side checks of the C ABI (no GPU): the library loads, exports every function the
+header declares, and validates arguments before touching the device."""
+import ctypes
+import os
+
+import pytest
+
+from post_weight_quantization_16_b200 import build as B
+from post_weight_quantization_16_b200 import gptq as G
+
+
+@pytest.fixture(scope="module")
+def L():
+    B.build()
+    return G.lib()
+
+
+def test_library_exports_every_header_function(L):
+    names = G.header_functions()
+    assert len(names) >= 13
+    for nm in names:
+        assert hasattr(L, nm), nm
+    # and the binding declares a signature for each of them
+    assert set(names) == set(G._SIGS)
+
+
+def test_status_strings(L):
+    for s in range(8):
+        assert L.gptq_status_string(s)
+    assert b"positive definite" in L.gptq_status_string(G.ERR_NOT_PD)
+
+
+def test_workspace_bytes(L):
+    n, m = 4096, 4096
+    b = L.gptq_workspace_bytes(n, m)
+    assert b >= 4 * n * n * 4 + m * n * 4
+    assert L.gptq_workspace_bytes(100, 4) == 0        # n % 128
+    assert L.gptq_workspace_bytes(4096, 0) == 0       # m_max
+    assert L.gptq_workspace_bytes(65536, 1) == 0      # n too large
+    assert L.gptq_workspace_bytes(28672, 8192) > 14e9
+
+
+def test_create_rejects_bad_arguments_before_any_device_call(L):
+    h = ctypes.c_void_p()
+    assert L.gptq_create(ctypes.byref(h), 100, 16, 0, None) == G.ERR_ARG
+    assert L.gptq_create(ctypes.byref(h), 512, 0, 0, None) == G.ERR_ARG
+    assert L.gptq_create(ctypes.byref(h), 512, 16, -1, None) == G.ERR_ARG
+    assert L.gptq_create(None, 512, 16, 0, None) == G.ERR_ARG
+
+
+def test_create_reports_oom_without_allocating(L, monkeypatch):
+    monkeypatch.setenv("GPTQ_MAX_WORKSPACE_BYTES", "1000")
+    h = ctypes.c_void_p()
+    assert L.gptq_create(ctypes.byref(h), 512, 16, 0, None) == G.ERR_OOM
+    assert not h.value
+
+
+def test_null_context_is_an_argument_error(L):
+    assert L.gptq_hessian_accumulate(None, None, 0, 0) == G.ERR_ARG
+    assert L.gptq_prepare(None, 0.01, 0, None) == G.ERR_ARG
+    assert L.gptq_quantize_layer(None, None, 1, G.QParams(4, 128, 0), None, None, None, None, None) == G.ERR_ARG
+    assert L.gptq_synchronize(None) == G.ERR_ARG
+    assert L.gptq_reset(None) == G.ERR_ARG
+    assert L.gptq_destroy(None) == G.OK
+
+
+@pytest.mark.skipif(os.path.exists("/dev/nvidia0"), reason="checks the no-GPU behaviour")
+def test_no_cpu_fallback_without_a_device(L):
+    h = ctypes.c_void_p()
+    assert L.gptq_create(ctypes.byref(h), 512, 16, 0, None) == G.ERR_CUDA
+
+
+def test_binding_fails_loudly_when_library_missing(monkeypatch, tmp_path):
+    monkeypatch.setattr(G, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(G, "_LIB", None)
+    with pytest.raises(RuntimeError, match="not built"):
+        G.lib()

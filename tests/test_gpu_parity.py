@@ -1,0 +1,185 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle on seeded inputs."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import gptq_oracle as O
+from post_weight_quantization_16_b200 import synth
+from post_weight_quantization_16_b200.gptq import GPTQContext, GPTQError, ERR_NOT_PD, ERR_STATE
+from tests import gpu_helpers as GH
+
+pytestmark = pytest.mark.gpu
+
+TINY, TINY_Q = synth.WORKLOADS["tiny_256x512"]
+
+
+def _h_rel(H, Href):
+    return np.linalg.norm(H - Href) / np.linalg.norm(Href)
+
+
+# ----------------------------------------------------------------------------------------
+# S1 Hessian
+# ----------------------------------------------------------------------------------------
+@pytest.mark.parametrize("n,n_tok", [(512, 2048), (384, 1000), (128, 64), (768, 4157)])
+def test_hessian_matches_fp64(n, n_tok):
+    layer = synth.scaled_layer(TINY, m=64, n=n, n_tok=n_tok)
+    X = synth.make_x_bf16(layer)
+    with GPTQContext(n, 64, 0) as ctx:
+        ctx.accumulate_hessian(GH.bf16_to_dev(X))
+        H, nt = ctx.get_hessian()
+    H = H.cpu().numpy().astype(np.float64)
+    Href = O.hessian(synth.bf16_bits_to_f32(X))
+    assert nt == n_tok
+    assert _h_rel(H, Href) <= GH.H_REL_FRO
+    assert np.array_equal(H, H.T)
+
+
+def test_hessian_batches_strides_and_chunks():
+    layer = synth.scaled_layer(TINY, m=64, n=512, n_tok=6000)
+    X = synth.make_x_bf16(layer)
+    Href = O.hessian(synth.bf16_bits_to_f32(X))
+    for chunk in (64, 1024, 1 << 20):
+        with GPTQContext(512, 64, 0) as ctx:
+            ctx.set_hessian_chunk(chunk)
+            # batches of uneven sizes, the middle one taken from a wider (padded) buffer
+            ctx.accumulate_hessian(GH.bf16_to_dev(X[:1000]))
+            pad = np.zeros((3000, 512 + 64), dtype=np.uint16)
+            pad[:, :512] = X[1000:4000]
+            Xp = GH.bf16_to_dev(pad)
+            ctx.accumulate_hessian(Xp[:, :512])
+            ctx.accumulate_hessian(GH.bf16_to_dev(X[4000:]))
+            H, nt = ctx.get_hessian()
+        assert nt == 6000
+        assert _h_rel(H.cpu().numpy().astype(np.float64), Href) <= GH.H_REL_FRO, chunk
+
+
+# ----------------------------------------------------------------------------------------
+# S2-S4 prepare
+# ----------------------------------------------------------------------------------------
+@pytest.mark.parametrize("desc_act", [False, True])
+@pytest.mark.parametrize("damp", [0.01, 0.1])
+def test_prepare_perm_and_factor(desc_act, damp):
+    layer = synth.scaled_layer(TINY, m=64, n=640, n_tok=3000)
+    X = synth.make_x_bf16(layer)
+    with GPTQContext(layer.n, 64, 0) as ctx:
+        ctx.accumulate_hessian(GH.bf16_to_dev(X))
+        H, _ = ctx.get_hessian()
+        perm = ctx.prepare(damp, desc_act).cpu().numpy()
+        U = ctx.get_factor().cpu().numpy().astype(np.float64)
+    H = H.cpu().numpy().astype(np.float64)
+    prep = O.prepare(H, damp, desc_act)          # the oracle on the GPU's H
+    assert np.array_equal(perm, prep["perm"])
+    assert np.allclose(np.tril(U, -1), 0)
+    err = np.abs(U - prep["U"]).max() / np.abs(prep["U"]).max()
+    assert err <= 2e-5, err
+    resid = np.abs(U.T @ U @ prep["Hd"] - np.eye(layer.n)).max()
+    assert resid <= 1e-3, resid
+
+
+def test_not_positive_definite_is_reported():
+    n = 256
+    H = np.eye(n, dtype=np.float32)
+    H[3, 7] = H[7, 3] = 4.0       # 2x2 minor [[1,4],[4,1]] is indefinite
+    with GPTQContext(n, 32, 0) as ctx:
+        ctx.set_hessian(torch.from_numpy(H).to(GH.DEV), 10)
+        with pytest.raises(GPTQError) as ei:
+            ctx.prepare(0.0, False)
+        assert ei.value.status == ERR_NOT_PD
+        # not prepared: quantizing is a state error
+        W = torch.zeros((32, n), dtype=torch.float16, device=GH.DEV)
+        with pytest.raises(GPTQError) as ei:
+            ctx.quantize_layer(W, 4, 128, False)
+        assert ei.value.status == ERR_STATE
+        # with damping the same H is fine
+        ctx.prepare(1.0, False)
+
+
+def test_state_machine():
+    layer = synth.scaled_layer(TINY, m=32, n=256, n_tok=512)
+    X = GH.bf16_to_dev(synth.make_x_bf16(layer))
+    with GPTQContext(256, 32, 0) as ctx:
+        W = torch.zeros((32, 256), dtype=torch.float16, device=GH.DEV)
+        with pytest.raises(GPTQError) as ei:
+            ctx.quantize_layer(W, 4, 128, False)
+        assert ei.value.status == ERR_STATE
+        ctx.accumulate_hessian(X)
+        ctx.prepare(0.01, True)
+        with pytest.raises(GPTQError) as ei:
+            ctx.accumulate_hessian(X)
+        assert ei.value.status == ERR_STATE
+        ctx.reset()
+        ctx.accumulate_hessian(X)
+        _, nt = ctx.get_hessian()
+        assert nt == 512
+
+
+# ----------------------------------------------------------------------------------------
+# S5-S7 sweep (stage-isolated replay against the oracle on the GPU's H)
+# ----------------------------------------------------------------------------------------
+SWEEP_CASES = [
+    # bits, group, sym, desc_act, damp
+    (4, 128, False, False, 0.01),
+    (4, 128, False, True, 0.01),
+    (4, 128, True, True, 0.01),
+    (3, 64, False, True, 0.1),
+    (2, 32, False, True, 0.01),
+    (2, -1, False, True, 0.1),
+    (3, 256, True, False, 0.01),
+    (8, 128, False, True, 0.01),
+    (4, 64, True, True, 0.1),
+]
+
+
+@pytest.mark.parametrize("bits,g,sym,desc_act,damp", SWEEP_CASES)
+def test_quantize_layer_parity(bits, g, sym, desc_act, damp):
+    layer = synth.scaled_layer(TINY, m=96, n=512, n_tok=2048)
+    qs = synth.QuantSetting(bits, g, sym, damp, desc_act)
+    gpu = GH.run_path(layer, qs)
+    prep = O.prepare(gpu["H"], damp, desc_act)
+    assert np.array_equal(gpu["perm"], prep["perm"])
+    st, rep = GH.check_sweep_replay(gpu["W"], prep, gpu, qs)
+    GH.assert_replay_ok(st, rep, gpu)
+    # g_idx and the dequantized weights in original order
+    assert np.array_equal(gpu["g_idx"], O.g_idx(prep["perm"], g))
+    what = O.unpermute_columns(rep["what"], prep["perm"])
+    scale_ref = np.repeat(rep["scales"], (layer.n if g == -1 else g), axis=1)[:, np.argsort(prep["perm"])]
+    assert np.all(np.abs(gpu["w_hat"] - what) <= 1e-5 * scale_ref + 1e-12)
+    # layer error within 1 % of the oracle's own (un-replayed) run, measured with the exact H
+    Href = O.hessian(synth.bf16_bits_to_f32(gpu["X"]))
+    own = O.quantize_layer(gpu["W"].astype(np.float64), gpu["H"], bits, g, sym, damp, desc_act)
+    e_gpu = O.layer_error(gpu["W"], gpu["w_hat"], Href)
+    e_own = O.layer_error(gpu["W"], own["what_orig"], Href)
+    assert abs(e_gpu - e_own) <= GH.LAYER_ERR_REL * e_own, (e_gpu, e_own)
+
+
+def test_end_to_end_tiny_config():
+    """The tiny workload end to end: H against the oracle's own H, then the full replay."""
+    gpu = GH.run_path(TINY, TINY_Q)
+    Href = O.hessian(synth.bf16_bits_to_f32(gpu["X"]))
+    assert _h_rel(gpu["H"], Href) <= GH.H_REL_FRO
+    prep = O.prepare(gpu["H"], TINY_Q.damp, TINY_Q.desc_act)
+    st, rep = GH.check_sweep_replay(gpu["W"], prep, gpu, TINY_Q)
+    GH.assert_replay_ok(st, rep, gpu)
+    assert np.array_equal(gpu["packed"], O.pack_codes(rep["codes"], TINY_Q.bits))
+
+
+def test_dead_columns_on_gpu():
+    layer = synth.scaled_layer(TINY, m=64, n=256, n_tok=1024)
+    X = synth.make_x_bf16(layer)
+    X[:, [5, 77, 200]] = 0
+    qs = synth.QuantSetting(4, 128, False, 0.01, True)
+    gpu = GH.run_path(layer, qs, X_bits=X)
+    assert np.all(gpu["w_hat"][:, [5, 77, 200]] == 0)
+    prep = O.prepare(gpu["H"], qs.damp, qs.desc_act)
+    assert prep["dead"][[5, 77, 200]].all()
+    st, rep = GH.check_sweep_replay(gpu["W"], prep, gpu, qs)
+    GH.assert_replay_ok(st, rep, gpu)
+
+
+def test_ragged_rows_and_wider_context():
+    layer = synth.scaled_layer(TINY, m=45, n=384, n_tok=777)
+    qs = synth.QuantSetting(4, 128, True, 0.01, True)
+    gpu = GH.run_path(layer, qs, ctx_m=300)
+    prep = O.prepare(gpu["H"], qs.damp, qs.desc_act)
+    st, rep = GH.check_sweep_replay(gpu["W"], prep, gpu, qs)
+    GH.assert_replay_ok(st, rep, gpu)
