@@ -145,8 +145,8 @@ int64_t gptq_launch_count(const gptq_ctx* ctx);
 const char* gptq_status_string(gptq_status s);
 
 /* Tokens per tensor-memory accumulation chunk of S1 (a multiple of 64).  Each chunk is
- * summed on the tensor cores, then added to H in fp32 by the CUDA cores, which bounds the
- * accumulation error of long calibration sets.  Default 4096. */
+ * summed on the tensor cores, then added to fp32 running sums with round-to-nearest adds,
+ * which bounds the accumulation error of long calibration sets.  Default 512. */
 gptq_status gptq_set_hessian_chunk(gptq_ctx* ctx, int64_t tokens);
 
 #ifdef __cplusplus

@@ -49,7 +49,7 @@ struct gptq_ctx {
   int64_t n_tok = 0;
   int state = ST_ACCUM;
   int mirrored = 0;           // H's lower triangle has been filled
-  int64_t chunk_tokens = 4096;
+  int64_t chunk_tokens = 512;
   int64_t launches = 0;       // kernels launched by this context (instrumentation)
   PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
 };
@@ -281,7 +281,7 @@ gptq_status gptq_create(gptq_ctx** out, int64_t n, int64_t m_max, int device, vo
   c->stream = static_cast<cudaStream_t>(stream);
   c->n = n;
   c->m_max = m_max;
-  c->chunk_tokens = 4096;
+  c->chunk_tokens = 512;
   c->encode = get_encode();
   const size_t nn = static_cast<size_t>(n) * n;
   cudaError_t e = cudaSuccess;

@@ -15,11 +15,13 @@
 //   warp 0      TMA producer (one elected lane), 4-stage ring of 48 KB stages
 //   warp 1      tensor-memory allocator + MMA issuer (one lane): tcgen05.mma kind::f16,
 //               M=128, N=256, K=16, bf16 x bf16 -> fp32 in TMEM
-//   warps 2-5   epilogue: TMEM -> registers -> H (fp32, L2-resident) += 2 * partial
+//   warps 2-9   epilogue: TMEM -> registers, fp32 running sums; H += 2 * sums at the end
 // The 512 TMEM columns hold two 128x256 fp32 accumulators.  Each accumulator sums one chunk
 // of `chunk_iters` x 64 tokens on the tensor cores; the epilogue then adds that partial sum
-// into H with the CUDA cores while the other accumulator takes the next chunk.  Chunking
-// bounds the error of the tensor cores' long fp32 accumulation.
+// to its register accumulators with round-to-nearest fp32 adds while the other accumulator
+// takes the next chunk.  The tensor cores' own accumulation is not round-to-nearest (on a
+// long sum of positive terms it drifts low by about 1e-5 relative per 4096 tokens), so
+// short chunks keep that drift at the 1e-6 level.
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -34,7 +36,7 @@ constexpr int HS_BOX_BYTES = 64 * HS_BK * 2;      // one TMA box: 64 features x 
 constexpr int HS_A_BYTES = HS_BM * HS_BK * 2;     // 16 KB
 constexpr int HS_B_BYTES = HS_BN * HS_BK * 2;     // 32 KB
 constexpr int HS_STAGE_BYTES = HS_A_BYTES + HS_B_BYTES;
-constexpr int HS_THREADS = 192;
+constexpr int HS_THREADS = 64 + 256;  // producer, MMA, 8 epilogue warps
 constexpr int HS_BAR_BYTES = 8 * (2 * HS_STAGES + 5) + 16;
 constexpr int HS_SMEM = HS_STAGES * HS_STAGE_BYTES + HS_BAR_BYTES + 1024;
 
@@ -98,7 +100,7 @@ __global__ void __launch_bounds__(HS_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar_tfull + 8 * b, 1);
-      mbar_init(bar_tempty + 8 * b, 4 * 32);
+      mbar_init(bar_tempty + 8 * b, 8 * 32);
     }
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
@@ -182,39 +184,58 @@ __global__ void __launch_bounds__(HS_THREADS, 1)
       }
     }
   } else {
-    // ---------------- epilogue: TMEM -> H ----------------
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    // ---------------- epilogue: TMEM -> registers (fp32) -> H ----------------
+    // Eight warps: warp w reads TMEM lane quarter (w % 4) and one 128-column half of the
+    // tile.  Each thread keeps its row's 128 running sums in registers across chunks and
+    // adds them into H once, at the end of the call.
+    const int q = warp & 3;
+    const int hh = (warp - 2) >> 2;
     const int r = row0 + q * 32 + lane;
+    float acc[HS_BN / 2];
+#pragma unroll
+    for (int j = 0; j < HS_BN / 2; ++j) acc[j] = 0.0f;
+    bool all_ok = true;
     for (int c = 0; c < n_chunks; ++c) {
       const int b = c & 1;
       const uint32_t ph = static_cast<uint32_t>(c >> 1) & 1u;
       int ok = 0;
       if (lane == 0) ok = mbar_wait_bounded(bar_tfull + 8 * b, ph, abort_flag) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
+      if (!ok) {
+        all_ok = false;
+        break;
+      }
       tc_fence_after();
-#pragma unroll 1
-      for (int cc = 0; cc < HS_BN / 32; ++cc) {
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
         uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * HS_BN + cc * 32),
+        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                               static_cast<uint32_t>(b * HS_BN + hh * (HS_BN / 2) + cc * 32),
                            v);
         tmem_ld_wait();
-        const int col = col0 + cc * 32;
-        if (r < n && col < n) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) acc[cc * 32 + j] += __uint_as_float(v[j]);
+      }
+      tc_fence_before();
+      mbar_arrive(bar_tempty + 8 * b);
+    }
+    if (all_ok && r < n) {
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        const int col = col0 + hh * (HS_BN / 2) + cc * 32;
+        if (col < n) {
           float4* dst = reinterpret_cast<float4*>(H + static_cast<size_t>(r) * n + col);
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             float4 h = dst[j];
-            h.x = fmaf(2.0f, __uint_as_float(v[4 * j + 0]), h.x);
-            h.y = fmaf(2.0f, __uint_as_float(v[4 * j + 1]), h.y);
-            h.z = fmaf(2.0f, __uint_as_float(v[4 * j + 2]), h.z);
-            h.w = fmaf(2.0f, __uint_as_float(v[4 * j + 3]), h.w);
+            h.x = fmaf(2.0f, acc[cc * 32 + 4 * j + 0], h.x);
+            h.y = fmaf(2.0f, acc[cc * 32 + 4 * j + 1], h.y);
+            h.z = fmaf(2.0f, acc[cc * 32 + 4 * j + 2], h.z);
+            h.w = fmaf(2.0f, acc[cc * 32 + 4 * j + 3], h.w);
             dst[j] = h;
           }
         }
       }
-      tc_fence_before();
-      mbar_arrive(bar_tempty + 8 * b);
     }
   }
 

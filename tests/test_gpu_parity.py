@@ -90,8 +90,8 @@ def test_not_positive_definite_is_reported():
         with pytest.raises(GPTQError) as ei:
             ctx.quantize_layer(W, 4, 128, False)
         assert ei.value.status == ERR_STATE
-        # with damping the same H is fine
-        ctx.prepare(1.0, False)
+        # with enough damping the same H is positive definite: [[1,4],[4,1]] + 10*mean(diag)*I
+        ctx.prepare(10.0, False)
 
 
 def test_state_machine():
@@ -143,7 +143,8 @@ def test_quantize_layer_parity(bits, g, sym, desc_act, damp):
     assert np.array_equal(gpu["g_idx"], O.g_idx(prep["perm"], g))
     what = O.unpermute_columns(rep["what"], prep["perm"])
     scale_ref = np.repeat(rep["scales"], (layer.n if g == -1 else g), axis=1)[:, np.argsort(prep["perm"])]
-    assert np.all(np.abs(gpu["w_hat"] - what) <= 1e-5 * scale_ref + 1e-12)
+    # (u - z) * s in fp32 on the GPU vs float64 in the oracle, with scales equal to 1e-5
+    assert np.all(np.abs(gpu["w_hat"] - what) <= 2e-7 * np.abs(what) + 1e-5 * scale_ref * (1 << bits) + 1e-12)
     # layer error within 1 % of the oracle's own (un-replayed) run, measured with the exact H
     Href = O.hessian(synth.bf16_bits_to_f32(gpu["X"]))
     own = O.quantize_layer(gpu["W"].astype(np.float64), gpu["H"], bits, g, sym, damp, desc_act)
