@@ -280,10 +280,12 @@ def run_gpu(args, rank, world, local_rank):
     t_roof = max(f_path / (peak * 1e12), b_sweep / (peaks["hbm_gbs"] * 1e9))
 
     # end to end through the public API with host buffers (pinned), copies inside the timed region
-    Xh = torch.from_numpy(X_host.view(np.int16)).view(torch.bfloat16).pin_memory()
-    Wh = torch.from_numpy(W_host).pin_memory()
-    e2e_ms = e2e_run(ctx, Xh, Wh, qs, dev, stream, reps=max(1, min(3, args.steps)))
-    e2e_ms = max_over_ranks(e2e_ms, world, dev)
+    e2e_ms = None
+    if not args.no_e2e:
+        Xh = torch.from_numpy(X_host.view(np.int16)).view(torch.bfloat16).pin_memory()
+        Wh = torch.from_numpy(W_host).pin_memory()
+        e2e_ms = e2e_run(ctx, Xh, Wh, qs, dev, stream, reps=max(1, min(3, args.steps)))
+        e2e_ms = max_over_ranks(e2e_ms, world, dev)
     G_ = n // (n if qs.group_size == -1 else qs.group_size)
     d2h = m * n * qs.bits // 8 + 2 * m * G_ * 4 + 2 * n * 4
     h2d = X_host.nbytes + W_host.nbytes
@@ -307,8 +309,9 @@ def run_gpu(args, rank, world, local_rank):
             "gweights_per_s_solve": weights / ((statistics.mean(t_p) + statistics.mean(t_q)) / 1e3) / 1e9,
             "path_roofline": {"t_roof_ms": t_roof * 1e3, "frac": t_roof * 1e3 / ms_step},
             "roofline": roofline,
-            "e2e": {"value": world * weights / (e2e_ms / 1e3) / 1e9, "unit": "Gweights/s",
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "e2e": None if e2e_ms is None else {
+                "value": world * weights / (e2e_ms / 1e3) / 1e9, "unit": "Gweights/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": launches,
             "clocks": clk,
             "cpu_baseline": cpu,
@@ -377,6 +380,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default=WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the separate host-buffer end-to-end measurement")
     args = ap.parse_args()
     rank, world, local_rank = dist_env()
     if args.impl == "reference":

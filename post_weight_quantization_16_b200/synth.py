@@ -109,6 +109,15 @@ def block7b_layers():
     return out
 
 
+def _register_block7b():
+    """Name each 7B-block layer as a workload too (4-bit, asymmetric, group 128, damp 0.01, act-order)."""
+    for lay in block7b_layers():
+        WORKLOADS[f"{lay.name}_{lay.m}x{lay.n}"] = (lay, QuantSetting(4, 128, False, 0.01, True))
+
+
+_register_block7b()
+
+
 def block7b_settings():
     """bits x group_size x damp grid of the 7B block sweep (desc_act on)."""
     out = []
