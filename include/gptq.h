@@ -141,6 +141,33 @@ gptq_status gptq_destroy(gptq_ctx* ctx);
  * NULL).  Pure host function. */
 int64_t gptq_launch_count(const gptq_ctx* ctx);
 
+/* Allocation-free variant of gptq_quantize_layer for callers that cannot allocate device
+ * memory themselves (a host that owns a fixed device-memory budget, or code that must not
+ * call cudaMalloc/cudaFree, which synchronize the device).  The page has no counterpart:
+ * it is a deployment convenience, not a step of the method.
+ * It runs the S5-S7 kernels with their scratch (the fp32 working copy of W and the
+ * per-block error tile) in a fixed array compiled into this library, so it calls no
+ * cudaMalloc, cudaFree or other allocating routine:
+ *   - the array holds 2^20 fp32 working weights plus 4096 x 128 fp32 errors (6 MiB); every
+ *     GPU that loads the library keeps it until the process exits;
+ *   - limits: m <= 4096, m * n <= 2^20, 128 <= n <= 32768 with n % 128 == 0; larger requests
+ *     return GPTQ_ERR_ARG before anything is launched;
+ *   - every call shares the one array (it keeps the last call's contents; nothing in it has
+ *     to start at zero), so calls that overlap on the GPU — on different streams, or from
+ *     different host threads — race and corrupt each other; serialize them;
+ *   - the first call on a device resolves the array's device address (and raises kernel
+ *     shared-memory limits) with that device current; make that first call before any
+ *     stream capture.
+ * Inputs (device): W_fp16 [m x n] fp16, original column order; U [n x n] fp32 upper factor
+ * in sweep order (as from gptq_get_factor); perm [n] int32 (as from gptq_prepare); dead
+ * [n] uint8 (1 = dead column, weights zeroed) or NULL for none.  Outputs as in
+ * gptq_quantize_layer.  `device` is the CUDA ordinal, `cuda_stream` a cudaStream_t the
+ * kernels are enqueued on (asynchronous). */
+gptq_status gptq_quantize_layer_noalloc(const void* W_fp16, int64_t m, int64_t n, const float* U,
+                                        const int32_t* perm, const uint8_t* dead, gptq_qparams qp,
+                                        uint32_t* codes_out, float* scales_out, float* zeros_out,
+                                        int32_t* g_idx_out, float* W_hat_out, int device, void* cuda_stream);
+
 /* Static description of a status code. */
 const char* gptq_status_string(gptq_status s);
 

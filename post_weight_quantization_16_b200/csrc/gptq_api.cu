@@ -9,6 +9,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <thread>
 
 #include "../../include/gptq.h"
@@ -525,3 +526,119 @@ gptq_status gptq_destroy(gptq_ctx* c) {
 }
 
 }  // extern "C"
+
+// ==========================================================================================
+// Allocation-free quantize: gptq_quantize_layer_noalloc
+//
+// Some callers must not allocate device memory on their own: an engine or plugin host that
+// owns a fixed device-memory budget and hands out every byte itself, or code that runs where
+// cudaMalloc/cudaFree would stall other work (both synchronize the device) or are not
+// permitted at all.  For them this entry point runs the same sweep kernels as
+// gptq_quantize_layer, but its scratch (the fp32 working copy of W and the per-block error
+// tile) lives in the fixed array below, which the library's module holds on every GPU that
+// loads it, until the process exits.
+// ==========================================================================================
+namespace {
+constexpr int64_t kNoAllocMaxWeights = int64_t(1) << 20;  // m * n  (4 MiB of fp32 working weights)
+constexpr int64_t kNoAllocMaxRows = 4096;                  // m      (2 MiB of block errors)
+constexpr int kNoAllocMaxDevices = 64;
+}  // namespace
+
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocMaxWeights + kNoAllocMaxRows * SW_B];
+static __device__ __align__(256) uint8_t g_noalloc_no_dead[kMaxN];  // all zero: no dead columns
+
+namespace {
+std::mutex g_noalloc_mu;
+float* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+uint8_t* g_noalloc_nodead_ptr[kNoAllocMaxDevices] = {};
+
+// Once per device, with that device current: resolve the device addresses of the static
+// arrays (host code must not use the symbols themselves as addresses) and raise the
+// dynamic shared-memory limits of the kernels this path launches.  Allocates nothing.
+gptq_status noalloc_setup(int device, float** scratch, uint8_t** nodead) {
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[device]) {
+    void* p = nullptr;
+    void* q = nullptr;
+    CK(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+    CK(cudaGetSymbolAddress(&q, g_noalloc_no_dead));
+    CK(cudaFuncSetAttribute(sweep_block_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, SW_SMEM));
+    CK(cudaFuncSetAttribute(sweep_block_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, SW_SMEM));
+    CK(cudaFuncSetAttribute(sweep_block_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, SW_SMEM));
+    CK(cudaFuncSetAttribute(init_w_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                            static_cast<int>(kMaxN * 2)));
+    g_noalloc_nodead_ptr[device] = static_cast<uint8_t*>(q);
+    g_noalloc_ptr[device] = static_cast<float*>(p);
+  }
+  *scratch = g_noalloc_ptr[device];
+  *nodead = g_noalloc_nodead_ptr[device];
+  return GPTQ_OK;
+}
+}  // namespace
+
+extern "C" gptq_status gptq_quantize_layer_noalloc(const void* W, int64_t m, int64_t n, const float* U,
+                                                   const int32_t* perm, const uint8_t* dead, gptq_qparams qp,
+                                                   uint32_t* codes, float* scales, float* zeros, int32_t* g_idx,
+                                                   float* W_hat, int device, void* cuda_stream) {
+  if (!W || !U || !perm || !codes || !scales || !zeros) return GPTQ_ERR_ARG;
+  if (n < 128 || n > kMaxN || n % 128 || m < 1) return GPTQ_ERR_ARG;
+  if (m > kNoAllocMaxRows || m * n > kNoAllocMaxWeights) return GPTQ_ERR_ARG;  // beyond the fixed scratch
+  if (!valid_qparams(qp, n)) return GPTQ_ERR_ARG;
+  if (!aligned16(U) || !aligned16(codes) || (W_hat && !aligned16(W_hat))) return GPTQ_ERR_ARG;
+  if (device < 0 || device >= kNoAllocMaxDevices) return GPTQ_ERR_ARG;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || device >= ndev) {
+    cudaGetLastError();
+    return GPTQ_ERR_CUDA;
+  }
+  DeviceGuard dg(device);
+  float* scratch = nullptr;
+  uint8_t* nodead = nullptr;
+  gptq_status s = noalloc_setup(device, &scratch, &nodead);
+  if (s != GPTQ_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  const int ni = static_cast<int>(n), mi = static_cast<int>(m);
+  const int g = (qp.group_size == -1) ? ni : qp.group_size;
+  float* Wq = scratch;                       // [m x n]
+  float* Err = scratch + kNoAllocMaxWeights; // [m x 128]
+  init_w_kernel<<<mi, 256, static_cast<size_t>(ni) * 2, st>>>(static_cast<const __half*>(W), ni, perm,
+                                                             dead ? dead : nodead, Wq);
+  CKL("noalloc init_w");
+  SweepArgs a;
+  a.Wq = Wq;
+  a.U = U;
+  a.Err = Err;
+  a.codes = codes;
+  a.scales = scales;
+  a.zeros = zeros;
+  a.W_hat = W_hat;
+  a.perm = perm;
+  a.m = mi;
+  a.n = ni;
+  a.bits = qp.bits;
+  a.sym = qp.sym;
+  a.g = g;
+  a.G = ni / g;
+  const int grid = (mi + SW_THREADS - 1) / SW_THREADS;
+  for (int i1 = 0; i1 < ni; i1 += SW_B) {
+    if (g >= SW_B)
+      sweep_block_kernel<0><<<grid, SW_THREADS, SW_SMEM, st>>>(a, i1);
+    else if (g == 64)
+      sweep_block_kernel<64><<<grid, SW_THREADS, SW_SMEM, st>>>(a, i1);
+    else
+      sweep_block_kernel<32><<<grid, SW_THREADS, SW_SMEM, st>>>(a, i1);
+    CKL("noalloc sweep");
+    const int i2 = i1 + SW_B;
+    if (i2 < ni) {
+      dim3 gg((ni - i2 + SG_BN - 1) / SG_BN, (mi + SG_BM - 1) / SG_BM);
+      sgemm_kernel<false><<<gg, SG_THREADS, 0, st>>>(mi, ni - i2, SW_B, -1.f, Err, SW_B,
+                                                     U + static_cast<size_t>(i1) * ni + i2, ni, 1.f, Wq + i2, ni, 0);
+      CKL("noalloc trailing");
+    }
+  }
+  if (g_idx) {
+    g_idx_kernel<<<(ni + 255) / 256, 256, 0, st>>>(perm, ni, g, g_idx);
+    CKL("noalloc g_idx");
+  }
+  return GPTQ_OK;
+}

@@ -51,6 +51,8 @@ _SIGS = {
     "gptq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "gptq_set_hessian_chunk": (ctypes.c_int, [_P, ctypes.c_int64]),
     "gptq_launch_count": (ctypes.c_int64, [_P]),
+    "gptq_quantize_layer_noalloc": (ctypes.c_int, [_P, ctypes.c_int64, ctypes.c_int64, _P, _P, _P, QParams,
+                                                   _P, _P, _P, _P, _P, ctypes.c_int, _P]),
 }
 
 
