@@ -36,6 +36,30 @@ METRIC = "GPTQ layer quant: Gweights/s + Hessian TFLOP/s, % of roofline, 1×B200
 WORKLOAD = "q_proj_4096x4096"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant kernel from one
+# ncu capture (profiles/hessian_syrk_kernel__block7b_q_65536tok_x4096.md), valid only while the
+# kernel's sources are the ones captured.  The capture ran 65536 tokens; X traffic grows in
+# proportion to the tokens, so it is scaled per token to a full launch.
+PROFILED_TRAFFIC = {
+    "hessian_syrk_kernel": {
+        "sources": {"post_weight_quantization_16_b200/csrc/hessian_tc.cuh": "e16be80c005318b5027207506433bafdc3b624a9",
+                    "post_weight_quantization_16_b200/csrc/sm100_ptx.cuh": "3becefca78c60eb64f9140ee7762b602f76919e6"},
+        "n": 4096, "tokens": 65536, "dram_bytes": 975.429376e6 + 23.913216e6,
+    },
+}
+
+
+def profiled_traffic(kernel: str, n: int, n_tok: int):
+    import hashlib
+    rec = PROFILED_TRAFFIC.get(kernel)
+    if rec is None or rec["n"] != n:
+        return None
+    for path, sha in rec["sources"].items():
+        with open(os.path.join(ROOT, path), "rb") as f:
+            if hashlib.sha1(f.read()).hexdigest() != sha:
+                return None
+    return rec["dram_bytes"] * n_tok / rec["tokens"]
+
 
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -95,7 +119,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
         except (OSError, FileNotFoundError):
@@ -269,12 +293,12 @@ def run_gpu(args, rank, world, local_rank):
     h_flops = layer.n_tok * layer.n * (layer.n + 1)           # algorithmic: upper triangle incl. diagonal
     h_tflops = h_flops / (h_ms / 1e3) / 1e12
     peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    n, m = layer.n, layer.m
     roofline = {"bound": "tensor", "kernel": "hessian_syrk_kernel", "achieved": h_tflops, "peak": peak,
-                "unit": "TFLOP/s", "frac": h_tflops / peak, "traffic": None,
+                "unit": "TFLOP/s", "frac": h_tflops / peak, "traffic": profiled_traffic("hessian_syrk_kernel", n, layer.n_tok),
                 "peak_source": f"{peaks_src} bf16 dense, sustained", "algorithmic_flops_per_launch": h_flops}
 
     # whole-path roofline: contraction flops at the bf16 peak vs the sweep's bytes at HBM bandwidth
-    n, m = layer.n, layer.m
     f_path = layer.n_tok * n * (n + 1) + 2 * n ** 3 / 3 + 2 * m * sum(128 * (n - i2) for i2 in range(128, n, 128))
     b_sweep = 2 * m * n + 2 * n * (n + 1) + m * n * qs.bits / 8 + 8 * m * n / qs.group_size + 8 * n
     t_roof = max(f_path / (peak * 1e12), b_sweep / (peaks["hbm_gbs"] * 1e9))
@@ -375,8 +399,8 @@ def e2e_run(ctx, Xh, Wh, qs, dev, stream, reps=2, batch_tokens=16384):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
-    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--steps", type=int, default=60)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default=WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -1,0 +1,35 @@
+/*
+ * gptq_testing.h — test hooks of libgptq.  Not part of the method's interface: they expose
+ * internal kernels so that the test-suite can check them in isolation.
+ */
+#ifndef GPTQ_B200_TESTING_H
+#define GPTQ_B200_TESTING_H
+
+#include "gptq.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* The three-product tf32 tensor-core GEMM of the factorization and of the lazy trailing
+ * update (S4, S6):  C = alpha * A * B^T (+ C when beta = 1).
+ *   A_hi/A_lo : device fp32 [M x K], leading dimension lda (A = A_hi + A_lo; hi/lo are tf32 values)
+ *   B_hi/B_lo : device fp32 [N x K], leading dimension ldb
+ *   k_lo_mode : 0 = K from 0; 1 = K from the first column of the output tile (B lower-triangular
+ *               in this form); 2 = K from the first row of the tile (A upper-triangular)
+ *   k_hi_mode : 0 = K to the end; 1 = K up to the last column of the tile (B upper-triangular)
+ *   upper_only: skip output tiles wholly below the diagonal of C
+ *   C         : fp32 output [M x N] (ldc) or NULL; C_hi/C_lo: hi/lo output (ldh) or NULL;
+ *   Ct_hi/Ct_lo: transposed hi/lo output [N x M] (ldt) or NULL (beta applies to C and C_hi/C_lo).
+ * Requirements: N % 32 == 0, K % 32 == 0, 16-byte aligned bases, leading dimensions % 4 == 0.
+ * Synchronizes the stream before returning.  Allocates a 4-byte status word (stream-ordered). */
+gptq_status gptq_test_gemm_tf32x3(int M, int N, int K, const float* A_hi, const float* A_lo, int lda, const float* B_hi,
+                                  const float* B_lo, int ldb, float alpha, int beta, int k_lo_mode, int k_hi_mode,
+                                  int upper_only, float* C, int ldc, float* C_hi, float* C_lo, int ldh, float* Ct_hi,
+                                  float* Ct_lo, int ldt, int device, void* cuda_stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GPTQ_B200_TESTING_H */

@@ -1,0 +1,281 @@
+// gemm_tc.cuh — fp32-faithful GEMM on the sm_100a tensor cores (three tf32 products).
+//
+//   C = alpha * A * B^T (+ C)      A [M x K] row-major, B [N x K] row-major (both K-major)
+//
+// Used by the factorization (its Schur-complement, panel and inverse products) and by the
+// lazy trailing update of the column sweep (W[:, i2:] -= Err * U[blk, i2:]).  Each operand
+// X is stored as two arrays X_hi = rn_tf32(X) and X_lo = rn_tf32(X - X_hi); the product is
+// A_hi B_hi + A_hi B_lo + A_lo B_hi, about 2^-21 relative per term, close to fp32.  The
+// tensor cores' own accumulation is not round-to-nearest, so every 32-wide K stage is
+// accumulated in its own TMEM buffer and then added into fp32 registers with
+// round-to-nearest adds (double-buffered TMEM, as in the Hessian kernel).
+//
+// Tile 128 x 256 (tcgen05.mma kind::tf32, M=128, N=256, K=8), 2-stage TMA ring of 96 KB
+// stages (A_hi, A_lo, B_hi, B_lo; 128-byte swizzle), warp roles:
+//   warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer, warps 2-9 epilogue.
+// Triangular operands: the K range of a tile can start at its first column (B lower in
+// K-major form) or its first row (A upper), or stop after its last column (B upper), so
+// the zero halves of triangular factors are skipped; tiles wholly below the diagonal of C
+// can be skipped for symmetric updates.
+// Outputs (any subset): plain fp32 C (optionally + C), hi/lo pair (optionally + hi+lo), and a
+// transposed hi/lo pair (coalesced: the 32 lanes of a warp write 32 consecutive rows).
+#pragma once
+
+#include "sm100_ptx.cuh"
+
+namespace gptq {
+
+constexpr int GT_BM = 128, GT_BN = 256, GT_BK = 32, GT_STAGES = 2;
+constexpr int GT_A_BYTES = GT_BM * GT_BK * 4;  // 16 KB
+constexpr int GT_B_BYTES = GT_BN * GT_BK * 4;  // 32 KB
+constexpr int GT_STAGE_BYTES = 2 * GT_A_BYTES + 2 * GT_B_BYTES;
+constexpr int GT_THREADS = 64 + 256;
+constexpr int GT_SMEM = GT_STAGES * GT_STAGE_BYTES + 256 + 1024;
+
+enum : int { GT_KLO_NONE = 0, GT_KLO_COL = 1, GT_KLO_ROW = 2 };
+enum : int { GT_KHI_NONE = 0, GT_KHI_COL = 1 };
+
+struct GemmTCArgs {
+  int M, N, K;
+  float alpha;
+  int beta;          // 0 or 1: add the existing C (plain or hi+lo)
+  int k_lo_mode, k_hi_mode, upper_only;
+  float* C;          // plain fp32 output (or nullptr)
+  int ldc;
+  float* Chi;        // hi/lo output (or nullptr)
+  float* Clo;
+  int ldh;
+  float* Cthi;       // transposed hi/lo output (or nullptr): Ct[c][r]
+  float* Ctlo;
+  int ldt;
+  int* status;
+};
+
+__device__ __forceinline__ float tf32_rn(float x) {
+  uint32_t u = __float_as_uint(x);
+  u += 0xFFFu + ((u >> 13) & 1u);
+  return __uint_as_float(u & 0xFFFFE000u);
+}
+
+__global__ void __launch_bounds__(GT_THREADS, 1)
+    gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_constant__ CUtensorMap a_lo,
+                       const __grid_constant__ CUtensorMap b_hi, const __grid_constant__ CUtensorMap b_lo,
+                       GemmTCArgs p) {
+  extern __shared__ uint8_t gt_smem_raw[];
+  const uint32_t raw_s = smem_u32(gt_smem_raw);
+  uint8_t* smem = gt_smem_raw + (((raw_s + 1023u) & ~1023u) - raw_s);
+  const uint32_t sbase = smem_u32(smem);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int m0 = blockIdx.y * GT_BM;
+  const int n0 = blockIdx.x * GT_BN;
+  if (p.upper_only && m0 >= n0 + GT_BN) return;  // uniform, before any barrier or TMEM use
+
+  int k_begin = 0, k_end = p.K;
+  if (p.k_lo_mode == GT_KLO_COL) k_begin = n0;
+  if (p.k_lo_mode == GT_KLO_ROW) k_begin = m0;
+  if (p.k_hi_mode == GT_KHI_COL) k_end = min(p.K, n0 + GT_BN);
+  k_begin = (k_begin / GT_BK) * GT_BK;
+  const int n_iters = (k_end > k_begin) ? (k_end - k_begin + GT_BK - 1) / GT_BK : 0;
+
+  const uint32_t bar_full = sbase + GT_STAGES * GT_STAGE_BYTES;
+  const uint32_t bar_empty = bar_full + 8 * GT_STAGES;
+  const uint32_t bar_tfull = bar_empty + 8 * GT_STAGES;
+  const uint32_t bar_tempty = bar_tfull + 16;
+  const uint32_t bar_drain = bar_tempty + 16;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + GT_STAGES * GT_STAGE_BYTES + 8 * (2 * GT_STAGES + 5));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < GT_STAGES; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_tfull + 8 * b, 1);
+      mbar_init(bar_tempty + 8 * b, 8 * 32);
+    }
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&a_hi);
+    tma_prefetch_desc(&a_lo);
+    tma_prefetch_desc(&b_hi);
+    tma_prefetch_desc(&b_lo);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      int issued = 0;
+      for (int it = 0; it < n_iters; ++it) {
+        const int s = it % GT_STAGES;
+        const uint32_t ph = static_cast<uint32_t>(it / GT_STAGES) & 1u;
+        if (!mbar_wait_bounded(bar_empty + 8 * s, ph ^ 1u, abort_flag)) break;
+        const uint32_t fb = bar_full + 8 * s;
+        mbar_arrive_expect_tx(fb, GT_STAGE_BYTES);
+        const uint32_t st = sbase + s * GT_STAGE_BYTES;
+        const int k = k_begin + it * GT_BK;
+        tma_load_2d(st, &a_hi, fb, k, m0);
+        tma_load_2d(st + GT_A_BYTES, &a_lo, fb, k, m0);
+        tma_load_2d(st + 2 * GT_A_BYTES, &b_hi, fb, k, n0);
+        tma_load_2d(st + 2 * GT_A_BYTES + GT_B_BYTES, &b_lo, fb, k, n0);
+        issued = it + 1;
+      }
+      for (int it = max(0, issued - GT_STAGES); it < issued; ++it)
+        mbar_wait_drain(bar_full + 8 * (it % GT_STAGES), static_cast<uint32_t>(it / GT_STAGES) & 1u);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer: one TMEM buffer per K stage ----------------
+      constexpr uint32_t idesc = idesc_make(2u, 2u, 0u, 0u, GT_BM, GT_BN);  // tf32, K-major A and B
+      bool ok = true;
+      for (int it = 0; it < n_iters; ++it) {
+        const int b = it & 1;
+        const uint32_t ph = static_cast<uint32_t>(it >> 1) & 1u;
+        if (!mbar_wait_bounded(bar_tempty + 8 * b, ph ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const int s = it % GT_STAGES;
+        const uint32_t phs = static_cast<uint32_t>(it / GT_STAGES) & 1u;
+        if (!mbar_wait_bounded(bar_full + 8 * s, phs, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * GT_BN);
+        const uint32_t st = sbase + s * GT_STAGE_BYTES;
+        const uint32_t sa_hi = st, sa_lo = st + GT_A_BYTES;
+        const uint32_t sb_hi = st + 2 * GT_A_BYTES, sb_lo = sb_hi + GT_B_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < GT_BK / 8; ++kk) {
+          const uint32_t off = kk * 32;  // 8 fp32 of K inside the 128-byte swizzle row
+          const uint64_t dah = sdesc_sw128(sa_hi + off, 16, 1024), dal = sdesc_sw128(sa_lo + off, 16, 1024);
+          const uint64_t dbh = sdesc_sw128(sb_hi + off, 16, 1024), dbl = sdesc_sw128(sb_lo + off, 16, 1024);
+          umma_tf32(d_tmem, dal, dbh, idesc, kk > 0 ? 1u : 0u);
+          umma_tf32(d_tmem, dah, dbl, idesc, 1u);
+          umma_tf32(d_tmem, dah, dbh, idesc, 1u);
+        }
+        umma_commit(bar_empty + 8 * s);
+        umma_commit(bar_tfull + 8 * b);
+      }
+      if (!ok) {
+        umma_commit(bar_drain);
+        mbar_wait_drain(bar_drain, 0);
+      }
+    }
+  } else {
+    // ---------------- epilogue ----------------
+    const int q = warp & 3;
+    const int hh = (warp - 2) >> 2;
+    const int r = m0 + q * 32 + lane;
+    const int cbase = n0 + hh * (GT_BN / 2);
+    float acc[GT_BN / 2];
+#pragma unroll
+    for (int j = 0; j < GT_BN / 2; ++j) acc[j] = 0.0f;
+    bool all_ok = true;
+    for (int it = 0; it < n_iters; ++it) {
+      const int b = it & 1;
+      const uint32_t ph = static_cast<uint32_t>(it >> 1) & 1u;
+      int ok = 0;
+      if (lane == 0) ok = mbar_wait_bounded(bar_tfull + 8 * b, ph, abort_flag) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) {
+        all_ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                               static_cast<uint32_t>(b * GT_BN + hh * (GT_BN / 2) + cc * 32),
+                           v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) acc[cc * 32 + j] += __uint_as_float(v[j]);
+      }
+      tc_fence_before();
+      mbar_arrive(bar_tempty + 8 * b);
+    }
+    if (all_ok) {
+      const bool row_ok = r < p.M;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        const int c0 = cbase + cc * 32;
+        if (c0 >= p.N) continue;  // N % 32 == 0: whole 32-column groups
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = p.alpha * acc[cc * 32 + j];
+        if (row_ok && p.C) {
+          float4* cp = reinterpret_cast<float4*>(p.C + static_cast<size_t>(r) * p.ldc + c0);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            float4 o = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+            if (p.beta) {
+              const float4 c = cp[j];
+              o.x += c.x;
+              o.y += c.y;
+              o.z += c.z;
+              o.w += c.w;
+            }
+            cp[j] = o;
+          }
+        }
+        if (row_ok && p.Chi) {
+          float4* hp = reinterpret_cast<float4*>(p.Chi + static_cast<size_t>(r) * p.ldh + c0);
+          float4* lp = reinterpret_cast<float4*>(p.Clo + static_cast<size_t>(r) * p.ldh + c0);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            float x[4] = {v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]};
+            if (p.beta) {
+              const float4 h = hp[j], l = lp[j];
+              x[0] += h.x + l.x;
+              x[1] += h.y + l.y;
+              x[2] += h.z + l.z;
+              x[3] += h.w + l.w;
+            }
+            float hi[4], lo[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              hi[e] = tf32_rn(x[e]);
+              lo[e] = tf32_rn(x[e] - hi[e]);
+            }
+            hp[j] = make_float4(hi[0], hi[1], hi[2], hi[3]);
+            lp[j] = make_float4(lo[0], lo[1], lo[2], lo[3]);
+          }
+        }
+        if (row_ok && p.Cthi) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float hi = tf32_rn(v[j]);
+            const size_t o = static_cast<size_t>(c0 + j) * p.ldt + r;
+            p.Cthi[o] = hi;
+            p.Ctlo[o] = tf32_rn(v[j] - hi);
+          }
+        }
+      }
+    }
+  }
+
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) atomicOr(p.status, ST_TIMEOUT);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+}  // namespace gptq

@@ -13,7 +13,9 @@
 #include <thread>
 
 #include "../../include/gptq.h"
+#include "../../include/gptq_testing.h"
 #include "factor_kernels.cuh"
+#include "gemm_tc.cuh"
 #include "hessian_tc.cuh"
 #include "prepare_kernels.cuh"
 #include "sgemm_simt.cuh"
@@ -34,13 +36,13 @@ struct gptq_ctx {
   int device = 0;
   cudaStream_t stream = nullptr;
   int64_t n = 0, m_max = 0;
-  float* H = nullptr;    // [n x n] accumulated Hessian (upper triangle valid until mirrored)
-  float* A = nullptr;    // [n x n] damped, permuted H (consumed by the factorization)
-  float* V = nullptr;    // [n x n] reverse Cholesky factor
-  float* U = nullptr;    // [n x n] U = V^-1
-  float* T = nullptr;    // [n/2 x n/2 + slack] temporary of the inverse recursion
-  float* Wq = nullptr;   // [m_max x n] fp32 working weights
-  float* Err = nullptr;  // [m_max x 128]
+  float* H = nullptr;                          // [n x n] accumulated Hessian (upper triangle until mirrored)
+  float *A_hi = nullptr, *A_lo = nullptr;      // [n x n] damped, permuted H; Schur complements
+  float *VT_hi = nullptr, *VT_lo = nullptr;    // [n x n] V12 blocks (upper) and T^T blocks (lower)
+  float *U_hi = nullptr, *U_lo = nullptr;      // [n x n] U (upper)
+  float *Ut_hi = nullptr, *Ut_lo = nullptr;    // [n x n] U^T
+  float* Wq = nullptr;                         // [m_max x n] fp32 working weights
+  float *Err_hi = nullptr, *Err_lo = nullptr;  // [m_max x 128]
   float* keys = nullptr;
   uint8_t* dead = nullptr;
   int32_t* perm = nullptr;
@@ -68,8 +70,6 @@ gptq_status cuda_fail(cudaError_t e, const char* what) {
     if (_s != GPTQ_OK) return _s;                        \
   } while (0)
 #define CKL(what) CK(cudaGetLastError())
-
-size_t t_elems(int64_t n) { return static_cast<size_t>((n / 2 + FB_NB) * (n / 2 + FB_NB)); }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -139,53 +139,119 @@ gptq_status status_from_flags(int f) {
   return GPTQ_OK;
 }
 
-gptq_status sgemm(gptq_ctx* c, bool transB, int M, int N, int K, float alpha, const float* A, int lda,
-                  const float* B, int ldb, float beta, float* C, int ldc, bool upper_only) {
+// 2-D fp32 tensor map of a row-major sub-matrix (rows x cols, leading dimension ld), boxes of
+// 32 columns x box_rows rows, 128-byte swizzle.
+gptq_status make_map(gptq_ctx* c, CUtensorMap* map, const float* base, int64_t rows, int64_t cols, int64_t ld,
+                     int box_rows) {
+  if (!aligned16(base) || ld % 4 || cols % GT_BK) return GPTQ_ERR_ARG;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 4};
+  const cuuint32_t box[2] = {GT_BK, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = c->encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? GPTQ_OK : GPTQ_ERR_CUDA;
+}
+
+// C (+)= alpha * A B^T on the tensor cores, operands as tf32 hi/lo pairs (gemm_tc.cuh).
+struct TcOut {
+  float* C = nullptr;
+  int ldc = 0;
+  float* Chi = nullptr;
+  float* Clo = nullptr;
+  int ldh = 0;
+  float* Cthi = nullptr;
+  float* Ctlo = nullptr;
+  int ldt = 0;
+};
+
+gptq_status gemm_tc(gptq_ctx* c, int M, int N, int K, const float* Ahi, const float* Alo, int lda, const float* Bhi,
+                    const float* Blo, int ldb, float alpha, int beta, int klo, int khi, int upper, const TcOut& o) {
   if (M <= 0 || N <= 0) return GPTQ_OK;
-  if (K % SG_BK || N % 4 || lda % 4 || ldb % 4 || ldc % 4 || !aligned16(A) || !aligned16(B) || !aligned16(C))
-    return GPTQ_ERR_ARG;
-  if (K == 0) return GPTQ_OK;
-  dim3 grid((N + SG_BN - 1) / SG_BN, (M + SG_BM - 1) / SG_BM);
-  cudaStream_t st = c->stream;
+  if (N % 32 || K % GT_BK) return GPTQ_ERR_ARG;
+  CUtensorMap ma_hi, ma_lo, mb_hi, mb_lo;
+  gptq_status s;
+  if ((s = make_map(c, &ma_hi, Ahi, M, K, lda, GT_BM)) != GPTQ_OK) return s;
+  if ((s = make_map(c, &ma_lo, Alo, M, K, lda, GT_BM)) != GPTQ_OK) return s;
+  if ((s = make_map(c, &mb_hi, Bhi, N, K, ldb, GT_BN)) != GPTQ_OK) return s;
+  if ((s = make_map(c, &mb_lo, Blo, N, K, ldb, GT_BN)) != GPTQ_OK) return s;
+  GemmTCArgs a;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.alpha = alpha;
+  a.beta = beta;
+  a.k_lo_mode = klo;
+  a.k_hi_mode = khi;
+  a.upper_only = upper;
+  a.C = o.C;
+  a.ldc = o.ldc;
+  a.Chi = o.Chi;
+  a.Clo = o.Clo;
+  a.ldh = o.ldh;
+  a.Cthi = o.Cthi;
+  a.Ctlo = o.Ctlo;
+  a.ldt = o.ldt;
+  a.status = c->status;
+  dim3 grid((N + GT_BN - 1) / GT_BN, (M + GT_BM - 1) / GT_BM);
+  gemm_tf32x3_kernel<<<grid, GT_THREADS, GT_SMEM, c->stream>>>(ma_hi, ma_lo, mb_hi, mb_lo, a);
   ++c->launches;
-  if (transB)
-    sgemm_kernel<true><<<grid, SG_THREADS, 0, st>>>(M, N, K, alpha, A, lda, B, ldb, beta, C, ldc, upper_only ? 1 : 0);
-  else
-    sgemm_kernel<false><<<grid, SG_THREADS, 0, st>>>(M, N, K, alpha, A, lda, B, ldb, beta, C, ldc, upper_only ? 1 : 0);
-  CKL("sgemm");
+  CKL("gemm_tc");
   return GPTQ_OK;
 }
 
-// [V,U] of the diagonal block [o, o+h) of A (h a multiple of FB_NB).
+// U (and U^T) of the diagonal block [o, o+h) of A, h a multiple of the 128-column leaf.
 gptq_status chol_inv(gptq_ctx* c, int o, int h) {
   const int n = static_cast<int>(c->n);
-  if (h <= FB_NB) {
-    chol_inv_base_kernel<<<1, FB_THREADS, 0, c->stream>>>(c->A, c->V, c->U, n, o, c->status);
+  if (h <= LF_NB) {
+    leaf_chol_inv_kernel<<<1, LF_THREADS, LF_SMEM, c->stream>>>(c->A_hi, c->A_lo, n, o, c->U_hi, c->U_lo, c->Ut_hi,
+                                                               c->Ut_lo, c->status);
     ++c->launches;
-    CKL("chol_inv_base");
+    CKL("leaf_chol_inv");
     return GPTQ_OK;
   }
-  const int h2 = ((h / FB_NB) / 2) * FB_NB;
+  const int h2 = ((h / LF_NB) / 2) * LF_NB;
   const int h1 = h - h2;
   const int o2 = o + h1;
-  gptq_status s;
   auto at = [n](float* M, int r, int col) { return M + static_cast<size_t>(r) * n + col; };
+  gptq_status s;
   if ((s = chol_inv(c, o2, h2)) != GPTQ_OK) return s;
-  // V12 = A12 U22^T
-  if ((s = sgemm(c, true, h1, h2, h2, 1.f, at(c->A, o, o2), n, at(c->U, o2, o2), n, 0.f, at(c->V, o, o2), n,
-                 false)) != GPTQ_OK)
+  // V12 = A12 U22^T                      (U22 rows are the K-major B; k >= column)
+  TcOut v12;
+  v12.Chi = at(c->VT_hi, o, o2);
+  v12.Clo = at(c->VT_lo, o, o2);
+  v12.ldh = n;
+  if ((s = gemm_tc(c, h1, h2, h2, at(c->A_hi, o, o2), at(c->A_lo, o, o2), n, at(c->U_hi, o2, o2), at(c->U_lo, o2, o2),
+                   n, 1.f, 0, GT_KLO_COL, GT_KHI_NONE, 0, v12)) != GPTQ_OK)
     return s;
-  // A11 -= V12 V12^T (upper tiles)
-  if ((s = sgemm(c, true, h1, h1, h2, -1.f, at(c->V, o, o2), n, at(c->V, o, o2), n, 1.f, at(c->A, o, o), n,
-                 true)) != GPTQ_OK)
+  // A11 -= V12 V12^T                     (upper tiles only)
+  TcOut a11;
+  a11.Chi = at(c->A_hi, o, o);
+  a11.Clo = at(c->A_lo, o, o);
+  a11.ldh = n;
+  if ((s = gemm_tc(c, h1, h1, h2, at(c->VT_hi, o, o2), at(c->VT_lo, o, o2), n, at(c->VT_hi, o, o2),
+                   at(c->VT_lo, o, o2), n, -1.f, 1, GT_KLO_NONE, GT_KHI_NONE, 1, a11)) != GPTQ_OK)
+    return s;
+  // T^T = (V12 U22)^T into the lower block [o2.., o..]   (Ut22 rows as B; k <= column)
+  TcOut tt;
+  tt.Cthi = at(c->VT_hi, o2, o);
+  tt.Ctlo = at(c->VT_lo, o2, o);
+  tt.ldt = n;
+  if ((s = gemm_tc(c, h1, h2, h2, at(c->VT_hi, o, o2), at(c->VT_lo, o, o2), n, at(c->Ut_hi, o2, o2),
+                   at(c->Ut_lo, o2, o2), n, 1.f, 0, GT_KLO_NONE, GT_KHI_COL, 0, tt)) != GPTQ_OK)
     return s;
   if ((s = chol_inv(c, o, h1)) != GPTQ_OK) return s;
-  // T = V12 U22 ; U12 = -U11 T
-  if ((s = sgemm(c, false, h1, h2, h2, 1.f, at(c->V, o, o2), n, at(c->U, o2, o2), n, 0.f, c->T, h2, false)) !=
-      GPTQ_OK)
-    return s;
-  if ((s = sgemm(c, false, h1, h2, h1, -1.f, at(c->U, o, o), n, c->T, h2, 0.f, at(c->U, o, o2), n, false)) !=
-      GPTQ_OK)
+  // U12 = -U11 T  (and Ut21 = U12^T)      (U11 rows as A; k >= row)
+  TcOut u12;
+  u12.Chi = at(c->U_hi, o, o2);
+  u12.Clo = at(c->U_lo, o, o2);
+  u12.ldh = n;
+  u12.Cthi = at(c->Ut_hi, o2, o);
+  u12.Ctlo = at(c->Ut_lo, o2, o);
+  u12.ldt = n;
+  if ((s = gemm_tc(c, h1, h2, h1, at(c->U_hi, o, o), at(c->U_lo, o, o), n, at(c->VT_hi, o2, o), at(c->VT_lo, o2, o),
+                   n, -1.f, 0, GT_KLO_ROW, GT_KHI_NONE, 0, u12)) != GPTQ_OK)
     return s;
   return GPTQ_OK;
 }
@@ -200,7 +266,8 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 }
 
 void free_all(gptq_ctx* c) {
-  float** fs[] = {&c->H, &c->A, &c->V, &c->U, &c->T, &c->Wq, &c->Err, &c->keys};
+  float** fs[] = {&c->H,     &c->A_hi,  &c->A_lo,  &c->VT_hi, &c->VT_lo,  &c->U_hi,   &c->U_lo,
+                  &c->Ut_hi, &c->Ut_lo, &c->Wq,    &c->Err_hi, &c->Err_lo, &c->keys};
   for (float** p : fs)
     if (*p) {
       cudaFree(*p);
@@ -248,10 +315,9 @@ const char* gptq_status_string(gptq_status s) {
 size_t gptq_workspace_bytes(int64_t n, int64_t m_max) {
   if (n < 128 || n > kMaxN || n % 128 || m_max < 1 || m_max > kMaxM) return 0;
   const size_t nn = static_cast<size_t>(n) * static_cast<size_t>(n);
-  size_t b = 4 * nn * sizeof(float);                                  // H, A, V, U
-  b += t_elems(n) * sizeof(float);                                    // T
-  b += static_cast<size_t>(m_max) * static_cast<size_t>(n) * sizeof(float);   // Wq
-  b += static_cast<size_t>(m_max) * SW_B * sizeof(float);             // Err
+  size_t b = 9 * nn * sizeof(float);                                              // H, A, VT, U, Ut (hi/lo)
+  b += static_cast<size_t>(m_max) * static_cast<size_t>(n) * sizeof(float);       // Wq
+  b += 2 * static_cast<size_t>(m_max) * SW_B * sizeof(float);                     // Err hi/lo
   b += static_cast<size_t>(n) * (sizeof(float) + 1 + sizeof(int32_t)) + sizeof(double) + sizeof(int);
   return b;
 }
@@ -290,12 +356,11 @@ gptq_status gptq_create(gptq_ctx** out, int64_t n, int64_t m_max, int device, vo
     if (e == cudaSuccess) e = cudaMalloc(p, bytes);
   };
   alloc(reinterpret_cast<void**>(&c->H), nn * 4);
-  alloc(reinterpret_cast<void**>(&c->A), nn * 4);
-  alloc(reinterpret_cast<void**>(&c->V), nn * 4);
-  alloc(reinterpret_cast<void**>(&c->U), nn * 4);
-  alloc(reinterpret_cast<void**>(&c->T), t_elems(n) * 4);
+  for (float** p : {&c->A_hi, &c->A_lo, &c->VT_hi, &c->VT_lo, &c->U_hi, &c->U_lo, &c->Ut_hi, &c->Ut_lo})
+    alloc(reinterpret_cast<void**>(p), nn * 4);
   alloc(reinterpret_cast<void**>(&c->Wq), static_cast<size_t>(m_max) * n * 4);
-  alloc(reinterpret_cast<void**>(&c->Err), static_cast<size_t>(m_max) * SW_B * 4);
+  alloc(reinterpret_cast<void**>(&c->Err_hi), static_cast<size_t>(m_max) * SW_B * 4);
+  alloc(reinterpret_cast<void**>(&c->Err_lo), static_cast<size_t>(m_max) * SW_B * 4);
   alloc(reinterpret_cast<void**>(&c->keys), n * 4);
   alloc(reinterpret_cast<void**>(&c->dead), n);
   alloc(reinterpret_cast<void**>(&c->perm), n * 4);
@@ -309,6 +374,10 @@ gptq_status gptq_create(gptq_ctx** out, int64_t n, int64_t m_max, int device, vo
     return (e == cudaErrorMemoryAllocation) ? GPTQ_ERR_OOM : GPTQ_ERR_CUDA;
   }
   e = cudaFuncSetAttribute(hessian_syrk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, HS_SMEM);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(gemm_tf32x3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GT_SMEM);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(leaf_chol_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, LF_SMEM);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(sweep_block_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, SW_SMEM);
   if (e == cudaSuccess)
@@ -415,12 +484,11 @@ gptq_status gptq_prepare(gptq_ctx* c, double damp, int desc_act, int32_t* perm_o
   ++c->launches;
   CKL("perm");
   gather_damp_kernel<<<n, 256, static_cast<size_t>(n) * 4, c->stream>>>(c->H, n, c->perm, c->keys, c->mean, damp,
-                                                                        c->A);
+                                                                        c->A_hi, c->A_lo);
   ++c->launches;
   CKL("gather");
   const size_t nn = static_cast<size_t>(n) * n;
-  CK(cudaMemsetAsync(c->U, 0, nn * 4, c->stream));
-  CK(cudaMemsetAsync(c->V, 0, nn * 4, c->stream));
+  for (float* p : {c->U_hi, c->U_lo, c->Ut_hi, c->Ut_lo}) CK(cudaMemsetAsync(p, 0, nn * 4, c->stream));
   if ((s = chol_inv(c, 0, n)) != GPTQ_OK) return s;
   if (perm_out) CK(cudaMemcpyAsync(perm_out, c->perm, n * 4, cudaMemcpyDeviceToDevice, c->stream));
   int flags = 0;
@@ -434,7 +502,10 @@ gptq_status gptq_get_factor(gptq_ctx* c, float* U_out) {
   if (!c || !U_out) return GPTQ_ERR_ARG;
   if (c->state != ST_PREPARED) return GPTQ_ERR_STATE;
   DeviceGuard dg(c->device);
-  CK(cudaMemcpyAsync(U_out, c->U, static_cast<size_t>(c->n) * c->n * 4, cudaMemcpyDeviceToDevice, c->stream));
+  const size_t nn = static_cast<size_t>(c->n) * c->n;
+  combine_hilo_kernel<<<592, 256, 0, c->stream>>>(c->U_hi, c->U_lo, nn, U_out);
+  ++c->launches;
+  CKL("combine");
   return GPTQ_OK;
 }
 
@@ -454,8 +525,10 @@ gptq_status gptq_quantize_layer(gptq_ctx* c, const void* W, int64_t m, gptq_qpar
   CKL("init_w");
   SweepArgs a;
   a.Wq = c->Wq;
-  a.U = c->U;
-  a.Err = c->Err;
+  a.U = c->U_hi;
+  a.U_lo = c->U_lo;
+  a.Err = c->Err_hi;
+  a.Err_lo = c->Err_lo;
   a.codes = codes;
   a.scales = scales;
   a.zeros = zeros;
@@ -479,8 +552,13 @@ gptq_status gptq_quantize_layer(gptq_ctx* c, const void* W, int64_t m, gptq_qpar
     CKL("sweep");
     const int i2 = i1 + SW_B;
     if (i2 < n) {
-      gptq_status s = sgemm(c, false, mi, n - i2, SW_B, -1.f, c->Err, SW_B,
-                            c->U + static_cast<size_t>(i1) * n + i2, n, 1.f, c->Wq + i2, n, false);
+      // W[:, i2:] -= Err * U[i1:i2, i2:]   (B in K-major form: rows i2.. of U^T, columns i1..i2)
+      TcOut w;
+      w.C = c->Wq + i2;
+      w.ldc = n;
+      const size_t ub = static_cast<size_t>(i2) * n + i1;
+      gptq_status s = gemm_tc(c, mi, n - i2, SW_B, c->Err_hi, c->Err_lo, SW_B, c->Ut_hi + ub, c->Ut_lo + ub, n, -1.f,
+                              1, GT_KLO_NONE, GT_KHI_NONE, 0, w);
       if (s != GPTQ_OK) return s;
     }
   }
@@ -512,6 +590,50 @@ gptq_status gptq_reset(gptq_ctx* c) {
 }
 
 int64_t gptq_launch_count(const gptq_ctx* c) { return c ? c->launches : -1; }
+
+gptq_status gptq_test_gemm_tf32x3(int M, int N, int K, const float* A_hi, const float* A_lo, int lda, const float* B_hi,
+                                  const float* B_lo, int ldb, float alpha, int beta, int k_lo_mode, int k_hi_mode,
+                                  int upper_only, float* C, int ldc, float* C_hi, float* C_lo, int ldh, float* Ct_hi,
+                                  float* Ct_lo, int ldt, int device, void* cuda_stream) {
+  if (!A_hi || !A_lo || !B_hi || !B_lo || M < 1 || N < 1 || K < GT_BK) return GPTQ_ERR_ARG;
+  if (k_lo_mode < 0 || k_lo_mode > 2 || k_hi_mode < 0 || k_hi_mode > 1 || (beta != 0 && beta != 1)) return GPTQ_ERR_ARG;
+  if ((C_hi == nullptr) != (C_lo == nullptr) || (Ct_hi == nullptr) != (Ct_lo == nullptr)) return GPTQ_ERR_ARG;
+  if ((C && (!aligned16(C) || ldc % 4)) || (C_hi && (!aligned16(C_hi) || !aligned16(C_lo) || ldh % 4)))
+    return GPTQ_ERR_ARG;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) {
+    cudaGetLastError();
+    return GPTQ_ERR_CUDA;
+  }
+  DeviceGuard dg(device);
+  gptq_ctx t;
+  t.device = device;
+  t.stream = static_cast<cudaStream_t>(cuda_stream);
+  t.encode = get_encode();
+  if (!t.encode) return GPTQ_ERR_CUDA;
+  CK(cudaFuncSetAttribute(gemm_tf32x3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GT_SMEM));
+  CK(cudaMallocAsync(reinterpret_cast<void**>(&t.status), sizeof(int), t.stream));
+  CK(cudaMemsetAsync(t.status, 0, sizeof(int), t.stream));
+  TcOut o;
+  o.C = C;
+  o.ldc = ldc;
+  o.Chi = C_hi;
+  o.Clo = C_lo;
+  o.ldh = ldh;
+  o.Cthi = Ct_hi;
+  o.Ctlo = Ct_lo;
+  o.ldt = ldt;
+  gptq_status s = gemm_tc(&t, M, N, K, A_hi, A_lo, lda, B_hi, B_lo, ldb, alpha, beta, k_lo_mode, k_hi_mode,
+                          upper_only, o);
+  int flags = 0;
+  cudaMemcpyAsync(&flags, t.status, sizeof(int), cudaMemcpyDeviceToHost, t.stream);
+  cudaError_t e = cudaStreamSynchronize(t.stream);
+  cudaFreeAsync(t.status, t.stream);
+  t.status = nullptr;
+  if (s != GPTQ_OK) return s;
+  if (e != cudaSuccess) return cuda_fail(e, "test gemm");
+  return status_from_flags(flags);
+}
 
 gptq_status gptq_destroy(gptq_ctx* c) {
   if (!c) return GPTQ_OK;
@@ -607,7 +729,9 @@ extern "C" gptq_status gptq_quantize_layer_noalloc(const void* W, int64_t m, int
   SweepArgs a;
   a.Wq = Wq;
   a.U = U;
+  a.U_lo = nullptr;
   a.Err = Err;
+  a.Err_lo = nullptr;
   a.codes = codes;
   a.scales = scales;
   a.zeros = zeros;

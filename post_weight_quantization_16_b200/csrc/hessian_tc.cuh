@@ -54,15 +54,6 @@ __device__ __forceinline__ void hs_tile_of(int t, int& bi, int& bj) {
   bi = t - b * (b + 1);
 }
 
-// Wait without the abort shortcut (used to drain copies/MMAs still in flight before exit).
-__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
-  }
-  return true;
-}
-
 __global__ void __launch_bounds__(HS_THREADS, 1)
     hessian_syrk_kernel(const __grid_constant__ CUtensorMap xmap, float* __restrict__ H, int n, int n_tok,
                         int chunk_iters, int* __restrict__ status) {

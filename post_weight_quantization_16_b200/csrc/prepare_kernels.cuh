@@ -14,6 +14,8 @@
 #include <cuda_fp16.h>
 #include <cstdint>
 
+#include "factor_kernels.cuh"
+
 namespace gptq {
 
 __global__ void mirror_upper_kernel(float* __restrict__ H, int n) {
@@ -81,21 +83,24 @@ __global__ void identity_perm_kernel(int n, int32_t* __restrict__ perm) {
 // One CTA per output row a; the source row perm[a] of the (mirrored) H is staged in smem.
 __global__ void gather_damp_kernel(const float* __restrict__ H, int n, const int32_t* __restrict__ perm,
                                    const float* __restrict__ keys, const double* __restrict__ mean,
-                                   double damp, float* __restrict__ A) {
+                                   double damp, float* __restrict__ A_hi, float* __restrict__ A_lo) {
   extern __shared__ float row_s[];
   const int a = blockIdx.x;
   const int pa = perm[a];
   const float4* src = reinterpret_cast<const float4*>(H + static_cast<size_t>(pa) * n);
   for (int k = threadIdx.x; k < n / 4; k += blockDim.x) reinterpret_cast<float4*>(row_s)[k] = src[k];
   __syncthreads();
-  float* dst = A + static_cast<size_t>(a) * n;
+  float* dh = A_hi + static_cast<size_t>(a) * n;
+  float* dl = A_lo + static_cast<size_t>(a) * n;
   for (int b = threadIdx.x; b < n; b += blockDim.x) {
     float v;
     if (b == a)
       v = static_cast<float>(static_cast<double>(keys[pa]) + damp * (*mean));
     else
       v = row_s[perm[b]];
-    dst[b] = v;
+    const float hi = tf32_round(v);
+    dh[b] = hi;
+    dl[b] = tf32_round(v - hi);
   }
 }
 
@@ -112,6 +117,14 @@ __global__ void init_w_kernel(const __half* __restrict__ W, int n, const int32_t
     const int p = perm[k];
     dst[k] = dead[p] ? 0.0f : __half2float(wrow_s[p]);
   }
+}
+
+// out = hi + lo (the fp32 value of a hi/lo pair)
+__global__ void combine_hilo_kernel(const float* __restrict__ hi, const float* __restrict__ lo, size_t count,
+                                    float* __restrict__ out) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < count;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    out[i] = hi[i] + lo[i];
 }
 
 __global__ void g_idx_kernel(const int32_t* __restrict__ perm, int n, int g, int32_t* __restrict__ g_idx) {

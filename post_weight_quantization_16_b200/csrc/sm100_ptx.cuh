@@ -84,6 +84,15 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
   }
 }
 
+// Wait without the abort shortcut (used to drain copies/MMAs still in flight before exit).
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+  }
+  return true;
+}
+
 // ----------------------------------------------------------------------------------------
 // TMA (per-CTA tensor loads from this GPU's own memory; no cluster multicast anywhere)
 // ----------------------------------------------------------------------------------------

@@ -23,6 +23,8 @@
 
 #include <cstdint>
 
+#include "factor_kernels.cuh"
+
 namespace gptq {
 
 constexpr int SW_B = 128;       // sweep block (columns)
@@ -31,8 +33,10 @@ constexpr int SW_SMEM = SW_B * SW_B * 4 + SW_B * 4 + SW_B * 4 + SW_B * SW_THREAD
 
 struct SweepArgs {
   float* Wq;          // [m x n] fp32 working weights, sweep order
-  const float* U;     // [n x n] upper factor
-  float* Err;         // [m x 128] scaled errors of the current block
+  const float* U;     // [n x n] upper factor (fp32, or the tf32 hi part when U_lo is set)
+  const float* U_lo;  // [n x n] tf32 lo part of U, or nullptr
+  float* Err;         // [m x 128] scaled errors of the current block (fp32, or hi part)
+  float* Err_lo;      // [m x 128] tf32 lo part of the errors, or nullptr
   uint32_t* codes;    // [m x n*bits/32]
   float* scales;      // [m x G]
   float* zeros;       // [m x G]
@@ -73,13 +77,20 @@ __global__ void __launch_bounds__(SW_THREADS)
   const int n = a.n;
   for (int idx = lane; idx < SW_B * SW_B / 4; idx += SW_THREADS) {
     const int k = idx / (SW_B / 4), j4 = idx % (SW_B / 4);
-    reinterpret_cast<float4*>(Us)[idx] =
-        *reinterpret_cast<const float4*>(a.U + static_cast<size_t>(i1 + k) * n + i1 + 4 * j4);
+    const size_t g = static_cast<size_t>(i1 + k) * n + i1 + 4 * j4;
+    float4 u = *reinterpret_cast<const float4*>(a.U + g);
+    if (a.U_lo) {
+      const float4 l = *reinterpret_cast<const float4*>(a.U_lo + g);
+      u.x += l.x;
+      u.y += l.y;
+      u.z += l.z;
+      u.w += l.w;
+    }
+    reinterpret_cast<float4*>(Us)[idx] = u;
   }
-  for (int k = lane; k < SW_B; k += SW_THREADS) {
-    rU[k] = 1.0f / a.U[static_cast<size_t>(i1 + k) * n + i1 + k];
-    perm_s[k] = a.perm[i1 + k];
-  }
+  for (int k = lane; k < SW_B; k += SW_THREADS) perm_s[k] = a.perm[i1 + k];
+  __syncthreads();
+  for (int k = lane; k < SW_B; k += SW_THREADS) rU[k] = 1.0f / Us[k * SW_B + k];
   __syncthreads();
 
   const int r = blockIdx.x * SW_THREADS + lane;
@@ -189,8 +200,23 @@ __global__ void __launch_bounds__(SW_THREADS)
     }
     if (valid) {
       float4* ep = reinterpret_cast<float4*>(err_row + c0);
+      if (a.Err_lo) {
+        float4* lp = reinterpret_cast<float4*>(a.Err_lo + static_cast<size_t>(rr) * SW_B + c0);
 #pragma unroll
-      for (int j4 = 0; j4 < 4; ++j4) ep[j4] = make_float4(E[4 * j4], E[4 * j4 + 1], E[4 * j4 + 2], E[4 * j4 + 3]);
+        for (int j4 = 0; j4 < 4; ++j4) {
+          float hi[4], lo[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            hi[e] = tf32_round(E[4 * j4 + e]);
+            lo[e] = tf32_round(E[4 * j4 + e] - hi[e]);
+          }
+          ep[j4] = make_float4(hi[0], hi[1], hi[2], hi[3]);
+          lp[j4] = make_float4(lo[0], lo[1], lo[2], lo[3]);
+        }
+      } else {
+#pragma unroll
+        for (int j4 = 0; j4 < 4; ++j4) ep[j4] = make_float4(E[4 * j4], E[4 * j4 + 1], E[4 * j4 + 2], E[4 * j4 + 3]);
+      }
     }
 #pragma unroll
     for (int t = 1; t < 8; ++t) {

@@ -17,6 +17,7 @@ import torch
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libgptq.so")
 HEADER = os.path.join(os.path.dirname(HERE), "include", "gptq.h")
+HEADERS = [HEADER, os.path.join(os.path.dirname(HERE), "include", "gptq_testing.h")]
 
 STATUS = {0: "GPTQ_OK", 1: "GPTQ_ERR_ARG", 2: "GPTQ_ERR_STATE", 3: "GPTQ_ERR_NOT_PD", 4: "GPTQ_ERR_OOM",
           5: "GPTQ_ERR_CUDA", 6: "GPTQ_ERR_TIMEOUT", 7: "GPTQ_ERR_UNSUPPORTED"}
@@ -53,6 +54,10 @@ _SIGS = {
     "gptq_launch_count": (ctypes.c_int64, [_P]),
     "gptq_quantize_layer_noalloc": (ctypes.c_int, [_P, ctypes.c_int64, ctypes.c_int64, _P, _P, _P, QParams,
                                                    _P, _P, _P, _P, _P, ctypes.c_int, _P]),
+    "gptq_test_gemm_tf32x3": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P, ctypes.c_int, _P, _P,
+                                             ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                             ctypes.c_int, _P, ctypes.c_int, _P, _P, ctypes.c_int, _P, _P,
+                                             ctypes.c_int, ctypes.c_int, _P]),
 }
 
 
@@ -73,10 +78,12 @@ def lib():
 
 
 def header_functions():
-    """Names of the functions include/gptq.h declares."""
-    text = open(HEADER).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(gptq_[a-z_]+)\s*\(", text)))
+    """Names of the functions the headers under include/ declare."""
+    names = set()
+    for h in HEADERS:
+        text = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        names |= set(re.findall(r"\b(gptq_[a-z0-9_]+)\s*\(", text))
+    return sorted(names)
 
 
 def _check(status: int, call: str):

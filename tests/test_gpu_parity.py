@@ -56,10 +56,10 @@ def test_hessian_batches_strides_and_chunks():
 # ----------------------------------------------------------------------------------------
 # S2-S4 prepare
 # ----------------------------------------------------------------------------------------
-@pytest.mark.parametrize("desc_act", [False, True])
-@pytest.mark.parametrize("damp", [0.01, 0.1])
-def test_prepare_perm_and_factor(desc_act, damp):
-    layer = synth.scaled_layer(TINY, m=64, n=640, n_tok=3000)
+@pytest.mark.parametrize("n,desc_act,damp", [(128, True, 0.01), (256, False, 0.1), (384, True, 0.01),
+                                             (640, False, 0.01), (640, True, 0.1), (1024, True, 0.01)])
+def test_prepare_perm_and_factor(n, desc_act, damp):
+    layer = synth.scaled_layer(TINY, m=64, n=n, n_tok=3000)
     X = synth.make_x_bf16(layer)
     with GPTQContext(layer.n, 64, 0) as ctx:
         ctx.accumulate_hessian(GH.bf16_to_dev(X))
