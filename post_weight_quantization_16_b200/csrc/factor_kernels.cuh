@@ -30,12 +30,18 @@ __device__ __forceinline__ float tf32_round(float x) {
 }
 
 // Warp 0: UL Cholesky of the 32 x 32 block S[P0.., P0..] (upper triangle) into V, and its
-// inverse into X.  Lane i holds row i in registers; columns are broadcast with shuffles.
+// inverse X = V^-1 in the same sweep.  Lane i holds row i of the block in registers
+// (columns are broadcast with shuffles) and column i of the inverse.  Step c produces
+// column c of V and row c of X: X[c][c] = 1/V[c][c], X[c][j] = -(sum_{c<l<=j} V[c][l] X[l][j]) / V[c][c];
+// the inverse row uses only earlier steps' results, so it fills the latency of the pivot chain.
 __device__ __forceinline__ void leaf_diag_factor(float (*S)[LF_LD], float (*V)[LF_LD], float (*X)[LF_LD], int P0,
                                                  int lane, int* bad) {
-  float d[LF_P];
+  float d[LF_P], x[LF_P];
 #pragma unroll
-  for (int j = 0; j < LF_P; ++j) d[j] = S[P0 + lane][P0 + j];
+  for (int j = 0; j < LF_P; ++j) {
+    d[j] = S[P0 + lane][P0 + j];
+    x[j] = 0.0f;
+  }
 #pragma unroll
   for (int c = LF_P - 1; c >= 0; --c) {
     float piv = __shfl_sync(0xffffffffu, d[c], c);
@@ -43,31 +49,26 @@ __device__ __forceinline__ void leaf_diag_factor(float (*S)[LF_LD], float (*V)[L
       if (lane == 0) *bad = 1;
       piv = 1.0f;
     }
-    const float s = sqrtf(piv);
-    const float rs = 1.0f / s;
-    const float col = (lane < c) ? d[c] * rs : (lane == c ? s : 0.0f);
+    const float rs = rsqrtf(piv);  // 1 / V[c][c]
+    const float sv = piv * rs;     // V[c][c]
+    const float col = (lane < c) ? d[c] * rs : (lane == c ? sv : 0.0f);
     d[c] = col;
+    V[P0 + lane][P0 + c] = col;
 #pragma unroll
-    for (int j = 0; j < c; ++j) {
+    for (int j = c - 1; j >= 0; --j) {  // the next pivot column first: it is on the critical path
       const float cj = __shfl_sync(0xffffffffu, col, j);
       d[j] = fmaf(-col, cj, d[j]);
     }
-  }
-#pragma unroll
-  for (int j = 0; j < LF_P; ++j) V[P0 + lane][P0 + j] = (j >= lane) ? d[j] : 0.0f;
-  __syncwarp();
-  // column `lane` of the inverse by back substitution (x[l] = 0 for l > lane)
-  float x[LF_P];
-#pragma unroll
-  for (int r = LF_P - 1; r >= 0; --r) {
+    // row c of the inverse (V[c][l] for l > c were written by earlier steps)
+    __syncwarp();
     float acc = 0.0f;
 #pragma unroll
-    for (int l = r + 1; l < LF_P; ++l) acc = fmaf(V[P0 + r][P0 + l], x[l], acc);
-    const float vrr = V[P0 + r][P0 + r];
-    x[r] = (r == lane) ? 1.0f / vrr : (r < lane ? -acc / vrr : 0.0f);
+    for (int l = c + 1; l < LF_P; ++l) acc = fmaf(V[P0 + c][P0 + l], x[l], acc);
+    x[c] = (lane == c) ? rs : (lane > c ? -acc * rs : 0.0f);
   }
 #pragma unroll
   for (int r = 0; r < LF_P; ++r) X[P0 + r][P0 + lane] = x[r];
+  __syncwarp();
 }
 
 // Leaf: U_kk (= V_kk^-1, V_kk V_kk^T = A_kk) for the diagonal block at offset o, read from
@@ -95,30 +96,82 @@ __global__ void __launch_bounds__(LF_THREADS, 1)
   __syncthreads();
 
   // ---- reverse right-looking Cholesky, 32-column panels from the bottom-right ----
+  // Lookahead: after the panel solve, warp 0 updates the next diagonal block itself and goes
+  // straight on to factor it, while warps 1-3 and 5-7 (warp 4 shares warp 0's scheduler)
+  // update the rest of the trailing triangle.
   for (int p = LF_NB / LF_P - 1; p >= 0; --p) {
     const int P0 = p * LF_P;
     if (warp == 0) leaf_diag_factor(S, V, X, P0, lane, bad);
     __syncthreads();
-    // panel: V[i][P0+c] = sum_{k >= c} S[i][P0+k] * Xd[c][k]   for rows i < P0
-    for (int item = tid; item < P0 * 8; item += LF_THREADS) {
-      const int i = item >> 3, cg = (item & 7) * 4;
+    // panel: V[i][P0+c] = sum_k S[i][P0+k] * Xd[c][k]   for rows i < P0 (Xd upper: zero for k < c);
+    // one 4 x 4 tile of (rows, panel columns) per thread
+    for (int item = tid; item < (P0 / 4) * (LF_P / 4); item += LF_THREADS) {
+      const int i0 = (item / (LF_P / 4)) * 4, c0 = (item % (LF_P / 4)) * 4;
+      float acc[4][4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int c = cg + e;
-        float acc = 0.0f;
-        for (int k = c; k < LF_P; ++k) acc = fmaf(S[i][P0 + k], X[P0 + c][P0 + k], acc);
-        V[i][P0 + c] = acc;
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
+#pragma unroll 8
+      for (int k = 0; k < LF_P; ++k) {
+        float sv[4], xv[4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          sv[a] = S[i0 + a][P0 + k];
+          xv[a] = X[P0 + c0 + a][P0 + k];
+        }
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+          for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(sv[a], xv[b], acc[a][b]);
       }
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) V[i0 + a][P0 + c0 + b] = acc[a][b];
     }
     __syncthreads();
-    // trailing update of the upper triangle: S[i][j] -= sum_c V[i][P0+c] V[j][P0+c], i <= j < P0
-    const int nb = P0 / 4;
-    const int npairs = nb * (nb + 1) / 2;
-    for (int t = tid; t < npairs; t += LF_THREADS) {
-      int bj = static_cast<int>((sqrtf(8.0f * t + 1.0f) - 1.0f) * 0.5f);
-      while (bj * (bj + 1) / 2 > t) --bj;
-      while ((bj + 1) * (bj + 2) / 2 <= t) ++bj;
-      const int bi = t - bj * (bj + 1) / 2;
+    if (p == 0) break;
+    // trailing update of the upper triangle: S[i][j] -= sum_c V[i][P0+c] V[j][P0+c], i <= j < P0,
+    // in 4 x 4 tiles (bi <= bj); the tiles of the next diagonal block go to warp 0
+    const int nb = P0 / 4, nd = LF_P / 4, d0 = nb - nd;  // next diagonal block = tile rows/cols [d0, nb)
+    int t_begin, t_step, t_end;
+    if (warp == 0) {
+      t_begin = lane;
+      t_step = 32;
+      t_end = nd * (nd + 1) / 2;  // tiles inside the next diagonal block
+    } else if (warp == 4) {
+      t_begin = 0;
+      t_step = 1;
+      t_end = 0;
+    } else {
+      const int wi = (warp < 4) ? warp - 1 : warp - 2;  // 0..5
+      t_begin = wi * 32 + lane;
+      t_step = 6 * 32;
+      t_end = nb * (nb + 1) / 2 - nd * (nd + 1) / 2;  // all other tiles
+    }
+    for (int t = t_begin; t < t_end; t += t_step) {
+      int bi, bj;
+      if (warp == 0) {  // enumerate the upper tiles of the next diagonal block
+        int jj = static_cast<int>((sqrtf(8.0f * t + 1.0f) - 1.0f) * 0.5f);
+        while (jj * (jj + 1) / 2 > t) --jj;
+        while ((jj + 1) * (jj + 2) / 2 <= t) ++jj;
+        bi = d0 + (t - jj * (jj + 1) / 2);
+        bj = d0 + jj;
+      } else {  // enumerate all upper tiles with bj < d0, then the block column bi < d0 <= bj
+        const int na = d0 * (d0 + 1) / 2;
+        if (t < na) {
+          int jj = static_cast<int>((sqrtf(8.0f * t + 1.0f) - 1.0f) * 0.5f);
+          while (jj * (jj + 1) / 2 > t) --jj;
+          while ((jj + 1) * (jj + 2) / 2 <= t) ++jj;
+          bi = t - jj * (jj + 1) / 2;
+          bj = jj;
+        } else {
+          const int u = t - na;
+          bi = u / nd;
+          bj = d0 + u % nd;
+        }
+      }
       const int i0 = 4 * bi, j0 = 4 * bj;
       float acc[4][4];
 #pragma unroll
@@ -144,41 +197,67 @@ __global__ void __launch_bounds__(LF_THREADS, 1)
         for (int b = 0; b < 4; ++b)
           if (i0 + a <= j0 + b) S[i0 + a][j0 + b] -= acc[a][b];
     }
-    __syncthreads();
+    if (warp == 0) __syncwarp();
   }
+  __syncthreads();
 
   // ---- U = V^-1: diagonal 32-blocks are in X; off-diagonal blocks by block rows ----
   //   U_ij = -Xd_i * sum_{l=i+1..j} V_il U_lj      (block row i from the bottom)
   for (int bi = LF_NB / LF_P - 2; bi >= 0; --bi) {
     const int I0 = bi * LF_P;
     const int ncols = LF_NB - I0 - LF_P;  // columns right of the diagonal block
-    // T[r][c] = sum_{k >= I0+32} V[I0+r][k] X[k][I0+32+c]  -> stored in S (free now)
-    for (int item = tid; item < LF_P * ncols / 4; item += LF_THREADS) {
-      const int r = item / (ncols / 4), c0 = (item % (ncols / 4)) * 4;
-      const int col = I0 + LF_P + c0;
-      const int kend = col + 4;  // X is upper: X[k][col..col+3] = 0 for k > col + 3
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int k = I0 + LF_P; k < kend; ++k) {
-        const float v = V[I0 + r][k];
+    // T[r][col] = sum_{k >= I0+32} V[I0+r][k] X[k][col]  -> stored in S (free now);
+    // one 4 x 4 tile per thread; X is upper, so X[k][col0..col0+3] = 0 for k > col0 + 3
+    const int nct = ncols / 4;
+    for (int item = tid; item < (LF_P / 4) * nct; item += LF_THREADS) {
+      const int r0 = (item / nct) * 4, col0 = I0 + LF_P + (item % nct) * 4;
+      float acc[4][4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) acc[e] = fmaf(v, X[k][col + e], acc[e]);
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
+      for (int k = I0 + LF_P; k < col0 + 4; ++k) {
+        float vv[4], xv[4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          vv[a] = V[I0 + r0 + a][k];
+          xv[a] = X[k][col0 + a];
+        }
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+          for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(vv[a], xv[b], acc[a][b]);
       }
 #pragma unroll
-      for (int e = 0; e < 4; ++e) S[I0 + r][col + e] = acc[e];
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) S[I0 + r0 + a][col0 + b] = acc[a][b];
     }
     __syncthreads();
-    // X[I0+r][col] = -sum_{k >= r} Xd[r][k] T[k][col]
-    for (int item = tid; item < LF_P * ncols / 4; item += LF_THREADS) {
-      const int r = item / (ncols / 4), c0 = (item % (ncols / 4)) * 4;
-      const int col = I0 + LF_P + c0;
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int k = r; k < LF_P; ++k) {
-        const float xd = X[I0 + r][I0 + k];
+    // X[I0+r][col] = -sum_{k >= r} Xd[r][k] T[k][col]      (Xd upper: zero for k < r)
+    for (int item = tid; item < (LF_P / 4) * nct; item += LF_THREADS) {
+      const int r0 = (item / nct) * 4, col0 = I0 + LF_P + (item % nct) * 4;
+      float acc[4][4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) acc[e] = fmaf(xd, S[I0 + k][col + e], acc[e]);
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
+      for (int k = r0; k < LF_P; ++k) {
+        float xd[4], tv[4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          xd[a] = X[I0 + r0 + a][I0 + k];
+          tv[a] = S[I0 + k][col0 + a];
+        }
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+          for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(xd[a], tv[b], acc[a][b]);
       }
 #pragma unroll
-      for (int e = 0; e < 4; ++e) X[I0 + r][col + e] = -acc[e];
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) X[I0 + r0 + a][col0 + b] = -acc[a][b];
     }
     __syncthreads();
   }

@@ -10,8 +10,9 @@
 // accumulated in its own TMEM buffer and then added into fp32 registers with
 // round-to-nearest adds (double-buffered TMEM, as in the Hessian kernel).
 //
-// Tile 128 x 256 (tcgen05.mma kind::tf32, M=128, N=256, K=8), 2-stage TMA ring of 96 KB
-// stages (A_hi, A_lo, B_hi, B_lo; 128-byte swizzle), warp roles:
+// Tile 128 x 256 (tcgen05.mma kind::tf32, M=128, N=256, K=8), persistent CTAs (one per SM)
+// over the tiles, 2-stage TMA ring of 96 KB stages (A_hi, A_lo, B_hi, B_lo; 128-byte
+// swizzle), warp roles:
 //   warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer, warps 2-9 epilogue.
 // Triangular operands: the K range of a tile can start at its first column (B lower in
 // K-major form) or its first row (A upper), or stop after its last column (B upper), so
@@ -19,6 +20,10 @@
 // can be skipped for symmetric updates.
 // Outputs (any subset): plain fp32 C (optionally + C), hi/lo pair (optionally + hi+lo), and a
 // transposed hi/lo pair (coalesced: the 32 lanes of a warp write 32 consecutive rows).
+// A and B are addressed as sub-blocks (row/column offsets) of the whole matrices their tensor
+// maps describe, so the maps are encoded once per context.  Rows or columns of a partial
+// tile that fall outside the sub-block read neighbouring data whose products land only in
+// outputs that are never stored.
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -37,6 +42,8 @@ enum : int { GT_KHI_NONE = 0, GT_KHI_COL = 1 };
 
 struct GemmTCArgs {
   int M, N, K;
+  int a_row0, a_col0;  // offset of A inside the matrix its tensor maps describe
+  int b_row0, b_col0;  // offset of B
   float alpha;
   int beta;          // 0 or 1: add the existing C (plain or hi+lo)
   int k_lo_mode, k_hi_mode, upper_only;
@@ -57,6 +64,26 @@ __device__ __forceinline__ float tf32_rn(float x) {
   return __uint_as_float(u & 0xFFFFE000u);
 }
 
+// Tile t of the output (n-tiles fastest); returns false for tiles skipped by upper_only.
+__device__ __forceinline__ bool gt_tile(const GemmTCArgs& p, int t, int ntn, int& m0, int& n0, int& k_begin,
+                                       int& n_iters) {
+  m0 = (t / ntn) * GT_BM;
+  n0 = (t % ntn) * GT_BN;
+  if (p.upper_only && m0 >= n0 + GT_BN) return false;
+  int kb = 0, ke = p.K;
+  if (p.k_lo_mode == GT_KLO_COL) kb = n0;
+  if (p.k_lo_mode == GT_KLO_ROW) kb = m0;
+  if (p.k_hi_mode == GT_KHI_COL) ke = min(p.K, n0 + GT_BN);
+  kb = (kb / GT_BK) * GT_BK;
+  k_begin = kb;
+  n_iters = (ke > kb) ? (ke - kb + GT_BK - 1) / GT_BK : 0;
+  return true;
+}
+
+// Persistent: CTA b handles tiles b, b + gridDim.x, ...  The producer and the MMA issuer run
+// ahead across tile boundaries; each K stage lands in one of two TMEM accumulators, which
+// the epilogue warps drain into registers that were pre-loaded with C (beta = 1) while the
+// tile's first stages were in flight, so a tile ends with stores only.
 __global__ void __launch_bounds__(GT_THREADS, 1)
     gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_constant__ CUtensorMap a_lo,
                        const __grid_constant__ CUtensorMap b_hi, const __grid_constant__ CUtensorMap b_lo,
@@ -68,16 +95,8 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int m0 = blockIdx.y * GT_BM;
-  const int n0 = blockIdx.x * GT_BN;
-  if (p.upper_only && m0 >= n0 + GT_BN) return;  // uniform, before any barrier or TMEM use
-
-  int k_begin = 0, k_end = p.K;
-  if (p.k_lo_mode == GT_KLO_COL) k_begin = n0;
-  if (p.k_lo_mode == GT_KLO_ROW) k_begin = m0;
-  if (p.k_hi_mode == GT_KHI_COL) k_end = min(p.K, n0 + GT_BN);
-  k_begin = (k_begin / GT_BK) * GT_BK;
-  const int n_iters = (k_end > k_begin) ? (k_end - k_begin + GT_BK - 1) / GT_BK : 0;
+  const int ntn = (p.N + GT_BN - 1) / GT_BN;
+  const int ntiles = ntn * ((p.M + GT_BM - 1) / GT_BM);
 
   const uint32_t bar_full = sbase + GT_STAGES * GT_STAGE_BYTES;
   const uint32_t bar_empty = bar_full + 8 * GT_STAGES;
@@ -117,59 +136,71 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------- TMA producer ----------------
-      int issued = 0;
-      for (int it = 0; it < n_iters; ++it) {
-        const int s = it % GT_STAGES;
-        const uint32_t ph = static_cast<uint32_t>(it / GT_STAGES) & 1u;
-        if (!mbar_wait_bounded(bar_empty + 8 * s, ph ^ 1u, abort_flag)) break;
-        const uint32_t fb = bar_full + 8 * s;
-        mbar_arrive_expect_tx(fb, GT_STAGE_BYTES);
-        const uint32_t st = sbase + s * GT_STAGE_BYTES;
-        const int k = k_begin + it * GT_BK;
-        tma_load_2d(st, &a_hi, fb, k, m0);
-        tma_load_2d(st + GT_A_BYTES, &a_lo, fb, k, m0);
-        tma_load_2d(st + 2 * GT_A_BYTES, &b_hi, fb, k, n0);
-        tma_load_2d(st + 2 * GT_A_BYTES + GT_B_BYTES, &b_lo, fb, k, n0);
-        issued = it + 1;
+      // ---------------- TMA producer (continuous stage ring over all tiles) ----------------
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        int m0, n0, kb, ni;
+        if (!gt_tile(p, t, ntn, m0, n0, kb, ni)) continue;
+        for (int j = 0; j < ni; ++j, ++it) {
+          const int s = it % GT_STAGES;
+          const uint32_t ph = static_cast<uint32_t>(it / GT_STAGES) & 1u;
+          if (!mbar_wait_bounded(bar_empty + 8 * s, ph ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = bar_full + 8 * s;
+          mbar_arrive_expect_tx(fb, GT_STAGE_BYTES);
+          const uint32_t st = sbase + s * GT_STAGE_BYTES;
+          const int k = kb + j * GT_BK;
+          tma_load_2d(st, &a_hi, fb, p.a_col0 + k, p.a_row0 + m0);
+          tma_load_2d(st + GT_A_BYTES, &a_lo, fb, p.a_col0 + k, p.a_row0 + m0);
+          tma_load_2d(st + 2 * GT_A_BYTES, &b_hi, fb, p.b_col0 + k, p.b_row0 + n0);
+          tma_load_2d(st + 2 * GT_A_BYTES + GT_B_BYTES, &b_lo, fb, p.b_col0 + k, p.b_row0 + n0);
+        }
       }
-      for (int it = max(0, issued - GT_STAGES); it < issued; ++it)
-        mbar_wait_drain(bar_full + 8 * (it % GT_STAGES), static_cast<uint32_t>(it / GT_STAGES) & 1u);
+      for (int i = max(0, it - GT_STAGES); i < it; ++i)
+        mbar_wait_drain(bar_full + 8 * (i % GT_STAGES), static_cast<uint32_t>(i / GT_STAGES) & 1u);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer: one TMEM buffer per K stage ----------------
       constexpr uint32_t idesc = idesc_make(2u, 2u, 0u, 0u, GT_BM, GT_BN);  // tf32, K-major A and B
       bool ok = true;
-      for (int it = 0; it < n_iters; ++it) {
-        const int b = it & 1;
-        const uint32_t ph = static_cast<uint32_t>(it >> 1) & 1u;
-        if (!mbar_wait_bounded(bar_tempty + 8 * b, ph ^ 1u, abort_flag)) {
-          ok = false;
-          break;
-        }
-        const int s = it % GT_STAGES;
-        const uint32_t phs = static_cast<uint32_t>(it / GT_STAGES) & 1u;
-        if (!mbar_wait_bounded(bar_full + 8 * s, phs, abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * GT_BN);
-        const uint32_t st = sbase + s * GT_STAGE_BYTES;
-        const uint32_t sa_hi = st, sa_lo = st + GT_A_BYTES;
-        const uint32_t sb_hi = st + 2 * GT_A_BYTES, sb_lo = sb_hi + GT_B_BYTES;
+      int it = 0;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        int m0, n0, kb, ni;
+        if (!gt_tile(p, t, ntn, m0, n0, kb, ni)) continue;
+        for (int j = 0; j < ni; ++j, ++it) {
+          const int b = it & 1;
+          const uint32_t ph = static_cast<uint32_t>(it >> 1) & 1u;
+          if (!mbar_wait_bounded(bar_tempty + 8 * b, ph ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const int s = it % GT_STAGES;
+          const uint32_t phs = static_cast<uint32_t>(it / GT_STAGES) & 1u;
+          if (!mbar_wait_bounded(bar_full + 8 * s, phs, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * GT_BN);
+          const uint32_t st = sbase + s * GT_STAGE_BYTES;
+          const uint32_t sa_hi = st, sa_lo = st + GT_A_BYTES;
+          const uint32_t sb_hi = st + 2 * GT_A_BYTES, sb_lo = sb_hi + GT_B_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < GT_BK / 8; ++kk) {
-          const uint32_t off = kk * 32;  // 8 fp32 of K inside the 128-byte swizzle row
-          const uint64_t dah = sdesc_sw128(sa_hi + off, 16, 1024), dal = sdesc_sw128(sa_lo + off, 16, 1024);
-          const uint64_t dbh = sdesc_sw128(sb_hi + off, 16, 1024), dbl = sdesc_sw128(sb_lo + off, 16, 1024);
-          umma_tf32(d_tmem, dal, dbh, idesc, kk > 0 ? 1u : 0u);
-          umma_tf32(d_tmem, dah, dbl, idesc, 1u);
-          umma_tf32(d_tmem, dah, dbh, idesc, 1u);
+          for (int kk = 0; kk < GT_BK / 8; ++kk) {
+            const uint32_t off = kk * 32;  // 8 fp32 of K inside the 128-byte swizzle row
+            const uint64_t dah = sdesc_sw128(sa_hi + off, 16, 1024), dal = sdesc_sw128(sa_lo + off, 16, 1024);
+            const uint64_t dbh = sdesc_sw128(sb_hi + off, 16, 1024), dbl = sdesc_sw128(sb_lo + off, 16, 1024);
+            umma_tf32(d_tmem, dal, dbh, idesc, kk > 0 ? 1u : 0u);
+            umma_tf32(d_tmem, dah, dbl, idesc, 1u);
+            umma_tf32(d_tmem, dah, dbh, idesc, 1u);
+          }
+          umma_commit(bar_empty + 8 * s);
+          umma_commit(bar_tfull + 8 * b);
         }
-        umma_commit(bar_empty + 8 * s);
-        umma_commit(bar_tfull + 8 * b);
       }
       if (!ok) {
         umma_commit(bar_drain);
@@ -180,90 +211,106 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
     // ---------------- epilogue ----------------
     const int q = warp & 3;
     const int hh = (warp - 2) >> 2;
-    const int r = m0 + q * 32 + lane;
-    const int cbase = n0 + hh * (GT_BN / 2);
-    float acc[GT_BN / 2];
-#pragma unroll
-    for (int j = 0; j < GT_BN / 2; ++j) acc[j] = 0.0f;
+    int it = 0;
     bool all_ok = true;
-    for (int it = 0; it < n_iters; ++it) {
-      const int b = it & 1;
-      const uint32_t ph = static_cast<uint32_t>(it >> 1) & 1u;
-      int ok = 0;
-      if (lane == 0) ok = mbar_wait_bounded(bar_tfull + 8 * b, ph, abort_flag) ? 1 : 0;
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) {
-        all_ok = false;
-        break;
-      }
-      tc_fence_after();
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                               static_cast<uint32_t>(b * GT_BN + hh * (GT_BN / 2) + cc * 32),
-                           v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < 32; ++j) acc[cc * 32 + j] += __uint_as_float(v[j]);
-      }
-      tc_fence_before();
-      mbar_arrive(bar_tempty + 8 * b);
-    }
-    if (all_ok) {
+    for (int t = blockIdx.x; t < ntiles && all_ok; t += gridDim.x) {
+      int m0, n0, kb, ni;
+      if (!gt_tile(p, t, ntn, m0, n0, kb, ni)) continue;
+      const int r = m0 + q * 32 + lane;
+      const int cbase = n0 + hh * (GT_BN / 2);
       const bool row_ok = r < p.M;
+      float acc[GT_BN / 2];
+      // pre-load C (beta = 1) into the accumulators while the first stages run
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         const int c0 = cbase + cc * 32;
-        if (c0 >= p.N) continue;  // N % 32 == 0: whole 32-column groups
-        float v[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = p.alpha * acc[cc * 32 + j];
-        if (row_ok && p.C) {
-          float4* cp = reinterpret_cast<float4*>(p.C + static_cast<size_t>(r) * p.ldc + c0);
+        const bool ld = p.beta && row_ok && c0 < p.N;
+        if (ld && p.C) {
+          const float4* cp = reinterpret_cast<const float4*>(p.C + static_cast<size_t>(r) * p.ldc + c0);
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            float4 o = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-            if (p.beta) {
-              const float4 c = cp[j];
-              o.x += c.x;
-              o.y += c.y;
-              o.z += c.z;
-              o.w += c.w;
-            }
-            cp[j] = o;
+            const float4 c = cp[j];
+            acc[cc * 32 + 4 * j + 0] = c.x;
+            acc[cc * 32 + 4 * j + 1] = c.y;
+            acc[cc * 32 + 4 * j + 2] = c.z;
+            acc[cc * 32 + 4 * j + 3] = c.w;
           }
+        } else if (ld && p.Chi) {
+          const float4* hp = reinterpret_cast<const float4*>(p.Chi + static_cast<size_t>(r) * p.ldh + c0);
+          const float4* lp = reinterpret_cast<const float4*>(p.Clo + static_cast<size_t>(r) * p.ldh + c0);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float4 h = hp[j], l = lp[j];
+            acc[cc * 32 + 4 * j + 0] = h.x + l.x;
+            acc[cc * 32 + 4 * j + 1] = h.y + l.y;
+            acc[cc * 32 + 4 * j + 2] = h.z + l.z;
+            acc[cc * 32 + 4 * j + 3] = h.w + l.w;
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) acc[cc * 32 + j] = 0.0f;
         }
-        if (row_ok && p.Chi) {
+      }
+      for (int j = 0; j < ni; ++j, ++it) {
+        const int b = it & 1;
+        const uint32_t ph = static_cast<uint32_t>(it >> 1) & 1u;
+        int ok = 0;
+        if (lane == 0) ok = mbar_wait_bounded(bar_tfull + 8 * b, ph, abort_flag) ? 1 : 0;
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) {
+          all_ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          uint32_t v[16];
+          tmem_ld_32x32b_x16(tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                 static_cast<uint32_t>(b * GT_BN + hh * (GT_BN / 2) + cc * 16),
+                             v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) acc[cc * 16 + jj] = fmaf(p.alpha, __uint_as_float(v[jj]), acc[cc * 16 + jj]);
+        }
+        tc_fence_before();
+        mbar_arrive(bar_tempty + 8 * b);
+      }
+      if (!all_ok) break;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        const int c0 = cbase + cc * 32;
+        if (!row_ok || c0 >= p.N) continue;  // N % 32 == 0: whole 32-column groups
+        if (p.C) {
+          float4* cp = reinterpret_cast<float4*>(p.C + static_cast<size_t>(r) * p.ldc + c0);
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            cp[j] = make_float4(acc[cc * 32 + 4 * j], acc[cc * 32 + 4 * j + 1], acc[cc * 32 + 4 * j + 2],
+                                acc[cc * 32 + 4 * j + 3]);
+        }
+        if (p.Chi) {
           float4* hp = reinterpret_cast<float4*>(p.Chi + static_cast<size_t>(r) * p.ldh + c0);
           float4* lp = reinterpret_cast<float4*>(p.Clo + static_cast<size_t>(r) * p.ldh + c0);
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            float x[4] = {v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]};
-            if (p.beta) {
-              const float4 h = hp[j], l = lp[j];
-              x[0] += h.x + l.x;
-              x[1] += h.y + l.y;
-              x[2] += h.z + l.z;
-              x[3] += h.w + l.w;
-            }
             float hi[4], lo[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              hi[e] = tf32_rn(x[e]);
-              lo[e] = tf32_rn(x[e] - hi[e]);
+              const float x = acc[cc * 32 + 4 * j + e];
+              hi[e] = tf32_rn(x);
+              lo[e] = tf32_rn(x - hi[e]);
             }
             hp[j] = make_float4(hi[0], hi[1], hi[2], hi[3]);
             lp[j] = make_float4(lo[0], lo[1], lo[2], lo[3]);
           }
         }
-        if (row_ok && p.Cthi) {
+        if (p.Cthi) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            const float hi = tf32_rn(v[j]);
+            const float x = acc[cc * 32 + j];
+            const float hi = tf32_rn(x);
             const size_t o = static_cast<size_t>(c0 + j) * p.ldt + r;
             p.Cthi[o] = hi;
-            p.Ctlo[o] = tf32_rn(v[j] - hi);
+            p.Ctlo[o] = tf32_rn(x - hi);
           }
         }
       }

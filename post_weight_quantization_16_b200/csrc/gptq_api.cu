@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <chrono>
 #include <cstdio>
 #include <cstdlib>
@@ -54,6 +55,14 @@ struct gptq_ctx {
   int mirrored = 0;           // H's lower triangle has been filled
   int64_t chunk_tokens = 512;
   int64_t launches = 0;       // kernels launched by this context (instrumentation)
+  int num_sms = 148;
+  // tensor maps of whole matrices, encoded once: A-operand maps (128-row boxes) and
+  // B-operand maps (256-row boxes), hi and lo
+  CUtensorMap mA_A[2], mA_VT[2], mA_U[2], mA_Err[2];
+  CUtensorMap mB_U[2], mB_VT[2], mB_Ut[2];
+  cudaStream_t capture_stream = nullptr;
+  cudaGraphExec_t factor_graph = nullptr;  // the factorization recursion, recorded once
+  int64_t factor_graph_launches = 0;
   PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
 };
 
@@ -166,20 +175,25 @@ struct TcOut {
   int ldt = 0;
 };
 
-gptq_status gemm_tc(gptq_ctx* c, int M, int N, int K, const float* Ahi, const float* Alo, int lda, const float* Bhi,
-                    const float* Blo, int ldb, float alpha, int beta, int klo, int khi, int upper, const TcOut& o) {
+// An operand of gemm_tc: the hi/lo tensor maps of a whole matrix and the sub-block offset.
+struct TcOperand {
+  const CUtensorMap* hi;
+  const CUtensorMap* lo;
+  int row0, col0;
+};
+
+gptq_status gemm_tc(gptq_ctx* c, int M, int N, int K, TcOperand A, TcOperand B, float alpha, int beta, int klo,
+                    int khi, int upper, const TcOut& o) {
   if (M <= 0 || N <= 0) return GPTQ_OK;
   if (N % 32 || K % GT_BK) return GPTQ_ERR_ARG;
-  CUtensorMap ma_hi, ma_lo, mb_hi, mb_lo;
-  gptq_status s;
-  if ((s = make_map(c, &ma_hi, Ahi, M, K, lda, GT_BM)) != GPTQ_OK) return s;
-  if ((s = make_map(c, &ma_lo, Alo, M, K, lda, GT_BM)) != GPTQ_OK) return s;
-  if ((s = make_map(c, &mb_hi, Bhi, N, K, ldb, GT_BN)) != GPTQ_OK) return s;
-  if ((s = make_map(c, &mb_lo, Blo, N, K, ldb, GT_BN)) != GPTQ_OK) return s;
   GemmTCArgs a;
   a.M = M;
   a.N = N;
   a.K = K;
+  a.a_row0 = A.row0;
+  a.a_col0 = A.col0;
+  a.b_row0 = B.row0;
+  a.b_col0 = B.col0;
   a.alpha = alpha;
   a.beta = beta;
   a.k_lo_mode = klo;
@@ -194,8 +208,9 @@ gptq_status gemm_tc(gptq_ctx* c, int M, int N, int K, const float* Ahi, const fl
   a.Ctlo = o.Ctlo;
   a.ldt = o.ldt;
   a.status = c->status;
-  dim3 grid((N + GT_BN - 1) / GT_BN, (M + GT_BM - 1) / GT_BM);
-  gemm_tf32x3_kernel<<<grid, GT_THREADS, GT_SMEM, c->stream>>>(ma_hi, ma_lo, mb_hi, mb_lo, a);
+  const int ntiles = ((N + GT_BN - 1) / GT_BN) * ((M + GT_BM - 1) / GT_BM);
+  gemm_tf32x3_kernel<<<std::min(ntiles, c->num_sms), GT_THREADS, GT_SMEM, c->stream>>>(*A.hi, *A.lo, *B.hi, *B.lo,
+                                                                                       a);
   ++c->launches;
   CKL("gemm_tc");
   return GPTQ_OK;
@@ -217,29 +232,30 @@ gptq_status chol_inv(gptq_ctx* c, int o, int h) {
   auto at = [n](float* M, int r, int col) { return M + static_cast<size_t>(r) * n + col; };
   gptq_status s;
   if ((s = chol_inv(c, o2, h2)) != GPTQ_OK) return s;
+  auto opA = [](CUtensorMap* m, int r0, int c0) { return TcOperand{&m[0], &m[1], r0, c0}; };
   // V12 = A12 U22^T                      (U22 rows are the K-major B; k >= column)
   TcOut v12;
   v12.Chi = at(c->VT_hi, o, o2);
   v12.Clo = at(c->VT_lo, o, o2);
   v12.ldh = n;
-  if ((s = gemm_tc(c, h1, h2, h2, at(c->A_hi, o, o2), at(c->A_lo, o, o2), n, at(c->U_hi, o2, o2), at(c->U_lo, o2, o2),
-                   n, 1.f, 0, GT_KLO_COL, GT_KHI_NONE, 0, v12)) != GPTQ_OK)
+  if ((s = gemm_tc(c, h1, h2, h2, opA(c->mA_A, o, o2), opA(c->mB_U, o2, o2), 1.f, 0, GT_KLO_COL, GT_KHI_NONE, 0,
+                   v12)) != GPTQ_OK)
     return s;
   // A11 -= V12 V12^T                     (upper tiles only)
   TcOut a11;
   a11.Chi = at(c->A_hi, o, o);
   a11.Clo = at(c->A_lo, o, o);
   a11.ldh = n;
-  if ((s = gemm_tc(c, h1, h1, h2, at(c->VT_hi, o, o2), at(c->VT_lo, o, o2), n, at(c->VT_hi, o, o2),
-                   at(c->VT_lo, o, o2), n, -1.f, 1, GT_KLO_NONE, GT_KHI_NONE, 1, a11)) != GPTQ_OK)
+  if ((s = gemm_tc(c, h1, h1, h2, opA(c->mA_VT, o, o2), opA(c->mB_VT, o, o2), -1.f, 1, GT_KLO_NONE, GT_KHI_NONE, 1,
+                   a11)) != GPTQ_OK)
     return s;
   // T^T = (V12 U22)^T into the lower block [o2.., o..]   (Ut22 rows as B; k <= column)
   TcOut tt;
   tt.Cthi = at(c->VT_hi, o2, o);
   tt.Ctlo = at(c->VT_lo, o2, o);
   tt.ldt = n;
-  if ((s = gemm_tc(c, h1, h2, h2, at(c->VT_hi, o, o2), at(c->VT_lo, o, o2), n, at(c->Ut_hi, o2, o2),
-                   at(c->Ut_lo, o2, o2), n, 1.f, 0, GT_KLO_NONE, GT_KHI_COL, 0, tt)) != GPTQ_OK)
+  if ((s = gemm_tc(c, h1, h2, h2, opA(c->mA_VT, o, o2), opA(c->mB_Ut, o2, o2), 1.f, 0, GT_KLO_NONE, GT_KHI_COL, 0,
+                   tt)) != GPTQ_OK)
     return s;
   if ((s = chol_inv(c, o, h1)) != GPTQ_OK) return s;
   // U12 = -U11 T  (and Ut21 = U12^T)      (U11 rows as A; k >= row)
@@ -250,9 +266,65 @@ gptq_status chol_inv(gptq_ctx* c, int o, int h) {
   u12.Cthi = at(c->Ut_hi, o2, o);
   u12.Ctlo = at(c->Ut_lo, o2, o);
   u12.ldt = n;
-  if ((s = gemm_tc(c, h1, h2, h1, at(c->U_hi, o, o), at(c->U_lo, o, o), n, at(c->VT_hi, o2, o), at(c->VT_lo, o2, o),
-                   n, -1.f, 0, GT_KLO_ROW, GT_KHI_NONE, 0, u12)) != GPTQ_OK)
+  if ((s = gemm_tc(c, h1, h2, h1, opA(c->mA_U, o, o), opA(c->mB_VT, o2, o), -1.f, 0, GT_KLO_ROW, GT_KHI_NONE, 0,
+                   u12)) != GPTQ_OK)
     return s;
+  return GPTQ_OK;
+}
+
+// Encode the context's whole-matrix tensor maps (once, at create).
+gptq_status encode_maps(gptq_ctx* c) {
+  const int64_t n = c->n;
+  gptq_status s;
+  struct M {
+    CUtensorMap* m;
+    float* p;
+    int64_t rows, cols, ld;
+    int box;
+  } list[] = {
+      {&c->mA_A[0], c->A_hi, n, n, n, GT_BM},        {&c->mA_A[1], c->A_lo, n, n, n, GT_BM},
+      {&c->mA_VT[0], c->VT_hi, n, n, n, GT_BM},      {&c->mA_VT[1], c->VT_lo, n, n, n, GT_BM},
+      {&c->mA_U[0], c->U_hi, n, n, n, GT_BM},        {&c->mA_U[1], c->U_lo, n, n, n, GT_BM},
+      {&c->mA_Err[0], c->Err_hi, c->m_max, SW_B, SW_B, GT_BM},
+      {&c->mA_Err[1], c->Err_lo, c->m_max, SW_B, SW_B, GT_BM},
+      {&c->mB_U[0], c->U_hi, n, n, n, GT_BN},        {&c->mB_U[1], c->U_lo, n, n, n, GT_BN},
+      {&c->mB_VT[0], c->VT_hi, n, n, n, GT_BN},      {&c->mB_VT[1], c->VT_lo, n, n, n, GT_BN},
+      {&c->mB_Ut[0], c->Ut_hi, n, n, n, GT_BN},      {&c->mB_Ut[1], c->Ut_lo, n, n, n, GT_BN},
+  };
+  for (auto& e : list)
+    if ((s = make_map(c, e.m, e.p, e.rows, e.cols, e.ld, e.box)) != GPTQ_OK) return s;
+  return GPTQ_OK;
+}
+
+// Run the factorization recursion: recorded as a CUDA graph on first use (on a private
+// stream), then replayed on the context's stream.
+gptq_status run_factorization(gptq_ctx* c) {
+  if (!c->factor_graph) {
+    if (!c->capture_stream) CK(cudaStreamCreateWithFlags(&c->capture_stream, cudaStreamNonBlocking));
+    cudaStream_t user = c->stream;
+    const int64_t l0 = c->launches;
+    c->stream = c->capture_stream;
+    CK(cudaStreamBeginCapture(c->capture_stream, cudaStreamCaptureModeThreadLocal));
+    gptq_status s = chol_inv(c, 0, static_cast<int>(c->n));
+    cudaGraph_t g = nullptr;
+    cudaError_t e = cudaStreamEndCapture(c->capture_stream, &g);
+    c->stream = user;
+    if (s != GPTQ_OK || e != cudaSuccess) {
+      if (g) cudaGraphDestroy(g);
+      c->launches = l0;
+      return s != GPTQ_OK ? s : cuda_fail(e, "capture");
+    }
+    e = cudaGraphInstantiate(&c->factor_graph, g, 0);
+    cudaGraphDestroy(g);
+    if (e != cudaSuccess) {
+      c->factor_graph = nullptr;
+      return cuda_fail(e, "instantiate");
+    }
+    c->factor_graph_launches = c->launches - l0;
+    c->launches = l0;
+  }
+  CK(cudaGraphLaunch(c->factor_graph, c->stream));
+  c->launches += c->factor_graph_launches;
   return GPTQ_OK;
 }
 
@@ -266,6 +338,10 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 }
 
 void free_all(gptq_ctx* c) {
+  if (c->factor_graph) cudaGraphExecDestroy(c->factor_graph);
+  if (c->capture_stream) cudaStreamDestroy(c->capture_stream);
+  c->factor_graph = nullptr;
+  c->capture_stream = nullptr;
   float** fs[] = {&c->H,     &c->A_hi,  &c->A_lo,  &c->VT_hi, &c->VT_lo,  &c->U_hi,   &c->U_lo,
                   &c->Ut_hi, &c->Ut_lo, &c->Wq,    &c->Err_hi, &c->Err_lo, &c->keys};
   for (float** p : fs)
@@ -350,6 +426,7 @@ gptq_status gptq_create(gptq_ctx** out, int64_t n, int64_t m_max, int device, vo
   c->m_max = m_max;
   c->chunk_tokens = 512;
   c->encode = get_encode();
+  cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, device);
   const size_t nn = static_cast<size_t>(n) * n;
   cudaError_t e = cudaSuccess;
   auto alloc = [&](void** p, size_t bytes) {
@@ -372,6 +449,11 @@ gptq_status gptq_create(gptq_ctx** out, int64_t n, int64_t m_max, int device, vo
     free_all(c);
     delete c;
     return (e == cudaErrorMemoryAllocation) ? GPTQ_ERR_OOM : GPTQ_ERR_CUDA;
+  }
+  if (encode_maps(c) != GPTQ_OK) {
+    free_all(c);
+    delete c;
+    return GPTQ_ERR_CUDA;
   }
   e = cudaFuncSetAttribute(hessian_syrk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, HS_SMEM);
   if (e == cudaSuccess)
@@ -489,7 +571,7 @@ gptq_status gptq_prepare(gptq_ctx* c, double damp, int desc_act, int32_t* perm_o
   CKL("gather");
   const size_t nn = static_cast<size_t>(n) * n;
   for (float* p : {c->U_hi, c->U_lo, c->Ut_hi, c->Ut_lo}) CK(cudaMemsetAsync(p, 0, nn * 4, c->stream));
-  if ((s = chol_inv(c, 0, n)) != GPTQ_OK) return s;
+  if ((s = run_factorization(c)) != GPTQ_OK) return s;
   if (perm_out) CK(cudaMemcpyAsync(perm_out, c->perm, n * 4, cudaMemcpyDeviceToDevice, c->stream));
   int flags = 0;
   if ((s = read_status(c, &flags)) != GPTQ_OK) return s;
@@ -540,7 +622,7 @@ gptq_status gptq_quantize_layer(gptq_ctx* c, const void* W, int64_t m, gptq_qpar
   a.sym = qp.sym;
   a.g = g;
   a.G = n / g;
-  const int grid = (mi + SW_THREADS - 1) / SW_THREADS;
+  const int grid = (mi + SW_ROWS - 1) / SW_ROWS;
   for (int i1 = 0; i1 < n; i1 += SW_B) {
     if (g >= SW_B)
       sweep_block_kernel<0><<<grid, SW_THREADS, SW_SMEM, c->stream>>>(a, i1);
@@ -556,9 +638,8 @@ gptq_status gptq_quantize_layer(gptq_ctx* c, const void* W, int64_t m, gptq_qpar
       TcOut w;
       w.C = c->Wq + i2;
       w.ldc = n;
-      const size_t ub = static_cast<size_t>(i2) * n + i1;
-      gptq_status s = gemm_tc(c, mi, n - i2, SW_B, c->Err_hi, c->Err_lo, SW_B, c->Ut_hi + ub, c->Ut_lo + ub, n, -1.f,
-                              1, GT_KLO_NONE, GT_KHI_NONE, 0, w);
+      gptq_status s = gemm_tc(c, mi, n - i2, SW_B, TcOperand{&c->mA_Err[0], &c->mA_Err[1], 0, 0},
+                              TcOperand{&c->mB_Ut[0], &c->mB_Ut[1], i2, i1}, -1.f, 1, GT_KLO_NONE, GT_KHI_NONE, 0, w);
       if (s != GPTQ_OK) return s;
     }
   }
@@ -611,6 +692,7 @@ gptq_status gptq_test_gemm_tf32x3(int M, int N, int K, const float* A_hi, const 
   t.stream = static_cast<cudaStream_t>(cuda_stream);
   t.encode = get_encode();
   if (!t.encode) return GPTQ_ERR_CUDA;
+  cudaDeviceGetAttribute(&t.num_sms, cudaDevAttrMultiProcessorCount, device);
   CK(cudaFuncSetAttribute(gemm_tf32x3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GT_SMEM));
   CK(cudaMallocAsync(reinterpret_cast<void**>(&t.status), sizeof(int), t.stream));
   CK(cudaMemsetAsync(t.status, 0, sizeof(int), t.stream));
@@ -623,8 +705,15 @@ gptq_status gptq_test_gemm_tf32x3(int M, int N, int K, const float* A_hi, const 
   o.Cthi = Ct_hi;
   o.Ctlo = Ct_lo;
   o.ldt = ldt;
-  gptq_status s = gemm_tc(&t, M, N, K, A_hi, A_lo, lda, B_hi, B_lo, ldb, alpha, beta, k_lo_mode, k_hi_mode,
-                          upper_only, o);
+  CUtensorMap ma[2], mb[2];
+  gptq_status s = GPTQ_OK;
+  if (s == GPTQ_OK) s = make_map(&t, &ma[0], A_hi, M, K, lda, GT_BM);
+  if (s == GPTQ_OK) s = make_map(&t, &ma[1], A_lo, M, K, lda, GT_BM);
+  if (s == GPTQ_OK) s = make_map(&t, &mb[0], B_hi, N, K, ldb, GT_BN);
+  if (s == GPTQ_OK) s = make_map(&t, &mb[1], B_lo, N, K, ldb, GT_BN);
+  if (s == GPTQ_OK)
+    s = gemm_tc(&t, M, N, K, TcOperand{&ma[0], &ma[1], 0, 0}, TcOperand{&mb[0], &mb[1], 0, 0}, alpha, beta, k_lo_mode,
+                k_hi_mode, upper_only, o);
   int flags = 0;
   cudaMemcpyAsync(&flags, t.status, sizeof(int), cudaMemcpyDeviceToHost, t.stream);
   cudaError_t e = cudaStreamSynchronize(t.stream);
@@ -743,7 +832,7 @@ extern "C" gptq_status gptq_quantize_layer_noalloc(const void* W, int64_t m, int
   a.sym = qp.sym;
   a.g = g;
   a.G = ni / g;
-  const int grid = (mi + SW_THREADS - 1) / SW_THREADS;
+  const int grid = (mi + SW_ROWS - 1) / SW_ROWS;
   for (int i1 = 0; i1 < ni; i1 += SW_B) {
     if (g >= SW_B)
       sweep_block_kernel<0><<<grid, SW_THREADS, SW_SMEM, st>>>(a, i1);

@@ -198,14 +198,14 @@ __global__ void __launch_bounds__(HS_THREADS, 1)
       }
       tc_fence_after();
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                               static_cast<uint32_t>(b * HS_BN + hh * (HS_BN / 2) + cc * 32),
+      for (int cc = 0; cc < 8; ++cc) {
+        uint32_t v[16];
+        tmem_ld_32x32b_x16(tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                               static_cast<uint32_t>(b * HS_BN + hh * (HS_BN / 2) + cc * 16),
                            v);
         tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) acc[cc * 32 + j] += __uint_as_float(v[j]);
+        for (int j = 0; j < 16; ++j) acc[cc * 16 + j] += __uint_as_float(v[j]);
       }
       tc_fence_before();
       mbar_arrive(bar_tempty + 8 * b);

@@ -4,18 +4,18 @@
 //  each column's error into the not-yet-quantized columns; "模型量化实战…" §3.2
 //  quantize_block: blocks of 128 columns.)
 //
-// Rows of W are independent once U is known, so each thread owns one row.  The row's 128
-// block columns live in registers as eight 16-column sub-blocks R[0..7]; the U block
-// (upper 128 x 128) is in shared memory and every U read is a warp-wide broadcast.
-// For sub-block sb the thread
-//   1. (re)computes the group's min-max scale/zero from the current values when a group
-//      starts (groups of 32/64 inside the block; groups >= 128 at block starts),
-//   2. quantizes the 16 columns in order, e = (w - q) / U[i,i], and updates the remaining
-//      columns of the sub-block,
-//   3. applies the 16 errors to the later sub-blocks of the block (a 16 x 16 rank update
-//      each), then rotates the registers so the next sub-block is R[0].
-// The errors of the whole block go to Err [m x 128]; the columns after the block receive
-// them through one GEMM per block (S6) launched by the host.
+// Rows of W are independent once U is known.  Eight lanes of a warp share one row: lane
+// l (0..7 within its group) holds the row's block columns 16l .. 16l+15 in registers, so a
+// warp sweeps four rows and a 256-thread CTA 32 rows.  For column i the owning lane
+// (i / 16) computes the code, the dequantized value and e = (w - q) / U[i][i]; e is broadcast
+// to the row's lanes with a warp shuffle and every lane updates its 16 columns,
+// w[j] -= e * U[i][j].  U is upper-triangular, so the update leaves columns left of i
+// untouched without any masking.  Group scales/zeros come from a min/max over the group's
+// current values reduced across the row's lanes with shuffles.  The U block (128 x 128) is
+// staged in shared memory with asynchronous copies, in a bank-skewed layout so the eight
+// 16-column segments a warp reads at once hit different banks.
+// The block's errors go to Err [m x 128]; the columns after the block receive them through
+// one GEMM per block (S6) launched by the host.
 //
 // The integer decisions (code and zero-point) are taken in fp32 with IEEE division and
 // round-half-to-even, the precision the pages' own sketches use.
@@ -27,9 +27,21 @@
 
 namespace gptq {
 
-constexpr int SW_B = 128;       // sweep block (columns)
-constexpr int SW_THREADS = 32;  // rows per CTA
-constexpr int SW_SMEM = SW_B * SW_B * 4 + SW_B * 4 + SW_B * 4 + SW_B * SW_THREADS;
+constexpr int SW_B = 128;            // sweep block (columns)
+constexpr int SW_LANES = 8;          // lanes per row
+constexpr int SW_COLS = SW_B / SW_LANES;  // 16 columns per lane
+constexpr int SW_THREADS = 256;
+constexpr int SW_ROWS = SW_THREADS / SW_LANES;  // 32 rows per CTA
+constexpr int SW_SEG = 20;                      // skewed segment stride (floats) in shared memory
+constexpr int SW_ULD = SW_LANES * SW_SEG;       // 160 floats per staged U row
+constexpr int SW_SMEM = 2 * SW_B * SW_ULD * 4 + SW_B * 4 + SW_B * 4 + SW_ROWS * 32 * 4;
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n cp.async.wait_group 0;" ::: "memory");
+}
 
 struct SweepArgs {
   float* Wq;          // [m x n] fp32 working weights, sweep order
@@ -64,36 +76,45 @@ __device__ __forceinline__ void group_scale_zero(float wmin, float wmax, float a
   }
 }
 
+// min / max / max|.| over the eight lanes of a row group
+__device__ __forceinline__ void group_reduce(float& wmin, float& wmax, float& amax) {
+#pragma unroll
+  for (int o = 1; o < SW_LANES; o <<= 1) {
+    wmin = fminf(wmin, __shfl_xor_sync(0xffffffffu, wmin, o));
+    wmax = fmaxf(wmax, __shfl_xor_sync(0xffffffffu, wmax, o));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  }
+}
+
 template <int GSUB>  // 0: groups of >= 128 columns (params at block starts); 32 or 64: inside the block
 __global__ void __launch_bounds__(SW_THREADS)
     sweep_block_kernel(SweepArgs a, int i1) {
   extern __shared__ __align__(16) float sw_smem[];
-  float* Us = sw_smem;                                        // [128][128]
-  float* rU = Us + SW_B * SW_B;                               // [128] 1 / U[i][i]
-  int* perm_s = reinterpret_cast<int*>(rU + SW_B);            // [128]
-  uint8_t* code_s = reinterpret_cast<uint8_t*>(perm_s + SW_B);  // [128][32]
+  float* Us = sw_smem;                                          // [128][160] U block (skewed)
+  float* Ul = Us + SW_B * SW_ULD;                               // [128][160] lo part while it lands
+  float* rU = Ul + SW_B * SW_ULD;                               // [128] 1 / U[i][i]
+  int* perm_s = reinterpret_cast<int*>(rU + SW_B);              // [128]
+  uint32_t* cw = reinterpret_cast<uint32_t*>(perm_s + SW_B);    // [32 rows][32 words] packed codes
 
-  const int lane = threadIdx.x;
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int l8 = lane & (SW_LANES - 1);      // segment of the row this lane holds
+  const int gbase = lane & ~(SW_LANES - 1);  // first lane of the row's group
+  const int rloc = tid / SW_LANES;           // row within the CTA
   const int n = a.n;
-  for (int idx = lane; idx < SW_B * SW_B / 4; idx += SW_THREADS) {
-    const int k = idx / (SW_B / 4), j4 = idx % (SW_B / 4);
-    const size_t g = static_cast<size_t>(i1 + k) * n + i1 + 4 * j4;
-    float4 u = *reinterpret_cast<const float4*>(a.U + g);
-    if (a.U_lo) {
-      const float4 l = *reinterpret_cast<const float4*>(a.U_lo + g);
-      u.x += l.x;
-      u.y += l.y;
-      u.z += l.z;
-      u.w += l.w;
-    }
-    reinterpret_cast<float4*>(Us)[idx] = u;
-  }
-  for (int k = lane; k < SW_B; k += SW_THREADS) perm_s[k] = a.perm[i1 + k];
-  __syncthreads();
-  for (int k = lane; k < SW_B; k += SW_THREADS) rU[k] = 1.0f / Us[k * SW_B + k];
-  __syncthreads();
 
-  const int r = blockIdx.x * SW_THREADS + lane;
+  // stage U[i1 + k][i1 + j] at Us[k][SEG * (j / 16) + j % 16]
+  for (int idx = tid; idx < SW_B * (SW_B / 4); idx += SW_THREADS) {
+    const int k = idx / (SW_B / 4), j = (idx % (SW_B / 4)) * 4;
+    const size_t g = static_cast<size_t>(i1 + k) * n + i1 + j;
+    const int so = k * SW_ULD + (j / SW_COLS) * SW_SEG + (j % SW_COLS);
+    cp_async16(Us + so, a.U + g);
+    if (a.U_lo) cp_async16(Ul + so, a.U_lo + g);
+  }
+  if (tid < SW_B) perm_s[tid] = a.perm[i1 + tid];
+  for (int idx = tid; idx < SW_ROWS * 32; idx += SW_THREADS) cw[idx] = 0u;
+
+  const int r = blockIdx.x * SW_ROWS + rloc;
   const bool valid = r < a.m;
   const int rr = valid ? r : 0;
 
@@ -101,53 +122,58 @@ __global__ void __launch_bounds__(SW_THREADS)
   if (a.sym) {
     qp.lo = -static_cast<float>(1 << (a.bits - 1));
     qp.hi = static_cast<float>((1 << (a.bits - 1)) - 1);
-    qp.qmax_f = qp.hi;
   } else {
     qp.lo = 0.0f;
     qp.hi = static_cast<float>((1 << a.bits) - 1);
-    qp.qmax_f = qp.hi;
   }
+  qp.qmax_f = qp.hi;
   qp.zsym = static_cast<float>(1 << (a.bits - 1));
 
-  float R[8][16];
+  // this lane's 16 columns of the row, while U lands
+  float w[SW_COLS];
   {
-    const float4* src = reinterpret_cast<const float4*>(a.Wq + static_cast<size_t>(rr) * n + i1);
+    const float4* src = reinterpret_cast<const float4*>(a.Wq + static_cast<size_t>(rr) * n + i1 + SW_COLS * l8);
 #pragma unroll
-    for (int t = 0; t < 8; ++t)
-#pragma unroll
-      for (int j4 = 0; j4 < 4; ++j4) {
-        const float4 v = valid ? src[t * 4 + j4] : make_float4(0.f, 0.f, 0.f, 0.f);
-        R[t][4 * j4 + 0] = v.x;
-        R[t][4 * j4 + 1] = v.y;
-        R[t][4 * j4 + 2] = v.z;
-        R[t][4 * j4 + 3] = v.w;
-      }
+    for (int j4 = 0; j4 < SW_COLS / 4; ++j4) {
+      const float4 v = valid ? src[j4] : make_float4(0.f, 0.f, 0.f, 0.f);
+      w[4 * j4 + 0] = v.x;
+      w[4 * j4 + 1] = v.y;
+      w[4 * j4 + 2] = v.z;
+      w[4 * j4 + 3] = v.w;
+    }
   }
+  cp_async_wait_all();
+  __syncthreads();
+  if (a.U_lo) {
+    for (int idx = tid; idx < SW_B * SW_ULD; idx += SW_THREADS) Us[idx] += Ul[idx];
+    __syncthreads();
+  }
+  if (tid < SW_B) rU[tid] = 1.0f / Us[tid * SW_ULD + (tid / SW_COLS) * SW_SEG + (tid % SW_COLS)];
+  __syncthreads();
 
   float s = 1.0f, z = 0.0f;
   if (GSUB == 0) {
     const int gi = i1 / a.g;
     if (i1 % a.g == 0) {
-      float wmin = R[0][0], wmax = R[0][0], amax = 0.0f;
+      float wmin = w[0], wmax = w[0], amax = 0.0f;
 #pragma unroll
-      for (int t = 0; t < 8; ++t)
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          wmin = fminf(wmin, R[t][j]);
-          wmax = fmaxf(wmax, R[t][j]);
-          amax = fmaxf(amax, fabsf(R[t][j]));
-        }
-      if (valid) {
-        const float* rest = a.Wq + static_cast<size_t>(rr) * n;
-        for (int c = i1 + SW_B; c < i1 + a.g; ++c) {
-          const float w = rest[c];
-          wmin = fminf(wmin, w);
-          wmax = fmaxf(wmax, w);
-          amax = fmaxf(amax, fabsf(w));
+      for (int j = 0; j < SW_COLS; ++j) {
+        wmin = fminf(wmin, w[j]);
+        wmax = fmaxf(wmax, w[j]);
+        amax = fmaxf(amax, fabsf(w[j]));
+      }
+      if (valid) {  // columns of the group beyond this block (already up to date)
+        const float* row = a.Wq + static_cast<size_t>(rr) * n;
+        for (int c = i1 + SW_B + l8; c < i1 + a.g; c += SW_LANES) {
+          const float x = row[c];
+          wmin = fminf(wmin, x);
+          wmax = fmaxf(wmax, x);
+          amax = fmaxf(amax, fabsf(x));
         }
       }
+      group_reduce(wmin, wmax, amax);
       group_scale_zero(wmin, wmax, amax, qp, a.sym, s, z);
-      if (valid) {
+      if (valid && l8 == 0) {
         a.scales[static_cast<size_t>(rr) * a.G + gi] = s;
         a.zeros[static_cast<size_t>(rr) * a.G + gi] = z;
       }
@@ -157,108 +183,113 @@ __global__ void __launch_bounds__(SW_THREADS)
     }
   }
 
-  float* err_row = a.Err + static_cast<size_t>(rr) * SW_B;
-  float* what_row = a.W_hat ? a.W_hat + static_cast<size_t>(rr) * n : nullptr;
+  uint32_t mycode[SW_COLS];
+  float myerr[SW_COLS], mywhat[SW_COLS];
+#pragma unroll
+  for (int t = 0; t < SW_COLS; ++t) {
+    mycode[t] = 0u;
+    myerr[t] = 0.0f;
+    mywhat[t] = 0.0f;
+  }
+  const float* urow_base = Us + l8 * SW_SEG;
 
 #pragma unroll 1
-  for (int sb = 0; sb < 8; ++sb) {
-    const int c0 = sb * 16;  // first block column of R[0]
-    if (GSUB > 0 && (c0 % (GSUB > 0 ? GSUB : 1)) == 0) {
-      constexpr int NT = (GSUB > 0 ? GSUB : 16) / 16;
-      float wmin = R[0][0], wmax = R[0][0], amax = 0.0f;
+  for (int c = 0; c < SW_LANES; ++c) {  // chunk c = columns 16c .. 16c+15, owned by lane c of each row
+    if (GSUB > 0 && ((c * SW_COLS) % (GSUB > 0 ? GSUB : SW_COLS)) == 0) {
+      constexpr int NL = (GSUB > 0 ? GSUB : SW_COLS) / SW_COLS;  // lanes covering one group
+      const bool in = (l8 >= c) && (l8 < c + NL);
+      float wmin = in ? w[0] : INFINITY, wmax = in ? w[0] : -INFINITY, amax = 0.0f;
+      if (in) {
 #pragma unroll
-      for (int t = 0; t < NT; ++t)
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          wmin = fminf(wmin, R[t][j]);
-          wmax = fmaxf(wmax, R[t][j]);
-          amax = fmaxf(amax, fabsf(R[t][j]));
+        for (int j = 0; j < SW_COLS; ++j) {
+          wmin = fminf(wmin, w[j]);
+          wmax = fmaxf(wmax, w[j]);
+          amax = fmaxf(amax, fabsf(w[j]));
         }
+      }
+      group_reduce(wmin, wmax, amax);
       group_scale_zero(wmin, wmax, amax, qp, a.sym, s, z);
-      if (valid) {
-        const int gi = (i1 + c0) / a.g;
+      if (valid && l8 == 0) {
+        const int gi = (i1 + c * SW_COLS) / a.g;
         a.scales[static_cast<size_t>(rr) * a.G + gi] = s;
         a.zeros[static_cast<size_t>(rr) * a.G + gi] = z;
       }
     }
-
-    float E[16];
+    const bool owner = (l8 == c);
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const float w = R[0][k];
-      float v = __fdiv_rn(w, s);
+    for (int t = 0; t < SW_COLS; ++t) {
+      const int i = c * SW_COLS + t;
+      // every lane quantizes its column t; the owner's result is the one that counts
+      const float x = w[t];
+      float v = __fdiv_rn(x, s);
       if (!a.sym) v = __fadd_rn(v, z);
       const float q = fminf(fmaxf(rintf(v), qp.lo), qp.hi);
       const float what = a.sym ? __fmul_rn(q, s) : __fmul_rn(__fsub_rn(q, z), s);
-      code_s[(c0 + k) * SW_THREADS + lane] = static_cast<uint8_t>(static_cast<int>(q - qp.lo));
-      const float e = __fmul_rn(__fsub_rn(w, what), rU[c0 + k]);
-      E[k] = e;
-      if (what_row && valid) what_row[perm_s[c0 + k]] = what;
-      const float* urow = Us + (c0 + k) * SW_B + c0;
+      const float e_own = __fmul_rn(__fsub_rn(x, what), rU[i]);
+      if (owner) {
+        mycode[t] = static_cast<uint32_t>(static_cast<int>(q - qp.lo));
+        myerr[t] = e_own;
+        mywhat[t] = what;
+      }
+      const float e = __shfl_sync(0xffffffffu, e_own, gbase + c);
+      const float4* urow = reinterpret_cast<const float4*>(urow_base + i * SW_ULD);
 #pragma unroll
-      for (int j = k + 1; j < 16; ++j) R[0][j] = fmaf(-e, urow[j], R[0][j]);
-    }
-    if (valid) {
-      float4* ep = reinterpret_cast<float4*>(err_row + c0);
-      if (a.Err_lo) {
-        float4* lp = reinterpret_cast<float4*>(a.Err_lo + static_cast<size_t>(rr) * SW_B + c0);
-#pragma unroll
-        for (int j4 = 0; j4 < 4; ++j4) {
-          float hi[4], lo[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            hi[e] = tf32_round(E[4 * j4 + e]);
-            lo[e] = tf32_round(E[4 * j4 + e] - hi[e]);
-          }
-          ep[j4] = make_float4(hi[0], hi[1], hi[2], hi[3]);
-          lp[j4] = make_float4(lo[0], lo[1], lo[2], lo[3]);
-        }
-      } else {
-#pragma unroll
-        for (int j4 = 0; j4 < 4; ++j4) ep[j4] = make_float4(E[4 * j4], E[4 * j4 + 1], E[4 * j4 + 2], E[4 * j4 + 3]);
+      for (int j4 = 0; j4 < SW_COLS / 4; ++j4) {
+        const float4 u = urow[j4];
+        w[4 * j4 + 0] = fmaf(-e, u.x, w[4 * j4 + 0]);
+        w[4 * j4 + 1] = fmaf(-e, u.y, w[4 * j4 + 1]);
+        w[4 * j4 + 2] = fmaf(-e, u.z, w[4 * j4 + 2]);
+        w[4 * j4 + 3] = fmaf(-e, u.w, w[4 * j4 + 3]);
       }
     }
-#pragma unroll
-    for (int t = 1; t < 8; ++t) {
-      if (sb + t < 8) {
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const float4* urow = reinterpret_cast<const float4*>(Us + (c0 + k) * SW_B + c0 + 16 * t);
-#pragma unroll
-          for (int j4 = 0; j4 < 4; ++j4) {
-            const float4 u = urow[j4];
-            R[t][4 * j4 + 0] = fmaf(-E[k], u.x, R[t][4 * j4 + 0]);
-            R[t][4 * j4 + 1] = fmaf(-E[k], u.y, R[t][4 * j4 + 1]);
-            R[t][4 * j4 + 2] = fmaf(-E[k], u.z, R[t][4 * j4 + 2]);
-            R[t][4 * j4 + 3] = fmaf(-E[k], u.w, R[t][4 * j4 + 3]);
-          }
-        }
-      }
-    }
-#pragma unroll
-    for (int t = 0; t < 7; ++t)
-#pragma unroll
-      for (int j = 0; j < 16; ++j) R[t][j] = R[t + 1][j];
   }
 
-  // pack this row's 128 codes (LSB-first bit stream) and store them
+  // errors of this lane's 16 columns (hi/lo for the tensor-core update, or fp32)
+  if (valid) {
+    const size_t eo = static_cast<size_t>(rr) * SW_B + SW_COLS * l8;
+    float4* ep = reinterpret_cast<float4*>(a.Err + eo);
+    if (a.Err_lo) {
+      float4* lp = reinterpret_cast<float4*>(a.Err_lo + eo);
+#pragma unroll
+      for (int j4 = 0; j4 < SW_COLS / 4; ++j4) {
+        float hi[4], lo[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          hi[e] = tf32_round(myerr[4 * j4 + e]);
+          lo[e] = tf32_round(myerr[4 * j4 + e] - hi[e]);
+        }
+        ep[j4] = make_float4(hi[0], hi[1], hi[2], hi[3]);
+        lp[j4] = make_float4(lo[0], lo[1], lo[2], lo[3]);
+      }
+    } else {
+#pragma unroll
+      for (int j4 = 0; j4 < SW_COLS / 4; ++j4)
+        ep[j4] = make_float4(myerr[4 * j4], myerr[4 * j4 + 1], myerr[4 * j4 + 2], myerr[4 * j4 + 3]);
+    }
+    if (a.W_hat) {
+      float* wh = a.W_hat + static_cast<size_t>(rr) * n;
+#pragma unroll
+      for (int t = 0; t < SW_COLS; ++t) wh[perm_s[SW_COLS * l8 + t]] = mywhat[t];
+    }
+  }
+
+  // pack the row's 128 codes (LSB-first bit stream): each lane ORs its 16 codes into the
+  // row's words in shared memory, then the row's lanes store the words
+  const int bits = a.bits;
+  uint32_t* rw = cw + rloc * 32;
+#pragma unroll
+  for (int t = 0; t < SW_COLS; ++t) {
+    const int pos = (SW_COLS * l8 + t) * bits;
+    const uint32_t code = mycode[t];
+    atomicOr(&rw[pos >> 5], code << (pos & 31));
+    if ((pos & 31) + bits > 32) atomicOr(&rw[(pos >> 5) + 1], code >> (32 - (pos & 31)));
+  }
   __syncwarp();
   if (valid) {
-    const int bits = a.bits;
     const int words = 4 * bits;  // 128 * bits / 32
     const int ldc = n * bits / 32;
     uint32_t* dst = a.codes + static_cast<size_t>(rr) * ldc + (i1 * bits) / 32;
-    for (int w = 0; w < words; ++w) {
-      const int bit0 = w * 32;
-      const int k0 = bit0 / bits, k1 = (bit0 + 31) / bits;
-      uint32_t acc = 0;
-      for (int k = k0; k <= k1; ++k) {
-        const uint32_t c = code_s[k * SW_THREADS + lane];
-        const int pos = k * bits - bit0;
-        acc |= (pos >= 0) ? (c << pos) : (c >> (-pos));
-      }
-      dst[w] = acc;
-    }
+    for (int wi = l8; wi < words; wi += SW_LANES) dst[wi] = rw[wi];
   }
 }
 
