@@ -21,12 +21,14 @@ extern "C" {
  *   upper_only: skip output tiles wholly below the diagonal of C
  *   C         : fp32 output [M x N] (ldc) or NULL; C_hi/C_lo: hi/lo output (ldh) or NULL;
  *   Ct_hi/Ct_lo: transposed hi/lo output [N x M] (ldt) or NULL (beta applies to C and C_hi/C_lo).
+ *   chunk_stages: 32-wide K stages summed in one tensor-memory accumulator before the fp32
+ *               register add (1 = every stage; the trailing update of the sweep uses 4).
  * Requirements: N % 32 == 0, K % 32 == 0, 16-byte aligned bases, leading dimensions % 4 == 0.
  * Synchronizes the stream before returning.  Allocates a 4-byte status word (stream-ordered). */
 gptq_status gptq_test_gemm_tf32x3(int M, int N, int K, const float* A_hi, const float* A_lo, int lda, const float* B_hi,
                                   const float* B_lo, int ldb, float alpha, int beta, int k_lo_mode, int k_hi_mode,
                                   int upper_only, float* C, int ldc, float* C_hi, float* C_lo, int ldh, float* Ct_hi,
-                                  float* Ct_lo, int ldt, int device, void* cuda_stream);
+                                  float* Ct_lo, int ldt, int chunk_stages, int device, void* cuda_stream);
 
 #ifdef __cplusplus
 }

@@ -22,6 +22,7 @@ constexpr int LF_P = 32;       // panel width (one warp)
 constexpr int LF_THREADS = 256;
 constexpr int LF_LD = LF_NB + 1;
 constexpr int LF_SMEM = 3 * LF_NB * LF_LD * 4 + 16;
+static_assert(LF_NB * LF_NB <= LF_NB * LF_LD, "a staged block must fit in V (and in X)");
 
 __device__ __forceinline__ float tf32_round(float x) {
   uint32_t u = __float_as_uint(x);
@@ -61,9 +62,10 @@ __device__ __forceinline__ void leaf_diag_factor(float (*S)[LF_LD], float (*V)[L
     }
     // row c of the inverse (V[c][l] for l > c were written by earlier steps)
     __syncwarp();
-    float acc = 0.0f;
+    float acc4[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // four partial sums: a short dependent chain
 #pragma unroll
-    for (int l = c + 1; l < LF_P; ++l) acc = fmaf(V[P0 + c][P0 + l], x[l], acc);
+    for (int l = c + 1; l < LF_P; ++l) acc4[l & 3] = fmaf(V[P0 + c][P0 + l], x[l], acc4[l & 3]);
+    const float acc = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
     x[c] = (lane == c) ? rs : (lane > c ? -acc * rs : 0.0f);
   }
 #pragma unroll
@@ -86,12 +88,30 @@ __global__ void __launch_bounds__(LF_THREADS, 1)
   int* bad = reinterpret_cast<int*>(lf_smem + 3 * LF_NB * LF_LD);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) *bad = 0;
-  for (int idx = tid; idx < LF_NB * LF_NB; idx += LF_THREADS) {
-    const int i = idx / LF_NB, j = idx % LF_NB;
-    const size_t g = static_cast<size_t>(o + i) * n + o + j;
-    S[i][j] = (i <= j) ? A_hi[g] + A_lo[g] : 0.0f;
-    V[i][j] = 0.0f;
-    X[i][j] = 0.0f;
+  // stage A_hi into V's storage and A_lo into X's with asynchronous 16-byte copies, at an
+  // unpadded 128-float pitch (the 129-float rows of S are not 16-byte aligned)
+  {
+    float* th = &V[0][0];
+    float* tl = &X[0][0];
+    for (int idx = tid; idx < LF_NB * (LF_NB / 4); idx += LF_THREADS) {
+      const int i = idx / (LF_NB / 4), j = (idx % (LF_NB / 4)) * 4;
+      const size_t g = static_cast<size_t>(o + i) * n + o + j;
+      const uint32_t dh = smem_u32(th + i * LF_NB + j), dl = smem_u32(tl + i * LF_NB + j);
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dh), "l"(A_hi + g) : "memory");
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dl), "l"(A_lo + g) : "memory");
+    }
+    asm volatile("cp.async.commit_group;\n cp.async.wait_group 0;" ::: "memory");
+    __syncthreads();
+    for (int idx = tid; idx < LF_NB * LF_NB; idx += LF_THREADS) {
+      const int i = idx / LF_NB, j = idx % LF_NB;
+      const float v = th[i * LF_NB + j] + tl[i * LF_NB + j];
+      S[i][j] = (i <= j) ? v : 0.0f;
+    }
+    __syncthreads();
+    for (int idx = tid; idx < LF_NB * LF_LD; idx += LF_THREADS) {
+      (&V[0][0])[idx] = 0.0f;
+      (&X[0][0])[idx] = 0.0f;
+    }
   }
   __syncthreads();
 
@@ -136,14 +156,10 @@ __global__ void __launch_bounds__(LF_THREADS, 1)
     // in 4 x 4 tiles (bi <= bj); the tiles of the next diagonal block go to warp 0
     const int nb = P0 / 4, nd = LF_P / 4, d0 = nb - nd;  // next diagonal block = tile rows/cols [d0, nb)
     int t_begin, t_step, t_end;
-    if (warp == 0) {
-      t_begin = lane;
-      t_step = 32;
+    if (warp == 0 || warp == 4) {  // the two warps of scheduler 0 update the next diagonal block
+      t_begin = (warp == 4 ? 32 : 0) + lane;
+      t_step = 64;
       t_end = nd * (nd + 1) / 2;  // tiles inside the next diagonal block
-    } else if (warp == 4) {
-      t_begin = 0;
-      t_step = 1;
-      t_end = 0;
     } else {
       const int wi = (warp < 4) ? warp - 1 : warp - 2;  // 0..5
       t_begin = wi * 32 + lane;
@@ -152,7 +168,7 @@ __global__ void __launch_bounds__(LF_THREADS, 1)
     }
     for (int t = t_begin; t < t_end; t += t_step) {
       int bi, bj;
-      if (warp == 0) {  // enumerate the upper tiles of the next diagonal block
+      if (warp == 0 || warp == 4) {  // enumerate the upper tiles of the next diagonal block
         int jj = static_cast<int>((sqrtf(8.0f * t + 1.0f) - 1.0f) * 0.5f);
         while (jj * (jj + 1) / 2 > t) --jj;
         while ((jj + 1) * (jj + 2) / 2 <= t) ++jj;
@@ -197,7 +213,7 @@ __global__ void __launch_bounds__(LF_THREADS, 1)
         for (int b = 0; b < 4; ++b)
           if (i0 + a <= j0 + b) S[i0 + a][j0 + b] -= acc[a][b];
     }
-    if (warp == 0) __syncwarp();
+    if (warp == 0 || warp == 4) asm volatile("bar.sync 1, 64;" ::: "memory");  // next block updated
   }
   __syncthreads();
 
@@ -262,22 +278,28 @@ __global__ void __launch_bounds__(LF_THREADS, 1)
     __syncthreads();
   }
 
-  // ---- write U (hi/lo) and Ut = U^T (hi/lo) ----
-  for (int idx = tid; idx < LF_NB * LF_NB; idx += LF_THREADS) {
-    const int i = idx / LF_NB, j = idx % LF_NB;
-    const float u = (i <= j) ? X[i][j] : 0.0f;
-    const float hi = tf32_round(u);
+  // ---- write U (hi/lo) and Ut = U^T (hi/lo), 16-byte stores ----
+  for (int idx = tid; idx < LF_NB * (LF_NB / 4); idx += LF_THREADS) {
+    const int i = idx / (LF_NB / 4), j = (idx % (LF_NB / 4)) * 4;
+    float u[4], ut[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      u[e] = (i <= j + e) ? X[i][j + e] : 0.0f;   // U[i][j+e]
+      ut[e] = (j + e <= i) ? X[j + e][i] : 0.0f;  // Ut[i][j+e] = U[j+e][i]
+    }
+    float uh[4], ul[4], th[4], tl[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      uh[e] = tf32_round(u[e]);
+      ul[e] = tf32_round(u[e] - uh[e]);
+      th[e] = tf32_round(ut[e]);
+      tl[e] = tf32_round(ut[e] - th[e]);
+    }
     const size_t g = static_cast<size_t>(o + i) * n + o + j;
-    U_hi[g] = hi;
-    U_lo[g] = tf32_round(u - hi);
-  }
-  for (int idx = tid; idx < LF_NB * LF_NB; idx += LF_THREADS) {
-    const int j = idx / LF_NB, i = idx % LF_NB;  // Ut[j][i] = U[i][j]
-    const float u = (i <= j) ? X[i][j] : 0.0f;
-    const float hi = tf32_round(u);
-    const size_t g = static_cast<size_t>(o + j) * n + o + i;
-    Ut_hi[g] = hi;
-    Ut_lo[g] = tf32_round(u - hi);
+    *reinterpret_cast<float4*>(U_hi + g) = make_float4(uh[0], uh[1], uh[2], uh[3]);
+    *reinterpret_cast<float4*>(U_lo + g) = make_float4(ul[0], ul[1], ul[2], ul[3]);
+    *reinterpret_cast<float4*>(Ut_hi + g) = make_float4(th[0], th[1], th[2], th[3]);
+    *reinterpret_cast<float4*>(Ut_lo + g) = make_float4(tl[0], tl[1], tl[2], tl[3]);
   }
   if (tid == 0 && *bad) atomicOr(status, ST_NOT_PD);
 }

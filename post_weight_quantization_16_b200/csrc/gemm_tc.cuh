@@ -47,6 +47,7 @@ struct GemmTCArgs {
   float alpha;
   int beta;          // 0 or 1: add the existing C (plain or hi+lo)
   int k_lo_mode, k_hi_mode, upper_only;
+  int chunk_stages;  // K stages summed in one TMEM accumulator before the fp32 register add
   float* C;          // plain fp32 output (or nullptr)
   int ldc;
   float* Chi;        // hi/lo output (or nullptr)
@@ -64,12 +65,32 @@ __device__ __forceinline__ float tf32_rn(float x) {
   return __uint_as_float(u & 0xFFFFE000u);
 }
 
-// Tile t of the output (n-tiles fastest); returns false for tiles skipped by upper_only.
-__device__ __forceinline__ bool gt_tile(const GemmTCArgs& p, int t, int ntn, int& m0, int& n0, int& k_begin,
-                                       int& n_iters) {
-  m0 = (t / ntn) * GT_BM;
-  n0 = (t % ntn) * GT_BN;
-  if (p.upper_only && m0 >= n0 + GT_BN) return false;
+// Number of output tiles the kernel visits: all of them, or with upper_only only the tiles
+// that reach the upper triangle (tile (mt, nt) is needed iff mt < 2 nt + 2).
+__host__ __device__ inline int gt_num_tiles(int M, int N, int upper_only) {
+  const int mtn = (M + GT_BM - 1) / GT_BM, ntn = (N + GT_BN - 1) / GT_BN;
+  if (!upper_only) return mtn * ntn;
+  int c = 0;
+  for (int nt = 0; nt < ntn; ++nt) c += min(mtn, 2 * nt + 2);
+  return c;
+}
+
+// Tile t (n-tiles fastest, or with upper_only column by column over the needed tiles).
+__device__ __forceinline__ void gt_tile(const GemmTCArgs& p, int t, int& m0, int& n0, int& k_begin, int& n_iters) {
+  const int mtn = (p.M + GT_BM - 1) / GT_BM, ntn = (p.N + GT_BN - 1) / GT_BN;
+  if (!p.upper_only) {
+    m0 = (t / ntn) * GT_BM;
+    n0 = (t % ntn) * GT_BN;
+  } else {
+    int nt = 0;
+    for (;; ++nt) {
+      const int cnt = min(mtn, 2 * nt + 2);
+      if (t < cnt || nt == ntn - 1) break;
+      t -= cnt;
+    }
+    m0 = t * GT_BM;
+    n0 = nt * GT_BN;
+  }
   int kb = 0, ke = p.K;
   if (p.k_lo_mode == GT_KLO_COL) kb = n0;
   if (p.k_lo_mode == GT_KLO_ROW) kb = m0;
@@ -77,7 +98,6 @@ __device__ __forceinline__ bool gt_tile(const GemmTCArgs& p, int t, int ntn, int
   kb = (kb / GT_BK) * GT_BK;
   k_begin = kb;
   n_iters = (ke > kb) ? (ke - kb + GT_BK - 1) / GT_BK : 0;
-  return true;
 }
 
 // Persistent: CTA b handles tiles b, b + gridDim.x, ...  The producer and the MMA issuer run
@@ -95,8 +115,7 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int ntn = (p.N + GT_BN - 1) / GT_BN;
-  const int ntiles = ntn * ((p.M + GT_BM - 1) / GT_BM);
+  const int ntiles = gt_num_tiles(p.M, p.N, p.upper_only);
 
   const uint32_t bar_full = sbase + GT_STAGES * GT_STAGE_BYTES;
   const uint32_t bar_empty = bar_full + 8 * GT_STAGES;
@@ -141,7 +160,7 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
         int m0, n0, kb, ni;
-        if (!gt_tile(p, t, ntn, m0, n0, kb, ni)) continue;
+        gt_tile(p, t, m0, n0, kb, ni);
         for (int j = 0; j < ni; ++j, ++it) {
           const int s = it % GT_STAGES;
           const uint32_t ph = static_cast<uint32_t>(it / GT_STAGES) & 1u;
@@ -164,19 +183,24 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      // ---------------- MMA issuer: one TMEM buffer per K stage ----------------
+      // ---------------- MMA issuer: one TMEM buffer per chunk of K stages ----------------
       constexpr uint32_t idesc = idesc_make(2u, 2u, 0u, 0u, GT_BM, GT_BN);  // tf32, K-major A and B
+      const int cs = p.chunk_stages;
       bool ok = true;
-      int it = 0;
+      int it = 0, ch = 0;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
         int m0, n0, kb, ni;
-        if (!gt_tile(p, t, ntn, m0, n0, kb, ni)) continue;
+        gt_tile(p, t, m0, n0, kb, ni);
+        int b = 0;
         for (int j = 0; j < ni; ++j, ++it) {
-          const int b = it & 1;
-          const uint32_t ph = static_cast<uint32_t>(it >> 1) & 1u;
-          if (!mbar_wait_bounded(bar_tempty + 8 * b, ph ^ 1u, abort_flag)) {
-            ok = false;
-            break;
+          const bool first = (j % cs) == 0;
+          if (first) {
+            b = ch & 1;
+            const uint32_t ph = static_cast<uint32_t>(ch >> 1) & 1u;
+            if (!mbar_wait_bounded(bar_tempty + 8 * b, ph ^ 1u, abort_flag)) {
+              ok = false;
+              break;
+            }
           }
           const int s = it % GT_STAGES;
           const uint32_t phs = static_cast<uint32_t>(it / GT_STAGES) & 1u;
@@ -194,12 +218,15 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
             const uint32_t off = kk * 32;  // 8 fp32 of K inside the 128-byte swizzle row
             const uint64_t dah = sdesc_sw128(sa_hi + off, 16, 1024), dal = sdesc_sw128(sa_lo + off, 16, 1024);
             const uint64_t dbh = sdesc_sw128(sb_hi + off, 16, 1024), dbl = sdesc_sw128(sb_lo + off, 16, 1024);
-            umma_tf32(d_tmem, dal, dbh, idesc, kk > 0 ? 1u : 0u);
+            umma_tf32(d_tmem, dal, dbh, idesc, (first && kk == 0) ? 0u : 1u);
             umma_tf32(d_tmem, dah, dbl, idesc, 1u);
             umma_tf32(d_tmem, dah, dbh, idesc, 1u);
           }
           umma_commit(bar_empty + 8 * s);
-          umma_commit(bar_tfull + 8 * b);
+          if ((j % cs) == cs - 1 || j == ni - 1) {
+            umma_commit(bar_tfull + 8 * b);
+            ++ch;
+          }
         }
       }
       if (!ok) {
@@ -211,11 +238,11 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
     // ---------------- epilogue ----------------
     const int q = warp & 3;
     const int hh = (warp - 2) >> 2;
-    int it = 0;
+    int ch = 0;
     bool all_ok = true;
     for (int t = blockIdx.x; t < ntiles && all_ok; t += gridDim.x) {
       int m0, n0, kb, ni;
-      if (!gt_tile(p, t, ntn, m0, n0, kb, ni)) continue;
+      gt_tile(p, t, m0, n0, kb, ni);
       const int r = m0 + q * 32 + lane;
       const int cbase = n0 + hh * (GT_BN / 2);
       const bool row_ok = r < p.M;
@@ -251,9 +278,10 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
           for (int j = 0; j < 32; ++j) acc[cc * 32 + j] = 0.0f;
         }
       }
-      for (int j = 0; j < ni; ++j, ++it) {
-        const int b = it & 1;
-        const uint32_t ph = static_cast<uint32_t>(it >> 1) & 1u;
+      const int nch = (ni + p.chunk_stages - 1) / p.chunk_stages;
+      for (int j = 0; j < nch; ++j, ++ch) {
+        const int b = ch & 1;
+        const uint32_t ph = static_cast<uint32_t>(ch >> 1) & 1u;
         int ok = 0;
         if (lane == 0) ok = mbar_wait_bounded(bar_tfull + 8 * b, ph, abort_flag) ? 1 : 0;
         ok = __shfl_sync(0xffffffffu, ok, 0);

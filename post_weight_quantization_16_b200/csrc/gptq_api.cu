@@ -29,6 +29,7 @@ namespace {
 enum CtxState { ST_ACCUM = 0, ST_PREPARED = 1 };
 
 constexpr int64_t kMaxN = 32768;
+constexpr int kSuperBlock = 1024;  // columns whose block errors are applied beyond them in one product
 constexpr int64_t kMaxM = int64_t(1) << 24;
 
 }  // namespace
@@ -43,7 +44,7 @@ struct gptq_ctx {
   float *U_hi = nullptr, *U_lo = nullptr;      // [n x n] U (upper)
   float *Ut_hi = nullptr, *Ut_lo = nullptr;    // [n x n] U^T
   float* Wq = nullptr;                         // [m_max x n] fp32 working weights
-  float *Err_hi = nullptr, *Err_lo = nullptr;  // [m_max x 128]
+  float *Err_hi = nullptr, *Err_lo = nullptr;  // [m_max x kSuperBlock] block errors of a super-block
   float* keys = nullptr;
   uint8_t* dead = nullptr;
   int32_t* perm = nullptr;
@@ -175,18 +176,62 @@ struct TcOut {
   int ldt = 0;
 };
 
-// An operand of gemm_tc: the hi/lo tensor maps of a whole matrix and the sub-block offset.
+// An operand of gemm_tc: the hi/lo tensor maps of a whole matrix and the sub-block offset,
+// plus the sub-block's hi/lo pointers and leading dimension (for the CUDA-core path).
 struct TcOperand {
   const CUtensorMap* hi;
   const CUtensorMap* lo;
   int row0, col0;
+  const float* phi;
+  const float* plo;
+  int ld;
 };
 
+// Products with fewer tensor-core tiles than this run on the CUDA cores (fp32, 64 x 64 tiles).
+constexpr int kMinTcTiles = 32;
+
 gptq_status gemm_tc(gptq_ctx* c, int M, int N, int K, TcOperand A, TcOperand B, float alpha, int beta, int klo,
-                    int khi, int upper, const TcOut& o) {
+                    int khi, int upper, const TcOut& o, int chunk_stages = 1) {
   if (M <= 0 || N <= 0) return GPTQ_OK;
   if (N % 32 || K % GT_BK) return GPTQ_ERR_ARG;
+  const int tc_tiles = gt_num_tiles(M, N, upper);
+  if (tc_tiles < kMinTcTiles && A.phi && B.phi) {
+    GemmSimtArgs g;
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    g.A_hi = A.phi;
+    g.A_lo = A.plo;
+    g.lda = A.ld;
+    g.B_hi = B.phi;
+    g.B_lo = B.plo;
+    g.ldb = B.ld;
+    g.alpha = alpha;
+    g.beta = beta;
+    g.k_lo_mode = klo;
+    g.k_hi_mode = khi;
+    g.upper_only = upper;
+    g.C = o.C;
+    g.ldc = o.ldc;
+    g.Chi = o.Chi;
+    g.Clo = o.Clo;
+    g.ldh = o.ldh;
+    g.Cthi = o.Cthi;
+    g.Ctlo = o.Ctlo;
+    g.ldt = o.ldt;
+    if (static_cast<int64_t>(M) * N <= 512 * 512) {  // 32 x 32 tiles: more CTAs for the smallest products
+      dim3 grid((N + 31) / 32, (M + 31) / 32);
+      gemm_hilo_simt_kernel<32, 32><<<grid, GS_THREADS, gs_smem_bytes<32, 32>(), c->stream>>>(g);
+    } else {
+      dim3 grid((N + 63) / 64, (M + 63) / 64);
+      gemm_hilo_simt_kernel<64, 64><<<grid, GS_THREADS, gs_smem_bytes<64, 64>(), c->stream>>>(g);
+    }
+    ++c->launches;
+    CKL("gemm_simt");
+    return GPTQ_OK;
+  }
   GemmTCArgs a;
+  a.chunk_stages = chunk_stages;
   a.M = M;
   a.N = N;
   a.K = K;
@@ -208,9 +253,8 @@ gptq_status gemm_tc(gptq_ctx* c, int M, int N, int K, TcOperand A, TcOperand B, 
   a.Ctlo = o.Ctlo;
   a.ldt = o.ldt;
   a.status = c->status;
-  const int ntiles = ((N + GT_BN - 1) / GT_BN) * ((M + GT_BM - 1) / GT_BM);
-  gemm_tf32x3_kernel<<<std::min(ntiles, c->num_sms), GT_THREADS, GT_SMEM, c->stream>>>(*A.hi, *A.lo, *B.hi, *B.lo,
-                                                                                       a);
+  gemm_tf32x3_kernel<<<std::min(tc_tiles, c->num_sms), GT_THREADS, GT_SMEM, c->stream>>>(*A.hi, *A.lo, *B.hi,
+                                                                                         *B.lo, a);
   ++c->launches;
   CKL("gemm_tc");
   return GPTQ_OK;
@@ -232,13 +276,16 @@ gptq_status chol_inv(gptq_ctx* c, int o, int h) {
   auto at = [n](float* M, int r, int col) { return M + static_cast<size_t>(r) * n + col; };
   gptq_status s;
   if ((s = chol_inv(c, o2, h2)) != GPTQ_OK) return s;
-  auto opA = [](CUtensorMap* m, int r0, int c0) { return TcOperand{&m[0], &m[1], r0, c0}; };
+  auto op = [n](CUtensorMap* m, float* hi, float* lo, int r0, int c0) {
+    return TcOperand{&m[0], &m[1], r0, c0, hi + static_cast<size_t>(r0) * n + c0, lo + static_cast<size_t>(r0) * n + c0,
+                     n};
+  };
   // V12 = A12 U22^T                      (U22 rows are the K-major B; k >= column)
   TcOut v12;
   v12.Chi = at(c->VT_hi, o, o2);
   v12.Clo = at(c->VT_lo, o, o2);
   v12.ldh = n;
-  if ((s = gemm_tc(c, h1, h2, h2, opA(c->mA_A, o, o2), opA(c->mB_U, o2, o2), 1.f, 0, GT_KLO_COL, GT_KHI_NONE, 0,
+  if ((s = gemm_tc(c, h1, h2, h2, op(c->mA_A, c->A_hi, c->A_lo, o, o2), op(c->mB_U, c->U_hi, c->U_lo, o2, o2), 1.f, 0, GT_KLO_COL, GT_KHI_NONE, 0,
                    v12)) != GPTQ_OK)
     return s;
   // A11 -= V12 V12^T                     (upper tiles only)
@@ -246,7 +293,7 @@ gptq_status chol_inv(gptq_ctx* c, int o, int h) {
   a11.Chi = at(c->A_hi, o, o);
   a11.Clo = at(c->A_lo, o, o);
   a11.ldh = n;
-  if ((s = gemm_tc(c, h1, h1, h2, opA(c->mA_VT, o, o2), opA(c->mB_VT, o, o2), -1.f, 1, GT_KLO_NONE, GT_KHI_NONE, 1,
+  if ((s = gemm_tc(c, h1, h1, h2, op(c->mA_VT, c->VT_hi, c->VT_lo, o, o2), op(c->mB_VT, c->VT_hi, c->VT_lo, o, o2), -1.f, 1, GT_KLO_NONE, GT_KHI_NONE, 1,
                    a11)) != GPTQ_OK)
     return s;
   // T^T = (V12 U22)^T into the lower block [o2.., o..]   (Ut22 rows as B; k <= column)
@@ -254,7 +301,7 @@ gptq_status chol_inv(gptq_ctx* c, int o, int h) {
   tt.Cthi = at(c->VT_hi, o2, o);
   tt.Ctlo = at(c->VT_lo, o2, o);
   tt.ldt = n;
-  if ((s = gemm_tc(c, h1, h2, h2, opA(c->mA_VT, o, o2), opA(c->mB_Ut, o2, o2), 1.f, 0, GT_KLO_NONE, GT_KHI_COL, 0,
+  if ((s = gemm_tc(c, h1, h2, h2, op(c->mA_VT, c->VT_hi, c->VT_lo, o, o2), op(c->mB_Ut, c->Ut_hi, c->Ut_lo, o2, o2), 1.f, 0, GT_KLO_NONE, GT_KHI_COL, 0,
                    tt)) != GPTQ_OK)
     return s;
   if ((s = chol_inv(c, o, h1)) != GPTQ_OK) return s;
@@ -266,7 +313,7 @@ gptq_status chol_inv(gptq_ctx* c, int o, int h) {
   u12.Cthi = at(c->Ut_hi, o2, o);
   u12.Ctlo = at(c->Ut_lo, o2, o);
   u12.ldt = n;
-  if ((s = gemm_tc(c, h1, h2, h1, opA(c->mA_U, o, o), opA(c->mB_VT, o2, o), -1.f, 0, GT_KLO_ROW, GT_KHI_NONE, 0,
+  if ((s = gemm_tc(c, h1, h2, h1, op(c->mA_U, c->U_hi, c->U_lo, o, o), op(c->mB_VT, c->VT_hi, c->VT_lo, o2, o), -1.f, 0, GT_KLO_ROW, GT_KHI_NONE, 0,
                    u12)) != GPTQ_OK)
     return s;
   return GPTQ_OK;
@@ -285,8 +332,8 @@ gptq_status encode_maps(gptq_ctx* c) {
       {&c->mA_A[0], c->A_hi, n, n, n, GT_BM},        {&c->mA_A[1], c->A_lo, n, n, n, GT_BM},
       {&c->mA_VT[0], c->VT_hi, n, n, n, GT_BM},      {&c->mA_VT[1], c->VT_lo, n, n, n, GT_BM},
       {&c->mA_U[0], c->U_hi, n, n, n, GT_BM},        {&c->mA_U[1], c->U_lo, n, n, n, GT_BM},
-      {&c->mA_Err[0], c->Err_hi, c->m_max, SW_B, SW_B, GT_BM},
-      {&c->mA_Err[1], c->Err_lo, c->m_max, SW_B, SW_B, GT_BM},
+      {&c->mA_Err[0], c->Err_hi, c->m_max, kSuperBlock, kSuperBlock, GT_BM},
+      {&c->mA_Err[1], c->Err_lo, c->m_max, kSuperBlock, kSuperBlock, GT_BM},
       {&c->mB_U[0], c->U_hi, n, n, n, GT_BN},        {&c->mB_U[1], c->U_lo, n, n, n, GT_BN},
       {&c->mB_VT[0], c->VT_hi, n, n, n, GT_BN},      {&c->mB_VT[1], c->VT_lo, n, n, n, GT_BN},
       {&c->mB_Ut[0], c->Ut_hi, n, n, n, GT_BN},      {&c->mB_Ut[1], c->Ut_lo, n, n, n, GT_BN},
@@ -393,7 +440,7 @@ size_t gptq_workspace_bytes(int64_t n, int64_t m_max) {
   const size_t nn = static_cast<size_t>(n) * static_cast<size_t>(n);
   size_t b = 9 * nn * sizeof(float);                                              // H, A, VT, U, Ut (hi/lo)
   b += static_cast<size_t>(m_max) * static_cast<size_t>(n) * sizeof(float);       // Wq
-  b += 2 * static_cast<size_t>(m_max) * SW_B * sizeof(float);                     // Err hi/lo
+  b += 2 * static_cast<size_t>(m_max) * kSuperBlock * sizeof(float);              // Err hi/lo
   b += static_cast<size_t>(n) * (sizeof(float) + 1 + sizeof(int32_t)) + sizeof(double) + sizeof(int);
   return b;
 }
@@ -436,8 +483,8 @@ gptq_status gptq_create(gptq_ctx** out, int64_t n, int64_t m_max, int device, vo
   for (float** p : {&c->A_hi, &c->A_lo, &c->VT_hi, &c->VT_lo, &c->U_hi, &c->U_lo, &c->Ut_hi, &c->Ut_lo})
     alloc(reinterpret_cast<void**>(p), nn * 4);
   alloc(reinterpret_cast<void**>(&c->Wq), static_cast<size_t>(m_max) * n * 4);
-  alloc(reinterpret_cast<void**>(&c->Err_hi), static_cast<size_t>(m_max) * SW_B * 4);
-  alloc(reinterpret_cast<void**>(&c->Err_lo), static_cast<size_t>(m_max) * SW_B * 4);
+  alloc(reinterpret_cast<void**>(&c->Err_hi), static_cast<size_t>(m_max) * kSuperBlock * 4);
+  alloc(reinterpret_cast<void**>(&c->Err_lo), static_cast<size_t>(m_max) * kSuperBlock * 4);
   alloc(reinterpret_cast<void**>(&c->keys), n * 4);
   alloc(reinterpret_cast<void**>(&c->dead), n);
   alloc(reinterpret_cast<void**>(&c->perm), n * 4);
@@ -460,6 +507,12 @@ gptq_status gptq_create(gptq_ctx** out, int64_t n, int64_t m_max, int device, vo
     e = cudaFuncSetAttribute(gemm_tf32x3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GT_SMEM);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(leaf_chol_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, LF_SMEM);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(gemm_hilo_simt_kernel<64, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             gs_smem_bytes<64, 64>());
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(gemm_hilo_simt_kernel<32, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             gs_smem_bytes<32, 32>());
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(sweep_block_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, SW_SMEM);
   if (e == cudaSuccess)
@@ -622,25 +675,45 @@ gptq_status gptq_quantize_layer(gptq_ctx* c, const void* W, int64_t m, gptq_qpar
   a.sym = qp.sym;
   a.g = g;
   a.G = n / g;
+  a.ld_err = kSuperBlock;
   const int grid = (mi + SW_ROWS - 1) / SW_ROWS;
-  for (int i1 = 0; i1 < n; i1 += SW_B) {
-    if (g >= SW_B)
-      sweep_block_kernel<0><<<grid, SW_THREADS, SW_SMEM, c->stream>>>(a, i1);
-    else if (g == 64)
-      sweep_block_kernel<64><<<grid, SW_THREADS, SW_SMEM, c->stream>>>(a, i1);
-    else
-      sweep_block_kernel<32><<<grid, SW_THREADS, SW_SMEM, c->stream>>>(a, i1);
-    ++c->launches;
-    CKL("sweep");
-    const int i2 = i1 + SW_B;
-    if (i2 < n) {
-      // W[:, i2:] -= Err * U[i1:i2, i2:]   (B in K-major form: rows i2.. of U^T, columns i1..i2)
+  // two-level lazy update: inside a super-block the columns after each 128-block are updated
+  // right away; the columns beyond the super-block receive all its block errors in one product
+  // (K = super-block width).  A group that starts inside a super-block must not reach past it.
+  const int sb = ((g <= kSuperBlock && kSuperBlock % g == 0) || g % kSuperBlock == 0 || g == n) ? kSuperBlock : SW_B;
+  for (int s0 = 0; s0 < n; s0 += sb) {
+    const int s1 = std::min(n, s0 + sb);
+    for (int i1 = s0; i1 < s1; i1 += SW_B) {
+      a.err_col0 = i1 - s0;
+      if (g >= SW_B)
+        sweep_block_kernel<0><<<grid, SW_THREADS, SW_SMEM, c->stream>>>(a, i1);
+      else if (g == 64)
+        sweep_block_kernel<64><<<grid, SW_THREADS, SW_SMEM, c->stream>>>(a, i1);
+      else
+        sweep_block_kernel<32><<<grid, SW_THREADS, SW_SMEM, c->stream>>>(a, i1);
+      ++c->launches;
+      CKL("sweep");
+      const int i2 = i1 + SW_B;
+      if (i2 < s1) {
+        // W[:, i2:s1] -= Err_blk * U[i1:i2, i2:s1]   (B in K-major form: rows of U^T)
+        TcOut w;
+        w.C = c->Wq + i2;
+        w.ldc = n;
+        gptq_status st = gemm_tc(c, mi, s1 - i2, SW_B, TcOperand{&c->mA_Err[0], &c->mA_Err[1], 0, i1 - s0, nullptr, nullptr, 0},
+                                 TcOperand{&c->mB_Ut[0], &c->mB_Ut[1], i2, i1, nullptr, nullptr, 0}, -1.f, 1,
+                                 GT_KLO_NONE, GT_KHI_NONE, 0, w, SW_B / GT_BK);
+        if (st != GPTQ_OK) return st;
+      }
+    }
+    if (s1 < n) {
+      // W[:, s1:] -= Err_super * U[s0:s1, s1:]   (K = s1 - s0; 128-wide TMEM chunks)
       TcOut w;
-      w.C = c->Wq + i2;
+      w.C = c->Wq + s1;
       w.ldc = n;
-      gptq_status s = gemm_tc(c, mi, n - i2, SW_B, TcOperand{&c->mA_Err[0], &c->mA_Err[1], 0, 0},
-                              TcOperand{&c->mB_Ut[0], &c->mB_Ut[1], i2, i1}, -1.f, 1, GT_KLO_NONE, GT_KHI_NONE, 0, w);
-      if (s != GPTQ_OK) return s;
+      gptq_status st = gemm_tc(c, mi, n - s1, s1 - s0, TcOperand{&c->mA_Err[0], &c->mA_Err[1], 0, 0, nullptr, nullptr, 0},
+                               TcOperand{&c->mB_Ut[0], &c->mB_Ut[1], s1, s0, nullptr, nullptr, 0}, -1.f, 1,
+                               GT_KLO_NONE, GT_KHI_NONE, 0, w, SW_B / GT_BK);
+      if (st != GPTQ_OK) return st;
     }
   }
   if (g_idx) {
@@ -675,7 +748,8 @@ int64_t gptq_launch_count(const gptq_ctx* c) { return c ? c->launches : -1; }
 gptq_status gptq_test_gemm_tf32x3(int M, int N, int K, const float* A_hi, const float* A_lo, int lda, const float* B_hi,
                                   const float* B_lo, int ldb, float alpha, int beta, int k_lo_mode, int k_hi_mode,
                                   int upper_only, float* C, int ldc, float* C_hi, float* C_lo, int ldh, float* Ct_hi,
-                                  float* Ct_lo, int ldt, int device, void* cuda_stream) {
+                                  float* Ct_lo, int ldt, int chunk_stages, int device, void* cuda_stream) {
+  if (chunk_stages < 1) return GPTQ_ERR_ARG;
   if (!A_hi || !A_lo || !B_hi || !B_lo || M < 1 || N < 1 || K < GT_BK) return GPTQ_ERR_ARG;
   if (k_lo_mode < 0 || k_lo_mode > 2 || k_hi_mode < 0 || k_hi_mode > 1 || (beta != 0 && beta != 1)) return GPTQ_ERR_ARG;
   if ((C_hi == nullptr) != (C_lo == nullptr) || (Ct_hi == nullptr) != (Ct_lo == nullptr)) return GPTQ_ERR_ARG;
@@ -712,8 +786,9 @@ gptq_status gptq_test_gemm_tf32x3(int M, int N, int K, const float* A_hi, const 
   if (s == GPTQ_OK) s = make_map(&t, &mb[0], B_hi, N, K, ldb, GT_BN);
   if (s == GPTQ_OK) s = make_map(&t, &mb[1], B_lo, N, K, ldb, GT_BN);
   if (s == GPTQ_OK)
-    s = gemm_tc(&t, M, N, K, TcOperand{&ma[0], &ma[1], 0, 0}, TcOperand{&mb[0], &mb[1], 0, 0}, alpha, beta, k_lo_mode,
-                k_hi_mode, upper_only, o);
+    s = gemm_tc(&t, M, N, K, TcOperand{&ma[0], &ma[1], 0, 0, nullptr, nullptr, 0},
+                TcOperand{&mb[0], &mb[1], 0, 0, nullptr, nullptr, 0}, alpha, beta, k_lo_mode, k_hi_mode, upper_only, o,
+                chunk_stages);
   int flags = 0;
   cudaMemcpyAsync(&flags, t.status, sizeof(int), cudaMemcpyDeviceToHost, t.stream);
   cudaError_t e = cudaStreamSynchronize(t.stream);
@@ -821,6 +896,8 @@ extern "C" gptq_status gptq_quantize_layer_noalloc(const void* W, int64_t m, int
   a.U_lo = nullptr;
   a.Err = Err;
   a.Err_lo = nullptr;
+  a.ld_err = SW_B;
+  a.err_col0 = 0;
   a.codes = codes;
   a.scales = scales;
   a.zeros = zeros;

@@ -14,8 +14,9 @@
 // current values reduced across the row's lanes with shuffles.  The U block (128 x 128) is
 // staged in shared memory with asynchronous copies, in a bank-skewed layout so the eight
 // 16-column segments a warp reads at once hit different banks.
-// The block's errors go to Err [m x 128]; the columns after the block receive them through
-// one GEMM per block (S6) launched by the host.
+// The block's errors go to Err; the columns after the block receive them through tensor-core
+// products (S6) launched by the host: within a super-block of columns right after each block,
+// beyond it once per super-block.
 //
 // The integer decisions (code and zero-point) are taken in fp32 with IEEE division and
 // round-half-to-even, the precision the pages' own sketches use.
@@ -47,8 +48,9 @@ struct SweepArgs {
   float* Wq;          // [m x n] fp32 working weights, sweep order
   const float* U;     // [n x n] upper factor (fp32, or the tf32 hi part when U_lo is set)
   const float* U_lo;  // [n x n] tf32 lo part of U, or nullptr
-  float* Err;         // [m x 128] scaled errors of the current block (fp32, or hi part)
-  float* Err_lo;      // [m x 128] tf32 lo part of the errors, or nullptr
+  float* Err;         // scaled errors (fp32, or hi part): block columns at Err[r * ld_err + err_col0 ..]
+  float* Err_lo;      // tf32 lo part of the errors (same layout), or nullptr
+  int ld_err, err_col0;
   uint32_t* codes;    // [m x n*bits/32]
   float* scales;      // [m x G]
   float* zeros;       // [m x G]
@@ -246,7 +248,7 @@ __global__ void __launch_bounds__(SW_THREADS)
 
   // errors of this lane's 16 columns (hi/lo for the tensor-core update, or fp32)
   if (valid) {
-    const size_t eo = static_cast<size_t>(rr) * SW_B + SW_COLS * l8;
+    const size_t eo = static_cast<size_t>(rr) * a.ld_err + a.err_col0 + SW_COLS * l8;
     float4* ep = reinterpret_cast<float4*>(a.Err + eo);
     if (a.Err_lo) {
       float4* lp = reinterpret_cast<float4*>(a.Err_lo + eo);

@@ -57,7 +57,7 @@ _SIGS = {
     "gptq_test_gemm_tf32x3": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P, ctypes.c_int, _P, _P,
                                              ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                              ctypes.c_int, _P, ctypes.c_int, _P, _P, ctypes.c_int, _P, _P,
-                                             ctypes.c_int, ctypes.c_int, _P]),
+                                             ctypes.c_int, ctypes.c_int, ctypes.c_int, _P]),
 }
 
 

@@ -32,7 +32,7 @@ def p(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def run_gemm(A, B, alpha=1.0, beta=0, C0=None, klo=0, khi=0, upper=0, plain=True, hilo=False, trans=False):
+def run_gemm(A, B, alpha=1.0, beta=0, C0=None, klo=0, khi=0, upper=0, plain=True, hilo=False, trans=False, chunk=1):
     M, K = A.shape
     N = B.shape[0]
     ah, al = split(A)
@@ -48,7 +48,7 @@ def run_gemm(A, B, alpha=1.0, beta=0, C0=None, klo=0, khi=0, upper=0, plain=True
     Cth = torch.zeros((N, M), dtype=torch.float32, device=DEV) if trans else None
     Ctl = torch.zeros((N, M), dtype=torch.float32, device=DEV) if trans else None
     st = G.lib().gptq_test_gemm_tf32x3(M, N, K, p(Ah), p(Al), K, p(Bh), p(Bl), K, float(alpha), int(beta), klo, khi,
-                                       upper, p(C), N, p(Ch), p(Cl), N, p(Cth), p(Ctl), M, 0,
+                                       upper, p(C), N, p(Ch), p(Cl), N, p(Cth), p(Ctl), M, chunk, 0,
                                        ctypes.c_void_p(torch.cuda.current_stream(DEV).cuda_stream))
     assert st == G.OK, G.STATUS.get(st)
     out = {}
@@ -69,14 +69,15 @@ def ref(A, B, alpha, beta, C0):
     return R, scale
 
 
-@pytest.mark.parametrize("M,N,K", [(128, 256, 32), (200, 320, 96), (64, 64, 128), (384, 512, 2048)])
+@pytest.mark.parametrize("M,N,K,chunk", [(128, 256, 32, 1), (200, 320, 96, 1), (64, 64, 128, 4), (384, 512, 2048, 1),
+                                         (4096, 768, 128, 4), (300, 1024, 256, 2)])
 @pytest.mark.parametrize("beta", [0, 1])
-def test_gemm_outputs_match_fp64(M, N, K, beta):
+def test_gemm_outputs_match_fp64(M, N, K, chunk, beta):
     r = np.random.default_rng(M + N + K + beta)
     A = r.standard_normal((M, K)).astype(np.float32)
     B = r.standard_normal((N, K)).astype(np.float32)
     C0 = r.standard_normal((M, N)).astype(np.float32)
-    out = run_gemm(A, B, alpha=-0.75, beta=beta, C0=C0, plain=True, hilo=True, trans=(beta == 0))
+    out = run_gemm(A, B, alpha=-0.75, beta=beta, C0=C0, plain=True, hilo=True, trans=(beta == 0), chunk=chunk)
     R, scale = ref(A, B, -0.75, beta, C0)
     for k in out:
         got = out[k].T if k == "Ct" else out[k]

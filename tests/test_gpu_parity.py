@@ -184,3 +184,18 @@ def test_ragged_rows_and_wider_context():
     prep = O.prepare(gpu["H"], qs.damp, qs.desc_act)
     st, rep = GH.check_sweep_replay(gpu["W"], prep, gpu, qs)
     GH.assert_replay_ok(st, rep, gpu)
+
+
+@pytest.mark.parametrize("n,g,sym,bits", [(2048, 128, False, 4), (1152, -1, False, 4), (1536, 384, True, 3),
+                                          (2048, 256, False, 2), (1280, 64, True, 4)])
+def test_quantize_layer_parity_across_super_blocks(n, g, sym, bits):
+    """Layers wider than one 1024-column super-block (the far columns are updated once per
+    super-block), including a partial last super-block and a group width that forces
+    per-block far updates."""
+    layer = synth.scaled_layer(TINY, m=80, n=n, n_tok=2 * n)
+    qs = synth.QuantSetting(bits, g, sym, 0.01, True)
+    gpu = GH.run_path(layer, qs)
+    prep = O.prepare(gpu["H"], qs.damp, qs.desc_act)
+    assert np.array_equal(gpu["perm"], prep["perm"])
+    st, rep = GH.check_sweep_replay(gpu["W"], prep, gpu, qs)
+    GH.assert_replay_ok(st, rep, gpu)
