@@ -87,6 +87,8 @@ __global__ void __launch_bounds__(LF_THREADS, 1)
   float(*X)[LF_LD] = reinterpret_cast<float(*)[LF_LD]>(lf_smem + 2 * LF_NB * LF_LD);
   int* bad = reinterpret_cast<int*>(lf_smem + 3 * LF_NB * LF_LD);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  griddep_wait();
+  griddep_launch_dependents();  // one CTA: the next kernel may take the other SMs right away
   if (tid == 0) *bad = 0;
   // stage A_hi into V's storage and A_lo into X's with asynchronous 16-byte copies, at an
   // unpadded 128-float pitch (the 129-float rows of S are not 16-byte aligned)

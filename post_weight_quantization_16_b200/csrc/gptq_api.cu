@@ -149,6 +149,25 @@ gptq_status status_from_flags(int f) {
   return GPTQ_OK;
 }
 
+// Launch a kernel on the context's stream with programmatic stream serialization, so that it
+// can be scheduled while its predecessor finishes (every kernel waits on griddepcontrol.wait
+// before it reads its inputs).
+template <typename... KArgs, typename... Args>
+cudaError_t launch(gptq_ctx* c, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = c->stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  ++c->launches;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // 2-D fp32 tensor map of a row-major sub-matrix (rows x cols, leading dimension ld), boxes of
 // 32 columns x box_rows rows, 128-byte swizzle.
 gptq_status make_map(gptq_ctx* c, CUtensorMap* map, const float* base, int64_t rows, int64_t cols, int64_t ld,
@@ -221,12 +240,11 @@ gptq_status gemm_tc(gptq_ctx* c, int M, int N, int K, TcOperand A, TcOperand B, 
     g.ldt = o.ldt;
     if (static_cast<int64_t>(M) * N <= 512 * 512) {  // 32 x 32 tiles: more CTAs for the smallest products
       dim3 grid((N + 31) / 32, (M + 31) / 32);
-      gemm_hilo_simt_kernel<32, 32><<<grid, GS_THREADS, gs_smem_bytes<32, 32>(), c->stream>>>(g);
+      CK(launch(c, gemm_hilo_simt_kernel<32, 32>, grid, dim3(GS_THREADS), gs_smem_bytes<32, 32>(), g));
     } else {
       dim3 grid((N + 63) / 64, (M + 63) / 64);
-      gemm_hilo_simt_kernel<64, 64><<<grid, GS_THREADS, gs_smem_bytes<64, 64>(), c->stream>>>(g);
+      CK(launch(c, gemm_hilo_simt_kernel<64, 64>, grid, dim3(GS_THREADS), gs_smem_bytes<64, 64>(), g));
     }
-    ++c->launches;
     CKL("gemm_simt");
     return GPTQ_OK;
   }
@@ -253,9 +271,8 @@ gptq_status gemm_tc(gptq_ctx* c, int M, int N, int K, TcOperand A, TcOperand B, 
   a.Ctlo = o.Ctlo;
   a.ldt = o.ldt;
   a.status = c->status;
-  gemm_tf32x3_kernel<<<std::min(tc_tiles, c->num_sms), GT_THREADS, GT_SMEM, c->stream>>>(*A.hi, *A.lo, *B.hi,
-                                                                                         *B.lo, a);
-  ++c->launches;
+  CK(launch(c, gemm_tf32x3_kernel, dim3(std::min(tc_tiles, c->num_sms)), dim3(GT_THREADS), GT_SMEM, *A.hi, *A.lo, *B.hi,
+                                                                                         *B.lo, a));
   CKL("gemm_tc");
   return GPTQ_OK;
 }
@@ -264,9 +281,8 @@ gptq_status gemm_tc(gptq_ctx* c, int M, int N, int K, TcOperand A, TcOperand B, 
 gptq_status chol_inv(gptq_ctx* c, int o, int h) {
   const int n = static_cast<int>(c->n);
   if (h <= LF_NB) {
-    leaf_chol_inv_kernel<<<1, LF_THREADS, LF_SMEM, c->stream>>>(c->A_hi, c->A_lo, n, o, c->U_hi, c->U_lo, c->Ut_hi,
-                                                               c->Ut_lo, c->status);
-    ++c->launches;
+    CK(launch(c, leaf_chol_inv_kernel, dim3(1), dim3(LF_THREADS), LF_SMEM, c->A_hi, c->A_lo, n, o, c->U_hi, c->U_lo, c->Ut_hi,
+                                                               c->Ut_lo, c->status));
     CKL("leaf_chol_inv");
     return GPTQ_OK;
   }
@@ -560,9 +576,7 @@ gptq_status gptq_hessian_accumulate(gptq_ctx* c, const void* X, int64_t n_tok, i
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return GPTQ_ERR_CUDA;
   const int chunk_iters = static_cast<int>(c->chunk_tokens / HS_BK);
-  hessian_syrk_kernel<<<hs_num_tiles(static_cast<int>(c->n)), HS_THREADS, HS_SMEM, c->stream>>>(
-      map, c->H, static_cast<int>(c->n), static_cast<int>(n_tok), chunk_iters, c->status);
-  ++c->launches;
+  CK(launch(c, hessian_syrk_kernel, dim3(hs_num_tiles(static_cast<int>(c->n))), dim3(HS_THREADS), HS_SMEM, map, c->H, static_cast<int>(c->n), static_cast<int>(n_tok), chunk_iters, c->status));
   CKL("hessian");
   c->n_tok += n_tok;
   c->mirrored = 0;
@@ -572,8 +586,7 @@ gptq_status gptq_hessian_accumulate(gptq_ctx* c, const void* X, int64_t n_tok, i
 static gptq_status ensure_mirrored(gptq_ctx* c) {
   if (c->mirrored) return GPTQ_OK;
   const int n = static_cast<int>(c->n);
-  mirror_upper_kernel<<<dim3(n / 32, n / 32), dim3(32, 8), 0, c->stream>>>(c->H, n);
-  ++c->launches;
+  CK(launch(c, mirror_upper_kernel, dim3(n / 32, n / 32), dim3(32, 8), 0, c->H, n));
   CKL("mirror");
   c->mirrored = 1;
   return GPTQ_OK;
@@ -609,18 +622,15 @@ gptq_status gptq_prepare(gptq_ctx* c, double damp, int desc_act, int32_t* perm_o
   gptq_status s;
   c->state = ST_ACCUM;
   if ((s = ensure_mirrored(c)) != GPTQ_OK) return s;
-  diag_stats_kernel<<<1, 1024, 0, c->stream>>>(c->H, n, c->keys, c->dead, c->mean);
-  ++c->launches;
+  CK(launch(c, diag_stats_kernel, dim3(1), dim3(1024), 0, c->H, n, c->keys, c->dead, c->mean));
   CKL("diag_stats");
   if (desc_act)
-    rank_perm_kernel<<<(n + 255) / 256, 256, 0, c->stream>>>(c->keys, n, c->perm);
+    CK(launch(c, rank_perm_kernel, dim3((n + 255) / 256), dim3(256), 0, c->keys, n, c->perm));
   else
-    identity_perm_kernel<<<(n + 255) / 256, 256, 0, c->stream>>>(n, c->perm);
-  ++c->launches;
+    CK(launch(c, identity_perm_kernel, dim3((n + 255) / 256), dim3(256), 0, n, c->perm));
   CKL("perm");
-  gather_damp_kernel<<<n, 256, static_cast<size_t>(n) * 4, c->stream>>>(c->H, n, c->perm, c->keys, c->mean, damp,
-                                                                        c->A_hi, c->A_lo);
-  ++c->launches;
+  CK(launch(c, gather_damp_kernel, dim3(n), dim3(256), static_cast<size_t>(n) * 4, c->H, n, c->perm, c->keys, c->mean, damp,
+                                                                        c->A_hi, c->A_lo));
   CKL("gather");
   const size_t nn = static_cast<size_t>(n) * n;
   for (float* p : {c->U_hi, c->U_lo, c->Ut_hi, c->Ut_lo}) CK(cudaMemsetAsync(p, 0, nn * 4, c->stream));
@@ -638,8 +648,7 @@ gptq_status gptq_get_factor(gptq_ctx* c, float* U_out) {
   if (c->state != ST_PREPARED) return GPTQ_ERR_STATE;
   DeviceGuard dg(c->device);
   const size_t nn = static_cast<size_t>(c->n) * c->n;
-  combine_hilo_kernel<<<592, 256, 0, c->stream>>>(c->U_hi, c->U_lo, nn, U_out);
-  ++c->launches;
+  CK(launch(c, combine_hilo_kernel, dim3(592), dim3(256), 0, c->U_hi, c->U_lo, nn, U_out));
   CKL("combine");
   return GPTQ_OK;
 }
@@ -654,9 +663,8 @@ gptq_status gptq_quantize_layer(gptq_ctx* c, const void* W, int64_t m, gptq_qpar
   const int n = static_cast<int>(c->n);
   const int mi = static_cast<int>(m);
   const int g = (qp.group_size == -1) ? n : qp.group_size;
-  init_w_kernel<<<mi, 256, static_cast<size_t>(n) * 2, c->stream>>>(static_cast<const __half*>(W), n, c->perm, c->dead,
-                                                                   c->Wq);
-  ++c->launches;
+  CK(launch(c, init_w_kernel, dim3(mi), dim3(256), static_cast<size_t>(n) * 2, static_cast<const __half*>(W), n, c->perm, c->dead,
+                                                                   c->Wq));
   CKL("init_w");
   SweepArgs a;
   a.Wq = c->Wq;
@@ -686,12 +694,11 @@ gptq_status gptq_quantize_layer(gptq_ctx* c, const void* W, int64_t m, gptq_qpar
     for (int i1 = s0; i1 < s1; i1 += SW_B) {
       a.err_col0 = i1 - s0;
       if (g >= SW_B)
-        sweep_block_kernel<0><<<grid, SW_THREADS, SW_SMEM, c->stream>>>(a, i1);
+        CK(launch(c, sweep_block_kernel<0>, dim3(grid), dim3(SW_THREADS), SW_SMEM, a, i1));
       else if (g == 64)
-        sweep_block_kernel<64><<<grid, SW_THREADS, SW_SMEM, c->stream>>>(a, i1);
+        CK(launch(c, sweep_block_kernel<64>, dim3(grid), dim3(SW_THREADS), SW_SMEM, a, i1));
       else
-        sweep_block_kernel<32><<<grid, SW_THREADS, SW_SMEM, c->stream>>>(a, i1);
-      ++c->launches;
+        CK(launch(c, sweep_block_kernel<32>, dim3(grid), dim3(SW_THREADS), SW_SMEM, a, i1));
       CKL("sweep");
       const int i2 = i1 + SW_B;
       if (i2 < s1) {
@@ -717,8 +724,7 @@ gptq_status gptq_quantize_layer(gptq_ctx* c, const void* W, int64_t m, gptq_qpar
     }
   }
   if (g_idx) {
-    g_idx_kernel<<<(n + 255) / 256, 256, 0, c->stream>>>(c->perm, n, g, g_idx);
-    ++c->launches;
+    CK(launch(c, g_idx_kernel, dim3((n + 255) / 256), dim3(256), 0, c->perm, n, g, g_idx));
     CKL("g_idx");
   }
   return GPTQ_OK;

@@ -106,6 +106,7 @@ __global__ void __launch_bounds__(HS_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  griddep_wait();  // inputs of the previous kernel are complete and visible from here on
 
   if (warp == 0) {
     if (lane == 0) {
@@ -230,6 +231,7 @@ __global__ void __launch_bounds__(HS_THREADS, 1)
     }
   }
 
+  griddep_launch_dependents();
   __syncthreads();
   if (threadIdx.x == 0 && *abort_flag) atomicOr(status, ST_TIMEOUT);
   if (warp == 1) {

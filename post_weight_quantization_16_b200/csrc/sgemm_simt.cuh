@@ -15,6 +15,8 @@
 
 #include <cstdint>
 
+#include "sm100_ptx.cuh"
+
 namespace gptq {
 
 constexpr int SG_BM = 128, SG_BN = 128, SG_BK = 16, SG_THREADS = 256;
@@ -198,6 +200,7 @@ __device__ __forceinline__ void gs_cp_async16(void* smem_dst, const void* gmem_s
 template <int TM, int TN>
 __global__ void __launch_bounds__(GS_THREADS) gemm_hilo_simt_kernel(GemmSimtArgs p) {
   constexpr int RI = TM / 16, RJ = TN / 16;
+  griddep_wait();
   const int m0 = blockIdx.y * TM, n0 = blockIdx.x * TN;
   if (p.upper_only && m0 >= n0 + TN) return;
   int kb = 0, ke = p.K;
@@ -283,6 +286,7 @@ __global__ void __launch_bounds__(GS_THREADS) gemm_hilo_simt_kernel(GemmSimtArgs
     }
   }
   asm volatile("cp.async.wait_group 0;" ::: "memory");
+  griddep_launch_dependents();
 
 #pragma unroll
   for (int i = 0; i < RI; ++i) {

@@ -39,6 +39,17 @@ __device__ __forceinline__ bool elect_one_sync() {
 }
 
 // ----------------------------------------------------------------------------------------
+// programmatic dependent launch: a kernel launched with programmatic stream serialization
+// may start while its predecessor still runs; it must wait here before touching data the
+// predecessor writes.  launch_dependents lets the next kernel's CTAs be scheduled early.
+// Both are no-ops for kernels launched without the attribute.
+// ----------------------------------------------------------------------------------------
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ----------------------------------------------------------------------------------------
 // mbarrier
 // ----------------------------------------------------------------------------------------
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {

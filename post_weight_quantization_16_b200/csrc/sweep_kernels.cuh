@@ -98,6 +98,7 @@ __global__ void __launch_bounds__(SW_THREADS)
   int* perm_s = reinterpret_cast<int*>(rU + SW_B);              // [128]
   uint32_t* cw = reinterpret_cast<uint32_t*>(perm_s + SW_B);    // [32 rows][32 words] packed codes
 
+  griddep_wait();
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int l8 = lane & (SW_LANES - 1);      // segment of the row this lane holds
@@ -246,6 +247,7 @@ __global__ void __launch_bounds__(SW_THREADS)
     }
   }
 
+  griddep_launch_dependents();
   // errors of this lane's 16 columns (hi/lo for the tensor-core update, or fp32)
   if (valid) {
     const size_t eo = static_cast<size_t>(rr) * a.ld_err + a.err_col0 + SW_COLS * l8;
