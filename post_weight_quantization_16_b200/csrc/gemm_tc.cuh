@@ -10,9 +10,10 @@
 // accumulated in its own TMEM buffer and then added into fp32 registers with
 // round-to-nearest adds (double-buffered TMEM, as in the Hessian kernel).
 //
-// Tile 128 x 256 (tcgen05.mma kind::tf32, M=128, N=256, K=8), persistent CTAs (one per SM)
-// over the tiles, 2-stage TMA ring of 96 KB stages (A_hi, A_lo, B_hi, B_lo; 128-byte
-// swizzle), warp roles:
+// Tile 128 x BN, BN in {64, 128, 256} chosen per product so that small products still spread
+// over many SMs (tcgen05.mma kind::tf32, M=128, N=BN, K=8), persistent CTAs (one per SM) over
+// the tiles, a TMA ring of about 192 KB (2, 3 or 4 stages of A_hi, A_lo, B_hi, B_lo; 128-byte
+// swizzle; B arrives as 64-row boxes, so one tensor map serves every BN), warp roles:
 //   warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer, warps 2-9 epilogue.
 // Triangular operands: the K range of a tile can start at its first column (B lower in
 // K-major form) or its first row (A upper), or stop after its last column (B upper), so
@@ -30,12 +31,19 @@
 
 namespace gptq {
 
-constexpr int GT_BM = 128, GT_BN = 256, GT_BK = 32, GT_STAGES = 2;
+constexpr int GT_BM = 128, GT_BK = 32, GT_BOX_N = 64;
 constexpr int GT_A_BYTES = GT_BM * GT_BK * 4;  // 16 KB
-constexpr int GT_B_BYTES = GT_BN * GT_BK * 4;  // 32 KB
-constexpr int GT_STAGE_BYTES = 2 * GT_A_BYTES + 2 * GT_B_BYTES;
 constexpr int GT_THREADS = 64 + 256;
-constexpr int GT_SMEM = GT_STAGES * GT_STAGE_BYTES + 256 + 1024;
+
+template <int BN>
+struct GtCfg {
+  static_assert(BN == 64 || BN == 128 || BN == 256, "tile width");
+  static constexpr int B_BYTES = BN * GT_BK * 4;
+  static constexpr int STAGE_BYTES = 2 * GT_A_BYTES + 2 * B_BYTES;  // 48, 64 or 96 KB
+  static constexpr int STAGES = BN == 256 ? 2 : (BN == 128 ? 3 : 4);
+  static constexpr int SMEM = STAGES * STAGE_BYTES + 256 + 1024;
+  static constexpr int TMEM_COLS = 2 * BN;  // two accumulators
+};
 
 enum : int { GT_KLO_NONE = 0, GT_KLO_COL = 1, GT_KLO_ROW = 2 };
 enum : int { GT_KHI_NONE = 0, GT_KHI_COL = 1 };
@@ -66,35 +74,36 @@ __device__ __forceinline__ float tf32_rn(float x) {
 }
 
 // Number of output tiles the kernel visits: all of them, or with upper_only only the tiles
-// that reach the upper triangle (tile (mt, nt) is needed iff mt < 2 nt + 2).
-__host__ __device__ inline int gt_num_tiles(int M, int N, int upper_only) {
-  const int mtn = (M + GT_BM - 1) / GT_BM, ntn = (N + GT_BN - 1) / GT_BN;
+// that reach the upper triangle (tile (mt, nt) is needed iff mt * BM < (nt + 1) * BN).
+__host__ __device__ inline int gt_num_tiles(int M, int N, int upper_only, int bn) {
+  const int mtn = (M + GT_BM - 1) / GT_BM, ntn = (N + bn - 1) / bn;
   if (!upper_only) return mtn * ntn;
   int c = 0;
-  for (int nt = 0; nt < ntn; ++nt) c += min(mtn, 2 * nt + 2);
+  for (int nt = 0; nt < ntn; ++nt) c += min(mtn, ((nt + 1) * bn + GT_BM - 1) / GT_BM);
   return c;
 }
 
 // Tile t (n-tiles fastest, or with upper_only column by column over the needed tiles).
+template <int BN>
 __device__ __forceinline__ void gt_tile(const GemmTCArgs& p, int t, int& m0, int& n0, int& k_begin, int& n_iters) {
-  const int mtn = (p.M + GT_BM - 1) / GT_BM, ntn = (p.N + GT_BN - 1) / GT_BN;
+  const int mtn = (p.M + GT_BM - 1) / GT_BM, ntn = (p.N + BN - 1) / BN;
   if (!p.upper_only) {
     m0 = (t / ntn) * GT_BM;
-    n0 = (t % ntn) * GT_BN;
+    n0 = (t % ntn) * BN;
   } else {
     int nt = 0;
     for (;; ++nt) {
-      const int cnt = min(mtn, 2 * nt + 2);
+      const int cnt = min(mtn, ((nt + 1) * BN + GT_BM - 1) / GT_BM);
       if (t < cnt || nt == ntn - 1) break;
       t -= cnt;
     }
     m0 = t * GT_BM;
-    n0 = nt * GT_BN;
+    n0 = nt * BN;
   }
   int kb = 0, ke = p.K;
   if (p.k_lo_mode == GT_KLO_COL) kb = n0;
   if (p.k_lo_mode == GT_KLO_ROW) kb = m0;
-  if (p.k_hi_mode == GT_KHI_COL) ke = min(p.K, n0 + GT_BN);
+  if (p.k_hi_mode == GT_KHI_COL) ke = min(p.K, n0 + BN);
   kb = (kb / GT_BK) * GT_BK;
   k_begin = kb;
   n_iters = (ke > kb) ? (ke - kb + GT_BK - 1) / GT_BK : 0;
@@ -104,6 +113,7 @@ __device__ __forceinline__ void gt_tile(const GemmTCArgs& p, int t, int& m0, int
 // ahead across tile boundaries; each K stage lands in one of two TMEM accumulators, which
 // the epilogue warps drain into registers that were pre-loaded with C (beta = 1) while the
 // tile's first stages were in flight, so a tile ends with stores only.
+template <int BN>
 __global__ void __launch_bounds__(GT_THREADS, 1)
     gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_constant__ CUtensorMap a_lo,
                        const __grid_constant__ CUtensorMap b_hi, const __grid_constant__ CUtensorMap b_lo,
@@ -115,18 +125,20 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int ntiles = gt_num_tiles(p.M, p.N, p.upper_only);
+  using Cfg = GtCfg<BN>;
+  constexpr int STAGES = Cfg::STAGES, STAGE_BYTES = Cfg::STAGE_BYTES, B_BYTES = Cfg::B_BYTES;
+  const int ntiles = gt_num_tiles(p.M, p.N, p.upper_only, BN);
 
-  const uint32_t bar_full = sbase + GT_STAGES * GT_STAGE_BYTES;
-  const uint32_t bar_empty = bar_full + 8 * GT_STAGES;
-  const uint32_t bar_tfull = bar_empty + 8 * GT_STAGES;
+  const uint32_t bar_full = sbase + STAGES * STAGE_BYTES;
+  const uint32_t bar_empty = bar_full + 8 * STAGES;
+  const uint32_t bar_tfull = bar_empty + 8 * STAGES;
   const uint32_t bar_tempty = bar_tfull + 16;
   const uint32_t bar_drain = bar_tempty + 16;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + GT_STAGES * GT_STAGE_BYTES + 8 * (2 * GT_STAGES + 5));
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + STAGES * STAGE_BYTES + 8 * (2 * STAGES + 5));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < GT_STAGES; ++s) {
+    for (int s = 0; s < STAGES; ++s) {
       mbar_init(bar_full + 8 * s, 1);
       mbar_init(bar_empty + 8 * s, 1);
     }
@@ -139,7 +151,7 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_alloc(smem_u32(tmem_slot), Cfg::TMEM_COLS);
     tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
@@ -161,37 +173,41 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
         int m0, n0, kb, ni;
-        gt_tile(p, t, m0, n0, kb, ni);
+        gt_tile<BN>(p, t, m0, n0, kb, ni);
         for (int j = 0; j < ni; ++j, ++it) {
-          const int s = it % GT_STAGES;
-          const uint32_t ph = static_cast<uint32_t>(it / GT_STAGES) & 1u;
+          const int s = it % STAGES;
+          const uint32_t ph = static_cast<uint32_t>(it / STAGES) & 1u;
           if (!mbar_wait_bounded(bar_empty + 8 * s, ph ^ 1u, abort_flag)) {
             ok = false;
             break;
           }
           const uint32_t fb = bar_full + 8 * s;
-          mbar_arrive_expect_tx(fb, GT_STAGE_BYTES);
-          const uint32_t st = sbase + s * GT_STAGE_BYTES;
+          mbar_arrive_expect_tx(fb, STAGE_BYTES);
+          const uint32_t st = sbase + s * STAGE_BYTES;
           const int k = kb + j * GT_BK;
           tma_load_2d(st, &a_hi, fb, p.a_col0 + k, p.a_row0 + m0);
           tma_load_2d(st + GT_A_BYTES, &a_lo, fb, p.a_col0 + k, p.a_row0 + m0);
-          tma_load_2d(st + 2 * GT_A_BYTES, &b_hi, fb, p.b_col0 + k, p.b_row0 + n0);
-          tma_load_2d(st + 2 * GT_A_BYTES + GT_B_BYTES, &b_lo, fb, p.b_col0 + k, p.b_row0 + n0);
+#pragma unroll
+          for (int bx = 0; bx < BN / GT_BOX_N; ++bx) {  // 64-row boxes, stacked at 8 KB
+            const uint32_t o8 = bx * (GT_BOX_N * GT_BK * 4);
+            tma_load_2d(st + 2 * GT_A_BYTES + o8, &b_hi, fb, p.b_col0 + k, p.b_row0 + n0 + bx * GT_BOX_N);
+            tma_load_2d(st + 2 * GT_A_BYTES + B_BYTES + o8, &b_lo, fb, p.b_col0 + k, p.b_row0 + n0 + bx * GT_BOX_N);
+          }
         }
       }
-      for (int i = max(0, it - GT_STAGES); i < it; ++i)
-        mbar_wait_drain(bar_full + 8 * (i % GT_STAGES), static_cast<uint32_t>(i / GT_STAGES) & 1u);
+      for (int i = max(0, it - STAGES); i < it; ++i)
+        mbar_wait_drain(bar_full + 8 * (i % STAGES), static_cast<uint32_t>(i / STAGES) & 1u);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer: one TMEM buffer per chunk of K stages ----------------
-      constexpr uint32_t idesc = idesc_make(2u, 2u, 0u, 0u, GT_BM, GT_BN);  // tf32, K-major A and B
+      constexpr uint32_t idesc = idesc_make(2u, 2u, 0u, 0u, GT_BM, BN);  // tf32, K-major A and B
       const int cs = p.chunk_stages;
       bool ok = true;
       int it = 0, ch = 0;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
         int m0, n0, kb, ni;
-        gt_tile(p, t, m0, n0, kb, ni);
+        gt_tile<BN>(p, t, m0, n0, kb, ni);
         int b = 0;
         for (int j = 0; j < ni; ++j, ++it) {
           const bool first = (j % cs) == 0;
@@ -203,17 +219,17 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
               break;
             }
           }
-          const int s = it % GT_STAGES;
-          const uint32_t phs = static_cast<uint32_t>(it / GT_STAGES) & 1u;
+          const int s = it % STAGES;
+          const uint32_t phs = static_cast<uint32_t>(it / STAGES) & 1u;
           if (!mbar_wait_bounded(bar_full + 8 * s, phs, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * GT_BN);
-          const uint32_t st = sbase + s * GT_STAGE_BYTES;
+          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * BN);
+          const uint32_t st = sbase + s * STAGE_BYTES;
           const uint32_t sa_hi = st, sa_lo = st + GT_A_BYTES;
-          const uint32_t sb_hi = st + 2 * GT_A_BYTES, sb_lo = sb_hi + GT_B_BYTES;
+          const uint32_t sb_hi = st + 2 * GT_A_BYTES, sb_lo = sb_hi + B_BYTES;
 #pragma unroll
           for (int kk = 0; kk < GT_BK / 8; ++kk) {
             const uint32_t off = kk * 32;  // 8 fp32 of K inside the 128-byte swizzle row
@@ -243,14 +259,15 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
     bool all_ok = true;
     for (int t = blockIdx.x; t < ntiles && all_ok; t += gridDim.x) {
       int m0, n0, kb, ni;
-      gt_tile(p, t, m0, n0, kb, ni);
+      gt_tile<BN>(p, t, m0, n0, kb, ni);
       const int r = m0 + q * 32 + lane;
-      const int cbase = n0 + hh * (GT_BN / 2);
+      constexpr int HALF = BN / 2;  // columns per epilogue warp
+      const int cbase = n0 + hh * HALF;
       const bool row_ok = r < p.M;
-      float acc[GT_BN / 2];
+      float acc[HALF];
       // pre-load C (beta = 1) into the accumulators while the first stages run
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 0; cc < HALF / 32; ++cc) {
         const int c0 = cbase + cc * 32;
         const bool ld = p.beta && row_ok && c0 < p.N;
         if (ld && p.C) {
@@ -292,10 +309,10 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
         }
         tc_fence_after();
 #pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
+        for (int cc = 0; cc < HALF / 16; ++cc) {
           uint32_t v[16];
           tmem_ld_32x32b_x16(tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                                 static_cast<uint32_t>(b * GT_BN + hh * (GT_BN / 2) + cc * 16),
+                                 static_cast<uint32_t>(b * BN + hh * HALF + cc * 16),
                              v);
           tmem_ld_wait();
 #pragma unroll
@@ -306,7 +323,7 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
       }
       if (!all_ok) break;
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 0; cc < HALF / 32; ++cc) {
         const int c0 = cbase + cc * 32;
         if (!row_ok || c0 >= p.N) continue;  // N % 32 == 0: whole 32-column groups
         if (p.C) {
@@ -351,7 +368,7 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
   if (threadIdx.x == 0 && *abort_flag) atomicOr(p.status, ST_TIMEOUT);
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, 512);
+    tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
   }
 }
 

@@ -206,15 +206,43 @@ struct TcOperand {
   int ld;
 };
 
-// Products with fewer tensor-core tiles than this run on the CUDA cores (fp32, 64 x 64 tiles).
+// Products with fewer tensor-core tiles (at the narrowest tile) than this run on the CUDA
+// cores (fp32, 32 x 32 or 64 x 64 tiles).
 constexpr int kMinTcTiles = 32;
 
+cudaError_t set_gemm_tc_attributes() {
+  cudaError_t e = cudaFuncSetAttribute(gemm_tf32x3_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       GtCfg<256>::SMEM);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(gemm_tf32x3_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, GtCfg<128>::SMEM);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(gemm_tf32x3_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, GtCfg<64>::SMEM);
+  return e;
+}
+
+// Tile width of a tensor-core product: the one with the least modelled time, waves of
+// persistent CTAs times a tile's cost (its width plus a fixed 64-column-equivalent overhead).
+int pick_bn(int M, int N, int upper, int sms) {
+  int best = 256;
+  int64_t best_cost = -1;
+  for (int bn : {256, 128, 64}) {
+    const int64_t waves = (gt_num_tiles(M, N, upper, bn) + sms - 1) / sms;
+    const int64_t cost = waves * (bn + 64);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = bn;
+    }
+  }
+  return best;
+}
+
 gptq_status gemm_tc(gptq_ctx* c, int M, int N, int K, TcOperand A, TcOperand B, float alpha, int beta, int klo,
-                    int khi, int upper, const TcOut& o, int chunk_stages = 1) {
+                    int khi, int upper, const TcOut& o, int chunk_stages = 1, int force_bn = 0) {
   if (M <= 0 || N <= 0) return GPTQ_OK;
   if (N % 32 || K % GT_BK) return GPTQ_ERR_ARG;
-  const int tc_tiles = gt_num_tiles(M, N, upper);
-  if (tc_tiles < kMinTcTiles && A.phi && B.phi) {
+  const int bn = force_bn ? force_bn : pick_bn(M, N, upper, c->num_sms);
+  const int tc_tiles = gt_num_tiles(M, N, upper, bn);
+  if (gt_num_tiles(M, N, upper, 64) < kMinTcTiles && A.phi && B.phi) {
     GemmSimtArgs g;
     g.M = M;
     g.N = N;
@@ -271,8 +299,13 @@ gptq_status gemm_tc(gptq_ctx* c, int M, int N, int K, TcOperand A, TcOperand B, 
   a.Ctlo = o.Ctlo;
   a.ldt = o.ldt;
   a.status = c->status;
-  CK(launch(c, gemm_tf32x3_kernel, dim3(std::min(tc_tiles, c->num_sms)), dim3(GT_THREADS), GT_SMEM, *A.hi, *A.lo, *B.hi,
-                                                                                         *B.lo, a));
+  const dim3 grid(std::min(tc_tiles, c->num_sms));
+  if (bn == 256)
+    CK(launch(c, gemm_tf32x3_kernel<256>, grid, dim3(GT_THREADS), GtCfg<256>::SMEM, *A.hi, *A.lo, *B.hi, *B.lo, a));
+  else if (bn == 128)
+    CK(launch(c, gemm_tf32x3_kernel<128>, grid, dim3(GT_THREADS), GtCfg<128>::SMEM, *A.hi, *A.lo, *B.hi, *B.lo, a));
+  else
+    CK(launch(c, gemm_tf32x3_kernel<64>, grid, dim3(GT_THREADS), GtCfg<64>::SMEM, *A.hi, *A.lo, *B.hi, *B.lo, a));
   CKL("gemm_tc");
   return GPTQ_OK;
 }
@@ -350,9 +383,9 @@ gptq_status encode_maps(gptq_ctx* c) {
       {&c->mA_U[0], c->U_hi, n, n, n, GT_BM},        {&c->mA_U[1], c->U_lo, n, n, n, GT_BM},
       {&c->mA_Err[0], c->Err_hi, c->m_max, kSuperBlock, kSuperBlock, GT_BM},
       {&c->mA_Err[1], c->Err_lo, c->m_max, kSuperBlock, kSuperBlock, GT_BM},
-      {&c->mB_U[0], c->U_hi, n, n, n, GT_BN},        {&c->mB_U[1], c->U_lo, n, n, n, GT_BN},
-      {&c->mB_VT[0], c->VT_hi, n, n, n, GT_BN},      {&c->mB_VT[1], c->VT_lo, n, n, n, GT_BN},
-      {&c->mB_Ut[0], c->Ut_hi, n, n, n, GT_BN},      {&c->mB_Ut[1], c->Ut_lo, n, n, n, GT_BN},
+      {&c->mB_U[0], c->U_hi, n, n, n, GT_BOX_N},        {&c->mB_U[1], c->U_lo, n, n, n, GT_BOX_N},
+      {&c->mB_VT[0], c->VT_hi, n, n, n, GT_BOX_N},      {&c->mB_VT[1], c->VT_lo, n, n, n, GT_BOX_N},
+      {&c->mB_Ut[0], c->Ut_hi, n, n, n, GT_BOX_N},      {&c->mB_Ut[1], c->Ut_lo, n, n, n, GT_BOX_N},
   };
   for (auto& e : list)
     if ((s = make_map(c, e.m, e.p, e.rows, e.cols, e.ld, e.box)) != GPTQ_OK) return s;
@@ -519,8 +552,7 @@ gptq_status gptq_create(gptq_ctx** out, int64_t n, int64_t m_max, int device, vo
     return GPTQ_ERR_CUDA;
   }
   e = cudaFuncSetAttribute(hessian_syrk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, HS_SMEM);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(gemm_tf32x3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GT_SMEM);
+  if (e == cudaSuccess) e = set_gemm_tc_attributes();
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(leaf_chol_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, LF_SMEM);
   if (e == cudaSuccess)
@@ -754,8 +786,9 @@ int64_t gptq_launch_count(const gptq_ctx* c) { return c ? c->launches : -1; }
 gptq_status gptq_test_gemm_tf32x3(int M, int N, int K, const float* A_hi, const float* A_lo, int lda, const float* B_hi,
                                   const float* B_lo, int ldb, float alpha, int beta, int k_lo_mode, int k_hi_mode,
                                   int upper_only, float* C, int ldc, float* C_hi, float* C_lo, int ldh, float* Ct_hi,
-                                  float* Ct_lo, int ldt, int chunk_stages, int device, void* cuda_stream) {
+                                  float* Ct_lo, int ldt, int chunk_stages, int tile_n, int device, void* cuda_stream) {
   if (chunk_stages < 1) return GPTQ_ERR_ARG;
+  if (tile_n != 0 && tile_n != 64 && tile_n != 128 && tile_n != 256) return GPTQ_ERR_ARG;
   if (!A_hi || !A_lo || !B_hi || !B_lo || M < 1 || N < 1 || K < GT_BK) return GPTQ_ERR_ARG;
   if (k_lo_mode < 0 || k_lo_mode > 2 || k_hi_mode < 0 || k_hi_mode > 1 || (beta != 0 && beta != 1)) return GPTQ_ERR_ARG;
   if ((C_hi == nullptr) != (C_lo == nullptr) || (Ct_hi == nullptr) != (Ct_lo == nullptr)) return GPTQ_ERR_ARG;
@@ -773,7 +806,7 @@ gptq_status gptq_test_gemm_tf32x3(int M, int N, int K, const float* A_hi, const 
   t.encode = get_encode();
   if (!t.encode) return GPTQ_ERR_CUDA;
   cudaDeviceGetAttribute(&t.num_sms, cudaDevAttrMultiProcessorCount, device);
-  CK(cudaFuncSetAttribute(gemm_tf32x3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GT_SMEM));
+  CK(set_gemm_tc_attributes());
   CK(cudaMallocAsync(reinterpret_cast<void**>(&t.status), sizeof(int), t.stream));
   CK(cudaMemsetAsync(t.status, 0, sizeof(int), t.stream));
   TcOut o;
@@ -789,12 +822,12 @@ gptq_status gptq_test_gemm_tf32x3(int M, int N, int K, const float* A_hi, const 
   gptq_status s = GPTQ_OK;
   if (s == GPTQ_OK) s = make_map(&t, &ma[0], A_hi, M, K, lda, GT_BM);
   if (s == GPTQ_OK) s = make_map(&t, &ma[1], A_lo, M, K, lda, GT_BM);
-  if (s == GPTQ_OK) s = make_map(&t, &mb[0], B_hi, N, K, ldb, GT_BN);
-  if (s == GPTQ_OK) s = make_map(&t, &mb[1], B_lo, N, K, ldb, GT_BN);
+  if (s == GPTQ_OK) s = make_map(&t, &mb[0], B_hi, N, K, ldb, GT_BOX_N);
+  if (s == GPTQ_OK) s = make_map(&t, &mb[1], B_lo, N, K, ldb, GT_BOX_N);
   if (s == GPTQ_OK)
     s = gemm_tc(&t, M, N, K, TcOperand{&ma[0], &ma[1], 0, 0, nullptr, nullptr, 0},
                 TcOperand{&mb[0], &mb[1], 0, 0, nullptr, nullptr, 0}, alpha, beta, k_lo_mode, k_hi_mode, upper_only, o,
-                chunk_stages);
+                chunk_stages, tile_n);
   int flags = 0;
   cudaMemcpyAsync(&flags, t.status, sizeof(int), cudaMemcpyDeviceToHost, t.stream);
   cudaError_t e = cudaStreamSynchronize(t.stream);
@@ -803,6 +836,36 @@ gptq_status gptq_test_gemm_tf32x3(int M, int N, int K, const float* A_hi, const 
   if (s != GPTQ_OK) return s;
   if (e != cudaSuccess) return cuda_fail(e, "test gemm");
   return status_from_flags(flags);
+}
+
+gptq_status gptq_test_div_rn(uint64_t seed, int64_t count, uint64_t* mismatches, float* example, int device,
+                             void* cuda_stream) {
+  if (count < 0 || !mismatches) return GPTQ_ERR_ARG;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) {
+    cudaGetLastError();
+    return GPTQ_ERR_CUDA;
+  }
+  DeviceGuard dg(device);
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  int sms = 0;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device);
+  unsigned long long* d_count = nullptr;
+  CK(cudaMallocAsync(reinterpret_cast<void**>(&d_count), 16, st));
+  float* d_ex = reinterpret_cast<float*>(d_count + 1);
+  cudaMemsetAsync(d_count, 0, 16, st);
+  div_rn_check_kernel<<<sms * 8, 256, 0, st>>>(seed, static_cast<long long>(count), d_count, d_ex);
+  cudaError_t e = cudaGetLastError();
+  unsigned long long h[2] = {0ull, 0ull};
+  cudaMemcpyAsync(h, d_count, 16, cudaMemcpyDeviceToHost, st);
+  cudaError_t e2 = cudaStreamSynchronize(st);
+  cudaFreeAsync(d_count, st);
+  cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "test div_rn");
+  if (e2 != cudaSuccess) return cuda_fail(e2, "test div_rn");
+  *mismatches = h[0];
+  if (example) std::memcpy(example, &h[1], 2 * sizeof(float));
+  return GPTQ_OK;
 }
 
 gptq_status gptq_destroy(gptq_ctx* c) {

@@ -7,10 +7,10 @@
 // Rows of W are independent once U is known.  Eight lanes of a warp share one row: lane
 // l (0..7 within its group) holds the row's block columns 16l .. 16l+15 in registers, so a
 // warp sweeps four rows and a 256-thread CTA 32 rows.  For column i the owning lane
-// (i / 16) computes the code, the dequantized value and e = (w - q) / U[i][i]; e is broadcast
-// to the row's lanes with a warp shuffle and every lane updates its 16 columns,
-// w[j] -= e * U[i][j].  U is upper-triangular, so the update leaves columns left of i
-// untouched without any masking.  Group scales/zeros come from a min/max over the group's
+// (i / 16) computes the code, the dequantized value and e = (w - q) / U[i][i] and updates
+// its own later columns, w[j] -= e * U[i][j], so the per-column dependent chain never
+// leaves the lane's registers.  After each 16-column chunk its errors reach the row's later
+// lanes in one batch (16 shuffles, then 16 x 16 fused multiply-adds per lane).  Group scales/zeros come from a min/max over the group's
 // current values reduced across the row's lanes with shuffles.  The U block (128 x 128) is
 // staged in shared memory with asynchronous copies, in a bank-skewed layout so the eight
 // 16-column segments a warp reads at once hit different banks.
@@ -18,8 +18,8 @@
 // products (S6) launched by the host: within a super-block of columns right after each block,
 // beyond it once per super-block.
 //
-// The integer decisions (code and zero-point) are taken in fp32 with IEEE division and
-// round-half-to-even, the precision the pages' own sketches use.
+// The integer decisions (code and zero-point) are taken in fp32 with correctly rounded
+// division and round-half-to-even, the precision the pages' own sketches use.
 #pragma once
 
 #include <cstdint>
@@ -85,6 +85,58 @@ __device__ __forceinline__ void group_reduce(float& wmin, float& wmax, float& am
     wmin = fminf(wmin, __shfl_xor_sync(0xffffffffu, wmin, o));
     wmax = fmaxf(wmax, __shfl_xor_sync(0xffffffffu, wmax, o));
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  }
+}
+
+// x / s rounded to nearest-even, from r = 1/s rounded to nearest: q0 = x r, then one
+// correction with the remainder x - q0 s taken by a fused multiply-add (Markstein's
+// correction step, "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Dev. 34(1), 1990).  Three dependent operations instead of a
+// full division on the sweep's per-column chain; the tests compare it bit for bit with
+// IEEE division over the quantizer's range.
+__device__ __forceinline__ float div_rn(float x, float s, float r) {
+  const float q0 = __fmul_rn(x, r);
+  const float rem = __fmaf_rn(-q0, s, x);
+  return __fmaf_rn(rem, r, q0);
+}
+
+// Test support: compare div_rn with IEEE division on count (x, s) pairs drawn from a
+// counter-based hash (splitmix64 of seed + index).  Even indices take random bit patterns
+// (|x| in [2^-60, 2^21), s in [2^-27, 2^11)); odd ones put x / s within a few ulps of a
+// half-integer k + 1/2, |k| <= 300, where a code's rounding is decided.
+__device__ __forceinline__ uint64_t splitmix64(uint64_t z) {
+  z += 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+__global__ void div_rn_check_kernel(uint64_t seed, long long count, unsigned long long* mismatches, float* example) {
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < count; i += stride) {
+    const uint64_t h1 = splitmix64(seed ^ (static_cast<uint64_t>(i) * 2u));
+    const uint64_t h2 = splitmix64(seed ^ (static_cast<uint64_t>(i) * 2u + 1u));
+    const uint32_t se = 100u + static_cast<uint32_t>(h2 % 38u);  // biased exponent of s: 2^-27 .. 2^10
+    const float s = __uint_as_float((se << 23) | static_cast<uint32_t>(h2 >> 41));
+    float x;
+    if ((i & 1) == 0) {
+      const uint32_t xe = 67u + static_cast<uint32_t>(h1 % 81u);  // 2^-60 .. 2^20
+      x = __uint_as_float(((static_cast<uint32_t>(h1 >> 63)) << 31) | (xe << 23) | static_cast<uint32_t>((h1 >> 8) & 0x7FFFFFu));
+    } else {
+      const int k = static_cast<int>(h1 % 601u) - 300;
+      const int d = static_cast<int>((h1 >> 20) % 9u) - 4;  // -4 .. 4 ulps
+      x = __fmul_rn(static_cast<float>(k) + 0.5f, s);
+      x = __int_as_float(__float_as_int(x) + d);
+    }
+    const float r = __frcp_rn(s);
+    const float a = div_rn(x, s, r);
+    const float b = __fdiv_rn(x, s);
+    if (__float_as_uint(a) != __float_as_uint(b)) {
+      if (atomicAdd(mismatches, 1ull) == 0ull) {
+        example[0] = x;
+        example[1] = s;
+      }
+    }
   }
 }
 
@@ -194,7 +246,9 @@ __global__ void __launch_bounds__(SW_THREADS)
     myerr[t] = 0.0f;
     mywhat[t] = 0.0f;
   }
-  const float* urow_base = Us + l8 * SW_SEG;
+  // inside the rounding the zero-point enters only for asymmetric codes
+  float zs = a.sym ? 0.0f : z;
+  float rs = __frcp_rn(s);
 
 #pragma unroll 1
   for (int c = 0; c < SW_LANES; ++c) {  // chunk c = columns 16c .. 16c+15, owned by lane c of each row
@@ -212,6 +266,8 @@ __global__ void __launch_bounds__(SW_THREADS)
       }
       group_reduce(wmin, wmax, amax);
       group_scale_zero(wmin, wmax, amax, qp, a.sym, s, z);
+      zs = a.sym ? 0.0f : z;
+      rs = __frcp_rn(s);
       if (valid && l8 == 0) {
         const int gi = (i1 + c * SW_COLS) / a.g;
         a.scales[static_cast<size_t>(rr) * a.G + gi] = s;
@@ -219,30 +275,51 @@ __global__ void __launch_bounds__(SW_THREADS)
       }
     }
     const bool owner = (l8 == c);
+    const float* useg = Us + (c * SW_COLS) * SW_ULD + l8 * SW_SEG;  // U rows of the chunk, this lane's columns
+    // The owner walks its 16 columns with nothing but its own registers on the dependent
+    // chain; the other lanes run the same instructions with a zero error (no effect).
+    float ec[SW_COLS];
 #pragma unroll
     for (int t = 0; t < SW_COLS; ++t) {
-      const int i = c * SW_COLS + t;
-      // every lane quantizes its column t; the owner's result is the one that counts
       const float x = w[t];
-      float v = __fdiv_rn(x, s);
-      if (!a.sym) v = __fadd_rn(v, z);
+      const float v = __fadd_rn(div_rn(x, s, rs), zs);
       const float q = fminf(fmaxf(rintf(v), qp.lo), qp.hi);
-      const float what = a.sym ? __fmul_rn(q, s) : __fmul_rn(__fsub_rn(q, z), s);
-      const float e_own = __fmul_rn(__fsub_rn(x, what), rU[i]);
+      const float qz = __fsub_rn(q, zs);
+      const float e = __fmul_rn(__fmaf_rn(-qz, s, x), rU[c * SW_COLS + t]);
+      ec[t] = e;
       if (owner) {
         mycode[t] = static_cast<uint32_t>(static_cast<int>(q - qp.lo));
-        myerr[t] = e_own;
-        mywhat[t] = what;
+        myerr[t] = e;
+        mywhat[t] = __fmul_rn(qz, s);
       }
-      const float e = __shfl_sync(0xffffffffu, e_own, gbase + c);
-      const float4* urow = reinterpret_cast<const float4*>(urow_base + i * SW_ULD);
+      const float eo = owner ? e : 0.0f;
+      const float4* urow = reinterpret_cast<const float4*>(useg + t * SW_ULD);
 #pragma unroll
-      for (int j4 = 0; j4 < SW_COLS / 4; ++j4) {
+      for (int j4 = (t + 1) / 4; j4 < SW_COLS / 4; ++j4) {
         const float4 u = urow[j4];
-        w[4 * j4 + 0] = fmaf(-e, u.x, w[4 * j4 + 0]);
-        w[4 * j4 + 1] = fmaf(-e, u.y, w[4 * j4 + 1]);
-        w[4 * j4 + 2] = fmaf(-e, u.z, w[4 * j4 + 2]);
-        w[4 * j4 + 3] = fmaf(-e, u.w, w[4 * j4 + 3]);
+        if (4 * j4 + 0 > t) w[4 * j4 + 0] = fmaf(-eo, u.x, w[4 * j4 + 0]);
+        if (4 * j4 + 1 > t) w[4 * j4 + 1] = fmaf(-eo, u.y, w[4 * j4 + 1]);
+        if (4 * j4 + 2 > t) w[4 * j4 + 2] = fmaf(-eo, u.z, w[4 * j4 + 2]);
+        w[4 * j4 + 3] = fmaf(-eo, u.w, w[4 * j4 + 3]);
+      }
+    }
+    // the chunk's 16 errors reach the row's later lanes in one batch:
+    // w[j] -= sum_t e_t U[16c + t][j] for the columns j of lanes l8 > c
+    if (c + 1 < SW_LANES) {
+      const bool later = l8 > c;
+#pragma unroll
+      for (int t = 0; t < SW_COLS; ++t) {
+        const float eb = __shfl_sync(0xffffffffu, ec[t], gbase + c);
+        const float e = later ? eb : 0.0f;
+        const float4* urow = reinterpret_cast<const float4*>(useg + t * SW_ULD);
+#pragma unroll
+        for (int j4 = 0; j4 < SW_COLS / 4; ++j4) {
+          const float4 u = urow[j4];
+          w[4 * j4 + 0] = fmaf(-e, u.x, w[4 * j4 + 0]);
+          w[4 * j4 + 1] = fmaf(-e, u.y, w[4 * j4 + 1]);
+          w[4 * j4 + 2] = fmaf(-e, u.z, w[4 * j4 + 2]);
+          w[4 * j4 + 3] = fmaf(-e, u.w, w[4 * j4 + 3]);
+        }
       }
     }
   }

@@ -32,7 +32,8 @@ def p(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def run_gemm(A, B, alpha=1.0, beta=0, C0=None, klo=0, khi=0, upper=0, plain=True, hilo=False, trans=False, chunk=1):
+def run_gemm(A, B, alpha=1.0, beta=0, C0=None, klo=0, khi=0, upper=0, plain=True, hilo=False, trans=False, chunk=1,
+             tile=0):
     M, K = A.shape
     N = B.shape[0]
     ah, al = split(A)
@@ -48,7 +49,7 @@ def run_gemm(A, B, alpha=1.0, beta=0, C0=None, klo=0, khi=0, upper=0, plain=True
     Cth = torch.zeros((N, M), dtype=torch.float32, device=DEV) if trans else None
     Ctl = torch.zeros((N, M), dtype=torch.float32, device=DEV) if trans else None
     st = G.lib().gptq_test_gemm_tf32x3(M, N, K, p(Ah), p(Al), K, p(Bh), p(Bl), K, float(alpha), int(beta), klo, khi,
-                                       upper, p(C), N, p(Ch), p(Cl), N, p(Cth), p(Ctl), M, chunk, 0,
+                                       upper, p(C), N, p(Ch), p(Cl), N, p(Cth), p(Ctl), M, chunk, tile, 0,
                                        ctypes.c_void_p(torch.cuda.current_stream(DEV).cuda_stream))
     assert st == G.OK, G.STATUS.get(st)
     out = {}
@@ -72,12 +73,14 @@ def ref(A, B, alpha, beta, C0):
 @pytest.mark.parametrize("M,N,K,chunk", [(128, 256, 32, 1), (200, 320, 96, 1), (64, 64, 128, 4), (384, 512, 2048, 1),
                                          (4096, 768, 128, 4), (300, 1024, 256, 2)])
 @pytest.mark.parametrize("beta", [0, 1])
-def test_gemm_outputs_match_fp64(M, N, K, chunk, beta):
+@pytest.mark.parametrize("tile", [0, 64, 128, 256])
+def test_gemm_outputs_match_fp64(M, N, K, chunk, beta, tile):
     r = np.random.default_rng(M + N + K + beta)
     A = r.standard_normal((M, K)).astype(np.float32)
     B = r.standard_normal((N, K)).astype(np.float32)
     C0 = r.standard_normal((M, N)).astype(np.float32)
-    out = run_gemm(A, B, alpha=-0.75, beta=beta, C0=C0, plain=True, hilo=True, trans=(beta == 0), chunk=chunk)
+    out = run_gemm(A, B, alpha=-0.75, beta=beta, C0=C0, plain=True, hilo=True, trans=(beta == 0), chunk=chunk,
+                   tile=tile)
     R, scale = ref(A, B, -0.75, beta, C0)
     for k in out:
         got = out[k].T if k == "Ct" else out[k]
@@ -85,35 +88,47 @@ def test_gemm_outputs_match_fp64(M, N, K, chunk, beta):
         assert err.max() <= 2e-6, (k, err.max())
 
 
-def test_gemm_triangular_k_ranges():
+@pytest.mark.parametrize("tile", [64, 128, 256])
+def test_gemm_triangular_k_ranges(tile):
     r = np.random.default_rng(7)
     n = 512
     # B lower in K-major form (B[c][k] = 0 for k < c): K from the tile's first column
     A = r.standard_normal((256, n)).astype(np.float32)
     B = np.triu(r.standard_normal((n, n)).astype(np.float32))
     R, scale = ref(A, B, 1.0, 0, None)
-    got = run_gemm(A, B, klo=1)["C"]
+    got = run_gemm(A, B, klo=1, tile=tile)["C"]
     assert (np.abs(got - R) / scale).max() <= 2e-6
     # B upper in K-major form (B[c][k] = 0 for k > c): K up to the tile's last column
     B2 = np.tril(r.standard_normal((n, n)).astype(np.float32))
     R, scale = ref(A, B2, 1.0, 0, None)
-    got = run_gemm(A, B2, khi=1)["C"]
+    got = run_gemm(A, B2, khi=1, tile=tile)["C"]
     assert (np.abs(got - R) / scale).max() <= 2e-6
     # A upper (A[r][k] = 0 for k < r): K from the tile's first row
     A3 = np.triu(r.standard_normal((n, n)).astype(np.float32))
     B3 = r.standard_normal((384, n)).astype(np.float32)
     R, scale = ref(A3, B3, 1.0, 0, None)
-    got = run_gemm(A3, B3, klo=2)["C"]
+    got = run_gemm(A3, B3, klo=2, tile=tile)["C"]
     assert (np.abs(got - R) / scale).max() <= 2e-6
 
 
-def test_gemm_upper_only_updates_upper_triangle():
+@pytest.mark.parametrize("tile", [64, 128, 256])
+def test_gemm_upper_only_updates_upper_triangle(tile):
     r = np.random.default_rng(9)
     n, K = 640, 128
     V = r.standard_normal((n, K)).astype(np.float32)
     C0 = r.standard_normal((n, n)).astype(np.float32)
-    out = run_gemm(V, V, alpha=-1.0, beta=1, C0=C0, upper=1, plain=False, hilo=True)
+    out = run_gemm(V, V, alpha=-1.0, beta=1, C0=C0, upper=1, plain=False, hilo=True, tile=tile)
     R, scale = ref(V, V, -1.0, 1, C0)
     iu = np.triu_indices(n)
     err = np.abs(out["Chilo"][iu] - R[iu]) / scale[iu]
     assert err.max() <= 2e-6
+
+
+def test_sweep_division_equals_ieee_division():
+    """The sweep's reciprocal-plus-correction quotient is the correctly rounded x / s,
+    bit for bit, on 2^30 pairs: random operands and quotients next to code boundaries."""
+    mism = ctypes.c_uint64(0)
+    ex = (ctypes.c_float * 2)()
+    st = G.lib().gptq_test_div_rn(12345, 1 << 30, ctypes.byref(mism), ex, 0, None)
+    assert st == 0, G.lib().gptq_status_string(st).decode()
+    assert mism.value == 0, f"{mism.value} differing quotients, e.g. x={ex[0]!r} s={ex[1]!r}"
