@@ -24,12 +24,15 @@ extern "C" {
  *   chunk_stages: 32-wide K stages summed in one tensor-memory accumulator before the fp32
  *               register add (1 = every stage; the trailing update of the sweep uses 4).
  *   tile_n    : output tile width 64, 128 or 256, or 0 for the library's own choice.
+ *   c_reduce  : 1 = C += alpha A B^T through TMA reduce-add boxes (needs C and beta = 1; C's
+ *               base 16-byte aligned, ldc % 4 == 0), the path of the sweep's trailing update.
  * Requirements: N % 32 == 0, K % 32 == 0, 16-byte aligned bases, leading dimensions % 4 == 0.
  * Synchronizes the stream before returning.  Allocates a 4-byte status word (stream-ordered). */
 gptq_status gptq_test_gemm_tf32x3(int M, int N, int K, const float* A_hi, const float* A_lo, int lda, const float* B_hi,
                                   const float* B_lo, int ldb, float alpha, int beta, int k_lo_mode, int k_hi_mode,
                                   int upper_only, float* C, int ldc, float* C_hi, float* C_lo, int ldh, float* Ct_hi,
-                                  float* Ct_lo, int ldt, int chunk_stages, int tile_n, int device, void* cuda_stream);
+                                  float* Ct_lo, int ldt, int chunk_stages, int tile_n, int c_reduce, int device,
+                                  void* cuda_stream);
 
 /* The sweep's division (S5): x / s from the rounded reciprocal of s plus one fused
  * multiply-add correction, compared bit for bit with IEEE division on `count` (x, s) pairs

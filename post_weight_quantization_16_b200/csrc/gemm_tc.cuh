@@ -20,7 +20,10 @@
 // the zero halves of triangular factors are skipped; tiles wholly below the diagonal of C
 // can be skipped for symmetric updates.
 // Outputs (any subset): plain fp32 C (optionally + C), hi/lo pair (optionally + hi+lo), and a
-// transposed hi/lo pair (coalesced: the 32 lanes of a warp write 32 consecutive rows).
+// transposed hi/lo pair (coalesced: the 32 lanes of a warp write 32 consecutive rows).  The
+// accumulating plain output of the sweep's trailing update (C += alpha A B^T) can instead go
+// out through TMA reduce-add: each epilogue warp stages 32 x 32 boxes in shared memory and
+// L2 adds them into C, so the tile never reads C and its stores are whole swizzled boxes.
 // A and B are addressed as sub-blocks (row/column offsets) of the whole matrices their tensor
 // maps describe, so the maps are encoded once per context.  Rows or columns of a partial
 // tile that fall outside the sub-block read neighbouring data whose products land only in
@@ -41,7 +44,8 @@ struct GtCfg {
   static constexpr int B_BYTES = BN * GT_BK * 4;
   static constexpr int STAGE_BYTES = 2 * GT_A_BYTES + 2 * B_BYTES;  // 48, 64 or 96 KB
   static constexpr int STAGES = BN == 256 ? 2 : (BN == 128 ? 3 : 4);
-  static constexpr int SMEM = STAGES * STAGE_BYTES + 256 + 1024;
+  static constexpr int STG_BYTES = 8 * 32 * 32 * 4;  // one 32 x 32 fp32 staging box per epilogue warp
+  static constexpr int SMEM = STAGES * STAGE_BYTES + STG_BYTES + 256 + 1024;
   static constexpr int TMEM_COLS = 2 * BN;  // two accumulators
 };
 
@@ -58,6 +62,8 @@ struct GemmTCArgs {
   int chunk_stages;  // K stages summed in one TMEM accumulator before the fp32 register add
   float* C;          // plain fp32 output (or nullptr)
   int ldc;
+  int c_reduce;        // 1: C += alpha A B^T by TMA reduce-add through the c_map tensor map (beta = 1)
+  int c_row0, c_col0;  // offset of C inside the matrix c_map describes
   float* Chi;        // hi/lo output (or nullptr)
   float* Clo;
   int ldh;
@@ -117,7 +123,7 @@ template <int BN>
 __global__ void __launch_bounds__(GT_THREADS, 1)
     gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_constant__ CUtensorMap a_lo,
                        const __grid_constant__ CUtensorMap b_hi, const __grid_constant__ CUtensorMap b_lo,
-                       GemmTCArgs p) {
+                       const __grid_constant__ CUtensorMap c_map, GemmTCArgs p) {
   extern __shared__ uint8_t gt_smem_raw[];
   const uint32_t raw_s = smem_u32(gt_smem_raw);
   uint8_t* smem = gt_smem_raw + (((raw_s + 1023u) & ~1023u) - raw_s);
@@ -129,12 +135,14 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
   constexpr int STAGES = Cfg::STAGES, STAGE_BYTES = Cfg::STAGE_BYTES, B_BYTES = Cfg::B_BYTES;
   const int ntiles = gt_num_tiles(p.M, p.N, p.upper_only, BN);
 
-  const uint32_t bar_full = sbase + STAGES * STAGE_BYTES;
+  const uint32_t stg_base = sbase + STAGES * STAGE_BYTES;  // 1024-aligned staging boxes
+  const uint32_t bar_full = stg_base + Cfg::STG_BYTES;
   const uint32_t bar_empty = bar_full + 8 * STAGES;
   const uint32_t bar_tfull = bar_empty + 8 * STAGES;
   const uint32_t bar_tempty = bar_tfull + 16;
   const uint32_t bar_drain = bar_tempty + 16;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + STAGES * STAGE_BYTES + 8 * (2 * STAGES + 5));
+  uint32_t* tmem_slot =
+      reinterpret_cast<uint32_t*>(smem + STAGES * STAGE_BYTES + Cfg::STG_BYTES + 8 * (2 * STAGES + 5));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   if (threadIdx.x == 0) {
@@ -159,12 +167,14 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
     tma_prefetch_desc(&a_lo);
     tma_prefetch_desc(&b_hi);
     tma_prefetch_desc(&b_lo);
+    if (p.c_reduce) tma_prefetch_desc(&c_map);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   griddep_wait();  // inputs of the previous kernel are complete and visible from here on
+  griddep_launch_dependents();  // the next kernel may start its prologue now; it waits for our completion
 
   if (warp == 0) {
     if (lane == 0) {
@@ -270,7 +280,7 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
       for (int cc = 0; cc < HALF / 32; ++cc) {
         const int c0 = cbase + cc * 32;
         const bool ld = p.beta && row_ok && c0 < p.N;
-        if (ld && p.C) {
+        if (ld && p.C && !p.c_reduce) {
           const float4* cp = reinterpret_cast<const float4*>(p.C + static_cast<size_t>(r) * p.ldc + c0);
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
@@ -325,7 +335,30 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
 #pragma unroll
       for (int cc = 0; cc < HALF / 32; ++cc) {
         const int c0 = cbase + cc * 32;
-        if (!row_ok || c0 >= p.N) continue;  // N % 32 == 0: whole 32-column groups
+        if (c0 >= p.N) continue;  // N % 32 == 0: whole 32-column groups
+        if (p.C && p.c_reduce) {
+          // stage the warp's 32 x 32 box (128-byte swizzle: 16-byte chunk k of row r at
+          // chunk k ^ (r % 8)) and add it into C with one TMA reduce; rows past M add zeros
+          const uint32_t stg = stg_base + static_cast<uint32_t>(warp - 2) * 4096u;
+          if (lane == 0) bulk_wait_read0();  // the previous box has left this buffer
+          __syncwarp();
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const float x0 = row_ok ? acc[cc * 32 + 4 * k + 0] : 0.0f, x1 = row_ok ? acc[cc * 32 + 4 * k + 1] : 0.0f;
+            const float x2 = row_ok ? acc[cc * 32 + 4 * k + 2] : 0.0f, x3 = row_ok ? acc[cc * 32 + 4 * k + 3] : 0.0f;
+            const uint32_t a = stg + static_cast<uint32_t>(lane * 128 + ((k ^ (lane & 7)) * 16));
+            asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(a), "f"(x0), "f"(x1), "f"(x2), "f"(x3)
+                         : "memory");
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_reduce_add_2d(&c_map, stg, p.c_col0 + c0, p.c_row0 + m0 + q * 32);
+            bulk_commit();
+          }
+          continue;
+        }
+        if (!row_ok) continue;
         if (p.C) {
           float4* cp = reinterpret_cast<float4*>(p.C + static_cast<size_t>(r) * p.ldc + c0);
 #pragma unroll
@@ -363,7 +396,7 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
     }
   }
 
-  griddep_launch_dependents();
+  if (warp >= 2 && lane == 0 && p.c_reduce) bulk_wait0();  // this warp's reduces are complete
   __syncthreads();
   if (threadIdx.x == 0 && *abort_flag) atomicOr(p.status, ST_TIMEOUT);
   if (warp == 1) {

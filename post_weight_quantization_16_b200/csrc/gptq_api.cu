@@ -61,7 +61,11 @@ struct gptq_ctx {
   // B-operand maps (256-row boxes), hi and lo
   CUtensorMap mA_A[2], mA_VT[2], mA_U[2], mA_Err[2];
   CUtensorMap mB_U[2], mB_VT[2], mB_Ut[2];
+  CUtensorMap mC_Wq;  // Wq as the reduce-add target of the trailing update (32 x 32 boxes)
   cudaStream_t capture_stream = nullptr;
+  cudaStream_t side_stream = nullptr;     // second branch of the captured factorization graph
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+  bool pdl = true;                        // launches overlap their predecessor (programmatic)
   cudaGraphExec_t factor_graph = nullptr;  // the factorization recursion, recorded once
   int64_t factor_graph_launches = 0;
   PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
@@ -163,7 +167,7 @@ cudaError_t launch(gptq_ctx* c, void (*kernel)(KArgs...), dim3 grid, dim3 block,
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = c->pdl ? 1 : 0;
   ++c->launches;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
@@ -193,6 +197,8 @@ struct TcOut {
   float* Cthi = nullptr;
   float* Ctlo = nullptr;
   int ldt = 0;
+  const CUtensorMap* c_map = nullptr;  // C += ... by TMA reduce-add (beta = 1, plain C)
+  int c_row0 = 0, c_col0 = 0;           // offset of C inside the matrix c_map describes
 };
 
 // An operand of gemm_tc: the hi/lo tensor maps of a whole matrix and the sub-block offset,
@@ -298,14 +304,19 @@ gptq_status gemm_tc(gptq_ctx* c, int M, int N, int K, TcOperand A, TcOperand B, 
   a.Cthi = o.Cthi;
   a.Ctlo = o.Ctlo;
   a.ldt = o.ldt;
+  a.c_reduce = o.c_map ? 1 : 0;
+  a.c_row0 = o.c_row0;
+  a.c_col0 = o.c_col0;
   a.status = c->status;
+  if (o.c_map && (beta != 1 || !o.C)) return GPTQ_ERR_ARG;
+  const CUtensorMap& cm = o.c_map ? *o.c_map : *A.hi;  // unused unless c_reduce
   const dim3 grid(std::min(tc_tiles, c->num_sms));
   if (bn == 256)
-    CK(launch(c, gemm_tf32x3_kernel<256>, grid, dim3(GT_THREADS), GtCfg<256>::SMEM, *A.hi, *A.lo, *B.hi, *B.lo, a));
+    CK(launch(c, gemm_tf32x3_kernel<256>, grid, dim3(GT_THREADS), GtCfg<256>::SMEM, *A.hi, *A.lo, *B.hi, *B.lo, cm, a));
   else if (bn == 128)
-    CK(launch(c, gemm_tf32x3_kernel<128>, grid, dim3(GT_THREADS), GtCfg<128>::SMEM, *A.hi, *A.lo, *B.hi, *B.lo, a));
+    CK(launch(c, gemm_tf32x3_kernel<128>, grid, dim3(GT_THREADS), GtCfg<128>::SMEM, *A.hi, *A.lo, *B.hi, *B.lo, cm, a));
   else
-    CK(launch(c, gemm_tf32x3_kernel<64>, grid, dim3(GT_THREADS), GtCfg<64>::SMEM, *A.hi, *A.lo, *B.hi, *B.lo, a));
+    CK(launch(c, gemm_tf32x3_kernel<64>, grid, dim3(GT_THREADS), GtCfg<64>::SMEM, *A.hi, *A.lo, *B.hi, *B.lo, cm, a));
   CKL("gemm_tc");
   return GPTQ_OK;
 }
@@ -345,15 +356,32 @@ gptq_status chol_inv(gptq_ctx* c, int o, int h) {
   if ((s = gemm_tc(c, h1, h1, h2, op(c->mA_VT, c->VT_hi, c->VT_lo, o, o2), op(c->mB_VT, c->VT_hi, c->VT_lo, o, o2), -1.f, 1, GT_KLO_NONE, GT_KHI_NONE, 1,
                    a11)) != GPTQ_OK)
     return s;
-  // T^T = (V12 U22)^T into the lower block [o2.., o..]   (Ut22 rows as B; k <= column)
+  // T^T = (V12 U22)^T into the lower block [o2.., o..]   (Ut22 rows as B; k <= column).
+  // Only U12 below needs it, so while the graph is being captured it runs on a second
+  // branch, beside the factorization of A11 (which touches only [o, o+h1)^2).
   TcOut tt;
   tt.Cthi = at(c->VT_hi, o2, o);
   tt.Ctlo = at(c->VT_lo, o2, o);
   tt.ldt = n;
-  if ((s = gemm_tc(c, h1, h2, h2, op(c->mA_VT, c->VT_hi, c->VT_lo, o, o2), op(c->mB_Ut, c->Ut_hi, c->Ut_lo, o2, o2), 1.f, 0, GT_KLO_NONE, GT_KHI_COL, 0,
-                   tt)) != GPTQ_OK)
-    return s;
+  const bool branch = c->side_stream != nullptr;
+  cudaStream_t main_stream = c->stream;
+  if (branch) {
+    CK(cudaEventRecord(c->ev_fork, main_stream));
+    CK(cudaStreamWaitEvent(c->side_stream, c->ev_fork, 0));
+    c->stream = c->side_stream;
+    c->pdl = false;
+  }
+  s = gemm_tc(c, h1, h2, h2, op(c->mA_VT, c->VT_hi, c->VT_lo, o, o2), op(c->mB_Ut, c->Ut_hi, c->Ut_lo, o2, o2), 1.f, 0,
+              GT_KLO_NONE, GT_KHI_COL, 0, tt);
+  if (branch) {
+    c->stream = main_stream;
+    c->pdl = true;
+    if (s == GPTQ_OK) CK(cudaEventRecord(c->ev_join, c->side_stream));
+  }
+  if (s != GPTQ_OK) return s;
   if ((s = chol_inv(c, o, h1)) != GPTQ_OK) return s;
+  // the join: the latest T on the branch (branch launches are in order, so this one too)
+  if (branch) CK(cudaStreamWaitEvent(main_stream, c->ev_join, 0));
   // U12 = -U11 T  (and Ut21 = U12^T)      (U11 rows as A; k >= row)
   TcOut u12;
   u12.Chi = at(c->U_hi, o, o2);
@@ -386,6 +414,7 @@ gptq_status encode_maps(gptq_ctx* c) {
       {&c->mB_U[0], c->U_hi, n, n, n, GT_BOX_N},        {&c->mB_U[1], c->U_lo, n, n, n, GT_BOX_N},
       {&c->mB_VT[0], c->VT_hi, n, n, n, GT_BOX_N},      {&c->mB_VT[1], c->VT_lo, n, n, n, GT_BOX_N},
       {&c->mB_Ut[0], c->Ut_hi, n, n, n, GT_BOX_N},      {&c->mB_Ut[1], c->Ut_lo, n, n, n, GT_BOX_N},
+      {&c->mC_Wq, c->Wq, c->m_max, n, n, 32},
   };
   for (auto& e : list)
     if ((s = make_map(c, e.m, e.p, e.rows, e.cols, e.ld, e.box)) != GPTQ_OK) return s;
@@ -397,6 +426,9 @@ gptq_status encode_maps(gptq_ctx* c) {
 gptq_status run_factorization(gptq_ctx* c) {
   if (!c->factor_graph) {
     if (!c->capture_stream) CK(cudaStreamCreateWithFlags(&c->capture_stream, cudaStreamNonBlocking));
+    if (!c->side_stream) CK(cudaStreamCreateWithFlags(&c->side_stream, cudaStreamNonBlocking));
+    if (!c->ev_fork) CK(cudaEventCreateWithFlags(&c->ev_fork, cudaEventDisableTiming));
+    if (!c->ev_join) CK(cudaEventCreateWithFlags(&c->ev_join, cudaEventDisableTiming));
     cudaStream_t user = c->stream;
     const int64_t l0 = c->launches;
     c->stream = c->capture_stream;
@@ -436,6 +468,11 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 void free_all(gptq_ctx* c) {
   if (c->factor_graph) cudaGraphExecDestroy(c->factor_graph);
   if (c->capture_stream) cudaStreamDestroy(c->capture_stream);
+  if (c->side_stream) cudaStreamDestroy(c->side_stream);
+  if (c->ev_fork) cudaEventDestroy(c->ev_fork);
+  if (c->ev_join) cudaEventDestroy(c->ev_join);
+  c->side_stream = nullptr;
+  c->ev_fork = c->ev_join = nullptr;
   c->factor_graph = nullptr;
   c->capture_stream = nullptr;
   float** fs[] = {&c->H,     &c->A_hi,  &c->A_lo,  &c->VT_hi, &c->VT_lo,  &c->U_hi,   &c->U_lo,
@@ -738,6 +775,8 @@ gptq_status gptq_quantize_layer(gptq_ctx* c, const void* W, int64_t m, gptq_qpar
         TcOut w;
         w.C = c->Wq + i2;
         w.ldc = n;
+        w.c_map = &c->mC_Wq;
+        w.c_col0 = i2;
         gptq_status st = gemm_tc(c, mi, s1 - i2, SW_B, TcOperand{&c->mA_Err[0], &c->mA_Err[1], 0, i1 - s0, nullptr, nullptr, 0},
                                  TcOperand{&c->mB_Ut[0], &c->mB_Ut[1], i2, i1, nullptr, nullptr, 0}, -1.f, 1,
                                  GT_KLO_NONE, GT_KHI_NONE, 0, w, SW_B / GT_BK);
@@ -749,6 +788,8 @@ gptq_status gptq_quantize_layer(gptq_ctx* c, const void* W, int64_t m, gptq_qpar
       TcOut w;
       w.C = c->Wq + s1;
       w.ldc = n;
+      w.c_map = &c->mC_Wq;
+      w.c_col0 = s1;
       gptq_status st = gemm_tc(c, mi, n - s1, s1 - s0, TcOperand{&c->mA_Err[0], &c->mA_Err[1], 0, 0, nullptr, nullptr, 0},
                                TcOperand{&c->mB_Ut[0], &c->mB_Ut[1], s1, s0, nullptr, nullptr, 0}, -1.f, 1,
                                GT_KLO_NONE, GT_KHI_NONE, 0, w, SW_B / GT_BK);
@@ -786,8 +827,10 @@ int64_t gptq_launch_count(const gptq_ctx* c) { return c ? c->launches : -1; }
 gptq_status gptq_test_gemm_tf32x3(int M, int N, int K, const float* A_hi, const float* A_lo, int lda, const float* B_hi,
                                   const float* B_lo, int ldb, float alpha, int beta, int k_lo_mode, int k_hi_mode,
                                   int upper_only, float* C, int ldc, float* C_hi, float* C_lo, int ldh, float* Ct_hi,
-                                  float* Ct_lo, int ldt, int chunk_stages, int tile_n, int device, void* cuda_stream) {
+                                  float* Ct_lo, int ldt, int chunk_stages, int tile_n, int c_reduce, int device,
+                                  void* cuda_stream) {
   if (chunk_stages < 1) return GPTQ_ERR_ARG;
+  if (c_reduce && (!C || beta != 1)) return GPTQ_ERR_ARG;
   if (tile_n != 0 && tile_n != 64 && tile_n != 128 && tile_n != 256) return GPTQ_ERR_ARG;
   if (!A_hi || !A_lo || !B_hi || !B_lo || M < 1 || N < 1 || K < GT_BK) return GPTQ_ERR_ARG;
   if (k_lo_mode < 0 || k_lo_mode > 2 || k_hi_mode < 0 || k_hi_mode > 1 || (beta != 0 && beta != 1)) return GPTQ_ERR_ARG;
@@ -818,8 +861,12 @@ gptq_status gptq_test_gemm_tf32x3(int M, int N, int K, const float* A_hi, const 
   o.Cthi = Ct_hi;
   o.Ctlo = Ct_lo;
   o.ldt = ldt;
-  CUtensorMap ma[2], mb[2];
+  CUtensorMap ma[2], mb[2], mc;
   gptq_status s = GPTQ_OK;
+  if (c_reduce) {
+    s = make_map(&t, &mc, C, M, N, ldc, 32);
+    o.c_map = &mc;
+  }
   if (s == GPTQ_OK) s = make_map(&t, &ma[0], A_hi, M, K, lda, GT_BM);
   if (s == GPTQ_OK) s = make_map(&t, &ma[1], A_lo, M, K, lda, GT_BM);
   if (s == GPTQ_OK) s = make_map(&t, &mb[0], B_hi, N, K, ldb, GT_BOX_N);

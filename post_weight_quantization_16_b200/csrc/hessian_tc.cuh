@@ -107,6 +107,7 @@ __global__ void __launch_bounds__(HS_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   griddep_wait();  // inputs of the previous kernel are complete and visible from here on
+  griddep_launch_dependents();  // the next kernel may start its prologue now; it waits for our completion
 
   if (warp == 0) {
     if (lane == 0) {
@@ -231,7 +232,6 @@ __global__ void __launch_bounds__(HS_THREADS, 1)
     }
   }
 
-  griddep_launch_dependents();
   __syncthreads();
   if (threadIdx.x == 0 && *abort_flag) atomicOr(status, ST_TIMEOUT);
   if (warp == 1) {

@@ -20,6 +20,7 @@ namespace gptq {
 
 __global__ void mirror_upper_kernel(float* __restrict__ H, int n) {
   griddep_wait();
+  griddep_launch_dependents();
   __shared__ float t[32][33];
   const int tr = blockIdx.y, tc = blockIdx.x;
   if (tr > tc) return;
@@ -37,6 +38,7 @@ __global__ void mirror_upper_kernel(float* __restrict__ H, int n) {
 __global__ void diag_stats_kernel(const float* __restrict__ H, int n, float* __restrict__ keys,
                                   uint8_t* __restrict__ dead, double* __restrict__ mean_out) {
   griddep_wait();
+  griddep_launch_dependents();
   __shared__ double red[32];
   double s = 0.0;
   for (int i = threadIdx.x; i < n; i += blockDim.x) {
@@ -61,6 +63,7 @@ __global__ void diag_stats_kernel(const float* __restrict__ H, int n, float* __r
 // perm[rank(i)] = i with rank(i) = #{j : key_j > key_i or (key_j == key_i and j < i)}.
 __global__ void rank_perm_kernel(const float* __restrict__ keys, int n, int32_t* __restrict__ perm) {
   griddep_wait();
+  griddep_launch_dependents();
   __shared__ float ks[1024];
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   const float ki = (i < n) ? keys[i] : 0.0f;
@@ -80,6 +83,7 @@ __global__ void rank_perm_kernel(const float* __restrict__ keys, int n, int32_t*
 
 __global__ void identity_perm_kernel(int n, int32_t* __restrict__ perm) {
   griddep_wait();
+  griddep_launch_dependents();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) perm[i] = i;
 }
@@ -89,6 +93,7 @@ __global__ void gather_damp_kernel(const float* __restrict__ H, int n, const int
                                    const float* __restrict__ keys, const double* __restrict__ mean,
                                    double damp, float* __restrict__ A_hi, float* __restrict__ A_lo) {
   griddep_wait();
+  griddep_launch_dependents();
   extern __shared__ float row_s[];
   const int a = blockIdx.x;
   const int pa = perm[a];
@@ -113,6 +118,7 @@ __global__ void gather_damp_kernel(const float* __restrict__ H, int n, const int
 __global__ void init_w_kernel(const __half* __restrict__ W, int n, const int32_t* __restrict__ perm,
                               const uint8_t* __restrict__ dead, float* __restrict__ Wq) {
   griddep_wait();
+  griddep_launch_dependents();
   extern __shared__ __half wrow_s[];
   const int r = blockIdx.x;
   const __half* src = W + static_cast<size_t>(r) * n;
@@ -129,6 +135,7 @@ __global__ void init_w_kernel(const __half* __restrict__ W, int n, const int32_t
 __global__ void combine_hilo_kernel(const float* __restrict__ hi, const float* __restrict__ lo, size_t count,
                                     float* __restrict__ out) {
   griddep_wait();
+  griddep_launch_dependents();
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < count;
        i += static_cast<size_t>(gridDim.x) * blockDim.x)
     out[i] = hi[i] + lo[i];
@@ -136,6 +143,7 @@ __global__ void combine_hilo_kernel(const float* __restrict__ hi, const float* _
 
 __global__ void g_idx_kernel(const int32_t* __restrict__ perm, int n, int g, int32_t* __restrict__ g_idx) {
   griddep_wait();
+  griddep_launch_dependents();
   const int k = blockIdx.x * blockDim.x + threadIdx.x;
   if (k < n) g_idx[perm[k]] = k / g;
 }

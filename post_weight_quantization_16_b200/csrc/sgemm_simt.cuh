@@ -201,6 +201,7 @@ template <int TM, int TN>
 __global__ void __launch_bounds__(GS_THREADS) gemm_hilo_simt_kernel(GemmSimtArgs p) {
   constexpr int RI = TM / 16, RJ = TN / 16;
   griddep_wait();
+  griddep_launch_dependents();
   const int m0 = blockIdx.y * TM, n0 = blockIdx.x * TN;
   if (p.upper_only && m0 >= n0 + TN) return;
   int kb = 0, ke = p.K;
@@ -286,7 +287,6 @@ __global__ void __launch_bounds__(GS_THREADS) gemm_hilo_simt_kernel(GemmSimtArgs
     }
   }
   asm volatile("cp.async.wait_group 0;" ::: "memory");
-  griddep_launch_dependents();
 
 #pragma unroll
   for (int i = 0; i < RI; ++i) {

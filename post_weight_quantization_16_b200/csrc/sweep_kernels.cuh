@@ -4,19 +4,23 @@
 //  each column's error into the not-yet-quantized columns; "模型量化实战…" §3.2
 //  quantize_block: blocks of 128 columns.)
 //
-// Rows of W are independent once U is known.  Eight lanes of a warp share one row: lane
-// l (0..7 within its group) holds the row's block columns 16l .. 16l+15 in registers, so a
-// warp sweeps four rows and a 256-thread CTA 32 rows.  For column i the owning lane
-// (i / 16) computes the code, the dequantized value and e = (w - q) / U[i][i] and updates
-// its own later columns, w[j] -= e * U[i][j], so the per-column dependent chain never
-// leaves the lane's registers.  After each 16-column chunk its errors reach the row's later
-// lanes in one batch (16 shuffles, then 16 x 16 fused multiply-adds per lane).  Group scales/zeros come from a min/max over the group's
-// current values reduced across the row's lanes with shuffles.  The U block (128 x 128) is
-// staged in shared memory with asynchronous copies, in a bank-skewed layout so the eight
-// 16-column segments a warp reads at once hit different banks.
-// The block's errors go to Err; the columns after the block receive them through tensor-core
-// products (S6) launched by the host: within a super-block of columns right after each block,
-// beyond it once per super-block.
+// Rows of W are independent once U is known.  A CTA takes 32 rows and keeps their 128
+// block columns in shared memory.  The block is walked in eight chunks of 16 columns:
+//   * warp 0, the walker, gives each lane one row.  For chunk k it loads the row's 16
+//     values, applies the previous chunk's errors to them, then walks the 16 columns:
+//     code, dequantized value, e = (w - q) / U[i][i], and w[j] -= e * U[i][j] for the
+//     chunk's later columns.  The per-column dependent chain stays in the lane's registers
+//     and every U value it needs is the same for all 32 lanes (a broadcast read).
+//   * warps 1-3, the updaters, apply chunk k's errors to chunks k+2 .. 7 of the tile while
+//     the walker is on chunk k+1 (a rank-16 update in shared memory).
+// Named barriers hand each chunk's errors to the updaters and each finished update back to
+// the walker.  Group scales/zeros come from a min/max over the group's current values.  The
+// U block (128 x 128, hi + lo) is staged in shared memory before the kernel waits on its
+// predecessor, so the staging overlaps the previous kernel's tail.  At the end the CTA writes
+// the block's errors to Err, the packed code words and the dequantized weights row by row.
+// The columns after the block receive the errors through tensor-core products (S6) launched
+// by the host: within a super-block of columns right after each block, beyond it once per
+// super-block.
 //
 // The integer decisions (code and zero-point) are taken in fp32 with correctly rounded
 // division and round-half-to-even, the precision the pages' own sketches use.
@@ -28,14 +32,17 @@
 
 namespace gptq {
 
-constexpr int SW_B = 128;            // sweep block (columns)
-constexpr int SW_LANES = 8;          // lanes per row
-constexpr int SW_COLS = SW_B / SW_LANES;  // 16 columns per lane
-constexpr int SW_THREADS = 256;
-constexpr int SW_ROWS = SW_THREADS / SW_LANES;  // 32 rows per CTA
-constexpr int SW_SEG = 20;                      // skewed segment stride (floats) in shared memory
-constexpr int SW_ULD = SW_LANES * SW_SEG;       // 160 floats per staged U row
-constexpr int SW_SMEM = 2 * SW_B * SW_ULD * 4 + SW_B * 4 + SW_B * 4 + SW_ROWS * 32 * 4;
+constexpr int SW_B = 128;        // sweep block (columns)
+constexpr int SW_ROWS = 32;      // rows per CTA (one walker lane each)
+constexpr int SW_CH = 16;        // chunk width
+constexpr int SW_NCH = SW_B / SW_CH;
+constexpr int SW_THREADS = 128;  // walker warp + three updater warps
+constexpr int SW_WLD = 132;      // W tile pitch (floats): 16-byte rows, quarter-warps in distinct banks
+constexpr int SW_ELD = 129;      // error / dequantized tile pitch (floats): odd, lane-per-row access
+constexpr int SW_CLD = 132;      // code tile pitch (bytes): 33 words, lane-per-row byte stores in distinct banks
+// U block | W tile | errors | dequantized values | 1/U[i][i] | perm | group partials | codes
+constexpr int SW_SMEM = SW_B * SW_B * 4 + SW_ROWS * SW_WLD * 4 + 2 * SW_ROWS * SW_ELD * 4 + SW_B * 4 + SW_B * 4 +
+                        3 * 4 * SW_ROWS * 4 + SW_ROWS * SW_CLD;
 
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
@@ -75,16 +82,6 @@ __device__ __forceinline__ void group_scale_zero(float wmin, float wmax, float a
     const float xmax = fmaxf(wmax, 0.0f);
     s = fmaxf(__fdiv_rn(__fsub_rn(xmax, xmin), qp.qmax_f), 1e-8f);
     z = -rintf(__fdiv_rn(xmin, s));
-  }
-}
-
-// min / max / max|.| over the eight lanes of a row group
-__device__ __forceinline__ void group_reduce(float& wmin, float& wmax, float& amax) {
-#pragma unroll
-  for (int o = 1; o < SW_LANES; o <<= 1) {
-    wmin = fminf(wmin, __shfl_xor_sync(0xffffffffu, wmin, o));
-    wmax = fmaxf(wmax, __shfl_xor_sync(0xffffffffu, wmax, o));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   }
 }
 
@@ -140,38 +137,67 @@ __global__ void div_rn_check_kernel(uint64_t seed, long long count, unsigned lon
   }
 }
 
-template <int GSUB>  // 0: groups of >= 128 columns (params at block starts); 32 or 64: inside the block
+__device__ __forceinline__ void named_arrive(int id) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(SW_THREADS) : "memory");
+}
+__device__ __forceinline__ void named_sync(int id) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(SW_THREADS) : "memory");
+}
+
+// GSUB 0: groups of >= 128 columns (parameters at block starts); 32 or 64: groups inside the block
+template <int GSUB>
 __global__ void __launch_bounds__(SW_THREADS)
     sweep_block_kernel(SweepArgs a, int i1) {
   extern __shared__ __align__(16) float sw_smem[];
-  float* Us = sw_smem;                                          // [128][160] U block (skewed)
-  float* Ul = Us + SW_B * SW_ULD;                               // [128][160] lo part while it lands
-  float* rU = Ul + SW_B * SW_ULD;                               // [128] 1 / U[i][i]
-  int* perm_s = reinterpret_cast<int*>(rU + SW_B);              // [128]
-  uint32_t* cw = reinterpret_cast<uint32_t*>(perm_s + SW_B);    // [32 rows][32 words] packed codes
+  float* Us = sw_smem;                                    // [128][128] U block
+  float* Ws = Us + SW_B * SW_B;                           // [32][132] W tile
+  float* Es = Ws + SW_ROWS * SW_WLD;                      // [32][129] scaled errors
+  float* Hs = Es + SW_ROWS * SW_ELD;                      // [32][129] dequantized values
+  float* rU = Hs + SW_ROWS * SW_ELD;                      // [128] 1 / U[i][i]
+  int* perm_s = reinterpret_cast<int*>(rU + SW_B);        // [128]
+  float* part = reinterpret_cast<float*>(perm_s + SW_B);  // [3][4][32] group min / max / max|.| partials
+  uint8_t* codes8 = reinterpret_cast<uint8_t*>(part + 3 * 4 * SW_ROWS);  // [32][132] codes
 
-  griddep_wait();
   const int tid = threadIdx.x;
-  const int lane = tid & 31;
-  const int l8 = lane & (SW_LANES - 1);      // segment of the row this lane holds
-  const int gbase = lane & ~(SW_LANES - 1);  // first lane of the row's group
-  const int rloc = tid / SW_LANES;           // row within the CTA
+  const int warp = tid >> 5, lane = tid & 31;
   const int n = a.n;
+  const int row0 = blockIdx.x * SW_ROWS;
 
-  // stage U[i1 + k][i1 + j] at Us[k][SEG * (j / 16) + j % 16]
+  griddep_launch_dependents();  // the next kernel may start its prologue now; it waits for our completion
+  // ---- before the predecessor is waited on: the U block (written long before) ----
   for (int idx = tid; idx < SW_B * (SW_B / 4); idx += SW_THREADS) {
     const int k = idx / (SW_B / 4), j = (idx % (SW_B / 4)) * 4;
-    const size_t g = static_cast<size_t>(i1 + k) * n + i1 + j;
-    const int so = k * SW_ULD + (j / SW_COLS) * SW_SEG + (j % SW_COLS);
-    cp_async16(Us + so, a.U + g);
-    if (a.U_lo) cp_async16(Ul + so, a.U_lo + g);
+    cp_async16(Us + k * SW_B + j, a.U + static_cast<size_t>(i1 + k) * n + i1 + j);
   }
   if (tid < SW_B) perm_s[tid] = a.perm[i1 + tid];
-  for (int idx = tid; idx < SW_ROWS * 32; idx += SW_THREADS) cw[idx] = 0u;
+  cp_async_wait_all();
+  __syncthreads();
+  if (a.U_lo) {
+    for (int idx = tid; idx < SW_B * (SW_B / 4); idx += SW_THREADS) {
+      const int k = idx / (SW_B / 4), j = (idx % (SW_B / 4)) * 4;
+      const float4 l = *reinterpret_cast<const float4*>(a.U_lo + static_cast<size_t>(i1 + k) * n + i1 + j);
+      float4* h = reinterpret_cast<float4*>(Us + k * SW_B + j);
+      float4 v = *h;
+      v.x += l.x;
+      v.y += l.y;
+      v.z += l.z;
+      v.w += l.w;
+      *h = v;
+    }
+    __syncthreads();
+  }
+  if (tid < SW_B) rU[tid] = 1.0f / Us[tid * SW_B + tid];
 
-  const int r = blockIdx.x * SW_ROWS + rloc;
-  const bool valid = r < a.m;
-  const int rr = valid ? r : 0;
+  // ---- the W tile (written by the previous kernel) ----
+  griddep_wait();
+  for (int idx = tid; idx < SW_ROWS * (SW_B / 4); idx += SW_THREADS) {
+    const int rl = idx / (SW_B / 4), j = (idx % (SW_B / 4)) * 4;
+    const float4 v = (row0 + rl < a.m)
+                         ? *reinterpret_cast<const float4*>(a.Wq + static_cast<size_t>(row0 + rl) * n + i1 + j)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+    *reinterpret_cast<float4*>(Ws + rl * SW_WLD + j) = v;
+  }
+  __syncthreads();
 
   QParams qp;
   if (a.sym) {
@@ -184,193 +210,215 @@ __global__ void __launch_bounds__(SW_THREADS)
   qp.qmax_f = qp.hi;
   qp.zsym = static_cast<float>(1 << (a.bits - 1));
 
-  // this lane's 16 columns of the row, while U lands
-  float w[SW_COLS];
-  {
-    const float4* src = reinterpret_cast<const float4*>(a.Wq + static_cast<size_t>(rr) * n + i1 + SW_COLS * l8);
-#pragma unroll
-    for (int j4 = 0; j4 < SW_COLS / 4; ++j4) {
-      const float4 v = valid ? src[j4] : make_float4(0.f, 0.f, 0.f, 0.f);
-      w[4 * j4 + 0] = v.x;
-      w[4 * j4 + 1] = v.y;
-      w[4 * j4 + 2] = v.z;
-      w[4 * j4 + 3] = v.w;
+  // group parameters at the block start (groups of >= 128 columns): each thread reduces a
+  // quarter of its row's block columns (and of the group's columns past the block)
+  if (GSUB == 0 && i1 % a.g == 0) {
+    const int rl = tid & 31, qtr = tid >> 5;
+    float wmin = INFINITY, wmax = -INFINITY, amax = 0.0f;
+    for (int j = qtr * 32; j < qtr * 32 + 32; ++j) {
+      const float x = Ws[rl * SW_WLD + j];
+      wmin = fminf(wmin, x);
+      wmax = fmaxf(wmax, x);
+      amax = fmaxf(amax, fabsf(x));
     }
+    if (row0 + rl < a.m) {
+      const float* row = a.Wq + static_cast<size_t>(row0 + rl) * n;
+      for (int c = i1 + SW_B + qtr; c < i1 + a.g; c += 4) {
+        const float x = row[c];
+        wmin = fminf(wmin, x);
+        wmax = fmaxf(wmax, x);
+        amax = fmaxf(amax, fabsf(x));
+      }
+    }
+    part[(0 * 4 + qtr) * SW_ROWS + rl] = wmin;
+    part[(1 * 4 + qtr) * SW_ROWS + rl] = wmax;
+    part[(2 * 4 + qtr) * SW_ROWS + rl] = amax;
   }
-  cp_async_wait_all();
-  __syncthreads();
-  if (a.U_lo) {
-    for (int idx = tid; idx < SW_B * SW_ULD; idx += SW_THREADS) Us[idx] += Ul[idx];
-    __syncthreads();
-  }
-  if (tid < SW_B) rU[tid] = 1.0f / Us[tid * SW_ULD + (tid / SW_COLS) * SW_SEG + (tid % SW_COLS)];
   __syncthreads();
 
-  float s = 1.0f, z = 0.0f;
-  if (GSUB == 0) {
-    const int gi = i1 / a.g;
-    if (i1 % a.g == 0) {
-      float wmin = w[0], wmax = w[0], amax = 0.0f;
+  if (warp == 0) {
+    // ================= walker: lane = row =================
+    const int rl = lane;
+    const bool valid = row0 + rl < a.m;
+    float s = 1.0f, z = 0.0f;
+    if (GSUB == 0) {
+      const int gi = i1 / a.g;
+      if (i1 % a.g == 0) {
+        float wmin = part[rl], wmax = part[4 * SW_ROWS + rl], amax = part[8 * SW_ROWS + rl];
 #pragma unroll
-      for (int j = 0; j < SW_COLS; ++j) {
-        wmin = fminf(wmin, w[j]);
-        wmax = fmaxf(wmax, w[j]);
-        amax = fmaxf(amax, fabsf(w[j]));
+        for (int q = 1; q < 4; ++q) {
+          wmin = fminf(wmin, part[q * SW_ROWS + rl]);
+          wmax = fmaxf(wmax, part[(4 + q) * SW_ROWS + rl]);
+          amax = fmaxf(amax, part[(8 + q) * SW_ROWS + rl]);
+        }
+        group_scale_zero(wmin, wmax, amax, qp, a.sym, s, z);
+        if (valid) {
+          a.scales[static_cast<size_t>(row0 + rl) * a.G + gi] = s;
+          a.zeros[static_cast<size_t>(row0 + rl) * a.G + gi] = z;
+        }
+      } else if (valid) {
+        s = a.scales[static_cast<size_t>(row0 + rl) * a.G + gi];
+        z = a.zeros[static_cast<size_t>(row0 + rl) * a.G + gi];
       }
-      if (valid) {  // columns of the group beyond this block (already up to date)
-        const float* row = a.Wq + static_cast<size_t>(rr) * n;
-        for (int c = i1 + SW_B + l8; c < i1 + a.g; c += SW_LANES) {
-          const float x = row[c];
-          wmin = fminf(wmin, x);
-          wmax = fmaxf(wmax, x);
-          amax = fmaxf(amax, fabsf(x));
+    }
+    // inside the rounding the zero-point enters only for asymmetric codes
+    float zs = a.sym ? 0.0f : z;
+    float rs = __frcp_rn(s);
+    const float rnd = 12582912.0f;  // 1.5 * 2^23: adding and subtracting it rounds half-to-even
+    const bool want_what = a.W_hat != nullptr;
+    float* wrow = Ws + rl * SW_WLD;
+    float ep[SW_CH];  // the previous chunk's errors
+#pragma unroll
+    for (int t = 0; t < SW_CH; ++t) ep[t] = 0.0f;
+    int u_seen = 0;  // updater passes waited for
+#pragma unroll 1
+    for (int k = 0; k < SW_NCH; ++k) {
+      // chunk k has chunks <= k-2 applied once the updaters' pass k-2 is done
+      for (; u_seen <= k - 2; ++u_seen) named_sync(3 + (u_seen & 1));
+      float w[SW_CH];
+#pragma unroll
+      for (int j4 = 0; j4 < SW_CH / 4; ++j4) {
+        const float4 v = *reinterpret_cast<const float4*>(wrow + k * SW_CH + 4 * j4);
+        w[4 * j4 + 0] = v.x;
+        w[4 * j4 + 1] = v.y;
+        w[4 * j4 + 2] = v.z;
+        w[4 * j4 + 3] = v.w;
+      }
+      if (k > 0) {  // chunk k-1's errors, in the walker's own registers
+#pragma unroll
+        for (int t = 0; t < SW_CH; ++t) {
+          const float4* urow = reinterpret_cast<const float4*>(Us + ((k - 1) * SW_CH + t) * SW_B + k * SW_CH);
+#pragma unroll
+          for (int j4 = 0; j4 < SW_CH / 4; ++j4) {
+            const float4 u = urow[j4];
+            w[4 * j4 + 0] = fmaf(-ep[t], u.x, w[4 * j4 + 0]);
+            w[4 * j4 + 1] = fmaf(-ep[t], u.y, w[4 * j4 + 1]);
+            w[4 * j4 + 2] = fmaf(-ep[t], u.z, w[4 * j4 + 2]);
+            w[4 * j4 + 3] = fmaf(-ep[t], u.w, w[4 * j4 + 3]);
+          }
         }
       }
-      group_reduce(wmin, wmax, amax);
-      group_scale_zero(wmin, wmax, amax, qp, a.sym, s, z);
-      if (valid && l8 == 0) {
-        a.scales[static_cast<size_t>(rr) * a.G + gi] = s;
-        a.zeros[static_cast<size_t>(rr) * a.G + gi] = z;
-      }
-    } else if (valid) {
-      s = a.scales[static_cast<size_t>(rr) * a.G + gi];
-      z = a.zeros[static_cast<size_t>(rr) * a.G + gi];
-    }
-  }
-
-  uint32_t mycode[SW_COLS];
-  float myerr[SW_COLS], mywhat[SW_COLS];
+      if (GSUB > 0 && ((k * SW_CH) % (GSUB > 0 ? GSUB : SW_CH)) == 0) {
+        // a group starts here: its later chunks need the updaters' pass k-1 as well
+        for (; u_seen <= k - 1; ++u_seen) named_sync(3 + (u_seen & 1));
+        float wmin = w[0], wmax = w[0], amax = 0.0f;
 #pragma unroll
-  for (int t = 0; t < SW_COLS; ++t) {
-    mycode[t] = 0u;
-    myerr[t] = 0.0f;
-    mywhat[t] = 0.0f;
-  }
-  // inside the rounding the zero-point enters only for asymmetric codes
-  float zs = a.sym ? 0.0f : z;
-  float rs = __frcp_rn(s);
-
-#pragma unroll 1
-  for (int c = 0; c < SW_LANES; ++c) {  // chunk c = columns 16c .. 16c+15, owned by lane c of each row
-    if (GSUB > 0 && ((c * SW_COLS) % (GSUB > 0 ? GSUB : SW_COLS)) == 0) {
-      constexpr int NL = (GSUB > 0 ? GSUB : SW_COLS) / SW_COLS;  // lanes covering one group
-      const bool in = (l8 >= c) && (l8 < c + NL);
-      float wmin = in ? w[0] : INFINITY, wmax = in ? w[0] : -INFINITY, amax = 0.0f;
-      if (in) {
-#pragma unroll
-        for (int j = 0; j < SW_COLS; ++j) {
+        for (int j = 0; j < SW_CH; ++j) {
           wmin = fminf(wmin, w[j]);
           wmax = fmaxf(wmax, w[j]);
           amax = fmaxf(amax, fabsf(w[j]));
         }
+        for (int j = (k + 1) * SW_CH; j < k * SW_CH + GSUB; ++j) {
+          const float x = wrow[j];
+          wmin = fminf(wmin, x);
+          wmax = fmaxf(wmax, x);
+          amax = fmaxf(amax, fabsf(x));
+        }
+        group_scale_zero(wmin, wmax, amax, qp, a.sym, s, z);
+        zs = a.sym ? 0.0f : z;
+        rs = __frcp_rn(s);
+        if (valid) {
+          const int gi = (i1 + k * SW_CH) / a.g;
+          a.scales[static_cast<size_t>(row0 + rl) * a.G + gi] = s;
+          a.zeros[static_cast<size_t>(row0 + rl) * a.G + gi] = z;
+        }
       }
-      group_reduce(wmin, wmax, amax);
-      group_scale_zero(wmin, wmax, amax, qp, a.sym, s, z);
-      zs = a.sym ? 0.0f : z;
-      rs = __frcp_rn(s);
-      if (valid && l8 == 0) {
-        const int gi = (i1 + c * SW_COLS) / a.g;
-        a.scales[static_cast<size_t>(rr) * a.G + gi] = s;
-        a.zeros[static_cast<size_t>(rr) * a.G + gi] = z;
-      }
-    }
-    const bool owner = (l8 == c);
-    const float* useg = Us + (c * SW_COLS) * SW_ULD + l8 * SW_SEG;  // U rows of the chunk, this lane's columns
-    // The owner walks its 16 columns with nothing but its own registers on the dependent
-    // chain; the other lanes run the same instructions with a zero error (no effect).
-    float ec[SW_COLS];
+      // the walk (no shared-memory stores inside it, so its loads can be issued early)
+      float qc[SW_CH];
 #pragma unroll
-    for (int t = 0; t < SW_COLS; ++t) {
-      const float x = w[t];
-      const float v = __fadd_rn(div_rn(x, s, rs), zs);
-      const float q = fminf(fmaxf(rintf(v), qp.lo), qp.hi);
-      const float qz = __fsub_rn(q, zs);
-      const float e = __fmul_rn(__fmaf_rn(-qz, s, x), rU[c * SW_COLS + t]);
-      ec[t] = e;
-      if (owner) {
-        mycode[t] = static_cast<uint32_t>(static_cast<int>(q - qp.lo));
-        myerr[t] = e;
-        mywhat[t] = __fmul_rn(qz, s);
-      }
-      const float eo = owner ? e : 0.0f;
-      const float4* urow = reinterpret_cast<const float4*>(useg + t * SW_ULD);
+      for (int t = 0; t < SW_CH; ++t) {
+        const int i = k * SW_CH + t;
+        const float x = w[t];
+        const float v = __fadd_rn(div_rn(x, s, rs), zs);
+        // clamp, then round half-to-even (clamping to integer bounds commutes with rounding)
+        const float q = __fsub_rn(__fadd_rn(fminf(fmaxf(v, qp.lo), qp.hi), rnd), rnd);
+        const float e = __fmul_rn(__fmaf_rn(-__fsub_rn(q, zs), s, x), rU[i]);
+        ep[t] = e;
+        qc[t] = q;
+        const float4* urow = reinterpret_cast<const float4*>(Us + i * SW_B + k * SW_CH);
 #pragma unroll
-      for (int j4 = (t + 1) / 4; j4 < SW_COLS / 4; ++j4) {
-        const float4 u = urow[j4];
-        if (4 * j4 + 0 > t) w[4 * j4 + 0] = fmaf(-eo, u.x, w[4 * j4 + 0]);
-        if (4 * j4 + 1 > t) w[4 * j4 + 1] = fmaf(-eo, u.y, w[4 * j4 + 1]);
-        if (4 * j4 + 2 > t) w[4 * j4 + 2] = fmaf(-eo, u.z, w[4 * j4 + 2]);
-        w[4 * j4 + 3] = fmaf(-eo, u.w, w[4 * j4 + 3]);
-      }
-    }
-    // the chunk's 16 errors reach the row's later lanes in one batch:
-    // w[j] -= sum_t e_t U[16c + t][j] for the columns j of lanes l8 > c
-    if (c + 1 < SW_LANES) {
-      const bool later = l8 > c;
-#pragma unroll
-      for (int t = 0; t < SW_COLS; ++t) {
-        const float eb = __shfl_sync(0xffffffffu, ec[t], gbase + c);
-        const float e = later ? eb : 0.0f;
-        const float4* urow = reinterpret_cast<const float4*>(useg + t * SW_ULD);
-#pragma unroll
-        for (int j4 = 0; j4 < SW_COLS / 4; ++j4) {
+        for (int j4 = (t + 1) / 4; j4 < SW_CH / 4; ++j4) {
           const float4 u = urow[j4];
-          w[4 * j4 + 0] = fmaf(-e, u.x, w[4 * j4 + 0]);
-          w[4 * j4 + 1] = fmaf(-e, u.y, w[4 * j4 + 1]);
-          w[4 * j4 + 2] = fmaf(-e, u.z, w[4 * j4 + 2]);
+          if (4 * j4 + 0 > t) w[4 * j4 + 0] = fmaf(-e, u.x, w[4 * j4 + 0]);
+          if (4 * j4 + 1 > t) w[4 * j4 + 1] = fmaf(-e, u.y, w[4 * j4 + 1]);
+          if (4 * j4 + 2 > t) w[4 * j4 + 2] = fmaf(-e, u.z, w[4 * j4 + 2]);
           w[4 * j4 + 3] = fmaf(-e, u.w, w[4 * j4 + 3]);
         }
       }
-    }
-  }
-
-  griddep_launch_dependents();
-  // errors of this lane's 16 columns (hi/lo for the tensor-core update, or fp32)
-  if (valid) {
-    const size_t eo = static_cast<size_t>(rr) * a.ld_err + a.err_col0 + SW_COLS * l8;
-    float4* ep = reinterpret_cast<float4*>(a.Err + eo);
-    if (a.Err_lo) {
-      float4* lp = reinterpret_cast<float4*>(a.Err_lo + eo);
 #pragma unroll
-      for (int j4 = 0; j4 < SW_COLS / 4; ++j4) {
-        float hi[4], lo[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          hi[e] = tf32_round(myerr[4 * j4 + e]);
-          lo[e] = tf32_round(myerr[4 * j4 + e] - hi[e]);
-        }
-        ep[j4] = make_float4(hi[0], hi[1], hi[2], hi[3]);
-        lp[j4] = make_float4(lo[0], lo[1], lo[2], lo[3]);
+      for (int t = 0; t < SW_CH; ++t) {
+        const int i = k * SW_CH + t;
+        Es[rl * SW_ELD + i] = ep[t];
+        codes8[rl * SW_CLD + i] = static_cast<uint8_t>(static_cast<int>(qc[t] - qp.lo));
+        if (want_what) Hs[rl * SW_ELD + i] = __fmul_rn(__fsub_rn(qc[t], zs), s);
       }
-    } else {
-#pragma unroll
-      for (int j4 = 0; j4 < SW_COLS / 4; ++j4)
-        ep[j4] = make_float4(myerr[4 * j4], myerr[4 * j4 + 1], myerr[4 * j4 + 2], myerr[4 * j4 + 3]);
+      if (k + 2 < SW_NCH) named_arrive(1 + (k & 1));  // chunk k's errors are in Es
     }
-    if (a.W_hat) {
-      float* wh = a.W_hat + static_cast<size_t>(rr) * n;
+  } else {
+    // ================= updaters: chunks k+2 .. 7 -= E_k U[chunk k, .] =================
+    const int ut = tid - 32;  // 0..95
+#pragma unroll 1
+    for (int k = 0; k + 2 < SW_NCH; ++k) {
+      named_sync(1 + (k & 1));
+      const int c0 = (k + 2) * SW_CH;
+      const int n4 = (SW_B - c0) / 4;  // 4-column groups to update
+      for (int item = ut; item < SW_ROWS * n4; item += SW_THREADS - 32) {
+        const int rl = item & 31, j = c0 + 4 * (item >> 5);
+        float4 acc = *reinterpret_cast<const float4*>(Ws + rl * SW_WLD + j);
 #pragma unroll
-      for (int t = 0; t < SW_COLS; ++t) wh[perm_s[SW_COLS * l8 + t]] = mywhat[t];
+        for (int t = 0; t < SW_CH; ++t) {
+          const float e = Es[rl * SW_ELD + k * SW_CH + t];
+          const float4 u = *reinterpret_cast<const float4*>(Us + (k * SW_CH + t) * SW_B + j);
+          acc.x = fmaf(-e, u.x, acc.x);
+          acc.y = fmaf(-e, u.y, acc.y);
+          acc.z = fmaf(-e, u.z, acc.z);
+          acc.w = fmaf(-e, u.w, acc.w);
+        }
+        *reinterpret_cast<float4*>(Ws + rl * SW_WLD + j) = acc;
+      }
+      named_arrive(3 + (k & 1));
     }
   }
 
-  // pack the row's 128 codes (LSB-first bit stream): each lane ORs its 16 codes into the
-  // row's words in shared memory, then the row's lanes store the words
-  const int bits = a.bits;
-  uint32_t* rw = cw + rloc * 32;
-#pragma unroll
-  for (int t = 0; t < SW_COLS; ++t) {
-    const int pos = (SW_COLS * l8 + t) * bits;
-    const uint32_t code = mycode[t];
-    atomicOr(&rw[pos >> 5], code << (pos & 31));
-    if ((pos & 31) + bits > 32) atomicOr(&rw[(pos >> 5) + 1], code >> (32 - (pos & 31)));
+  __syncthreads();
+  // errors of the block's rows (hi/lo for the tensor-core update, or fp32), row by row
+  for (int idx = tid; idx < SW_ROWS * SW_B; idx += SW_THREADS) {
+    const int rl = idx / SW_B, j = idx % SW_B;
+    if (row0 + rl >= a.m) continue;
+    const float e = Es[rl * SW_ELD + j];
+    const size_t eo = static_cast<size_t>(row0 + rl) * a.ld_err + a.err_col0 + j;
+    if (a.Err_lo) {
+      const float hi = tf32_round(e);
+      a.Err[eo] = hi;
+      a.Err_lo[eo] = tf32_round(e - hi);
+    } else {
+      a.Err[eo] = e;
+    }
   }
-  __syncwarp();
-  if (valid) {
+  if (a.W_hat) {  // dequantized weights back to the original column order
+    for (int idx = tid; idx < SW_ROWS * SW_B; idx += SW_THREADS) {
+      const int rl = idx / SW_B, j = idx % SW_B;
+      if (row0 + rl < a.m) a.W_hat[static_cast<size_t>(row0 + rl) * n + perm_s[j]] = Hs[rl * SW_ELD + j];
+    }
+  }
+  // pack each row's 128 codes into its LSB-first bit stream: one 32-bit word per thread
+  {
+    const int bits = a.bits;
     const int words = 4 * bits;  // 128 * bits / 32
     const int ldc = n * bits / 32;
-    uint32_t* dst = a.codes + static_cast<size_t>(rr) * ldc + (i1 * bits) / 32;
-    for (int wi = l8; wi < words; wi += SW_LANES) dst[wi] = rw[wi];
+    for (int idx = tid; idx < SW_ROWS * words; idx += SW_THREADS) {
+      const int rl = idx / words, wi = idx % words;
+      if (row0 + rl >= a.m) continue;
+      const uint8_t* cr = codes8 + rl * SW_CLD;
+      const int b0 = 32 * wi;
+      uint32_t word = 0u;
+      for (int k = b0 / bits; k * bits < b0 + 32; ++k) {
+        const int pos = k * bits - b0;
+        const uint32_t code = cr[k];
+        word |= (pos >= 0) ? (code << pos) : (code >> (-pos));
+      }
+      a.codes[static_cast<size_t>(row0 + rl) * ldc + (i1 * bits) / 32 + wi] = word;
+    }
   }
 }
 

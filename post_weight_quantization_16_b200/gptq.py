@@ -57,7 +57,8 @@ _SIGS = {
     "gptq_test_gemm_tf32x3": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P, ctypes.c_int, _P, _P,
                                              ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                              ctypes.c_int, _P, ctypes.c_int, _P, _P, ctypes.c_int, _P, _P,
-                                             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _P]),
+                                             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                             _P]),
     "gptq_test_div_rn": (ctypes.c_int, [ctypes.c_uint64, ctypes.c_int64, ctypes.POINTER(ctypes.c_uint64),
                                         ctypes.POINTER(ctypes.c_float), ctypes.c_int, _P]),
 }

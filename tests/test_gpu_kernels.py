@@ -33,7 +33,7 @@ def p(t):
 
 
 def run_gemm(A, B, alpha=1.0, beta=0, C0=None, klo=0, khi=0, upper=0, plain=True, hilo=False, trans=False, chunk=1,
-             tile=0):
+             tile=0, reduce=0):
     M, K = A.shape
     N = B.shape[0]
     ah, al = split(A)
@@ -49,7 +49,7 @@ def run_gemm(A, B, alpha=1.0, beta=0, C0=None, klo=0, khi=0, upper=0, plain=True
     Cth = torch.zeros((N, M), dtype=torch.float32, device=DEV) if trans else None
     Ctl = torch.zeros((N, M), dtype=torch.float32, device=DEV) if trans else None
     st = G.lib().gptq_test_gemm_tf32x3(M, N, K, p(Ah), p(Al), K, p(Bh), p(Bl), K, float(alpha), int(beta), klo, khi,
-                                       upper, p(C), N, p(Ch), p(Cl), N, p(Cth), p(Ctl), M, chunk, tile, 0,
+                                       upper, p(C), N, p(Ch), p(Cl), N, p(Cth), p(Ctl), M, chunk, tile, reduce, 0,
                                        ctypes.c_void_p(torch.cuda.current_stream(DEV).cuda_stream))
     assert st == G.OK, G.STATUS.get(st)
     out = {}
@@ -122,6 +122,30 @@ def test_gemm_upper_only_updates_upper_triangle(tile):
     iu = np.triu_indices(n)
     err = np.abs(out["Chilo"][iu] - R[iu]) / scale[iu]
     assert err.max() <= 2e-6
+
+
+@pytest.mark.parametrize("M,N,K,chunk", [(4096, 896, 128, 4), (300, 320, 1024, 4), (128, 64, 32, 1), (1000, 3072, 256, 4)])
+@pytest.mark.parametrize("tile", [64, 128, 256])
+def test_gemm_reduce_add_epilogue(M, N, K, chunk, tile):
+    """C += alpha A B^T through TMA reduce-add boxes: equals the fp64 result, and C's columns
+    right of the product (inside the same allocation) are untouched."""
+    r = np.random.default_rng(M + N + K + tile)
+    A = r.standard_normal((M, K)).astype(np.float32)
+    B = r.standard_normal((N, K)).astype(np.float32)
+    pad = 96  # C lives in a wider matrix: the product covers its first N columns
+    C0 = r.standard_normal((M, N + pad)).astype(np.float32)
+    ah, al = split(A)
+    bh, bl = split(B)
+    Ah, Al, Bh, Bl = dev(ah), dev(al), dev(bh), dev(bl)
+    C = dev(C0)
+    st = G.lib().gptq_test_gemm_tf32x3(M, N, K, p(Ah), p(Al), K, p(Bh), p(Bl), K, -1.0, 1, 0, 0, 0, p(C), N + pad,
+                                       None, None, 0, None, None, 0, chunk, tile, 1, 0,
+                                       ctypes.c_void_p(torch.cuda.current_stream(DEV).cuda_stream))
+    assert st == G.OK, G.STATUS.get(st)
+    got = C.cpu().numpy().astype(np.float64)
+    R, scale = ref(A, B, -1.0, 1, C0[:, :N])
+    assert (np.abs(got[:, :N] - R) / scale).max() <= 2e-6
+    assert np.array_equal(got[:, N:], C0[:, N:].astype(np.float64))
 
 
 def test_sweep_division_equals_ieee_division():
