@@ -21,7 +21,7 @@ constexpr int LF_NB = 128;     // leaf block
 constexpr int LF_P = 32;       // panel width (one warp)
 constexpr int LF_THREADS = 256;
 constexpr int LF_LD = LF_NB + 1;
-constexpr int LF_SMEM = 3 * LF_NB * LF_LD * 4 + 16;
+constexpr int LF_SMEM = 3 * LF_NB * LF_LD * 4 + LF_NB * 4 + 16;  // S, V, X, 1/V[c][c], flag
 static_assert(LF_NB * LF_NB <= LF_NB * LF_LD, "a staged block must fit in V (and in X)");
 
 __device__ __forceinline__ float tf32_round(float x) {
@@ -30,53 +30,129 @@ __device__ __forceinline__ float tf32_round(float x) {
   return __uint_as_float(u & 0xFFFFE000u);
 }
 
-// Warp 0: UL Cholesky of the 32 x 32 block S[P0.., P0..] (upper triangle) into V, and its
-// inverse X = V^-1 in the same sweep.  Lane i holds row i of the block in registers
-// (columns are broadcast with shuffles) and column i of the inverse.  Step c produces
-// column c of V and row c of X: X[c][c] = 1/V[c][c], X[c][j] = -(sum_{c<l<=j} V[c][l] X[l][j]) / V[c][c];
-// the inverse row uses only earlier steps' results, so it fills the latency of the pivot chain.
-__device__ __forceinline__ void leaf_diag_factor(float (*S)[LF_LD], float (*V)[LF_LD], float (*X)[LF_LD], int P0,
-                                                 int lane, int* bad) {
-  float d[LF_P], x[LF_P];
+// Warp 0: one 32-column panel of the UL Cholesky, P0 = 32 p.  Lane l carries row P0 + l of
+// the diagonal block (and, for NR > 0, row 32 r + l of block row r < NR above it) in
+// registers; step c (from the panel's last column down) produces column P0 + c of V for
+// those rows, eliminating it from the panel's earlier columns:
+//   V[c][c] = sqrt(S[c][c]),   V[i][c] = S[i][c] / V[c][c],   S[i][j] -= V[i][c] V[j][c].
+// The pivot chain is kept short: lane c-1's diagonal after column c is its own column value
+// squared off its diagonal, so the next pivot is broadcast without waiting for the column
+// broadcast.  1 / V[c][c] goes to rsv for the inverse of the diagonal block.
+template <int NR>
+__device__ __forceinline__ void leaf_sweep(float (*S)[LF_LD], float (*V)[LF_LD], float* rsv, int P0, int lane,
+                                           int* bad) {
+  float d[NR + 1][LF_P];
 #pragma unroll
   for (int j = 0; j < LF_P; ++j) {
-    d[j] = S[P0 + lane][P0 + j];
-    x[j] = 0.0f;
+    d[0][j] = S[P0 + lane][P0 + j];
+#pragma unroll
+    for (int r = 0; r < NR; ++r) d[r + 1][j] = S[LF_P * r + lane][P0 + j];
   }
+  float pnext = __shfl_sync(0xffffffffu, d[0][LF_P - 1], LF_P - 1);
 #pragma unroll
   for (int c = LF_P - 1; c >= 0; --c) {
-    float piv = __shfl_sync(0xffffffffu, d[c], c);
+    float piv = pnext;
     if (!(piv > 0.0f) || !isfinite(piv)) {
       if (lane == 0) *bad = 1;
       piv = 1.0f;
     }
     const float rs = rsqrtf(piv);  // 1 / V[c][c]
     const float sv = piv * rs;     // V[c][c]
-    const float col = (lane < c) ? d[c] * rs : (lane == c ? sv : 0.0f);
-    d[c] = col;
-    V[P0 + lane][P0 + c] = col;
+    float col[NR + 1];
+    col[0] = (lane < c) ? d[0][c] * rs : (lane == c ? sv : 0.0f);
 #pragma unroll
-    for (int j = c - 1; j >= 0; --j) {  // the next pivot column first: it is on the critical path
-      const float cj = __shfl_sync(0xffffffffu, col, j);
-      d[j] = fmaf(-col, cj, d[j]);
+    for (int r = 0; r < NR; ++r) col[r + 1] = d[r + 1][c] * rs;
+    if (c > 0) pnext = __shfl_sync(0xffffffffu, fmaf(-col[0], col[0], d[0][c - 1]), c - 1);
+    V[P0 + lane][P0 + c] = col[0];
+#pragma unroll
+    for (int r = 0; r < NR; ++r) V[LF_P * r + lane][P0 + c] = col[r + 1];
+    if (lane == 0) rsv[P0 + c] = rs;
+#pragma unroll
+    for (int j = c - 1; j >= 0; --j) {
+      const float cj = __shfl_sync(0xffffffffu, col[0], j);  // V[P0 + j][P0 + c]
+#pragma unroll
+      for (int r = 0; r <= NR; ++r) d[r][j] = fmaf(-col[r], cj, d[r][j]);
     }
-    // row c of the inverse (V[c][l] for l > c were written by earlier steps)
-    __syncwarp();
+  }
+  __syncwarp();
+}
+
+// One warp, lane l: row 32 r + l above diagonal block P0 (r < P0 / 32), its panel-p part
+// from the block's factor (V's diagonal block and 1 / V[c][c] in shared memory):
+//   V[i][P0+c] = (S[i][P0+c] - sum_{k>c} V[i][P0+k] V[P0+c][P0+k]) / V[c][c],  c from the last.
+// Every lane reads the same V entries (broadcast) and works on its own row.
+__device__ __forceinline__ void leaf_rows_above(float (*S)[LF_LD], float (*V)[LF_LD], const float* rsv, int P0,
+                                                int row) {
+  float d[LF_P];
+#pragma unroll
+  for (int j = 0; j < LF_P; ++j) d[j] = S[row][P0 + j];
+#pragma unroll
+  for (int c = LF_P - 1; c >= 0; --c) {
+    const float col = d[c] * rsv[P0 + c];
+    V[row][P0 + c] = col;
+#pragma unroll
+    for (int j = c - 1; j >= 0; --j) d[j] = fmaf(-col, V[P0 + j][P0 + c], d[j]);
+  }
+}
+
+// One warp: the inverse X = V^-1 of diagonal block P0 (upper, 32 x 32), lane j holding column
+// j: X[c][c] = 1/V[c][c], X[c][j] = -(sum_{c<l<=j} V[c][l] X[l][j]) / V[c][c], rows from the
+// last up.  Written to X's diagonal block (zeros below the diagonal).
+__device__ __forceinline__ void leaf_inv_diag(const float (*V)[LF_LD], float (*X)[LF_LD], const float* rsv, int P0,
+                                              int lane) {
+  float x[LF_P];
+#pragma unroll
+  for (int c = LF_P - 1; c >= 0; --c) {
     float acc4[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // four partial sums: a short dependent chain
 #pragma unroll
     for (int l = c + 1; l < LF_P; ++l) acc4[l & 3] = fmaf(V[P0 + c][P0 + l], x[l], acc4[l & 3]);
     const float acc = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
+    const float rs = rsv[P0 + c];
     x[c] = (lane == c) ? rs : (lane > c ? -acc * rs : 0.0f);
   }
 #pragma unroll
   for (int r = 0; r < LF_P; ++r) X[P0 + r][P0 + lane] = x[r];
-  __syncwarp();
+}
+
+// 4 x 4 tile of C[i0.., j0..] = sum_k P[i0 + a][k] Q[j0 + b][k] over k in [k0, k1), rows of
+// P and Q in shared memory at pitch LF_LD.
+__device__ __forceinline__ void lf_tile_nt(const float (*P)[LF_LD], const float (*Q)[LF_LD], int i0, int j0, int k0,
+                                           int k1, float (&acc)[4][4]) {
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
+#pragma unroll 4
+  for (int k = k0; k < k1; ++k) {
+    float pv[4], qv[4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      pv[a] = P[i0 + a][k];
+      qv[a] = Q[j0 + a][k];
+    }
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(pv[a], qv[b], acc[a][b]);
+  }
+}
+
+__device__ __forceinline__ void lf_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // Leaf: U_kk (= V_kk^-1, V_kk V_kk^T = A_kk) for the diagonal block at offset o, read from
 // the upper triangle of A = A_hi + A_lo.  Writes U (upper, zeros below) and Ut = U^T as
 // hi/lo pairs.  A non-positive or non-finite pivot sets ST_NOT_PD (and is replaced by 1
 // so the kernel still finishes with finite work).
+//
+// Reverse right-looking Cholesky over four 32-column panels, bottom-right first.  The chain
+// from one panel to the next is kept short: warp 0 factors diagonal block p in registers,
+// warps 1 .. p solve the rows above it (one row a lane) while warp 5 inverts the diagonal
+// block, all warps update column block p-1 (lookahead), and warp 0 goes on to block p-1
+// while the six warps 1-3, 5-7 finish the trailing update and form block row p of the
+// inverse U = V^-1:
+//   U_pj = -Xd_p * sum_{l=p+1..j} V_pl U_lj      (Xd_p = the diagonal block's inverse).
 __global__ void __launch_bounds__(LF_THREADS, 1)
     leaf_chol_inv_kernel(const float* __restrict__ A_hi, const float* __restrict__ A_lo, int n, int o,
                          float* __restrict__ U_hi, float* __restrict__ U_lo, float* __restrict__ Ut_hi,
@@ -85,7 +161,7 @@ __global__ void __launch_bounds__(LF_THREADS, 1)
   float(*S)[LF_LD] = reinterpret_cast<float(*)[LF_LD]>(lf_smem);
   float(*V)[LF_LD] = reinterpret_cast<float(*)[LF_LD]>(lf_smem + LF_NB * LF_LD);
   float(*X)[LF_LD] = reinterpret_cast<float(*)[LF_LD]>(lf_smem + 2 * LF_NB * LF_LD);
-  int* bad = reinterpret_cast<int*>(lf_smem + 3 * LF_NB * LF_LD);
+  int* bad = reinterpret_cast<int*>(lf_smem + 3 * LF_NB * LF_LD + LF_NB);  // after rsv
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   griddep_wait();
   griddep_launch_dependents();  // one CTA: the next kernel may take the other SMs right away
@@ -109,176 +185,126 @@ __global__ void __launch_bounds__(LF_THREADS, 1)
       const float v = th[i * LF_NB + j] + tl[i * LF_NB + j];
       S[i][j] = (i <= j) ? v : 0.0f;
     }
-    __syncthreads();
-    for (int idx = tid; idx < LF_NB * LF_LD; idx += LF_THREADS) {
-      (&V[0][0])[idx] = 0.0f;
-      (&X[0][0])[idx] = 0.0f;
-    }
   }
   __syncthreads();
+  // (every entry of V and X that is read below is written first: no clearing needed)
 
-  // ---- reverse right-looking Cholesky, 32-column panels from the bottom-right ----
-  // Lookahead: after the panel solve, warp 0 updates the next diagonal block itself and goes
-  // straight on to factor it, while warps 1-3 and 5-7 (warp 4 shares warp 0's scheduler)
-  // update the rest of the trailing triangle.
+  float* rsv = &X[0][0] + LF_NB * LF_LD;  // [128] 1 / V[c][c]
+  // the six warps 1-3, 5-7 (warp 4 shares warp 0's scheduler and stays out of its way)
+  const bool g1 = (warp != 0 && warp != 4);
+  const int t1 = tid - 32 * ((warp > 0) + (warp > 4));  // 0..191 within the six warps
+  constexpr int NG1 = LF_THREADS - 64;
+
+#pragma unroll 1
   for (int p = LF_NB / LF_P - 1; p >= 0; --p) {
     const int P0 = p * LF_P;
-    if (warp == 0) leaf_diag_factor(S, V, X, P0, lane, bad);
-    __syncthreads();
-    // panel: V[i][P0+c] = sum_k S[i][P0+k] * Xd[c][k]   for rows i < P0 (Xd upper: zero for k < c);
-    // one 4 x 4 tile of (rows, panel columns) per thread
-    for (int item = tid; item < (P0 / 4) * (LF_P / 4); item += LF_THREADS) {
-      const int i0 = (item / (LF_P / 4)) * 4, c0 = (item % (LF_P / 4)) * 4;
-      float acc[4][4];
-#pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
-#pragma unroll 8
-      for (int k = 0; k < LF_P; ++k) {
-        float sv[4], xv[4];
-#pragma unroll
-        for (int a = 0; a < 4; ++a) {
-          sv[a] = S[i0 + a][P0 + k];
-          xv[a] = X[P0 + c0 + a][P0 + k];
-        }
+    // panel p: the diagonal block (warp 0, the chain), then the rows above it (warps 1 .. p,
+    // one row a lane) while warp 5 inverts the diagonal block
+    if (warp == 0) leaf_sweep<0>(S, V, rsv, P0, lane, bad);
+    __syncthreads();  // diagonal block p in V; the six warps' work of the step before is done
+    if (warp >= 1 && warp <= p) leaf_rows_above(S, V, rsv, P0, LF_P * (warp - 1) + lane);
+    if (warp == 5) leaf_inv_diag(V, X, rsv, P0, lane);  // Xd_p
+    __syncthreads();  // panel p in V for every row; Xd_p in X
+    if (p > 0) {
+      // lookahead: column block p-1 of the trailing update, all warps
+      //   S[i][j] -= sum_c V[i][P0+c] V[j][P0+c],  j in [P0-32, P0), i <= j
+      const int nrt = P0 / 4;  // row tiles 0 .. nrt-1; column tiles of block p-1: 8
+      for (int t = tid; t < nrt * 8; t += LF_THREADS) {
+        const int bi = t / 8, bj = (P0 - LF_P) / 4 + t % 8;
+        if (bi > bj) continue;
+        const int i0 = 4 * bi, j0 = 4 * bj;
+        float acc[4][4];
+        lf_tile_nt(V, V, i0, j0, P0, P0 + LF_P, acc);
 #pragma unroll
         for (int a = 0; a < 4; ++a)
 #pragma unroll
-          for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(sv[a], xv[b], acc[a][b]);
+          for (int b = 0; b < 4; ++b)
+            if (i0 + a <= j0 + b) S[i0 + a][j0 + b] -= acc[a][b];
       }
-#pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) V[i0 + a][P0 + c0 + b] = acc[a][b];
+      __syncthreads();  // column block p-1 is up to date: warp 0 may factor it
     }
-    __syncthreads();
-    if (p == 0) break;
-    // trailing update of the upper triangle: S[i][j] -= sum_c V[i][P0+c] V[j][P0+c], i <= j < P0,
-    // in 4 x 4 tiles (bi <= bj); the tiles of the next diagonal block go to warp 0
-    const int nb = P0 / 4, nd = LF_P / 4, d0 = nb - nd;  // next diagonal block = tile rows/cols [d0, nb)
-    int t_begin, t_step, t_end;
-    if (warp == 0 || warp == 4) {  // the two warps of scheduler 0 update the next diagonal block
-      t_begin = (warp == 4 ? 32 : 0) + lane;
-      t_step = 64;
-      t_end = nd * (nd + 1) / 2;  // tiles inside the next diagonal block
-    } else {
-      const int wi = (warp < 4) ? warp - 1 : warp - 2;  // 0..5
-      t_begin = wi * 32 + lane;
-      t_step = 6 * 32;
-      t_end = nb * (nb + 1) / 2 - nd * (nd + 1) / 2;  // all other tiles
-    }
-    for (int t = t_begin; t < t_end; t += t_step) {
-      int bi, bj;
-      if (warp == 0 || warp == 4) {  // enumerate the upper tiles of the next diagonal block
-        int jj = static_cast<int>((sqrtf(8.0f * t + 1.0f) - 1.0f) * 0.5f);
-        while (jj * (jj + 1) / 2 > t) --jj;
-        while ((jj + 1) * (jj + 2) / 2 <= t) ++jj;
-        bi = d0 + (t - jj * (jj + 1) / 2);
-        bj = d0 + jj;
-      } else {  // enumerate all upper tiles with bj < d0, then the block column bi < d0 <= bj
-        const int na = d0 * (d0 + 1) / 2;
-        if (t < na) {
-          int jj = static_cast<int>((sqrtf(8.0f * t + 1.0f) - 1.0f) * 0.5f);
-          while (jj * (jj + 1) / 2 > t) --jj;
-          while ((jj + 1) * (jj + 2) / 2 <= t) ++jj;
-          bi = t - jj * (jj + 1) / 2;
-          bj = jj;
-        } else {
-          const int u = t - na;
-          bi = u / nd;
-          bj = d0 + u % nd;
+    if (g1) {
+      {
+        // the rest of the trailing update: S[i][j] -= sum_c V[i][P0+c] V[j][P0+c], i <= j < P0-32
+        const int nb2 = (P0 - LF_P) / 4;
+        const int ntiles = nb2 > 0 ? nb2 * (nb2 + 1) / 2 : 0;
+        for (int t = t1; t < ntiles; t += NG1) {
+          int bj = 0, tt = t;
+          while (tt > bj) {
+            tt -= bj + 1;
+            ++bj;
+          }
+          const int i0 = 4 * tt, j0 = 4 * bj;
+          float acc[4][4];
+          lf_tile_nt(V, V, i0, j0, P0, P0 + LF_P, acc);
+#pragma unroll
+          for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+              if (i0 + a <= j0 + b) S[i0 + a][j0 + b] -= acc[a][b];
         }
       }
-      const int i0 = 4 * bi, j0 = 4 * bj;
-      float acc[4][4];
+      // block row p of the inverse, right of the diagonal block:
+      //   U_pj = -Xd_p * sum_{l=p+1..j} V_pl U_lj
+      // (S's block row p right of its diagonal block is no longer needed and holds T)
+      const int ncols = LF_NB - P0 - LF_P;
+      if (ncols > 0) {
+        const int nct = ncols / 4;
+        // T[r][col] = sum_{k >= P0+32} V[P0+r][k] X[k][col]   (X upper: k <= col)
+        for (int item = t1; item < (LF_P / 4) * nct; item += NG1) {
+          const int r0 = (item / nct) * 4, col0 = P0 + LF_P + (item % nct) * 4;
+          float acc[4][4];
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
+          for (int a = 0; a < 4; ++a)
 #pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
-#pragma unroll 4
-      for (int c = 0; c < LF_P; ++c) {
-        float vi[4], vj[4];
+            for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
+          for (int k = P0 + LF_P; k < col0 + 4; ++k) {
+            float vv[4], xv[4];
 #pragma unroll
-        for (int a = 0; a < 4; ++a) {
-          vi[a] = V[i0 + a][P0 + c];
-          vj[a] = V[j0 + a][P0 + c];
+            for (int a = 0; a < 4; ++a) {
+              vv[a] = V[P0 + r0 + a][k];
+              xv[a] = X[k][col0 + a];
+            }
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+              for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(vv[a], xv[b], acc[a][b]);
+          }
+#pragma unroll
+          for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) S[P0 + r0 + a][col0 + b] = acc[a][b];
         }
+        lf_bar_sync(3, NG1);
+        // X[P0+r][col] = -sum_{k >= r} Xd[r][k] T[k][col]
+        for (int item = t1; item < (LF_P / 4) * nct; item += NG1) {
+          const int r0 = (item / nct) * 4, col0 = P0 + LF_P + (item % nct) * 4;
+          float acc[4][4];
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+          for (int a = 0; a < 4; ++a)
 #pragma unroll
-          for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(vi[a], vj[b], acc[a][b]);
+            for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
+          for (int k = r0; k < LF_P; ++k) {
+            float xd[4], tv[4];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+              xd[a] = X[P0 + r0 + a][P0 + k];
+              tv[a] = S[P0 + k][col0 + a];
+            }
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+              for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(xd[a], tv[b], acc[a][b]);
+          }
+#pragma unroll
+          for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) X[P0 + r0 + a][col0 + b] = -acc[a][b];
+        }
       }
-#pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b)
-          if (i0 + a <= j0 + b) S[i0 + a][j0 + b] -= acc[a][b];
     }
-    if (warp == 0 || warp == 4) asm volatile("bar.sync 1, 64;" ::: "memory");  // next block updated
   }
   __syncthreads();
-
-  // ---- U = V^-1: diagonal 32-blocks are in X; off-diagonal blocks by block rows ----
-  //   U_ij = -Xd_i * sum_{l=i+1..j} V_il U_lj      (block row i from the bottom)
-  for (int bi = LF_NB / LF_P - 2; bi >= 0; --bi) {
-    const int I0 = bi * LF_P;
-    const int ncols = LF_NB - I0 - LF_P;  // columns right of the diagonal block
-    // T[r][col] = sum_{k >= I0+32} V[I0+r][k] X[k][col]  -> stored in S (free now);
-    // one 4 x 4 tile per thread; X is upper, so X[k][col0..col0+3] = 0 for k > col0 + 3
-    const int nct = ncols / 4;
-    for (int item = tid; item < (LF_P / 4) * nct; item += LF_THREADS) {
-      const int r0 = (item / nct) * 4, col0 = I0 + LF_P + (item % nct) * 4;
-      float acc[4][4];
-#pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
-      for (int k = I0 + LF_P; k < col0 + 4; ++k) {
-        float vv[4], xv[4];
-#pragma unroll
-        for (int a = 0; a < 4; ++a) {
-          vv[a] = V[I0 + r0 + a][k];
-          xv[a] = X[k][col0 + a];
-        }
-#pragma unroll
-        for (int a = 0; a < 4; ++a)
-#pragma unroll
-          for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(vv[a], xv[b], acc[a][b]);
-      }
-#pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) S[I0 + r0 + a][col0 + b] = acc[a][b];
-    }
-    __syncthreads();
-    // X[I0+r][col] = -sum_{k >= r} Xd[r][k] T[k][col]      (Xd upper: zero for k < r)
-    for (int item = tid; item < (LF_P / 4) * nct; item += LF_THREADS) {
-      const int r0 = (item / nct) * 4, col0 = I0 + LF_P + (item % nct) * 4;
-      float acc[4][4];
-#pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
-      for (int k = r0; k < LF_P; ++k) {
-        float xd[4], tv[4];
-#pragma unroll
-        for (int a = 0; a < 4; ++a) {
-          xd[a] = X[I0 + r0 + a][I0 + k];
-          tv[a] = S[I0 + k][col0 + a];
-        }
-#pragma unroll
-        for (int a = 0; a < 4; ++a)
-#pragma unroll
-          for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(xd[a], tv[b], acc[a][b]);
-      }
-#pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) X[I0 + r0 + a][col0 + b] = -acc[a][b];
-    }
-    __syncthreads();
-  }
 
   // ---- write U (hi/lo) and Ut = U^T (hi/lo), 16-byte stores ----
   for (int idx = tid; idx < LF_NB * (LF_NB / 4); idx += LF_THREADS) {
