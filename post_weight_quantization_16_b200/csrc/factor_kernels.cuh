@@ -141,9 +141,28 @@ __device__ __forceinline__ void lf_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// Rows [R0, R0 + 32) of U = X (zeros left of the diagonal) as a hi/lo pair, 16-byte stores,
+// by threads t = 0 .. nt-1.  (U^T is formed off the critical path.)
+__device__ __forceinline__ void leaf_store_rows(const float (*X)[LF_LD], float* __restrict__ U_hi,
+                                                float* __restrict__ U_lo, int n, int o, int R0, int t, int nt) {
+  for (int idx = t; idx < LF_P * (LF_NB / 4); idx += nt) {
+    const int i = R0 + idx / (LF_NB / 4), j = (idx % (LF_NB / 4)) * 4;
+    float uh[4], ul[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float u = (i <= j + e) ? X[i][j + e] : 0.0f;  // U[i][j+e]
+      uh[e] = tf32_round(u);
+      ul[e] = tf32_round(u - uh[e]);
+    }
+    const size_t g = static_cast<size_t>(o + i) * n + o + j;
+    *reinterpret_cast<float4*>(U_hi + g) = make_float4(uh[0], uh[1], uh[2], uh[3]);
+    *reinterpret_cast<float4*>(U_lo + g) = make_float4(ul[0], ul[1], ul[2], ul[3]);
+  }
+}
+
 // Leaf: U_kk (= V_kk^-1, V_kk V_kk^T = A_kk) for the diagonal block at offset o, read from
-// the upper triangle of A = A_hi + A_lo.  Writes U (upper, zeros below) and Ut = U^T as
-// hi/lo pairs.  A non-positive or non-finite pivot sets ST_NOT_PD (and is replaced by 1
+// the upper triangle of A = A_hi + A_lo.  Writes U (upper, zeros below) as a hi/lo pair
+// (transpose_block_kernel forms U^T on the graph's second branch).  A non-positive or non-finite pivot sets ST_NOT_PD (and is replaced by 1
 // so the kernel still finishes with finite work).
 //
 // Reverse right-looking Cholesky over four 32-column panels, bottom-right first.  The chain
@@ -155,8 +174,7 @@ __device__ __forceinline__ void lf_bar_sync(int id, int count) {
 //   U_pj = -Xd_p * sum_{l=p+1..j} V_pl U_lj      (Xd_p = the diagonal block's inverse).
 __global__ void __launch_bounds__(LF_THREADS, 1)
     leaf_chol_inv_kernel(const float* __restrict__ A_hi, const float* __restrict__ A_lo, int n, int o,
-                         float* __restrict__ U_hi, float* __restrict__ U_lo, float* __restrict__ Ut_hi,
-                         float* __restrict__ Ut_lo, int* __restrict__ status) {
+                         float* __restrict__ U_hi, float* __restrict__ U_lo, int* __restrict__ status) {
   extern __shared__ float lf_smem[];
   float(*S)[LF_LD] = reinterpret_cast<float(*)[LF_LD]>(lf_smem);
   float(*V)[LF_LD] = reinterpret_cast<float(*)[LF_LD]>(lf_smem + LF_NB * LF_LD);
@@ -223,6 +241,8 @@ __global__ void __launch_bounds__(LF_THREADS, 1)
       }
       __syncthreads();  // column block p-1 is up to date: warp 0 may factor it
     }
+    // block row p+1 of U is final (since the last step): warp 4, otherwise idle here, writes it
+    if (warp == 4 && p + 1 < LF_NB / LF_P) leaf_store_rows(X, U_hi, U_lo, n, o, (p + 1) * LF_P, lane, 32);
     if (g1) {
       {
         // the rest of the trailing update: S[i][j] -= sum_c V[i][P0+c] V[j][P0+c], i <= j < P0-32
@@ -306,30 +326,34 @@ __global__ void __launch_bounds__(LF_THREADS, 1)
   }
   __syncthreads();
 
-  // ---- write U (hi/lo) and Ut = U^T (hi/lo), 16-byte stores ----
-  for (int idx = tid; idx < LF_NB * (LF_NB / 4); idx += LF_THREADS) {
-    const int i = idx / (LF_NB / 4), j = (idx % (LF_NB / 4)) * 4;
-    float u[4], ut[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      u[e] = (i <= j + e) ? X[i][j + e] : 0.0f;   // U[i][j+e]
-      ut[e] = (j + e <= i) ? X[j + e][i] : 0.0f;  // Ut[i][j+e] = U[j+e][i]
-    }
-    float uh[4], ul[4], th[4], tl[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      uh[e] = tf32_round(u[e]);
-      ul[e] = tf32_round(u[e] - uh[e]);
-      th[e] = tf32_round(ut[e]);
-      tl[e] = tf32_round(ut[e] - th[e]);
-    }
-    const size_t g = static_cast<size_t>(o + i) * n + o + j;
-    *reinterpret_cast<float4*>(U_hi + g) = make_float4(uh[0], uh[1], uh[2], uh[3]);
-    *reinterpret_cast<float4*>(U_lo + g) = make_float4(ul[0], ul[1], ul[2], ul[3]);
-    *reinterpret_cast<float4*>(Ut_hi + g) = make_float4(th[0], th[1], th[2], th[3]);
-    *reinterpret_cast<float4*>(Ut_lo + g) = make_float4(tl[0], tl[1], tl[2], tl[3]);
-  }
+  // block row 0 of U (the others went out during the factorization)
+  leaf_store_rows(X, U_hi, U_lo, n, o, 0, tid, LF_THREADS);
   if (tid == 0 && *bad) atomicOr(status, ST_NOT_PD);
+}
+
+// U^T of one 128 x 128 diagonal block (hi and lo), 32 x 32 tiles through shared memory:
+// Ut[o + c][o + r] = U[o + r][o + c].  Grid (4, 4), block (32, 8).
+__global__ void __launch_bounds__(256) transpose_block_kernel(const float* __restrict__ U_hi,
+                                                              const float* __restrict__ U_lo, int n, int o,
+                                                              float* __restrict__ Ut_hi, float* __restrict__ Ut_lo) {
+  __shared__ float th[32][33], tl[32][33];
+  griddep_wait();
+  griddep_launch_dependents();
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  const int r0 = o + blockIdx.y * 32, c0 = o + blockIdx.x * 32;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const size_t g = static_cast<size_t>(r0 + ty + 8 * k) * n + c0 + tx;
+    th[ty + 8 * k][tx] = U_hi[g];
+    tl[ty + 8 * k][tx] = U_lo[g];
+  }
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const size_t g = static_cast<size_t>(c0 + ty + 8 * k) * n + r0 + tx;
+    Ut_hi[g] = th[tx][ty + 8 * k];
+    Ut_lo[g] = tl[tx][ty + 8 * k];
+  }
 }
 
 }  // namespace gptq

@@ -325,9 +325,27 @@ gptq_status gemm_tc(gptq_ctx* c, int M, int N, int K, TcOperand A, TcOperand B, 
 gptq_status chol_inv(gptq_ctx* c, int o, int h) {
   const int n = static_cast<int>(c->n);
   if (h <= LF_NB) {
-    CK(launch(c, leaf_chol_inv_kernel, dim3(1), dim3(LF_THREADS), LF_SMEM, c->A_hi, c->A_lo, n, o, c->U_hi, c->U_lo, c->Ut_hi,
-                                                               c->Ut_lo, c->status));
+    CK(launch(c, leaf_chol_inv_kernel, dim3(1), dim3(LF_THREADS), LF_SMEM, c->A_hi, c->A_lo, n, o, c->U_hi, c->U_lo,
+              c->status));
     CKL("leaf_chol_inv");
+    // U^T of the block, needed only by later T products and the sweep's trailing update: on
+    // the second branch while it exists (the factorization graph), in line otherwise
+    const bool branch = c->side_stream != nullptr;
+    cudaStream_t main_stream = c->stream;
+    if (branch) {
+      CK(cudaEventRecord(c->ev_fork, main_stream));
+      CK(cudaStreamWaitEvent(c->side_stream, c->ev_fork, 0));
+      c->stream = c->side_stream;
+      c->pdl = false;
+    }
+    const cudaError_t e = launch(c, transpose_block_kernel, dim3(4, 4), dim3(32, 8), 0, c->U_hi, c->U_lo, n, o,
+                                 c->Ut_hi, c->Ut_lo);
+    if (branch) {
+      c->stream = main_stream;
+      c->pdl = true;
+    }
+    CK(e);
+    CKL("transpose_block");
     return GPTQ_OK;
   }
   const int h2 = ((h / LF_NB) / 2) * LF_NB;
@@ -434,6 +452,11 @@ gptq_status run_factorization(gptq_ctx* c) {
     c->stream = c->capture_stream;
     CK(cudaStreamBeginCapture(c->capture_stream, cudaStreamCaptureModeThreadLocal));
     gptq_status s = chol_inv(c, 0, static_cast<int>(c->n));
+    if (s == GPTQ_OK) {  // join the second branch (the last block's U^T)
+      cudaError_t e1 = cudaEventRecord(c->ev_join, c->side_stream);
+      if (e1 == cudaSuccess) e1 = cudaStreamWaitEvent(c->capture_stream, c->ev_join, 0);
+      if (e1 != cudaSuccess) s = cuda_fail(e1, "join");
+    }
     cudaGraph_t g = nullptr;
     cudaError_t e = cudaStreamEndCapture(c->capture_stream, &g);
     c->stream = user;
