@@ -89,33 +89,54 @@ __host__ __device__ inline int gt_num_tiles(int M, int N, int upper_only, int bn
   return c;
 }
 
-// Tile t (n-tiles fastest, or with upper_only column by column over the needed tiles).
-template <int BN>
-__device__ __forceinline__ void gt_tile(const GemmTCArgs& p, int t, int& m0, int& n0, int& k_begin, int& n_iters) {
-  const int mtn = (p.M + GT_BM - 1) / GT_BM, ntn = (p.N + BN - 1) / BN;
-  if (!p.upper_only) {
-    m0 = (t / ntn) * GT_BM;
-    n0 = (t % ntn) * BN;
+// Tile t of a product.  Tiles are numbered in order of decreasing K range where the operands
+// are triangular (K from the tile's first column: columns ascending; K up to its last column:
+// columns descending; K from its first row, or full K: rows ascending), so that the snake
+// assignment below pairs long tiles with short ones; with upper_only, column by column over
+// the needed tiles (all of full K).
+__host__ __device__ inline void gt_tile_at(int M, int N, int K, int k_lo_mode, int k_hi_mode, int upper_only, int bn,
+                                           int t, int& m0, int& n0, int& k_begin, int& n_iters) {
+  const int mtn = (M + GT_BM - 1) / GT_BM, ntn = (N + bn - 1) / bn;
+  if (!upper_only) {
+    if (k_lo_mode == GT_KLO_COL) {
+      n0 = (t / mtn) * bn;
+      m0 = (t % mtn) * GT_BM;
+    } else if (k_hi_mode == GT_KHI_COL) {
+      n0 = (ntn - 1 - t / mtn) * bn;
+      m0 = (t % mtn) * GT_BM;
+    } else {
+      m0 = (t / ntn) * GT_BM;
+      n0 = (t % ntn) * bn;
+    }
   } else {
     int nt = 0;
     for (;; ++nt) {
-      const int cnt = min(mtn, ((nt + 1) * BN + GT_BM - 1) / GT_BM);
+      const int cnt = min(mtn, ((nt + 1) * bn + GT_BM - 1) / GT_BM);
       if (t < cnt || nt == ntn - 1) break;
       t -= cnt;
     }
     m0 = t * GT_BM;
-    n0 = nt * BN;
+    n0 = nt * bn;
   }
-  int kb = 0, ke = p.K;
-  if (p.k_lo_mode == GT_KLO_COL) kb = n0;
-  if (p.k_lo_mode == GT_KLO_ROW) kb = m0;
-  if (p.k_hi_mode == GT_KHI_COL) ke = min(p.K, n0 + BN);
+  int kb = 0, ke = K;
+  if (k_lo_mode == GT_KLO_COL) kb = n0;
+  if (k_lo_mode == GT_KLO_ROW) kb = m0;
+  if (k_hi_mode == GT_KHI_COL) ke = min(K, n0 + bn);
   kb = (kb / GT_BK) * GT_BK;
   k_begin = kb;
   n_iters = (ke > kb) ? (ke - kb + GT_BK - 1) / GT_BK : 0;
 }
 
-// Persistent: CTA b handles tiles b, b + gridDim.x, ...  The producer and the MMA issuer run
+template <int BN>
+__device__ __forceinline__ void gt_tile(const GemmTCArgs& p, int t, int& m0, int& n0, int& k_begin, int& n_iters) {
+  gt_tile_at(p.M, p.N, p.K, p.k_lo_mode, p.k_hi_mode, p.upper_only, BN, t, m0, n0, k_begin, n_iters);
+}
+
+// Snake assignment of tiles to the G persistent CTAs: round i goes b = 0 .. G-1 on even
+// rounds and G-1 .. 0 on odd ones, so a CTA's long first tile meets a short second one.
+__host__ __device__ inline int gt_sched(int i, int b, int G) { return i * G + ((i & 1) ? G - 1 - b : b); }
+
+// Persistent: CTA b handles the tiles gt_sched gives it.  The producer and the MMA issuer run
 // ahead across tile boundaries; each K stage lands in one of two TMEM accumulators, which
 // the epilogue warps drain into registers that were pre-loaded with C (beta = 1) while the
 // tile's first stages were in flight, so a tile ends with stores only.
@@ -181,7 +202,9 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
       // ---------------- TMA producer (continuous stage ring over all tiles) ----------------
       int it = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+      for (int rnd = 0; rnd * static_cast<int>(gridDim.x) < ntiles && ok; ++rnd) {
+        const int t = gt_sched(rnd, blockIdx.x, gridDim.x);
+        if (t >= ntiles) continue;
         int m0, n0, kb, ni;
         gt_tile<BN>(p, t, m0, n0, kb, ni);
         for (int j = 0; j < ni; ++j, ++it) {
@@ -215,7 +238,9 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
       const int cs = p.chunk_stages;
       bool ok = true;
       int it = 0, ch = 0;
-      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+      for (int rnd = 0; rnd * static_cast<int>(gridDim.x) < ntiles && ok; ++rnd) {
+        const int t = gt_sched(rnd, blockIdx.x, gridDim.x);
+        if (t >= ntiles) continue;
         int m0, n0, kb, ni;
         gt_tile<BN>(p, t, m0, n0, kb, ni);
         int b = 0;
@@ -267,7 +292,9 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
     const int hh = (warp - 2) >> 2;
     int ch = 0;
     bool all_ok = true;
-    for (int t = blockIdx.x; t < ntiles && all_ok; t += gridDim.x) {
+    for (int rnd = 0; rnd * static_cast<int>(gridDim.x) < ntiles && all_ok; ++rnd) {
+      const int t = gt_sched(rnd, blockIdx.x, gridDim.x);
+      if (t >= ntiles) continue;
       int m0, n0, kb, ni;
       gt_tile<BN>(p, t, m0, n0, kb, ni);
       const int r = m0 + q * 32 + lane;

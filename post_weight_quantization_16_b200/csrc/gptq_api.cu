@@ -11,6 +11,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <vector>
 #include <thread>
 
 #include "../../include/gptq.h"
@@ -226,14 +227,36 @@ cudaError_t set_gemm_tc_attributes() {
   return e;
 }
 
-// Tile width of a tensor-core product: the one with the least modelled time, waves of
-// persistent CTAs times a tile's cost (its width plus a fixed 64-column-equivalent overhead).
-int pick_bn(int M, int N, int upper, int sms) {
+// Tile width of a tensor-core product: the one with the least modelled time.  A tile costs
+// (K stages + 2 for the pipeline fill and the epilogue) x (BN + 64): a stage's MMAs grow with
+// the tile width, plus a part that does not (issue, barriers, the A operand).  The CTAs take
+// tiles in the snake order of gt_sched and the time is that of the busiest CTA.  Products with
+// triangular K ranges are simulated tile by tile (they are recorded once, in the factorization
+// graph); the others have equal tiles.
+int64_t gemm_cost(int M, int N, int K, int klo, int khi, int upper, int bn, int sms) {
+  const int ntiles = gt_num_tiles(M, N, upper, bn);
+  const int G = std::min(ntiles, sms);
+  if (G <= 0) return 0;
+  if (klo == GT_KLO_NONE && khi == GT_KHI_NONE) {
+    const int64_t waves = (ntiles + G - 1) / G;
+    return waves * ((K + GT_BK - 1) / GT_BK + 2) * (bn + 64);
+  }
+  std::vector<int64_t> load(G, 0);
+  for (int t = 0; t < ntiles; ++t) {
+    int m0, n0, kb, ni;
+    gt_tile_at(M, N, K, klo, khi, upper, bn, t, m0, n0, kb, ni);
+    const int r = t / G, q = t % G;
+    const int b = (r & 1) ? G - 1 - q : q;
+    load[b] += static_cast<int64_t>(ni + 2) * (bn + 64);
+  }
+  return *std::max_element(load.begin(), load.end());
+}
+
+int pick_bn(int M, int N, int K, int klo, int khi, int upper, int sms) {
   int best = 256;
   int64_t best_cost = -1;
   for (int bn : {256, 128, 64}) {
-    const int64_t waves = (gt_num_tiles(M, N, upper, bn) + sms - 1) / sms;
-    const int64_t cost = waves * (bn + 64);
+    const int64_t cost = gemm_cost(M, N, K, klo, khi, upper, bn, sms);
     if (best_cost < 0 || cost < best_cost) {
       best_cost = cost;
       best = bn;
@@ -246,7 +269,7 @@ gptq_status gemm_tc(gptq_ctx* c, int M, int N, int K, TcOperand A, TcOperand B, 
                     int khi, int upper, const TcOut& o, int chunk_stages = 1, int force_bn = 0) {
   if (M <= 0 || N <= 0) return GPTQ_OK;
   if (N % 32 || K % GT_BK) return GPTQ_ERR_ARG;
-  const int bn = force_bn ? force_bn : pick_bn(M, N, upper, c->num_sms);
+  const int bn = force_bn ? force_bn : pick_bn(M, N, K, klo, khi, upper, c->num_sms);
   const int tc_tiles = gt_num_tiles(M, N, upper, bn);
   if (gt_num_tiles(M, N, upper, 64) < kMinTcTiles && A.phi && B.phi) {
     GemmSimtArgs g;
