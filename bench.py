@@ -41,7 +41,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # kernel's sources are the ones captured.  The capture ran 65536 tokens; X traffic grows in
 # proportion to the tokens, so it is scaled per token to a full launch.
 PROFILED_TRAFFIC = {
-    "hessian_syrk_kernel": {
+    "hessian_syrk_pair_kernel": {
         "sources": {"post_weight_quantization_16_b200/csrc/hessian_tc.cuh": "0407c38d802bbd8cf2150eb1a81037799abe762b",
                     "post_weight_quantization_16_b200/csrc/sm100_ptx.cuh": "e9de838590f26e9845d60943020e63915adb0b72"},
         "n": 4096, "tokens": 65536, "dram_bytes": 975.245824e6 + 23.945472e6,
@@ -294,8 +294,8 @@ def run_gpu(args, rank, world, local_rank):
     h_tflops = h_flops / (h_ms / 1e3) / 1e12
     peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
     n, m = layer.n, layer.m
-    roofline = {"bound": "tensor", "kernel": "hessian_syrk_kernel", "achieved": h_tflops, "peak": peak,
-                "unit": "TFLOP/s", "frac": h_tflops / peak, "traffic": profiled_traffic("hessian_syrk_kernel", n, layer.n_tok),
+    roofline = {"bound": "tensor", "kernel": "hessian_syrk_pair_kernel", "achieved": h_tflops, "peak": peak,
+                "unit": "TFLOP/s", "frac": h_tflops / peak, "traffic": profiled_traffic("hessian_syrk_pair_kernel", n, layer.n_tok),
                 "peak_source": f"{peaks_src} bf16 dense, sustained", "algorithmic_flops_per_launch": h_flops}
 
     # whole-path roofline: contraction flops at the bf16 peak vs the sweep's bytes at HBM bandwidth

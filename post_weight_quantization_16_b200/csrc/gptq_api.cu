@@ -634,7 +634,7 @@ gptq_status gptq_create(gptq_ctx** out, int64_t n, int64_t m_max, int device, vo
     delete c;
     return GPTQ_ERR_CUDA;
   }
-  e = cudaFuncSetAttribute(hessian_syrk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, HS_SMEM);
+  e = cudaFuncSetAttribute(hessian_syrk_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, HP_SMEM);
   if (e == cudaSuccess) e = set_gemm_tc_attributes();
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(leaf_chol_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, LF_SMEM);
@@ -691,7 +691,8 @@ gptq_status gptq_hessian_accumulate(gptq_ctx* c, const void* X, int64_t n_tok, i
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return GPTQ_ERR_CUDA;
   const int chunk_iters = static_cast<int>(c->chunk_tokens / HS_BK);
-  CK(launch(c, hessian_syrk_kernel, dim3(hs_num_tiles(static_cast<int>(c->n))), dim3(HS_THREADS), HS_SMEM, map, c->H, static_cast<int>(c->n), static_cast<int>(n_tok), chunk_iters, c->status));
+  CK(launch(c, hessian_syrk_pair_kernel, dim3(2 * hp_num_pairs(static_cast<int>(c->n))), dim3(HS_THREADS), HP_SMEM, map,
+            c->H, static_cast<int>(c->n), static_cast<int>(n_tok), chunk_iters, c->status));
   CKL("hessian");
   c->n_tok += n_tok;
   c->mirrored = 0;
