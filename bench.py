@@ -37,14 +37,14 @@ WORKLOAD = "q_proj_4096x4096"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant kernel from one
-# ncu capture (profiles/hessian_syrk_kernel__block7b_q_65536tok_x4096.md), valid only while the
+# ncu capture (profiles/hessian_syrk_pair_kernel__block7b_q_65536tok_x4096.md), valid only while the
 # kernel's sources are the ones captured.  The capture ran 65536 tokens; X traffic grows in
 # proportion to the tokens, so it is scaled per token to a full launch.
 PROFILED_TRAFFIC = {
     "hessian_syrk_pair_kernel": {
-        "sources": {"post_weight_quantization_16_b200/csrc/hessian_tc.cuh": "0407c38d802bbd8cf2150eb1a81037799abe762b",
-                    "post_weight_quantization_16_b200/csrc/sm100_ptx.cuh": "e9de838590f26e9845d60943020e63915adb0b72"},
-        "n": 4096, "tokens": 65536, "dram_bytes": 975.245824e6 + 23.945472e6,
+        "sources": {"post_weight_quantization_16_b200/csrc/hessian_tc.cuh": "99d3e9d95b42960505710a519acfa15b724aa743",
+                    "post_weight_quantization_16_b200/csrc/sm100_ptx.cuh": "fa523347e627c8a77d87a07310da3ca52cf8c71e"},
+        "n": 4096, "tokens": 65536, "dram_bytes": 975.479040e6 + 24.431360e6,
     },
 }
 
