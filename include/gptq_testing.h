@@ -44,6 +44,17 @@ gptq_status gptq_test_gemm_tf32x3(int M, int N, int K, const float* A_hi, const 
 gptq_status gptq_test_div_rn(uint64_t seed, int64_t count, uint64_t* mismatches, float* example, int device,
                              void* cuda_stream);
 
+/* Host-only checks of the tensor-core GEMM's work split (no GPU needed).
+ * gptq_test_pick_tile_n: the output tile width (64, 128 or 256) the library picks for an
+ *   M x N x K product with the given K-range modes on `sms` persistent CTAs; -1 on bad sizes.
+ * gptq_test_tile_schedule: walks the schedule of `ctas` persistent CTAs over the tiles of
+ *   width tile_n and returns 0 when every tile is visited exactly once, the tiles are
+ *   distinct, aligned and in range (with upper_only: exactly the tiles that reach the upper
+ *   triangle, otherwise all of them), and every non-empty K range is aligned and within K; otherwise
+ *   the number (1-8) of the first check that failed, or -1 on bad arguments. */
+int gptq_test_pick_tile_n(int M, int N, int K, int k_lo_mode, int k_hi_mode, int upper_only, int sms);
+int gptq_test_tile_schedule(int M, int N, int K, int k_lo_mode, int k_hi_mode, int upper_only, int tile_n, int ctas);
+
 #ifdef __cplusplus
 }
 #endif

@@ -962,6 +962,44 @@ gptq_status gptq_test_div_rn(uint64_t seed, int64_t count, uint64_t* mismatches,
   return GPTQ_OK;
 }
 
+int gptq_test_pick_tile_n(int M, int N, int K, int k_lo_mode, int k_hi_mode, int upper_only, int sms) {
+  if (M < 1 || N < 1 || K < 1 || sms < 1) return -1;
+  return pick_bn(M, N, K, k_lo_mode, k_hi_mode, upper_only, sms);
+}
+
+int gptq_test_tile_schedule(int M, int N, int K, int k_lo_mode, int k_hi_mode, int upper_only, int tile_n,
+                                    int ctas) {
+  if (M < 1 || N < 1 || K < 1 || ctas < 1 || (tile_n != 64 && tile_n != 128 && tile_n != 256)) return -1;
+  const int ntiles = gt_num_tiles(M, N, upper_only, tile_n);
+  const int mtn = (M + GT_BM - 1) / GT_BM, ntn = (N + tile_n - 1) / tile_n;
+  std::vector<int> seen(ntiles, 0), cell(static_cast<size_t>(mtn) * ntn, 0);
+  for (int b = 0; b < ctas; ++b)
+    for (int r = 0; r * ctas < ntiles; ++r) {
+      const int t = gt_sched(r, b, ctas);
+      if (t < 0) return 1;
+      if (t >= ntiles) continue;
+      ++seen[t];
+    }
+  for (int t = 0; t < ntiles; ++t) {
+    if (seen[t] != 1) return 2;  // every tile exactly once
+    int m0, n0, kb, ni;
+    gt_tile_at(M, N, K, k_lo_mode, k_hi_mode, upper_only, tile_n, t, m0, n0, kb, ni);
+    if (m0 < 0 || m0 >= mtn * GT_BM || n0 < 0 || n0 >= ntn * tile_n || m0 % GT_BM || n0 % tile_n) return 3;
+    if (kb < 0 || kb % GT_BK || ni < 0 || (ni > 0 && kb + ni * GT_BK > ((K + GT_BK - 1) / GT_BK) * GT_BK)) return 4;
+    if (upper_only && m0 >= n0 + tile_n) return 5;  // wholly below the diagonal
+    if (++cell[static_cast<size_t>(m0 / GT_BM) * ntn + n0 / tile_n] != 1) return 6;  // distinct tiles
+  }
+  if (!upper_only) {
+    for (int v : cell)
+      if (v != 1) return 7;  // and all of them
+  } else {
+    for (int mt = 0; mt < mtn; ++mt)
+      for (int nt = 0; nt < ntn; ++nt)
+        if ((mt * GT_BM < (nt + 1) * tile_n) != (cell[static_cast<size_t>(mt) * ntn + nt] == 1)) return 8;
+  }
+  return 0;
+}
+
 gptq_status gptq_destroy(gptq_ctx* c) {
   if (!c) return GPTQ_OK;
   gptq_status s;

@@ -61,6 +61,8 @@ _SIGS = {
                                              _P]),
     "gptq_test_div_rn": (ctypes.c_int, [ctypes.c_uint64, ctypes.c_int64, ctypes.POINTER(ctypes.c_uint64),
                                         ctypes.POINTER(ctypes.c_float), ctypes.c_int, _P]),
+    "gptq_test_pick_tile_n": (ctypes.c_int, [ctypes.c_int] * 7),
+    "gptq_test_tile_schedule": (ctypes.c_int, [ctypes.c_int] * 8),
 }
 
 
