@@ -161,26 +161,36 @@ class ClockSampler:
 # ----------------------------------------------------------------------------------------
 # CPU oracle baseline (bounded sample of the same workload)
 # ----------------------------------------------------------------------------------------
-def cpu_oracle_baseline(layer, qs, tok_sample=16384, row_sample=256):
+def cpu_oracle_baseline(layer, qs, tok_sample=16384, row_sample=256, prep_n=None, data=None):
+    """The oracle timed on a bounded sample of the layer, scaled to the whole layer: the Hessian
+    on tok_sample tokens (time x n_tok / tok_sample); prepare on the leading prep_n x prep_n
+    block of H (time x (n / prep_n)^3; the whole H when prep_n is None) and the sweep of
+    row_sample rows over those prep_n columns (time x (m / row_sample) x (n / prep_n)).
+    `data` = (X sample, W) generated beforehand, outside the timing."""
     from oracle import gptq_oracle as O
     cores = len(os.sched_getaffinity(0))
-    X = synth.bf16_bits_to_f32(synth.make_x_bf16(layer, 0, tok_sample))
-    W = synth.make_w_fp16(layer).astype(np.float64)
+    if data is None:
+        data = (synth.bf16_bits_to_f32(synth.make_x_bf16(layer, 0, tok_sample)),
+                synth.make_w_fp16(layer).astype(np.float64))
+    X, W = data
     t0 = time.perf_counter()
     H = O.hessian(X)
-    t_h = (time.perf_counter() - t0) * (layer.n_tok / tok_sample)
+    t_h = (time.perf_counter() - t0) * (layer.n_tok / X.shape[0])
+    pn = layer.n if prep_n is None else min(prep_n, layer.n)
     t0 = time.perf_counter()
-    prep = O.prepare(H, qs.damp, qs.desc_act)
-    t_p = time.perf_counter() - t0
-    Wp = W[:row_sample][:, prep["perm"]]
+    prep = O.prepare(H[:pn, :pn], qs.damp, qs.desc_act)
+    t_p = (time.perf_counter() - t0) * (layer.n / pn) ** 3
+    g = qs.group_size if (qs.group_size != -1 and pn % qs.group_size == 0) else -1
+    Wp = W[:row_sample, :pn][:, prep["perm"]]
     t0 = time.perf_counter()
-    O.gptq_sweep(Wp, prep["U"], qs.bits, qs.group_size, bool(qs.sym), block=128)
-    t_s = (time.perf_counter() - t0) * (layer.m / row_sample)
+    O.gptq_sweep(Wp, prep["U"], qs.bits, g, bool(qs.sym), block=128)
+    t_s = (time.perf_counter() - t0) * (layer.m / row_sample) * (layer.n / pn)
     t_layer = t_h + t_p + t_s
     return {
         "value": layer.m * layer.n / t_layer / 1e9, "unit": "Gweights/s", "cores": cores, "kind": "oracle",
-        "sample": (f"Hessian on {tok_sample} of {layer.n_tok} tokens (scaled), full prepare at n={layer.n}, "
-                   f"sweep of {row_sample} of {layer.m} rows (scaled); float64 numpy"),
+        "sample": (f"Hessian on {X.shape[0]} of {layer.n_tok} tokens (scaled), prepare and sweep on the leading "
+                   f"{pn} of {layer.n} columns (scaled by n^3 and n), sweep of {row_sample} of {layer.m} rows "
+                   f"(scaled); float64 numpy"),
         "seconds_per_layer": t_layer, "stage_seconds": {"hessian": t_h, "prepare": t_p, "sweep": t_s},
     }
 
@@ -190,10 +200,20 @@ def run_reference(args, rank, world):
     if rank != 0:
         return
     layer, qs = synth.WORKLOADS[args.config]
-    tok, rows = 4096, 64
+    # each step a sample small enough that all warm-up and timed steps end within a few minutes
+    n_steps = args.warmup + args.steps
+    if n_steps <= 4:
+        tok, rows, pn = 4096, 64, None
+    elif n_steps <= 20:
+        tok, rows, pn = 2048, 32, 2048
+    else:
+        tok, rows, pn = 1024, 16, 2048
+    tok = max(64, int(tok * min(1.0, (4096 / layer.n) ** 2)))  # the Hessian sample's cost grows as n^2
+    data = (synth.bf16_bits_to_f32(synth.make_x_bf16(layer, 0, tok)), synth.make_w_fp16(layer).astype(np.float64))
     times = []
-    for step in range(args.warmup + args.steps):
-        r = cpu_oracle_baseline(layer, qs, tok_sample=tok, row_sample=rows)
+    r = None
+    for step in range(n_steps):
+        r = cpu_oracle_baseline(layer, qs, tok_sample=tok, row_sample=rows, prep_n=pn, data=data)
         if step >= args.warmup:
             times.append(r["seconds_per_layer"])
     t = sum(times) / len(times)
@@ -206,8 +226,7 @@ def run_reference(args, rank, world):
         "config": {"workload": args.config, "m": layer.m, "n": layer.n, "n_tok": layer.n_tok, "bits": qs.bits,
                    "group_size": qs.group_size, "sym": qs.sym, "damp": qs.damp, "desc_act": qs.desc_act},
         "cpu_baseline": {"value": val, "unit": "Gweights/s", "cores": cores, "kind": "oracle",
-                         "sample": f"each step: Hessian on {tok} tokens, full prepare, sweep of {rows} rows; "
-                                   "times scaled to the full layer"},
+                         "sample": "each step: " + r["sample"]},
         "e2e": {"value": val, "unit": "Gweights/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
