@@ -362,6 +362,27 @@ def layer_error(W, What, H0) -> float:
 
 
 # ==================================================================================
+# the packed result's consumer (the step after the path: a layer that keeps its weights as
+# codes and dequantizes them for the product, [P4] §4.3 "INT4 ... 反量化到 FP16 再计算")
+# ==================================================================================
+def dequantize_packed(packed, scales, zeros, perm, n: int, bits: int, group_size: int) -> np.ndarray:
+    """W_hat in ORIGINAL column order from the packed output of the path: code k of a row
+    (sweep order) belongs to group k // g and dequantizes as (code - zero) * scale ([P4] §3.1
+    dequantize), formed exactly in float64 from the stored float32 scale and zero; sweep
+    position k goes back to original column perm[k]."""
+    codes = unpack_codes(packed, n, bits)
+    grp = np.arange(n) // _group_width(group_size, n)
+    s = np.asarray(scales, dtype=np.float32).astype(np.float64)[:, grp]
+    z = np.asarray(zeros, dtype=np.float32).astype(np.float64)[:, grp]
+    return unpermute_columns((codes.astype(np.float64) - z) * s, perm)
+
+
+def dequant_matmul(X, packed, scales, zeros, perm, n: int, bits: int, group_size: int) -> np.ndarray:
+    """Y = X W_hat^T for activations X [tokens, n] in original column order (float64)."""
+    return np.asarray(X, dtype=np.float64) @ dequantize_packed(packed, scales, zeros, perm, n, bits, group_size).T
+
+
+# ==================================================================================
 # whole layer
 # ==================================================================================
 def quantize_layer(W, H, bits: int, group_size: int, sym: bool, damp: float, desc_act: bool,

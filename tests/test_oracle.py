@@ -386,3 +386,27 @@ def test_replay_adopts_in_band_flip_and_flags_out_of_band_flip():
     assert st.adopted == 1 and st.hard_mismatch == 0
     assert st.identical == st.total - 1
     assert np.array_equal(out["codes"], planted["codes"])
+
+
+# ----------------------------------------------------------------------------------------
+# the packed result's consumer: decoding the stream with its documented layout (LSB-first
+# per row, sweep order, groups of g sweep positions, perm back to original columns) gives
+# back exactly the dequantized weights the sweep formed, and the product with them
+# ----------------------------------------------------------------------------------------
+@pytest.mark.parametrize("bits,g,sym,desc_act", [(4, 64, False, True), (3, 32, True, True), (2, -1, False, False),
+                                                 (8, 128, True, True)])
+def test_dequantize_packed_round_trip(bits, g, sym, desc_act):
+    r = np.random.default_rng(bits * 10 + (g if g > 0 else 1))
+    m, n, N = 12, 256, 600
+    X = r.standard_normal((N, n))
+    X[:, r.choice(n, 4, replace=False)] *= 15.0
+    W = 0.02 * r.standard_normal((m, n))
+    H = O.hessian(X)
+    res = O.quantize_layer(W, H, bits, g, sym, 0.01, desc_act)
+    What = O.dequantize_packed(res["packed"], res["scales"], res["zeros"], res["perm"], n, bits, g)
+    assert np.array_equal(What, res["what_orig"])
+    Y = O.dequant_matmul(X[:7], res["packed"], res["scales"], res["zeros"], res["perm"], n, bits, g)
+    assert np.allclose(Y, X[:7] @ res["what_orig"].T, rtol=1e-12, atol=1e-12)
+    if desc_act:  # the permutation matters: decoding without it does not give W_hat back
+        wrong = O.dequantize_packed(res["packed"], res["scales"], res["zeros"], np.arange(n), n, bits, g)
+        assert not np.array_equal(wrong, res["what_orig"])
