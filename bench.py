@@ -169,6 +169,8 @@ def cpu_oracle_baseline(layer, qs, tok_sample=16384, row_sample=256, prep_n=None
     `data` = (X sample, W) generated beforehand, outside the timing."""
     from oracle import gptq_oracle as O
     cores = len(os.sched_getaffinity(0))
+    tok_sample = min(tok_sample, layer.n_tok)
+    row_sample = min(row_sample, layer.m)
     if data is None:
         data = (synth.bf16_bits_to_f32(synth.make_x_bf16(layer, 0, tok_sample)),
                 synth.make_w_fp16(layer).astype(np.float64))
@@ -208,7 +210,7 @@ def run_reference(args, rank, world):
         tok, rows, pn = 2048, 32, 2048
     else:
         tok, rows, pn = 1024, 16, 2048
-    tok = max(64, int(tok * min(1.0, (4096 / layer.n) ** 2)))  # the Hessian sample's cost grows as n^2
+    tok = min(layer.n_tok, max(64, int(tok * min(1.0, (4096 / layer.n) ** 2))))  # its cost grows as n^2
     data = (synth.bf16_bits_to_f32(synth.make_x_bf16(layer, 0, tok)), synth.make_w_fp16(layer).astype(np.float64))
     times = []
     r = None
