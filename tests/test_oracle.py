@@ -410,3 +410,94 @@ def test_dequantize_packed_round_trip(bits, g, sym, desc_act):
     if desc_act:  # the permutation matters: decoding without it does not give W_hat back
         wrong = O.dequantize_packed(res["packed"], res["scales"], res["zeros"], np.arange(n), n, bits, g)
         assert not np.array_equal(wrong, res["what_orig"])
+
+
+# ----------------------------------------------------------------------------------------
+# the replay's zero-point branch: a reference whose zero-point took the other side of an
+# in-band rounding decision is adopted; one outside the band, or more than one step away,
+# is a hard mismatch (asymmetric quantizer of "模型量化实战…" §3.1: z = -round(xmin / s))
+# ----------------------------------------------------------------------------------------
+def test_zero_boundary_distance_closed_form():
+    t = np.array([-2.4999, 3.2, 0.5, -0.7, 7.0, -3.5, 1e-9])
+    want = np.array([1e-4, 0.3, 0.0, 0.2, 0.5, 0.0, 0.5 - 1e-9])
+    assert np.allclose(O.zero_boundary_distance(t), want, atol=1e-12)
+
+
+def _zero_rows():
+    """Three rows whose first 32-column group has xmax = 12.5 (4-bit: s close to 1) and an
+    xmin that puts t = xmin / s at 8e-5 (row 0), 0.25 (row 1) and 8e-5 (row 2) from a
+    half-integer; the remaining values are small and inside the range."""
+    rng = _rng(77)
+    W = rng.uniform(-1.0, 1.0, (3, 64))
+    W[:, 1] = 12.5
+    W[0, 0] = -2.5 + 1e-4
+    W[1, 0] = -2.25
+    W[2, 0] = -2.5 - 1e-4
+    return W
+
+
+def test_replay_adopts_in_band_zero_flip():
+    W = _zero_rows()
+    U = np.eye(W.shape[1])
+    ref = O.gptq_sweep(W, U, 4, 32, False)
+    s, z, t = O.group_params(W[:, :32], 4, False)
+    assert O.zero_boundary_distance(t[0]) < 1e-3 and z[0] == 2.0
+    planted = ref["zeros"].copy()
+    planted[0, 0] = 3.0                      # the other side of row 0's in-band decision
+    st = O.ReplayStats()
+    out = O.gptq_sweep(W, U, 4, 32, False, ref_zeros=planted, stats=st)
+    assert st.zero_adopted == 1 and st.zero_hard_mismatch == 0
+    assert np.array_equal(out["zeros"], planted)
+    # the group's codes and dequantized values are formed with the adopted zero-point
+    w32 = W[0, :32].astype(np.float32)
+    u = np.clip(np.rint(w32 / s[0] + np.float32(3.0)), 0, 15)
+    assert np.array_equal(out["codes"][0, :32], u.astype(np.int64))
+    assert np.allclose(out["what"][0, :32], (u - 3.0) * np.float64(s[0]), rtol=0, atol=0)
+    # the other rows are untouched
+    assert np.array_equal(out["codes"][1:], ref["codes"][1:])
+
+
+def test_replay_flags_out_of_band_or_far_zero_flip():
+    W = _zero_rows()
+    U = np.eye(W.shape[1])
+    ref = O.gptq_sweep(W, U, 4, 32, False)
+    _, z, t = O.group_params(W[:, :32], 4, False)
+    assert O.zero_boundary_distance(t[1]) > 0.2
+    planted = ref["zeros"].copy()
+    planted[1, 0] = z[1] + 1                 # row 1: one step away, but far from a boundary
+    planted[2, 0] = z[2] - 2                 # row 2: in band, but two steps away
+    st = O.ReplayStats()
+    out = O.gptq_sweep(W, U, 4, 32, False, ref_zeros=planted, stats=st)
+    assert st.zero_adopted == 0 and st.zero_hard_mismatch == 2
+    assert np.array_equal(out["zeros"], ref["zeros"])  # the oracle keeps its own decisions
+
+
+def test_replay_ignores_zeros_of_symmetric_codes():
+    """Symmetric zero-points are the constant 2^(b-1); the replay has nothing to adopt."""
+    W = _zero_rows()
+    U = np.eye(W.shape[1])
+    planted = np.full((3, 2), 7.0, dtype=np.float32)
+    st = O.ReplayStats()
+    out = O.gptq_sweep(W, U, 4, 32, True, ref_zeros=planted, stats=st)
+    assert st.zero_adopted == 0 and st.zero_hard_mismatch == 0
+    assert (out["zeros"] == 8.0).all()
+
+
+def test_dequant_matmul_equals_sum_in_sweep_order():
+    """Y[t, r] = sum_k X[t, perm[k]] (code[r, k] - z[r, k // g]) s[r, k // g]: the product
+    taken in sweep order with the activations gathered by perm, on a tiny case by loops."""
+    rng = _rng(31)
+    m, n, g, bits = 5, 64, 16, 4
+    codes = rng.integers(0, 16, (m, n))
+    s = rng.uniform(0.01, 0.1, (m, n // g)).astype(np.float32)
+    z = rng.integers(0, 16, (m, n // g)).astype(np.float32)
+    perm = rng.permutation(n)
+    X = rng.normal(0, 1, (3, n))
+    packed = O.pack_codes(codes, bits)
+    Y = O.dequant_matmul(X, packed, s, z, perm, n, bits, g)
+    for t in range(3):
+        for r in range(m):
+            acc = 0.0
+            for k in range(n):
+                acc += X[t, perm[k]] * (codes[r, k] - float(z[r, k // g])) * float(s[r, k // g])
+            assert abs(Y[t, r] - acc) <= 1e-12 * (1 + abs(acc))
