@@ -112,6 +112,13 @@ gptq_status gptq_prepare(gptq_ctx* ctx, double damp, int desc_act, int32_t* perm
  * buffer U_out.  GPTQ_ERR_STATE before gptq_prepare.  Asynchronous. */
 gptq_status gptq_get_factor(gptq_ctx* ctx, float* U_out);
 
+/* Copy the dead-column mask of the last gptq_prepare to the device buffer dead_out
+ * (uint8 [n], ORIGINAL column order): 1 where diag(H) was 0, so that the column was treated
+ * as unexcited (H_ii = 1) and its weights are zeroed by gptq_quantize_layer; 0 elsewhere.
+ * This is the `dead` input gptq_quantize_layer_noalloc needs to reproduce the context's
+ * result.  GPTQ_ERR_STATE before gptq_prepare.  Asynchronous. */
+gptq_status gptq_get_dead_columns(gptq_ctx* ctx, uint8_t* dead_out);
+
 /* S5-S7 (asynchronous): quantize W with the prepared factor.
  *   W_fp16     : device fp16 [m x n] row-major (ld n), ORIGINAL column order, 1 <= m <= m_max.
  *   codes_out  : device uint32 [m x n*bits/32]; row r holds its codes in SWEEP order as an
@@ -167,6 +174,32 @@ gptq_status gptq_quantize_layer_noalloc(const void* W_fp16, int64_t m, int64_t n
                                         const int32_t* perm, const uint8_t* dead, gptq_qparams qp,
                                         uint32_t* codes_out, float* scales_out, float* zeros_out,
                                         int32_t* g_idx_out, float* W_hat_out, int device, void* cuda_stream);
+
+/* Per-kernel instrumentation (off by default).  While profiling is on, every kernel the
+ * context launches is bracketed by CUDA timing events on the context's stream and the
+ * factorization runs as individual launches instead of its recorded graph (so launches no
+ * longer overlap their predecessor: totals are slightly above those of normal runs).
+ * gptq_get_profile waits for the stream (bounded), folds the records into one entry per
+ * kernel role and clears them.
+ *   name     : kernel and role, e.g. "gemm_tf32x3:factor"
+ *   launches : launches recorded
+ *   ms       : sum of the launches' event durations
+ *   flops    : algorithmic floating-point operations of those launches (the product's nonzero
+ *              multiply-adds x 2, counted once however many partial products the kernel forms;
+ *              0 for kernels that are not contractions)
+ *   bytes    : algorithmic bytes read and written by those launches (0 where not stated)
+ * gptq_get_profile writes at most `capacity` entries to the host array `out` and the number
+ * of roles recorded to *count (which may exceed capacity). */
+typedef struct {
+  char name[40];
+  int64_t launches;
+  double ms;
+  double flops;
+  double bytes;
+} gptq_kernel_stat;
+
+gptq_status gptq_set_profiling(gptq_ctx* ctx, int on);
+gptq_status gptq_get_profile(gptq_ctx* ctx, gptq_kernel_stat* out, int capacity, int* count);
 
 /* Static description of a status code. */
 const char* gptq_status_string(gptq_status s);

@@ -44,6 +44,14 @@ gptq_status gptq_test_gemm_tf32x3(int M, int N, int K, const float* A_hi, const 
 gptq_status gptq_test_div_rn(uint64_t seed, int64_t count, uint64_t* mismatches, float* example, int device,
                              void* cuda_stream);
 
+/* Failure detection of the device-side waits: enqueue on the context's stream a one-CTA
+ * kernel that waits on an mbarrier no thread ever arrives on, with the same bounded wait the
+ * tcgen05 kernels use but a limit of limit_ns nanoseconds (1 <= limit_ns <= 10 s).  When the
+ * wait gives up the kernel records ST_TIMEOUT in the context's status word and returns, so
+ * the next gptq_synchronize (or gptq_prepare) reports GPTQ_ERR_TIMEOUT and the context stays
+ * usable.  Asynchronous. */
+gptq_status gptq_test_bounded_wait(gptq_ctx* ctx, uint64_t limit_ns);
+
 /* Host-only checks of the tensor-core GEMM's work split (no GPU needed).
  * gptq_test_pick_tile_n: the output tile width (64, 128 or 256) the library picks for an
  *   M x N x K product with the given K-range modes on `sms` persistent CTAs; -1 on bad sizes.

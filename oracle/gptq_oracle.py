@@ -363,7 +363,8 @@ def layer_error(W, What, H0) -> float:
 
 # ==================================================================================
 # the packed result's consumer (the step after the path: a layer that keeps its weights as
-# codes and dequantizes them for the product, [P4] §4.3 "INT4 ... 反量化到 FP16 再计算")
+# codes and dequantizes them for the product: per [P4] §4.3, INT4 weights are turned back
+# into FP16 values before the matrix product, and the gain is memory bandwidth)
 # ==================================================================================
 def dequantize_packed(packed, scales, zeros, perm, n: int, bits: int, group_size: int) -> np.ndarray:
     """W_hat in ORIGINAL column order from the packed output of the path: code k of a row

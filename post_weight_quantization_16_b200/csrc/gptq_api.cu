@@ -69,7 +69,20 @@ struct gptq_ctx {
   bool pdl = true;                        // launches overlap their predecessor (programmatic)
   cudaGraphExec_t factor_graph = nullptr;  // the factorization recursion, recorded once
   int64_t factor_graph_launches = 0;
+  int gemm_role = 0;                      // 0: factorization product, 1: trailing update (instrumentation)
   PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  // per-kernel instrumentation (gptq_set_profiling): the role and algorithmic work of the next
+  // launch, and one record (two timing events) per launch while profiling is on
+  bool prof = false;
+  const char* tag = "other";
+  double tag_flops = 0.0, tag_bytes = 0.0;
+  struct ProfRec {
+    const char* tag;
+    double flops, bytes;
+    cudaEvent_t e0, e1;
+  };
+  std::vector<ProfRec> prof_recs;
+  bool prof_error = false;
 };
 
 namespace {
@@ -168,9 +181,51 @@ cudaError_t launch(gptq_ctx* c, void (*kernel)(KArgs...), dim3 grid, dim3 block,
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = c->pdl ? 1 : 0;
+  cfg.numAttrs = (c->pdl && !c->prof) ? 1 : 0;
   ++c->launches;
-  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  const char* tag = c->tag;
+  const double fl = c->tag_flops, by = c->tag_bytes;
+  c->tag = "other";
+  c->tag_flops = c->tag_bytes = 0.0;
+  if (!c->prof) return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  gptq_ctx::ProfRec r{tag, fl, by, nullptr, nullptr};
+  if (cudaEventCreate(&r.e0) != cudaSuccess || cudaEventCreate(&r.e1) != cudaSuccess) {
+    if (r.e0) cudaEventDestroy(r.e0);
+    c->prof_error = true;
+    cudaGetLastError();
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  }
+  cudaEventRecord(r.e0, c->stream);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  cudaEventRecord(r.e1, c->stream);
+  c->prof_recs.push_back(r);
+  return e;
+}
+
+// Role and algorithmic work of the next launch (instrumentation only).
+void tag(gptq_ctx* c, const char* name, double flops, double bytes) {
+  c->tag = name;
+  c->tag_flops = flops;
+  c->tag_bytes = bytes;
+}
+
+// Algorithmic flops of C (+)= A B^T with the K ranges and output triangle gemm_tc uses:
+// 2 x the nonzero multiply-adds, element (r, c) of C taking k in [kb, ke) with kb = c (B
+// lower in K-major form), r (A upper) or 0, ke = c + 1 (B upper) or K; upper_only keeps r <= c.
+double gemm_algo_flops(int M, int N, int K, int klo, int khi, int upper) {
+  double total = 0.0;
+  for (int col = 0; col < N; ++col) {
+    const int64_t R = upper ? std::min<int64_t>(M, col + 1) : M;
+    const int64_t ke = (khi == GT_KHI_COL) ? std::min<int64_t>(K, col + 1) : K;
+    if (klo == GT_KLO_ROW) {
+      const int64_t q = std::min<int64_t>(R, ke);
+      total += static_cast<double>(q * ke - q * (q - 1) / 2);
+    } else {
+      const int64_t kb = (klo == GT_KLO_COL) ? col : 0;
+      total += static_cast<double>(R) * static_cast<double>(std::max<int64_t>(0, ke - kb));
+    }
+  }
+  return 2.0 * total;
 }
 
 // 2-D fp32 tensor map of a row-major sub-matrix (rows x cols, leading dimension ld), boxes of
@@ -295,6 +350,8 @@ gptq_status gemm_tc(gptq_ctx* c, int M, int N, int K, TcOperand A, TcOperand B, 
     g.Cthi = o.Cthi;
     g.Ctlo = o.Ctlo;
     g.ldt = o.ldt;
+    tag(c, c->gemm_role ? "gemm_hilo_simt:trailing" : "gemm_hilo_simt:factor",
+        gemm_algo_flops(M, N, K, klo, khi, upper), 0.0);
     if (static_cast<int64_t>(M) * N <= 512 * 512) {  // 32 x 32 tiles: more CTAs for the smallest products
       dim3 grid((N + 31) / 32, (M + 31) / 32);
       CK(launch(c, gemm_hilo_simt_kernel<32, 32>, grid, dim3(GS_THREADS), gs_smem_bytes<32, 32>(), g));
@@ -334,6 +391,7 @@ gptq_status gemm_tc(gptq_ctx* c, int M, int N, int K, TcOperand A, TcOperand B, 
   if (o.c_map && (beta != 1 || !o.C)) return GPTQ_ERR_ARG;
   const CUtensorMap& cm = o.c_map ? *o.c_map : *A.hi;  // unused unless c_reduce
   const dim3 grid(std::min(tc_tiles, c->num_sms));
+  tag(c, c->gemm_role ? "gemm_tf32x3:trailing" : "gemm_tf32x3:factor", gemm_algo_flops(M, N, K, klo, khi, upper), 0.0);
   if (bn == 256)
     CK(launch(c, gemm_tf32x3_kernel<256>, grid, dim3(GT_THREADS), GtCfg<256>::SMEM, *A.hi, *A.lo, *B.hi, *B.lo, cm, a));
   else if (bn == 128)
@@ -348,6 +406,7 @@ gptq_status gemm_tc(gptq_ctx* c, int M, int N, int K, TcOperand A, TcOperand B, 
 gptq_status chol_inv(gptq_ctx* c, int o, int h) {
   const int n = static_cast<int>(c->n);
   if (h <= LF_NB) {
+    tag(c, "leaf_chol_inv", 2.0 * LF_NB * LF_NB * LF_NB / 3.0, 4.0 * LF_NB * LF_NB * 4);
     CK(launch(c, leaf_chol_inv_kernel, dim3(1), dim3(LF_THREADS), LF_SMEM, c->A_hi, c->A_lo, n, o, c->U_hi, c->U_lo,
               c->status));
     CKL("leaf_chol_inv");
@@ -361,6 +420,7 @@ gptq_status chol_inv(gptq_ctx* c, int o, int h) {
       c->stream = c->side_stream;
       c->pdl = false;
     }
+    tag(c, "transpose_block", 0.0, 4.0 * LF_NB * LF_NB * 4);
     const cudaError_t e = launch(c, transpose_block_kernel, dim3(4, 4), dim3(32, 8), 0, c->U_hi, c->U_lo, n, o,
                                  c->Ut_hi, c->Ut_lo);
     if (branch) {
@@ -465,6 +525,14 @@ gptq_status encode_maps(gptq_ctx* c) {
 // Run the factorization recursion: recorded as a CUDA graph on first use (on a private
 // stream), then replayed on the context's stream.
 gptq_status run_factorization(gptq_ctx* c) {
+  c->gemm_role = 0;
+  if (c->prof) {  // instrumented: every launch on its own, timed, on the context's stream
+    cudaStream_t side = c->side_stream;
+    c->side_stream = nullptr;
+    const gptq_status s = chol_inv(c, 0, static_cast<int>(c->n));
+    c->side_stream = side;
+    return s;
+  }
   if (!c->factor_graph) {
     if (!c->capture_stream) CK(cudaStreamCreateWithFlags(&c->capture_stream, cudaStreamNonBlocking));
     if (!c->side_stream) CK(cudaStreamCreateWithFlags(&c->side_stream, cudaStreamNonBlocking));
@@ -511,7 +579,16 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
 }
 
+void free_prof(gptq_ctx* c) {
+  for (auto& r : c->prof_recs) {
+    cudaEventDestroy(r.e0);
+    cudaEventDestroy(r.e1);
+  }
+  c->prof_recs.clear();
+}
+
 void free_all(gptq_ctx* c) {
+  free_prof(c);
   if (c->factor_graph) cudaGraphExecDestroy(c->factor_graph);
   if (c->capture_stream) cudaStreamDestroy(c->capture_stream);
   if (c->side_stream) cudaStreamDestroy(c->side_stream);
@@ -691,6 +768,8 @@ gptq_status gptq_hessian_accumulate(gptq_ctx* c, const void* X, int64_t n_tok, i
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return GPTQ_ERR_CUDA;
   const int chunk_iters = static_cast<int>(c->chunk_tokens / HS_BK);
+  const double nn1 = static_cast<double>(c->n) * (c->n + 1);
+  tag(c, "hessian_syrk_pair", static_cast<double>(n_tok) * nn1, 2.0 * n_tok * c->n + 4.0 * nn1);
   CK(launch(c, hessian_syrk_pair_kernel, dim3(2 * hp_num_pairs(static_cast<int>(c->n))), dim3(HS_THREADS), HP_SMEM, map,
             c->H, static_cast<int>(c->n), static_cast<int>(n_tok), chunk_iters, c->status));
   CKL("hessian");
@@ -702,6 +781,7 @@ gptq_status gptq_hessian_accumulate(gptq_ctx* c, const void* X, int64_t n_tok, i
 static gptq_status ensure_mirrored(gptq_ctx* c) {
   if (c->mirrored) return GPTQ_OK;
   const int n = static_cast<int>(c->n);
+  tag(c, "prepare:mirror", 0.0, 4.0 * n * n);
   CK(launch(c, mirror_upper_kernel, dim3(n / 32, n / 32), dim3(32, 8), 0, c->H, n));
   CKL("mirror");
   c->mirrored = 1;
@@ -738,13 +818,16 @@ gptq_status gptq_prepare(gptq_ctx* c, double damp, int desc_act, int32_t* perm_o
   gptq_status s;
   c->state = ST_ACCUM;
   if ((s = ensure_mirrored(c)) != GPTQ_OK) return s;
+  tag(c, "prepare:diag_stats", 0.0, 9.0 * n);
   CK(launch(c, diag_stats_kernel, dim3(1), dim3(1024), 0, c->H, n, c->keys, c->dead, c->mean));
   CKL("diag_stats");
+  tag(c, "prepare:perm", 0.0, 8.0 * n);
   if (desc_act)
     CK(launch(c, rank_perm_kernel, dim3((n + 255) / 256), dim3(256), 0, c->keys, n, c->perm));
   else
     CK(launch(c, identity_perm_kernel, dim3((n + 255) / 256), dim3(256), 0, n, c->perm));
   CKL("perm");
+  tag(c, "prepare:gather_damp", 0.0, 12.0 * n * n);
   CK(launch(c, gather_damp_kernel, dim3(n), dim3(256), static_cast<size_t>(n) * 4, c->H, n, c->perm, c->keys, c->mean, damp,
                                                                         c->A_hi, c->A_lo));
   CKL("gather");
@@ -764,8 +847,67 @@ gptq_status gptq_get_factor(gptq_ctx* c, float* U_out) {
   if (c->state != ST_PREPARED) return GPTQ_ERR_STATE;
   DeviceGuard dg(c->device);
   const size_t nn = static_cast<size_t>(c->n) * c->n;
+  tag(c, "combine_hilo", 0.0, 12.0 * static_cast<double>(nn));
   CK(launch(c, combine_hilo_kernel, dim3(592), dim3(256), 0, c->U_hi, c->U_lo, nn, U_out));
   CKL("combine");
+  return GPTQ_OK;
+}
+
+gptq_status gptq_get_dead_columns(gptq_ctx* c, uint8_t* dead_out) {
+  if (!c || !dead_out) return GPTQ_ERR_ARG;
+  if (c->state != ST_PREPARED) return GPTQ_ERR_STATE;
+  DeviceGuard dg(c->device);
+  CK(cudaMemcpyAsync(dead_out, c->dead, static_cast<size_t>(c->n), cudaMemcpyDeviceToDevice, c->stream));
+  return GPTQ_OK;
+}
+
+gptq_status gptq_set_profiling(gptq_ctx* c, int on) {
+  if (!c || (on != 0 && on != 1)) return GPTQ_ERR_ARG;
+  c->prof = on != 0;
+  return GPTQ_OK;
+}
+
+gptq_status gptq_get_profile(gptq_ctx* c, gptq_kernel_stat* out, int capacity, int* count) {
+  if (!c || capacity < 0 || (capacity > 0 && !out)) return GPTQ_ERR_ARG;
+  DeviceGuard dg(c->device);
+  gptq_status st = wait_stream(c);
+  if (st != GPTQ_OK) return st;
+  std::vector<gptq_kernel_stat> agg;
+  bool bad = c->prof_error;
+  for (const auto& r : c->prof_recs) {
+    float ms = 0.0f;
+    if (cudaEventElapsedTime(&ms, r.e0, r.e1) != cudaSuccess) {
+      bad = true;
+      cudaGetLastError();
+      continue;
+    }
+    gptq_kernel_stat* e = nullptr;
+    for (auto& a : agg)
+      if (std::strncmp(a.name, r.tag, sizeof(a.name)) == 0) e = &a;
+    if (!e) {
+      gptq_kernel_stat z{};
+      std::strncpy(z.name, r.tag, sizeof(z.name) - 1);
+      agg.push_back(z);
+      e = &agg.back();
+    }
+    e->launches += 1;
+    e->ms += ms;
+    e->flops += r.flops;
+    e->bytes += r.bytes;
+  }
+  free_prof(c);
+  c->prof_error = false;
+  for (int i = 0; i < capacity && i < static_cast<int>(agg.size()); ++i) out[i] = agg[i];
+  if (count) *count = static_cast<int>(agg.size());
+  return bad ? GPTQ_ERR_CUDA : GPTQ_OK;
+}
+
+gptq_status gptq_test_bounded_wait(gptq_ctx* c, uint64_t limit_ns) {
+  if (!c || limit_ns < 1 || limit_ns > 10000000000ull) return GPTQ_ERR_ARG;
+  DeviceGuard dg(c->device);
+  tag(c, "test:bounded_wait", 0.0, 0.0);
+  CK(launch(c, bounded_wait_probe_kernel, dim3(1), dim3(32), 0, limit_ns, c->status));
+  CKL("bounded_wait_probe");
   return GPTQ_OK;
 }
 
@@ -779,6 +921,7 @@ gptq_status gptq_quantize_layer(gptq_ctx* c, const void* W, int64_t m, gptq_qpar
   const int n = static_cast<int>(c->n);
   const int mi = static_cast<int>(m);
   const int g = (qp.group_size == -1) ? n : qp.group_size;
+  tag(c, "quantize:init_w", 0.0, 6.0 * static_cast<double>(m) * n);
   CK(launch(c, init_w_kernel, dim3(mi), dim3(256), static_cast<size_t>(n) * 2, static_cast<const __half*>(W), n, c->perm, c->dead,
                                                                    c->Wq));
   CKL("init_w");
@@ -801,6 +944,11 @@ gptq_status gptq_quantize_layer(gptq_ctx* c, const void* W, int64_t m, gptq_qpar
   a.G = n / g;
   a.ld_err = kSuperBlock;
   const int grid = (mi + SW_ROWS - 1) / SW_ROWS;
+  // algorithmic bytes of one sweep block: W tile in, scaled errors out (hi/lo), codes,
+  // scales/zeros of the groups that start in it, the U block (hi/lo)
+  const double sweep_bytes = 4.0 * mi * SW_B + 8.0 * mi * SW_B + mi * SW_B * qp.bits / 8.0 +
+                             8.0 * mi * std::max(1, SW_B / g) + 8.0 * SW_B * SW_B + (W_hat ? 4.0 * mi * SW_B : 0.0);
+  c->gemm_role = 1;
   // two-level lazy update: inside a super-block the columns after each 128-block are updated
   // right away; the columns beyond the super-block receive all its block errors in one product
   // (K = super-block width).  A group that starts inside a super-block must not reach past it.
@@ -809,6 +957,7 @@ gptq_status gptq_quantize_layer(gptq_ctx* c, const void* W, int64_t m, gptq_qpar
     const int s1 = std::min(n, s0 + sb);
     for (int i1 = s0; i1 < s1; i1 += SW_B) {
       a.err_col0 = i1 - s0;
+      tag(c, "sweep_block", 0.0, sweep_bytes);
       if (g >= SW_B)
         CK(launch(c, sweep_block_kernel<0>, dim3(grid), dim3(SW_THREADS), SW_SMEM, a, i1));
       else if (g == 64)
@@ -843,7 +992,9 @@ gptq_status gptq_quantize_layer(gptq_ctx* c, const void* W, int64_t m, gptq_qpar
       if (st != GPTQ_OK) return st;
     }
   }
+  c->gemm_role = 0;
   if (g_idx) {
+    tag(c, "quantize:g_idx", 0.0, 8.0 * n);
     CK(launch(c, g_idx_kernel, dim3((n + 255) / 256), dim3(256), 0, c->perm, n, g, g_idx));
     CKL("g_idx");
   }

@@ -78,16 +78,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Wait for the phase of parity `parity` of barrier `bar` to complete.  Gives up (returns
-// false) when *abort is set by another role or when the deadline passes; in the latter case
+// false) when *abort is set by another role or when limit_ns have passed; in the latter case
 // it sets *abort itself so the CTA's other roles stop too.
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 255u) == 0) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         *abort = 1;
         return false;
       }
@@ -122,6 +123,20 @@ __device__ __forceinline__ bool mbar_wait_bounded_cl(uint32_t bar, uint32_t pari
   }
 }
 
+// One CTA waits on a barrier nobody arrives on, with a short limit: the failure path of the
+// bounded wait (records ST_TIMEOUT and returns; used by the tests of failure detection).
+__global__ void bounded_wait_probe_kernel(uint64_t limit_ns, int* status) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !mbar_wait_bounded(smem_u32(&bar), 0u, &abort_flag, limit_ns)) atomicOr(status, ST_TIMEOUT);
+}
+
 // Wait without the abort shortcut (used to drain copies/MMAs still in flight before exit).
 __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
   const uint64_t t0 = globaltimer_ns();
@@ -132,7 +147,9 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
 }
 
 // ----------------------------------------------------------------------------------------
-// TMA (per-CTA tensor loads from this GPU's own memory; no cluster multicast anywhere)
+// TMA (per-CTA tensor loads from this GPU's own memory).  No TMA or bulk load uses cluster
+// multicast; the only multicast in this library is the CTA-pair MMA's completion signal
+// (tcgen05.commit ... multicast::cluster) to the two CTAs' barriers.
 // ----------------------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");

@@ -35,6 +35,11 @@ class QParams(ctypes.Structure):
     _fields_ = [("bits", ctypes.c_int), ("group_size", ctypes.c_int), ("sym", ctypes.c_int)]
 
 
+class KernelStat(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 40), ("launches", ctypes.c_int64), ("ms", ctypes.c_double),
+                ("flops", ctypes.c_double), ("bytes", ctypes.c_double)]
+
+
 _LIB = None
 _P = ctypes.c_void_p
 _SIGS = {
@@ -52,6 +57,10 @@ _SIGS = {
     "gptq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "gptq_set_hessian_chunk": (ctypes.c_int, [_P, ctypes.c_int64]),
     "gptq_launch_count": (ctypes.c_int64, [_P]),
+    "gptq_get_dead_columns": (ctypes.c_int, [_P, _P]),
+    "gptq_set_profiling": (ctypes.c_int, [_P, ctypes.c_int]),
+    "gptq_get_profile": (ctypes.c_int, [_P, ctypes.POINTER(KernelStat), ctypes.c_int, ctypes.POINTER(ctypes.c_int)]),
+    "gptq_test_bounded_wait": (ctypes.c_int, [_P, ctypes.c_uint64]),
     "gptq_quantize_layer_noalloc": (ctypes.c_int, [_P, ctypes.c_int64, ctypes.c_int64, _P, _P, _P, QParams,
                                                    _P, _P, _P, _P, _P, ctypes.c_int, _P]),
     "gptq_test_gemm_tf32x3": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P, ctypes.c_int, _P, _P,
@@ -160,6 +169,12 @@ class GPTQContext:
         _check(lib().gptq_prepare(self._h, float(damp), int(bool(desc_act)), _ptr(perm)), "gptq_prepare")
         return perm
 
+    def get_dead_columns(self) -> torch.Tensor:
+        """uint8 [n] mask (original column order) of the columns the last prepare found unexcited."""
+        d = torch.empty(self.n, dtype=torch.uint8, device=self.device)
+        _check(lib().gptq_get_dead_columns(self._h, _ptr(d)), "gptq_get_dead_columns")
+        return d
+
     def get_factor(self) -> torch.Tensor:
         U = torch.empty((self.n, self.n), dtype=torch.float32, device=self.device)
         _check(lib().gptq_get_factor(self._h, _ptr(U)), "gptq_get_factor")
@@ -192,6 +207,19 @@ class GPTQContext:
 
     def synchronize(self):
         _check(lib().gptq_synchronize(self._h), "gptq_synchronize")
+
+    # -- instrumentation ---------------------------------------------------------------------
+    def set_profiling(self, on: bool):
+        _check(lib().gptq_set_profiling(self._h, int(bool(on))), "gptq_set_profiling")
+
+    def get_profile(self) -> dict:
+        """{role: {"launches", "ms", "flops", "bytes"}} of the launches recorded since the last call."""
+        cap = 64
+        arr = (KernelStat * cap)()
+        cnt = ctypes.c_int()
+        _check(lib().gptq_get_profile(self._h, arr, cap, ctypes.byref(cnt)), "gptq_get_profile")
+        return {arr[i].name.decode(): {"launches": int(arr[i].launches), "ms": arr[i].ms, "flops": arr[i].flops,
+                                      "bytes": arr[i].bytes} for i in range(min(cap, cnt.value))}
 
     def launch_count(self) -> int:
         return int(lib().gptq_launch_count(self._h))

@@ -75,3 +75,11 @@ def test_binding_fails_loudly_when_library_missing(monkeypatch, tmp_path):
     monkeypatch.setattr(G, "_LIB", None)
     with pytest.raises(RuntimeError, match="not built"):
         G.lib()
+
+
+def test_new_calls_reject_a_null_context(L):
+    assert L.gptq_get_dead_columns(None, None) == G.ERR_ARG
+    assert L.gptq_set_profiling(None, 1) == G.ERR_ARG
+    cnt = ctypes.c_int()
+    assert L.gptq_get_profile(None, None, 0, ctypes.byref(cnt)) == G.ERR_ARG
+    assert L.gptq_test_bounded_wait(None, 1000) == G.ERR_ARG

@@ -44,8 +44,12 @@ def test_cpu_oracle_baseline_on_tiny_layer():
     r = bench.cpu_oracle_baseline(layer, qs, tok_sample=512, row_sample=32)
     assert r["value"] > 0 and r["kind"] == "oracle" and r["cores"] >= 1
     assert set(r["stage_seconds"]) == {"hessian", "prepare", "sweep"}
-    r2 = bench.cpu_oracle_baseline(layer, qs, tok_sample=256, row_sample=16, prep_n=256)
-    assert r2["value"] > 0 and "256 of 512 columns" in r2["sample"]
+    r2 = bench.cpu_oracle_baseline(layer, qs, tok_sample=256, row_sample=16, col_sample=256)
+    assert r2["value"] > 0 and "leading 256 of 512 columns" in r2["sample"]
+    # a wide layer stays bounded: only the leading columns are generated and timed
+    big, bq = synth.WORKLOADS["down_proj_8192x28672"]
+    r3 = bench.cpu_oracle_baseline(big, bq, tok_sample=256, row_sample=8, col_sample=256)
+    assert r3["value"] > 0 and r3["seconds_per_layer"] > r2["seconds_per_layer"]
 
 
 def test_reference_arm_line(capsys):
@@ -59,3 +63,31 @@ def test_reference_arm_line(capsys):
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
     bench.run_reference(args, 1, 2)  # other ranks do nothing
     assert capsys.readouterr().out == ""
+
+
+def test_peak_choice_follows_the_clocks():
+    peaks = {"bf16_tflops": 1644.2, "bf16_tflops_sustained": 1385.2, "hbm_gbs": 6468.0}
+    capped = {"sm_mhz": 1440.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    full = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
+    assert bench.choose_peak(peaks, 4.4, capped)[:2] == (1385.2, "sustained")
+    assert bench.choose_peak(peaks, 0.15, capped)[:2] == (1644.2, "burst")     # too short
+    assert bench.choose_peak(peaks, 4.4, full)[:2] == (1644.2, "burst")        # not capped
+    assert bench.choose_peak(peaks, 4.4, None)[:2] == (1644.2, "burst")
+
+
+def test_dominant_kernel_folds_roles():
+    prof = {"gemm_tf32x3:factor": {"launches": 10, "ms": 50.0, "flops": 1e13, "bytes": 0.0},
+            "gemm_tf32x3:trailing": {"launches": 20, "ms": 30.0, "flops": 5e12, "bytes": 0.0},
+            "hessian_syrk_pair": {"launches": 1, "ms": 45.0, "flops": 5e13, "bytes": 4e9},
+            "sweep_block": {"launches": 224, "ms": 10.0, "flops": 0.0, "bytes": 3e9}}
+    name, k = bench.dominant_kernel(prof)
+    assert name == "gemm_tf32x3" and k["ms"] == 80.0 and k["launches"] == 30 and k["flops"] == 1.5e13
+    assert sorted(k["roles"]) == ["gemm_tf32x3:factor", "gemm_tf32x3:trailing"]
+
+
+def test_path_rooflines_of_the_q_proj_layer():
+    layer, qs = synth.WORKLOADS["q_proj_4096x4096"]
+    t_bf16, t_prec, work = bench.path_rooflines(layer, qs, 1644.2, 6468.0)
+    assert abs(work["hessian"] - 4.399e12) / 4.399e12 < 1e-3
+    assert abs(t_bf16 * 1e3 - 2.74) < 0.01          # every product at the bf16 peak
+    assert t_prec > t_bf16                            # fp32-faithful products at the tf32 rate / 3

@@ -1,0 +1,85 @@
+"""Failure detection on the GPU without a GPU fault: a device-side bounded wait that runs out
+(an mbarrier nothing arrives on, with a 1 ms limit) is reported as GPTQ_ERR_TIMEOUT by the
+next gptq_synchronize and leaves the context usable; a host wait with a short limit returns
+GPTQ_ERR_TIMEOUT while a kernel is still running.  Also the per-kernel instrumentation, which
+must not change any result."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import gptq_oracle as O
+from post_weight_quantization_16_b200 import synth
+from post_weight_quantization_16_b200 import gptq as G
+from tests import gpu_helpers as GH
+
+pytestmark = pytest.mark.gpu
+TINY = synth.WORKLOADS["tiny_256x512"][0]
+
+
+def _small_run(ctx, layer, qs, X, W):
+    ctx.reset()
+    ctx.accumulate_hessian(GH.bf16_to_dev(X))
+    perm = ctx.prepare(qs.damp, qs.desc_act)
+    out = ctx.quantize_layer(torch.from_numpy(W).to(GH.DEV), qs.bits, qs.group_size, qs.sym)
+    ctx.synchronize()
+    return perm.cpu().numpy(), {k: v.cpu().numpy() for k, v in out.items() if v is not None}
+
+
+def test_device_wait_that_runs_out_is_reported_and_the_context_survives():
+    layer = synth.scaled_layer(TINY, m=64, n=256, n_tok=512)
+    qs = synth.QuantSetting(4, 128, False, 0.01, True)
+    X, W = synth.make_x_bf16(layer), synth.make_w_fp16(layer)
+    with G.GPTQContext(layer.n, layer.m, 0) as ctx:
+        perm0, ref = _small_run(ctx, layer, qs, X, W)
+        assert G.lib().gptq_test_bounded_wait(ctx._h, 1_000_000) == G.OK   # 1 ms
+        with pytest.raises(G.GPTQError) as ei:
+            ctx.synchronize()
+        assert ei.value.status == G.ERR_TIMEOUT
+        ctx.synchronize()                       # the status word was cleared
+        perm1, out = _small_run(ctx, layer, qs, X, W)
+        assert np.array_equal(perm0, perm1)
+        for k in ref:
+            assert np.array_equal(ref[k], out[k]), k
+
+
+def test_host_wait_with_a_short_limit_returns_timeout(monkeypatch):
+    with G.GPTQContext(256, 16, 0) as ctx:
+        assert G.lib().gptq_test_bounded_wait(ctx._h, 300_000_000) == G.OK  # a 300 ms kernel
+        monkeypatch.setenv("GPTQ_SYNC_TIMEOUT_MS", "5")
+        with pytest.raises(G.GPTQError) as ei:
+            ctx.synchronize()                   # the host gives up after 5 ms
+        assert ei.value.status == G.ERR_TIMEOUT
+        monkeypatch.delenv("GPTQ_SYNC_TIMEOUT_MS")
+        with pytest.raises(G.GPTQError) as ei:
+            ctx.synchronize()                   # the kernel itself gave up and said so
+        assert ei.value.status == G.ERR_TIMEOUT
+        ctx.synchronize()
+
+
+def test_profiling_records_every_role_and_changes_no_result():
+    layer = synth.scaled_layer(TINY, m=96, n=1024, n_tok=2048)
+    qs = synth.QuantSetting(4, 128, False, 0.01, True)
+    X, W = synth.make_x_bf16(layer), synth.make_w_fp16(layer)
+    with G.GPTQContext(layer.n, layer.m, 0) as ctx:
+        perm0, ref = _small_run(ctx, layer, qs, X, W)
+        ctx.set_profiling(True)
+        perm1, out = _small_run(ctx, layer, qs, X, W)
+        prof = ctx.get_profile()
+        ctx.set_profiling(False)
+        assert ctx.get_profile() == {}
+    assert np.array_equal(perm0, perm1)
+    for k in ref:
+        assert np.array_equal(ref[k], out[k]), k
+    n = layer.n
+    assert prof["hessian_syrk_pair"]["launches"] == 1
+    assert prof["hessian_syrk_pair"]["flops"] == layer.n_tok * n * (n + 1)
+    assert prof["leaf_chol_inv"]["launches"] == n // 128
+    assert prof["sweep_block"]["launches"] == n // 128
+    # the factorization's algorithmic work: n^3/3 for the Cholesky factor and n^3/3 for its
+    # inverse, plus lower-order terms of the diagonals
+    f = sum(v["flops"] for k, v in prof.items() if k.endswith(":factor") or k == "leaf_chol_inv")
+    assert 2 * n ** 3 / 3 <= f <= 1.02 * 2 * n ** 3 / 3, f
+    # the trailing update: 2 m sum over blocks of 128 (n - i2)
+    t = sum(v["flops"] for k, v in prof.items() if k.endswith(":trailing"))
+    assert t == 2 * layer.m * sum(128 * (n - i2) for i2 in range(128, n, 128))
+    assert all(v["ms"] > 0 for v in prof.values())
