@@ -106,11 +106,39 @@ def upper_cholesky_of_inverse(Hd) -> np.ndarray:
         raise NotPositiveDefinite(str(exc)) from None
 
 
-def prepare(H, damp: float, desc_act: bool) -> dict:
-    """Steps S2-S4 on an accumulated H (any scale).
+def upper_cholesky_of_inverse_leading(Hd, k: int) -> np.ndarray:
+    """The leading k x k block of U = upper_cholesky_of_inverse(Hd), without forming all of U.
 
-    Returns ``dead`` (bool [n]), ``perm`` (int [n]: sweep position k holds original
-    column perm[k]), ``Hd`` (damped, permuted H) and ``U``.
+    U is upper-triangular, so column j < k of U has no entries below row j and the leading
+    block of H^-1 = U^T U is U[:k, :k]^T U[:k, :k]: U[:k, :k] is the upper Cholesky factor of
+    (H^-1)[:k, :k], whose columns come from a Cholesky solve of H against the first k unit
+    vectors.
+    """
+    Hd = np.asarray(Hd, dtype=np.float64)
+    n = Hd.shape[0]
+    try:
+        c = scipy.linalg.cho_factor(Hd, lower=True)
+    except np.linalg.LinAlgError as exc:
+        raise NotPositiveDefinite(str(exc)) from None
+    E = np.zeros((n, k))
+    E[np.arange(k), np.arange(k)] = 1.0
+    Y = scipy.linalg.cho_solve(c, E)[:k]
+    Y = 0.5 * (Y + Y.T)
+    return np.linalg.cholesky(Y).T.copy()
+
+
+def upper_cholesky_of_inverse_trailing(Hd, k: int) -> np.ndarray:
+    """The trailing k x k block of U = upper_cholesky_of_inverse(Hd), which depends only on
+    the trailing k x k block of Hd: with H = V V^T, V upper, the trailing block of V V^T is
+    V22 V22^T, and U = V^-1 has U22 = V22^-1, the factor of Hd[-k:, -k:] alone."""
+    Hd = np.asarray(Hd, dtype=np.float64)
+    return upper_cholesky_of_inverse(Hd[-k:, -k:])
+
+
+def prepare_order(H, damp: float, desc_act: bool) -> dict:
+    """Steps S2-S3 and the damping of S4 on an accumulated H (any scale): ``dead`` (bool [n]),
+    ``perm`` (int [n]: sweep position k holds original column perm[k]), ``Hd`` (damped,
+    permuted H) and ``mean_diag``.
     Damping: H += damp * mean(diag H) * I  ([P4] §3.2 prepare; [P3] §3.3 damp_percent).
     """
     H1 = np.array(H, dtype=np.float64)
@@ -119,10 +147,17 @@ def prepare(H, damp: float, desc_act: bool) -> dict:
     H1[dead, dead] = 1.0
     perm = act_order(H1) if desc_act else np.arange(n)
     mean_diag = float(np.mean(np.diag(H1)))
-    H2 = H1 + damp * mean_diag * np.eye(n)
-    Hd = H2[np.ix_(perm, perm)]
-    U = upper_cholesky_of_inverse(Hd)
-    return {"dead": dead, "perm": perm, "Hd": Hd, "U": U, "mean_diag": mean_diag}
+    H1[np.arange(n), np.arange(n)] += damp * mean_diag
+    Hd = H1[np.ix_(perm, perm)]
+    return {"dead": dead, "perm": perm, "Hd": Hd, "mean_diag": mean_diag}
+
+
+def prepare(H, damp: float, desc_act: bool) -> dict:
+    """Steps S2-S4 on an accumulated H (any scale): prepare_order, then U, the upper
+    Cholesky factor of the damped, permuted H's inverse."""
+    p = prepare_order(H, damp, desc_act)
+    p["U"] = upper_cholesky_of_inverse(p["Hd"])
+    return p
 
 
 # ==================================================================================

@@ -69,7 +69,7 @@ struct gptq_ctx {
   bool pdl = true;                        // launches overlap their predecessor (programmatic)
   cudaGraphExec_t factor_graph = nullptr;  // the factorization recursion, recorded once
   int64_t factor_graph_launches = 0;
-  int gemm_role = 0;                      // 0: factorization product, 1: trailing update (instrumentation)
+  int gemm_role = 0;                      // which product gemm_tc runs (instrumentation): GR_*
   PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
   // per-kernel instrumentation (gptq_set_profiling): the role and algorithmic work of the next
   // launch, and one record (two timing events) per launch while profiling is on
@@ -268,6 +268,17 @@ struct TcOperand {
   int ld;
 };
 
+// Roles of the products gemm_tc runs (instrumentation names: kernel:role).
+enum : int { GR_V12 = 0, GR_SYRK, GR_T, GR_U12, GR_NEAR, GR_FAR, GR_TEST, GR_COUNT };
+const char* const kGemmTcNames[GR_COUNT] = {"gemm_tf32x3:factor_v12",    "gemm_tf32x3:factor_syrk",
+                                            "gemm_tf32x3:factor_t",      "gemm_tf32x3:factor_u12",
+                                            "gemm_tf32x3:trailing_near", "gemm_tf32x3:trailing_far",
+                                            "gemm_tf32x3:test"};
+const char* const kGemmSimtNames[GR_COUNT] = {"gemm_hilo_simt:factor_v12",    "gemm_hilo_simt:factor_syrk",
+                                              "gemm_hilo_simt:factor_t",      "gemm_hilo_simt:factor_u12",
+                                              "gemm_hilo_simt:trailing_near", "gemm_hilo_simt:trailing_far",
+                                              "gemm_hilo_simt:test"};
+
 // Products with fewer tensor-core tiles (at the narrowest tile) than this run on the CUDA
 // cores (fp32, 32 x 32 or 64 x 64 tiles).
 constexpr int kMinTcTiles = 32;
@@ -350,8 +361,7 @@ gptq_status gemm_tc(gptq_ctx* c, int M, int N, int K, TcOperand A, TcOperand B, 
     g.Cthi = o.Cthi;
     g.Ctlo = o.Ctlo;
     g.ldt = o.ldt;
-    tag(c, c->gemm_role ? "gemm_hilo_simt:trailing" : "gemm_hilo_simt:factor",
-        gemm_algo_flops(M, N, K, klo, khi, upper), 0.0);
+    tag(c, kGemmSimtNames[c->gemm_role], gemm_algo_flops(M, N, K, klo, khi, upper), 0.0);
     if (static_cast<int64_t>(M) * N <= 512 * 512) {  // 32 x 32 tiles: more CTAs for the smallest products
       dim3 grid((N + 31) / 32, (M + 31) / 32);
       CK(launch(c, gemm_hilo_simt_kernel<32, 32>, grid, dim3(GS_THREADS), gs_smem_bytes<32, 32>(), g));
@@ -391,7 +401,7 @@ gptq_status gemm_tc(gptq_ctx* c, int M, int N, int K, TcOperand A, TcOperand B, 
   if (o.c_map && (beta != 1 || !o.C)) return GPTQ_ERR_ARG;
   const CUtensorMap& cm = o.c_map ? *o.c_map : *A.hi;  // unused unless c_reduce
   const dim3 grid(std::min(tc_tiles, c->num_sms));
-  tag(c, c->gemm_role ? "gemm_tf32x3:trailing" : "gemm_tf32x3:factor", gemm_algo_flops(M, N, K, klo, khi, upper), 0.0);
+  tag(c, kGemmTcNames[c->gemm_role], gemm_algo_flops(M, N, K, klo, khi, upper), 0.0);
   if (bn == 256)
     CK(launch(c, gemm_tf32x3_kernel<256>, grid, dim3(GT_THREADS), GtCfg<256>::SMEM, *A.hi, *A.lo, *B.hi, *B.lo, cm, a));
   else if (bn == 128)
@@ -446,6 +456,7 @@ gptq_status chol_inv(gptq_ctx* c, int o, int h) {
   v12.Chi = at(c->VT_hi, o, o2);
   v12.Clo = at(c->VT_lo, o, o2);
   v12.ldh = n;
+  c->gemm_role = GR_V12;
   if ((s = gemm_tc(c, h1, h2, h2, op(c->mA_A, c->A_hi, c->A_lo, o, o2), op(c->mB_U, c->U_hi, c->U_lo, o2, o2), 1.f, 0, GT_KLO_COL, GT_KHI_NONE, 0,
                    v12)) != GPTQ_OK)
     return s;
@@ -454,6 +465,7 @@ gptq_status chol_inv(gptq_ctx* c, int o, int h) {
   a11.Chi = at(c->A_hi, o, o);
   a11.Clo = at(c->A_lo, o, o);
   a11.ldh = n;
+  c->gemm_role = GR_SYRK;
   if ((s = gemm_tc(c, h1, h1, h2, op(c->mA_VT, c->VT_hi, c->VT_lo, o, o2), op(c->mB_VT, c->VT_hi, c->VT_lo, o, o2), -1.f, 1, GT_KLO_NONE, GT_KHI_NONE, 1,
                    a11)) != GPTQ_OK)
     return s;
@@ -472,6 +484,7 @@ gptq_status chol_inv(gptq_ctx* c, int o, int h) {
     c->stream = c->side_stream;
     c->pdl = false;
   }
+  c->gemm_role = GR_T;
   s = gemm_tc(c, h1, h2, h2, op(c->mA_VT, c->VT_hi, c->VT_lo, o, o2), op(c->mB_Ut, c->Ut_hi, c->Ut_lo, o2, o2), 1.f, 0,
               GT_KLO_NONE, GT_KHI_COL, 0, tt);
   if (branch) {
@@ -491,6 +504,7 @@ gptq_status chol_inv(gptq_ctx* c, int o, int h) {
   u12.Cthi = at(c->Ut_hi, o2, o);
   u12.Ctlo = at(c->Ut_lo, o2, o);
   u12.ldt = n;
+  c->gemm_role = GR_U12;
   if ((s = gemm_tc(c, h1, h2, h1, op(c->mA_U, c->U_hi, c->U_lo, o, o), op(c->mB_VT, c->VT_hi, c->VT_lo, o2, o), -1.f, 0, GT_KLO_ROW, GT_KHI_NONE, 0,
                    u12)) != GPTQ_OK)
     return s;
@@ -525,7 +539,6 @@ gptq_status encode_maps(gptq_ctx* c) {
 // Run the factorization recursion: recorded as a CUDA graph on first use (on a private
 // stream), then replayed on the context's stream.
 gptq_status run_factorization(gptq_ctx* c) {
-  c->gemm_role = 0;
   if (c->prof) {  // instrumented: every launch on its own, timed, on the context's stream
     cudaStream_t side = c->side_stream;
     c->side_stream = nullptr;
@@ -782,7 +795,7 @@ static gptq_status ensure_mirrored(gptq_ctx* c) {
   if (c->mirrored) return GPTQ_OK;
   const int n = static_cast<int>(c->n);
   tag(c, "prepare:mirror", 0.0, 4.0 * n * n);
-  CK(launch(c, mirror_upper_kernel, dim3(n / 32, n / 32), dim3(32, 8), 0, c->H, n));
+  CK(launch(c, mirror_upper_kernel, dim3(n / MIR_T, n / MIR_T), dim3(32, 8), 0, c->H, n));
   CKL("mirror");
   c->mirrored = 1;
   return GPTQ_OK;
@@ -828,7 +841,7 @@ gptq_status gptq_prepare(gptq_ctx* c, double damp, int desc_act, int32_t* perm_o
     CK(launch(c, identity_perm_kernel, dim3((n + 255) / 256), dim3(256), 0, n, c->perm));
   CKL("perm");
   tag(c, "prepare:gather_damp", 0.0, 12.0 * n * n);
-  CK(launch(c, gather_damp_kernel, dim3(n), dim3(256), static_cast<size_t>(n) * 4, c->H, n, c->perm, c->keys, c->mean, damp,
+  CK(launch(c, gather_damp_kernel, dim3(n), dim3(GD_THREADS), static_cast<size_t>(n) * 4, c->H, n, c->perm, c->keys, c->mean, damp,
                                                                         c->A_hi, c->A_lo));
   CKL("gather");
   const size_t nn = static_cast<size_t>(n) * n;
@@ -948,7 +961,6 @@ gptq_status gptq_quantize_layer(gptq_ctx* c, const void* W, int64_t m, gptq_qpar
   // scales/zeros of the groups that start in it, the U block (hi/lo)
   const double sweep_bytes = 4.0 * mi * SW_B + 8.0 * mi * SW_B + mi * SW_B * qp.bits / 8.0 +
                              8.0 * mi * std::max(1, SW_B / g) + 8.0 * SW_B * SW_B + (W_hat ? 4.0 * mi * SW_B : 0.0);
-  c->gemm_role = 1;
   // two-level lazy update: inside a super-block the columns after each 128-block are updated
   // right away; the columns beyond the super-block receive all its block errors in one product
   // (K = super-block width).  A group that starts inside a super-block must not reach past it.
@@ -973,6 +985,7 @@ gptq_status gptq_quantize_layer(gptq_ctx* c, const void* W, int64_t m, gptq_qpar
         w.ldc = n;
         w.c_map = &c->mC_Wq;
         w.c_col0 = i2;
+        c->gemm_role = GR_NEAR;
         gptq_status st = gemm_tc(c, mi, s1 - i2, SW_B, TcOperand{&c->mA_Err[0], &c->mA_Err[1], 0, i1 - s0, nullptr, nullptr, 0},
                                  TcOperand{&c->mB_Ut[0], &c->mB_Ut[1], i2, i1, nullptr, nullptr, 0}, -1.f, 1,
                                  GT_KLO_NONE, GT_KHI_NONE, 0, w, SW_B / GT_BK);
@@ -986,13 +999,13 @@ gptq_status gptq_quantize_layer(gptq_ctx* c, const void* W, int64_t m, gptq_qpar
       w.ldc = n;
       w.c_map = &c->mC_Wq;
       w.c_col0 = s1;
+      c->gemm_role = GR_FAR;
       gptq_status st = gemm_tc(c, mi, n - s1, s1 - s0, TcOperand{&c->mA_Err[0], &c->mA_Err[1], 0, 0, nullptr, nullptr, 0},
                                TcOperand{&c->mB_Ut[0], &c->mB_Ut[1], s1, s0, nullptr, nullptr, 0}, -1.f, 1,
                                GT_KLO_NONE, GT_KHI_NONE, 0, w, SW_B / GT_BK);
       if (st != GPTQ_OK) return st;
     }
   }
-  c->gemm_role = 0;
   if (g_idx) {
     tag(c, "quantize:g_idx", 0.0, 8.0 * n);
     CK(launch(c, g_idx_kernel, dim3((n + 255) / 256), dim3(256), 0, c->perm, n, g, g_idx));
@@ -1061,6 +1074,7 @@ gptq_status gptq_test_gemm_tf32x3(int M, int N, int K, const float* A_hi, const 
   o.ldt = ldt;
   CUtensorMap ma[2], mb[2], mc;
   gptq_status s = GPTQ_OK;
+  t.gemm_role = GR_TEST;
   if (c_reduce) {
     s = make_map(&t, &mc, C, M, N, ldc, 32);
     o.c_map = &mc;

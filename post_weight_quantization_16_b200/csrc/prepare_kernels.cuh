@@ -18,20 +18,25 @@
 
 namespace gptq {
 
-__global__ void mirror_upper_kernel(float* __restrict__ H, int n) {
+// 64 x 64 tiles, 256 threads: a tile of the upper triangle is staged in shared memory and
+// written transposed into the lower triangle (the diagonal tile only below its diagonal).
+constexpr int MIR_T = 64;
+__global__ void __launch_bounds__(256) mirror_upper_kernel(float* __restrict__ H, int n) {
   griddep_wait();
   griddep_launch_dependents();
-  __shared__ float t[32][33];
+  __shared__ float t[MIR_T][MIR_T + 1];
   const int tr = blockIdx.y, tc = blockIdx.x;
   if (tr > tc) return;
   const int x = threadIdx.x, y = threadIdx.y;  // 32 x 8
-  for (int k = y; k < 32; k += 8) t[k][x] = H[static_cast<size_t>(tr * 32 + k) * n + tc * 32 + x];
+  for (int k = y; k < MIR_T; k += 8)
+    for (int c = x; c < MIR_T; c += 32) t[k][c] = H[static_cast<size_t>(tr * MIR_T + k) * n + tc * MIR_T + c];
   __syncthreads();
-  // write the transpose into block (tc, tr); on the diagonal block only the strictly lower part
-  for (int k = y; k < 32; k += 8) {
-    const int r = tc * 32 + k, c = tr * 32 + x;
-    if (r > c) H[static_cast<size_t>(r) * n + c] = t[x][k];
-  }
+  // block (tc, tr) receives the transpose; on the diagonal tile only the strictly lower part
+  for (int k = y; k < MIR_T; k += 8)
+    for (int c = x; c < MIR_T; c += 32) {
+      const int r = tc * MIR_T + k, col = tr * MIR_T + c;
+      if (r > col) H[static_cast<size_t>(r) * n + col] = t[c][k];
+    }
 }
 
 // One CTA of 1024 threads.
@@ -88,10 +93,15 @@ __global__ void identity_perm_kernel(int n, int32_t* __restrict__ perm) {
   if (i < n) perm[i] = i;
 }
 
-// One CTA per output row a; the source row perm[a] of the (mirrored) H is staged in smem.
-__global__ void gather_damp_kernel(const float* __restrict__ H, int n, const int32_t* __restrict__ perm,
-                                   const float* __restrict__ keys, const double* __restrict__ mean,
-                                   double damp, float* __restrict__ A_hi, float* __restrict__ A_lo) {
+// One CTA (1024 threads) per output row a: the source row perm[a] of the (mirrored) H is
+// staged in shared memory, then gathered by perm four columns at a time (16-byte loads of
+// perm, 16-byte stores of the hi and lo parts).  n % 4 == 0.
+constexpr int GD_THREADS = 1024;
+__global__ void __launch_bounds__(GD_THREADS) gather_damp_kernel(const float* __restrict__ H, int n,
+                                                                 const int32_t* __restrict__ perm,
+                                                                 const float* __restrict__ keys,
+                                                                 const double* __restrict__ mean, double damp,
+                                                                 float* __restrict__ A_hi, float* __restrict__ A_lo) {
   griddep_wait();
   griddep_launch_dependents();
   extern __shared__ float row_s[];
@@ -99,18 +109,23 @@ __global__ void gather_damp_kernel(const float* __restrict__ H, int n, const int
   const int pa = perm[a];
   const float4* src = reinterpret_cast<const float4*>(H + static_cast<size_t>(pa) * n);
   for (int k = threadIdx.x; k < n / 4; k += blockDim.x) reinterpret_cast<float4*>(row_s)[k] = src[k];
+  const float dval = static_cast<float>(static_cast<double>(keys[pa]) + damp * (*mean));
   __syncthreads();
-  float* dh = A_hi + static_cast<size_t>(a) * n;
-  float* dl = A_lo + static_cast<size_t>(a) * n;
-  for (int b = threadIdx.x; b < n; b += blockDim.x) {
-    float v;
-    if (b == a)
-      v = static_cast<float>(static_cast<double>(keys[pa]) + damp * (*mean));
-    else
-      v = row_s[perm[b]];
-    const float hi = tf32_round(v);
-    dh[b] = hi;
-    dl[b] = tf32_round(v - hi);
+  float4* dh = reinterpret_cast<float4*>(A_hi + static_cast<size_t>(a) * n);
+  float4* dl = reinterpret_cast<float4*>(A_lo + static_cast<size_t>(a) * n);
+  const int4* p4 = reinterpret_cast<const int4*>(perm);
+  for (int b4 = threadIdx.x; b4 < n / 4; b4 += blockDim.x) {
+    const int4 pb = p4[b4];
+    float v[4] = {row_s[pb.x], row_s[pb.y], row_s[pb.z], row_s[pb.w]};
+    float hi[4], lo[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (4 * b4 + e == a) v[e] = dval;
+      hi[e] = tf32_round(v[e]);
+      lo[e] = tf32_round(v[e] - hi[e]);
+    }
+    dh[b4] = make_float4(hi[0], hi[1], hi[2], hi[3]);
+    dl[b4] = make_float4(lo[0], lo[1], lo[2], lo[3]);
   }
 }
 

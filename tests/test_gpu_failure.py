@@ -77,9 +77,9 @@ def test_profiling_records_every_role_and_changes_no_result():
     assert prof["sweep_block"]["launches"] == n // 128
     # the factorization's algorithmic work: n^3/3 for the Cholesky factor and n^3/3 for its
     # inverse, plus lower-order terms of the diagonals
-    f = sum(v["flops"] for k, v in prof.items() if k.endswith(":factor") or k == "leaf_chol_inv")
+    f = sum(v["flops"] for k, v in prof.items() if ":factor" in k or k == "leaf_chol_inv")
     assert 2 * n ** 3 / 3 <= f <= 1.02 * 2 * n ** 3 / 3, f
     # the trailing update: 2 m sum over blocks of 128 (n - i2)
-    t = sum(v["flops"] for k, v in prof.items() if k.endswith(":trailing"))
+    t = sum(v["flops"] for k, v in prof.items() if ":trailing" in k)
     assert t == 2 * layer.m * sum(128 * (n - i2) for i2 in range(128, n, 128))
     assert all(v["ms"] > 0 for v in prof.values())

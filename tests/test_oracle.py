@@ -501,3 +501,23 @@ def test_dequant_matmul_equals_sum_in_sweep_order():
             for k in range(n):
                 acc += X[t, perm[k]] * (codes[r, k] - float(z[r, k // g])) * float(s[r, k // g])
             assert abs(Y[t, r] - acc) <= 1e-12 * (1 + abs(acc))
+
+
+# ----------------------------------------------------------------------------------------
+# blocks of U without forming all of it (the full-width parity checks use them)
+# ----------------------------------------------------------------------------------------
+@pytest.mark.parametrize("n,k", [(64, 16), (96, 32), (40, 40)])
+def test_leading_and_trailing_blocks_of_U(n, k):
+    H = _spd(n, 5, cond_boost=10.0)
+    p = O.prepare(H, 0.01, True)
+    U = p["U"]
+    assert np.allclose(O.upper_cholesky_of_inverse_leading(p["Hd"], k), U[:k, :k], rtol=1e-10, atol=1e-14)
+    assert np.allclose(O.upper_cholesky_of_inverse_trailing(p["Hd"], k), U[-k:, -k:], rtol=1e-10, atol=1e-14)
+
+
+def test_prepare_order_is_prepare_without_the_factor():
+    H = _spd(48, 8)
+    H[7, :] = H[:, 7] = 0.0
+    a, b = O.prepare_order(H, 0.1, True), O.prepare(H, 0.1, True)
+    assert np.array_equal(a["perm"], b["perm"]) and np.array_equal(a["dead"], b["dead"])
+    assert np.array_equal(a["Hd"], b["Hd"]) and a["mean_diag"] == b["mean_diag"]

@@ -92,8 +92,9 @@ def test_noalloc_matches_oracle_and_context_path_on_two_calls(bits, g, sym, want
         rs, rep = GH.check_sweep_replay(W, prep, gpu, qs)
         GH.assert_replay_ok(rs, rep, gpu)
         assert np.array_equal(out["g_idx"].cpu().numpy(), O.g_idx(prep["perm"], qs.group_size)), call
-        # and the context path's outputs
-        same = (out["codes"] == ref["codes"]).float().mean().item()
+        # and the context path's outputs (codes compared one by one, not as packed words)
+        ref_codes = O.unpack_codes(ref["codes"].cpu().numpy().view(np.uint32), layer.n, qs.bits)
+        same = float(np.mean(gpu["codes"] == ref_codes))
         assert same >= GH.CODES_IDENTICAL, (call, same)
         assert torch.equal(out["zeros"], ref["zeros"]), call
         if want_what:
