@@ -318,6 +318,7 @@ def run_gpu(args, rank, world, local_rank):
     stream = torch.cuda.current_stream(dev)
     ctx = G.GPTQContext(layer.n, layer.m, local_rank, stream)
     out = None
+    perm_holder = [None]
 
     def step(timing=None):
         nonlocal out
@@ -327,7 +328,7 @@ def run_gpu(args, rank, world, local_rank):
         ctx.accumulate_hessian(X)
         if timing is not None:
             timing[1].record(stream)
-        ctx.prepare(qs.damp, qs.desc_act)
+        perm_holder[0] = ctx.prepare(qs.damp, qs.desc_act)
         if timing is not None:
             timing[2].record(stream)
         out = ctx.quantize_layer(W, qs.bits, qs.group_size, bool(qs.sym), want_w_hat=False, out=out)
@@ -402,6 +403,9 @@ def run_gpu(args, rank, world, local_rank):
                         "peak_source": f"{peaks_src} bf16 dense {peak_kind}"}
     t_roof, t_prec, work = path_rooflines(layer, qs, peak, peaks["hbm_gbs"])
 
+    # the packed result's consumer on this layer's own output (W4A16 product)
+    w4a16 = None if args.no_w4a16 else w4a16_measure(G, out, perm_holder[0], layer, qs, dev, stream, peaks, peak)
+
     # end to end through the public API with host buffers (pinned), copies inside the timed region
     e2e_ms = None
     G_ = n // (n if qs.group_size == -1 else qs.group_size)
@@ -438,6 +442,7 @@ def run_gpu(args, rank, world, local_rank):
             "roofline": roofline,
             "hessian_roofline": hessian_roofline,
             "kernels": prof,
+            "w4a16": w4a16,
             "e2e": None if e2e_ms is None else {
                 "value": world * weights / (e2e_ms / 1e3) / 1e9, "unit": "Gweights/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
@@ -450,6 +455,46 @@ def run_gpu(args, rank, world, local_rank):
         import torch.distributed as dist
         dist.barrier()
         dist.destroy_process_group()
+
+
+def w4a16_measure(G, out, perm, layer, qs, dev, stream, peaks, peak_bf16, reps=8):
+    """Y = X W16^T from the step's packed codes (gptq_dequant_matmul) for a decode-sized and a
+    prefill-sized batch of fp16 activations; each launch timed alone with CUDA events, L2
+    flushed (a 256 MB write) before every repetition."""
+    import torch
+    n, m = layer.n, layer.m
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    res = {}
+    for T in (16, 4096):
+        X = torch.randn((T, n), device=dev, dtype=torch.float32).to(torch.float16)
+        Y = torch.empty((T, m), dtype=torch.float32, device=dev)
+        ws = torch.empty(int(G.lib().gptq_dequant_matmul_workspace_bytes(T, m, n, 1)), dtype=torch.uint8, device=dev)
+        ms = []
+        for r in range(reps + 2):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            G.dequant_matmul(X, out["codes"], out["scales"], out["zeros"], perm, qs.bits, qs.group_size, out=Y,
+                             workspace=ws, stream=stream)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            if r >= 2:
+                ms.append(e0.elapsed_time(e1))
+        t = statistics.median(ms)
+        g = n if qs.group_size == -1 else qs.group_size
+        byts = m * n * qs.bits / 8 + 8 * m * (n // g) + 2 * T * n + 4 * T * m + 4 * n
+        flops = 2.0 * T * m * n
+        if T <= 64:
+            ach = byts / (t / 1e3) / 1e9
+            res[f"T{T}"] = {"ms": t, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                            "frac": ach / peaks["hbm_gbs"], "algorithmic_bytes": byts}
+        else:
+            ach = flops / (t / 1e3) / 1e12
+            res[f"T{T}"] = {"ms": t, "bound": "tensor", "achieved": ach, "peak": peak_bf16, "unit": "TFLOP/s",
+                            "frac": ach / peak_bf16, "algorithmic_flops": flops}
+    res["note"] = ("fp16 activations x fp16-dequantized weights, fp32 accumulation; act-order gather included; "
+                   "median of %d launches, L2 flushed before each" % reps)
+    return res
 
 
 def e2e_run(ctx, Xh, Wh, qs, dev, stream, reps=2, batch_tokens=16384):
@@ -505,19 +550,85 @@ def e2e_run(ctx, Xh, Wh, qs, dev, stream, reps=2, batch_tokens=16384):
     return statistics.mean(times[1:])
 
 
+def run_block(args, rank, world, local_rank):
+    """The 7B-shaped block sweep as one pipelined call per step: seven layers with their own
+    calibration sets (65536 tokens each), each quantized under the 18 settings of bits x
+    group_size x damp (126 quantize runs, 14 factorizations, 7 Hessians).  The same jobs run
+    one layer at a time through the context calls give the sequential time for comparison."""
+    import torch
+    from post_weight_quantization_16_b200 import build as B
+    from post_weight_quantization_16_b200 import gptq as G
+    B.build()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    layers = synth.block7b_layers()
+    settings = synth.block7b_settings()
+    Xs = [torch.from_numpy(synth.make_x_bf16(L).view(np.int16)).to(dev).view(torch.bfloat16) for L in layers]
+    Ws = [torch.from_numpy(synth.make_w_fp16(L)).to(dev) for L in layers]
+    jobs = [dict(X=X, W=W, bits=q.bits, group_size=q.group_size, sym=q.sym, damp=q.damp, desc_act=q.desc_act)
+            for X, W in zip(Xs, Ws) for q in settings]
+    weights = sum(j["W"].shape[0] * j["W"].shape[1] for j in jobs)
+
+    def sequential():
+        for X, W in zip(Xs, Ws):
+            with G.GPTQContext(W.shape[1], W.shape[0], local_rank, stream) as ctx:
+                ctx.accumulate_hessian(X)
+                for damp in (0.01, 0.1):
+                    ctx.prepare(damp, True)
+                    for q in settings:
+                        if q.damp == damp:
+                            ctx.quantize_layer(W, q.bits, q.group_size, q.sym, want_w_hat=False)
+                ctx.synchronize()
+
+    def timed(fn, k, w):
+        for _ in range(w):
+            fn()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(k):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / k
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    ms = timed(lambda: G.quantize_layers(jobs, local_rank, stream), args.steps, args.warmup)
+    clk = clocks.stop()
+    ms_seq = timed(sequential, max(1, args.steps // 2), 1)
+    line = {
+        "metric": METRIC, "value": weights / (ms / 1e3) / 1e9, "unit": "Gweights/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16->f32", "data": "synthetic",
+        "config": {"workload": "block7b: q,k,v,o 4096x4096, gate,up 11008x4096, down 4096x11008; 65536 tokens "
+                               "each; 18 settings (bits 2/3/4 x group 64/128/per-channel x damp 0.01/0.1)",
+                   "jobs": len(jobs), "factorizations": 14, "hessians": 7},
+        "sequential_ms_per_step": ms_seq, "pipeline_speedup": ms_seq / ms, "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--config", default=WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--config", default=WORKLOAD, choices=sorted(synth.WORKLOADS) + ["block7b"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the separate host-buffer end-to-end measurement")
+    ap.add_argument("--no-w4a16", action="store_true", help="skip the dequantizing product on the layer's output")
     args = ap.parse_args()
     rank, world, local_rank = dist_env()
     if args.impl == "reference":
+        if args.config == "block7b":
+            args.config = "block7b_q_4096x4096"
         run_reference(args, rank, world)
+        return
+    if args.config == "block7b":
+        run_block(args, rank, world, local_rank)
         return
     run_gpu(args, rank, world, local_rank)
 

@@ -175,6 +175,78 @@ gptq_status gptq_quantize_layer_noalloc(const void* W_fp16, int64_t m, int64_t n
                                         uint32_t* codes_out, float* scales_out, float* zeros_out,
                                         int32_t* g_idx_out, float* W_hat_out, int device, void* cuda_stream);
 
+/* ---------------------------------------------------------------------------------------
+ * Many layers in one call, pipelined ("大模型量化：GPTQ/AWQ/GGUF 原理对比…", AWQ vs GPTQ section:
+ * quantizing a whole 7B model layer by layer takes hours on one A100; here the per-layer solves
+ * of a block overlap on one GPU).
+ *
+ * Each job is one layer: its calibration activations, its weights, its quantizer settings and
+ * its outputs (the arguments of gptq_hessian_accumulate, gptq_prepare and gptq_quantize_layer):
+ *   X_bf16, n_tok, ld_x : device bf16 [n_tok x n] calibration activations (leading dimension ld_x)
+ *   W_fp16, m, n        : device fp16 [m x n] weights, original column order
+ *   qp, damp, desc_act  : quantizer settings and prepare settings
+ *   codes_out, scales_out, zeros_out, g_idx_out (may be NULL), perm_out (device int32 [n], may
+ *   be NULL), W_hat_out (may be NULL): as in gptq_prepare / gptq_quantize_layer.
+ * Jobs whose X_bf16, n_tok, ld_x and n are equal share one Hessian (e.g. the q, k and v
+ * projections of a transformer block read the same input); within such a group, jobs with the
+ * same damp and desc_act share one factorization.  Groups run in order of first appearance on
+ * two internal contexts and streams: the Hessian of group i+1 and the quantization of group i-1
+ * run while group i is factored.  The call allocates its contexts (two per distinct width n;
+ * GPTQ_ERR_OOM before any launch if they do not fit), waits for `cuda_stream` before starting,
+ * returns once every job is done (bounded waits) and frees the contexts.
+ * Returns the first error (GPTQ_ERR_NOT_PD names no job; the outputs of later jobs are then
+ * undefined). */
+typedef struct {
+  const void* X_bf16;
+  int64_t n_tok, ld_x;
+  const void* W_fp16;
+  int64_t m, n;
+  gptq_qparams qp;
+  double damp;
+  int desc_act;
+  uint32_t* codes_out;
+  float* scales_out;
+  float* zeros_out;
+  int32_t* g_idx_out;
+  int32_t* perm_out;
+  float* W_hat_out;
+} gptq_layer_job;
+
+gptq_status gptq_quantize_layers(const gptq_layer_job* jobs, int count, int device, void* cuda_stream);
+
+/* ---------------------------------------------------------------------------------------
+ * The packed result's consumer: Y = X W16^T
+ * ("模型量化实战：从 INT8 PTQ 到 GPTQ 的精度保持与推理加速全解析" §4.3: INT4 weights are turned
+ *  back into FP16 before the matrix product; the low-bit storage saves memory bandwidth.)
+ *
+ *   W16[r][k] = fp16( fp32(code[r][k] - zero[r][k / g]) * scale[r][k / g] )   (sweep order k)
+ *   Y[t][r]   = sum_k X[t][perm[k]] * W16[r][k]      (fp16 products, fp32 accumulation)
+ *
+ * gptq_dequant_matmul_workspace_bytes: device bytes of caller-provided workspace the call
+ *   needs for T tokens, m output rows and n input features (act_order: 1 when a perm is
+ *   passed); 0 for sizes the call rejects.  Pure host function.
+ * gptq_dequant_matmul (asynchronous, on cuda_stream):
+ *   X_fp16    : device fp16 [T x n] row-major, ORIGINAL column order, 16-byte aligned;
+ *               1 <= T <= 2^24
+ *   codes     : device uint32 [m x n*bits/32], scales/zeros: device fp32 [m x G], exactly as
+ *               gptq_quantize_layer writes them (16-byte aligned codes)
+ *   perm      : device int32 [n] (sweep position k holds original column perm[k]) or NULL for
+ *               the identity order
+ *   qp        : bits and group_size as quantized (sym is encoded in the zeros and not read)
+ *   Y         : device fp32 [T x m] row-major output
+ *   workspace : device, 256-byte aligned, at least gptq_dequant_matmul_workspace_bytes; holds a
+ *               status word, the activations gathered into sweep order and split-K partial
+ *               sums; owned by the caller, may be reused by later calls on the same stream
+ *   n % 128 == 0, 128 <= n <= 2^20, 1 <= m <= 2^24.  Arguments are checked before any launch
+ *   (GPTQ_ERR_ARG); the result is deterministic (split-K partials are summed in a fixed order).
+ * gptq_dequant_matmul_check: waits (bounded) for cuda_stream and returns GPTQ_ERR_TIMEOUT if
+ *   a bounded wait of the last gptq_dequant_matmul on this workspace ran out, else GPTQ_OK. */
+size_t gptq_dequant_matmul_workspace_bytes(int64_t T, int64_t m, int64_t n, int act_order);
+gptq_status gptq_dequant_matmul(const void* X_fp16, int64_t T, const uint32_t* codes, const float* scales,
+                                const float* zeros, const int32_t* perm, int64_t m, int64_t n, gptq_qparams qp,
+                                float* Y, void* workspace, size_t workspace_bytes, int device, void* cuda_stream);
+gptq_status gptq_dequant_matmul_check(void* workspace, int device, void* cuda_stream);
+
 /* Per-kernel instrumentation (off by default).  While profiling is on, every kernel the
  * context launches is bracketed by CUDA timing events on the context's stream and the
  * factorization runs as individual launches instead of its recorded graph (so launches no

@@ -418,6 +418,63 @@ def dequant_matmul(X, packed, scales, zeros, perm, n: int, bits: int, group_size
     return np.asarray(X, dtype=np.float64) @ dequantize_packed(packed, scales, zeros, perm, n, bits, group_size).T
 
 
+def dequantize_packed_fp16(packed, scales, zeros, perm, n: int, bits: int, group_size: int) -> np.ndarray:
+    """The FP16 weights an INT4 layer is turned back into before its product ([P4] §4.3):
+    (code - zero) * scale formed in float32, the precision the scales are stored in (the
+    difference of two small integers is exact; the product is rounded to nearest), then
+    rounded to nearest fp16.  ORIGINAL column order, like dequantize_packed."""
+    codes = unpack_codes(packed, n, bits)
+    grp = np.arange(n) // _group_width(group_size, n)
+    s = np.asarray(scales, dtype=np.float32)[:, grp]
+    z = np.asarray(zeros, dtype=np.float32)[:, grp]
+    w32 = (codes.astype(np.float32) - z) * s
+    return unpermute_columns(w32.astype(np.float16), perm)
+
+
+def dequant_matmul_fp16(X16, packed, scales, zeros, perm, n: int, bits: int, group_size: int) -> np.ndarray:
+    """Y = X W16^T in float64 for fp16 activations X16 [tokens, n] (original column order) and
+    the fp16 weights of dequantize_packed_fp16: every product of two fp16 values is exact in
+    float64 and the sum is taken in float64."""
+    W16 = dequantize_packed_fp16(packed, scales, zeros, perm, n, bits, group_size)
+    return np.asarray(X16, dtype=np.float16).astype(np.float64) @ W16.astype(np.float64).T
+
+
+# ==================================================================================
+# AWQ: activation-aware channel scaling before round-to-nearest ([P5] "AWQ：激活值感知 +
+# 通道缩放，又快又好": importance = mean |x| per input channel; the channels above the median
+# importance are multiplied by s (2.0 in the page's sketch); the scaled weights are quantized
+# to nearest and the dequantized weights are divided by the scale again)
+# ==================================================================================
+def awq_channel_importance(X) -> np.ndarray:
+    """Mean |x| of each input channel over the calibration tokens X [tokens, n] (float64)."""
+    X = np.asarray(X, dtype=np.float64)
+    return np.abs(X).sum(axis=0) / X.shape[0]
+
+
+def awq_channel_scale(importance, s_protect: float) -> np.ndarray:
+    """s_protect for the channels whose importance exceeds the median, 1 for the others.  The
+    page's torch.median gives the lower of the two middle values of an even count."""
+    v = np.asarray(importance, dtype=np.float64)
+    med = np.sort(v)[(v.shape[0] - 1) // 2]
+    return np.where(v > med, np.float32(s_protect), np.float32(1.0)).astype(np.float32)
+
+
+def awq_quantize(W, X, s_protect: float, bits: int, group_size: int, sym: bool) -> dict:
+    """The page's AWQ on one layer: W_scaled = W * scale (each input channel; float32 product),
+    round-to-nearest of W_scaled with the min-max groups of this module (original column
+    order), W_hat = dequantized / scale.  Returns rtn's dict plus channel_scale, importance,
+    packed codes and what (float64, original order)."""
+    imp = awq_channel_importance(X)
+    scale = awq_channel_scale(imp, s_protect)
+    Ws = np.asarray(W, dtype=np.float32) * scale[None, :]
+    r = rtn(Ws.astype(np.float64), bits, group_size, sym)
+    r["channel_scale"] = scale
+    r["importance"] = imp
+    r["what"] = r["what"] / scale[None, :].astype(np.float64)
+    r["packed"] = pack_codes(r["codes"], bits)
+    return r
+
+
 # ==================================================================================
 # whole layer
 # ==================================================================================

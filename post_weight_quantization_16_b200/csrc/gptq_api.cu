@@ -16,6 +16,7 @@
 
 #include "../../include/gptq.h"
 #include "../../include/gptq_testing.h"
+#include "dequant_gemm.cuh"
 #include "factor_kernels.cuh"
 #include "gemm_tc.cuh"
 #include "hessian_tc.cuh"
@@ -1297,4 +1298,323 @@ extern "C" gptq_status gptq_quantize_layer_noalloc(const void* W, int64_t m, int
     CKL("noalloc g_idx");
   }
   return GPTQ_OK;
+}
+
+// ==========================================================================================
+// The consumer of the packed result: gptq_dequant_matmul (dequant_gemm.cuh)
+// ==========================================================================================
+namespace {
+
+constexpr int kDqPlanSms = 148;  // the split-K plan is fixed so that the workspace size is a pure function
+
+struct DqPlan {
+  int tn = 0, tiles_m = 0, tiles_t = 0, k_tiles = 0, k_per = 0, splits = 0;
+  size_t xp_off = 0, part_off = 0, total = 0;
+};
+
+bool dq_plan(int64_t T, int64_t m, int64_t n, int act_order, DqPlan* p) {
+  if (T < 1 || T > (int64_t(1) << 24) || m < 1 || m > (int64_t(1) << 24) || n < 128 || n > (int64_t(1) << 20) ||
+      n % 128)
+    return false;
+  p->tn = T <= 16 ? 16 : T <= 32 ? 32 : T <= 64 ? 64 : T <= 128 ? 128 : 256;
+  p->tiles_m = static_cast<int>((m + DQ_BM - 1) / DQ_BM);
+  p->tiles_t = static_cast<int>((T + p->tn - 1) / p->tn);
+  p->k_tiles = static_cast<int>(n / DQ_BK);
+  const int64_t base = static_cast<int64_t>(p->tiles_m) * p->tiles_t;
+  int splits = base >= kDqPlanSms ? 1 : static_cast<int>(std::min<int64_t>(p->k_tiles, kDqPlanSms / base));
+  splits = std::max(1, splits);
+  p->k_per = (p->k_tiles + splits - 1) / splits;
+  p->splits = (p->k_tiles + p->k_per - 1) / p->k_per;
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  size_t off = 256;  // status word
+  p->xp_off = off;
+  if (act_order) off += up(static_cast<size_t>(T) * n * 2);
+  p->part_off = off;
+  if (p->splits > 1) off += up(static_cast<size_t>(p->splits) * T * m * 4);
+  p->total = off;
+  return true;
+}
+
+template <int BITS>
+cudaError_t set_dq_attr(int smem) {
+  return cudaFuncSetAttribute(dequant_gemm_kernel<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+}
+
+}  // namespace
+
+extern "C" size_t gptq_dequant_matmul_workspace_bytes(int64_t T, int64_t m, int64_t n, int act_order) {
+  DqPlan p;
+  if (!dq_plan(T, m, n, act_order ? 1 : 0, &p)) return 0;
+  return p.total;
+}
+
+extern "C" gptq_status gptq_dequant_matmul(const void* X, int64_t T, const uint32_t* codes, const float* scales,
+                                           const float* zeros, const int32_t* perm, int64_t m, int64_t n,
+                                           gptq_qparams qp, float* Y, void* workspace, size_t workspace_bytes,
+                                           int device, void* cuda_stream) {
+  if (!X || !codes || !scales || !zeros || !Y || !workspace) return GPTQ_ERR_ARG;
+  DqPlan pl;
+  if (!dq_plan(T, m, n, perm ? 1 : 0, &pl)) return GPTQ_ERR_ARG;
+  if (!valid_qparams(qp, n)) return GPTQ_ERR_ARG;
+  if (!aligned16(X) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return GPTQ_ERR_ARG;
+  if (workspace_bytes < pl.total) return GPTQ_ERR_ARG;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) {
+    cudaGetLastError();
+    return GPTQ_ERR_CUDA;
+  }
+  DeviceGuard dg(device);
+  PFN_cuTensorMapEncodeTiled_v12000 encode = get_encode();
+  if (!encode) return GPTQ_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int* status = reinterpret_cast<int*>(ws);
+  const int ni = static_cast<int>(n), mi = static_cast<int>(m), Ti = static_cast<int>(T);
+  const int bits = qp.bits;
+  CK(cudaMemsetAsync(status, 0, sizeof(int), st));
+  // the activations in sweep order (act-order), else as given
+  const __half* Xs = static_cast<const __half*>(X);
+  if (perm) {
+    __half* Xp = reinterpret_cast<__half*>(ws + pl.xp_off);
+    CK(cudaFuncSetAttribute(permute_x_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ni * 2));
+    permute_x_kernel<<<Ti, 256, static_cast<size_t>(ni) * 2, st>>>(Xs, ni, perm, Xp);
+    CKL("permute_x");
+    Xs = Xp;
+  }
+  CUtensorMap cmap, xmap;
+  {
+    const int64_t words = n * bits / 32;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(words), static_cast<cuuint64_t>(m)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(words) * 4};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(4 * bits), static_cast<cuuint32_t>(DQ_BM)};
+    const cuuint32_t estr[2] = {1, 1};
+    if (encode(&cmap, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(codes), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return GPTQ_ERR_CUDA;
+  }
+  {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(n), static_cast<cuuint64_t>(T)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(n) * 2};
+    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(pl.tn)};
+    const cuuint32_t estr[2] = {1, 1};
+    if (encode(&xmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half*>(Xs), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return GPTQ_ERR_CUDA;
+  }
+  DqArgs a;
+  a.T = Ti;
+  a.m = mi;
+  a.n = ni;
+  a.tn = pl.tn;
+  a.g = (qp.group_size == -1) ? ni : qp.group_size;
+  a.G = ni / a.g;
+  a.k_tiles = pl.k_tiles;
+  a.k_tiles_per_split = pl.k_per;
+  a.out = pl.splits > 1 ? reinterpret_cast<float*>(ws + pl.part_off) : Y;
+  a.scales = scales;
+  a.zeros = zeros;
+  a.status = status;
+  const int smem = dq_smem_bytes(pl.tn, bits);
+  const dim3 grid(pl.tiles_m, pl.tiles_t, pl.splits);
+  switch (bits) {
+    case 2:
+      CK(set_dq_attr<2>(smem));
+      dequant_gemm_kernel<2><<<grid, DQ_THREADS, smem, st>>>(cmap, xmap, a);
+      break;
+    case 3:
+      CK(set_dq_attr<3>(smem));
+      dequant_gemm_kernel<3><<<grid, DQ_THREADS, smem, st>>>(cmap, xmap, a);
+      break;
+    case 4:
+      CK(set_dq_attr<4>(smem));
+      dequant_gemm_kernel<4><<<grid, DQ_THREADS, smem, st>>>(cmap, xmap, a);
+      break;
+    default:
+      CK(set_dq_attr<8>(smem));
+      dequant_gemm_kernel<8><<<grid, DQ_THREADS, smem, st>>>(cmap, xmap, a);
+      break;
+  }
+  CKL("dequant_gemm");
+  if (pl.splits > 1) {
+    splitk_reduce_kernel<<<592, 256, 0, st>>>(a.out, pl.splits, static_cast<size_t>(T) * m, Y);
+    CKL("splitk_reduce");
+  }
+  return GPTQ_OK;
+}
+
+extern "C" gptq_status gptq_dequant_matmul_check(void* workspace, int device, void* cuda_stream) {
+  if (!workspace) return GPTQ_ERR_ARG;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) {
+    cudaGetLastError();
+    return GPTQ_ERR_CUDA;
+  }
+  DeviceGuard dg(device);
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  int flags = 0;
+  CK(cudaMemcpyAsync(&flags, workspace, sizeof(int), cudaMemcpyDeviceToHost, st));
+  gptq_ctx tmp;
+  tmp.stream = st;
+  const gptq_status s = wait_stream(&tmp);
+  if (s != GPTQ_OK) return s;
+  return status_from_flags(flags);
+}
+
+// ==========================================================================================
+// Many layers in one call: gptq_quantize_layers (two contexts per width, two streams)
+// ==========================================================================================
+namespace {
+
+struct LayerGroup {
+  const gptq_layer_job* first;
+  std::vector<int> jobs;
+};
+
+bool same_input(const gptq_layer_job& a, const gptq_layer_job& b) {
+  return a.X_bf16 == b.X_bf16 && a.n_tok == b.n_tok && a.ld_x == b.ld_x && a.n == b.n;
+}
+
+// The slot's context for width n (created on first use with the batch's largest m for that n).
+struct Slot {
+  cudaStream_t stream = nullptr;
+  std::vector<std::pair<int64_t, gptq_ctx*>> ctx;
+  gptq_ctx* get(int64_t n) {
+    for (auto& e : ctx)
+      if (e.first == n) return e.second;
+    return nullptr;
+  }
+};
+
+gptq_status run_group(gptq_ctx* c, const gptq_layer_job* jobs, const LayerGroup& g) {
+  // one factorization per distinct (damp, desc_act), each followed by its jobs' quantization
+  std::vector<int> done(g.jobs.size(), 0);
+  for (size_t i = 0; i < g.jobs.size(); ++i) {
+    if (done[i]) continue;
+    const gptq_layer_job& a = jobs[g.jobs[i]];
+    gptq_status s = gptq_prepare(c, a.damp, a.desc_act, nullptr);
+    if (s != GPTQ_OK) return s;
+    for (size_t j = i; j < g.jobs.size(); ++j) {
+      const gptq_layer_job& b = jobs[g.jobs[j]];
+      if (done[j] || b.damp != a.damp || b.desc_act != a.desc_act) continue;
+      done[j] = 1;
+      if (b.perm_out)
+        CK(cudaMemcpyAsync(b.perm_out, c->perm, static_cast<size_t>(c->n) * 4, cudaMemcpyDeviceToDevice, c->stream));
+      s = gptq_quantize_layer(c, b.W_fp16, b.m, b.qp, b.codes_out, b.scales_out, b.zeros_out, b.g_idx_out,
+                              b.W_hat_out);
+      if (s != GPTQ_OK) return s;
+    }
+  }
+  return GPTQ_OK;
+}
+
+gptq_status enqueue_hessian(gptq_ctx* c, const gptq_layer_job& a) {
+  gptq_status s = gptq_reset(c);
+  if (s == GPTQ_OK) s = gptq_hessian_accumulate(c, a.X_bf16, a.n_tok, a.ld_x);
+  return s;
+}
+
+}  // namespace
+
+extern "C" gptq_status gptq_quantize_layers(const gptq_layer_job* jobs, int count, int device, void* cuda_stream) {
+  if (!jobs || count < 1) return GPTQ_ERR_ARG;
+  for (int i = 0; i < count; ++i) {
+    const gptq_layer_job& j = jobs[i];
+    if (!j.W_fp16 || !j.codes_out || !j.scales_out || !j.zeros_out || j.m < 1 || j.n_tok < 0 ||
+        (j.n_tok > 0 && !j.X_bf16) || !valid_qparams(j.qp, j.n) || gptq_workspace_bytes(j.n, j.m) == 0 ||
+        !(j.damp >= 0.0) || j.damp > 1e6 || !(j.desc_act == 0 || j.desc_act == 1))
+      return GPTQ_ERR_ARG;
+  }
+  // groups of jobs that share their calibration input, in order of first appearance
+  std::vector<LayerGroup> groups;
+  for (int i = 0; i < count; ++i) {
+    LayerGroup* g = nullptr;
+    for (auto& e : groups)
+      if (same_input(*e.first, jobs[i])) g = &e;
+    if (!g) {
+      groups.push_back(LayerGroup{&jobs[i], {}});
+      g = &groups.back();
+    }
+    g->jobs.push_back(i);
+  }
+  // contexts: two per distinct width, sized for the batch's largest m at that width
+  std::vector<std::pair<int64_t, int64_t>> widths;  // (n, m_max)
+  for (int i = 0; i < count; ++i) {
+    bool found = false;
+    for (auto& w : widths)
+      if (w.first == jobs[i].n) {
+        w.second = std::max(w.second, jobs[i].m);
+        found = true;
+      }
+    if (!found) widths.emplace_back(jobs[i].n, jobs[i].m);
+  }
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) {
+    cudaGetLastError();
+    return GPTQ_ERR_CUDA;
+  }
+  DeviceGuard dg(device);
+  size_t need = 0;
+  for (auto& w : widths) need += 2 * gptq_workspace_bytes(w.first, w.second);
+  size_t free_b = 0, total_b = 0;
+  CK(cudaMemGetInfo(&free_b, &total_b));
+  const int64_t env_limit = env_int("GPTQ_MAX_WORKSPACE_BYTES", -1);
+  if (need > free_b || (env_limit >= 0 && static_cast<int64_t>(need) > env_limit)) return GPTQ_ERR_OOM;
+
+  Slot slot[2];
+  gptq_status st = GPTQ_OK;
+  cudaEvent_t ev = nullptr;
+  auto cleanup = [&]() {
+    for (auto& sl : slot) {
+      for (auto& e : sl.ctx) {
+        const gptq_status d = gptq_destroy(e.second);
+        if (st == GPTQ_OK) st = d;
+      }
+      if (sl.stream) cudaStreamDestroy(sl.stream);
+    }
+    if (ev) cudaEventDestroy(ev);
+  };
+  for (auto& sl : slot) {
+    if (cudaStreamCreateWithFlags(&sl.stream, cudaStreamNonBlocking) != cudaSuccess) {
+      st = GPTQ_ERR_CUDA;
+      cleanup();
+      return st;
+    }
+    for (auto& w : widths) {
+      gptq_ctx* c = nullptr;
+      st = gptq_create(&c, w.first, w.second, device, sl.stream);
+      if (st != GPTQ_OK) {
+        cleanup();
+        return st;
+      }
+      sl.ctx.emplace_back(w.first, c);
+    }
+  }
+  // start after the caller's stream
+  if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventRecord(ev, static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess ||
+      cudaStreamWaitEvent(slot[0].stream, ev, 0) != cudaSuccess || cudaStreamWaitEvent(slot[1].stream, ev, 0) != cudaSuccess) {
+    st = GPTQ_ERR_CUDA;
+    cleanup();
+    return st;
+  }
+  const int G = static_cast<int>(groups.size());
+  st = enqueue_hessian(slot[0].get(groups[0].first->n), *groups[0].first);
+  for (int i = 0; i < G && st == GPTQ_OK; ++i) {
+    if (i + 1 < G) {  // the next group's Hessian on the other slot, behind that slot's last quantization
+      const LayerGroup& nx = groups[i + 1];
+      st = enqueue_hessian(slot[(i + 1) & 1].get(nx.first->n), *nx.first);
+      if (st != GPTQ_OK) break;
+    }
+    st = run_group(slot[i & 1].get(groups[i].first->n), jobs, groups[i]);
+  }
+  // wait for both slots and collect any device-side failure
+  for (auto& sl : slot)
+    for (auto& e : sl.ctx) {
+      const gptq_status s = gptq_synchronize(e.second);
+      if (st == GPTQ_OK) st = s;
+    }
+  cleanup();
+  return st;
 }

@@ -35,6 +35,14 @@ class QParams(ctypes.Structure):
     _fields_ = [("bits", ctypes.c_int), ("group_size", ctypes.c_int), ("sym", ctypes.c_int)]
 
 
+class LayerJob(ctypes.Structure):
+    _fields_ = [("X_bf16", ctypes.c_void_p), ("n_tok", ctypes.c_int64), ("ld_x", ctypes.c_int64),
+                ("W_fp16", ctypes.c_void_p), ("m", ctypes.c_int64), ("n", ctypes.c_int64), ("qp", QParams),
+                ("damp", ctypes.c_double), ("desc_act", ctypes.c_int), ("codes_out", ctypes.c_void_p),
+                ("scales_out", ctypes.c_void_p), ("zeros_out", ctypes.c_void_p), ("g_idx_out", ctypes.c_void_p),
+                ("perm_out", ctypes.c_void_p), ("W_hat_out", ctypes.c_void_p)]
+
+
 class KernelStat(ctypes.Structure):
     _fields_ = [("name", ctypes.c_char * 40), ("launches", ctypes.c_int64), ("ms", ctypes.c_double),
                 ("flops", ctypes.c_double), ("bytes", ctypes.c_double)]
@@ -61,6 +69,12 @@ _SIGS = {
     "gptq_set_profiling": (ctypes.c_int, [_P, ctypes.c_int]),
     "gptq_get_profile": (ctypes.c_int, [_P, ctypes.POINTER(KernelStat), ctypes.c_int, ctypes.POINTER(ctypes.c_int)]),
     "gptq_test_bounded_wait": (ctypes.c_int, [_P, ctypes.c_uint64]),
+    "gptq_dequant_matmul_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                                              ctypes.c_int]),
+    "gptq_dequant_matmul": (ctypes.c_int, [_P, ctypes.c_int64, _P, _P, _P, _P, ctypes.c_int64, ctypes.c_int64,
+                                           QParams, _P, _P, ctypes.c_size_t, ctypes.c_int, _P]),
+    "gptq_dequant_matmul_check": (ctypes.c_int, [_P, ctypes.c_int, _P]),
+    "gptq_quantize_layers": (ctypes.c_int, [ctypes.POINTER(LayerJob), ctypes.c_int, ctypes.c_int, _P]),
     "gptq_quantize_layer_noalloc": (ctypes.c_int, [_P, ctypes.c_int64, ctypes.c_int64, _P, _P, _P, QParams,
                                                    _P, _P, _P, _P, _P, ctypes.c_int, _P]),
     "gptq_test_gemm_tf32x3": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P, ctypes.c_int, _P, _P,
@@ -230,3 +244,62 @@ class GPTQContext:
 
 def workspace_bytes(n: int, m_max: int) -> int:
     return int(lib().gptq_workspace_bytes(int(n), int(m_max)))
+
+
+def dequant_matmul(X: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor,
+                   perm: torch.Tensor | None, bits: int, group_size: int, out: torch.Tensor | None = None,
+                   workspace: torch.Tensor | None = None, stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+    """Y = X W16^T from the packed result (gptq_dequant_matmul).  X: fp16 [T, n] device tensor in
+    original column order; codes/scales/zeros as gptq_quantize_layer wrote them; perm or None.
+    Returns fp32 Y [T, m] (asynchronous on `stream`)."""
+    if X.dtype != torch.float16 or X.dim() != 2 or not X.is_contiguous():
+        raise ValueError("X must be a contiguous fp16 [T, n] device tensor")
+    T, n = X.shape
+    m = codes.shape[0]
+    dev = X.device
+    stream = stream if stream is not None else torch.cuda.current_stream(dev)
+    need = int(lib().gptq_dequant_matmul_workspace_bytes(T, m, n, int(perm is not None)))
+    if need == 0:
+        raise GPTQError(ERR_ARG, "gptq_dequant_matmul_workspace_bytes")
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    if out is None:
+        out = torch.empty((T, m), dtype=torch.float32, device=dev)
+    qp = QParams(int(bits), int(group_size), 0)
+    _check(lib().gptq_dequant_matmul(_ptr(X), T, _ptr(codes), _ptr(scales), _ptr(zeros), _ptr(perm), m, n, qp,
+                                     _ptr(out), _ptr(workspace), workspace.numel(), dev.index,
+                                     ctypes.c_void_p(stream.cuda_stream)), "gptq_dequant_matmul")
+    return out
+
+
+def quantize_layers(layers: list, device: int = 0, stream: torch.cuda.Stream | None = None) -> list:
+    """Quantize many layers in one pipelined call (gptq_quantize_layers).  `layers` is a list of
+    dicts with X (bf16 [n_tok, n] device tensor; the same tensor object for layers that share an
+    input), W (fp16 [m, n]), bits, group_size, sym, damp, desc_act and optional want_w_hat.
+    Returns one dict of device outputs per layer (codes, scales, zeros, g_idx, perm, w_hat)."""
+    dev = torch.device("cuda", device)
+    stream = stream if stream is not None else torch.cuda.current_stream(dev)
+    jobs = (LayerJob * len(layers))()
+    outs = []
+    for i, L in enumerate(layers):
+        X, W = L["X"], L["W"]
+        m, n = W.shape
+        g = n if L["group_size"] == -1 else L["group_size"]
+        o = {"codes": torch.empty((m, n * L["bits"] // 32), dtype=torch.int32, device=dev),
+             "scales": torch.empty((m, n // g), dtype=torch.float32, device=dev),
+             "zeros": torch.empty((m, n // g), dtype=torch.float32, device=dev),
+             "g_idx": torch.empty(n, dtype=torch.int32, device=dev),
+             "perm": torch.empty(n, dtype=torch.int32, device=dev),
+             "w_hat": torch.empty((m, n), dtype=torch.float32, device=dev) if L.get("want_w_hat") else None}
+        outs.append(o)
+        j = jobs[i]
+        j.X_bf16, j.n_tok, j.ld_x = X.data_ptr(), X.shape[0], X.stride(0)
+        j.W_fp16, j.m, j.n = W.data_ptr(), m, n
+        j.qp = QParams(int(L["bits"]), int(L["group_size"]), int(bool(L["sym"])))
+        j.damp, j.desc_act = float(L["damp"]), int(bool(L["desc_act"]))
+        j.codes_out, j.scales_out, j.zeros_out = o["codes"].data_ptr(), o["scales"].data_ptr(), o["zeros"].data_ptr()
+        j.g_idx_out, j.perm_out = o["g_idx"].data_ptr(), o["perm"].data_ptr()
+        j.W_hat_out = o["w_hat"].data_ptr() if o["w_hat"] is not None else None
+    _check(lib().gptq_quantize_layers(jobs, len(layers), dev.index, ctypes.c_void_p(stream.cuda_stream)),
+           "gptq_quantize_layers")
+    return outs

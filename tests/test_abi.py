@@ -83,3 +83,13 @@ def test_new_calls_reject_a_null_context(L):
     cnt = ctypes.c_int()
     assert L.gptq_get_profile(None, None, 0, ctypes.byref(cnt)) == G.ERR_ARG
     assert L.gptq_test_bounded_wait(None, 1000) == G.ERR_ARG
+
+
+def test_dequant_matmul_workspace_is_a_pure_size_function(L):
+    assert L.gptq_dequant_matmul_workspace_bytes(16, 4096, 4096, 1) >= 256 + 16 * 4096 * 2
+    assert L.gptq_dequant_matmul_workspace_bytes(16, 4096, 4096, 0) < L.gptq_dequant_matmul_workspace_bytes(
+        16, 4096, 4096, 1)
+    assert L.gptq_dequant_matmul_workspace_bytes(16, 4096, 100, 0) == 0      # n % 128
+    assert L.gptq_dequant_matmul_workspace_bytes(0, 4096, 4096, 0) == 0      # no tokens
+    assert L.gptq_dequant_matmul(None, 1, None, None, None, None, 1, 128, G.QParams(4, 128, 0), None, None, 0, 0,
+                                 None) == G.ERR_ARG

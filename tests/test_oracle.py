@@ -521,3 +521,106 @@ def test_prepare_order_is_prepare_without_the_factor():
     a, b = O.prepare_order(H, 0.1, True), O.prepare(H, 0.1, True)
     assert np.array_equal(a["perm"], b["perm"]) and np.array_equal(a["dead"], b["dead"])
     assert np.array_equal(a["Hd"], b["Hd"]) and a["mean_diag"] == b["mean_diag"]
+
+
+# ----------------------------------------------------------------------------------------
+# the fp16 weights of the dequantizing product ("模型量化实战…" §4.3: INT4 weights are turned
+# back into FP16 before the product)
+# ----------------------------------------------------------------------------------------
+def test_fp16_dequant_is_within_half_an_fp16_ulp_and_exact_for_power_of_two_scales():
+    rng = _rng(41)
+    m, n, g, bits = 6, 128, 32, 4
+    codes = rng.integers(0, 16, (m, n))
+    s = rng.uniform(1e-3, 0.05, (m, n // g)).astype(np.float32)
+    z = rng.integers(0, 16, (m, n // g)).astype(np.float32)
+    perm = rng.permutation(n)
+    packed = O.pack_codes(codes, bits)
+    w64 = O.dequantize_packed(packed, s, z, perm, n, bits, g)
+    w16 = O.dequantize_packed_fp16(packed, s, z, perm, n, bits, g)
+    assert w16.dtype == np.float16
+    # round to nearest fp16: within half an ulp of the exact value (all values are normal here)
+    ulp = np.spacing(np.abs(w16).astype(np.float16)).astype(np.float64)
+    assert np.all(np.abs(w16.astype(np.float64) - w64) <= 0.5 * ulp * (1 + 1e-6) + 1e-30)
+    # power-of-two scales: every (code - zero) * scale is representable, so nothing rounds
+    s2 = np.full_like(s, np.float32(2.0 ** -7))
+    assert np.array_equal(O.dequantize_packed_fp16(packed, s2, z, perm, n, bits, g).astype(np.float64),
+                          O.dequantize_packed(packed, s2, z, perm, n, bits, g))
+
+
+def test_fp16_dequant_rounds_the_float32_product():
+    """One weight whose exact product lies just past an fp16 rounding midpoint, but whose float32
+    product lands exactly on it (then round-half-even decides): the fp16 value follows the
+    float32 product, as the reading states."""
+    # (u - z) = 5 and s = 13428327 * 2^-26 (exact in float32): 5 s = 1 + 2^-11 + 3 * 2^-26,
+    # which float32 rounds to 1 + 2^-11, the fp16 midpoint between 1 and 1 + 2^-10
+    s = np.float32(13428327 * 2.0 ** -26)
+    assert float(s) == 13428327 * 2.0 ** -26
+    exact = 5.0 * np.float64(s)
+    f32 = np.float32(5.0) * s
+    assert exact == 1 + 2.0 ** -11 + 3 * 2.0 ** -26 and f32 == np.float32(1 + 2.0 ** -11)
+    codes = np.array([[5] + [0] * 31])
+    packed = O.pack_codes(codes, 4)
+    w16 = O.dequantize_packed_fp16(packed, np.array([[s]]), np.array([[0.0]], dtype=np.float32),
+                                   np.arange(32), 32, 4, -1)
+    # half-even from the float32 midpoint goes down to 1.0; the exact product would round up
+    assert w16[0, 0] == np.float16(1.0)
+    assert np.float16(exact) == np.float16(1 + 2.0 ** -10)
+
+
+def test_dequant_matmul_fp16_by_loops():
+    rng = _rng(43)
+    m, n, g, bits = 4, 64, 16, 3
+    codes = rng.integers(0, 8, (m, n))
+    s = rng.uniform(0.01, 0.1, (m, n // g)).astype(np.float32)
+    z = rng.integers(0, 8, (m, n // g)).astype(np.float32)
+    perm = rng.permutation(n)
+    X16 = rng.normal(0, 1, (3, n)).astype(np.float16)
+    Y = O.dequant_matmul_fp16(X16, O.pack_codes(codes, bits), s, z, perm, n, bits, g)
+    for t in range(3):
+        for r in range(m):
+            acc = 0.0
+            for k in range(n):
+                w = np.float16(np.float32(codes[r, k] - z[r, k // g]) * s[r, k // g])
+                acc += float(X16[t, perm[k]]) * float(w)
+            assert abs(Y[t, r] - acc) <= 1e-12 * (1 + abs(acc))
+
+
+# ----------------------------------------------------------------------------------------
+# AWQ ("大模型量化…", AWQ section): importance, the median mask, scaling before rounding
+# ----------------------------------------------------------------------------------------
+def test_awq_importance_and_median_mask_on_a_worked_case():
+    X = np.array([[1.0, -2.0, 0.5, 4.0], [-3.0, 2.0, 0.5, 0.0]])
+    imp = O.awq_channel_importance(X)
+    assert imp.tolist() == [2.0, 2.0, 0.5, 2.0]
+    # sorted 0.5, 2, 2, 2: the lower median is 2; no channel is strictly above it
+    assert O.awq_channel_scale(imp, 2.0).tolist() == [1.0, 1.0, 1.0, 1.0]
+    imp2 = np.array([3.0, 1.0, 4.0, 2.0])          # lower median 2: channels 0 and 2 above it
+    assert O.awq_channel_scale(imp2, 2.0).tolist() == [2.0, 1.0, 2.0, 1.0]
+    imp3 = np.array([5.0, 1.0, 3.0])               # odd count: the middle value 3
+    assert O.awq_channel_scale(imp3, 1.5).tolist() == [1.5, 1.0, 1.0]
+
+
+def test_awq_with_unit_scale_is_round_to_nearest():
+    rng = _rng(61)
+    W = rng.normal(0, 0.02, (16, 128)).astype(np.float16).astype(np.float64)
+    X = rng.normal(0, 1, (64, 128))
+    a = O.awq_quantize(W, X, 1.0, 4, 32, False)
+    r = O.rtn(W, 4, 32, False)
+    assert np.array_equal(a["codes"], r["codes"]) and np.array_equal(a["scales"], r["scales"])
+    assert np.array_equal(a["what"], r["what"])
+
+
+@pytest.mark.parametrize("sym", [False, True])
+def test_awq_protected_channels_get_a_finer_step(sym):
+    """Dividing by the scale after rounding: a protected channel's error is at most half a
+    quantization step divided by s (the page's reason the method works), an unprotected one's
+    at most half a step."""
+    rng = _rng(62)
+    W = rng.normal(0, 0.02, (32, 256)).astype(np.float16).astype(np.float64)
+    X = rng.normal(0, 1, (128, 256)) * np.where(np.arange(256) % 7 == 0, 20.0, 1.0)[None, :]
+    a = O.awq_quantize(W, X, 2.0, 4, 64, sym)
+    sc = a["channel_scale"].astype(np.float64)
+    assert (sc == 2.0).sum() == 128                                    # half of an even count
+    step = np.repeat(a["scales"].astype(np.float64), 64, axis=1)
+    err = np.abs(W - a["what"])
+    assert np.all(err <= 0.5 * step / sc[None, :] * (1 + 1e-5) + 1e-12)
