@@ -215,6 +215,28 @@ typedef struct {
 gptq_status gptq_quantize_layers(const gptq_layer_job* jobs, int count, int device, void* cuda_stream);
 
 /* ---------------------------------------------------------------------------------------
+ * AWQ on the same calibration activations and weights
+ * ("大模型量化：GPTQ/AWQ/GGUF 原理对比，4-bit 量化对推理精度的影响", AWQ section):
+ *   importance[c] = mean_t |X[t][c]|      (summed in fp64)
+ *   scale[c]      = s_protect if importance[c] > median(importance) else 1
+ *                   (median of an even count: the lower of the two middle values)
+ *   W'            = fp32(W) * scale[c]     (each input channel)
+ *   codes, scales, zeros: round-to-nearest of W' with the min-max groups of gptq_qparams in
+ *                   ORIGINAL column order (no act-order, no error compensation); codes packed
+ *                   LSB-first per row as in gptq_quantize_layer
+ *   W_hat         = (code - zero) * group scale / scale[c]   (optional)
+ * At inference the activations are divided by scale[c].  s_protect = 1 is plain round-to-
+ * nearest.  X_bf16: device bf16 [n_tok x n] (ld_x >= n, ld_x % 8 == 0, 16-byte aligned;
+ * n_tok may be 0: every scale is 1); W_fp16: device fp16 [m x n]; channel_scale_out: device
+ * fp32 [n]; workspace: device, 256-byte aligned, gptq_awq_workspace_bytes(n) bytes (fp64 channel
+ * sums and the median).  Asynchronous on cuda_stream; arguments checked before any launch. */
+size_t gptq_awq_workspace_bytes(int64_t n);
+gptq_status gptq_awq_quantize(const void* X_bf16, int64_t n_tok, int64_t ld_x, const void* W_fp16, int64_t m, int64_t n,
+                              float s_protect, gptq_qparams qp, uint32_t* codes_out, float* scales_out,
+                              float* zeros_out, float* channel_scale_out, float* W_hat_out, void* workspace,
+                              size_t workspace_bytes, int device, void* cuda_stream);
+
+/* ---------------------------------------------------------------------------------------
  * The packed result's consumer: Y = X W16^T
  * ("模型量化实战：从 INT8 PTQ 到 GPTQ 的精度保持与推理加速全解析" §4.3: INT4 weights are turned
  *  back into FP16 before the matrix product; the low-bit storage saves memory bandwidth.)

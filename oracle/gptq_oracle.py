@@ -393,7 +393,7 @@ def layer_error(W, What, H0) -> float:
     W = np.asarray(W, dtype=np.float64)
     D = W - np.asarray(What, dtype=np.float64)
     H0 = np.asarray(H0, dtype=np.float64)
-    return float(np.einsum("ij,jk,ik->", D, H0, D) / np.einsum("ij,jk,ik->", W, H0, W))
+    return float(np.sum((D @ H0) * D) / np.sum((W @ H0) * W))
 
 
 # ==================================================================================

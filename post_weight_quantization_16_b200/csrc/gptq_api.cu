@@ -16,6 +16,7 @@
 
 #include "../../include/gptq.h"
 #include "../../include/gptq_testing.h"
+#include "awq_kernels.cuh"
 #include "dequant_gemm.cuh"
 #include "factor_kernels.cuh"
 #include "gemm_tc.cuh"
@@ -1617,4 +1618,66 @@ extern "C" gptq_status gptq_quantize_layers(const gptq_layer_job* jobs, int coun
     }
   cleanup();
   return st;
+}
+
+// ==========================================================================================
+// AWQ channel scaling and round-to-nearest on the same inputs (awq_kernels.cuh)
+// ==========================================================================================
+extern "C" size_t gptq_awq_workspace_bytes(int64_t n) {
+  if (n < 128 || n > kMaxN || n % 128) return 0;
+  return 256 + static_cast<size_t>(n) * sizeof(double);
+}
+
+extern "C" gptq_status gptq_awq_quantize(const void* X, int64_t n_tok, int64_t ld_x, const void* W, int64_t m, int64_t n,
+                                         float s_protect, gptq_qparams qp, uint32_t* codes, float* scales,
+                                         float* zeros, float* channel_scale, float* W_hat, void* workspace,
+                                         size_t workspace_bytes, int device, void* cuda_stream) {
+  if (!W || !codes || !scales || !zeros || !channel_scale || !workspace) return GPTQ_ERR_ARG;
+  if (gptq_awq_workspace_bytes(n) == 0 || workspace_bytes < gptq_awq_workspace_bytes(n)) return GPTQ_ERR_ARG;
+  if (m < 1 || m > kMaxM || n_tok < 0 || n_tok >= (int64_t(1) << 40) || (n_tok > 0 && !X)) return GPTQ_ERR_ARG;
+  if (!valid_qparams(qp, n) || !(s_protect > 0.0f) || !(s_protect < 1e30f)) return GPTQ_ERR_ARG;
+  if ((X && (!aligned16(X) || ld_x < n || ld_x % 8)) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return GPTQ_ERR_ARG;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) {
+    cudaGetLastError();
+    return GPTQ_ERR_CUDA;
+  }
+  DeviceGuard dg(device);
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  const int ni = static_cast<int>(n), mi = static_cast<int>(m);
+  double* median = reinterpret_cast<double*>(workspace);
+  double* sums = reinterpret_cast<double*>(static_cast<uint8_t*>(workspace) + 256);
+  CK(cudaMemsetAsync(workspace, 0, gptq_awq_workspace_bytes(n), st));
+  if (n_tok > 0) {
+    int sms = 148;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device);
+    const int gx = (ni + AWQ_SUM_COLS - 1) / AWQ_SUM_COLS;
+    const int gy = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((4 * sms + gx - 1) / gx, (n_tok + 7) / 8)));
+    channel_abs_sum_kernel<<<dim3(gx, gy), dim3(32, 8), 0, st>>>(static_cast<const __nv_bfloat16*>(X), n_tok, ld_x, ni,
+                                                                 sums);
+    CKL("channel_abs_sum");
+  }
+  awq_median_kernel<<<(ni + 255) / 256, 256, 0, st>>>(sums, ni, median);
+  CKL("awq_median");
+  awq_scale_kernel<<<(ni + 255) / 256, 256, 0, st>>>(sums, ni, n_tok, median, s_protect, channel_scale);
+  CKL("awq_scale");
+  AwqRtnArgs a;
+  a.W = static_cast<const __half*>(W);
+  a.scale = channel_scale;
+  a.m = mi;
+  a.n = ni;
+  a.bits = qp.bits;
+  a.sym = qp.sym;
+  a.g = (qp.group_size == -1) ? ni : qp.group_size;
+  a.G = ni / a.g;
+  a.codes = codes;
+  a.scales = scales;
+  a.zeros = zeros;
+  a.W_hat = W_hat;
+  const size_t smem = static_cast<size_t>(ni + 2 * a.G) * 4;
+  CK(cudaFuncSetAttribute(awq_rtn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
+  awq_rtn_kernel<<<mi, 256, smem, st>>>(a);
+  CKL("awq_rtn");
+  return GPTQ_OK;
 }

@@ -75,6 +75,10 @@ _SIGS = {
                                            QParams, _P, _P, ctypes.c_size_t, ctypes.c_int, _P]),
     "gptq_dequant_matmul_check": (ctypes.c_int, [_P, ctypes.c_int, _P]),
     "gptq_quantize_layers": (ctypes.c_int, [ctypes.POINTER(LayerJob), ctypes.c_int, ctypes.c_int, _P]),
+    "gptq_awq_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int64]),
+    "gptq_awq_quantize": (ctypes.c_int, [_P, ctypes.c_int64, ctypes.c_int64, _P, ctypes.c_int64, ctypes.c_int64,
+                                         ctypes.c_float, QParams, _P, _P, _P, _P, _P, _P, ctypes.c_size_t,
+                                         ctypes.c_int, _P]),
     "gptq_quantize_layer_noalloc": (ctypes.c_int, [_P, ctypes.c_int64, ctypes.c_int64, _P, _P, _P, QParams,
                                                    _P, _P, _P, _P, _P, ctypes.c_int, _P]),
     "gptq_test_gemm_tf32x3": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P, ctypes.c_int, _P, _P,
@@ -303,3 +307,27 @@ def quantize_layers(layers: list, device: int = 0, stream: torch.cuda.Stream | N
     _check(lib().gptq_quantize_layers(jobs, len(layers), dev.index, ctypes.c_void_p(stream.cuda_stream)),
            "gptq_quantize_layers")
     return outs
+
+
+def awq_quantize(X: torch.Tensor | None, W: torch.Tensor, s_protect: float = 2.0, bits: int = 4, group_size: int = 128,
+                 sym: bool = False, want_w_hat: bool = True, stream: torch.cuda.Stream | None = None) -> dict:
+    """AWQ channel scaling plus round-to-nearest (gptq_awq_quantize).  X: bf16 [n_tok, n] device
+    tensor (or None: no calibration tokens), W: fp16 [m, n].  Returns device tensors codes,
+    scales, zeros, channel_scale and (optionally) w_hat, all in original column order."""
+    m, n = W.shape
+    dev = W.device
+    stream = stream if stream is not None else torch.cuda.current_stream(dev)
+    g = n if group_size == -1 else group_size
+    out = {"codes": torch.empty((m, n * bits // 32), dtype=torch.int32, device=dev),
+           "scales": torch.empty((m, n // g), dtype=torch.float32, device=dev),
+           "zeros": torch.empty((m, n // g), dtype=torch.float32, device=dev),
+           "channel_scale": torch.empty(n, dtype=torch.float32, device=dev),
+           "w_hat": torch.empty((m, n), dtype=torch.float32, device=dev) if want_w_hat else None}
+    ws = torch.empty(int(lib().gptq_awq_workspace_bytes(n)), dtype=torch.uint8, device=dev)
+    n_tok, ld = (0, n) if X is None else (X.shape[0], X.stride(0))
+    qp = QParams(int(bits), int(group_size), int(bool(sym)))
+    _check(lib().gptq_awq_quantize(_ptr(X), n_tok, ld, _ptr(W), m, n, float(s_protect), qp, _ptr(out["codes"]),
+                                   _ptr(out["scales"]), _ptr(out["zeros"]), _ptr(out["channel_scale"]),
+                                   _ptr(out["w_hat"]), _ptr(ws), ws.numel(), dev.index,
+                                   ctypes.c_void_p(stream.cuda_stream)), "gptq_awq_quantize")
+    return out

@@ -11,6 +11,8 @@ check takes what it can compute one by one or what holds at any size:
 * the sweep: replayed by the oracle on sampled rows (stage-isolated: on the GPU's H; at 28672
   on the GPU's factor, checked above), with the layer error of those rows against the
   oracle's own run on them."""
+import time
+
 import numpy as np
 import pytest
 import torch
@@ -76,16 +78,24 @@ def _gpu_layer(layer, settings, seed=123, n_pairs=2048, full_factor=True, rows=2
     pairs = pairs[pairs[:, 0] != pairs[:, 1]]
     sample = np.sort(rng.choice(layer.m, min(rows, layer.m), replace=False))
     with GPTQContext(layer.n, layer.m, 0) as ctx:
+        t0 = time.perf_counter()
         d_ref, o_ref = _accumulate_and_sample(ctx, layer, pairs)
+        print(f"[{layer.name}] X streamed and sampled {time.perf_counter() - t0:.1f} s", flush=True)
         Ht, nt = ctx.get_hessian()
         H = Ht.cpu().numpy().astype(np.float64)
         del Ht
         assert nt == layer.n_tok
         _check_sampled_hessian(H, pairs, d_ref, o_ref)
         preps = {}
+        current = None
         for qs in settings:
             key = (qs.damp, qs.desc_act)
+            if key != current and key in preps:   # the context holds another damp's factor: redo it
+                ctx.prepare(qs.damp, qs.desc_act)
+                current = key
             if key not in preps:
+                current = key
+                t0 = time.perf_counter()
                 perm = ctx.prepare(qs.damp, qs.desc_act).cpu().numpy()
                 dead = ctx.get_dead_columns().cpu().numpy().astype(bool)
                 Ut = ctx.get_factor()
@@ -109,9 +119,11 @@ def _gpu_layer(layer, settings, seed=123, n_pairs=2048, full_factor=True, rows=2
                     uref = U   # the sweep replays on the GPU's factor, checked above
                 res = _u_probe_residual(U, po["Hd"], rng)
                 assert res <= 1e-3, res
+                print(f"[{layer.name}] prepare and factor checks {time.perf_counter() - t0:.1f} s", flush=True)
                 preps[key] = {"perm": perm, "dead": dead, "U": uref, "Hd": None}
                 del U
             prep = preps[key]
+            t0 = time.perf_counter()
             out = ctx.quantize_layer(Wd, qs.bits, qs.group_size, bool(qs.sym))
             ctx.synchronize()
             gpu = {"codes": O.unpack_codes(out["codes"][sample].cpu().numpy().view(np.uint32), layer.n, qs.bits),
@@ -131,6 +143,7 @@ def _gpu_layer(layer, settings, seed=123, n_pairs=2048, full_factor=True, rows=2
             e_gpu = O.layer_error(Wf, what, H)
             e_own = O.layer_error(Wf, own_what, H)
             assert abs(e_gpu - e_own) <= GH.LAYER_ERR_REL * e_own, (qs, e_gpu, e_own)
+            print(f"[{layer.name}] {qs} sweep checks {time.perf_counter() - t0:.1f} s", flush=True)
 
 
 def test_q_proj_full_size():
