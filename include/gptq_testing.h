@@ -11,30 +11,28 @@
 extern "C" {
 #endif
 
-/* The three-product bf16 tensor-core GEMM of the factorization and of the lazy trailing
+/* The three-product tf32 tensor-core GEMM of the factorization and of the lazy trailing
  * update (S4, S6):  C = alpha * A * B^T (+ C when beta = 1).
- *   A_hi/A_lo : device bf16 [M x K], leading dimension lda (A ~ A_hi + A_lo, the bf16 pair of A)
- *   B_hi/B_lo : device bf16 [N x K], leading dimension ldb
+ *   A_hi/A_lo : device fp32 [M x K], leading dimension lda (A = A_hi + A_lo; hi/lo are tf32 values)
+ *   B_hi/B_lo : device fp32 [N x K], leading dimension ldb
  *   k_lo_mode : 0 = K from 0; 1 = K from the first column of the output tile (B lower-triangular
  *               in this form); 2 = K from the first row of the tile (A upper-triangular)
  *   k_hi_mode : 0 = K to the end; 1 = K up to the last column of the tile (B upper-triangular)
  *   upper_only: skip output tiles wholly below the diagonal of C
- *   C         : fp32 output [M x N] (ldc) or NULL (beta = 1 needs it: C += ...);
- *   C_hi/C_lo : bf16 pair of the result [M x N] (ldh) or NULL;
- *   Ct        : transposed fp32 result [N x M] (ldt) or NULL; Ct_hi/Ct_lo: its bf16 pair or NULL.
- *   chunk_stages: 64-wide K stages summed in one tensor-memory accumulator before the fp32
- *               register add (1 = every stage; the trailing update of the sweep uses 2).
+ *   C         : fp32 output [M x N] (ldc) or NULL; C_hi/C_lo: hi/lo output (ldh) or NULL;
+ *   Ct_hi/Ct_lo: transposed hi/lo output [N x M] (ldt) or NULL (beta applies to C and C_hi/C_lo).
+ *   chunk_stages: 32-wide K stages summed in one tensor-memory accumulator before the fp32
+ *               register add (1 = every stage; the trailing update of the sweep uses 4).
  *   tile_n    : output tile width 64, 128 or 256, or 0 for the library's own choice.
  *   c_reduce  : 1 = C += alpha A B^T through TMA reduce-add boxes (needs C and beta = 1; C's
  *               base 16-byte aligned, ldc % 4 == 0), the path of the sweep's trailing update.
- * Requirements: N % 32 == 0, K % 64 == 0, 16-byte aligned bases, lda, ldb, ldh % 8 == 0,
- * ldc % 4 == 0.  Synchronizes the stream before returning.  Allocates a 4-byte status word
- * (stream-ordered). */
-gptq_status gptq_test_gemm_bf16x3(int M, int N, int K, const void* A_hi, const void* A_lo, int lda, const void* B_hi,
-                                  const void* B_lo, int ldb, float alpha, int beta, int k_lo_mode, int k_hi_mode,
-                                  int upper_only, float* C, int ldc, void* C_hi, void* C_lo, int ldh, float* Ct,
-                                  void* Ct_hi, void* Ct_lo, int ldt, int chunk_stages, int tile_n, int c_reduce,
-                                  int device, void* cuda_stream);
+ * Requirements: N % 32 == 0, K % 32 == 0, 16-byte aligned bases, leading dimensions % 4 == 0.
+ * Synchronizes the stream before returning.  Allocates a 4-byte status word (stream-ordered). */
+gptq_status gptq_test_gemm_tf32x3(int M, int N, int K, const float* A_hi, const float* A_lo, int lda, const float* B_hi,
+                                  const float* B_lo, int ldb, float alpha, int beta, int k_lo_mode, int k_hi_mode,
+                                  int upper_only, float* C, int ldc, float* C_hi, float* C_lo, int ldh, float* Ct_hi,
+                                  float* Ct_lo, int ldt, int chunk_stages, int tile_n, int c_reduce, int device,
+                                  void* cuda_stream);
 
 /* The sweep's division (S5): x / s from the rounded reciprocal of s plus one fused
  * multiply-add correction, compared bit for bit with IEEE division on `count` (x, s) pairs

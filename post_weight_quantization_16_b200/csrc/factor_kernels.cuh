@@ -9,12 +9,9 @@
 //   [U22] = f(A22);  V12 = A12 U22^T;  A11 -= V12 V12^T;  T = V12 U22;  [U11] = f(A11);
 //   U12 = -U11 T
 // whose products run on the tensor cores (gemm_tc.cuh) and whose leaves are the 128 x 128
-// diagonal blocks handled by leaf_chol_inv_kernel below.  Every matrix of the recursion
-// lives as an fp32 master (read by the leaves, the sweep and the CUDA-core products) and as a
-// bf16 hi/lo pair (the operands of the three-product tensor-core GEMM).
+// diagonal blocks handled by leaf_chol_inv_kernel below.  Matrices live as tf32 hi/lo
+// pairs (X = hi + lo to about 2^-23) so that they can feed the three-product GEMM.
 #pragma once
-
-#include <cuda_bf16.h>
 
 #include "sm100_ptx.cuh"
 
@@ -26,6 +23,12 @@ constexpr int LF_THREADS = 256;
 constexpr int LF_LD = LF_NB + 1;
 constexpr int LF_SMEM = 3 * LF_NB * LF_LD * 4 + LF_NB * 4 + 16;  // S, V, X, 1/V[c][c], flag
 static_assert(LF_NB * LF_NB <= LF_NB * LF_LD, "a staged block must fit in V (and in X)");
+
+__device__ __forceinline__ float tf32_round(float x) {
+  uint32_t u = __float_as_uint(x);
+  u += 0xFFFu + ((u >> 13) & 1u);
+  return __uint_as_float(u & 0xFFFFE000u);
+}
 
 // Warp 0: one 32-column panel of the UL Cholesky, P0 = 32 p.  Lane l carries row P0 + l of
 // the diagonal block (and, for NR > 0, row 32 r + l of block row r < NR above it) in
@@ -138,37 +141,28 @@ __device__ __forceinline__ void lf_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-// Two fp32 values as one word of two bf16 (the first in the low half).
-__device__ __forceinline__ uint32_t bf16x2_bits(__nv_bfloat16 a, __nv_bfloat16 b) {
-  return static_cast<uint32_t>(__bfloat16_as_ushort(a)) | (static_cast<uint32_t>(__bfloat16_as_ushort(b)) << 16);
-}
-
-// Rows [R0, R0 + 32) of U = X (zeros left of the diagonal): the fp32 master (16-byte stores)
-// and its bf16 hi/lo pair (8-byte stores), by threads t = 0 .. nt-1.  (U^T is formed off the
-// critical path.)
-__device__ __forceinline__ void leaf_store_rows(const float (*X)[LF_LD], float* __restrict__ U,
-                                                __nv_bfloat16* __restrict__ U_hi, __nv_bfloat16* __restrict__ U_lo,
-                                                int n, int o, int R0, int t, int nt) {
+// Rows [R0, R0 + 32) of U = X (zeros left of the diagonal) as a hi/lo pair, 16-byte stores,
+// by threads t = 0 .. nt-1.  (U^T is formed off the critical path.)
+__device__ __forceinline__ void leaf_store_rows(const float (*X)[LF_LD], float* __restrict__ U_hi,
+                                                float* __restrict__ U_lo, int n, int o, int R0, int t, int nt) {
   for (int idx = t; idx < LF_P * (LF_NB / 4); idx += nt) {
     const int i = R0 + idx / (LF_NB / 4), j = (idx % (LF_NB / 4)) * 4;
-    float u[4];
-    __nv_bfloat16 uh[4], ul[4];
+    float uh[4], ul[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      u[e] = (i <= j + e) ? X[i][j + e] : 0.0f;  // U[i][j+e]
-      uh[e] = __float2bfloat16_rn(u[e]);
-      ul[e] = __float2bfloat16_rn(u[e] - __bfloat162float(uh[e]));
+      const float u = (i <= j + e) ? X[i][j + e] : 0.0f;  // U[i][j+e]
+      uh[e] = tf32_round(u);
+      ul[e] = tf32_round(u - uh[e]);
     }
     const size_t g = static_cast<size_t>(o + i) * n + o + j;
-    *reinterpret_cast<float4*>(U + g) = make_float4(u[0], u[1], u[2], u[3]);
-    *reinterpret_cast<uint2*>(U_hi + g) = make_uint2(bf16x2_bits(uh[0], uh[1]), bf16x2_bits(uh[2], uh[3]));
-    *reinterpret_cast<uint2*>(U_lo + g) = make_uint2(bf16x2_bits(ul[0], ul[1]), bf16x2_bits(ul[2], ul[3]));
+    *reinterpret_cast<float4*>(U_hi + g) = make_float4(uh[0], uh[1], uh[2], uh[3]);
+    *reinterpret_cast<float4*>(U_lo + g) = make_float4(ul[0], ul[1], ul[2], ul[3]);
   }
 }
 
 // Leaf: U_kk (= V_kk^-1, V_kk V_kk^T = A_kk) for the diagonal block at offset o, read from
-// the upper triangle of the fp32 master A.  Writes U (upper, zeros below) as fp32 master and
-// bf16 pair (transpose_block_kernel forms U^T on the graph's second branch).  A non-positive or non-finite pivot sets ST_NOT_PD (and is replaced by 1
+// the upper triangle of A = A_hi + A_lo.  Writes U (upper, zeros below) as a hi/lo pair
+// (transpose_block_kernel forms U^T on the graph's second branch).  A non-positive or non-finite pivot sets ST_NOT_PD (and is replaced by 1
 // so the kernel still finishes with finite work).
 //
 // Reverse right-looking Cholesky over four 32-column panels, bottom-right first.  The chain
@@ -179,8 +173,8 @@ __device__ __forceinline__ void leaf_store_rows(const float (*X)[LF_LD], float* 
 // inverse U = V^-1:
 //   U_pj = -Xd_p * sum_{l=p+1..j} V_pl U_lj      (Xd_p = the diagonal block's inverse).
 __global__ void __launch_bounds__(LF_THREADS, 1)
-    leaf_chol_inv_kernel(const float* __restrict__ A, int n, int o, float* __restrict__ U,
-                         __nv_bfloat16* __restrict__ U_hi, __nv_bfloat16* __restrict__ U_lo, int* __restrict__ status) {
+    leaf_chol_inv_kernel(const float* __restrict__ A_hi, const float* __restrict__ A_lo, int n, int o,
+                         float* __restrict__ U_hi, float* __restrict__ U_lo, int* __restrict__ status) {
   extern __shared__ float lf_smem[];
   float(*S)[LF_LD] = reinterpret_cast<float(*)[LF_LD]>(lf_smem);
   float(*V)[LF_LD] = reinterpret_cast<float(*)[LF_LD]>(lf_smem + LF_NB * LF_LD);
@@ -190,21 +184,23 @@ __global__ void __launch_bounds__(LF_THREADS, 1)
   griddep_wait();
   griddep_launch_dependents();  // one CTA: the next kernel may take the other SMs right away
   if (tid == 0) *bad = 0;
-  // stage A into V's storage with asynchronous 16-byte copies, at an unpadded 128-float pitch
-  // (the 129-float rows of S are not 16-byte aligned)
+  // stage A_hi into V's storage and A_lo into X's with asynchronous 16-byte copies, at an
+  // unpadded 128-float pitch (the 129-float rows of S are not 16-byte aligned)
   {
     float* th = &V[0][0];
+    float* tl = &X[0][0];
     for (int idx = tid; idx < LF_NB * (LF_NB / 4); idx += LF_THREADS) {
       const int i = idx / (LF_NB / 4), j = (idx % (LF_NB / 4)) * 4;
       const size_t g = static_cast<size_t>(o + i) * n + o + j;
-      const uint32_t dh = smem_u32(th + i * LF_NB + j);
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dh), "l"(A + g) : "memory");
+      const uint32_t dh = smem_u32(th + i * LF_NB + j), dl = smem_u32(tl + i * LF_NB + j);
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dh), "l"(A_hi + g) : "memory");
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dl), "l"(A_lo + g) : "memory");
     }
     asm volatile("cp.async.commit_group;\n cp.async.wait_group 0;" ::: "memory");
     __syncthreads();
     for (int idx = tid; idx < LF_NB * LF_NB; idx += LF_THREADS) {
       const int i = idx / LF_NB, j = idx % LF_NB;
-      const float v = th[i * LF_NB + j];
+      const float v = th[i * LF_NB + j] + tl[i * LF_NB + j];
       S[i][j] = (i <= j) ? v : 0.0f;
     }
   }
@@ -246,7 +242,7 @@ __global__ void __launch_bounds__(LF_THREADS, 1)
       __syncthreads();  // column block p-1 is up to date: warp 0 may factor it
     }
     // block row p+1 of U is final (since the last step): warp 4, otherwise idle here, writes it
-    if (warp == 4 && p + 1 < LF_NB / LF_P) leaf_store_rows(X, U, U_hi, U_lo, n, o, (p + 1) * LF_P, lane, 32);
+    if (warp == 4 && p + 1 < LF_NB / LF_P) leaf_store_rows(X, U_hi, U_lo, n, o, (p + 1) * LF_P, lane, 32);
     if (g1) {
       {
         // the rest of the trailing update: S[i][j] -= sum_c V[i][P0+c] V[j][P0+c], i <= j < P0-32
@@ -331,32 +327,32 @@ __global__ void __launch_bounds__(LF_THREADS, 1)
   __syncthreads();
 
   // block row 0 of U (the others went out during the factorization)
-  leaf_store_rows(X, U, U_hi, U_lo, n, o, 0, tid, LF_THREADS);
+  leaf_store_rows(X, U_hi, U_lo, n, o, 0, tid, LF_THREADS);
   if (tid == 0 && *bad) atomicOr(status, ST_NOT_PD);
 }
 
-// U^T of one 128 x 128 diagonal block from the fp32 master, as fp32 master and bf16 pair,
-// 32 x 32 tiles through shared memory: Ut[o + c][o + r] = U[o + r][o + c].  Grid (4, 4),
-// block (32, 8).
-__global__ void __launch_bounds__(256) transpose_block_kernel(const float* __restrict__ U, int n, int o,
-                                                              float* __restrict__ Ut, __nv_bfloat16* __restrict__ Ut_hi,
-                                                              __nv_bfloat16* __restrict__ Ut_lo) {
-  __shared__ float th[32][33];
+// U^T of one 128 x 128 diagonal block (hi and lo), 32 x 32 tiles through shared memory:
+// Ut[o + c][o + r] = U[o + r][o + c].  Grid (4, 4), block (32, 8).
+__global__ void __launch_bounds__(256) transpose_block_kernel(const float* __restrict__ U_hi,
+                                                              const float* __restrict__ U_lo, int n, int o,
+                                                              float* __restrict__ Ut_hi, float* __restrict__ Ut_lo) {
+  __shared__ float th[32][33], tl[32][33];
   griddep_wait();
   griddep_launch_dependents();
   const int tx = threadIdx.x, ty = threadIdx.y;
   const int r0 = o + blockIdx.y * 32, c0 = o + blockIdx.x * 32;
 #pragma unroll
-  for (int k = 0; k < 4; ++k) th[ty + 8 * k][tx] = U[static_cast<size_t>(r0 + ty + 8 * k) * n + c0 + tx];
+  for (int k = 0; k < 4; ++k) {
+    const size_t g = static_cast<size_t>(r0 + ty + 8 * k) * n + c0 + tx;
+    th[ty + 8 * k][tx] = U_hi[g];
+    tl[ty + 8 * k][tx] = U_lo[g];
+  }
   __syncthreads();
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const size_t g = static_cast<size_t>(c0 + ty + 8 * k) * n + r0 + tx;
-    const float v = th[tx][ty + 8 * k];
-    const __nv_bfloat16 h = __float2bfloat16_rn(v);
-    Ut[g] = v;
-    Ut_hi[g] = h;
-    Ut_lo[g] = __float2bfloat16_rn(v - __bfloat162float(h));
+    Ut_hi[g] = th[tx][ty + 8 * k];
+    Ut_lo[g] = tl[tx][ty + 8 * k];
   }
 }
 

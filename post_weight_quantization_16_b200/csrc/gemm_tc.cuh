@@ -1,54 +1,47 @@
-// gemm_tc.cuh — fp32-faithful GEMM on the sm_100a tensor cores (three bf16 products).
+// gemm_tc.cuh — fp32-faithful GEMM on the sm_100a tensor cores (three tf32 products).
 //
 //   C = alpha * A * B^T (+ C)      A [M x K] row-major, B [N x K] row-major (both K-major)
 //
 // Used by the factorization (its Schur-complement, panel and inverse products) and by the
 // lazy trailing update of the column sweep (W[:, i2:] -= Err * U[blk, i2:]).  Each operand
-// X is given as two bf16 arrays X_hi = rn_bf16(X) and X_lo = rn_bf16(X - X_hi) (X to about
-// 2^-17); the product is A_hi B_hi + A_hi B_lo + A_lo B_hi, the missing A_lo B_lo term being
-// about 2^-16 of the product.  (A numpy emulation of the whole blocked factorization and of
-// the sweep's trailing update with these products, on a 4096-wide layer of the q_proj recipe,
-// kept U within 2.1e-6 of float64 and changed one code of 786432, inside the rounding band.)
-// The tensor cores' own accumulation is not round-to-nearest, so every 64-wide K stage is
+// X is stored as two arrays X_hi = rn_tf32(X) and X_lo = rn_tf32(X - X_hi); the product is
+// A_hi B_hi + A_hi B_lo + A_lo B_hi, about 2^-21 relative per term, close to fp32.  The
+// tensor cores' own accumulation is not round-to-nearest, so every 32-wide K stage is
 // accumulated in its own TMEM buffer and then added into fp32 registers with
 // round-to-nearest adds (double-buffered TMEM, as in the Hessian kernel).
 //
 // Tile 128 x BN, BN in {64, 128, 256} chosen per product so that small products still spread
-// over many SMs (tcgen05.mma kind::f16 with bf16 operands, M=128, N=BN, K=16), persistent CTAs
-// (one per SM) over the tiles, a TMA ring of about 192 KB (2, 3 or 4 stages of A_hi, A_lo,
-// B_hi, B_lo; 128-byte swizzle; B arrives as 64-row boxes, so one tensor map serves every
-// BN), warp roles:
+// over many SMs (tcgen05.mma kind::tf32, M=128, N=BN, K=8), persistent CTAs (one per SM) over
+// the tiles, a TMA ring of about 192 KB (2, 3 or 4 stages of A_hi, A_lo, B_hi, B_lo; 128-byte
+// swizzle; B arrives as 64-row boxes, so one tensor map serves every BN), warp roles:
 //   warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer, warps 2-9 epilogue.
 // Triangular operands: the K range of a tile can start at its first column (B lower in
 // K-major form) or its first row (A upper), or stop after its last column (B upper), so
 // the zero halves of triangular factors are skipped; tiles wholly below the diagonal of C
 // can be skipped for symmetric updates.
-// Outputs (any subset): plain fp32 C (optionally + C), a bf16 hi/lo pair of the result, and
-// the transposed result as fp32 and as a bf16 pair (coalesced: the 32 lanes of a warp write
-// 32 consecutive rows).  The accumulating plain output of the sweep's trailing update
-// (C += alpha A B^T) can instead go out through TMA reduce-add: each epilogue warp stages
-// 32 x 32 boxes in shared memory and L2 adds them into C, so the tile never reads C and its
-// stores are whole swizzled boxes.
+// Outputs (any subset): plain fp32 C (optionally + C), hi/lo pair (optionally + hi+lo), and a
+// transposed hi/lo pair (coalesced: the 32 lanes of a warp write 32 consecutive rows).  The
+// accumulating plain output of the sweep's trailing update (C += alpha A B^T) can instead go
+// out through TMA reduce-add: each epilogue warp stages 32 x 32 boxes in shared memory and
+// L2 adds them into C, so the tile never reads C and its stores are whole swizzled boxes.
 // A and B are addressed as sub-blocks (row/column offsets) of the whole matrices their tensor
 // maps describe, so the maps are encoded once per context.  Rows or columns of a partial
 // tile that fall outside the sub-block read neighbouring data whose products land only in
 // outputs that are never stored.
 #pragma once
 
-#include <cuda_bf16.h>
-
 #include "sm100_ptx.cuh"
 
 namespace gptq {
 
-constexpr int GT_BM = 128, GT_BK = 64, GT_BOX_N = 64;  // GT_BK bf16 = one 128-byte swizzle row
-constexpr int GT_A_BYTES = GT_BM * GT_BK * 2;  // 16 KB
+constexpr int GT_BM = 128, GT_BK = 32, GT_BOX_N = 64;
+constexpr int GT_A_BYTES = GT_BM * GT_BK * 4;  // 16 KB
 constexpr int GT_THREADS = 64 + 256;
 
 template <int BN>
 struct GtCfg {
   static_assert(BN == 64 || BN == 128 || BN == 256, "tile width");
-  static constexpr int B_BYTES = BN * GT_BK * 2;
+  static constexpr int B_BYTES = BN * GT_BK * 4;
   static constexpr int STAGE_BYTES = 2 * GT_A_BYTES + 2 * B_BYTES;  // 48, 64 or 96 KB
   static constexpr int STAGES = BN == 256 ? 2 : (BN == 128 ? 3 : 4);
   static constexpr int STG_BYTES = 8 * 32 * 32 * 4;  // one 32 x 32 fp32 staging box per epilogue warp
@@ -64,27 +57,26 @@ struct GemmTCArgs {
   int a_row0, a_col0;  // offset of A inside the matrix its tensor maps describe
   int b_row0, b_col0;  // offset of B
   float alpha;
-  int beta;          // 0 or 1: add the existing fp32 C
+  int beta;          // 0 or 1: add the existing C (plain or hi+lo)
   int k_lo_mode, k_hi_mode, upper_only;
   int chunk_stages;  // K stages summed in one TMEM accumulator before the fp32 register add
-  float* C;          // plain fp32 output (or nullptr); with beta = 1 also the added C
+  float* C;          // plain fp32 output (or nullptr)
   int ldc;
   int c_reduce;        // 1: C += alpha A B^T by TMA reduce-add through the c_map tensor map (beta = 1)
   int c_row0, c_col0;  // offset of C inside the matrix c_map describes
-  __nv_bfloat16* Chi;  // bf16 hi/lo pair of the result (or nullptr)
-  __nv_bfloat16* Clo;
+  float* Chi;        // hi/lo output (or nullptr)
+  float* Clo;
   int ldh;
-  float* Ct;           // transposed fp32 result (or nullptr): Ct[c][r]
-  __nv_bfloat16* Cthi; // transposed bf16 pair (or nullptr)
-  __nv_bfloat16* Ctlo;
+  float* Cthi;       // transposed hi/lo output (or nullptr): Ct[c][r]
+  float* Ctlo;
   int ldt;
   int* status;
 };
 
-// bf16 pair of an fp32 value: hi = rn_bf16(x), lo = rn_bf16(x - hi) (x - hi is exact in fp32)
-__device__ __forceinline__ void bf16_split(float x, __nv_bfloat16& hi, __nv_bfloat16& lo) {
-  hi = __float2bfloat16_rn(x);
-  lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+__device__ __forceinline__ float tf32_rn(float x) {
+  uint32_t u = __float_as_uint(x);
+  u += 0xFFFu + ((u >> 13) & 1u);
+  return __uint_as_float(u & 0xFFFFE000u);
 }
 
 // Number of output tiles the kernel visits: all of them, or with upper_only only the tiles
@@ -150,7 +142,7 @@ __host__ __device__ inline int gt_sched(int i, int b, int G) { return i * G + ((
 // tile's first stages were in flight, so a tile ends with stores only.
 template <int BN>
 __global__ void __launch_bounds__(GT_THREADS, 1)
-    gemm_bf16x3_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_constant__ CUtensorMap a_lo,
+    gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_constant__ CUtensorMap a_lo,
                        const __grid_constant__ CUtensorMap b_hi, const __grid_constant__ CUtensorMap b_lo,
                        const __grid_constant__ CUtensorMap c_map, GemmTCArgs p) {
   extern __shared__ uint8_t gt_smem_raw[];
@@ -230,7 +222,7 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
           tma_load_2d(st + GT_A_BYTES, &a_lo, fb, p.a_col0 + k, p.a_row0 + m0);
 #pragma unroll
           for (int bx = 0; bx < BN / GT_BOX_N; ++bx) {  // 64-row boxes, stacked at 8 KB
-            const uint32_t o8 = bx * (GT_BOX_N * GT_BK * 2);
+            const uint32_t o8 = bx * (GT_BOX_N * GT_BK * 4);
             tma_load_2d(st + 2 * GT_A_BYTES + o8, &b_hi, fb, p.b_col0 + k, p.b_row0 + n0 + bx * GT_BOX_N);
             tma_load_2d(st + 2 * GT_A_BYTES + B_BYTES + o8, &b_lo, fb, p.b_col0 + k, p.b_row0 + n0 + bx * GT_BOX_N);
           }
@@ -242,7 +234,7 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer: one TMEM buffer per chunk of K stages ----------------
-      constexpr uint32_t idesc = idesc_make(1u, 1u, 0u, 0u, GT_BM, BN);  // bf16, K-major A and B
+      constexpr uint32_t idesc = idesc_make(2u, 2u, 0u, 0u, GT_BM, BN);  // tf32, K-major A and B
       const int cs = p.chunk_stages;
       bool ok = true;
       int it = 0, ch = 0;
@@ -274,13 +266,13 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
           const uint32_t sa_hi = st, sa_lo = st + GT_A_BYTES;
           const uint32_t sb_hi = st + 2 * GT_A_BYTES, sb_lo = sb_hi + B_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < GT_BK / 16; ++kk) {
-            const uint32_t off = kk * 32;  // 16 bf16 of K inside the 128-byte swizzle row
+          for (int kk = 0; kk < GT_BK / 8; ++kk) {
+            const uint32_t off = kk * 32;  // 8 fp32 of K inside the 128-byte swizzle row
             const uint64_t dah = sdesc_sw128(sa_hi + off, 16, 1024), dal = sdesc_sw128(sa_lo + off, 16, 1024);
             const uint64_t dbh = sdesc_sw128(sb_hi + off, 16, 1024), dbl = sdesc_sw128(sb_lo + off, 16, 1024);
-            umma_f16(d_tmem, dal, dbh, idesc, (first && kk == 0) ? 0u : 1u);
-            umma_f16(d_tmem, dah, dbl, idesc, 1u);
-            umma_f16(d_tmem, dah, dbh, idesc, 1u);
+            umma_tf32(d_tmem, dal, dbh, idesc, (first && kk == 0) ? 0u : 1u);
+            umma_tf32(d_tmem, dah, dbl, idesc, 1u);
+            umma_tf32(d_tmem, dah, dbh, idesc, 1u);
           }
           umma_commit(bar_empty + 8 * s);
           if ((j % cs) == cs - 1 || j == ni - 1) {
@@ -324,6 +316,17 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
             acc[cc * 32 + 4 * j + 1] = c.y;
             acc[cc * 32 + 4 * j + 2] = c.z;
             acc[cc * 32 + 4 * j + 3] = c.w;
+          }
+        } else if (ld && p.Chi) {
+          const float4* hp = reinterpret_cast<const float4*>(p.Chi + static_cast<size_t>(r) * p.ldh + c0);
+          const float4* lp = reinterpret_cast<const float4*>(p.Clo + static_cast<size_t>(r) * p.ldh + c0);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float4 h = hp[j], l = lp[j];
+            acc[cc * 32 + 4 * j + 0] = h.x + l.x;
+            acc[cc * 32 + 4 * j + 1] = h.y + l.y;
+            acc[cc * 32 + 4 * j + 2] = h.z + l.z;
+            acc[cc * 32 + 4 * j + 3] = h.w + l.w;
           }
         } else {
 #pragma unroll
@@ -391,30 +394,29 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
                                 acc[cc * 32 + 4 * j + 3]);
         }
         if (p.Chi) {
-          uint4* hp = reinterpret_cast<uint4*>(p.Chi + static_cast<size_t>(r) * p.ldh + c0);
-          uint4* lp = reinterpret_cast<uint4*>(p.Clo + static_cast<size_t>(r) * p.ldh + c0);
+          float4* hp = reinterpret_cast<float4*>(p.Chi + static_cast<size_t>(r) * p.ldh + c0);
+          float4* lp = reinterpret_cast<float4*>(p.Clo + static_cast<size_t>(r) * p.ldh + c0);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            uint32_t hw[4], lw[4];
+          for (int j = 0; j < 8; ++j) {
+            float hi[4], lo[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              __nv_bfloat16 h0, l0, h1, l1;
-              bf16_split(acc[cc * 32 + 8 * j + 2 * e], h0, l0);
-              bf16_split(acc[cc * 32 + 8 * j + 2 * e + 1], h1, l1);
-              hw[e] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) | (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
-              lw[e] = static_cast<uint32_t>(__bfloat16_as_ushort(l0)) | (static_cast<uint32_t>(__bfloat16_as_ushort(l1)) << 16);
+              const float x = acc[cc * 32 + 4 * j + e];
+              hi[e] = tf32_rn(x);
+              lo[e] = tf32_rn(x - hi[e]);
             }
-            hp[j] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-            lp[j] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            hp[j] = make_float4(hi[0], hi[1], hi[2], hi[3]);
+            lp[j] = make_float4(lo[0], lo[1], lo[2], lo[3]);
           }
         }
-        if (p.Ct || p.Cthi) {
+        if (p.Cthi) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const float x = acc[cc * 32 + j];
+            const float hi = tf32_rn(x);
             const size_t o = static_cast<size_t>(c0 + j) * p.ldt + r;
-            if (p.Ct) p.Ct[o] = x;
-            if (p.Cthi) bf16_split(x, p.Cthi[o], p.Ctlo[o]);
+            p.Cthi[o] = hi;
+            p.Ctlo[o] = tf32_rn(x - hi);
           }
         }
       }

@@ -41,18 +41,13 @@ struct gptq_ctx {
   int device = 0;
   cudaStream_t stream = nullptr;
   int64_t n = 0, m_max = 0;
-  // Each matrix of the factorization as an fp32 master and a bf16 hi/lo pair (tensor operands).
-  float* H = nullptr;                                  // [n x n] accumulated Hessian (upper triangle until mirrored)
-  float* A = nullptr;                                  // [n x n] damped, permuted H; Schur complements
-  __nv_bfloat16 *A_hi = nullptr, *A_lo = nullptr;
-  float* VT = nullptr;                                 // [n x n] V12 blocks (upper) and T^T blocks (lower)
-  __nv_bfloat16 *VT_hi = nullptr, *VT_lo = nullptr;
-  float* U = nullptr;                                  // [n x n] U (upper)
-  __nv_bfloat16 *U_hi = nullptr, *U_lo = nullptr;
-  float* Ut = nullptr;                                 // [n x n] U^T
-  __nv_bfloat16 *Ut_hi = nullptr, *Ut_lo = nullptr;
-  float* Wq = nullptr;                                 // [m_max x n] fp32 working weights
-  __nv_bfloat16 *Err_hi = nullptr, *Err_lo = nullptr;  // [m_max x kSuperBlock] block errors of a super-block
+  float* H = nullptr;                          // [n x n] accumulated Hessian (upper triangle until mirrored)
+  float *A_hi = nullptr, *A_lo = nullptr;      // [n x n] damped, permuted H; Schur complements
+  float *VT_hi = nullptr, *VT_lo = nullptr;    // [n x n] V12 blocks (upper) and T^T blocks (lower)
+  float *U_hi = nullptr, *U_lo = nullptr;      // [n x n] U (upper)
+  float *Ut_hi = nullptr, *Ut_lo = nullptr;    // [n x n] U^T
+  float* Wq = nullptr;                         // [m_max x n] fp32 working weights
+  float *Err_hi = nullptr, *Err_lo = nullptr;  // [m_max x kSuperBlock] block errors of a super-block
   float* keys = nullptr;
   uint8_t* dead = nullptr;
   int32_t* perm = nullptr;
@@ -235,72 +230,68 @@ double gemm_algo_flops(int M, int N, int K, int klo, int khi, int upper) {
   return 2.0 * total;
 }
 
-// 2-D tensor map of a row-major matrix (rows x cols, leading dimension ld elements): boxes of
-// 128 bytes (64 bf16 or 32 fp32) x box_rows rows, 128-byte swizzle.
-gptq_status make_map(gptq_ctx* c, CUtensorMap* map, const void* base, bool bf16, int64_t rows, int64_t cols,
-                     int64_t ld, int box_rows) {
-  const int esz = bf16 ? 2 : 4, box_cols = 128 / esz;
-  if (!aligned16(base) || (ld * esz) % 16 || cols % box_cols) return GPTQ_ERR_ARG;
+// 2-D fp32 tensor map of a row-major sub-matrix (rows x cols, leading dimension ld), boxes of
+// 32 columns x box_rows rows, 128-byte swizzle.
+gptq_status make_map(gptq_ctx* c, CUtensorMap* map, const float* base, int64_t rows, int64_t cols, int64_t ld,
+                     int box_rows) {
+  if (!aligned16(base) || ld % 4 || cols % GT_BK) return GPTQ_ERR_ARG;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * esz};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 4};
+  const cuuint32_t box[2] = {GT_BK, static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[2] = {1, 1};
-  CUresult r = c->encode(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
-                         const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  CUresult r = c->encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? GPTQ_OK : GPTQ_ERR_CUDA;
 }
 
-// C (+)= alpha * A B^T on the tensor cores, operands as bf16 hi/lo pairs (gemm_tc.cuh).
-// Outputs: fp32 C (with beta = 1 also the added C), its bf16 pair, the transposed fp32 result
-// and its bf16 pair (Ct and Cthi/Ctlo share ldt; C and Chi/Clo have their own leading dims).
+// C (+)= alpha * A B^T on the tensor cores, operands as tf32 hi/lo pairs (gemm_tc.cuh).
 struct TcOut {
   float* C = nullptr;
   int ldc = 0;
-  __nv_bfloat16* Chi = nullptr;
-  __nv_bfloat16* Clo = nullptr;
+  float* Chi = nullptr;
+  float* Clo = nullptr;
   int ldh = 0;
-  float* Ct = nullptr;
-  __nv_bfloat16* Cthi = nullptr;
-  __nv_bfloat16* Ctlo = nullptr;
+  float* Cthi = nullptr;
+  float* Ctlo = nullptr;
   int ldt = 0;
   const CUtensorMap* c_map = nullptr;  // C += ... by TMA reduce-add (beta = 1, plain C)
   int c_row0 = 0, c_col0 = 0;           // offset of C inside the matrix c_map describes
 };
 
 // An operand of gemm_tc: the hi/lo tensor maps of a whole matrix and the sub-block offset,
-// plus the sub-block's fp32 master pointer and leading dimension (for the CUDA-core path).
+// plus the sub-block's hi/lo pointers and leading dimension (for the CUDA-core path).
 struct TcOperand {
   const CUtensorMap* hi;
   const CUtensorMap* lo;
   int row0, col0;
-  const float* p32;
+  const float* phi;
+  const float* plo;
   int ld;
 };
 
 // Roles of the products gemm_tc runs (instrumentation names: kernel:role).
 enum : int { GR_V12 = 0, GR_SYRK, GR_T, GR_U12, GR_NEAR, GR_FAR, GR_TEST, GR_COUNT };
-const char* const kGemmTcNames[GR_COUNT] = {"gemm_bf16x3:factor_v12",    "gemm_bf16x3:factor_syrk",
-                                            "gemm_bf16x3:factor_t",      "gemm_bf16x3:factor_u12",
-                                            "gemm_bf16x3:trailing_near", "gemm_bf16x3:trailing_far",
-                                            "gemm_bf16x3:test"};
-const char* const kGemmSimtNames[GR_COUNT] = {"gemm_f32_simt:factor_v12",    "gemm_f32_simt:factor_syrk",
-                                              "gemm_f32_simt:factor_t",      "gemm_f32_simt:factor_u12",
-                                              "gemm_f32_simt:trailing_near", "gemm_f32_simt:trailing_far",
-                                              "gemm_f32_simt:test"};
+const char* const kGemmTcNames[GR_COUNT] = {"gemm_tf32x3:factor_v12",    "gemm_tf32x3:factor_syrk",
+                                            "gemm_tf32x3:factor_t",      "gemm_tf32x3:factor_u12",
+                                            "gemm_tf32x3:trailing_near", "gemm_tf32x3:trailing_far",
+                                            "gemm_tf32x3:test"};
+const char* const kGemmSimtNames[GR_COUNT] = {"gemm_hilo_simt:factor_v12",    "gemm_hilo_simt:factor_syrk",
+                                              "gemm_hilo_simt:factor_t",      "gemm_hilo_simt:factor_u12",
+                                              "gemm_hilo_simt:trailing_near", "gemm_hilo_simt:trailing_far",
+                                              "gemm_hilo_simt:test"};
 
 // Products with fewer tensor-core tiles (at the narrowest tile) than this run on the CUDA
 // cores (fp32, 32 x 32 or 64 x 64 tiles).
 constexpr int kMinTcTiles = 32;
 
 cudaError_t set_gemm_tc_attributes() {
-  cudaError_t e = cudaFuncSetAttribute(gemm_bf16x3_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(gemm_tf32x3_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        GtCfg<256>::SMEM);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(gemm_bf16x3_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, GtCfg<128>::SMEM);
+    e = cudaFuncSetAttribute(gemm_tf32x3_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, GtCfg<128>::SMEM);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(gemm_bf16x3_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, GtCfg<64>::SMEM);
+    e = cudaFuncSetAttribute(gemm_tf32x3_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, GtCfg<64>::SMEM);
   return e;
 }
 
@@ -348,15 +339,16 @@ gptq_status gemm_tc(gptq_ctx* c, int M, int N, int K, TcOperand A, TcOperand B, 
   if (N % 32 || K % GT_BK) return GPTQ_ERR_ARG;
   const int bn = force_bn ? force_bn : pick_bn(M, N, K, klo, khi, upper, c->num_sms);
   const int tc_tiles = gt_num_tiles(M, N, upper, bn);
-  if (beta && !o.C) return GPTQ_ERR_ARG;  // the added C is the fp32 one
-  if (gt_num_tiles(M, N, upper, 64) < kMinTcTiles && A.p32 && B.p32) {
+  if (gt_num_tiles(M, N, upper, 64) < kMinTcTiles && A.phi && B.phi) {
     GemmSimtArgs g;
     g.M = M;
     g.N = N;
     g.K = K;
-    g.A = A.p32;
+    g.A_hi = A.phi;
+    g.A_lo = A.plo;
     g.lda = A.ld;
-    g.B = B.p32;
+    g.B_hi = B.phi;
+    g.B_lo = B.plo;
     g.ldb = B.ld;
     g.alpha = alpha;
     g.beta = beta;
@@ -368,17 +360,16 @@ gptq_status gemm_tc(gptq_ctx* c, int M, int N, int K, TcOperand A, TcOperand B, 
     g.Chi = o.Chi;
     g.Clo = o.Clo;
     g.ldh = o.ldh;
-    g.Ct = o.Ct;
     g.Cthi = o.Cthi;
     g.Ctlo = o.Ctlo;
     g.ldt = o.ldt;
     tag(c, kGemmSimtNames[c->gemm_role], gemm_algo_flops(M, N, K, klo, khi, upper), 0.0);
     if (static_cast<int64_t>(M) * N <= 512 * 512) {  // 32 x 32 tiles: more CTAs for the smallest products
       dim3 grid((N + 31) / 32, (M + 31) / 32);
-      CK(launch(c, gemm_f32_simt_kernel<32, 32>, grid, dim3(GS_THREADS), gs_smem_bytes<32, 32>(), g));
+      CK(launch(c, gemm_hilo_simt_kernel<32, 32>, grid, dim3(GS_THREADS), gs_smem_bytes<32, 32>(), g));
     } else {
       dim3 grid((N + 63) / 64, (M + 63) / 64);
-      CK(launch(c, gemm_f32_simt_kernel<64, 64>, grid, dim3(GS_THREADS), gs_smem_bytes<64, 64>(), g));
+      CK(launch(c, gemm_hilo_simt_kernel<64, 64>, grid, dim3(GS_THREADS), gs_smem_bytes<64, 64>(), g));
     }
     CKL("gemm_simt");
     return GPTQ_OK;
@@ -402,7 +393,6 @@ gptq_status gemm_tc(gptq_ctx* c, int M, int N, int K, TcOperand A, TcOperand B, 
   a.Chi = o.Chi;
   a.Clo = o.Clo;
   a.ldh = o.ldh;
-  a.Ct = o.Ct;
   a.Cthi = o.Cthi;
   a.Ctlo = o.Ctlo;
   a.ldt = o.ldt;
@@ -415,11 +405,11 @@ gptq_status gemm_tc(gptq_ctx* c, int M, int N, int K, TcOperand A, TcOperand B, 
   const dim3 grid(std::min(tc_tiles, c->num_sms));
   tag(c, kGemmTcNames[c->gemm_role], gemm_algo_flops(M, N, K, klo, khi, upper), 0.0);
   if (bn == 256)
-    CK(launch(c, gemm_bf16x3_kernel<256>, grid, dim3(GT_THREADS), GtCfg<256>::SMEM, *A.hi, *A.lo, *B.hi, *B.lo, cm, a));
+    CK(launch(c, gemm_tf32x3_kernel<256>, grid, dim3(GT_THREADS), GtCfg<256>::SMEM, *A.hi, *A.lo, *B.hi, *B.lo, cm, a));
   else if (bn == 128)
-    CK(launch(c, gemm_bf16x3_kernel<128>, grid, dim3(GT_THREADS), GtCfg<128>::SMEM, *A.hi, *A.lo, *B.hi, *B.lo, cm, a));
+    CK(launch(c, gemm_tf32x3_kernel<128>, grid, dim3(GT_THREADS), GtCfg<128>::SMEM, *A.hi, *A.lo, *B.hi, *B.lo, cm, a));
   else
-    CK(launch(c, gemm_bf16x3_kernel<64>, grid, dim3(GT_THREADS), GtCfg<64>::SMEM, *A.hi, *A.lo, *B.hi, *B.lo, cm, a));
+    CK(launch(c, gemm_tf32x3_kernel<64>, grid, dim3(GT_THREADS), GtCfg<64>::SMEM, *A.hi, *A.lo, *B.hi, *B.lo, cm, a));
   CKL("gemm_tc");
   return GPTQ_OK;
 }
@@ -428,8 +418,8 @@ gptq_status gemm_tc(gptq_ctx* c, int M, int N, int K, TcOperand A, TcOperand B, 
 gptq_status chol_inv(gptq_ctx* c, int o, int h) {
   const int n = static_cast<int>(c->n);
   if (h <= LF_NB) {
-    tag(c, "leaf_chol_inv", 2.0 * LF_NB * LF_NB * LF_NB / 3.0, 4.0 * LF_NB * LF_NB * 3);
-    CK(launch(c, leaf_chol_inv_kernel, dim3(1), dim3(LF_THREADS), LF_SMEM, c->A, n, o, c->U, c->U_hi, c->U_lo,
+    tag(c, "leaf_chol_inv", 2.0 * LF_NB * LF_NB * LF_NB / 3.0, 4.0 * LF_NB * LF_NB * 4);
+    CK(launch(c, leaf_chol_inv_kernel, dim3(1), dim3(LF_THREADS), LF_SMEM, c->A_hi, c->A_lo, n, o, c->U_hi, c->U_lo,
               c->status));
     CKL("leaf_chol_inv");
     // U^T of the block, needed only by later T products and the sweep's trailing update: on
@@ -442,9 +432,9 @@ gptq_status chol_inv(gptq_ctx* c, int o, int h) {
       c->stream = c->side_stream;
       c->pdl = false;
     }
-    tag(c, "transpose_block", 0.0, 4.0 * LF_NB * LF_NB * 3);
-    const cudaError_t e = launch(c, transpose_block_kernel, dim3(4, 4), dim3(32, 8), 0, c->U, n, o, c->Ut, c->Ut_hi,
-                                 c->Ut_lo);
+    tag(c, "transpose_block", 0.0, 4.0 * LF_NB * LF_NB * 4);
+    const cudaError_t e = launch(c, transpose_block_kernel, dim3(4, 4), dim3(32, 8), 0, c->U_hi, c->U_lo, n, o,
+                                 c->Ut_hi, c->Ut_lo);
     if (branch) {
       c->stream = main_stream;
       c->pdl = true;
@@ -457,41 +447,36 @@ gptq_status chol_inv(gptq_ctx* c, int o, int h) {
   const int h1 = h - h2;
   const int o2 = o + h1;
   auto at = [n](float* M, int r, int col) { return M + static_cast<size_t>(r) * n + col; };
-  auto at16 = [n](__nv_bfloat16* M, int r, int col) { return M + static_cast<size_t>(r) * n + col; };
   gptq_status s;
   if ((s = chol_inv(c, o2, h2)) != GPTQ_OK) return s;
-  auto op = [n](CUtensorMap* m, float* p32, int r0, int c0) {
-    return TcOperand{&m[0], &m[1], r0, c0, p32 + static_cast<size_t>(r0) * n + c0, n};
+  auto op = [n](CUtensorMap* m, float* hi, float* lo, int r0, int c0) {
+    return TcOperand{&m[0], &m[1], r0, c0, hi + static_cast<size_t>(r0) * n + c0, lo + static_cast<size_t>(r0) * n + c0,
+                     n};
   };
   // V12 = A12 U22^T                      (U22 rows are the K-major B; k >= column)
   TcOut v12;
-  v12.C = at(c->VT, o, o2);
-  v12.ldc = n;
-  v12.Chi = at16(c->VT_hi, o, o2);
-  v12.Clo = at16(c->VT_lo, o, o2);
+  v12.Chi = at(c->VT_hi, o, o2);
+  v12.Clo = at(c->VT_lo, o, o2);
   v12.ldh = n;
   c->gemm_role = GR_V12;
-  if ((s = gemm_tc(c, h1, h2, h2, op(c->mA_A, c->A, o, o2), op(c->mB_U, c->U, o2, o2), 1.f, 0, GT_KLO_COL,
-                   GT_KHI_NONE, 0, v12)) != GPTQ_OK)
+  if ((s = gemm_tc(c, h1, h2, h2, op(c->mA_A, c->A_hi, c->A_lo, o, o2), op(c->mB_U, c->U_hi, c->U_lo, o2, o2), 1.f, 0, GT_KLO_COL, GT_KHI_NONE, 0,
+                   v12)) != GPTQ_OK)
     return s;
   // A11 -= V12 V12^T                     (upper tiles only)
   TcOut a11;
-  a11.C = at(c->A, o, o);
-  a11.ldc = n;
-  a11.Chi = at16(c->A_hi, o, o);
-  a11.Clo = at16(c->A_lo, o, o);
+  a11.Chi = at(c->A_hi, o, o);
+  a11.Clo = at(c->A_lo, o, o);
   a11.ldh = n;
   c->gemm_role = GR_SYRK;
-  if ((s = gemm_tc(c, h1, h1, h2, op(c->mA_VT, c->VT, o, o2), op(c->mB_VT, c->VT, o, o2), -1.f, 1, GT_KLO_NONE,
-                   GT_KHI_NONE, 1, a11)) != GPTQ_OK)
+  if ((s = gemm_tc(c, h1, h1, h2, op(c->mA_VT, c->VT_hi, c->VT_lo, o, o2), op(c->mB_VT, c->VT_hi, c->VT_lo, o, o2), -1.f, 1, GT_KLO_NONE, GT_KHI_NONE, 1,
+                   a11)) != GPTQ_OK)
     return s;
   // T^T = (V12 U22)^T into the lower block [o2.., o..]   (Ut22 rows as B; k <= column).
   // Only U12 below needs it, so while the graph is being captured it runs on a second
   // branch, beside the factorization of A11 (which touches only [o, o+h1)^2).
   TcOut tt;
-  tt.Ct = at(c->VT, o2, o);
-  tt.Cthi = at16(c->VT_hi, o2, o);
-  tt.Ctlo = at16(c->VT_lo, o2, o);
+  tt.Cthi = at(c->VT_hi, o2, o);
+  tt.Ctlo = at(c->VT_lo, o2, o);
   tt.ldt = n;
   const bool branch = c->side_stream != nullptr;
   cudaStream_t main_stream = c->stream;
@@ -502,8 +487,8 @@ gptq_status chol_inv(gptq_ctx* c, int o, int h) {
     c->pdl = false;
   }
   c->gemm_role = GR_T;
-  s = gemm_tc(c, h1, h2, h2, op(c->mA_VT, c->VT, o, o2), op(c->mB_Ut, c->Ut, o2, o2), 1.f, 0, GT_KLO_NONE,
-              GT_KHI_COL, 0, tt);
+  s = gemm_tc(c, h1, h2, h2, op(c->mA_VT, c->VT_hi, c->VT_lo, o, o2), op(c->mB_Ut, c->Ut_hi, c->Ut_lo, o2, o2), 1.f, 0,
+              GT_KLO_NONE, GT_KHI_COL, 0, tt);
   if (branch) {
     c->stream = main_stream;
     c->pdl = true;
@@ -515,18 +500,15 @@ gptq_status chol_inv(gptq_ctx* c, int o, int h) {
   if (branch) CK(cudaStreamWaitEvent(main_stream, c->ev_join, 0));
   // U12 = -U11 T  (and Ut21 = U12^T)      (U11 rows as A; k >= row)
   TcOut u12;
-  u12.C = at(c->U, o, o2);
-  u12.ldc = n;
-  u12.Chi = at16(c->U_hi, o, o2);
-  u12.Clo = at16(c->U_lo, o, o2);
+  u12.Chi = at(c->U_hi, o, o2);
+  u12.Clo = at(c->U_lo, o, o2);
   u12.ldh = n;
-  u12.Ct = at(c->Ut, o2, o);
-  u12.Cthi = at16(c->Ut_hi, o2, o);
-  u12.Ctlo = at16(c->Ut_lo, o2, o);
+  u12.Cthi = at(c->Ut_hi, o2, o);
+  u12.Ctlo = at(c->Ut_lo, o2, o);
   u12.ldt = n;
   c->gemm_role = GR_U12;
-  if ((s = gemm_tc(c, h1, h2, h1, op(c->mA_U, c->U, o, o), op(c->mB_VT, c->VT, o2, o), -1.f, 0, GT_KLO_ROW,
-                   GT_KHI_NONE, 0, u12)) != GPTQ_OK)
+  if ((s = gemm_tc(c, h1, h2, h1, op(c->mA_U, c->U_hi, c->U_lo, o, o), op(c->mB_VT, c->VT_hi, c->VT_lo, o2, o), -1.f, 0, GT_KLO_ROW, GT_KHI_NONE, 0,
+                   u12)) != GPTQ_OK)
     return s;
   return GPTQ_OK;
 }
@@ -537,23 +519,22 @@ gptq_status encode_maps(gptq_ctx* c) {
   gptq_status s;
   struct M {
     CUtensorMap* m;
-    const void* p;
-    bool bf16;
+    float* p;
     int64_t rows, cols, ld;
     int box;
   } list[] = {
-      {&c->mA_A[0], c->A_hi, true, n, n, n, GT_BM},        {&c->mA_A[1], c->A_lo, true, n, n, n, GT_BM},
-      {&c->mA_VT[0], c->VT_hi, true, n, n, n, GT_BM},      {&c->mA_VT[1], c->VT_lo, true, n, n, n, GT_BM},
-      {&c->mA_U[0], c->U_hi, true, n, n, n, GT_BM},        {&c->mA_U[1], c->U_lo, true, n, n, n, GT_BM},
-      {&c->mA_Err[0], c->Err_hi, true, c->m_max, kSuperBlock, kSuperBlock, GT_BM},
-      {&c->mA_Err[1], c->Err_lo, true, c->m_max, kSuperBlock, kSuperBlock, GT_BM},
-      {&c->mB_U[0], c->U_hi, true, n, n, n, GT_BOX_N},     {&c->mB_U[1], c->U_lo, true, n, n, n, GT_BOX_N},
-      {&c->mB_VT[0], c->VT_hi, true, n, n, n, GT_BOX_N},   {&c->mB_VT[1], c->VT_lo, true, n, n, n, GT_BOX_N},
-      {&c->mB_Ut[0], c->Ut_hi, true, n, n, n, GT_BOX_N},   {&c->mB_Ut[1], c->Ut_lo, true, n, n, n, GT_BOX_N},
-      {&c->mC_Wq, c->Wq, false, c->m_max, n, n, 32},
+      {&c->mA_A[0], c->A_hi, n, n, n, GT_BM},        {&c->mA_A[1], c->A_lo, n, n, n, GT_BM},
+      {&c->mA_VT[0], c->VT_hi, n, n, n, GT_BM},      {&c->mA_VT[1], c->VT_lo, n, n, n, GT_BM},
+      {&c->mA_U[0], c->U_hi, n, n, n, GT_BM},        {&c->mA_U[1], c->U_lo, n, n, n, GT_BM},
+      {&c->mA_Err[0], c->Err_hi, c->m_max, kSuperBlock, kSuperBlock, GT_BM},
+      {&c->mA_Err[1], c->Err_lo, c->m_max, kSuperBlock, kSuperBlock, GT_BM},
+      {&c->mB_U[0], c->U_hi, n, n, n, GT_BOX_N},        {&c->mB_U[1], c->U_lo, n, n, n, GT_BOX_N},
+      {&c->mB_VT[0], c->VT_hi, n, n, n, GT_BOX_N},      {&c->mB_VT[1], c->VT_lo, n, n, n, GT_BOX_N},
+      {&c->mB_Ut[0], c->Ut_hi, n, n, n, GT_BOX_N},      {&c->mB_Ut[1], c->Ut_lo, n, n, n, GT_BOX_N},
+      {&c->mC_Wq, c->Wq, c->m_max, n, n, 32},
   };
   for (auto& e : list)
-    if ((s = make_map(c, e.m, e.p, e.bf16, e.rows, e.cols, e.ld, e.box)) != GPTQ_OK) return s;
+    if ((s = make_map(c, e.m, e.p, e.rows, e.cols, e.ld, e.box)) != GPTQ_OK) return s;
   return GPTQ_OK;
 }
 
@@ -605,17 +586,12 @@ gptq_status run_factorization(gptq_ctx* c) {
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
-  static PFN_cuTensorMapEncodeTiled_v12000 cached = nullptr;
-  static std::mutex mu;
-  std::lock_guard<std::mutex> lk(mu);
-  if (cached) return cached;
   void* fn = nullptr;
   cudaDriverEntryPointQueryResult q;
   if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
       q != cudaDriverEntryPointSuccess)
     return nullptr;
-  cached = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-  return cached;
+  return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
 }
 
 void free_prof(gptq_ctx* c) {
@@ -637,15 +613,9 @@ void free_all(gptq_ctx* c) {
   c->ev_fork = c->ev_join = nullptr;
   c->factor_graph = nullptr;
   c->capture_stream = nullptr;
-  float** fs[] = {&c->H, &c->A, &c->VT, &c->U, &c->Ut, &c->Wq, &c->keys};
+  float** fs[] = {&c->H,     &c->A_hi,  &c->A_lo,  &c->VT_hi, &c->VT_lo,  &c->U_hi,   &c->U_lo,
+                  &c->Ut_hi, &c->Ut_lo, &c->Wq,    &c->Err_hi, &c->Err_lo, &c->keys};
   for (float** p : fs)
-    if (*p) {
-      cudaFree(*p);
-      *p = nullptr;
-    }
-  __nv_bfloat16** bs[] = {&c->A_hi, &c->A_lo, &c->VT_hi, &c->VT_lo, &c->U_hi,
-                          &c->U_lo, &c->Ut_hi, &c->Ut_lo, &c->Err_hi, &c->Err_lo};
-  for (__nv_bfloat16** p : bs)
     if (*p) {
       cudaFree(*p);
       *p = nullptr;
@@ -692,9 +662,9 @@ const char* gptq_status_string(gptq_status s) {
 size_t gptq_workspace_bytes(int64_t n, int64_t m_max) {
   if (n < 128 || n > kMaxN || n % 128 || m_max < 1 || m_max > kMaxM) return 0;
   const size_t nn = static_cast<size_t>(n) * static_cast<size_t>(n);
-  size_t b = 5 * nn * sizeof(float) + 8 * nn * 2;                                 // H, A, VT, U, Ut; bf16 pairs
+  size_t b = 9 * nn * sizeof(float);                                              // H, A, VT, U, Ut (hi/lo)
   b += static_cast<size_t>(m_max) * static_cast<size_t>(n) * sizeof(float);       // Wq
-  b += 2 * static_cast<size_t>(m_max) * kSuperBlock * 2;                          // Err hi/lo (bf16)
+  b += 2 * static_cast<size_t>(m_max) * kSuperBlock * sizeof(float);              // Err hi/lo
   b += static_cast<size_t>(n) * (sizeof(float) + 1 + sizeof(int32_t)) + sizeof(double) + sizeof(int);
   return b;
 }
@@ -733,12 +703,12 @@ gptq_status gptq_create(gptq_ctx** out, int64_t n, int64_t m_max, int device, vo
   auto alloc = [&](void** p, size_t bytes) {
     if (e == cudaSuccess) e = cudaMalloc(p, bytes);
   };
-  for (float** p : {&c->H, &c->A, &c->VT, &c->U, &c->Ut}) alloc(reinterpret_cast<void**>(p), nn * 4);
-  for (__nv_bfloat16** p : {&c->A_hi, &c->A_lo, &c->VT_hi, &c->VT_lo, &c->U_hi, &c->U_lo, &c->Ut_hi, &c->Ut_lo})
-    alloc(reinterpret_cast<void**>(p), nn * 2);
+  alloc(reinterpret_cast<void**>(&c->H), nn * 4);
+  for (float** p : {&c->A_hi, &c->A_lo, &c->VT_hi, &c->VT_lo, &c->U_hi, &c->U_lo, &c->Ut_hi, &c->Ut_lo})
+    alloc(reinterpret_cast<void**>(p), nn * 4);
   alloc(reinterpret_cast<void**>(&c->Wq), static_cast<size_t>(m_max) * n * 4);
-  alloc(reinterpret_cast<void**>(&c->Err_hi), static_cast<size_t>(m_max) * kSuperBlock * 2);
-  alloc(reinterpret_cast<void**>(&c->Err_lo), static_cast<size_t>(m_max) * kSuperBlock * 2);
+  alloc(reinterpret_cast<void**>(&c->Err_hi), static_cast<size_t>(m_max) * kSuperBlock * 4);
+  alloc(reinterpret_cast<void**>(&c->Err_lo), static_cast<size_t>(m_max) * kSuperBlock * 4);
   alloc(reinterpret_cast<void**>(&c->keys), n * 4);
   alloc(reinterpret_cast<void**>(&c->dead), n);
   alloc(reinterpret_cast<void**>(&c->perm), n * 4);
@@ -761,10 +731,10 @@ gptq_status gptq_create(gptq_ctx** out, int64_t n, int64_t m_max, int device, vo
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(leaf_chol_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, LF_SMEM);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(gemm_f32_simt_kernel<64, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(gemm_hilo_simt_kernel<64, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              gs_smem_bytes<64, 64>());
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(gemm_f32_simt_kernel<32, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(gemm_hilo_simt_kernel<32, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              gs_smem_bytes<32, 32>());
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(sweep_block_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, SW_SMEM);
@@ -873,13 +843,11 @@ gptq_status gptq_prepare(gptq_ctx* c, double damp, int desc_act, int32_t* perm_o
     CK(launch(c, identity_perm_kernel, dim3((n + 255) / 256), dim3(256), 0, n, c->perm));
   CKL("perm");
   tag(c, "prepare:gather_damp", 0.0, 12.0 * n * n);
-  CK(launch(c, gather_damp_kernel, dim3(n), dim3(GD_THREADS), static_cast<size_t>(n) * 4, c->H, n, c->perm, c->keys,
-            c->mean, damp, c->A, c->A_hi, c->A_lo));
+  CK(launch(c, gather_damp_kernel, dim3(n), dim3(GD_THREADS), static_cast<size_t>(n) * 4, c->H, n, c->perm, c->keys, c->mean, damp,
+                                                                        c->A_hi, c->A_lo));
   CKL("gather");
   const size_t nn = static_cast<size_t>(n) * n;
-  // U and U^T below (above) their diagonals stay zero: the recursion writes only the other half
-  for (float* p : {c->U, c->Ut}) CK(cudaMemsetAsync(p, 0, nn * 4, c->stream));
-  for (__nv_bfloat16* p : {c->U_hi, c->U_lo, c->Ut_hi, c->Ut_lo}) CK(cudaMemsetAsync(p, 0, nn * 2, c->stream));
+  for (float* p : {c->U_hi, c->U_lo, c->Ut_hi, c->Ut_lo}) CK(cudaMemsetAsync(p, 0, nn * 4, c->stream));
   if ((s = run_factorization(c)) != GPTQ_OK) return s;
   if (perm_out) CK(cudaMemcpyAsync(perm_out, c->perm, n * 4, cudaMemcpyDeviceToDevice, c->stream));
   int flags = 0;
@@ -894,7 +862,9 @@ gptq_status gptq_get_factor(gptq_ctx* c, float* U_out) {
   if (c->state != ST_PREPARED) return GPTQ_ERR_STATE;
   DeviceGuard dg(c->device);
   const size_t nn = static_cast<size_t>(c->n) * c->n;
-  CK(cudaMemcpyAsync(U_out, c->U, nn * 4, cudaMemcpyDeviceToDevice, c->stream));
+  tag(c, "combine_hilo", 0.0, 12.0 * static_cast<double>(nn));
+  CK(launch(c, combine_hilo_kernel, dim3(592), dim3(256), 0, c->U_hi, c->U_lo, nn, U_out));
+  CKL("combine");
   return GPTQ_OK;
 }
 
@@ -972,9 +942,9 @@ gptq_status gptq_quantize_layer(gptq_ctx* c, const void* W, int64_t m, gptq_qpar
   CKL("init_w");
   SweepArgs a;
   a.Wq = c->Wq;
-  a.U = c->U;
-  a.Err = nullptr;
-  a.Err_hi = c->Err_hi;
+  a.U = c->U_hi;
+  a.U_lo = c->U_lo;
+  a.Err = c->Err_hi;
   a.Err_lo = c->Err_lo;
   a.codes = codes;
   a.scales = scales;
@@ -991,8 +961,8 @@ gptq_status gptq_quantize_layer(gptq_ctx* c, const void* W, int64_t m, gptq_qpar
   const int grid = (mi + SW_ROWS - 1) / SW_ROWS;
   // algorithmic bytes of one sweep block: W tile in, scaled errors out (hi/lo), codes,
   // scales/zeros of the groups that start in it, the U block (hi/lo)
-  const double sweep_bytes = 4.0 * mi * SW_B + 4.0 * mi * SW_B + mi * SW_B * qp.bits / 8.0 +
-                             8.0 * mi * std::max(1, SW_B / g) + 4.0 * SW_B * SW_B + (W_hat ? 4.0 * mi * SW_B : 0.0);
+  const double sweep_bytes = 4.0 * mi * SW_B + 8.0 * mi * SW_B + mi * SW_B * qp.bits / 8.0 +
+                             8.0 * mi * std::max(1, SW_B / g) + 8.0 * SW_B * SW_B + (W_hat ? 4.0 * mi * SW_B : 0.0);
   // two-level lazy update: inside a super-block the columns after each 128-block are updated
   // right away; the columns beyond the super-block receive all its block errors in one product
   // (K = super-block width).  A group that starts inside a super-block must not reach past it.
@@ -1018,8 +988,8 @@ gptq_status gptq_quantize_layer(gptq_ctx* c, const void* W, int64_t m, gptq_qpar
         w.c_map = &c->mC_Wq;
         w.c_col0 = i2;
         c->gemm_role = GR_NEAR;
-        gptq_status st = gemm_tc(c, mi, s1 - i2, SW_B, TcOperand{&c->mA_Err[0], &c->mA_Err[1], 0, i1 - s0, nullptr, 0},
-                                 TcOperand{&c->mB_Ut[0], &c->mB_Ut[1], i2, i1, nullptr, 0}, -1.f, 1,
+        gptq_status st = gemm_tc(c, mi, s1 - i2, SW_B, TcOperand{&c->mA_Err[0], &c->mA_Err[1], 0, i1 - s0, nullptr, nullptr, 0},
+                                 TcOperand{&c->mB_Ut[0], &c->mB_Ut[1], i2, i1, nullptr, nullptr, 0}, -1.f, 1,
                                  GT_KLO_NONE, GT_KHI_NONE, 0, w, SW_B / GT_BK);
         if (st != GPTQ_OK) return st;
       }
@@ -1032,8 +1002,8 @@ gptq_status gptq_quantize_layer(gptq_ctx* c, const void* W, int64_t m, gptq_qpar
       w.c_map = &c->mC_Wq;
       w.c_col0 = s1;
       c->gemm_role = GR_FAR;
-      gptq_status st = gemm_tc(c, mi, n - s1, s1 - s0, TcOperand{&c->mA_Err[0], &c->mA_Err[1], 0, 0, nullptr, 0},
-                               TcOperand{&c->mB_Ut[0], &c->mB_Ut[1], s1, s0, nullptr, 0}, -1.f, 1,
+      gptq_status st = gemm_tc(c, mi, n - s1, s1 - s0, TcOperand{&c->mA_Err[0], &c->mA_Err[1], 0, 0, nullptr, nullptr, 0},
+                               TcOperand{&c->mB_Ut[0], &c->mB_Ut[1], s1, s0, nullptr, nullptr, 0}, -1.f, 1,
                                GT_KLO_NONE, GT_KHI_NONE, 0, w, SW_B / GT_BK);
       if (st != GPTQ_OK) return st;
     }
@@ -1067,19 +1037,18 @@ gptq_status gptq_reset(gptq_ctx* c) {
 
 int64_t gptq_launch_count(const gptq_ctx* c) { return c ? c->launches : -1; }
 
-gptq_status gptq_test_gemm_bf16x3(int M, int N, int K, const void* A_hi, const void* A_lo, int lda, const void* B_hi,
-                                  const void* B_lo, int ldb, float alpha, int beta, int k_lo_mode, int k_hi_mode,
-                                  int upper_only, float* C, int ldc, void* C_hi, void* C_lo, int ldh, float* Ct,
-                                  void* Ct_hi, void* Ct_lo, int ldt, int chunk_stages, int tile_n, int c_reduce,
-                                  int device, void* cuda_stream) {
+gptq_status gptq_test_gemm_tf32x3(int M, int N, int K, const float* A_hi, const float* A_lo, int lda, const float* B_hi,
+                                  const float* B_lo, int ldb, float alpha, int beta, int k_lo_mode, int k_hi_mode,
+                                  int upper_only, float* C, int ldc, float* C_hi, float* C_lo, int ldh, float* Ct_hi,
+                                  float* Ct_lo, int ldt, int chunk_stages, int tile_n, int c_reduce, int device,
+                                  void* cuda_stream) {
   if (chunk_stages < 1) return GPTQ_ERR_ARG;
   if (c_reduce && (!C || beta != 1)) return GPTQ_ERR_ARG;
-  if (beta && !C) return GPTQ_ERR_ARG;
   if (tile_n != 0 && tile_n != 64 && tile_n != 128 && tile_n != 256) return GPTQ_ERR_ARG;
-  if (!A_hi || !A_lo || !B_hi || !B_lo || M < 1 || N < 1 || K < GT_BK || K % GT_BK || N % 32) return GPTQ_ERR_ARG;
+  if (!A_hi || !A_lo || !B_hi || !B_lo || M < 1 || N < 1 || K < GT_BK) return GPTQ_ERR_ARG;
   if (k_lo_mode < 0 || k_lo_mode > 2 || k_hi_mode < 0 || k_hi_mode > 1 || (beta != 0 && beta != 1)) return GPTQ_ERR_ARG;
   if ((C_hi == nullptr) != (C_lo == nullptr) || (Ct_hi == nullptr) != (Ct_lo == nullptr)) return GPTQ_ERR_ARG;
-  if ((C && (!aligned16(C) || ldc % 4)) || (C_hi && (!aligned16(C_hi) || !aligned16(C_lo) || ldh % 8)))
+  if ((C && (!aligned16(C) || ldc % 4)) || (C_hi && (!aligned16(C_hi) || !aligned16(C_lo) || ldh % 4)))
     return GPTQ_ERR_ARG;
   int ndev = 0;
   if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) {
@@ -1099,27 +1068,26 @@ gptq_status gptq_test_gemm_bf16x3(int M, int N, int K, const void* A_hi, const v
   TcOut o;
   o.C = C;
   o.ldc = ldc;
-  o.Chi = static_cast<__nv_bfloat16*>(C_hi);
-  o.Clo = static_cast<__nv_bfloat16*>(C_lo);
+  o.Chi = C_hi;
+  o.Clo = C_lo;
   o.ldh = ldh;
-  o.Ct = Ct;
-  o.Cthi = static_cast<__nv_bfloat16*>(Ct_hi);
-  o.Ctlo = static_cast<__nv_bfloat16*>(Ct_lo);
+  o.Cthi = Ct_hi;
+  o.Ctlo = Ct_lo;
   o.ldt = ldt;
   CUtensorMap ma[2], mb[2], mc;
   gptq_status s = GPTQ_OK;
   t.gemm_role = GR_TEST;
   if (c_reduce) {
-    s = make_map(&t, &mc, C, false, M, N, ldc, 32);
+    s = make_map(&t, &mc, C, M, N, ldc, 32);
     o.c_map = &mc;
   }
-  if (s == GPTQ_OK) s = make_map(&t, &ma[0], A_hi, true, M, K, lda, GT_BM);
-  if (s == GPTQ_OK) s = make_map(&t, &ma[1], A_lo, true, M, K, lda, GT_BM);
-  if (s == GPTQ_OK) s = make_map(&t, &mb[0], B_hi, true, N, K, ldb, GT_BOX_N);
-  if (s == GPTQ_OK) s = make_map(&t, &mb[1], B_lo, true, N, K, ldb, GT_BOX_N);
+  if (s == GPTQ_OK) s = make_map(&t, &ma[0], A_hi, M, K, lda, GT_BM);
+  if (s == GPTQ_OK) s = make_map(&t, &ma[1], A_lo, M, K, lda, GT_BM);
+  if (s == GPTQ_OK) s = make_map(&t, &mb[0], B_hi, N, K, ldb, GT_BOX_N);
+  if (s == GPTQ_OK) s = make_map(&t, &mb[1], B_lo, N, K, ldb, GT_BOX_N);
   if (s == GPTQ_OK)
-    s = gemm_tc(&t, M, N, K, TcOperand{&ma[0], &ma[1], 0, 0, nullptr, 0},
-                TcOperand{&mb[0], &mb[1], 0, 0, nullptr, 0}, alpha, beta, k_lo_mode, k_hi_mode, upper_only, o,
+    s = gemm_tc(&t, M, N, K, TcOperand{&ma[0], &ma[1], 0, 0, nullptr, nullptr, 0},
+                TcOperand{&mb[0], &mb[1], 0, 0, nullptr, nullptr, 0}, alpha, beta, k_lo_mode, k_hi_mode, upper_only, o,
                 chunk_stages, tile_n);
   int flags = 0;
   cudaMemcpyAsync(&flags, t.status, sizeof(int), cudaMemcpyDeviceToHost, t.stream);
@@ -1293,8 +1261,8 @@ extern "C" gptq_status gptq_quantize_layer_noalloc(const void* W, int64_t m, int
   SweepArgs a;
   a.Wq = Wq;
   a.U = U;
+  a.U_lo = nullptr;
   a.Err = Err;
-  a.Err_hi = nullptr;
   a.Err_lo = nullptr;
   a.ld_err = SW_B;
   a.err_col0 = 0;
@@ -1339,7 +1307,6 @@ extern "C" gptq_status gptq_quantize_layer_noalloc(const void* W, int64_t m, int
 namespace {
 
 constexpr int kDqPlanSms = 148;  // the split-K plan is fixed so that the workspace size is a pure function
-constexpr int kNoAllocMaxDevicesFwd = 64;
 
 struct DqPlan {
   int tn = 0, tiles_m = 0, tiles_t = 0, k_tiles = 0, k_per = 0, splits = 0;
@@ -1369,19 +1336,9 @@ bool dq_plan(int64_t T, int64_t m, int64_t n, int act_order, DqPlan* p) {
   return true;
 }
 
-// Raise a kernel's dynamic shared-memory limit once per device (later calls, which may be
-// recorded into a graph, then make no attribute call).
-std::mutex g_attr_mu;
-int g_attr_smem[kNoAllocMaxDevicesFwd][8] = {};
-
-template <typename K>
-cudaError_t ensure_smem_attr(int device, int slot, K kernel, int smem) {
-  std::lock_guard<std::mutex> lk(g_attr_mu);
-  if (device < 0 || device >= kNoAllocMaxDevicesFwd) return cudaErrorInvalidDevice;
-  if (g_attr_smem[device][slot] >= smem) return cudaSuccess;
-  const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e == cudaSuccess) g_attr_smem[device][slot] = smem;
-  return e;
+template <int BITS>
+cudaError_t set_dq_attr(int smem) {
+  return cudaFuncSetAttribute(dequant_gemm_kernel<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
 }
 
 }  // namespace
@@ -1420,7 +1377,7 @@ extern "C" gptq_status gptq_dequant_matmul(const void* X, int64_t T, const uint3
   const __half* Xs = static_cast<const __half*>(X);
   if (perm) {
     __half* Xp = reinterpret_cast<__half*>(ws + pl.xp_off);
-    CK(ensure_smem_attr(device, 4, permute_x_kernel, ni * 2));
+    CK(cudaFuncSetAttribute(permute_x_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ni * 2));
     permute_x_kernel<<<Ti, 256, static_cast<size_t>(ni) * 2, st>>>(Xs, ni, perm, Xp);
     CKL("permute_x");
     Xs = Xp;
@@ -1464,19 +1421,19 @@ extern "C" gptq_status gptq_dequant_matmul(const void* X, int64_t T, const uint3
   const dim3 grid(pl.tiles_m, pl.tiles_t, pl.splits);
   switch (bits) {
     case 2:
-      CK(ensure_smem_attr(device, 0, dequant_gemm_kernel<2>, smem));
+      CK(set_dq_attr<2>(smem));
       dequant_gemm_kernel<2><<<grid, DQ_THREADS, smem, st>>>(cmap, xmap, a);
       break;
     case 3:
-      CK(ensure_smem_attr(device, 1, dequant_gemm_kernel<3>, smem));
+      CK(set_dq_attr<3>(smem));
       dequant_gemm_kernel<3><<<grid, DQ_THREADS, smem, st>>>(cmap, xmap, a);
       break;
     case 4:
-      CK(ensure_smem_attr(device, 2, dequant_gemm_kernel<4>, smem));
+      CK(set_dq_attr<4>(smem));
       dequant_gemm_kernel<4><<<grid, DQ_THREADS, smem, st>>>(cmap, xmap, a);
       break;
     default:
-      CK(ensure_smem_attr(device, 3, dequant_gemm_kernel<8>, smem));
+      CK(set_dq_attr<8>(smem));
       dequant_gemm_kernel<8><<<grid, DQ_THREADS, smem, st>>>(cmap, xmap, a);
       break;
   }

@@ -6,8 +6,7 @@
 //                         ("模型量化实战…" §3.2 prepare: damp = 0.01 * mean(diag H))
 //   rank_perm_kernel      desc_act: stable descending order of diag H by rank counting
 //                         ("GPTQ量化损失深度解析…": desc_act=True, 按敏感度排序)
-//   gather_damp_kernel    A = H[perm][:, perm] + damp * mean(diag) * I  (row staged in smem),
-//                         as fp32 master and bf16 hi/lo pair
+//   gather_damp_kernel    A = H[perm][:, perm] + damp * mean(diag) * I  (row staged in smem)
 //   init_w_kernel         Wq = fp32(W[:, perm]) with dead columns zeroed
 //   g_idx_kernel          g_idx[perm[k]] = k / group_size
 #pragma once
@@ -96,15 +95,13 @@ __global__ void identity_perm_kernel(int n, int32_t* __restrict__ perm) {
 
 // One CTA (1024 threads) per output row a: the source row perm[a] of the (mirrored) H is
 // staged in shared memory, then gathered by perm four columns at a time (16-byte loads of
-// perm; 16-byte stores of the fp32 master, 8-byte stores of its bf16 hi and lo parts).
-// n % 4 == 0.
+// perm, 16-byte stores of the hi and lo parts).  n % 4 == 0.
 constexpr int GD_THREADS = 1024;
 __global__ void __launch_bounds__(GD_THREADS) gather_damp_kernel(const float* __restrict__ H, int n,
                                                                  const int32_t* __restrict__ perm,
                                                                  const float* __restrict__ keys,
                                                                  const double* __restrict__ mean, double damp,
-                                                                 float* __restrict__ A, __nv_bfloat16* __restrict__ A_hi,
-                                                                 __nv_bfloat16* __restrict__ A_lo) {
+                                                                 float* __restrict__ A_hi, float* __restrict__ A_lo) {
   griddep_wait();
   griddep_launch_dependents();
   extern __shared__ float row_s[];
@@ -114,23 +111,21 @@ __global__ void __launch_bounds__(GD_THREADS) gather_damp_kernel(const float* __
   for (int k = threadIdx.x; k < n / 4; k += blockDim.x) reinterpret_cast<float4*>(row_s)[k] = src[k];
   const float dval = static_cast<float>(static_cast<double>(keys[pa]) + damp * (*mean));
   __syncthreads();
-  float4* dm = reinterpret_cast<float4*>(A + static_cast<size_t>(a) * n);
-  uint2* dh = reinterpret_cast<uint2*>(A_hi + static_cast<size_t>(a) * n);
-  uint2* dl = reinterpret_cast<uint2*>(A_lo + static_cast<size_t>(a) * n);
+  float4* dh = reinterpret_cast<float4*>(A_hi + static_cast<size_t>(a) * n);
+  float4* dl = reinterpret_cast<float4*>(A_lo + static_cast<size_t>(a) * n);
   const int4* p4 = reinterpret_cast<const int4*>(perm);
   for (int b4 = threadIdx.x; b4 < n / 4; b4 += blockDim.x) {
     const int4 pb = p4[b4];
     float v[4] = {row_s[pb.x], row_s[pb.y], row_s[pb.z], row_s[pb.w]};
-    __nv_bfloat16 hi[4], lo[4];
+    float hi[4], lo[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       if (4 * b4 + e == a) v[e] = dval;
-      hi[e] = __float2bfloat16_rn(v[e]);
-      lo[e] = __float2bfloat16_rn(v[e] - __bfloat162float(hi[e]));
+      hi[e] = tf32_round(v[e]);
+      lo[e] = tf32_round(v[e] - hi[e]);
     }
-    dm[b4] = make_float4(v[0], v[1], v[2], v[3]);
-    dh[b4] = make_uint2(bf16x2_bits(hi[0], hi[1]), bf16x2_bits(hi[2], hi[3]));
-    dl[b4] = make_uint2(bf16x2_bits(lo[0], lo[1]), bf16x2_bits(lo[2], lo[3]));
+    dh[b4] = make_float4(hi[0], hi[1], hi[2], hi[3]);
+    dl[b4] = make_float4(lo[0], lo[1], lo[2], lo[3]);
   }
 }
 
@@ -149,6 +144,16 @@ __global__ void init_w_kernel(const __half* __restrict__ W, int n, const int32_t
     const int p = perm[k];
     dst[k] = dead[p] ? 0.0f : __half2float(wrow_s[p]);
   }
+}
+
+// out = hi + lo (the fp32 value of a hi/lo pair)
+__global__ void combine_hilo_kernel(const float* __restrict__ hi, const float* __restrict__ lo, size_t count,
+                                    float* __restrict__ out) {
+  griddep_wait();
+  griddep_launch_dependents();
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < count;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    out[i] = hi[i] + lo[i];
 }
 
 __global__ void g_idx_kernel(const int32_t* __restrict__ perm, int n, int g, int32_t* __restrict__ g_idx) {

@@ -13,8 +13,6 @@
 // buffering of the shared-memory tiles.
 #pragma once
 
-#include <cuda_bf16.h>
-
 #include <cstdint>
 
 #include "sm100_ptx.cuh"
@@ -154,27 +152,25 @@ __global__ void __launch_bounds__(SG_THREADS)
 
 namespace gptq {
 
-// CUDA-core fp32 GEMM with the same interface as the tensor-core GEMM (gemm_tc.cuh):
-// C = alpha * A * B^T (+ C), A [M x K] and B [N x K] row-major fp32 (the masters of the
-// factorization's matrices), the same K-range rules for triangular operands and the same
-// outputs (fp32, bf16 pair, transposed fp32, transposed bf16 pair).  Used for the
-// factorization's small products, where 32 x 32 or 64 x 64 tiles spread the work over more
-// SMs than the 128 x 256 tensor-core tiles and the fixed cost of a tensor-core pipeline would
-// dominate.
+// CUDA-core fp32 GEMM on hi/lo operands, with the same interface as the tensor-core GEMM
+// (gemm_tc.cuh): C = alpha * A * B^T (+ C), A [M x K] and B [N x K] given as hi/lo pairs
+// (summed to fp32 on load), the same K-range rules for triangular operands and the same
+// outputs.  Used for the factorization's small products, where 64 x 64 tiles spread the
+// work over more SMs than the 128 x 256 tensor-core tiles and the fixed cost of a
+// tensor-core pipeline would dominate.
 struct GemmSimtArgs {
   int M, N, K;
-  const float* A;
+  const float *A_hi, *A_lo;
   int lda;
-  const float* B;
+  const float *B_hi, *B_lo;
   int ldb;
   float alpha;
   int beta, k_lo_mode, k_hi_mode, upper_only;
   float* C;
   int ldc;
-  __nv_bfloat16 *Chi, *Clo;
+  float *Chi, *Clo;
   int ldh;
-  float* Ct;
-  __nv_bfloat16 *Cthi, *Ctlo;
+  float *Cthi, *Ctlo;
   int ldt;
 };
 
@@ -182,7 +178,13 @@ constexpr int GS_BK = 32, GS_STAGES = 3, GS_THREADS = 256, GS_LD = GS_BK + 4;
 
 template <int TM, int TN>
 constexpr int gs_smem_bytes() {
-  return GS_STAGES * (TM + TN) * GS_LD * 4;
+  return GS_STAGES * 2 * (TM + TN) * GS_LD * 4;
+}
+
+__device__ __forceinline__ float tf32_rn_simt(float x) {
+  uint32_t u = __float_as_uint(x);
+  u += 0xFFFu + ((u >> 13) & 1u);
+  return __uint_as_float(u & 0xFFFFE000u);
 }
 
 __device__ __forceinline__ void gs_cp_async16(void* smem_dst, const void* gmem_src, bool pred) {
@@ -193,10 +195,10 @@ __device__ __forceinline__ void gs_cp_async16(void* smem_dst, const void* gmem_s
 
 // TM x TN output tile, 256 threads laid out 16 x 16; thread (tx, ty) owns rows ty + 16 i and
 // columns tx + 16 j (strided, so that the shared-memory reads of a warp hit distinct banks).
-// K streams through a 3-stage cp.async ring of 32-wide tiles of A and B (K-major, 36-float
-// padded rows).
+// K streams through a 3-stage cp.async ring of 32-wide tiles of A_hi, A_lo, B_hi, B_lo
+// (K-major, 36-float padded rows); hi + lo are summed as they are read.
 template <int TM, int TN>
-__global__ void __launch_bounds__(GS_THREADS) gemm_f32_simt_kernel(GemmSimtArgs p) {
+__global__ void __launch_bounds__(GS_THREADS) gemm_hilo_simt_kernel(GemmSimtArgs p) {
   constexpr int RI = TM / 16, RJ = TN / 16;
   griddep_wait();
   griddep_launch_dependents();
@@ -212,23 +214,27 @@ __global__ void __launch_bounds__(GS_THREADS) gemm_f32_simt_kernel(GemmSimtArgs 
   extern __shared__ __align__(16) float gs_smem[];
   const int tid = threadIdx.x;
   const int tx = tid & 15, ty = tid >> 4;
-  auto stage_ptr = [&](int s) { return gs_smem + s * (TM + TN) * GS_LD; };
+  auto stage_ptr = [&](int s) { return gs_smem + s * 2 * (TM + TN) * GS_LD; };
 
   auto load_stage = [&](int s, int kt) {
-    float* As = stage_ptr(s);
-    float* Bs = As + TM * GS_LD;
+    float* Ah = stage_ptr(s);
+    float* Al = Ah + TM * GS_LD;
+    float* Bh = Al + TM * GS_LD;
+    float* Bl = Bh + TN * GS_LD;
     const int k0 = kb + kt * GS_BK;
     for (int idx = tid; idx < TM * (GS_BK / 4); idx += GS_THREADS) {
       const int r = idx / (GS_BK / 4), k4 = (idx % (GS_BK / 4)) * 4;
       const bool ok = (m0 + r) < p.M && (k0 + k4) < ke;
       const size_t o = ok ? static_cast<size_t>(m0 + r) * p.lda + k0 + k4 : 0;
-      gs_cp_async16(As + r * GS_LD + k4, p.A + o, ok);
+      gs_cp_async16(Ah + r * GS_LD + k4, p.A_hi + o, ok);
+      gs_cp_async16(Al + r * GS_LD + k4, p.A_lo + o, ok);
     }
     for (int idx = tid; idx < TN * (GS_BK / 4); idx += GS_THREADS) {
       const int r = idx / (GS_BK / 4), k4 = (idx % (GS_BK / 4)) * 4;
       const bool ok = (n0 + r) < p.N && (k0 + k4) < ke;
       const size_t o = ok ? static_cast<size_t>(n0 + r) * p.ldb + k0 + k4 : 0;
-      gs_cp_async16(Bs + r * GS_LD + k4, p.B + o, ok);
+      gs_cp_async16(Bh + r * GS_LD + k4, p.B_hi + o, ok);
+      gs_cp_async16(Bl + r * GS_LD + k4, p.B_lo + o, ok);
     }
   };
 
@@ -250,15 +256,25 @@ __global__ void __launch_bounds__(GS_THREADS) gemm_f32_simt_kernel(GemmSimtArgs 
     // refill the stage consumed one iteration ago
     if (kt + GS_STAGES - 1 < nk) load_stage((kt + GS_STAGES - 1) % GS_STAGES, kt + GS_STAGES - 1);
     asm volatile("cp.async.commit_group;" ::: "memory");
-    const float* As = stage_ptr(kt % GS_STAGES);
-    const float* Bs = As + TM * GS_LD;
+    const float* Ah = stage_ptr(kt % GS_STAGES);
+    const float* Al = Ah + TM * GS_LD;
+    const float* Bh = Al + TM * GS_LD;
+    const float* Bl = Bh + TN * GS_LD;
 #pragma unroll
     for (int k4 = 0; k4 < GS_BK; k4 += 4) {
       float4 a[RI], b[RJ];
 #pragma unroll
-      for (int i = 0; i < RI; ++i) a[i] = *reinterpret_cast<const float4*>(As + (ty + 16 * i) * GS_LD + k4);
+      for (int i = 0; i < RI; ++i) {
+        const float4 h = *reinterpret_cast<const float4*>(Ah + (ty + 16 * i) * GS_LD + k4);
+        const float4 l = *reinterpret_cast<const float4*>(Al + (ty + 16 * i) * GS_LD + k4);
+        a[i] = make_float4(h.x + l.x, h.y + l.y, h.z + l.z, h.w + l.w);
+      }
 #pragma unroll
-      for (int j = 0; j < RJ; ++j) b[j] = *reinterpret_cast<const float4*>(Bs + (tx + 16 * j) * GS_LD + k4);
+      for (int j = 0; j < RJ; ++j) {
+        const float4 h = *reinterpret_cast<const float4*>(Bh + (tx + 16 * j) * GS_LD + k4);
+        const float4 l = *reinterpret_cast<const float4*>(Bl + (tx + 16 * j) * GS_LD + k4);
+        b[j] = make_float4(h.x + l.x, h.y + l.y, h.z + l.z, h.w + l.w);
+      }
 #pragma unroll
       for (int i = 0; i < RI; ++i)
 #pragma unroll
@@ -280,26 +296,23 @@ __global__ void __launch_bounds__(GS_THREADS) gemm_f32_simt_kernel(GemmSimtArgs 
     for (int j = 0; j < RJ; ++j) {
       const int c = n0 + tx + 16 * j;
       if (c >= p.N) continue;
-      float v = p.alpha * acc[i][j];
+      const float v = p.alpha * acc[i][j];
       if (p.C) {
         float* cp = p.C + static_cast<size_t>(r) * p.ldc + c;
-        if (p.beta) v += *cp;
-        *cp = v;
+        *cp = p.beta ? v + *cp : v;
       }
       if (p.Chi) {
         const size_t o = static_cast<size_t>(r) * p.ldh + c;
-        const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+        const float x = p.beta ? v + (p.Chi[o] + p.Clo[o]) : v;
+        const float hi = tf32_rn_simt(x);
         p.Chi[o] = hi;
-        p.Clo[o] = __float2bfloat16_rn(v - __bfloat162float(hi));
+        p.Clo[o] = tf32_rn_simt(x - hi);
       }
-      if (p.Ct || p.Cthi) {
+      if (p.Cthi) {
         const size_t o = static_cast<size_t>(c) * p.ldt + r;
-        if (p.Ct) p.Ct[o] = v;
-        if (p.Cthi) {
-          const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-          p.Cthi[o] = hi;
-          p.Ctlo[o] = __float2bfloat16_rn(v - __bfloat162float(hi));
-        }
+        const float hi = tf32_rn_simt(v);
+        p.Cthi[o] = hi;
+        p.Ctlo[o] = tf32_rn_simt(v - hi);
       }
     }
   }

@@ -15,7 +15,7 @@
 //     the walker is on chunk k+1 (a rank-16 update in shared memory).
 // Named barriers hand each chunk's errors to the updaters and each finished update back to
 // the walker.  Group scales/zeros come from a min/max over the group's current values.  The
-// U block (128 x 128, fp32) is staged in shared memory before the kernel waits on its
+// U block (128 x 128, hi + lo) is staged in shared memory before the kernel waits on its
 // predecessor, so the staging overlaps the previous kernel's tail.  At the end the CTA writes
 // the block's errors to Err, the packed code words and the dequantized weights row by row.
 // The columns after the block receive the errors through tensor-core products (S6) launched
@@ -53,10 +53,10 @@ __device__ __forceinline__ void cp_async_wait_all() {
 
 struct SweepArgs {
   float* Wq;          // [m x n] fp32 working weights, sweep order
-  const float* U;     // [n x n] upper factor, fp32
-  float* Err;         // scaled errors as fp32 (or nullptr): block columns at Err[r * ld_err + err_col0 ..]
-  __nv_bfloat16* Err_hi;  // or as a bf16 hi/lo pair (same layout), the trailing product's operand
-  __nv_bfloat16* Err_lo;
+  const float* U;     // [n x n] upper factor (fp32, or the tf32 hi part when U_lo is set)
+  const float* U_lo;  // [n x n] tf32 lo part of U, or nullptr
+  float* Err;         // scaled errors (fp32, or hi part): block columns at Err[r * ld_err + err_col0 ..]
+  float* Err_lo;      // tf32 lo part of the errors (same layout), or nullptr
   int ld_err, err_col0;
   uint32_t* codes;    // [m x n*bits/32]
   float* scales;      // [m x G]
@@ -172,6 +172,20 @@ __global__ void __launch_bounds__(SW_THREADS)
   if (tid < SW_B) perm_s[tid] = a.perm[i1 + tid];
   cp_async_wait_all();
   __syncthreads();
+  if (a.U_lo) {
+    for (int idx = tid; idx < SW_B * (SW_B / 4); idx += SW_THREADS) {
+      const int k = idx / (SW_B / 4), j = (idx % (SW_B / 4)) * 4;
+      const float4 l = *reinterpret_cast<const float4*>(a.U_lo + static_cast<size_t>(i1 + k) * n + i1 + j);
+      float4* h = reinterpret_cast<float4*>(Us + k * SW_B + j);
+      float4 v = *h;
+      v.x += l.x;
+      v.y += l.y;
+      v.z += l.z;
+      v.w += l.w;
+      *h = v;
+    }
+    __syncthreads();
+  }
   if (tid < SW_B) rU[tid] = 1.0f / Us[tid * SW_B + tid];
 
   // ---- the W tile (written by the previous kernel) ----
@@ -367,16 +381,16 @@ __global__ void __launch_bounds__(SW_THREADS)
   }
 
   __syncthreads();
-  // errors of the block's rows (a bf16 pair for the tensor-core update, or fp32), row by row
+  // errors of the block's rows (hi/lo for the tensor-core update, or fp32), row by row
   for (int idx = tid; idx < SW_ROWS * SW_B; idx += SW_THREADS) {
     const int rl = idx / SW_B, j = idx % SW_B;
     if (row0 + rl >= a.m) continue;
     const float e = Es[rl * SW_ELD + j];
     const size_t eo = static_cast<size_t>(row0 + rl) * a.ld_err + a.err_col0 + j;
-    if (a.Err_hi) {
-      const __nv_bfloat16 hi = __float2bfloat16_rn(e);
-      a.Err_hi[eo] = hi;
-      a.Err_lo[eo] = __float2bfloat16_rn(e - __bfloat162float(hi));
+    if (a.Err_lo) {
+      const float hi = tf32_round(e);
+      a.Err[eo] = hi;
+      a.Err_lo[eo] = tf32_round(e - hi);
     } else {
       a.Err[eo] = e;
     }

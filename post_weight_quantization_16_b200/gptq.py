@@ -81,9 +81,9 @@ _SIGS = {
                                          ctypes.c_int, _P]),
     "gptq_quantize_layer_noalloc": (ctypes.c_int, [_P, ctypes.c_int64, ctypes.c_int64, _P, _P, _P, QParams,
                                                    _P, _P, _P, _P, _P, ctypes.c_int, _P]),
-    "gptq_test_gemm_bf16x3": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P, ctypes.c_int, _P, _P,
+    "gptq_test_gemm_tf32x3": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P, ctypes.c_int, _P, _P,
                                              ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                                             ctypes.c_int, _P, ctypes.c_int, _P, _P, ctypes.c_int, _P, _P, _P,
+                                             ctypes.c_int, _P, ctypes.c_int, _P, _P, ctypes.c_int, _P, _P,
                                              ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                              _P]),
     "gptq_test_div_rn": (ctypes.c_int, [ctypes.c_uint64, ctypes.c_int64, ctypes.POINTER(ctypes.c_uint64),

@@ -11,22 +11,16 @@ pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda", 0)
 
 
-def bf16_rn(x):
-    """bf16 bit patterns of fp32 values, round to nearest even."""
+def tf32_rn(x):
     u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
-    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
-    return u.astype(np.uint16)
-
-
-def bf16_f32(b):
-    return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+    u = (u + 0xFFF + ((u >> 13) & 1)) & 0xFFFFE000
+    return u.astype(np.uint32).view(np.float32)
 
 
 def split(x):
-    """The bf16 pair of x: hi = rn(x), lo = rn(x - hi)."""
     x = np.asarray(x, dtype=np.float32)
-    hi = bf16_rn(x)
-    lo = bf16_rn(x - bf16_f32(hi))
+    hi = tf32_rn(x)
+    lo = tf32_rn(x - hi)
     return hi, lo
 
 
@@ -34,25 +28,8 @@ def dev(a):
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(DEV)
 
 
-def dev16(b):
-    return torch.from_numpy(np.ascontiguousarray(b, dtype=np.uint16).view(np.int16)).to(DEV)
-
-
-def pair_value(h, l):
-    return bf16_f32(h.cpu().numpy().view(np.uint16)).astype(np.float64) + \
-        bf16_f32(l.cpu().numpy().view(np.uint16)).astype(np.float64)
-
-
 def p(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
-
-
-# Tolerances of the three-product bf16 GEMM, relative to sum_k |a_k b_k| (+ |C|): each operand
-# is its bf16 pair to 2^-17 and the dropped lo x lo product is below 2^-18 of |a b|, so an fp32
-# result is within about 3 * 2^-17 (TOL_F32); a result returned as a bf16 pair adds the
-# pair's own 2^-17 of |C| (TOL_PAIR).
-TOL_F32 = 3e-5
-TOL_PAIR = 4e-5
 
 
 def run_gemm(A, B, alpha=1.0, beta=0, C0=None, klo=0, khi=0, upper=0, plain=True, hilo=False, trans=False, chunk=1,
@@ -61,25 +38,27 @@ def run_gemm(A, B, alpha=1.0, beta=0, C0=None, klo=0, khi=0, upper=0, plain=True
     N = B.shape[0]
     ah, al = split(A)
     bh, bl = split(B)
-    Ah, Al, Bh, Bl = dev16(ah), dev16(al), dev16(bh), dev16(bl)
-    C = dev(C0 if C0 is not None else np.zeros((M, N))) if (plain or beta) else None
-    Ch = torch.zeros((M, N), dtype=torch.int16, device=DEV) if hilo else None
-    Cl = torch.zeros((M, N), dtype=torch.int16, device=DEV) if hilo else None
-    Ct = torch.zeros((N, M), dtype=torch.float32, device=DEV) if trans else None
-    Cth = torch.zeros((N, M), dtype=torch.int16, device=DEV) if trans else None
-    Ctl = torch.zeros((N, M), dtype=torch.int16, device=DEV) if trans else None
-    st = G.lib().gptq_test_gemm_bf16x3(M, N, K, p(Ah), p(Al), K, p(Bh), p(Bl), K, float(alpha), int(beta), klo, khi,
-                                       upper, p(C), N, p(Ch), p(Cl), N, p(Ct), p(Cth), p(Ctl), M, chunk, tile, reduce,
-                                       0, ctypes.c_void_p(torch.cuda.current_stream(DEV).cuda_stream))
+    Ah, Al, Bh, Bl = dev(ah), dev(al), dev(bh), dev(bl)
+    C = dev(C0 if C0 is not None else np.zeros((M, N))) if plain else None
+    if hilo:
+        c0 = C0 if C0 is not None else np.zeros((M, N))
+        h0, l0 = split(c0)
+        Ch, Cl = dev(h0), dev(l0)
+    else:
+        Ch = Cl = None
+    Cth = torch.zeros((N, M), dtype=torch.float32, device=DEV) if trans else None
+    Ctl = torch.zeros((N, M), dtype=torch.float32, device=DEV) if trans else None
+    st = G.lib().gptq_test_gemm_tf32x3(M, N, K, p(Ah), p(Al), K, p(Bh), p(Bl), K, float(alpha), int(beta), klo, khi,
+                                       upper, p(C), N, p(Ch), p(Cl), N, p(Cth), p(Ctl), M, chunk, tile, reduce, 0,
+                                       ctypes.c_void_p(torch.cuda.current_stream(DEV).cuda_stream))
     assert st == G.OK, G.STATUS.get(st)
     out = {}
-    if plain or beta:
+    if plain:
         out["C"] = C.cpu().numpy().astype(np.float64)
     if hilo:
-        out["Chilo"] = pair_value(Ch, Cl)
+        out["Chilo"] = Ch.cpu().numpy().astype(np.float64) + Cl.cpu().numpy().astype(np.float64)
     if trans:
-        out["Ct"] = Ct.cpu().numpy().astype(np.float64)
-        out["Cthilo"] = pair_value(Cth, Ctl)
+        out["Ct"] = Cth.cpu().numpy().astype(np.float64) + Ctl.cpu().numpy().astype(np.float64)
     return out
 
 
@@ -91,8 +70,8 @@ def ref(A, B, alpha, beta, C0):
     return R, scale
 
 
-@pytest.mark.parametrize("M,N,K,chunk", [(128, 256, 64, 1), (200, 320, 192, 1), (64, 64, 128, 2), (384, 512, 2048, 1),
-                                         (4096, 768, 128, 2), (300, 1024, 256, 2)])
+@pytest.mark.parametrize("M,N,K,chunk", [(128, 256, 32, 1), (200, 320, 96, 1), (64, 64, 128, 4), (384, 512, 2048, 1),
+                                         (4096, 768, 128, 4), (300, 1024, 256, 2)])
 @pytest.mark.parametrize("beta", [0, 1])
 @pytest.mark.parametrize("tile", [0, 64, 128, 256])
 def test_gemm_outputs_match_fp64(M, N, K, chunk, beta, tile):
@@ -104,9 +83,9 @@ def test_gemm_outputs_match_fp64(M, N, K, chunk, beta, tile):
                    tile=tile)
     R, scale = ref(A, B, -0.75, beta, C0)
     for k in out:
-        got = out[k].T if k.startswith("Ct") else out[k]
+        got = out[k].T if k == "Ct" else out[k]
         err = np.abs(got - R) / scale
-        assert err.max() <= (TOL_PAIR if "hilo" in k else TOL_F32), (k, err.max())
+        assert err.max() <= 2e-6, (k, err.max())
 
 
 @pytest.mark.parametrize("tile", [64, 128, 256])
@@ -118,18 +97,18 @@ def test_gemm_triangular_k_ranges(tile):
     B = np.triu(r.standard_normal((n, n)).astype(np.float32))
     R, scale = ref(A, B, 1.0, 0, None)
     got = run_gemm(A, B, klo=1, tile=tile)["C"]
-    assert (np.abs(got - R) / scale).max() <= TOL_F32
+    assert (np.abs(got - R) / scale).max() <= 2e-6
     # B upper in K-major form (B[c][k] = 0 for k > c): K up to the tile's last column
     B2 = np.tril(r.standard_normal((n, n)).astype(np.float32))
     R, scale = ref(A, B2, 1.0, 0, None)
     got = run_gemm(A, B2, khi=1, tile=tile)["C"]
-    assert (np.abs(got - R) / scale).max() <= TOL_F32
+    assert (np.abs(got - R) / scale).max() <= 2e-6
     # A upper (A[r][k] = 0 for k < r): K from the tile's first row
     A3 = np.triu(r.standard_normal((n, n)).astype(np.float32))
     B3 = r.standard_normal((384, n)).astype(np.float32)
     R, scale = ref(A3, B3, 1.0, 0, None)
     got = run_gemm(A3, B3, klo=2, tile=tile)["C"]
-    assert (np.abs(got - R) / scale).max() <= TOL_F32
+    assert (np.abs(got - R) / scale).max() <= 2e-6
 
 
 @pytest.mark.parametrize("tile", [64, 128, 256])
@@ -138,14 +117,14 @@ def test_gemm_upper_only_updates_upper_triangle(tile):
     n, K = 640, 128
     V = r.standard_normal((n, K)).astype(np.float32)
     C0 = r.standard_normal((n, n)).astype(np.float32)
-    out = run_gemm(V, V, alpha=-1.0, beta=1, C0=C0, upper=1, plain=True, hilo=True, tile=tile)
+    out = run_gemm(V, V, alpha=-1.0, beta=1, C0=C0, upper=1, plain=False, hilo=True, tile=tile)
     R, scale = ref(V, V, -1.0, 1, C0)
     iu = np.triu_indices(n)
-    assert (np.abs(out["C"][iu] - R[iu]) / scale[iu]).max() <= TOL_F32
-    assert (np.abs(out["Chilo"][iu] - R[iu]) / scale[iu]).max() <= TOL_PAIR
+    err = np.abs(out["Chilo"][iu] - R[iu]) / scale[iu]
+    assert err.max() <= 2e-6
 
 
-@pytest.mark.parametrize("M,N,K,chunk", [(4096, 896, 128, 2), (300, 320, 1024, 2), (128, 64, 64, 1), (1000, 3072, 256, 2)])
+@pytest.mark.parametrize("M,N,K,chunk", [(4096, 896, 128, 4), (300, 320, 1024, 4), (128, 64, 32, 1), (1000, 3072, 256, 4)])
 @pytest.mark.parametrize("tile", [64, 128, 256])
 def test_gemm_reduce_add_epilogue(M, N, K, chunk, tile):
     """C += alpha A B^T through TMA reduce-add boxes: equals the fp64 result, and C's columns
@@ -157,15 +136,15 @@ def test_gemm_reduce_add_epilogue(M, N, K, chunk, tile):
     C0 = r.standard_normal((M, N + pad)).astype(np.float32)
     ah, al = split(A)
     bh, bl = split(B)
-    Ah, Al, Bh, Bl = dev16(ah), dev16(al), dev16(bh), dev16(bl)
+    Ah, Al, Bh, Bl = dev(ah), dev(al), dev(bh), dev(bl)
     C = dev(C0)
-    st = G.lib().gptq_test_gemm_bf16x3(M, N, K, p(Ah), p(Al), K, p(Bh), p(Bl), K, -1.0, 1, 0, 0, 0, p(C), N + pad,
-                                       None, None, 0, None, None, None, 0, chunk, tile, 1, 0,
+    st = G.lib().gptq_test_gemm_tf32x3(M, N, K, p(Ah), p(Al), K, p(Bh), p(Bl), K, -1.0, 1, 0, 0, 0, p(C), N + pad,
+                                       None, None, 0, None, None, 0, chunk, tile, 1, 0,
                                        ctypes.c_void_p(torch.cuda.current_stream(DEV).cuda_stream))
     assert st == G.OK, G.STATUS.get(st)
     got = C.cpu().numpy().astype(np.float64)
     R, scale = ref(A, B, -1.0, 1, C0[:, :N])
-    assert (np.abs(got[:, :N] - R) / scale).max() <= TOL_F32
+    assert (np.abs(got[:, :N] - R) / scale).max() <= 2e-6
     assert np.array_equal(got[:, N:], C0[:, N:].astype(np.float64))
 
 
