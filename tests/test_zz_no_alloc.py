@@ -98,7 +98,12 @@ def test_noalloc_matches_oracle_and_context_path_on_two_calls(bits, g, sym, want
         assert same >= GH.CODES_IDENTICAL, (call, same)
         assert torch.equal(out["zeros"], ref["zeros"]), call
         if want_what:
-            what = out["w_hat"].cpu().numpy()
-            assert np.allclose(what, ref["w_hat"].cpu().numpy(), rtol=1e-6, atol=1e-9), call
+            # where both paths chose the same code the dequantized weights agree to the scales'
+            # tolerance; an in-band code flip (allowed above) moves one weight by a whole step
+            what = out["w_hat"].cpu().numpy().astype(np.float64)
+            same_orig = np.empty_like(gpu["codes"], dtype=bool)
+            same_orig[:, prep["perm"]] = gpu["codes"] == ref_codes
+            ref_what = ref["w_hat"].cpu().numpy().astype(np.float64)
+            assert np.allclose(what[same_orig], ref_what[same_orig], rtol=GH.SZ_REL, atol=1e-12), call
             if with_dead:
                 assert not what[:, [3, 500, 1000]].any()
