@@ -141,20 +141,23 @@ __device__ __forceinline__ void lf_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-// Rows [R0, R0 + 32) of U = X (zeros left of the diagonal) as a hi/lo pair, 16-byte stores,
-// by threads t = 0 .. nt-1.  (U^T is formed off the critical path.)
+// Rows [R0, R0 + 32) of U = X (zeros left of the diagonal) as a hi/lo pair and as plain fp32,
+// 16-byte stores, by threads t = 0 .. nt-1.  (U^T is formed off the critical path.)
 __device__ __forceinline__ void leaf_store_rows(const float (*X)[LF_LD], float* __restrict__ U_hi,
-                                                float* __restrict__ U_lo, int n, int o, int R0, int t, int nt) {
+                                                float* __restrict__ U_lo, float* __restrict__ U32, int n, int o,
+                                                int R0, int t, int nt) {
   for (int idx = t; idx < LF_P * (LF_NB / 4); idx += nt) {
     const int i = R0 + idx / (LF_NB / 4), j = (idx % (LF_NB / 4)) * 4;
-    float uh[4], ul[4];
+    float uh[4], ul[4], u4[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const float u = (i <= j + e) ? X[i][j + e] : 0.0f;  // U[i][j+e]
+      u4[e] = u;
       uh[e] = tf32_round(u);
       ul[e] = tf32_round(u - uh[e]);
     }
     const size_t g = static_cast<size_t>(o + i) * n + o + j;
+    *reinterpret_cast<float4*>(U32 + g) = make_float4(u4[0], u4[1], u4[2], u4[3]);
     *reinterpret_cast<float4*>(U_hi + g) = make_float4(uh[0], uh[1], uh[2], uh[3]);
     *reinterpret_cast<float4*>(U_lo + g) = make_float4(ul[0], ul[1], ul[2], ul[3]);
   }
@@ -174,7 +177,8 @@ __device__ __forceinline__ void leaf_store_rows(const float (*X)[LF_LD], float* 
 //   U_pj = -Xd_p * sum_{l=p+1..j} V_pl U_lj      (Xd_p = the diagonal block's inverse).
 __global__ void __launch_bounds__(LF_THREADS, 1)
     leaf_chol_inv_kernel(const float* __restrict__ A_hi, const float* __restrict__ A_lo, int n, int o,
-                         float* __restrict__ U_hi, float* __restrict__ U_lo, int* __restrict__ status) {
+                         float* __restrict__ U_hi, float* __restrict__ U_lo, float* __restrict__ U32,
+                         int* __restrict__ status) {
   extern __shared__ float lf_smem[];
   float(*S)[LF_LD] = reinterpret_cast<float(*)[LF_LD]>(lf_smem);
   float(*V)[LF_LD] = reinterpret_cast<float(*)[LF_LD]>(lf_smem + LF_NB * LF_LD);
@@ -242,7 +246,7 @@ __global__ void __launch_bounds__(LF_THREADS, 1)
       __syncthreads();  // column block p-1 is up to date: warp 0 may factor it
     }
     // block row p+1 of U is final (since the last step): warp 4, otherwise idle here, writes it
-    if (warp == 4 && p + 1 < LF_NB / LF_P) leaf_store_rows(X, U_hi, U_lo, n, o, (p + 1) * LF_P, lane, 32);
+    if (warp == 4 && p + 1 < LF_NB / LF_P) leaf_store_rows(X, U_hi, U_lo, U32, n, o, (p + 1) * LF_P, lane, 32);
     if (g1) {
       {
         // the rest of the trailing update: S[i][j] -= sum_c V[i][P0+c] V[j][P0+c], i <= j < P0-32
@@ -327,7 +331,7 @@ __global__ void __launch_bounds__(LF_THREADS, 1)
   __syncthreads();
 
   // block row 0 of U (the others went out during the factorization)
-  leaf_store_rows(X, U_hi, U_lo, n, o, 0, tid, LF_THREADS);
+  leaf_store_rows(X, U_hi, U_lo, U32, n, o, 0, tid, LF_THREADS);
   if (tid == 0 && *bad) atomicOr(status, ST_NOT_PD);
 }
 

@@ -23,6 +23,7 @@
 #include "hessian_tc.cuh"
 #include "prepare_kernels.cuh"
 #include "sgemm_simt.cuh"
+#include "slab_sweep.cuh"
 #include "sweep_kernels.cuh"
 
 using namespace gptq;
@@ -45,6 +46,7 @@ struct gptq_ctx {
   float *A_hi = nullptr, *A_lo = nullptr;      // [n x n] damped, permuted H; Schur complements
   float *VT_hi = nullptr, *VT_lo = nullptr;    // [n x n] V12 blocks (upper) and T^T blocks (lower)
   float *U_hi = nullptr, *U_lo = nullptr;      // [n x n] U (upper)
+  float* U32 = nullptr;                        // [n x n] U as plain fp32 (upper; read by the sweep)
   float *Ut_hi = nullptr, *Ut_lo = nullptr;    // [n x n] U^T
   float* Wq = nullptr;                         // [m_max x n] fp32 working weights
   float *Err_hi = nullptr, *Err_lo = nullptr;  // [m_max x kSuperBlock] block errors of a super-block
@@ -420,7 +422,7 @@ gptq_status chol_inv(gptq_ctx* c, int o, int h) {
   if (h <= LF_NB) {
     tag(c, "leaf_chol_inv", 2.0 * LF_NB * LF_NB * LF_NB / 3.0, 4.0 * LF_NB * LF_NB * 4);
     CK(launch(c, leaf_chol_inv_kernel, dim3(1), dim3(LF_THREADS), LF_SMEM, c->A_hi, c->A_lo, n, o, c->U_hi, c->U_lo,
-              c->status));
+              c->U32, c->status));
     CKL("leaf_chol_inv");
     // U^T of the block, needed only by later T products and the sweep's trailing update: on
     // the second branch while it exists (the factorization graph), in line otherwise
@@ -500,6 +502,8 @@ gptq_status chol_inv(gptq_ctx* c, int o, int h) {
   if (branch) CK(cudaStreamWaitEvent(main_stream, c->ev_join, 0));
   // U12 = -U11 T  (and Ut21 = U12^T)      (U11 rows as A; k >= row)
   TcOut u12;
+  u12.C = at(c->U32, o, o2);
+  u12.ldc = n;
   u12.Chi = at(c->U_hi, o, o2);
   u12.Clo = at(c->U_lo, o, o2);
   u12.ldh = n;
@@ -618,8 +622,8 @@ void free_all(gptq_ctx* c) {
   c->ev_fork = c->ev_join = nullptr;
   c->factor_graph = nullptr;
   c->capture_stream = nullptr;
-  float** fs[] = {&c->H,     &c->A_hi,  &c->A_lo,  &c->VT_hi, &c->VT_lo,  &c->U_hi,   &c->U_lo,
-                  &c->Ut_hi, &c->Ut_lo, &c->Wq,    &c->Err_hi, &c->Err_lo, &c->keys};
+  float** fs[] = {&c->H,     &c->A_hi,  &c->A_lo, &c->VT_hi,  &c->VT_lo,  &c->U_hi, &c->U_lo,
+                  &c->U32,   &c->Ut_hi, &c->Ut_lo, &c->Wq,     &c->Err_hi, &c->Err_lo, &c->keys};
   for (float** p : fs)
     if (*p) {
       cudaFree(*p);
@@ -667,7 +671,7 @@ const char* gptq_status_string(gptq_status s) {
 size_t gptq_workspace_bytes(int64_t n, int64_t m_max) {
   if (n < 128 || n > kMaxN || n % 128 || m_max < 1 || m_max > kMaxM) return 0;
   const size_t nn = static_cast<size_t>(n) * static_cast<size_t>(n);
-  size_t b = 9 * nn * sizeof(float);                                              // H, A, VT, U, Ut (hi/lo)
+  size_t b = 10 * nn * sizeof(float);                                             // H, A, VT, U, Ut (hi/lo), U
   b += static_cast<size_t>(m_max) * static_cast<size_t>(n) * sizeof(float);       // Wq
   b += 2 * static_cast<size_t>(m_max) * kSuperBlock * sizeof(float);              // Err hi/lo
   b += static_cast<size_t>(n) * (sizeof(float) + 1 + sizeof(int32_t)) + sizeof(double) + sizeof(int);
@@ -709,7 +713,7 @@ gptq_status gptq_create(gptq_ctx** out, int64_t n, int64_t m_max, int device, vo
     if (e == cudaSuccess) e = cudaMalloc(p, bytes);
   };
   alloc(reinterpret_cast<void**>(&c->H), nn * 4);
-  for (float** p : {&c->A_hi, &c->A_lo, &c->VT_hi, &c->VT_lo, &c->U_hi, &c->U_lo, &c->Ut_hi, &c->Ut_lo})
+  for (float** p : {&c->A_hi, &c->A_lo, &c->VT_hi, &c->VT_lo, &c->U_hi, &c->U_lo, &c->U32, &c->Ut_hi, &c->Ut_lo})
     alloc(reinterpret_cast<void**>(p), nn * 4);
   alloc(reinterpret_cast<void**>(&c->Wq), static_cast<size_t>(m_max) * n * 4);
   alloc(reinterpret_cast<void**>(&c->Err_hi), static_cast<size_t>(m_max) * kSuperBlock * 4);
@@ -741,6 +745,12 @@ gptq_status gptq_create(gptq_ctx** out, int64_t n, int64_t m_max, int device, vo
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(gemm_hilo_simt_kernel<32, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              gs_smem_bytes<32, 32>());
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(sweep_slab_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, SS_SMEM);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(sweep_slab_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, SS_SMEM);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(sweep_slab_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, SS_SMEM);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(sweep_block_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, SW_SMEM);
   if (e == cudaSuccess)
@@ -852,7 +862,7 @@ gptq_status gptq_prepare(gptq_ctx* c, double damp, int desc_act, int32_t* perm_o
                                                                         c->A_hi, c->A_lo));
   CKL("gather");
   const size_t nn = static_cast<size_t>(n) * n;
-  for (float* p : {c->U_hi, c->U_lo, c->Ut_hi, c->Ut_lo}) CK(cudaMemsetAsync(p, 0, nn * 4, c->stream));
+  for (float* p : {c->U_hi, c->U_lo, c->U32, c->Ut_hi, c->Ut_lo}) CK(cudaMemsetAsync(p, 0, nn * 4, c->stream));
   if ((s = run_factorization(c)) != GPTQ_OK) return s;
   if (perm_out) CK(cudaMemcpyAsync(perm_out, c->perm, n * 4, cudaMemcpyDeviceToDevice, c->stream));
   int flags = 0;
@@ -867,9 +877,7 @@ gptq_status gptq_get_factor(gptq_ctx* c, float* U_out) {
   if (c->state != ST_PREPARED) return GPTQ_ERR_STATE;
   DeviceGuard dg(c->device);
   const size_t nn = static_cast<size_t>(c->n) * c->n;
-  tag(c, "combine_hilo", 0.0, 12.0 * static_cast<double>(nn));
-  CK(launch(c, combine_hilo_kernel, dim3(592), dim3(256), 0, c->U_hi, c->U_lo, nn, U_out));
-  CKL("combine");
+  CK(cudaMemcpyAsync(U_out, c->U32, nn * 4, cudaMemcpyDeviceToDevice, c->stream));
   return GPTQ_OK;
 }
 
@@ -947,8 +955,8 @@ gptq_status gptq_quantize_layer(gptq_ctx* c, const void* W, int64_t m, gptq_qpar
   CKL("init_w");
   SweepArgs a;
   a.Wq = c->Wq;
-  a.U = c->U_hi;
-  a.U_lo = c->U_lo;
+  a.U = c->U32;
+  a.U_lo = nullptr;
   a.Err = c->Err_hi;
   a.Err_lo = c->Err_lo;
   a.codes = codes;
@@ -963,42 +971,28 @@ gptq_status gptq_quantize_layer(gptq_ctx* c, const void* W, int64_t m, gptq_qpar
   a.g = g;
   a.G = n / g;
   a.ld_err = kSuperBlock;
+  a.err_col0 = 0;
   const int grid = (mi + SW_ROWS - 1) / SW_ROWS;
-  // algorithmic bytes of one sweep block: W tile in, scaled errors out (hi/lo), codes,
-  // scales/zeros of the groups that start in it, the U block (hi/lo)
-  const double sweep_bytes = 4.0 * mi * SW_B + 8.0 * mi * SW_B + mi * SW_B * qp.bits / 8.0 +
-                             8.0 * mi * std::max(1, SW_B / g) + 8.0 * SW_B * SW_B + (W_hat ? 4.0 * mi * SW_B : 0.0);
-  // two-level lazy update: inside a super-block the columns after each 128-block are updated
-  // right away; the columns beyond the super-block receive all its block errors in one product
-  // (K = super-block width).  A group that starts inside a super-block must not reach past it.
+  // Two-level lazy update: inside a super-block of columns the slab kernel applies each block's
+  // errors to the later columns itself; the columns beyond the super-block receive all its
+  // block errors in one tensor-core product (K = super-block width).  A group that starts
+  // inside a super-block must not reach past it; other group widths use 128-column super-blocks.
   const int sb = ((g <= kSuperBlock && kSuperBlock % g == 0) || g % kSuperBlock == 0 || g == n) ? kSuperBlock : SW_B;
   for (int s0 = 0; s0 < n; s0 += sb) {
     const int s1 = std::min(n, s0 + sb);
-    for (int i1 = s0; i1 < s1; i1 += SW_B) {
-      a.err_col0 = i1 - s0;
-      tag(c, "sweep_block", 0.0, sweep_bytes);
-      if (g >= SW_B)
-        CK(launch(c, sweep_block_kernel<0>, dim3(grid), dim3(SW_THREADS), SW_SMEM, a, i1));
-      else if (g == 64)
-        CK(launch(c, sweep_block_kernel<64>, dim3(grid), dim3(SW_THREADS), SW_SMEM, a, i1));
-      else
-        CK(launch(c, sweep_block_kernel<32>, dim3(grid), dim3(SW_THREADS), SW_SMEM, a, i1));
-      CKL("sweep");
-      const int i2 = i1 + SW_B;
-      if (i2 < s1) {
-        // W[:, i2:s1] -= Err_blk * U[i1:i2, i2:s1]   (B in K-major form: rows of U^T)
-        TcOut w;
-        w.C = c->Wq + i2;
-        w.ldc = n;
-        w.c_map = &c->mC_Wq;
-        w.c_col0 = i2;
-        c->gemm_role = GR_NEAR;
-        gptq_status st = gemm_tc(c, mi, s1 - i2, SW_B, TcOperand{&c->mA_Err[0], &c->mA_Err[1], 0, i1 - s0, nullptr, nullptr, 0},
-                                 TcOperand{&c->mB_Ut[0], &c->mB_Ut[1], i2, i1, nullptr, nullptr, 0}, -1.f, 1,
-                                 GT_KLO_NONE, GT_KHI_NONE, 0, w, SW_B / GT_BK);
-        if (st != GPTQ_OK) return st;
-      }
-    }
+    const double S = static_cast<double>(s1 - s0);
+    // algorithmic bytes: the slab in, its scaled errors out (hi/lo), codes, scales/zeros of its
+    // groups, its U blocks, the dequantized weights when asked for
+    tag(c, "sweep_slab", 0.0,
+        4.0 * mi * S + 8.0 * mi * S + mi * S * qp.bits / 8.0 + 8.0 * mi * std::max(1.0, S / g) + 4.0 * SW_B * S +
+            (W_hat ? 4.0 * mi * S : 0.0));
+    if (g >= SW_B)
+      CK(launch(c, sweep_slab_kernel<0>, dim3(grid), dim3(SS_THREADS), SS_SMEM, a, s0, s1));
+    else if (g == 64)
+      CK(launch(c, sweep_slab_kernel<64>, dim3(grid), dim3(SS_THREADS), SS_SMEM, a, s0, s1));
+    else
+      CK(launch(c, sweep_slab_kernel<32>, dim3(grid), dim3(SS_THREADS), SS_SMEM, a, s0, s1));
+    CKL("sweep_slab");
     if (s1 < n) {
       // W[:, s1:] -= Err_super * U[s0:s1, s1:]   (K = s1 - s0; 128-wide TMEM chunks)
       TcOut w;
