@@ -471,22 +471,26 @@ def w4a16_measure(G, out, perm, layer, qs, dev, stream, peaks, peak_bf16, reps=8
         X = torch.randn((T, n), device=dev, dtype=torch.float32).to(torch.float16)
         Y = torch.empty((T, m), dtype=torch.float32, device=dev)
         ws = torch.empty(int(G.lib().gptq_dequant_matmul_workspace_bytes(T, m, n, 1)), dtype=torch.uint8, device=dev)
-        call = lambda: G.dequant_matmul(X, out["codes"], out["scales"], out["zeros"], perm, qs.bits, qs.group_size,
-                                        out=Y, workspace=ws, stream=stream)
-        call()  # first call: kernel attributes and tensor-map encoding outside the capture
+        cap = torch.cuda.Stream(dev)  # graphs are captured on a stream of their own
+        call = lambda st: G.dequant_matmul(X, out["codes"], out["scales"], out["zeros"], perm, qs.bits,
+                                           qs.group_size, out=Y, workspace=ws, stream=st)
+        call(stream)  # first call: kernel attributes and tensor-map encoding outside the capture
         torch.cuda.synchronize(dev)
         # the call as a CUDA graph, so that its host-side setup does not sit inside the timed window
         graph = torch.cuda.CUDAGraph()
-        with torch.cuda.stream(stream):
+        cap.wait_stream(stream)
+        with torch.cuda.stream(cap):
             graph.capture_begin(capture_error_mode="thread_local")
-            call()
+            call(cap)
             graph.capture_end()
+        torch.cuda.synchronize(dev)
         ms = []
         for r in range(reps + 2):
             flush.zero_()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            graph.replay()
+            with torch.cuda.stream(stream):
+                graph.replay()
             e1.record(stream)
             torch.cuda.synchronize(dev)
             if r >= 2:
