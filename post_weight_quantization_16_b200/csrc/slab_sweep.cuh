@@ -15,9 +15,10 @@
 //     as broadcasts): code, dequantized value, e = (w - q) / U[i][i], w[j] -= e U[i][j] for the
 //     chunk's later columns;
 //   * warps 1-7, the updaters, take each finished chunk's errors and apply them, first to the
-//     block's chunks two and more ahead (from the staged U block), then to every later column
-//     of the slab (U rows read through the L1 cache, the same address for all 32 lanes), in
-//     fp32 fused multiply-adds;
+//     block's chunks two and more ahead (from the staged U block, a lane per row), then to
+//     every later column of the slab (a lane per four columns, their 16 U values loaded once,
+//     coalesced across the warp, and used for all 32 rows; the errors read as shared-memory
+//     broadcasts), in fp32 fused multiply-adds;
 //   * the block's scaled errors go out as tf32 hi/lo pairs for the one product that updates
 //     the columns beyond the super-block, and its codes are packed.
 // So the per-block product on the later columns of the super-block, and its launch, leave the
@@ -34,9 +35,9 @@ constexpr int SS_THREADS = 256;            // walker warp + seven updater warps
 constexpr int SS_NW = SS_THREADS / 32;
 constexpr int SS_MAXW = 1024;              // slab width (columns)
 constexpr int SS_WLD = SS_MAXW + 4;        // slab pitch (floats): lane-per-row float4 access without conflicts
-// U block | slab | errors | 1/U[i][i] | perm | group partials | codes
-constexpr int SS_SMEM = SW_B * SW_B * 4 + SW_ROWS * SS_WLD * 4 + SW_ROWS * SW_ELD * 4 + SW_B * 4 + SW_B * 4 +
-                        3 * SS_NW * SW_ROWS * 4 + SW_ROWS * SW_CLD;
+// U block | slab | errors | the chunk's errors (compact) | 1/U[i][i] | perm | group partials | codes
+constexpr int SS_SMEM = SW_B * SW_B * 4 + SW_ROWS * SS_WLD * 4 + SW_ROWS * SW_ELD * 4 + 2 * SW_ROWS * SW_CH * 4 +
+                        SW_B * 4 + SW_B * 4 + 3 * SS_NW * SW_ROWS * 4 + SW_ROWS * SW_CLD;
 
 __device__ __forceinline__ void ss_arrive(int id) {
   asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(SS_THREADS) : "memory");
@@ -53,7 +54,8 @@ __global__ void __launch_bounds__(SS_THREADS, 1) sweep_slab_kernel(SweepArgs a, 
   float* Us = ss_smem;                                    // [128][128] U block
   float* Ws = Us + SW_B * SW_B;                           // [32][SS_WLD] slab
   float* Es = Ws + SW_ROWS * SS_WLD;                      // [32][129] scaled errors of the block
-  float* rU = Es + SW_ROWS * SW_ELD;                      // [128] 1 / U[i][i]
+  float* Ek = Es + SW_ROWS * SW_ELD;                      // [2][32][16] errors of the last two chunks
+  float* rU = Ek + 2 * SW_ROWS * SW_CH;                   // [128] 1 / U[i][i]
   int* perm_s = reinterpret_cast<int*>(rU + SW_B);        // [128]
   float* part = reinterpret_cast<float*>(perm_s + SW_B);  // [3][8][32] group min / max / max|.| partials
   uint8_t* codes8 = reinterpret_cast<uint8_t*>(part + 3 * SS_NW * SW_ROWS);  // [32][132] codes
@@ -252,6 +254,12 @@ __global__ void __launch_bounds__(SS_THREADS, 1) sweep_slab_kernel(SweepArgs a, 
           Es[rl * SW_ELD + i] = ep[t];
           codes8[rl * SW_CLD + i] = static_cast<uint8_t>(static_cast<int>(qc[t] - qp.lo));
         }
+        if (slab_rest) {  // the chunk's errors again, 16-byte aligned per row, for the slab pass
+          float4* ek = reinterpret_cast<float4*>(Ek + ((k & 1) * SW_ROWS + rl) * SW_CH);
+#pragma unroll
+          for (int j4 = 0; j4 < SW_CH / 4; ++j4)
+            ek[j4] = make_float4(ep[4 * j4], ep[4 * j4 + 1], ep[4 * j4 + 2], ep[4 * j4 + 3]);
+        }
         if (k + 2 < SW_NCH || slab_rest) ss_arrive(1 + (k & 1));  // chunk k's errors are in Es
         if (want_what && valid) {  // dequantized weights, straight to the original column order
 #pragma unroll
@@ -288,27 +296,38 @@ __global__ void __launch_bounds__(SS_THREADS, 1) sweep_slab_kernel(SweepArgs a, 
             *reinterpret_cast<float4*>(Ws + rl * SS_WLD + bo + j) = acc;
           }
         }
-        // (2) the slab's later columns, U rows i1 + 16 k .. + 15 read through L1 (one address
-        // per warp-wide load: the lanes are rows)
+        // (2) the slab's later columns: a lane takes four columns, holds their 16 U values
+        // (rows i1 + 16 k .. + 15, coalesced loads across the warp) in registers and walks the
+        // 32 rows, the chunk's errors read as shared-memory broadcasts
         if (slab_rest) {
           const int cb = bo + SW_B;
           const int nq = (S - cb) / 4;
-          float e[SW_CH];
-#pragma unroll
-          for (int t = 0; t < SW_CH; ++t) e[t] = Es[lane * SW_ELD + k * SW_CH + t];
           const float* ub = a.U + static_cast<size_t>(i1 + k * SW_CH) * n + s0 + cb;
-          for (int q = uw; q < nq; q += SS_NW - 1) {
-            float* wp = Ws + lane * SS_WLD + cb + 4 * q;
-            float4 acc = *reinterpret_cast<const float4*>(wp);
+          const float4* ek = reinterpret_cast<const float4*>(Ek + (k & 1) * SW_ROWS * SW_CH);
+          for (int q = uw * 32 + lane; q < nq; q += (SS_NW - 1) * 32) {
+            float4 u[SW_CH];
 #pragma unroll
-            for (int t = 0; t < SW_CH; ++t) {
-              const float4 u = __ldg(reinterpret_cast<const float4*>(ub + static_cast<size_t>(t) * n + 4 * q));
-              acc.x = fmaf(-e[t], u.x, acc.x);
-              acc.y = fmaf(-e[t], u.y, acc.y);
-              acc.z = fmaf(-e[t], u.z, acc.z);
-              acc.w = fmaf(-e[t], u.w, acc.w);
+            for (int t = 0; t < SW_CH; ++t)
+              u[t] = __ldg(reinterpret_cast<const float4*>(ub + static_cast<size_t>(t) * n + 4 * q));
+#pragma unroll 2
+            for (int r = 0; r < SW_ROWS; ++r) {
+              float* wp = Ws + r * SS_WLD + cb + 4 * q;
+              float4 acc = *reinterpret_cast<const float4*>(wp);
+#pragma unroll
+              for (int t4 = 0; t4 < SW_CH / 4; ++t4) {
+                const float4 e = ek[r * (SW_CH / 4) + t4];
+                const float ev[4] = {e.x, e.y, e.z, e.w};
+#pragma unroll
+                for (int tt = 0; tt < 4; ++tt) {
+                  const float4 uu = u[4 * t4 + tt];
+                  acc.x = fmaf(-ev[tt], uu.x, acc.x);
+                  acc.y = fmaf(-ev[tt], uu.y, acc.y);
+                  acc.z = fmaf(-ev[tt], uu.z, acc.z);
+                  acc.w = fmaf(-ev[tt], uu.w, acc.w);
+                }
+              }
+              *reinterpret_cast<float4*>(wp) = acc;
             }
-            *reinterpret_cast<float4*>(wp) = acc;
           }
         }
         ss_arrive(3 + (k & 1));
