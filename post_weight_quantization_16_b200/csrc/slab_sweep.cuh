@@ -304,13 +304,17 @@ __global__ void __launch_bounds__(SS_THREADS, 1) sweep_slab_kernel(SweepArgs a, 
           const int nq = (S - cb) / 4;
           const float* ub = a.U + static_cast<size_t>(i1 + k * SW_CH) * n + s0 + cb;
           const float4* ek = reinterpret_cast<const float4*>(Ek + (k & 1) * SW_ROWS * SW_CH);
-          for (int q = uw * 32 + lane; q < nq; q += (SS_NW - 1) * 32) {
+          // items (row chunk of 8 rows, column quad), quads fastest: every updater lane has work
+          // however narrow the rest of the slab, and a quad's U values are reused from L1
+          constexpr int RCH = 8;
+          for (int item = uw * 32 + lane; item < (SW_ROWS / RCH) * nq; item += (SS_NW - 1) * 32) {
+            const int q = item % nq, r0 = (item / nq) * RCH;
             float4 u[SW_CH];
 #pragma unroll
             for (int t = 0; t < SW_CH; ++t)
               u[t] = __ldg(reinterpret_cast<const float4*>(ub + static_cast<size_t>(t) * n + 4 * q));
 #pragma unroll 2
-            for (int r = 0; r < SW_ROWS; ++r) {
+            for (int r = r0; r < r0 + RCH; ++r) {
               float* wp = Ws + r * SS_WLD + cb + 4 * q;
               float4 acc = *reinterpret_cast<const float4*>(wp);
 #pragma unroll
