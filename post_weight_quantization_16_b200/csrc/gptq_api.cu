@@ -33,7 +33,8 @@ namespace {
 enum CtxState { ST_ACCUM = 0, ST_PREPARED = 1 };
 
 constexpr int64_t kMaxN = 32768;
-constexpr int kSuperBlock = 1024;  // columns whose block errors are applied beyond them in one product
+constexpr int kSuperBlock = 1024;  // widest slab: the block-error buffer holds this many columns
+constexpr int kSlabDefault = 256;  // columns per slab (super-block) of the sweep
 constexpr int64_t kMaxM = int64_t(1) << 24;
 
 }  // namespace
@@ -977,7 +978,10 @@ gptq_status gptq_quantize_layer(gptq_ctx* c, const void* W, int64_t m, gptq_qpar
   // errors to the later columns itself; the columns beyond the super-block receive all its
   // block errors in one tensor-core product (K = super-block width).  A group that starts
   // inside a super-block must not reach past it; other group widths use 128-column super-blocks.
-  const int sb = ((g <= kSuperBlock && kSuperBlock % g == 0) || g % kSuperBlock == 0 || g == n) ? kSuperBlock : SW_B;
+  // slab width: kSlabDefault, or GPTQ_SLAB_WIDTH (a multiple of 128 up to kSuperBlock) for tuning
+  const int slab = static_cast<int>(
+      std::min<int64_t>(kSuperBlock, std::max<int64_t>(SW_B, env_int("GPTQ_SLAB_WIDTH", kSlabDefault) / SW_B * SW_B)));
+  const int sb = ((g <= slab && slab % g == 0) || g % slab == 0 || g == n) ? slab : SW_B;
   for (int s0 = 0; s0 < n; s0 += sb) {
     const int s1 = std::min(n, s0 + sb);
     const double S = static_cast<double>(s1 - s0);
@@ -986,12 +990,13 @@ gptq_status gptq_quantize_layer(gptq_ctx* c, const void* W, int64_t m, gptq_qpar
     tag(c, "sweep_slab", 0.0,
         4.0 * mi * S + 8.0 * mi * S + mi * S * qp.bits / 8.0 + 8.0 * mi * std::max(1.0, S / g) + 4.0 * SW_B * S +
             (W_hat ? 4.0 * mi * S : 0.0));
+    const size_t smem = static_cast<size_t>(ss_smem_bytes(s1 - s0));
     if (g >= SW_B)
-      CK(launch(c, sweep_slab_kernel<0>, dim3(grid), dim3(SS_THREADS), SS_SMEM, a, s0, s1));
+      CK(launch(c, sweep_slab_kernel<0>, dim3(grid), dim3(SS_THREADS), smem, a, s0, s1));
     else if (g == 64)
-      CK(launch(c, sweep_slab_kernel<64>, dim3(grid), dim3(SS_THREADS), SS_SMEM, a, s0, s1));
+      CK(launch(c, sweep_slab_kernel<64>, dim3(grid), dim3(SS_THREADS), smem, a, s0, s1));
     else
-      CK(launch(c, sweep_slab_kernel<32>, dim3(grid), dim3(SS_THREADS), SS_SMEM, a, s0, s1));
+      CK(launch(c, sweep_slab_kernel<32>, dim3(grid), dim3(SS_THREADS), smem, a, s0, s1));
     CKL("sweep_slab");
     if (s1 < n) {
       // W[:, s1:] -= Err_super * U[s0:s1, s1:]   (K = s1 - s0; 128-wide TMEM chunks)

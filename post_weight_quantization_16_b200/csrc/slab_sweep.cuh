@@ -33,11 +33,15 @@ namespace gptq {
 
 constexpr int SS_THREADS = 256;            // walker warp + seven updater warps
 constexpr int SS_NW = SS_THREADS / 32;
-constexpr int SS_MAXW = 1024;              // slab width (columns)
-constexpr int SS_WLD = SS_MAXW + 4;        // slab pitch (floats): lane-per-row float4 access without conflicts
+constexpr int SS_MAXW = 1024;              // widest slab (columns)
+// slab pitch (floats) for a slab of S columns: lane-per-row float4 access without conflicts
+__host__ __device__ constexpr int ss_wld(int S) { return S + 4; }
 // U block | slab | errors | the chunk's errors (compact) | 1/U[i][i] | perm | group partials | codes
-constexpr int SS_SMEM = SW_B * SW_B * 4 + SW_ROWS * SS_WLD * 4 + SW_ROWS * SW_ELD * 4 + 2 * SW_ROWS * SW_CH * 4 +
-                        SW_B * 4 + SW_B * 4 + 3 * SS_NW * SW_ROWS * 4 + SW_ROWS * SW_CLD;
+__host__ __device__ constexpr int ss_smem_bytes(int S) {
+  return SW_B * SW_B * 4 + SW_ROWS * ss_wld(S) * 4 + SW_ROWS * SW_ELD * 4 + 2 * SW_ROWS * SW_CH * 4 + SW_B * 4 +
+         SW_B * 4 + 3 * SS_NW * SW_ROWS * 4 + SW_ROWS * SW_CLD;
+}
+constexpr int SS_SMEM = ss_smem_bytes(SS_MAXW);
 
 __device__ __forceinline__ void ss_arrive(int id) {
   asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(SS_THREADS) : "memory");
@@ -51,20 +55,20 @@ __device__ __forceinline__ void ss_sync(int id) {
 template <int GSUB>
 __global__ void __launch_bounds__(SS_THREADS, 1) sweep_slab_kernel(SweepArgs a, int s0, int s1) {
   extern __shared__ __align__(16) float ss_smem[];
-  float* Us = ss_smem;                                    // [128][128] U block
-  float* Ws = Us + SW_B * SW_B;                           // [32][SS_WLD] slab
-  float* Es = Ws + SW_ROWS * SS_WLD;                      // [32][129] scaled errors of the block
-  float* Ek = Es + SW_ROWS * SW_ELD;                      // [2][32][16] errors of the last two chunks
-  float* rU = Ek + 2 * SW_ROWS * SW_CH;                   // [128] 1 / U[i][i]
-  int* perm_s = reinterpret_cast<int*>(rU + SW_B);        // [128]
-  float* part = reinterpret_cast<float*>(perm_s + SW_B);  // [3][8][32] group min / max / max|.| partials
-  uint8_t* codes8 = reinterpret_cast<uint8_t*>(part + 3 * SS_NW * SW_ROWS);  // [32][132] codes
-
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int n = a.n;
   const int row0 = blockIdx.x * SW_ROWS;
   const int S = s1 - s0;
+  const int WLD = ss_wld(S);
+  float* Us = ss_smem;                                    // [128][128] U block
+  float* Ws = Us + SW_B * SW_B;                           // [32][WLD] slab
+  float* Es = Ws + SW_ROWS * WLD;                         // [32][129] scaled errors of the block
+  float* Ek = Es + SW_ROWS * SW_ELD;                      // [2][32][16] errors of the last two chunks
+  float* rU = Ek + 2 * SW_ROWS * SW_CH;                   // [128] 1 / U[i][i]
+  int* perm_s = reinterpret_cast<int*>(rU + SW_B);        // [128]
+  float* part = reinterpret_cast<float*>(perm_s + SW_B);  // [3][8][32] group min / max / max|.| partials
+  uint8_t* codes8 = reinterpret_cast<uint8_t*>(part + 3 * SS_NW * SW_ROWS);  // [32][132] codes
 
   auto stage_block = [&](int i1) {
     for (int idx = tid; idx < SW_B * (SW_B / 4); idx += SS_THREADS) {
@@ -81,7 +85,7 @@ __global__ void __launch_bounds__(SS_THREADS, 1) sweep_slab_kernel(SweepArgs a, 
   griddep_wait();
   for (int idx = tid; idx < SW_ROWS * (S / 4); idx += SS_THREADS) {
     const int rl = idx / (S / 4), j = (idx % (S / 4)) * 4;
-    float* dst = Ws + rl * SS_WLD + j;
+    float* dst = Ws + rl * WLD + j;
     if (row0 + rl < a.m)
       cp_async16(dst, a.Wq + static_cast<size_t>(row0 + rl) * n + s0 + j);
     else
@@ -121,7 +125,7 @@ __global__ void __launch_bounds__(SS_THREADS, 1) sweep_slab_kernel(SweepArgs a, 
       float wmin = INFINITY, wmax = -INFINITY, amax = 0.0f;
       const int in_end = min(S, bo + a.g);
       for (int j = bo + q; j < in_end; j += SS_NW) {
-        const float x = Ws[rl * SS_WLD + j];
+        const float x = Ws[rl * WLD + j];
         wmin = fminf(wmin, x);
         wmax = fmaxf(wmax, x);
         amax = fmaxf(amax, fabsf(x));
@@ -169,7 +173,7 @@ __global__ void __launch_bounds__(SS_THREADS, 1) sweep_slab_kernel(SweepArgs a, 
       // inside the rounding the zero-point enters only for asymmetric codes
       float zs = a.sym ? 0.0f : z;
       float rs = __frcp_rn(s);
-      float* wrow = Ws + rl * SS_WLD + bo;
+      float* wrow = Ws + rl * WLD + bo;
       float ep[SW_CH];  // the previous chunk's errors
 #pragma unroll
       for (int t = 0; t < SW_CH; ++t) ep[t] = 0.0f;
@@ -283,7 +287,7 @@ __global__ void __launch_bounds__(SS_THREADS, 1) sweep_slab_kernel(SweepArgs a, 
           const int n4 = (SW_B - c0) / 4;
           for (int item = tid - 32; item < SW_ROWS * n4; item += SS_THREADS - 32) {
             const int rl = item & 31, j = c0 + 4 * (item >> 5);
-            float4 acc = *reinterpret_cast<const float4*>(Ws + rl * SS_WLD + bo + j);
+            float4 acc = *reinterpret_cast<const float4*>(Ws + rl * WLD + bo + j);
 #pragma unroll
             for (int t = 0; t < SW_CH; ++t) {
               const float e = Es[rl * SW_ELD + k * SW_CH + t];
@@ -293,7 +297,7 @@ __global__ void __launch_bounds__(SS_THREADS, 1) sweep_slab_kernel(SweepArgs a, 
               acc.z = fmaf(-e, u.z, acc.z);
               acc.w = fmaf(-e, u.w, acc.w);
             }
-            *reinterpret_cast<float4*>(Ws + rl * SS_WLD + bo + j) = acc;
+            *reinterpret_cast<float4*>(Ws + rl * WLD + bo + j) = acc;
           }
         }
         // (2) the slab's later columns: a lane takes four columns, holds their 16 U values
@@ -315,7 +319,7 @@ __global__ void __launch_bounds__(SS_THREADS, 1) sweep_slab_kernel(SweepArgs a, 
               u[t] = __ldg(reinterpret_cast<const float4*>(ub + static_cast<size_t>(t) * n + 4 * q));
 #pragma unroll 2
             for (int r = r0; r < r0 + RCH; ++r) {
-              float* wp = Ws + r * SS_WLD + cb + 4 * q;
+              float* wp = Ws + r * WLD + cb + 4 * q;
               float4 acc = *reinterpret_cast<const float4*>(wp);
 #pragma unroll
               for (int t4 = 0; t4 < SW_CH / 4; ++t4) {

@@ -199,3 +199,16 @@ def test_quantize_layer_parity_across_super_blocks(n, g, sym, bits):
     assert np.array_equal(gpu["perm"], prep["perm"])
     st, rep = GH.check_sweep_replay(gpu["W"], prep, gpu, qs)
     GH.assert_replay_ok(st, rep, gpu)
+
+
+@pytest.mark.parametrize("slab", [128, 512, 1024])
+def test_quantize_layer_parity_other_slab_widths(slab, monkeypatch):
+    """The sweep's slab width (columns per launch, whose later columns are updated inside the
+    launch) changes only the order of the fp32 updates: parity at other widths than the default."""
+    monkeypatch.setenv("GPTQ_SLAB_WIDTH", str(slab))
+    layer = synth.scaled_layer(TINY, m=80, n=2048, n_tok=4096)
+    qs = synth.QuantSetting(4, 128, False, 0.01, True)
+    gpu = GH.run_path(layer, qs)
+    prep = O.prepare(gpu["H"], qs.damp, qs.desc_act)
+    st, rep = GH.check_sweep_replay(gpu["W"], prep, gpu, qs)
+    GH.assert_replay_ok(st, rep, gpu)
