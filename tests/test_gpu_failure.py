@@ -56,7 +56,8 @@ def test_host_wait_with_a_short_limit_returns_timeout(monkeypatch):
         ctx.synchronize()
 
 
-def test_profiling_records_every_role_and_changes_no_result():
+def test_profiling_records_every_role_and_changes_no_result(monkeypatch):
+    monkeypatch.setenv("GPTQ_SLAB_WIDTH", "256")
     layer = synth.scaled_layer(TINY, m=96, n=2304, n_tok=2048)
     qs = synth.QuantSetting(4, 128, False, 0.01, True)
     X, W = synth.make_x_bf16(layer), synth.make_w_fp16(layer)
@@ -74,13 +75,13 @@ def test_profiling_records_every_role_and_changes_no_result():
     assert prof["hessian_syrk_pair"]["launches"] == 1
     assert prof["hessian_syrk_pair"]["flops"] == layer.n_tok * n * (n + 1)
     assert prof["leaf_chol_inv"]["launches"] == n // 128
-    assert prof["sweep_slab"]["launches"] == (n + 1023) // 1024   # one per 1024-column super-block
+    assert prof["sweep_slab"]["launches"] == (n + 255) // 256   # one per 256-column slab
     # the factorization's algorithmic work: n^3/3 for the Cholesky factor and n^3/3 for its
     # inverse, plus lower-order terms of the diagonals
     f = sum(v["flops"] for k, v in prof.items() if ":factor" in k or k == "leaf_chol_inv")
     assert 2 * n ** 3 / 3 <= f <= 1.02 * 2 * n ** 3 / 3, f
-    # the tensor-core trailing update: the columns past each 1024-column super-block (the
-    # updates inside a super-block run in the slab kernel)
+    # the tensor-core trailing update: the columns past each 256-column slab (the updates
+    # inside a slab run in the slab kernel)
     t = sum(v["flops"] for k, v in prof.items() if ":trailing" in k)
-    assert t == 2 * layer.m * sum(min(1024, n - s0) * (n - s0 - 1024) for s0 in range(0, n - 1024, 1024))
+    assert t == 2 * layer.m * sum(min(256, n - s0) * (n - s0 - 256) for s0 in range(0, n - 256, 256))
     assert all(v["ms"] > 0 for v in prof.values())
