@@ -190,8 +190,8 @@ gptq_status gptq_quantize_layer_noalloc(const void* W_fp16, int64_t m, int64_t n
  * Jobs whose X_bf16, n_tok, ld_x and n are equal share one Hessian (e.g. the q, k and v
  * projections of a transformer block read the same input); within such a group, jobs with the
  * same damp and desc_act share one factorization.  Groups run in order of first appearance on
- * two internal contexts and streams: the Hessian of group i+1 and the quantization of group i-1
- * run while group i is factored.  The call allocates its contexts (two per distinct width n;
+ * two internal contexts and streams: the Hessian and the factorization of group i run while the
+ * quantization of group i-1 runs.  The call allocates its contexts (two per distinct width n;
  * GPTQ_ERR_OOM before any launch if they do not fit), waits for `cuda_stream` before starting,
  * returns once every job is done (bounded waits) and frees the contexts.
  * Returns the first error (GPTQ_ERR_NOT_PD names no job; the outputs of later jobs are then
@@ -213,6 +213,22 @@ typedef struct {
 } gptq_layer_job;
 
 gptq_status gptq_quantize_layers(const gptq_layer_job* jobs, int count, int device, void* cuda_stream);
+
+/* The same pipeline with its contexts kept between calls (gptq_quantize_layers creates and frees
+ * them on every call).  gptq_pipeline_create allocates two contexts for each of the `count`
+ * distinct widths widths[i] (up to m_max[i] rows each; GPTQ_ERR_OOM before allocating if they
+ * do not fit) and two streams; each gptq_pipeline_run waits for `cuda_stream` (the stream given
+ * at create) before starting, quantizes its jobs as gptq_quantize_layers does (GPTQ_ERR_ARG if
+ * a job's width has no context or its m exceeds that width's m_max) and returns when they are
+ * done.  Group i of a run (jobs sharing an input) runs on the two contexts alternately: its
+ * Hessian and factorization overlap the quantization of group i-1.  gptq_pipeline_destroy
+ * waits for the streams and frees everything (NULL is accepted).  A pipeline is used by one
+ * host thread at a time. */
+typedef struct gptq_pipeline gptq_pipeline;
+gptq_status gptq_pipeline_create(gptq_pipeline** out, const int64_t* widths, const int64_t* m_max, int count,
+                                 int device, void* cuda_stream);
+gptq_status gptq_pipeline_run(gptq_pipeline* pipeline, const gptq_layer_job* jobs, int count);
+gptq_status gptq_pipeline_destroy(gptq_pipeline* pipeline);
 
 /* ---------------------------------------------------------------------------------------
  * AWQ on the same calibration activations and weights

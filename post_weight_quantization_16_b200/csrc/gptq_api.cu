@@ -1537,14 +1537,93 @@ gptq_status enqueue_hessian(gptq_ctx* c, const gptq_layer_job& a) {
 
 }  // namespace
 
-extern "C" gptq_status gptq_quantize_layers(const gptq_layer_job* jobs, int count, int device, void* cuda_stream) {
-  if (!jobs || count < 1) return GPTQ_ERR_ARG;
+struct gptq_pipeline {
+  int device = 0;
+  cudaStream_t user = nullptr;
+  Slot slot[2];
+  cudaEvent_t ev = nullptr;
+};
+
+namespace {
+
+gptq_status pipeline_free(gptq_pipeline* p) {
+  gptq_status st = GPTQ_OK;
+  for (auto& sl : p->slot) {
+    for (auto& e : sl.ctx) {
+      const gptq_status d = gptq_destroy(e.second);
+      if (st == GPTQ_OK) st = d;
+    }
+    sl.ctx.clear();
+    if (sl.stream) cudaStreamDestroy(sl.stream);
+    sl.stream = nullptr;
+  }
+  if (p->ev) cudaEventDestroy(p->ev);
+  p->ev = nullptr;
+  return st;
+}
+
+bool valid_job(const gptq_layer_job& j) {
+  return j.W_fp16 && j.codes_out && j.scales_out && j.zeros_out && j.m >= 1 && j.n_tok >= 0 &&
+         (j.n_tok == 0 || j.X_bf16) && valid_qparams(j.qp, j.n) && gptq_workspace_bytes(j.n, j.m) != 0 &&
+         j.damp >= 0.0 && j.damp <= 1e6 && (j.desc_act == 0 || j.desc_act == 1);
+}
+
+}  // namespace
+
+extern "C" gptq_status gptq_pipeline_create(gptq_pipeline** out, const int64_t* widths, const int64_t* m_max, int count,
+                                            int device, void* cuda_stream) {
+  if (!out || !widths || !m_max || count < 1) return GPTQ_ERR_ARG;
+  *out = nullptr;
+  size_t need = 0;
   for (int i = 0; i < count; ++i) {
-    const gptq_layer_job& j = jobs[i];
-    if (!j.W_fp16 || !j.codes_out || !j.scales_out || !j.zeros_out || j.m < 1 || j.n_tok < 0 ||
-        (j.n_tok > 0 && !j.X_bf16) || !valid_qparams(j.qp, j.n) || gptq_workspace_bytes(j.n, j.m) == 0 ||
-        !(j.damp >= 0.0) || j.damp > 1e6 || !(j.desc_act == 0 || j.desc_act == 1))
-      return GPTQ_ERR_ARG;
+    const size_t b = gptq_workspace_bytes(widths[i], m_max[i]);
+    if (b == 0) return GPTQ_ERR_ARG;
+    for (int j = 0; j < i; ++j)
+      if (widths[j] == widths[i]) return GPTQ_ERR_ARG;  // one entry per width
+    need += 2 * b;
+  }
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) {
+    cudaGetLastError();
+    return GPTQ_ERR_CUDA;
+  }
+  DeviceGuard dg(device);
+  size_t free_b = 0, total_b = 0;
+  CK(cudaMemGetInfo(&free_b, &total_b));
+  const int64_t env_limit = env_int("GPTQ_MAX_WORKSPACE_BYTES", -1);
+  if (need > free_b || (env_limit >= 0 && static_cast<int64_t>(need) > env_limit)) return GPTQ_ERR_OOM;
+  gptq_pipeline* p = new gptq_pipeline();
+  p->device = device;
+  p->user = static_cast<cudaStream_t>(cuda_stream);
+  gptq_status st = GPTQ_OK;
+  for (auto& sl : p->slot) {
+    if (cudaStreamCreateWithFlags(&sl.stream, cudaStreamNonBlocking) != cudaSuccess) {
+      st = GPTQ_ERR_CUDA;
+      break;
+    }
+    for (int i = 0; i < count && st == GPTQ_OK; ++i) {
+      gptq_ctx* c = nullptr;
+      st = gptq_create(&c, widths[i], m_max[i], device, sl.stream);
+      if (st == GPTQ_OK) sl.ctx.emplace_back(widths[i], c);
+    }
+    if (st != GPTQ_OK) break;
+  }
+  if (st == GPTQ_OK && cudaEventCreateWithFlags(&p->ev, cudaEventDisableTiming) != cudaSuccess) st = GPTQ_ERR_CUDA;
+  if (st != GPTQ_OK) {
+    pipeline_free(p);
+    delete p;
+    return st;
+  }
+  *out = p;
+  return GPTQ_OK;
+}
+
+extern "C" gptq_status gptq_pipeline_run(gptq_pipeline* p, const gptq_layer_job* jobs, int count) {
+  if (!p || !jobs || count < 1) return GPTQ_ERR_ARG;
+  for (int i = 0; i < count; ++i) {
+    if (!valid_job(jobs[i])) return GPTQ_ERR_ARG;
+    gptq_ctx* c = p->slot[0].get(jobs[i].n);
+    if (!c || jobs[i].m > c->m_max) return GPTQ_ERR_ARG;  // no context of that width, or too many rows
   }
   // groups of jobs that share their calibration input, in order of first appearance
   std::vector<LayerGroup> groups;
@@ -1558,85 +1637,61 @@ extern "C" gptq_status gptq_quantize_layers(const gptq_layer_job* jobs, int coun
     }
     g->jobs.push_back(i);
   }
-  // contexts: two per distinct width, sized for the batch's largest m at that width
-  std::vector<std::pair<int64_t, int64_t>> widths;  // (n, m_max)
-  for (int i = 0; i < count; ++i) {
-    bool found = false;
-    for (auto& w : widths)
-      if (w.first == jobs[i].n) {
-        w.second = std::max(w.second, jobs[i].m);
-        found = true;
-      }
-    if (!found) widths.emplace_back(jobs[i].n, jobs[i].m);
-  }
-  int ndev = 0;
-  if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) {
-    cudaGetLastError();
-    return GPTQ_ERR_CUDA;
-  }
-  DeviceGuard dg(device);
-  size_t need = 0;
-  for (auto& w : widths) need += 2 * gptq_workspace_bytes(w.first, w.second);
-  size_t free_b = 0, total_b = 0;
-  CK(cudaMemGetInfo(&free_b, &total_b));
-  const int64_t env_limit = env_int("GPTQ_MAX_WORKSPACE_BYTES", -1);
-  if (need > free_b || (env_limit >= 0 && static_cast<int64_t>(need) > env_limit)) return GPTQ_ERR_OOM;
-
-  Slot slot[2];
-  gptq_status st = GPTQ_OK;
-  cudaEvent_t ev = nullptr;
-  auto cleanup = [&]() {
-    for (auto& sl : slot) {
-      for (auto& e : sl.ctx) {
-        const gptq_status d = gptq_destroy(e.second);
-        if (st == GPTQ_OK) st = d;
-      }
-      if (sl.stream) cudaStreamDestroy(sl.stream);
-    }
-    if (ev) cudaEventDestroy(ev);
-  };
-  for (auto& sl : slot) {
-    if (cudaStreamCreateWithFlags(&sl.stream, cudaStreamNonBlocking) != cudaSuccess) {
-      st = GPTQ_ERR_CUDA;
-      cleanup();
-      return st;
-    }
-    for (auto& w : widths) {
-      gptq_ctx* c = nullptr;
-      st = gptq_create(&c, w.first, w.second, device, sl.stream);
-      if (st != GPTQ_OK) {
-        cleanup();
-        return st;
-      }
-      sl.ctx.emplace_back(w.first, c);
-    }
-  }
+  DeviceGuard dg(p->device);
   // start after the caller's stream
-  if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess ||
-      cudaEventRecord(ev, static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess ||
-      cudaStreamWaitEvent(slot[0].stream, ev, 0) != cudaSuccess || cudaStreamWaitEvent(slot[1].stream, ev, 0) != cudaSuccess) {
-    st = GPTQ_ERR_CUDA;
-    cleanup();
-    return st;
+  CK(cudaEventRecord(p->ev, p->user));
+  for (auto& sl : p->slot) CK(cudaStreamWaitEvent(sl.stream, p->ev, 0));
+  // Group i runs on slot i % 2: its Hessian and factorization are enqueued behind that slot's
+  // earlier work, while the quantization of group i-1, enqueued on the other slot, runs; the
+  // host waits only inside each factorization (for its pivot check).
+  gptq_status st = GPTQ_OK;
+  for (size_t i = 0; i < groups.size() && st == GPTQ_OK; ++i) {
+    gptq_ctx* c = p->slot[i & 1].get(groups[i].first->n);
+    st = enqueue_hessian(c, *groups[i].first);
+    if (st == GPTQ_OK) st = run_group(c, jobs, groups[i]);
   }
-  const int G = static_cast<int>(groups.size());
-  st = enqueue_hessian(slot[0].get(groups[0].first->n), *groups[0].first);
-  for (int i = 0; i < G && st == GPTQ_OK; ++i) {
-    if (i + 1 < G) {  // the next group's Hessian on the other slot, behind that slot's last quantization
-      const LayerGroup& nx = groups[i + 1];
-      st = enqueue_hessian(slot[(i + 1) & 1].get(nx.first->n), *nx.first);
-      if (st != GPTQ_OK) break;
-    }
-    st = run_group(slot[i & 1].get(groups[i].first->n), jobs, groups[i]);
-  }
-  // wait for both slots and collect any device-side failure
-  for (auto& sl : slot)
+  // wait for both slots, collect any device-side failure, and order the caller's stream after
+  for (auto& sl : p->slot)
     for (auto& e : sl.ctx) {
       const gptq_status s = gptq_synchronize(e.second);
       if (st == GPTQ_OK) st = s;
     }
-  cleanup();
   return st;
+}
+
+extern "C" gptq_status gptq_pipeline_destroy(gptq_pipeline* p) {
+  if (!p) return GPTQ_OK;
+  gptq_status st;
+  {
+    DeviceGuard dg(p->device);
+    st = pipeline_free(p);
+  }
+  delete p;
+  return st;
+}
+
+extern "C" gptq_status gptq_quantize_layers(const gptq_layer_job* jobs, int count, int device, void* cuda_stream) {
+  if (!jobs || count < 1) return GPTQ_ERR_ARG;
+  std::vector<int64_t> widths, mm;
+  for (int i = 0; i < count; ++i) {
+    if (!valid_job(jobs[i])) return GPTQ_ERR_ARG;
+    bool found = false;
+    for (size_t w = 0; w < widths.size(); ++w)
+      if (widths[w] == jobs[i].n) {
+        mm[w] = std::max(mm[w], jobs[i].m);
+        found = true;
+      }
+    if (!found) {
+      widths.push_back(jobs[i].n);
+      mm.push_back(jobs[i].m);
+    }
+  }
+  gptq_pipeline* p = nullptr;
+  gptq_status st = gptq_pipeline_create(&p, widths.data(), mm.data(), static_cast<int>(widths.size()), device, cuda_stream);
+  if (st != GPTQ_OK) return st;
+  st = gptq_pipeline_run(p, jobs, count);
+  const gptq_status d = gptq_pipeline_destroy(p);
+  return st != GPTQ_OK ? st : d;
 }
 
 // ==========================================================================================

@@ -75,6 +75,10 @@ _SIGS = {
                                            QParams, _P, _P, ctypes.c_size_t, ctypes.c_int, _P]),
     "gptq_dequant_matmul_check": (ctypes.c_int, [_P, ctypes.c_int, _P]),
     "gptq_quantize_layers": (ctypes.c_int, [ctypes.POINTER(LayerJob), ctypes.c_int, ctypes.c_int, _P]),
+    "gptq_pipeline_create": (ctypes.c_int, [ctypes.POINTER(_P), ctypes.POINTER(ctypes.c_int64),
+                                            ctypes.POINTER(ctypes.c_int64), ctypes.c_int, ctypes.c_int, _P]),
+    "gptq_pipeline_run": (ctypes.c_int, [_P, ctypes.POINTER(LayerJob), ctypes.c_int]),
+    "gptq_pipeline_destroy": (ctypes.c_int, [_P]),
     "gptq_awq_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int64]),
     "gptq_awq_quantize": (ctypes.c_int, [_P, ctypes.c_int64, ctypes.c_int64, _P, ctypes.c_int64, ctypes.c_int64,
                                          ctypes.c_float, QParams, _P, _P, _P, _P, _P, _P, ctypes.c_size_t,
@@ -276,25 +280,20 @@ def dequant_matmul(X: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, z
     return out
 
 
-def quantize_layers(layers: list, device: int = 0, stream: torch.cuda.Stream | None = None) -> list:
-    """Quantize many layers in one pipelined call (gptq_quantize_layers).  `layers` is a list of
-    dicts with X (bf16 [n_tok, n] device tensor; the same tensor object for layers that share an
-    input), W (fp16 [m, n]), bits, group_size, sym, damp, desc_act and optional want_w_hat.
-    Returns one dict of device outputs per layer (codes, scales, zeros, g_idx, perm, w_hat)."""
-    dev = torch.device("cuda", device)
-    stream = stream if stream is not None else torch.cuda.current_stream(dev)
+def _jobs(layers: list, dev: torch.device):
     jobs = (LayerJob * len(layers))()
     outs = []
     for i, L in enumerate(layers):
         X, W = L["X"], L["W"]
         m, n = W.shape
         g = n if L["group_size"] == -1 else L["group_size"]
-        o = {"codes": torch.empty((m, n * L["bits"] // 32), dtype=torch.int32, device=dev),
-             "scales": torch.empty((m, n // g), dtype=torch.float32, device=dev),
-             "zeros": torch.empty((m, n // g), dtype=torch.float32, device=dev),
-             "g_idx": torch.empty(n, dtype=torch.int32, device=dev),
-             "perm": torch.empty(n, dtype=torch.int32, device=dev),
-             "w_hat": torch.empty((m, n), dtype=torch.float32, device=dev) if L.get("want_w_hat") else None}
+        o = L.get("out") or {
+            "codes": torch.empty((m, n * L["bits"] // 32), dtype=torch.int32, device=dev),
+            "scales": torch.empty((m, n // g), dtype=torch.float32, device=dev),
+            "zeros": torch.empty((m, n // g), dtype=torch.float32, device=dev),
+            "g_idx": torch.empty(n, dtype=torch.int32, device=dev),
+            "perm": torch.empty(n, dtype=torch.int32, device=dev),
+            "w_hat": torch.empty((m, n), dtype=torch.float32, device=dev) if L.get("want_w_hat") else None}
         outs.append(o)
         j = jobs[i]
         j.X_bf16, j.n_tok, j.ld_x = X.data_ptr(), X.shape[0], X.stride(0)
@@ -303,7 +302,50 @@ def quantize_layers(layers: list, device: int = 0, stream: torch.cuda.Stream | N
         j.damp, j.desc_act = float(L["damp"]), int(bool(L["desc_act"]))
         j.codes_out, j.scales_out, j.zeros_out = o["codes"].data_ptr(), o["scales"].data_ptr(), o["zeros"].data_ptr()
         j.g_idx_out, j.perm_out = o["g_idx"].data_ptr(), o["perm"].data_ptr()
-        j.W_hat_out = o["w_hat"].data_ptr() if o["w_hat"] is not None else None
+        j.W_hat_out = o["w_hat"].data_ptr() if o.get("w_hat") is not None else None
+    return jobs, outs
+
+
+class Pipeline:
+    """Contexts kept between batches of layers (gptq_pipeline_*): `widths` maps each input width
+    to the largest number of rows its layers have."""
+
+    def __init__(self, widths: dict, device: int = 0, stream: torch.cuda.Stream | None = None):
+        self.device = torch.device("cuda", device)
+        self.stream = stream if stream is not None else torch.cuda.current_stream(self.device)
+        ws = (ctypes.c_int64 * len(widths))(*[int(w) for w in widths])
+        ms = (ctypes.c_int64 * len(widths))(*[int(m) for m in widths.values()])
+        h = ctypes.c_void_p()
+        _check(lib().gptq_pipeline_create(ctypes.byref(h), ws, ms, len(widths), self.device.index,
+                                          ctypes.c_void_p(self.stream.cuda_stream)), "gptq_pipeline_create")
+        self._h = h
+
+    def run(self, layers: list) -> list:
+        jobs, outs = _jobs(layers, self.device)
+        _check(lib().gptq_pipeline_run(self._h, jobs, len(layers)), "gptq_pipeline_run")
+        return outs
+
+    def close(self):
+        if getattr(self, "_h", None):
+            st = lib().gptq_pipeline_destroy(self._h)
+            self._h = None
+            _check(st, "gptq_pipeline_destroy")
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        self.close()
+
+
+def quantize_layers(layers: list, device: int = 0, stream: torch.cuda.Stream | None = None) -> list:
+    """Quantize many layers in one pipelined call (gptq_quantize_layers).  `layers` is a list of
+    dicts with X (bf16 [n_tok, n] device tensor; the same tensor object for layers that share an
+    input), W (fp16 [m, n]), bits, group_size, sym, damp, desc_act and optional want_w_hat.
+    Returns one dict of device outputs per layer (codes, scales, zeros, g_idx, perm, w_hat)."""
+    dev = torch.device("cuda", device)
+    stream = stream if stream is not None else torch.cuda.current_stream(dev)
+    jobs, outs = _jobs(layers, dev)
     _check(lib().gptq_quantize_layers(jobs, len(layers), dev.index, ctypes.c_void_p(stream.cuda_stream)),
            "gptq_quantize_layers")
     return outs

@@ -67,3 +67,28 @@ def test_pipeline_equals_layers_quantized_alone():
            "scales": outs[2]["scales"].cpu().numpy(), "zeros": outs[2]["zeros"].cpu().numpy()}
     st, rep = GH.check_sweep_replay(Wa2.cpu().numpy(), prep, gpu, synth.QuantSetting(2, -1, False, 0.1, True))
     GH.assert_replay_ok(st, rep, gpu)
+
+
+@pytest.mark.gpu
+def test_pipeline_handle_reused_for_two_batches():
+    """One pipeline, two batches of different layers: each job equals the layer quantized alone."""
+    import dataclasses
+    lays = [dataclasses.replace(synth.scaled_layer(TINY, m=64, n=512, n_tok=1024, name=f"p{i}"), x_seed=20 + i,
+                                w_seed=40 + i) for i in range(3)]
+    Xs = [GH.bf16_to_dev(synth.make_x_bf16(l)) for l in lays]
+    Ws = [torch.from_numpy(synth.make_w_fp16(l)).to(GH.DEV) for l in lays]
+    with G.Pipeline({512: 64}) as pipe:
+        for batch in ([0, 1], [2, 0]):
+            layers = [dict(X=Xs[i], W=Ws[i], bits=4, group_size=128, sym=False, damp=0.01, desc_act=True)
+                      for i in batch]
+            outs = pipe.run(layers)
+            torch.cuda.synchronize(GH.DEV)
+            for i, o in zip(batch, outs):
+                ref, _ = _alone(Xs[i], Ws[i], 4, 128, False, 0.01, True)
+                for k in ("codes", "scales", "zeros", "g_idx", "perm"):
+                    assert np.array_equal(o[k].cpu().numpy(), ref[k]), (batch, i, k)
+        # a job wider than the pipeline's contexts is refused
+        with pytest.raises(G.GPTQError) as ei:
+            pipe.run([dict(X=Xs[0], W=torch.zeros((65, 512), dtype=torch.float16, device=GH.DEV), bits=4,
+                           group_size=128, sym=False, damp=0.01, desc_act=True)])
+        assert ei.value.status == G.ERR_ARG
