@@ -285,6 +285,19 @@ gptq_status gptq_dequant_matmul(const void* X_fp16, int64_t T, const uint32_t* c
                                 float* Y, void* workspace, size_t workspace_bytes, int device, void* cuda_stream);
 gptq_status gptq_dequant_matmul_check(void* workspace, int device, void* cuda_stream);
 
+/* ---------------------------------------------------------------------------------------
+ * Sequential (cross-layer) quantization ("GPTQ算法原理深度解析" §2.1: the quantization error of a
+ * layer reaches the next layer through its input): layer l+1 is calibrated on the outputs of
+ * the already-quantized layer l, y = X_l W16_l^T (gptq_dequant_matmul), through the model's
+ * activation.  This call forms those inputs:
+ *   x = act(y)   act 0 = identity, 1 = ReLU (y if y > 0, else 0)
+ *   Y        : device, `count` values, fp32 (in_bf16 = 0) or bf16 (in_bf16 = 1)
+ *   out_bf16 : device bf16 [count] or NULL (the next Hessian's input), round to nearest even
+ *   out_fp16 : device fp16 [count] or NULL (the next product's input), round to nearest even
+ * At least one output.  Asynchronous on cuda_stream. */
+gptq_status gptq_activation_convert(const void* Y, int in_bf16, int64_t count, int act, void* out_bf16, void* out_fp16,
+                                    int device, void* cuda_stream);
+
 /* Per-kernel instrumentation (off by default).  While profiling is on, every kernel the
  * context launches is bracketed by CUDA timing events on the context's stream and the
  * factorization runs as individual launches instead of its recorded graph (so launches no

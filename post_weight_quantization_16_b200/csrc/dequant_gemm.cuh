@@ -24,6 +24,7 @@
 // nearest fp16 (cvt.rn.f16x2.f32).
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
 #include <cstdint>
@@ -320,6 +321,20 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ P, int splits, si
     float acc = P[i];
     for (int s = 1; s < splits; ++s) acc += P[static_cast<size_t>(s) * count + i];
     Y[i] = acc;
+  }
+}
+
+// The next layer's inputs from a layer's output (sequential quantization): x = act(y), act 0 =
+// identity, 1 = ReLU (y if y > 0, else 0), from fp32 or bf16 y, written as bf16 and/or fp16
+// (round to nearest even).  Grid-stride, one element per thread and step.
+__global__ void activation_convert_kernel(const void* __restrict__ Y, int in_bf16, size_t count, int act,
+                                          __nv_bfloat16* __restrict__ out_bf16, __half* __restrict__ out_fp16) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < count;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    float y = in_bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(Y)[i]) : static_cast<const float*>(Y)[i];
+    if (act == 1) y = (y > 0.0f) ? y : 0.0f;
+    if (out_bf16) out_bf16[i] = __float2bfloat16_rn(y);
+    if (out_fp16) out_fp16[i] = __float2half_rn(y);
   }
 }
 

@@ -1755,3 +1755,24 @@ extern "C" gptq_status gptq_awq_quantize(const void* X, int64_t n_tok, int64_t l
   CKL("awq_rtn");
   return GPTQ_OK;
 }
+
+// ==========================================================================================
+// Sequential quantization: a layer's output, through its activation, as the next layer's inputs
+// ==========================================================================================
+extern "C" gptq_status gptq_activation_convert(const void* Y, int in_bf16, int64_t count, int act, void* out_bf16,
+                                               void* out_fp16, int device, void* cuda_stream) {
+  if (count < 0 || (count > 0 && !Y) || (!out_bf16 && !out_fp16) || (act != 0 && act != 1) ||
+      (in_bf16 != 0 && in_bf16 != 1))
+    return GPTQ_ERR_ARG;
+  if (count == 0) return GPTQ_OK;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) {
+    cudaGetLastError();
+    return GPTQ_ERR_CUDA;
+  }
+  DeviceGuard dg(device);
+  activation_convert_kernel<<<4 * 148, 256, 0, static_cast<cudaStream_t>(cuda_stream)>>>(
+      Y, in_bf16, static_cast<size_t>(count), act, static_cast<__nv_bfloat16*>(out_bf16), static_cast<__half*>(out_fp16));
+  CKL("activation_convert");
+  return GPTQ_OK;
+}

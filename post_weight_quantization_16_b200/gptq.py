@@ -79,6 +79,8 @@ _SIGS = {
                                             ctypes.POINTER(ctypes.c_int64), ctypes.c_int, ctypes.c_int, _P]),
     "gptq_pipeline_run": (ctypes.c_int, [_P, ctypes.POINTER(LayerJob), ctypes.c_int]),
     "gptq_pipeline_destroy": (ctypes.c_int, [_P]),
+    "gptq_activation_convert": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_int64, ctypes.c_int, _P, _P, ctypes.c_int,
+                                               _P]),
     "gptq_awq_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int64]),
     "gptq_awq_quantize": (ctypes.c_int, [_P, ctypes.c_int64, ctypes.c_int64, _P, ctypes.c_int64, ctypes.c_int64,
                                          ctypes.c_float, QParams, _P, _P, _P, _P, _P, _P, ctypes.c_size_t,
@@ -373,3 +375,54 @@ def awq_quantize(X: torch.Tensor | None, W: torch.Tensor, s_protect: float = 2.0
                                    _ptr(out["w_hat"]), _ptr(ws), ws.numel(), dev.index,
                                    ctypes.c_void_p(stream.cuda_stream)), "gptq_awq_quantize")
     return out
+
+
+def activation_convert(Y: torch.Tensor, act: int = 1, want_bf16: bool = True, want_fp16: bool = True,
+                       stream: torch.cuda.Stream | None = None):
+    """x = act(y) (0 identity, 1 ReLU) of an fp32 or bf16 device tensor, as bf16 and fp16 copies
+    (gptq_activation_convert)."""
+    if Y.dtype not in (torch.float32, torch.bfloat16) or not Y.is_contiguous():
+        raise ValueError("Y must be a contiguous fp32 or bf16 device tensor")
+    dev = Y.device
+    stream = stream if stream is not None else torch.cuda.current_stream(dev)
+    xb = torch.empty(Y.shape, dtype=torch.bfloat16, device=dev) if want_bf16 else None
+    xh = torch.empty(Y.shape, dtype=torch.float16, device=dev) if want_fp16 else None
+    _check(lib().gptq_activation_convert(_ptr(Y), int(Y.dtype == torch.bfloat16), Y.numel(), int(act), _ptr(xb),
+                                         _ptr(xh), dev.index, ctypes.c_void_p(stream.cuda_stream)),
+           "gptq_activation_convert")
+    return xb, xh
+
+
+def quantize_sequential(X0: torch.Tensor, layers: list, act: int = 1, stream: torch.cuda.Stream | None = None,
+                        keep_hessian: bool = False) -> list:
+    """Sequential quantization of a stack of linear layers ("GPTQ算法原理深度解析" §2.1: the error
+    of a layer reaches the next one through its input).  X0: bf16 [N, n0] calibration inputs of
+    layer 0; layers: dicts with W (fp16 [m_l, n_l], n_{l+1} = m_l), bits, group_size, sym, damp,
+    desc_act.  Layer l is calibrated on X_l; X_{l+1} = act(X_l W16_l^T), the product taken with
+    layer l's quantized weights (gptq_dequant_matmul on the fp16 copy of X_l).  Every step runs in
+    the library's kernels; this function only sequences the calls.  Returns, per layer, its
+    outputs (codes, scales, zeros, g_idx, perm), its calibration inputs X (bf16) and X16 (the
+    fp16 copy its product reads), and with keep_hessian its H (fp32 [n, n])."""
+    dev = X0.device
+    stream = stream if stream is not None else torch.cuda.current_stream(dev)
+    xb = X0
+    _, xh = activation_convert(X0, act=0, want_bf16=False, stream=stream)
+    res = []
+    for li, L in enumerate(layers):
+        W = L["W"]
+        m, n = W.shape
+        if xb.shape[1] != n:
+            raise ValueError(f"layer {li}: {n} inputs, but the previous layer gives {xb.shape[1]}")
+        with GPTQContext(n, m, dev.index, stream) as ctx:
+            ctx.accumulate_hessian(xb)
+            H = ctx.get_hessian()[0] if keep_hessian else None
+            perm = ctx.prepare(L["damp"], L["desc_act"])
+            out = ctx.quantize_layer(W, L["bits"], L["group_size"], L["sym"], want_w_hat=False)
+            ctx.synchronize()
+        out = dict(out, perm=perm, X=xb, X16=xh, H=H)
+        res.append(out)
+        if li + 1 < len(layers):
+            Y = dequant_matmul(xh, out["codes"], out["scales"], out["zeros"], perm, L["bits"], L["group_size"],
+                               stream=stream)
+            xb, xh = activation_convert(Y, act=act, stream=stream)
+    return res
