@@ -19,7 +19,7 @@ pytestmark = pytest.mark.gpu
 
 
 def _bits_to_f64(t, bf16):
-    a = t.cpu().numpy().view(np.uint16 if bf16 else np.float16)
+    a = t.cpu().view(torch.int16).numpy().view(np.uint16) if bf16 else t.cpu().numpy()
     return (synth.bf16_bits_to_f32(a) if bf16 else a.astype(np.float32)).astype(np.float64)
 
 
@@ -31,10 +31,10 @@ def test_activation_convert_rounds_to_nearest():
     xb, xh = G.activation_convert(Y, act=1)
     torch.cuda.synchronize(GH.DEV)
     relu = np.where(y > 0, y, np.float32(0))
-    assert np.array_equal(xb.cpu().numpy().view(np.uint16), synth.f32_to_bf16_bits(relu))
+    assert np.array_equal(xb.cpu().view(torch.int16).numpy().view(np.uint16), synth.f32_to_bf16_bits(relu))
     assert np.array_equal(xh.cpu().numpy(), relu.astype(np.float16))
     xb2, _ = G.activation_convert(Y, act=0, want_fp16=False)
-    assert np.array_equal(xb2.cpu().numpy().view(np.uint16), synth.f32_to_bf16_bits(y))
+    assert np.array_equal(xb2.cpu().view(torch.int16).numpy().view(np.uint16), synth.f32_to_bf16_bits(y))
 
 
 def test_three_layer_relu_stack_stage_by_stage():

@@ -98,12 +98,17 @@ def test_noalloc_matches_oracle_and_context_path_on_two_calls(bits, g, sym, want
         assert same >= GH.CODES_IDENTICAL, (call, same)
         assert torch.equal(out["zeros"], ref["zeros"]), call
         if want_what:
-            # where both paths chose the same code the dequantized weights agree to the scales'
-            # tolerance; an in-band code flip (allowed above) moves one weight by a whole step
-            what = out["w_hat"].cpu().numpy().astype(np.float64)
-            same_orig = np.empty_like(gpu["codes"], dtype=bool)
-            same_orig[:, prep["perm"]] = gpu["codes"] == ref_codes
-            ref_what = ref["w_hat"].cpu().numpy().astype(np.float64)
-            assert np.allclose(what[same_orig], ref_what[same_orig], rtol=GH.SZ_REL, atol=1e-12), call
+            # the dequantized weights are (code - zero) * scale of this call's own outputs, taken in
+            # fp32 and stored in the original column order (the scales themselves were checked
+            # against the oracle's replay above; the context path, which accumulates the
+            # propagated errors in another order, may differ from this one by a scale tolerance
+            # on each side, so its weights are not the yardstick here)
+            what = out["w_hat"].cpu().numpy()
+            gw = qs.group_size if qs.group_size > 0 else layer.n
+            grp = np.arange(layer.n) // gw
+            expect = np.empty_like(what)
+            expect[:, prep["perm"]] = ((gpu["codes"].astype(np.float32) - gpu["zeros"][:, grp].astype(np.float32))
+                                       * gpu["scales"][:, grp].astype(np.float32))
+            assert np.array_equal(what, expect), call
             if with_dead:
                 assert not what[:, [3, 500, 1000]].any()
