@@ -255,6 +255,27 @@ def test_blocked_equals_unblocked(n, B, g):
     assert np.allclose(a["what"], b["what"], rtol=1e-12, atol=1e-14)
 
 
+@pytest.mark.parametrize("n,g,sym,block", [(256, 64, False, None), (384, 128, True, 128), (320, -1, False, 64)])
+def test_sweep_errors_satisfy_E_U_equals_W_minus_Q(n, g, sym, block):
+    """Column i's weight after the updates of the columns before it is w_i - sum_{k<i} e_k U[k, i],
+    and e_i U[i, i] is its rounding residual, so E U = W - Q exactly (W the weights the sweep
+    starts from, Q the dequantized values): a dropped, transposed or mis-signed update breaks
+    it.  Consequence used by the CUDA path: the errors of all columns before a column block S
+    reach it as -E[:, <S] U[<S, S] = (W - Q)[:, <S] V[<S, S] U[S, S] with V = U^-1."""
+    H = _spd(n, 31, cond_boost=20.0)
+    p = O.prepare(H, 0.01, True)
+    Wp = _rng(32).normal(0, 0.02, (24, n))[:, p["perm"]]
+    sw = O.gptq_sweep(Wp, p["U"], 3, g, sym, block=block)
+    U = p["U"]
+    D = Wp - sw["what"]
+    assert np.allclose(sw["err"] @ U, D, rtol=0, atol=1e-12 * np.abs(Wp).max())
+    V = np.linalg.inv(U)
+    for s0, s1 in ((128, 256), (64, 192), (n - 64, n)):
+        lhs = -sw["err"][:, :s0] @ U[:s0, s0:s1]
+        rhs = D[:, :s0] @ V[:s0, s0:s1] @ U[s0:s1, s0:s1]
+        assert np.allclose(lhs, rhs, rtol=0, atol=1e-10 * np.abs(lhs).max())
+
+
 def test_brute_force_optimum_and_gptq_beats_rtn_on_average():
     bits, n = 4, 4
     e_gptq, e_rtn = [], []
