@@ -252,6 +252,23 @@ class GPTQContext:
         _check(lib().gptq_reset(self._h), "gptq_reset")
 
 
+def allreduce_hessian(ctx, group=None) -> int:
+    """Token-split calibration across the ranks of a torch.distributed group: each rank has
+    accumulated 2 X^T X over its own share of the tokens ("模型量化实战…" §3.2 accumulate_hessian:
+    the Hessian is a sum over tokens, so partial sums add).  The partial H and token counts are
+    summed with one all-reduce each (n^2 fp32 on the group's backend: NCCL over NVLink between
+    GPUs) and every rank's context continues from the full H.  Returns the total token count.
+    Every rank must call it, in the same order as its other collectives."""
+    import torch.distributed as dist
+    H, nt = ctx.get_hessian()
+    dist.all_reduce(H, op=dist.ReduceOp.SUM, group=group)
+    t = torch.tensor([nt], dtype=torch.int64, device=H.device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM, group=group)
+    total = int(t.item())
+    ctx.set_hessian(H, total)
+    return total
+
+
 def workspace_bytes(n: int, m_max: int) -> int:
     return int(lib().gptq_workspace_bytes(int(n), int(m_max)))
 

@@ -2,9 +2,9 @@
 
 The layer solve itself runs on one GPU.  Under torchrun the benchmark gives each rank its
 own independent layer (weak scaling, no collective on the data path) and reduces only the
-timing (max over ranks).  The natural data-parallel form of the Hessian (each rank sums
-2 x^T x over its own calibration tokens, one all-reduce of H) is checked here too, on the
-oracle, as the exchange a multi-GPU calibration would need.
+timing (max over ranks).  The data-parallel form of the Hessian (each rank sums 2 x^T x over
+its own calibration tokens, one all-reduce of H: gptq.allreduce_hessian) is checked here too,
+with the oracle standing in for the device context.
 """
 import os
 import socket
@@ -17,7 +17,27 @@ import torch.multiprocessing as mp
 
 import bench
 from oracle import gptq_oracle as O
+from post_weight_quantization_16_b200 import gptq as G
 from post_weight_quantization_16_b200 import synth
+
+
+class _OracleContext:
+    """The host-side face of a context (get_hessian / set_hessian) over the oracle's Hessian."""
+
+    def __init__(self, n):
+        self.H = torch.zeros((n, n), dtype=torch.float64)
+        self.n_tok = 0
+
+    def accumulate_hessian(self, X):
+        self.H += torch.from_numpy(O.hessian(X))
+        self.n_tok += X.shape[0]
+
+    def get_hessian(self):
+        return self.H.clone(), self.n_tok
+
+    def set_hessian(self, H, n_tok):
+        self.H = H.clone()
+        self.n_tok = n_tok
 
 
 def _free_port():
@@ -36,13 +56,15 @@ def _worker(rank, world, port, q):
         layer = bench.rank_layer(layer0, r)
         # timing reduction: the job time is the slowest rank's
         t = bench.max_over_ranks(1.0 + r, w)
-        # token-split Hessian: each rank accumulates its own share, one sum all-reduce
+        # token-split Hessian through the binding's exchange step (gptq.allreduce_hessian), the
+        # oracle standing in for the device context: each rank accumulates its own share
         X = synth.bf16_bits_to_f32(synth.make_x_bf16(layer0)).astype(np.float64)
         shard = np.array_split(X, w)[r]
-        Hp = torch.from_numpy(O.hessian(shard))
-        dist.all_reduce(Hp, op=dist.ReduceOp.SUM)
+        ctx = _OracleContext(X.shape[1])
+        ctx.accumulate_hessian(shard)
+        total = G.allreduce_hessian(ctx)
         bench.barrier(w)
-        q.put((r, w, lr, layer.x_seed, layer.w_seed, t, Hp.numpy()))
+        q.put((r, w, lr, layer.x_seed, layer.w_seed, t, ctx.H.numpy(), total, ctx.n_tok))
     finally:
         dist.destroy_process_group()
 
@@ -59,7 +81,7 @@ def test_two_ranks_gloo():
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    (r0, w0, l0, xs0, ws0, t0, H0), (r1, w1, l1, xs1, ws1, t1, H1) = res
+    (r0, w0, l0, xs0, ws0, t0, H0, tot0, nt0), (r1, w1, l1, xs1, ws1, t1, H1, tot1, nt1) = res
     assert (r0, r1) == (0, 1) and w0 == w1 == 2 and (l0, l1) == (0, 1)
     # independent layers: rank 0 keeps the workload's own seeds, rank 1 gets other ones
     layer0, _ = synth.WORKLOADS["tiny_256x512"]
@@ -70,6 +92,8 @@ def test_two_ranks_gloo():
     # all ranks hold the Hessian of the whole calibration set
     Href = O.hessian(synth.bf16_bits_to_f32(synth.make_x_bf16(layer0)))
     assert np.allclose(H0, Href, rtol=1e-12, atol=0) and np.array_equal(H0, H1)
+    n_tok = layer0.n_tok
+    assert tot0 == tot1 == nt0 == nt1 == n_tok
 
 
 def test_single_rank_helpers_without_process_group():
