@@ -16,7 +16,10 @@ extern "C" {
  *   A_hi/A_lo : device fp32 [M x K], leading dimension lda (A = A_hi + A_lo; hi/lo are tf32 values)
  *   B_hi/B_lo : device fp32 [N x K], leading dimension ldb
  *   k_lo_mode : 0 = K from 0; 1 = K from the first column of the output tile (B lower-triangular
- *               in this form); 2 = K from the first row of the tile (A upper-triangular)
+ *               in this form); 2 = K from the first row of the tile (A upper-triangular);
+ *               3 + j (j = 0..3) = K over the aligned block of kblk = 128 * 2^j columns that
+ *               holds the output tile only (B block-diagonal with kblk x kblk blocks; the tile
+ *               width is then at most kblk; k_hi_mode 1 still stops K at the tile's last column)
  *   k_hi_mode : 0 = K to the end; 1 = K up to the last column of the tile (B upper-triangular)
  *   upper_only: skip output tiles wholly below the diagonal of C
  *   C         : fp32 output [M x N] (ldc) or NULL; C_hi/C_lo: hi/lo output (ldh) or NULL;

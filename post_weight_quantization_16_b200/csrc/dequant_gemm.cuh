@@ -39,8 +39,12 @@ constexpr int DQ_THREADS = 64 + 256;             // producer, MMA, 8 dequant/epi
 constexpr int DQ_A_ATOM = DQ_BM * 64 * 2;        // 16 KB: 128 rows x 64 fp16
 constexpr int DQ_A_BYTES = 2 * DQ_A_ATOM;        // 32 KB per dequantized tile
 constexpr int DQ_NA = 2;                         // dequantized tiles in flight
-constexpr int DQ_SMEM_BUDGET = 224 * 1024;
+constexpr int DQ_SMEM_BUDGET = 224 * 1024;       // one CTA per SM
+constexpr int DQ_SMEM_BUDGET2 = 113 * 1024;      // two CTAs per SM (each also costs the SM 1 KB)
 
+// Few tokens (decode-sized T): the dequantization, not the MMA, sets the pace, so two CTAs share
+// an SM (16 dequantizing warps) with fewer stages each; 8-bit codes keep one (their registers).
+__host__ __device__ inline int dq_minb(int tn, int bits) { return (tn <= 32 && bits != 8) ? 2 : 1; }
 __host__ __device__ inline int dq_code_bytes(int bits) { return DQ_BM * DQ_BK * bits / 8; }
 __host__ __device__ inline int dq_x_atom_bytes(int tn) { return tn * 128; }
 __host__ __device__ inline int dq_stage_bytes(int tn, int bits) {
@@ -48,7 +52,8 @@ __host__ __device__ inline int dq_stage_bytes(int tn, int bits) {
   return c + 2 * dq_x_atom_bytes(tn);
 }
 __host__ __device__ inline int dq_stages(int tn, int bits) {
-  const int avail = DQ_SMEM_BUDGET - 1024 - 256 - DQ_NA * DQ_A_BYTES;
+  const int budget = dq_minb(tn, bits) == 2 ? DQ_SMEM_BUDGET2 : DQ_SMEM_BUDGET;
+  const int avail = budget - 1024 - 256 - DQ_NA * DQ_A_BYTES;
   int s = avail / dq_stage_bytes(tn, bits);
   return s < 2 ? 2 : (s > 8 ? 8 : s);
 }
@@ -67,33 +72,51 @@ struct DqArgs {
   int* status;
 };
 
+// Two dequantized values as one fp16 pair: (f0, f1) hold 2^23 + u as fp32 bit patterns;
+// f + (-(2^23 + z)) is u - z exactly, times s rounded to nearest in fp32 (the packed fp32x2
+// intrinsics: each lane an ordinary correctly rounded operation), then rounded to nearest fp16.
+// The low half of the result is f0's value.
+__device__ __forceinline__ uint32_t dq_pair(uint32_t f0, uint32_t f1, float2 nzz, float2 ss) {
+  const float2 d = __fmul2_rn(__fadd2_rn(make_float2(__uint_as_float(f0), __uint_as_float(f1)), nzz), ss);
+  const __half2 h = __floats2half2_rn(d.x, d.y);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
 // Dequantize the 64 codes of one half row (BITS-bit LSB-first stream in `w`) into 8 swizzled
-// 16-byte chunks of the fp16 tile.
+// 16-byte chunks of the fp16 tile.  zm = 2^23 + z.
 template <int BITS>
 __device__ __forceinline__ void dq_half_row(const uint32_t* w, float s0, float zm0, float s1, float zm1, int g32,
                                             uint32_t dst_row, int r7) {
+  const float2 ss0 = make_float2(s0, s0), zz0 = make_float2(-zm0, -zm0), ss1 = make_float2(s1, s1),
+               zz1 = make_float2(-zm1, -zm1);
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
+    const bool second = g32 && c >= 4;  // columns 32..63 of the half row: the next 32-column group
+    const float2 ss = second ? ss1 : ss0, zz = second ? zz1 : zz0;
     uint32_t h2[4];
+    if (BITS == 4) {
+      // one word holds the chunk's 8 codes: the even ones in the low nibbles of its bytes, the
+      // odd ones in the high nibbles; a byte permute puts each under the exponent of 2^23
+      const uint32_t ev = w[c] & 0x0F0F0F0Fu, od = (w[c] >> 4) & 0x0F0F0F0Fu;
 #pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      float d[2];
+      for (int p = 0; p < 4; ++p)
+        h2[p] = dq_pair(__byte_perm(ev, 0x4B000000u, 0x7540u + p), __byte_perm(od, 0x4B000000u, 0x7540u + p), zz, ss);
+    } else {
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int j = 8 * c + 2 * p + e;  // column within the half row
-        constexpr uint32_t mask = (1u << BITS) - 1u;
-        const int bit = j * BITS;
-        const int wi = bit >> 5, off = bit & 31;
-        uint32_t u = w[wi] >> off;
-        if (off + BITS > 32) u |= w[wi + 1] << (32 - off);
-        u &= mask;
-        // u - z exactly: (2^23 + u) - (2^23 + z), both operands exact in fp32
-        const bool second = g32 && j >= 32;
-        const float f = __fsub_rn(__uint_as_float(0x4B000000u | u), second ? zm1 : zm0);
-        d[e] = __fmul_rn(f, second ? s1 : s0);
+      for (int p = 0; p < 4; ++p) {
+        uint32_t f[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int j = 8 * c + 2 * p + e;  // column within the half row
+          constexpr uint32_t mask = (1u << BITS) - 1u;
+          const int bit = j * BITS;
+          const int wi = bit >> 5, off = bit & 31;
+          uint32_t u = w[wi] >> off;
+          if (off + BITS > 32) u |= w[wi + 1] << (32 - off);
+          f[e] = 0x4B000000u | (u & mask);
+        }
+        h2[p] = dq_pair(f[0], f[1], zz, ss);
       }
-      const __half2 hv = __floats2half2_rn(d[0], d[1]);
-      h2[p] = *reinterpret_cast<const uint32_t*>(&hv);
     }
     const uint32_t a = dst_row + static_cast<uint32_t>(((c ^ r7) << 4));
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(h2[0]), "r"(h2[1]), "r"(h2[2]), "r"(h2[3])
@@ -101,8 +124,8 @@ __device__ __forceinline__ void dq_half_row(const uint32_t* w, float s0, float z
   }
 }
 
-template <int BITS>
-__global__ void __launch_bounds__(DQ_THREADS, 1)
+template <int BITS, int MINB>
+__global__ void __launch_bounds__(DQ_THREADS, MINB)
     dequant_gemm_kernel(const __grid_constant__ CUtensorMap codes_map, const __grid_constant__ CUtensorMap x_map,
                         DqArgs p) {
   extern __shared__ uint8_t dq_smem_raw[];

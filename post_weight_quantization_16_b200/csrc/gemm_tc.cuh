@@ -49,7 +49,14 @@ struct GtCfg {
   static constexpr int TMEM_COLS = 2 * BN;  // two accumulators
 };
 
-enum : int { GT_KLO_NONE = 0, GT_KLO_COL = 1, GT_KLO_ROW = 2 };
+// K range of an output tile: from 0, from the tile's first column or first row, or (modes
+// GT_KLO_BLK + j) over the kblk = 128 * 2^j columns of the aligned block that holds the tile's
+// first column only -- the product with a block-diagonal B of kblk x kblk blocks (tiles at
+// most kblk wide; K_HI_COL still cuts the range at the tile's last column).
+enum : int { GT_KLO_NONE = 0, GT_KLO_COL = 1, GT_KLO_ROW = 2, GT_KLO_BLK = 3, GT_KLO_BLK_LAST = 6 };
+__host__ __device__ constexpr int gt_kblk(int k_lo_mode) {
+  return k_lo_mode >= GT_KLO_BLK ? (128 << (k_lo_mode - GT_KLO_BLK)) : 0;
+}
 enum : int { GT_KHI_NONE = 0, GT_KHI_COL = 1 };
 
 struct GemmTCArgs {
@@ -121,7 +128,12 @@ __host__ __device__ inline void gt_tile_at(int M, int N, int K, int k_lo_mode, i
   int kb = 0, ke = K;
   if (k_lo_mode == GT_KLO_COL) kb = n0;
   if (k_lo_mode == GT_KLO_ROW) kb = m0;
-  if (k_hi_mode == GT_KHI_COL) ke = min(K, n0 + bn);
+  if (k_lo_mode >= GT_KLO_BLK) {
+    const int kblk = gt_kblk(k_lo_mode);
+    kb = (n0 / kblk) * kblk;
+    ke = min(K, kb + kblk);
+  }
+  if (k_hi_mode == GT_KHI_COL) ke = min(ke, n0 + bn);
   kb = (kb / GT_BK) * GT_BK;
   k_begin = kb;
   n_iters = (ke > kb) ? (ke - kb + GT_BK - 1) / GT_BK : 0;

@@ -48,12 +48,15 @@ struct gptq_ctx {
   cudaStream_t stream = nullptr;
   int64_t n = 0, m_max = 0;
   float* H = nullptr;                          // [n x n] accumulated Hessian (upper triangle until mirrored)
-  float *A_hi = nullptr, *A_lo = nullptr;      // [n x n] damped, permuted H; Schur complements
+  float *A_hi = nullptr, *A_lo = nullptr;      // [n x n] damped, permuted H; Schur complements.  After the
+                                               // factorization: Vs^T = (V blockdiag(U_SS))^T as tf32
+                                               // hi/lo in their lower triangles (vs_width = S)
   float *VT_hi = nullptr, *VT_lo = nullptr;    // [n x n] V12 blocks (upper) and T^T blocks (lower)
   float *U_hi = nullptr, *U_lo = nullptr;      // [n x n] U (upper)
   float* U32 = nullptr;                        // [n x n] U as plain fp32 (upper; read by the sweep)
   float *Ut_hi = nullptr, *Ut_lo = nullptr;    // [n x n] U^T
   float* Wq = nullptr;                         // [m_max x n] fp32 working weights
+  __half* W0h = nullptr;                       // [m_max x n] the layer's weights in sweep order (dead columns 0)
   float *Err_hi = nullptr, *Err_lo = nullptr;  // [m_max x kSuperBlock] block errors of a super-block
   float* keys = nullptr;
   uint8_t* dead = nullptr;
@@ -64,13 +67,15 @@ struct gptq_ctx {
   int64_t n_tok = 0;
   int state = ST_ACCUM;
   int mirrored = 0;           // H's lower triangle has been filled
+  bool u_complete = false;    // U holds every block (the factorization leaves the blocks no step needs)
+  int vs_width = 0;           // slab width S of the Vs held in A (0: none since the last prepare)
   int64_t chunk_tokens = 512;
   int64_t launches = 0;       // kernels launched by this context (instrumentation)
   int num_sms = 148;
   // tensor maps of whole matrices, encoded once: A-operand maps (128-row boxes) and
   // B-operand maps (256-row boxes), hi and lo
   CUtensorMap mA_A[2], mA_VT[2], mA_U[2], mA_Err[2];
-  CUtensorMap mB_U[2], mB_VT[2], mB_Ut[2];
+  CUtensorMap mB_U[2], mB_VT[2], mB_Ut[2], mB_Vb[2];
   CUtensorMap mC_Wq;  // Wq as the reduce-add target of the trailing update (32 x 32 boxes)
   cudaStream_t capture_stream = nullptr;
   cudaStream_t side_stream = nullptr;     // second branch of the captured factorization graph
@@ -223,6 +228,15 @@ void tag(gptq_ctx* c, const char* name, double flops, double bytes) {
 // lower in K-major form), r (A upper) or 0, ke = c + 1 (B upper) or K; upper_only keeps r <= c.
 double gemm_algo_flops(int M, int N, int K, int klo, int khi, int upper) {
   double total = 0.0;
+  if (klo >= GT_KLO_BLK) {  // block-diagonal B (upper-triangular blocks with K_HI_COL): the rows
+    const int kblk = gt_kblk(klo);  // above the column's block are the ones a caller reads
+    for (int col = 0; col < N; ++col) {
+      const int64_t b0 = (col / kblk) * kblk;
+      const int64_t kc = (khi == GT_KHI_COL) ? col - b0 + 1 : std::min<int64_t>(kblk, K - b0);
+      total += static_cast<double>(std::min<int64_t>(M, b0)) * static_cast<double>(kc);
+    }
+    return 2.0 * total;
+  }
   for (int col = 0; col < N; ++col) {
     const int64_t R = upper ? std::min<int64_t>(M, col + 1) : M;
     const int64_t ke = (khi == GT_KHI_COL) ? std::min<int64_t>(K, col + 1) : K;
@@ -278,15 +292,15 @@ struct TcOperand {
 };
 
 // Roles of the products gemm_tc runs (instrumentation names: kernel:role).
-enum : int { GR_V12 = 0, GR_SYRK, GR_T, GR_U12, GR_NEAR, GR_FAR, GR_TEST, GR_COUNT };
+enum : int { GR_V12 = 0, GR_SYRK, GR_T, GR_U12, GR_VB, GR_NEAR, GR_FAR, GR_TEST, GR_COUNT };
 const char* const kGemmTcNames[GR_COUNT] = {"gemm_tf32x3:factor_v12",    "gemm_tf32x3:factor_syrk",
                                             "gemm_tf32x3:factor_t",      "gemm_tf32x3:factor_u12",
-                                            "gemm_tf32x3:trailing_near", "gemm_tf32x3:trailing_far",
-                                            "gemm_tf32x3:test"};
+                                            "gemm_tf32x3:trailing_vs",   "gemm_tf32x3:trailing_near",
+                                            "gemm_tf32x3:trailing_far",  "gemm_tf32x3:test"};
 const char* const kGemmSimtNames[GR_COUNT] = {"gemm_hilo_simt:factor_v12",    "gemm_hilo_simt:factor_syrk",
                                               "gemm_hilo_simt:factor_t",      "gemm_hilo_simt:factor_u12",
-                                              "gemm_hilo_simt:trailing_near", "gemm_hilo_simt:trailing_far",
-                                              "gemm_hilo_simt:test"};
+                                              "gemm_hilo_simt:trailing_vs",   "gemm_hilo_simt:trailing_near",
+                                              "gemm_hilo_simt:trailing_far",  "gemm_hilo_simt:test"};
 
 // Products with fewer tensor-core tiles (at the narrowest tile) than this run on the CUDA
 // cores (fp32, 32 x 32 or 64 x 64 tiles).
@@ -331,6 +345,7 @@ int pick_bn(int M, int N, int K, int klo, int khi, int upper, int sms) {
   int best = 256;
   int64_t best_cost = -1;
   for (int bn : {256, 128, 64}) {
+    if (klo >= GT_KLO_BLK && bn > gt_kblk(klo)) continue;  // a tile must not span two blocks of B
     const int64_t cost = gemm_cost(M, N, K, klo, khi, upper, bn, sms);
     if (best_cost < 0 || cost < best_cost) {
       best_cost = cost;
@@ -344,6 +359,7 @@ gptq_status gemm_tc(gptq_ctx* c, int M, int N, int K, TcOperand A, TcOperand B, 
                     int khi, int upper, const TcOut& o, int chunk_stages = 1, int force_bn = 0) {
   if (M <= 0 || N <= 0) return GPTQ_OK;
   if (N % 32 || K % GT_BK) return GPTQ_ERR_ARG;
+  if (klo > GT_KLO_BLK_LAST || (klo >= GT_KLO_BLK && force_bn > gt_kblk(klo))) return GPTQ_ERR_ARG;
   const int bn = force_bn ? force_bn : pick_bn(M, N, K, klo, khi, upper, c->num_sms);
   const int tc_tiles = gt_num_tiles(M, N, upper, bn);
   if (gt_num_tiles(M, N, upper, 64) < kMinTcTiles && A.phi && B.phi) {
@@ -421,15 +437,69 @@ gptq_status gemm_tc(gptq_ctx* c, int M, int N, int K, TcOperand A, TcOperand B, 
   return GPTQ_OK;
 }
 
-// U (and U^T) of the diagonal block [o, o+h) of A, h a multiple of the 128-column leaf.
-gptq_status chol_inv(gptq_ctx* c, int o, int h) {
+// The recursion's products, for the node [o, o+h) = [o, o2) + [o2, o+h) (h1 + h2 columns).
+// A, V, T and U share the n x n index space: the node's V12 sits at rows [o, o2), columns
+// [o2, o+h) of VT (upper), T^T below the diagonal of VT, U and U^T in their own arrays.
+TcOperand fop(CUtensorMap* m, float* hi, float* lo, int n, int r0, int c0) {
+  return TcOperand{&m[0], &m[1], r0, c0, hi + static_cast<size_t>(r0) * n + c0, lo + static_cast<size_t>(r0) * n + c0, n};
+}
+float* at(float* M, int n, int r, int col) { return M + static_cast<size_t>(r) * n + col; }
+
+// T^T = (V12 U22)^T into the lower block [o2.., o..]   (Ut22 rows as B; k <= column)
+gptq_status t_product(gptq_ctx* c, int o, int o2, int h1, int h2) {
+  const int n = static_cast<int>(c->n);
+  TcOut tt;
+  tt.Cthi = at(c->VT_hi, n, o2, o);
+  tt.Ctlo = at(c->VT_lo, n, o2, o);
+  tt.ldt = n;
+  c->gemm_role = GR_T;
+  return gemm_tc(c, h1, h2, h2, fop(c->mA_VT, c->VT_hi, c->VT_lo, n, o, o2), fop(c->mB_Ut, c->Ut_hi, c->Ut_lo, n, o2, o2),
+                 1.f, 0, GT_KLO_NONE, GT_KHI_COL, 0, tt);
+}
+
+// U12 = -U11 T  (and Ut21 = U12^T)      (U11 rows as A; k >= row)
+gptq_status u12_product(gptq_ctx* c, int o, int o2, int h1, int h2) {
+  const int n = static_cast<int>(c->n);
+  TcOut u12;
+  u12.C = at(c->U32, n, o, o2);
+  u12.ldc = n;
+  u12.Chi = at(c->U_hi, n, o, o2);
+  u12.Clo = at(c->U_lo, n, o, o2);
+  u12.ldh = n;
+  u12.Cthi = at(c->Ut_hi, n, o2, o);
+  u12.Ctlo = at(c->Ut_lo, n, o2, o);
+  u12.ldt = n;
+  c->gemm_role = GR_U12;
+  return gemm_tc(c, h1, h2, h1, fop(c->mA_U, c->U_hi, c->U_lo, n, o, o), fop(c->mB_VT, c->VT_hi, c->VT_lo, n, o2, o),
+                 -1.f, 0, GT_KLO_ROW, GT_KHI_NONE, 0, u12);
+}
+
+// Width of the left part of a node of h columns: half the leaves; on the recursion's left edge
+// (need_u false) a multiple of kSuperBlock, so that every aligned slab of up to kSuperBlock
+// columns lies inside one node whose U is computed in full.
+int split_left(int h, bool need_u) {
+  if (need_u) return h - ((h / LF_NB) / 2) * LF_NB;
+  const int h1 = ((h / 2 + kSuperBlock / 2) / kSuperBlock) * kSuperBlock;
+  return std::min(std::max(h1, kSuperBlock), h - LF_NB);
+}
+
+// The reverse-ordered Cholesky factor V (H = V V^T, V upper) of the diagonal block [o, o+h) of
+// A, h a multiple of the 128-column leaf, and U = V^-1 of that block when need_u:
+//   V22 = f(A22); V12 = A12 U22^T; A11 -= V12 V12^T; V11 = f(A11); U12 = -U11 V12 U22.
+// Every V12 needs the whole U of its node's right part, so right parts are inverted in full;
+// the nodes wider than kSuperBlock on the left edge of the recursion (the root, its left
+// part, ...) skip T and U12.  The sweep reads V and the diagonal slab blocks of U only (its
+// errors satisfy E U = W0 - Q, so the errors of the columns before a slab reach it as
+// (W0 - Q) V[., slab] U[slab, slab], see quantize); gptq_get_factor computes the skipped
+// blocks when asked (complete_factor).
+gptq_status chol_inv(gptq_ctx* c, int o, int h, bool need_u) {
   const int n = static_cast<int>(c->n);
   if (h <= LF_NB) {
     tag(c, "leaf_chol_inv", 2.0 * LF_NB * LF_NB * LF_NB / 3.0, 4.0 * LF_NB * LF_NB * 4);
     CK(launch(c, leaf_chol_inv_kernel, dim3(1), dim3(LF_THREADS), LF_SMEM, c->A_hi, c->A_lo, n, o, c->U_hi, c->U_lo,
               c->U32, c->status));
     CKL("leaf_chol_inv");
-    // U^T of the block, needed only by later T products and the sweep's trailing update: on
+    // U^T of the block, needed only by later T products and the block-diagonal product Vb: on
     // the second branch while it exists (the factorization graph), in line otherwise
     const bool branch = c->side_stream != nullptr;
     cudaStream_t main_stream = c->stream;
@@ -450,41 +520,32 @@ gptq_status chol_inv(gptq_ctx* c, int o, int h) {
     CKL("transpose_block");
     return GPTQ_OK;
   }
-  const int h2 = ((h / LF_NB) / 2) * LF_NB;
-  const int h1 = h - h2;
+  if (h <= kSuperBlock) need_u = true;
+  const int h1 = split_left(h, need_u), h2 = h - h1;
   const int o2 = o + h1;
-  auto at = [n](float* M, int r, int col) { return M + static_cast<size_t>(r) * n + col; };
   gptq_status s;
-  if ((s = chol_inv(c, o2, h2)) != GPTQ_OK) return s;
-  auto op = [n](CUtensorMap* m, float* hi, float* lo, int r0, int c0) {
-    return TcOperand{&m[0], &m[1], r0, c0, hi + static_cast<size_t>(r0) * n + c0, lo + static_cast<size_t>(r0) * n + c0,
-                     n};
-  };
+  if ((s = chol_inv(c, o2, h2, true)) != GPTQ_OK) return s;
   // V12 = A12 U22^T                      (U22 rows are the K-major B; k >= column)
   TcOut v12;
-  v12.Chi = at(c->VT_hi, o, o2);
-  v12.Clo = at(c->VT_lo, o, o2);
+  v12.Chi = at(c->VT_hi, n, o, o2);
+  v12.Clo = at(c->VT_lo, n, o, o2);
   v12.ldh = n;
   c->gemm_role = GR_V12;
-  if ((s = gemm_tc(c, h1, h2, h2, op(c->mA_A, c->A_hi, c->A_lo, o, o2), op(c->mB_U, c->U_hi, c->U_lo, o2, o2), 1.f, 0, GT_KLO_COL, GT_KHI_NONE, 0,
-                   v12)) != GPTQ_OK)
+  if ((s = gemm_tc(c, h1, h2, h2, fop(c->mA_A, c->A_hi, c->A_lo, n, o, o2), fop(c->mB_U, c->U_hi, c->U_lo, n, o2, o2),
+                   1.f, 0, GT_KLO_COL, GT_KHI_NONE, 0, v12)) != GPTQ_OK)
     return s;
   // A11 -= V12 V12^T                     (upper tiles only)
   TcOut a11;
-  a11.Chi = at(c->A_hi, o, o);
-  a11.Clo = at(c->A_lo, o, o);
+  a11.Chi = at(c->A_hi, n, o, o);
+  a11.Clo = at(c->A_lo, n, o, o);
   a11.ldh = n;
   c->gemm_role = GR_SYRK;
-  if ((s = gemm_tc(c, h1, h1, h2, op(c->mA_VT, c->VT_hi, c->VT_lo, o, o2), op(c->mB_VT, c->VT_hi, c->VT_lo, o, o2), -1.f, 1, GT_KLO_NONE, GT_KHI_NONE, 1,
-                   a11)) != GPTQ_OK)
+  if ((s = gemm_tc(c, h1, h1, h2, fop(c->mA_VT, c->VT_hi, c->VT_lo, n, o, o2), fop(c->mB_VT, c->VT_hi, c->VT_lo, n, o, o2),
+                   -1.f, 1, GT_KLO_NONE, GT_KHI_NONE, 1, a11)) != GPTQ_OK)
     return s;
-  // T^T = (V12 U22)^T into the lower block [o2.., o..]   (Ut22 rows as B; k <= column).
-  // Only U12 below needs it, so while the graph is being captured it runs on a second
+  if (!need_u) return chol_inv(c, o, h1, false);
+  // T is needed only by U12 below, so while the graph is being captured it runs on a second
   // branch, beside the factorization of A11 (which touches only [o, o+h1)^2).
-  TcOut tt;
-  tt.Cthi = at(c->VT_hi, o2, o);
-  tt.Ctlo = at(c->VT_lo, o2, o);
-  tt.ldt = n;
   const bool branch = c->side_stream != nullptr;
   cudaStream_t main_stream = c->stream;
   if (branch) {
@@ -493,32 +554,51 @@ gptq_status chol_inv(gptq_ctx* c, int o, int h) {
     c->stream = c->side_stream;
     c->pdl = false;
   }
-  c->gemm_role = GR_T;
-  s = gemm_tc(c, h1, h2, h2, op(c->mA_VT, c->VT_hi, c->VT_lo, o, o2), op(c->mB_Ut, c->Ut_hi, c->Ut_lo, o2, o2), 1.f, 0,
-              GT_KLO_NONE, GT_KHI_COL, 0, tt);
+  s = t_product(c, o, o2, h1, h2);
   if (branch) {
     c->stream = main_stream;
     c->pdl = true;
     if (s == GPTQ_OK) CK(cudaEventRecord(c->ev_join, c->side_stream));
   }
   if (s != GPTQ_OK) return s;
-  if ((s = chol_inv(c, o, h1)) != GPTQ_OK) return s;
+  if ((s = chol_inv(c, o, h1, true)) != GPTQ_OK) return s;
   // the join: the latest T on the branch (branch launches are in order, so this one too)
   if (branch) CK(cudaStreamWaitEvent(main_stream, c->ev_join, 0));
-  // U12 = -U11 T  (and Ut21 = U12^T)      (U11 rows as A; k >= row)
-  TcOut u12;
-  u12.C = at(c->U32, o, o2);
-  u12.ldc = n;
-  u12.Chi = at(c->U_hi, o, o2);
-  u12.Clo = at(c->U_lo, o, o2);
-  u12.ldh = n;
-  u12.Cthi = at(c->Ut_hi, o2, o);
-  u12.Ctlo = at(c->Ut_lo, o2, o);
-  u12.ldt = n;
-  c->gemm_role = GR_U12;
-  if ((s = gemm_tc(c, h1, h2, h1, op(c->mA_U, c->U_hi, c->U_lo, o, o), op(c->mB_VT, c->VT_hi, c->VT_lo, o2, o), -1.f, 0, GT_KLO_ROW, GT_KHI_NONE, 0,
-                   u12)) != GPTQ_OK)
-    return s;
+  return u12_product(c, o, o2, h1, h2);
+}
+
+// Vs = V blockdiag(U_SS) for slabs of S columns: every aligned S-column block of V above the
+// diagonal times the U block of its columns, in one launch (block-diagonal K ranges), written
+// transposed as tf32 hi/lo into the lower triangles of A_hi and A_lo (the K-major operand of
+// the product past a slab).  Tiles on the diagonal compute values nothing reads.
+gptq_status vs_product(gptq_ctx* c, int S) {
+  const int n = static_cast<int>(c->n);
+  int mode = GT_KLO_BLK;
+  while (gt_kblk(mode) < S) ++mode;
+  if (gt_kblk(mode) != S || mode > GT_KLO_BLK_LAST) return GPTQ_ERR_ARG;
+  TcOut vo;
+  vo.Cthi = c->A_hi;
+  vo.Ctlo = c->A_lo;
+  vo.ldt = n;
+  c->gemm_role = GR_VB;
+  // the tile width is fixed (the widest that fits a block): this product is launched from the
+  // quantize call, where simulating its many uneven tiles on the host would leave the GPU idle
+  return gemm_tc(c, n, n, n, fop(c->mA_VT, c->VT_hi, c->VT_lo, n, 0, 0), fop(c->mB_Ut, c->Ut_hi, c->Ut_lo, n, 0, 0),
+                 1.f, 0, mode, GT_KHI_COL, 1, vo, 1, S >= 256 ? 256 : 128);
+}
+
+// The U blocks the factorization leaves out: T and U12 of the nodes on the recursion's left
+// edge, smallest first (each U12 needs the complete U of its left part).
+gptq_status complete_factor(gptq_ctx* c) {
+  const int n = static_cast<int>(c->n);
+  std::vector<int> hs;
+  for (int h = n; h > kSuperBlock; h = split_left(h, false)) hs.push_back(h);
+  for (auto it = hs.rbegin(); it != hs.rend(); ++it) {
+    const int h = *it, h1 = split_left(h, false), h2 = h - h1;
+    gptq_status s;
+    if ((s = t_product(c, 0, h1, h1, h2)) != GPTQ_OK) return s;
+    if ((s = u12_product(c, 0, h1, h1, h2)) != GPTQ_OK) return s;
+  }
   return GPTQ_OK;
 }
 
@@ -540,6 +620,7 @@ gptq_status encode_maps(gptq_ctx* c) {
       {&c->mB_U[0], c->U_hi, n, n, n, GT_BOX_N},        {&c->mB_U[1], c->U_lo, n, n, n, GT_BOX_N},
       {&c->mB_VT[0], c->VT_hi, n, n, n, GT_BOX_N},      {&c->mB_VT[1], c->VT_lo, n, n, n, GT_BOX_N},
       {&c->mB_Ut[0], c->Ut_hi, n, n, n, GT_BOX_N},      {&c->mB_Ut[1], c->Ut_lo, n, n, n, GT_BOX_N},
+      {&c->mB_Vb[0], c->A_hi, n, n, n, GT_BOX_N},       {&c->mB_Vb[1], c->A_lo, n, n, n, GT_BOX_N},
       {&c->mC_Wq, c->Wq, c->m_max, n, n, 32},
   };
   for (auto& e : list)
@@ -553,7 +634,7 @@ gptq_status run_factorization(gptq_ctx* c) {
   if (c->prof) {  // instrumented: every launch on its own, timed, on the context's stream
     cudaStream_t side = c->side_stream;
     c->side_stream = nullptr;
-    const gptq_status s = chol_inv(c, 0, static_cast<int>(c->n));
+    const gptq_status s = chol_inv(c, 0, static_cast<int>(c->n), false);
     c->side_stream = side;
     return s;
   }
@@ -566,7 +647,7 @@ gptq_status run_factorization(gptq_ctx* c) {
     const int64_t l0 = c->launches;
     c->stream = c->capture_stream;
     CK(cudaStreamBeginCapture(c->capture_stream, cudaStreamCaptureModeThreadLocal));
-    gptq_status s = chol_inv(c, 0, static_cast<int>(c->n));
+    gptq_status s = chol_inv(c, 0, static_cast<int>(c->n), false);
     if (s == GPTQ_OK) {  // join the second branch (the last block's U^T)
       cudaError_t e1 = cudaEventRecord(c->ev_join, c->side_stream);
       if (e1 == cudaSuccess) e1 = cudaStreamWaitEvent(c->capture_stream, c->ev_join, 0);
@@ -634,6 +715,8 @@ void free_all(gptq_ctx* c) {
       cudaFree(*p);
       *p = nullptr;
     }
+  if (c->W0h) cudaFree(c->W0h);
+  c->W0h = nullptr;
   if (c->dead) cudaFree(c->dead);
   if (c->perm) cudaFree(c->perm);
   if (c->mean) cudaFree(c->mean);
@@ -677,7 +760,7 @@ size_t gptq_workspace_bytes(int64_t n, int64_t m_max) {
   if (n < 128 || n > kMaxN || n % 128 || m_max < 1 || m_max > kMaxM) return 0;
   const size_t nn = static_cast<size_t>(n) * static_cast<size_t>(n);
   size_t b = 10 * nn * sizeof(float);                                             // H, A, VT, U, Ut (hi/lo), U
-  b += static_cast<size_t>(m_max) * static_cast<size_t>(n) * sizeof(float);       // Wq
+  b += static_cast<size_t>(m_max) * static_cast<size_t>(n) * (sizeof(float) + 2);   // Wq, W0h
   b += 2 * static_cast<size_t>(m_max) * kSuperBlock * sizeof(float);              // Err hi/lo
   b += static_cast<size_t>(n) * (sizeof(float) + 1 + sizeof(int32_t)) + sizeof(double) + sizeof(int);
   return b;
@@ -721,6 +804,7 @@ gptq_status gptq_create(gptq_ctx** out, int64_t n, int64_t m_max, int device, vo
   for (float** p : {&c->A_hi, &c->A_lo, &c->VT_hi, &c->VT_lo, &c->U_hi, &c->U_lo, &c->U32, &c->Ut_hi, &c->Ut_lo})
     alloc(reinterpret_cast<void**>(p), nn * 4);
   alloc(reinterpret_cast<void**>(&c->Wq), static_cast<size_t>(m_max) * n * 4);
+  alloc(reinterpret_cast<void**>(&c->W0h), static_cast<size_t>(m_max) * n * 2);
   alloc(reinterpret_cast<void**>(&c->Err_hi), static_cast<size_t>(m_max) * kSuperBlock * 4);
   alloc(reinterpret_cast<void**>(&c->Err_lo), static_cast<size_t>(m_max) * kSuperBlock * 4);
   alloc(reinterpret_cast<void**>(&c->keys), n * 4);
@@ -869,6 +953,8 @@ gptq_status gptq_prepare(gptq_ctx* c, double damp, int desc_act, int32_t* perm_o
   const size_t nn = static_cast<size_t>(n) * n;
   for (float* p : {c->U_hi, c->U_lo, c->U32, c->Ut_hi, c->Ut_lo}) CK(cudaMemsetAsync(p, 0, nn * 4, c->stream));
   if ((s = run_factorization(c)) != GPTQ_OK) return s;
+  c->u_complete = n <= kSuperBlock;
+  c->vs_width = 0;
   if (perm_out) CK(cudaMemcpyAsync(perm_out, c->perm, n * 4, cudaMemcpyDeviceToDevice, c->stream));
   int flags = 0;
   if ((s = read_status(c, &flags)) != GPTQ_OK) return s;
@@ -881,6 +967,11 @@ gptq_status gptq_get_factor(gptq_ctx* c, float* U_out) {
   if (!c || !U_out) return GPTQ_ERR_ARG;
   if (c->state != ST_PREPARED) return GPTQ_ERR_STATE;
   DeviceGuard dg(c->device);
+  if (!c->u_complete) {
+    gptq_status s;
+    if ((s = complete_factor(c)) != GPTQ_OK) return s;
+    c->u_complete = true;
+  }
   const size_t nn = static_cast<size_t>(c->n) * c->n;
   CK(cudaMemcpyAsync(U_out, c->U32, nn * 4, cudaMemcpyDeviceToDevice, c->stream));
   return GPTQ_OK;
@@ -954,14 +1045,15 @@ gptq_status gptq_quantize_layer(gptq_ctx* c, const void* W, int64_t m, gptq_qpar
   const int n = static_cast<int>(c->n);
   const int mi = static_cast<int>(m);
   const int g = (qp.group_size == -1) ? n : qp.group_size;
-  tag(c, "quantize:init_w", 0.0, 6.0 * static_cast<double>(m) * n);
-  CK(launch(c, init_w_kernel, dim3(mi), dim3(256), static_cast<size_t>(n) * 2, static_cast<const __half*>(W), n, c->perm, c->dead,
-                                                                   c->Wq));
+  tag(c, "quantize:init_w", 0.0, 8.0 * static_cast<double>(m) * n);
+  CK(launch(c, init_w_kernel, dim3(mi), dim3(256), static_cast<size_t>(n) * 2, static_cast<const __half*>(W), n, c->perm,
+            c->dead, c->Wq, c->W0h));
   CKL("init_w");
   SweepArgs a;
   a.Wq = c->Wq;
   a.U = c->U32;
   a.U_lo = nullptr;
+  a.W0 = c->W0h;
   a.Err = c->Err_hi;
   a.Err_lo = c->Err_lo;
   a.codes = codes;
@@ -978,22 +1070,52 @@ gptq_status gptq_quantize_layer(gptq_ctx* c, const void* W, int64_t m, gptq_qpar
   a.ld_err = kSuperBlock;
   a.err_col0 = 0;
   const int grid = (mi + SW_ROWS - 1) / SW_ROWS;
-  // Two-level lazy update: inside a super-block of columns the slab kernel applies each block's
-  // errors to the later columns itself; the columns beyond the super-block receive all its
-  // block errors in one tensor-core product (K = super-block width).  A group that starts
-  // inside a super-block must not reach past it; other group widths use 128-column super-blocks.
-  // slab width: slab_default(n), or GPTQ_SLAB_WIDTH (a multiple of 128 up to kSuperBlock) for tuning
+  // Two-level lazy update.  Inside a super-block of columns (the slab) the slab kernel carries
+  // every column's error forward itself; the columns beyond the slab receive the slab's
+  // contribution in one tensor-core product (K = slab width).  The sweep's errors satisfy
+  // E U = W0 - Q column by column (W0 the original weights, Q their dequantized values), so the
+  // errors of all columns before a slab reach it as -E U[., slab] = D V[., slab] U[slab, slab]
+  // with D = W0 - Q.  That product is taken in this form, D Vs with Vs = V blockdiag(U_SS)
+  // (computed once per prepared factor and slab width): the factorization then needs U only
+  // inside the aligned slab blocks.  The slab's columns are exact once every earlier slab is
+  // in, not before, so every group must start and end inside one slab (or be the whole row).
+  // Group widths that cannot (wider than kSuperBlock, or not dividing a power-of-two slab)
+  // take the form -E U[slab, rest] instead, on the completed U, which also lets groups reach
+  // past a slab.  Slab width: slab_default(n), or GPTQ_SLAB_WIDTH (a multiple of 128 up to
+  // kSuperBlock) for tuning.
   const int slab = static_cast<int>(
       std::min<int64_t>(kSuperBlock, std::max<int64_t>(SW_B, env_int("GPTQ_SLAB_WIDTH", slab_default(n)) / SW_B * SW_B)));
-  const int sb = ((g <= slab && slab % g == 0) || g % slab == 0 || g == n) ? slab : SW_B;
+  int sd = SW_B;  // the widest power-of-two multiple of 128 up to the slab width
+  while (sd * 2 <= slab) sd *= 2;
+  const bool g_pow2 = g >= SW_B && g <= kSuperBlock && (g & (g - 1)) == 0;
+  if (g_pow2 && g > sd) sd = g;
+  const bool d_form = g < SW_B || g == n || g_pow2;
+  int sb;
+  if (d_form) {
+    sb = sd;
+    if (c->vs_width != sb) {
+      gptq_status st;
+      if ((st = vs_product(c, sb)) != GPTQ_OK) return st;
+      c->vs_width = sb;
+    }
+  } else {
+    sb = ((g <= slab && slab % g == 0) || g % slab == 0) ? slab : SW_B;
+    if (!c->u_complete) {
+      gptq_status st;
+      if ((st = complete_factor(c)) != GPTQ_OK) return st;
+      c->u_complete = true;
+    }
+  }
+  a.d_form = d_form ? 1 : 0;
   for (int s0 = 0; s0 < n; s0 += sb) {
     const int s1 = std::min(n, s0 + sb);
     const double S = static_cast<double>(s1 - s0);
-    // algorithmic bytes: the slab in, its scaled errors out (hi/lo), codes, scales/zeros of its
-    // groups, its U blocks, the dequantized weights when asked for
+    // algorithmic bytes: the slab in, its original weights (d form), its D or errors out
+    // (hi/lo) when a product follows, codes, scales/zeros of its groups, the upper half of its
+    // U block, the dequantized weights when asked for
     tag(c, "sweep_slab", 0.0,
-        4.0 * mi * S + 8.0 * mi * S + mi * S * qp.bits / 8.0 + 8.0 * mi * std::max(1.0, S / g) + 4.0 * SW_B * S +
-            (W_hat ? 4.0 * mi * S : 0.0));
+        4.0 * mi * S + (s1 < n ? (d_form ? 10.0 : 8.0) * mi * S : 0.0) + mi * S * qp.bits / 8.0 +
+            8.0 * mi * std::max(1.0, S / g) + 2.0 * S * S + (W_hat ? 4.0 * mi * S : 0.0));
     const size_t smem = static_cast<size_t>(ss_smem_bytes(s1 - s0));
     if (g >= SW_B)
       CK(launch(c, sweep_slab_kernel<0>, dim3(grid), dim3(SS_THREADS), smem, a, s0, s1));
@@ -1003,16 +1125,18 @@ gptq_status gptq_quantize_layer(gptq_ctx* c, const void* W, int64_t m, gptq_qpar
       CK(launch(c, sweep_slab_kernel<32>, dim3(grid), dim3(SS_THREADS), smem, a, s0, s1));
     CKL("sweep_slab");
     if (s1 < n) {
-      // W[:, s1:] -= Err_super * U[s0:s1, s1:]   (K = s1 - s0; 128-wide TMEM chunks)
+      // W[:, s1:] += D_slab Vs[s0:s1, s1:], or -= E_slab U[s0:s1, s1:]   (K = s1 - s0; 128-wide
+      // TMEM chunks)
       TcOut w;
       w.C = c->Wq + s1;
       w.ldc = n;
       w.c_map = &c->mC_Wq;
       w.c_col0 = s1;
       c->gemm_role = GR_FAR;
+      const TcOperand B = d_form ? TcOperand{&c->mB_Vb[0], &c->mB_Vb[1], s1, s0, nullptr, nullptr, 0}
+                                 : TcOperand{&c->mB_Ut[0], &c->mB_Ut[1], s1, s0, nullptr, nullptr, 0};
       gptq_status st = gemm_tc(c, mi, n - s1, s1 - s0, TcOperand{&c->mA_Err[0], &c->mA_Err[1], 0, 0, nullptr, nullptr, 0},
-                               TcOperand{&c->mB_Ut[0], &c->mB_Ut[1], s1, s0, nullptr, nullptr, 0}, -1.f, 1,
-                               GT_KLO_NONE, GT_KHI_NONE, 0, w, SW_B / GT_BK);
+                               B, d_form ? 1.f : -1.f, 1, GT_KLO_NONE, GT_KHI_NONE, 0, w, SW_B / GT_BK);
       if (st != GPTQ_OK) return st;
     }
   }
@@ -1054,7 +1178,7 @@ gptq_status gptq_test_gemm_tf32x3(int M, int N, int K, const float* A_hi, const 
   if (c_reduce && (!C || beta != 1)) return GPTQ_ERR_ARG;
   if (tile_n != 0 && tile_n != 64 && tile_n != 128 && tile_n != 256) return GPTQ_ERR_ARG;
   if (!A_hi || !A_lo || !B_hi || !B_lo || M < 1 || N < 1 || K < GT_BK) return GPTQ_ERR_ARG;
-  if (k_lo_mode < 0 || k_lo_mode > 2 || k_hi_mode < 0 || k_hi_mode > 1 || (beta != 0 && beta != 1)) return GPTQ_ERR_ARG;
+  if (k_lo_mode < 0 || k_lo_mode > GT_KLO_BLK_LAST || k_hi_mode < 0 || k_hi_mode > 1 || (beta != 0 && beta != 1)) return GPTQ_ERR_ARG;
   if ((C_hi == nullptr) != (C_lo == nullptr) || (Ct_hi == nullptr) != (Ct_lo == nullptr)) return GPTQ_ERR_ARG;
   if ((C && (!aligned16(C) || ldc % 4)) || (C_hi && (!aligned16(C_hi) || !aligned16(C_lo) || ldh % 4)))
     return GPTQ_ERR_ARG;
@@ -1264,12 +1388,14 @@ extern "C" gptq_status gptq_quantize_layer_noalloc(const void* W, int64_t m, int
   float* Wq = scratch;                       // [m x n]
   float* Err = scratch + kNoAllocMaxWeights; // [m x 128]
   init_w_kernel<<<mi, 256, static_cast<size_t>(ni) * 2, st>>>(static_cast<const __half*>(W), ni, perm,
-                                                             dead ? dead : nodead, Wq);
+                                                             dead ? dead : nodead, Wq, nullptr);
   CKL("noalloc init_w");
   SweepArgs a;
   a.Wq = Wq;
   a.U = U;
   a.U_lo = nullptr;
+  a.W0 = nullptr;
+  a.d_form = 0;
   a.Err = Err;
   a.Err_lo = nullptr;
   a.ld_err = SW_B;
@@ -1331,7 +1457,9 @@ bool dq_plan(int64_t T, int64_t m, int64_t n, int act_order, DqPlan* p) {
   p->tiles_t = static_cast<int>((T + p->tn - 1) / p->tn);
   p->k_tiles = static_cast<int>(n / DQ_BK);
   const int64_t base = static_cast<int64_t>(p->tiles_m) * p->tiles_t;
-  int splits = base >= kDqPlanSms ? 1 : static_cast<int>(std::min<int64_t>(p->k_tiles, kDqPlanSms / base));
+  // fill every SM (two CTAs each when the tile is decode-sized, see dq_minb) with K splits
+  const int64_t target = kDqPlanSms * (p->tn <= 32 ? 2 : 1);
+  int splits = base >= target ? 1 : static_cast<int>(std::min<int64_t>(p->k_tiles, target / base));
   splits = std::max(1, splits);
   p->k_per = (p->k_tiles + splits - 1) / splits;
   p->splits = (p->k_tiles + p->k_per - 1) / p->k_per;
@@ -1348,7 +1476,7 @@ bool dq_plan(int64_t T, int64_t m, int64_t n, int act_order, DqPlan* p) {
 // Raise a kernel's dynamic shared-memory limit once per device (later calls, which may be
 // recorded into a graph, then make no attribute call).
 std::mutex g_attr_mu;
-int g_attr_smem[kMaxDevicesAttr][8] = {};
+int g_attr_smem[kMaxDevicesAttr][12] = {};
 
 template <typename K>
 cudaError_t ensure_smem_attr(int device, int slot, K kernel, int smem) {
@@ -1438,22 +1566,38 @@ extern "C" gptq_status gptq_dequant_matmul(const void* X, int64_t T, const uint3
   a.status = status;
   const int smem = dq_smem_bytes(pl.tn, bits);
   const dim3 grid(pl.tiles_m, pl.tiles_t, pl.splits);
+  const bool two = dq_minb(pl.tn, bits) == 2;
   switch (bits) {
     case 2:
-      CK(ensure_smem_attr(device, 0, dequant_gemm_kernel<2>, smem));
-      dequant_gemm_kernel<2><<<grid, DQ_THREADS, smem, st>>>(cmap, xmap, a);
+      if (two) {
+        CK(ensure_smem_attr(device, 0, dequant_gemm_kernel<2, 2>, smem));
+        dequant_gemm_kernel<2, 2><<<grid, DQ_THREADS, smem, st>>>(cmap, xmap, a);
+      } else {
+        CK(ensure_smem_attr(device, 8, dequant_gemm_kernel<2, 1>, smem));
+        dequant_gemm_kernel<2, 1><<<grid, DQ_THREADS, smem, st>>>(cmap, xmap, a);
+      }
       break;
     case 3:
-      CK(ensure_smem_attr(device, 1, dequant_gemm_kernel<3>, smem));
-      dequant_gemm_kernel<3><<<grid, DQ_THREADS, smem, st>>>(cmap, xmap, a);
+      if (two) {
+        CK(ensure_smem_attr(device, 1, dequant_gemm_kernel<3, 2>, smem));
+        dequant_gemm_kernel<3, 2><<<grid, DQ_THREADS, smem, st>>>(cmap, xmap, a);
+      } else {
+        CK(ensure_smem_attr(device, 9, dequant_gemm_kernel<3, 1>, smem));
+        dequant_gemm_kernel<3, 1><<<grid, DQ_THREADS, smem, st>>>(cmap, xmap, a);
+      }
       break;
     case 4:
-      CK(ensure_smem_attr(device, 2, dequant_gemm_kernel<4>, smem));
-      dequant_gemm_kernel<4><<<grid, DQ_THREADS, smem, st>>>(cmap, xmap, a);
+      if (two) {
+        CK(ensure_smem_attr(device, 2, dequant_gemm_kernel<4, 2>, smem));
+        dequant_gemm_kernel<4, 2><<<grid, DQ_THREADS, smem, st>>>(cmap, xmap, a);
+      } else {
+        CK(ensure_smem_attr(device, 10, dequant_gemm_kernel<4, 1>, smem));
+        dequant_gemm_kernel<4, 1><<<grid, DQ_THREADS, smem, st>>>(cmap, xmap, a);
+      }
       break;
     default:
-      CK(ensure_smem_attr(device, 3, dequant_gemm_kernel<8>, smem));
-      dequant_gemm_kernel<8><<<grid, DQ_THREADS, smem, st>>>(cmap, xmap, a);
+      CK(ensure_smem_attr(device, 3, dequant_gemm_kernel<8, 1>, smem));
+      dequant_gemm_kernel<8, 1><<<grid, DQ_THREADS, smem, st>>>(cmap, xmap, a);
       break;
   }
   CKL("dequant_gemm");

@@ -129,9 +129,10 @@ __global__ void __launch_bounds__(GD_THREADS) gather_damp_kernel(const float* __
   }
 }
 
-// One CTA per row r: Wq[r][k] = dead[perm[k]] ? 0 : float(W[r][perm[k]]).
+// One CTA per row r: Wq[r][k] = dead[perm[k]] ? 0 : float(W[r][perm[k]]), and the same weights
+// kept in fp16 (exact) in W0h when it is given.
 __global__ void init_w_kernel(const __half* __restrict__ W, int n, const int32_t* __restrict__ perm,
-                              const uint8_t* __restrict__ dead, float* __restrict__ Wq) {
+                              const uint8_t* __restrict__ dead, float* __restrict__ Wq, __half* __restrict__ W0h) {
   griddep_wait();
   griddep_launch_dependents();
   extern __shared__ __half wrow_s[];
@@ -140,9 +141,12 @@ __global__ void init_w_kernel(const __half* __restrict__ W, int n, const int32_t
   for (int k = threadIdx.x; k < n; k += blockDim.x) wrow_s[k] = src[k];
   __syncthreads();
   float* dst = Wq + static_cast<size_t>(r) * n;
+  __half* dst0 = W0h ? W0h + static_cast<size_t>(r) * n : nullptr;
   for (int k = threadIdx.x; k < n; k += blockDim.x) {
     const int p = perm[k];
-    dst[k] = dead[p] ? 0.0f : __half2float(wrow_s[p]);
+    const __half w = dead[p] ? __float2half_rn(0.0f) : wrow_s[p];
+    dst[k] = __half2float(w);
+    if (dst0) dst0[k] = w;
   }
 }
 

@@ -207,7 +207,12 @@ __global__ void __launch_bounds__(GS_THREADS) gemm_hilo_simt_kernel(GemmSimtArgs
   int kb = 0, ke = p.K;
   if (p.k_lo_mode == 1) kb = n0;
   if (p.k_lo_mode == 2) kb = m0;
-  if (p.k_hi_mode == 1) ke = min(p.K, n0 + TN);
+  if (p.k_lo_mode >= 3) {  // the aligned block of 128 << (mode - 3) columns of the tile (block-diagonal B)
+    const int kblk = 128 << (p.k_lo_mode - 3);
+    kb = (n0 / kblk) * kblk;
+    ke = min(p.K, kb + kblk);
+  }
+  if (p.k_hi_mode == 1) ke = min(ke, n0 + TN);
   kb = (kb / GS_BK) * GS_BK;
   const int nk = (ke > kb) ? (ke - kb + GS_BK - 1) / GS_BK : 0;
 

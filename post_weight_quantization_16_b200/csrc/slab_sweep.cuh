@@ -19,8 +19,13 @@
 //     every later column of the slab (a lane per four columns, their 16 U values loaded once,
 //     coalesced across the warp, and used for all 32 rows; the errors read as shared-memory
 //     broadcasts), in fp32 fused multiply-adds;
-//   * the block's scaled errors go out as tf32 hi/lo pairs for the one product that updates
-//     the columns beyond the super-block, and its codes are packed.
+//   * for the one product that updates the columns beyond the super-block the block's columns
+//     go out as tf32 hi/lo pairs: d = w0 - q (original weight minus dequantized value), or
+//     with d_form = 0 the scaled errors e; and its codes are packed.
+// The two forms of that product carry the same compensation: the sweep's errors satisfy
+// E U = W0 - Q, so the errors of every column before a super-block reach it as
+// -E U[., sb] = (W0 - Q) V[., sb] U[sb, sb] (V = U^-1), which needs only the diagonal
+// super-block of U; it holds for the super-block as a whole, once every earlier column is in.
 // So the per-block product on the later columns of the super-block, and its launch, leave the
 // critical path: within a super-block the updates run beside the walker on the same SM.
 #pragma once
@@ -36,10 +41,11 @@ constexpr int SS_NW = SS_THREADS / 32;
 constexpr int SS_MAXW = 1024;              // widest slab (columns)
 // slab pitch (floats) for a slab of S columns: lane-per-row float4 access without conflicts
 __host__ __device__ constexpr int ss_wld(int S) { return S + 4; }
-// U block | slab | errors | the chunk's errors (compact) | 1/U[i][i] | perm | group partials | codes
+// U block | slab | errors | the chunk's errors (compact) | 1/U[i][i] | perm | group partials | codes |
+// the block's group parameters (s, and the zero-point inside the rounding, per row and group)
 __host__ __device__ constexpr int ss_smem_bytes(int S) {
   return SW_B * SW_B * 4 + SW_ROWS * ss_wld(S) * 4 + SW_ROWS * SW_ELD * 4 + 2 * SW_ROWS * SW_CH * 4 + SW_B * 4 +
-         SW_B * 4 + 3 * SS_NW * SW_ROWS * 4 + SW_ROWS * SW_CLD;
+         SW_B * 4 + 3 * SS_NW * SW_ROWS * 4 + SW_ROWS * SW_CLD + 2 * SW_ROWS * 4 * 4;
 }
 constexpr int SS_SMEM = ss_smem_bytes(SS_MAXW);
 
@@ -69,6 +75,8 @@ __global__ void __launch_bounds__(SS_THREADS, 1) sweep_slab_kernel(SweepArgs a, 
   int* perm_s = reinterpret_cast<int*>(rU + SW_B);        // [128]
   float* part = reinterpret_cast<float*>(perm_s + SW_B);  // [3][8][32] group min / max / max|.| partials
   uint8_t* codes8 = reinterpret_cast<uint8_t*>(part + 3 * SS_NW * SW_ROWS);  // [32][132] codes
+  float* gs_s = reinterpret_cast<float*>(codes8 + SW_ROWS * SW_CLD);          // [32][4] s of the block's groups
+  float* gz_s = gs_s + SW_ROWS * 4;                                           // [32][4] zero-point in the rounding
 
   auto stage_block = [&](int i1) {
     for (int idx = tid; idx < SW_B * (SW_B / 4); idx += SS_THREADS) {
@@ -173,6 +181,10 @@ __global__ void __launch_bounds__(SS_THREADS, 1) sweep_slab_kernel(SweepArgs a, 
       // inside the rounding the zero-point enters only for asymmetric codes
       float zs = a.sym ? 0.0f : z;
       float rs = __frcp_rn(s);
+      if (GSUB == 0) {
+        gs_s[rl * 4] = s;
+        gz_s[rl * 4] = zs;
+      }
       float* wrow = Ws + rl * WLD + bo;
       float ep[SW_CH];  // the previous chunk's errors
 #pragma unroll
@@ -224,6 +236,8 @@ __global__ void __launch_bounds__(SS_THREADS, 1) sweep_slab_kernel(SweepArgs a, 
           group_scale_zero(wmin, wmax, amax, qp, a.sym, s, z);
           zs = a.sym ? 0.0f : z;
           rs = __frcp_rn(s);
+          gs_s[rl * 4 + (k * SW_CH) / (GSUB > 0 ? GSUB : SW_B)] = s;
+          gz_s[rl * 4 + (k * SW_CH) / (GSUB > 0 ? GSUB : SW_B)] = zs;
           if (valid) {
             const int gi = (i1 + k * SW_CH) / a.g;
             a.scales[static_cast<size_t>(row0 + rl) * a.G + gi] = s;
@@ -343,18 +357,54 @@ __global__ void __launch_bounds__(SS_THREADS, 1) sweep_slab_kernel(SweepArgs a, 
     }
 
     __syncthreads();
-    // the block's errors (tf32 hi/lo for the tensor-core update past the super-block), row by row
-    for (int idx = tid; idx < SW_ROWS * SW_B; idx += SS_THREADS) {
-      const int rl = idx / SW_B, j = idx % SW_B;
-      if (row0 + rl >= a.m) continue;
-      const float e = Es[rl * SW_ELD + j];
-      const size_t eo = static_cast<size_t>(row0 + rl) * a.ld_err + a.err_col0 + bo + j;
-      if (a.Err_lo) {
-        const float hi = tf32_round(e);
-        a.Err[eo] = hi;
-        a.Err_lo[eo] = tf32_round(e - hi);
-      } else {
-        a.Err[eo] = e;
+    // the block's columns for the tensor-core update past the super-block (tf32 hi/lo), row by
+    // row: d = w0 - q from the codes and the group parameters (the walker's dequantization), eight
+    // columns an item, or the scaled errors
+    if (s1 < n && a.d_form) {
+      for (int it = tid; it < SW_ROWS * (SW_B / 8); it += SS_THREADS) {
+        const int rl = it / (SW_B / 8), j0 = (it % (SW_B / 8)) * 8;
+        if (row0 + rl >= a.m) continue;
+        const size_t row = static_cast<size_t>(row0 + rl);
+        const int slot = GSUB > 0 ? j0 / (GSUB > 0 ? GSUB : SW_B) : 0;
+        const float sc = gs_s[rl * 4 + slot], zc = gz_s[rl * 4 + slot];
+        const uint4 wv = __ldg(reinterpret_cast<const uint4*>(a.W0 + row * n + i1 + j0));
+        const uint32_t cw[2] = {*reinterpret_cast<const uint32_t*>(codes8 + rl * SW_CLD + j0),
+                                *reinterpret_cast<const uint32_t*>(codes8 + rl * SW_CLD + j0 + 4)};
+        const uint32_t hw[4] = {wv.x, wv.y, wv.z, wv.w};
+        float hi[8], lo[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          __half2 h2;
+          *reinterpret_cast<uint32_t*>(&h2) = hw[t >> 1];
+          const float w0 = (t & 1) ? __high2float(h2) : __low2float(h2);
+          const float q = static_cast<float>((cw[t >> 2] >> (8 * (t & 3))) & 0xffu) + qp.lo;
+          const float d = __fsub_rn(w0, __fmul_rn(__fsub_rn(q, zc), sc));
+          hi[t] = a.Err_lo ? tf32_round(d) : d;
+          lo[t] = tf32_round(d - hi[t]);
+        }
+        const size_t eo = row * a.ld_err + a.err_col0 + bo + j0;
+        float4* eh = reinterpret_cast<float4*>(a.Err + eo);
+        eh[0] = make_float4(hi[0], hi[1], hi[2], hi[3]);
+        eh[1] = make_float4(hi[4], hi[5], hi[6], hi[7]);
+        if (a.Err_lo) {
+          float4* el = reinterpret_cast<float4*>(a.Err_lo + eo);
+          el[0] = make_float4(lo[0], lo[1], lo[2], lo[3]);
+          el[1] = make_float4(lo[4], lo[5], lo[6], lo[7]);
+        }
+      }
+    } else if (s1 < n) {
+      for (int idx = tid; idx < SW_ROWS * SW_B; idx += SS_THREADS) {
+        const int rl = idx / SW_B, j = idx % SW_B;
+        if (row0 + rl >= a.m) continue;
+        const float e = Es[rl * SW_ELD + j];
+        const size_t eo = static_cast<size_t>(row0 + rl) * a.ld_err + a.err_col0 + bo + j;
+        if (a.Err_lo) {
+          const float hi = tf32_round(e);
+          a.Err[eo] = hi;
+          a.Err_lo[eo] = tf32_round(e - hi);
+        } else {
+          a.Err[eo] = e;
+        }
       }
     }
     // pack each row's 128 codes into its LSB-first bit stream: one 32-bit word per thread

@@ -26,6 +26,7 @@
 // division and round-half-to-even, the precision the pages' own sketches use.
 #pragma once
 
+#include <cuda_fp16.h>
 #include <cstdint>
 
 #include "factor_kernels.cuh"
@@ -55,7 +56,10 @@ struct SweepArgs {
   float* Wq;          // [m x n] fp32 working weights, sweep order
   const float* U;     // [n x n] upper factor (fp32, or the tf32 hi part when U_lo is set)
   const float* U_lo;  // [n x n] tf32 lo part of U, or nullptr
-  float* Err;         // scaled errors (fp32, or hi part): block columns at Err[r * ld_err + err_col0 ..]
+  const __half* W0;   // [m x n] original weights in sweep order, dead columns 0 (slab kernel, d_form)
+  int d_form;         // slab kernel: 1 = hand out W0 - Q for the product past the slab, 0 = the errors
+  float* Err;         // scaled errors, or W0 - Q (slab kernel, d_form), fp32 or the hi part:
+                      // block columns at Err[r * ld_err + err_col0 ..]
   float* Err_lo;      // tf32 lo part of the errors (same layout), or nullptr
   int ld_err, err_col0;
   uint32_t* codes;    // [m x n*bits/32]

@@ -111,6 +111,37 @@ def test_gemm_triangular_k_ranges(tile):
     assert (np.abs(got - R) / scale).max() <= 2e-6
 
 
+@pytest.mark.parametrize("kblk,tile", [(128, 64), (128, 128), (256, 128), (256, 256), (512, 256), (1024, 0)])
+def test_gemm_block_diagonal_k_ranges(kblk, tile):
+    """k_lo_mode 3 + log2(kblk / 128): K over the output column's aligned kblk block only, cut at
+    the tile's last column (B block-diagonal with upper-triangular blocks): the rows above each
+    block equal the fp64 product with that masked B, in the plain and the transposed output."""
+    r = np.random.default_rng(kblk + tile)
+    n = 1536
+    A = r.standard_normal((n, n)).astype(np.float32)
+    B = r.standard_normal((n, n)).astype(np.float32)
+    col = np.arange(n)[:, None]
+    k = np.arange(n)[None, :]
+    Bm = np.where((k // kblk == col // kblk) & (k <= col), B, np.float32(0))
+    mode = 3 + int(np.log2(kblk // 128))
+    out = run_gemm(A, Bm, klo=mode, khi=1, upper=1, plain=True, trans=True, tile=tile)
+    R, scale = ref(A, Bm, 1.0, 0, None)
+    rows_above = np.arange(n)[:, None] < (np.arange(n)[None, :] // kblk) * kblk
+    for key in ("C", "Ct"):
+        got = out[key].T if key == "Ct" else out[key]
+        err = np.abs(got - R) / (scale + 1e-30)
+        assert err[rows_above].max() <= 2e-6, (key, err[rows_above].max())
+
+
+def test_gemm_block_diagonal_rejects_wide_tiles():
+    A = np.ones((256, 256), np.float32)
+    Ah, Al = dev(A), dev(np.zeros_like(A))
+    st = G.lib().gptq_test_gemm_tf32x3(256, 256, 256, p(Ah), p(Al), 256, p(Ah), p(Al), 256, 1.0, 0, 3, 1, 1, p(Ah), 256,
+                                       None, None, 256, None, None, 256, 1, 256, 0, 0,
+                                       ctypes.c_void_p(torch.cuda.current_stream(DEV).cuda_stream))
+    assert st == G.ERR_ARG
+
+
 @pytest.mark.parametrize("tile", [64, 128, 256])
 def test_gemm_upper_only_updates_upper_triangle(tile):
     r = np.random.default_rng(9)

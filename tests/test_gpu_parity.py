@@ -57,8 +57,11 @@ def test_hessian_batches_strides_and_chunks():
 # S2-S4 prepare
 # ----------------------------------------------------------------------------------------
 @pytest.mark.parametrize("n,desc_act,damp", [(128, True, 0.01), (256, False, 0.1), (384, True, 0.01),
-                                             (640, False, 0.01), (640, True, 0.1), (1024, True, 0.01)])
+                                             (640, False, 0.01), (640, True, 0.1), (1024, True, 0.01),
+                                             (2304, True, 0.01), (3200, False, 0.01)])
 def test_prepare_perm_and_factor(n, desc_act, damp):
+    """Past 1024 columns the factorization leaves out the U blocks of the recursion's left edge
+    and gptq_get_factor completes them: the whole U is checked."""
     layer = synth.scaled_layer(TINY, m=64, n=n, n_tok=3000)
     X = synth.make_x_bf16(layer)
     with GPTQContext(layer.n, 64, 0) as ctx:
@@ -187,11 +190,13 @@ def test_ragged_rows_and_wider_context():
 
 
 @pytest.mark.parametrize("n,g,sym,bits", [(2048, 128, False, 4), (1152, -1, False, 4), (1536, 384, True, 3),
-                                          (2048, 256, False, 2), (1280, 64, True, 4)])
+                                          (2048, 256, False, 2), (1280, 64, True, 4), (2048, 1024, False, 4),
+                                          (4096, 2048, False, 4)])
 def test_quantize_layer_parity_across_super_blocks(n, g, sym, bits):
-    """Layers wider than one 1024-column super-block (the far columns are updated once per
-    super-block), including a partial last super-block and a group width that forces
-    per-block far updates."""
+    """Layers wider than one super-block (the far columns are updated once per super-block),
+    including a partial last super-block; groups of 256 and 1024 columns (the super-block
+    widens to hold a whole group) and groups of 384 and 2048 columns (the update past a
+    super-block taken as -E U on the completed factor, groups reaching past super-blocks)."""
     layer = synth.scaled_layer(TINY, m=80, n=n, n_tok=2 * n)
     qs = synth.QuantSetting(bits, g, sym, 0.01, True)
     gpu = GH.run_path(layer, qs)
@@ -212,3 +217,29 @@ def test_quantize_layer_parity_other_slab_widths(slab, monkeypatch):
     prep = O.prepare(gpu["H"], qs.damp, qs.desc_act)
     st, rep = GH.check_sweep_replay(gpu["W"], prep, gpu, qs)
     GH.assert_replay_ok(st, rep, gpu)
+
+
+def test_quantize_before_and_after_the_factor_is_completed():
+    """Quantizing needs only the diagonal super-blocks of U; completing U for gptq_get_factor
+    changes no output, whichever form the update past a super-block takes."""
+    layer = synth.scaled_layer(TINY, m=72, n=2304, n_tok=4608)
+    X, W = synth.make_x_bf16(layer), synth.make_w_fp16(layer)
+    Wd = torch.from_numpy(W).to(GH.DEV)
+    for qs in (synth.QuantSetting(4, 128, False, 0.01, True), synth.QuantSetting(3, 384, True, 0.01, True)):
+        with GPTQContext(layer.n, layer.m, 0) as ctx:
+            ctx.accumulate_hessian(GH.bf16_to_dev(X))
+            H, _ = ctx.get_hessian()
+            ctx.prepare(qs.damp, qs.desc_act)
+            a = ctx.quantize_layer(Wd, qs.bits, qs.group_size, qs.sym)
+            a = {k: v.clone() for k, v in a.items() if v is not None}
+            U = ctx.get_factor().cpu().numpy().astype(np.float64)
+            b = ctx.quantize_layer(Wd, qs.bits, qs.group_size, qs.sym)
+            ctx.synchronize()
+        for k in a:
+            assert torch.equal(a[k], b[k]), k
+        prep = O.prepare(H.cpu().numpy().astype(np.float64), qs.damp, qs.desc_act)
+        assert np.abs(U - prep["U"]).max() / np.abs(prep["U"]).max() <= 2e-5
+        gpu = {"codes": O.unpack_codes(a["codes"].cpu().numpy().view(np.uint32), layer.n, qs.bits),
+               "scales": a["scales"].cpu().numpy(), "zeros": a["zeros"].cpu().numpy()}
+        st, rep = GH.check_sweep_replay(W, prep, gpu, qs)
+        GH.assert_replay_ok(st, rep, gpu)
