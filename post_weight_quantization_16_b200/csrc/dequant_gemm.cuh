@@ -275,14 +275,42 @@ __global__ void __launch_bounds__(DQ_THREADS, MINB)
         ok = false;
         break;
       }
-      // this half row's 2 * BITS code words
+      // this half row's 2 * BITS code words.  A warp reads 16 rows: with 16-byte loads the
+      // first chunk each thread takes is rotated by its row so that the warp's 32 loads fall
+      // on distinct bank groups (4-bit: 2 chunks, rotated by row / 2; 8-bit: 4, by row)
       const uint8_t* cw = smem + (st_base - sbase) + s * stage_bytes + r * (16 * BITS) + h * (8 * BITS);
       uint32_t w[2 * BITS];
+      if (BITS == 2) {
+        const uint4 v = *reinterpret_cast<const uint4*>(cw);
+        w[0] = v.x;
+        w[1] = v.y;
+        w[2] = v.z;
+        w[3] = v.w;
+      } else if (BITS == 4 || BITS == 8) {
+        constexpr int NCH = BITS / 2;  // 16-byte chunks in the half row
+        const int rot = (BITS == 4) ? ((r >> 1) & 1) : (r & 3);
+        uint4 v[NCH];
 #pragma unroll
-      for (int q = 0; q < BITS; ++q) {
-        const uint2 v = *reinterpret_cast<const uint2*>(cw + 8 * q);
-        w[2 * q] = v.x;
-        w[2 * q + 1] = v.y;
+        for (int q = 0; q < NCH; ++q) v[q] = *reinterpret_cast<const uint4*>(cw + 16 * ((q + rot) & (NCH - 1)));
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+          // chunk c was loaded as v[(c - rot) mod NCH] (compile-time indices per rotation)
+          const uint4 x = (rot == 0) ? v[c]
+                        : (rot == 1) ? v[(c + NCH - 1) & (NCH - 1)]
+                        : (rot == 2) ? v[(c + NCH - 2) & (NCH - 1)]
+                                     : v[(c + NCH - 3) & (NCH - 1)];
+          w[4 * c] = x.x;
+          w[4 * c + 1] = x.y;
+          w[4 * c + 2] = x.z;
+          w[4 * c + 3] = x.w;
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < BITS; ++q) {
+          const uint2 v = *reinterpret_cast<const uint2*>(cw + 8 * q);
+          w[2 * q] = v.x;
+          w[2 * q + 1] = v.y;
+        }
       }
       const uint32_t dst_row = a_base + j * DQ_A_BYTES + h * DQ_A_ATOM + (r >> 3) * 1024 + r7 * 128;
       dq_half_row<BITS>(w, s0, zm0, s1, zm1, g32 ? 1 : 0, dst_row, r7);

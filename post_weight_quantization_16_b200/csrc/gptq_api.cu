@@ -942,7 +942,7 @@ gptq_status gptq_prepare(gptq_ctx* c, double damp, int desc_act, int32_t* perm_o
   CKL("diag_stats");
   tag(c, "prepare:perm", 0.0, 8.0 * n);
   if (desc_act)
-    CK(launch(c, rank_perm_kernel, dim3((n + 255) / 256), dim3(256), 0, c->keys, n, c->perm));
+    CK(launch(c, rank_perm_kernel, dim3((n + 7) / 8), dim3(256), 0, c->keys, n, c->perm));
   else
     CK(launch(c, identity_perm_kernel, dim3((n + 255) / 256), dim3(256), 0, n, c->perm));
   CKL("perm");

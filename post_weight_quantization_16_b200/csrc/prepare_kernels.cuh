@@ -65,25 +65,29 @@ __global__ void diag_stats_kernel(const float* __restrict__ H, int n, float* __r
   }
 }
 
-// perm[rank(i)] = i with rank(i) = #{j : key_j > key_i or (key_j == key_i and j < i)}.
-__global__ void rank_perm_kernel(const float* __restrict__ keys, int n, int32_t* __restrict__ perm) {
+// perm[rank(i)] = i with rank(i) = #{j : key_j > key_i or (key_j == key_i and j < i)}.  One warp
+// per element: the lanes count over the keys four at a time (float4, n % 128 == 0), then a warp
+// sum.  Grid: ceil(n / 8) CTAs of 256 threads.
+__global__ void __launch_bounds__(256) rank_perm_kernel(const float* __restrict__ keys, int n,
+                                                        int32_t* __restrict__ perm) {
   griddep_wait();
   griddep_launch_dependents();
-  __shared__ float ks[1024];
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  const float ki = (i < n) ? keys[i] : 0.0f;
+  const int i = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (i >= n) return;
+  const float ki = keys[i];
   int rank = 0;
-  for (int j0 = 0; j0 < n; j0 += 1024) {
-    __syncthreads();
-    for (int t = threadIdx.x; t < 1024; t += blockDim.x) ks[t] = (j0 + t < n) ? keys[j0 + t] : 0.0f;
-    __syncthreads();
-    const int jn = min(1024, n - j0);
-    for (int t = 0; t < jn; ++t) {
-      const float kj = ks[t];
-      rank += (kj > ki) || (kj == ki && j0 + t < i);
-    }
+  const float4* k4 = reinterpret_cast<const float4*>(keys);
+  for (int q = lane; q < n / 4; q += 32) {
+    const float4 v = __ldg(k4 + q);
+    const int j = 4 * q;
+    rank += (v.x > ki) || (v.x == ki && j < i);
+    rank += (v.y > ki) || (v.y == ki && j + 1 < i);
+    rank += (v.z > ki) || (v.z == ki && j + 2 < i);
+    rank += (v.w > ki) || (v.w == ki && j + 3 < i);
   }
-  if (i < n) perm[rank] = i;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) rank += __shfl_xor_sync(0xffffffffu, rank, o);
+  if (lane == 0) perm[rank] = i;
 }
 
 __global__ void identity_perm_kernel(int n, int32_t* __restrict__ perm) {

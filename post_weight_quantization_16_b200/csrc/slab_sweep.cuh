@@ -153,6 +153,18 @@ __global__ void __launch_bounds__(SS_THREADS, 1) sweep_slab_kernel(SweepArgs a, 
     }
     __syncthreads();
 
+    // the block-end hand-out's original weights (two items of eight columns per thread), loaded
+    // now so that their latency hides behind the walk
+    uint4 w0pre[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+    if (a.d_form && s1 < n) {
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int it = tid + r * SS_THREADS, rl = it / (SW_B / 8), j0 = (it % (SW_B / 8)) * 8;
+        if (row0 + rl < a.m)
+          w0pre[r] = __ldg(reinterpret_cast<const uint4*>(a.W0 + static_cast<size_t>(row0 + rl) * n + i1 + j0));
+      }
+    }
+
     if (warp == 0) {
       // ================= walker: lane = row =================
       const int rl = lane;
@@ -291,9 +303,22 @@ __global__ void __launch_bounds__(SS_THREADS, 1) sweep_slab_kernel(SweepArgs a, 
     } else {
       // ================= updaters: warps 1 .. 7, lane = row =================
       const int uw = warp - 1;  // 0 .. 6
+      // the slab pass's geometry (fixed within the block) and this lane's first item
+      constexpr int RCH = 8;
+      const int cb = bo + SW_B;
+      const int nq = slab_rest ? (S - cb) / 4 : 0;
+      const int first = uw * 32 + lane;
+      const bool have_first = first < (SW_ROWS / RCH) * nq;
 #pragma unroll 1
       for (int k = 0; k < SW_NCH; ++k) {
         if (!(k + 2 < SW_NCH || slab_rest)) continue;
+        // the first item's 16 U values do not depend on the walker: load them before waiting
+        float4 u[SW_CH];
+        if (have_first) {
+          const float* ub = a.U + static_cast<size_t>(i1 + k * SW_CH) * n + s0 + cb + 4 * (first % nq);
+#pragma unroll
+          for (int t = 0; t < SW_CH; ++t) u[t] = __ldg(reinterpret_cast<const float4*>(ub + static_cast<size_t>(t) * n));
+        }
         ss_sync(1 + (k & 1));
         // (1) the block's chunks k+2 .. 7, from the staged U block
         if (k + 2 < SW_NCH) {
@@ -318,19 +343,17 @@ __global__ void __launch_bounds__(SS_THREADS, 1) sweep_slab_kernel(SweepArgs a, 
         // (rows i1 + 16 k .. + 15, coalesced loads across the warp) in registers and walks the
         // 32 rows, the chunk's errors read as shared-memory broadcasts
         if (slab_rest) {
-          const int cb = bo + SW_B;
-          const int nq = (S - cb) / 4;
           const float* ub = a.U + static_cast<size_t>(i1 + k * SW_CH) * n + s0 + cb;
           const float4* ek = reinterpret_cast<const float4*>(Ek + (k & 1) * SW_ROWS * SW_CH);
           // items (row chunk of 8 rows, column quad), quads fastest: every updater lane has work
           // however narrow the rest of the slab, and a quad's U values are reused from L1
-          constexpr int RCH = 8;
-          for (int item = uw * 32 + lane; item < (SW_ROWS / RCH) * nq; item += (SS_NW - 1) * 32) {
+          for (int item = first; item < (SW_ROWS / RCH) * nq; item += (SS_NW - 1) * 32) {
             const int q = item % nq, r0 = (item / nq) * RCH;
-            float4 u[SW_CH];
+            if (item != first) {
 #pragma unroll
-            for (int t = 0; t < SW_CH; ++t)
-              u[t] = __ldg(reinterpret_cast<const float4*>(ub + static_cast<size_t>(t) * n + 4 * q));
+              for (int t = 0; t < SW_CH; ++t)
+                u[t] = __ldg(reinterpret_cast<const float4*>(ub + static_cast<size_t>(t) * n + 4 * q));
+            }
 #pragma unroll 2
             for (int r = r0; r < r0 + RCH; ++r) {
               float* wp = Ws + r * WLD + cb + 4 * q;
@@ -361,13 +384,16 @@ __global__ void __launch_bounds__(SS_THREADS, 1) sweep_slab_kernel(SweepArgs a, 
     // row: d = w0 - q from the codes and the group parameters (the walker's dequantization), eight
     // columns an item, or the scaled errors
     if (s1 < n && a.d_form) {
-      for (int it = tid; it < SW_ROWS * (SW_B / 8); it += SS_THREADS) {
+      static_assert(SW_ROWS * (SW_B / 8) == 2 * SS_THREADS, "two hand-out items per thread");
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int it = tid + r * SS_THREADS;
         const int rl = it / (SW_B / 8), j0 = (it % (SW_B / 8)) * 8;
         if (row0 + rl >= a.m) continue;
         const size_t row = static_cast<size_t>(row0 + rl);
         const int slot = GSUB > 0 ? j0 / (GSUB > 0 ? GSUB : SW_B) : 0;
         const float sc = gs_s[rl * 4 + slot], zc = gz_s[rl * 4 + slot];
-        const uint4 wv = __ldg(reinterpret_cast<const uint4*>(a.W0 + row * n + i1 + j0));
+        const uint4 wv = w0pre[r];
         const uint32_t cw[2] = {*reinterpret_cast<const uint32_t*>(codes8 + rl * SW_CLD + j0),
                                 *reinterpret_cast<const uint32_t*>(codes8 + rl * SW_CLD + j0 + 4)};
         const uint32_t hw[4] = {wv.x, wv.y, wv.z, wv.w};
