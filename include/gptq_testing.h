@@ -26,7 +26,8 @@ extern "C" {
  *   Ct_hi/Ct_lo: transposed hi/lo output [N x M] (ldt) or NULL (beta applies to C and C_hi/C_lo).
  *   chunk_stages: 32-wide K stages summed in one tensor-memory accumulator before the fp32
  *               register add (1 = every stage; the trailing update of the sweep uses 4).
- *   tile_n    : output tile width 64, 128 or 256, or 0 for the library's own choice.
+ *   tile_n    : output tile width 64, 128 or 256, 512 for the CTA-pair kernel (256 x 256 tiles on
+ *               two CTAs), or 0 for the library's own choice.
  *   c_reduce  : 1 = C += alpha A B^T through TMA reduce-add boxes (needs C and beta = 1; C's
  *               base 16-byte aligned, ldc % 4 == 0), the path of the sweep's trailing update.
  * Requirements: N % 32 == 0, K % 32 == 0, 16-byte aligned bases, leading dimensions % 4 == 0.

@@ -313,6 +313,8 @@ cudaError_t set_gemm_tc_attributes() {
     e = cudaFuncSetAttribute(gemm_tf32x3_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, GtCfg<128>::SMEM);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(gemm_tf32x3_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, GtCfg<64>::SMEM);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(gemm_tf32x3_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GP_SMEM);
   return e;
 }
 
@@ -360,7 +362,9 @@ gptq_status gemm_tc(gptq_ctx* c, int M, int N, int K, TcOperand A, TcOperand B, 
   if (M <= 0 || N <= 0) return GPTQ_OK;
   if (N % 32 || K % GT_BK) return GPTQ_ERR_ARG;
   if (klo > GT_KLO_BLK_LAST || (klo >= GT_KLO_BLK && force_bn > gt_kblk(klo))) return GPTQ_ERR_ARG;
-  const int bn = force_bn ? force_bn : pick_bn(M, N, K, klo, khi, upper, c->num_sms);
+  // force_bn 512: the CTA-pair kernel (256 x 256 tiles), for tests
+  if (force_bn == 2 * GP_BN && klo >= GT_KLO_BLK) return GPTQ_ERR_ARG;
+  const int bn = force_bn == 2 * GP_BN ? GP_BN : (force_bn ? force_bn : pick_bn(M, N, K, klo, khi, upper, c->num_sms));
   const int tc_tiles = gt_num_tiles(M, N, upper, bn);
   if (gt_num_tiles(M, N, upper, 64) < kMinTcTiles && A.phi && B.phi) {
     GemmSimtArgs g;
@@ -427,7 +431,20 @@ gptq_status gemm_tc(gptq_ctx* c, int M, int N, int K, TcOperand A, TcOperand B, 
   const CUtensorMap& cm = o.c_map ? *o.c_map : *A.hi;  // unused unless c_reduce
   const dim3 grid(std::min(tc_tiles, c->num_sms));
   tag(c, kGemmTcNames[c->gemm_role], gemm_algo_flops(M, N, K, klo, khi, upper), 0.0);
-  if (bn == 256)
+  // Dense products (full K range on every tile) with wide tiles and work for at least two waves
+  // of SM pairs run on CTA pairs (256 x 256 tiles, each CTA loading half of B: a third fewer L2
+  // bytes per flop).  Measured on the 8192 x 28672 layer: the updates past a slab 27.5 ms against
+  // 32.8 ms; the factorization's triangular products gained nothing, so they stay on single CTAs.
+  // GPTQ_GEMM_PAIR=0 turns pairs off.
+  const int pair_tiles = gt_num_tiles(M, N, upper, GP_BN, GP_BM);
+  const bool dense = klo == GT_KLO_NONE && khi == GT_KHI_NONE && !upper;
+  const bool pair = bn == GP_BN && klo < GT_KLO_BLK &&
+                    (force_bn == 2 * GP_BN ||
+                     (force_bn == 0 && dense && pair_tiles >= c->num_sms && env_int("GPTQ_GEMM_PAIR", 1) != 0));
+  if (pair) {
+    const dim3 pgrid(2 * std::min(pair_tiles, c->num_sms / 2));
+    CK(launch(c, gemm_tf32x3_pair_kernel, pgrid, dim3(GT_THREADS), GP_SMEM, *A.hi, *A.lo, *B.hi, *B.lo, cm, a));
+  } else if (bn == 256)
     CK(launch(c, gemm_tf32x3_kernel<256>, grid, dim3(GT_THREADS), GtCfg<256>::SMEM, *A.hi, *A.lo, *B.hi, *B.lo, cm, a));
   else if (bn == 128)
     CK(launch(c, gemm_tf32x3_kernel<128>, grid, dim3(GT_THREADS), GtCfg<128>::SMEM, *A.hi, *A.lo, *B.hi, *B.lo, cm, a));
@@ -1176,7 +1193,7 @@ gptq_status gptq_test_gemm_tf32x3(int M, int N, int K, const float* A_hi, const 
                                   void* cuda_stream) {
   if (chunk_stages < 1) return GPTQ_ERR_ARG;
   if (c_reduce && (!C || beta != 1)) return GPTQ_ERR_ARG;
-  if (tile_n != 0 && tile_n != 64 && tile_n != 128 && tile_n != 256) return GPTQ_ERR_ARG;
+  if (tile_n != 0 && tile_n != 64 && tile_n != 128 && tile_n != 256 && tile_n != 512) return GPTQ_ERR_ARG;
   if (!A_hi || !A_lo || !B_hi || !B_lo || M < 1 || N < 1 || K < GT_BK) return GPTQ_ERR_ARG;
   if (k_lo_mode < 0 || k_lo_mode > GT_KLO_BLK_LAST || k_hi_mode < 0 || k_hi_mode > 1 || (beta != 0 && beta != 1)) return GPTQ_ERR_ARG;
   if ((C_hi == nullptr) != (C_lo == nullptr) || (Ct_hi == nullptr) != (Ct_lo == nullptr)) return GPTQ_ERR_ARG;

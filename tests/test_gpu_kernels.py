@@ -73,7 +73,7 @@ def ref(A, B, alpha, beta, C0):
 @pytest.mark.parametrize("M,N,K,chunk", [(128, 256, 32, 1), (200, 320, 96, 1), (64, 64, 128, 4), (384, 512, 2048, 1),
                                          (4096, 768, 128, 4), (300, 1024, 256, 2)])
 @pytest.mark.parametrize("beta", [0, 1])
-@pytest.mark.parametrize("tile", [0, 64, 128, 256])
+@pytest.mark.parametrize("tile", [0, 64, 128, 256, 512])
 def test_gemm_outputs_match_fp64(M, N, K, chunk, beta, tile):
     r = np.random.default_rng(M + N + K + beta)
     A = r.standard_normal((M, K)).astype(np.float32)
@@ -88,7 +88,7 @@ def test_gemm_outputs_match_fp64(M, N, K, chunk, beta, tile):
         assert err.max() <= 2e-6, (k, err.max())
 
 
-@pytest.mark.parametrize("tile", [64, 128, 256])
+@pytest.mark.parametrize("tile", [64, 128, 256, 512])
 def test_gemm_triangular_k_ranges(tile):
     r = np.random.default_rng(7)
     n = 512
@@ -142,7 +142,7 @@ def test_gemm_block_diagonal_rejects_wide_tiles():
     assert st == G.ERR_ARG
 
 
-@pytest.mark.parametrize("tile", [64, 128, 256])
+@pytest.mark.parametrize("tile", [64, 128, 256, 512])
 def test_gemm_upper_only_updates_upper_triangle(tile):
     r = np.random.default_rng(9)
     n, K = 640, 128
@@ -156,7 +156,7 @@ def test_gemm_upper_only_updates_upper_triangle(tile):
 
 
 @pytest.mark.parametrize("M,N,K,chunk", [(4096, 896, 128, 4), (300, 320, 1024, 4), (128, 64, 32, 1), (1000, 3072, 256, 4)])
-@pytest.mark.parametrize("tile", [64, 128, 256])
+@pytest.mark.parametrize("tile", [64, 128, 256, 512])
 def test_gemm_reduce_add_epilogue(M, N, K, chunk, tile):
     """C += alpha A B^T through TMA reduce-add boxes: equals the fp64 result, and C's columns
     right of the product (inside the same allocation) are untouched."""
