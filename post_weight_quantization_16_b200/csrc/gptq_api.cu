@@ -84,6 +84,7 @@ struct gptq_ctx {
   cudaGraphExec_t factor_graph = nullptr;  // the factorization recursion, recorded once
   int64_t factor_graph_launches = 0;
   int gemm_role = 0;                      // which product gemm_tc runs (instrumentation): GR_*
+  int factor_chunk = 4;                   // K stages per TMEM accumulator in the factorization's products
   PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
   // per-kernel instrumentation (gptq_set_profiling): the role and algorithmic work of the next
   // launch, and one record (two timing events) per launch while profiling is on
@@ -471,7 +472,7 @@ gptq_status t_product(gptq_ctx* c, int o, int o2, int h1, int h2) {
   tt.ldt = n;
   c->gemm_role = GR_T;
   return gemm_tc(c, h1, h2, h2, fop(c->mA_VT, c->VT_hi, c->VT_lo, n, o, o2), fop(c->mB_Ut, c->Ut_hi, c->Ut_lo, n, o2, o2),
-                 1.f, 0, GT_KLO_NONE, GT_KHI_COL, 0, tt);
+                 1.f, 0, GT_KLO_NONE, GT_KHI_COL, 0, tt, c->factor_chunk);
 }
 
 // U12 = -U11 T  (and Ut21 = U12^T)      (U11 rows as A; k >= row)
@@ -488,7 +489,7 @@ gptq_status u12_product(gptq_ctx* c, int o, int o2, int h1, int h2) {
   u12.ldt = n;
   c->gemm_role = GR_U12;
   return gemm_tc(c, h1, h2, h1, fop(c->mA_U, c->U_hi, c->U_lo, n, o, o), fop(c->mB_VT, c->VT_hi, c->VT_lo, n, o2, o),
-                 -1.f, 0, GT_KLO_ROW, GT_KHI_NONE, 0, u12);
+                 -1.f, 0, GT_KLO_ROW, GT_KHI_NONE, 0, u12, c->factor_chunk);
 }
 
 // Width of the left part of a node of h columns: half the leaves; on the recursion's left edge
@@ -549,7 +550,7 @@ gptq_status chol_inv(gptq_ctx* c, int o, int h, bool need_u) {
   v12.ldh = n;
   c->gemm_role = GR_V12;
   if ((s = gemm_tc(c, h1, h2, h2, fop(c->mA_A, c->A_hi, c->A_lo, n, o, o2), fop(c->mB_U, c->U_hi, c->U_lo, n, o2, o2),
-                   1.f, 0, GT_KLO_COL, GT_KHI_NONE, 0, v12)) != GPTQ_OK)
+                   1.f, 0, GT_KLO_COL, GT_KHI_NONE, 0, v12, c->factor_chunk)) != GPTQ_OK)
     return s;
   // A11 -= V12 V12^T                     (upper tiles only)
   TcOut a11;
@@ -558,7 +559,7 @@ gptq_status chol_inv(gptq_ctx* c, int o, int h, bool need_u) {
   a11.ldh = n;
   c->gemm_role = GR_SYRK;
   if ((s = gemm_tc(c, h1, h1, h2, fop(c->mA_VT, c->VT_hi, c->VT_lo, n, o, o2), fop(c->mB_VT, c->VT_hi, c->VT_lo, n, o, o2),
-                   -1.f, 1, GT_KLO_NONE, GT_KHI_NONE, 1, a11)) != GPTQ_OK)
+                   -1.f, 1, GT_KLO_NONE, GT_KHI_NONE, 1, a11, c->factor_chunk)) != GPTQ_OK)
     return s;
   if (!need_u) return chol_inv(c, o, h1, false);
   // T is needed only by U12 below, so while the graph is being captured it runs on a second
@@ -810,6 +811,11 @@ gptq_status gptq_create(gptq_ctx** out, int64_t n, int64_t m_max, int device, vo
   c->n = n;
   c->m_max = m_max;
   c->chunk_tokens = 512;
+  // K stages (32 wide) summed in tensor memory before each round-to-nearest register add, in the
+  // factorization's products: 4 (as the updates past a slab), measured on B200: the factor's
+  // max-abs relative error against float64 1.1e-6 at n = 3200 (6.6e-7 with 1 stage), the 70B
+  // layer's factorization products 20 % faster; GPTQ_FACTOR_CHUNK (1, 2 or 4) for tuning
+  c->factor_chunk = static_cast<int>(std::min<int64_t>(4, std::max<int64_t>(1, env_int("GPTQ_FACTOR_CHUNK", 4))));
   c->encode = get_encode();
   cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, device);
   const size_t nn = static_cast<size_t>(n) * n;
