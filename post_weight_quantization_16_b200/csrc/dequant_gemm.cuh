@@ -38,27 +38,36 @@ constexpr int DQ_BK = 128;                       // K per stage (two 64-column s
 constexpr int DQ_THREADS = 64 + 256;             // producer, MMA, 8 dequant/epilogue warps
 constexpr int DQ_A_ATOM = DQ_BM * 64 * 2;        // 16 KB: 128 rows x 64 fp16
 constexpr int DQ_A_BYTES = 2 * DQ_A_ATOM;        // 32 KB per dequantized tile
-constexpr int DQ_NA = 2;                         // dequantized tiles in flight
+constexpr int DQ_NA_MAX = 4;                     // dequantized tiles in flight: 2, or 4 (decode tiles)
 constexpr int DQ_SMEM_BUDGET = 224 * 1024;       // one CTA per SM
 constexpr int DQ_SMEM_BUDGET2 = 113 * 1024;      // two CTAs per SM (each also costs the SM 1 KB)
 
-// Few tokens (decode-sized T): the dequantization, not the MMA, sets the pace, so two CTAs share
-// an SM (16 dequantizing warps) with fewer stages each; 8-bit codes keep one (their registers).
-__host__ __device__ inline int dq_minb(int tn, int bits) { return (tn <= 32 && bits != 8) ? 2 : 1; }
+// Launch shape of a tile width and code width: CTAs per SM (minb) and dequantized tiles in flight
+// (na).  Few tokens (decode-sized T): the dequantization and the round trip through the MMA set
+// the pace, not the MMA's work.  Shape 2 (default there): two CTAs per SM (16 dequantizing warps)
+// with two tiles each; shape 4: one CTA with four tiles in flight.  8-bit codes keep one CTA.
+struct DqShape {
+  int minb, na;
+};
+__host__ __device__ inline DqShape dq_shape(int tn, int bits, int decode_shape) {
+  if (tn <= 32 && decode_shape == 4) return DqShape{1, 4};
+  if (tn <= 32 && bits != 8) return DqShape{2, 2};
+  return DqShape{1, 2};
+}
 __host__ __device__ inline int dq_code_bytes(int bits) { return DQ_BM * DQ_BK * bits / 8; }
 __host__ __device__ inline int dq_x_atom_bytes(int tn) { return tn * 128; }
 __host__ __device__ inline int dq_stage_bytes(int tn, int bits) {
   const int c = (dq_code_bytes(bits) + 1023) / 1024 * 1024;
   return c + 2 * dq_x_atom_bytes(tn);
 }
-__host__ __device__ inline int dq_stages(int tn, int bits) {
-  const int budget = dq_minb(tn, bits) == 2 ? DQ_SMEM_BUDGET2 : DQ_SMEM_BUDGET;
-  const int avail = budget - 1024 - 256 - DQ_NA * DQ_A_BYTES;
+__host__ __device__ inline int dq_stages(int tn, int bits, int minb, int na) {
+  const int budget = minb == 2 ? DQ_SMEM_BUDGET2 : DQ_SMEM_BUDGET;
+  const int avail = budget - 1024 - 256 - na * DQ_A_BYTES;
   int s = avail / dq_stage_bytes(tn, bits);
   return s < 2 ? 2 : (s > 8 ? 8 : s);
 }
-__host__ __device__ inline int dq_smem_bytes(int tn, int bits) {
-  return 1024 + DQ_NA * DQ_A_BYTES + dq_stages(tn, bits) * dq_stage_bytes(tn, bits) + 256;
+__host__ __device__ inline int dq_smem_bytes(int tn, int bits, int minb, int na) {
+  return 1024 + na * DQ_A_BYTES + dq_stages(tn, bits, minb, na) * dq_stage_bytes(tn, bits) + 256;
 }
 __host__ __device__ inline int dq_tmem_cols(int tn) { return tn <= 32 ? 32 : tn; }
 
@@ -124,7 +133,7 @@ __device__ __forceinline__ void dq_half_row(const uint32_t* w, float s0, float z
   }
 }
 
-template <int BITS, int MINB>
+template <int BITS, int MINB, int NA>
 __global__ void __launch_bounds__(DQ_THREADS, MINB)
     dequant_gemm_kernel(const __grid_constant__ CUtensorMap codes_map, const __grid_constant__ CUtensorMap x_map,
                         DqArgs p) {
@@ -133,16 +142,16 @@ __global__ void __launch_bounds__(DQ_THREADS, MINB)
   uint8_t* smem = dq_smem_raw + (((raw_s + 1023u) & ~1023u) - raw_s);
   const uint32_t sbase = smem_u32(smem);
   const int tn = p.tn;
-  const int stages = dq_stages(tn, BITS);
+  const int stages = dq_stages(tn, BITS, MINB, NA);
   const int stage_bytes = dq_stage_bytes(tn, BITS);
   const int code_bytes = dq_code_bytes(BITS);
   const int code_pad = (code_bytes + 1023) / 1024 * 1024;
-  const uint32_t a_base = sbase;                                    // DQ_NA dequantized tiles
-  const uint32_t st_base = sbase + DQ_NA * DQ_A_BYTES;              // stages: codes | X atom 0 | X atom 1
+  const uint32_t a_base = sbase;                                    // NA dequantized tiles
+  const uint32_t st_base = sbase + NA * DQ_A_BYTES;                 // stages: codes | X atom 0 | X atom 1
   const uint32_t bar = st_base + stages * stage_bytes;
-  const uint32_t bar_full = bar, bar_empty = bar + 8 * 8, bar_afull = bar + 16 * 8, bar_aempty = bar + 18 * 8,
-                 bar_acc = bar + 20 * 8, bar_drain = bar + 21 * 8;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + (bar - sbase) + 22 * 8);
+  const uint32_t bar_full = bar, bar_empty = bar + 8 * 8, bar_afull = bar + 16 * 8, bar_aempty = bar_afull + 8 * NA,
+                 bar_acc = bar_aempty + 8 * NA, bar_drain = bar_acc + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + (bar_drain + 8 - sbase));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -158,7 +167,7 @@ __global__ void __launch_bounds__(DQ_THREADS, MINB)
       mbar_init(bar_full + 8 * s, 1);
       mbar_init(bar_empty + 8 * s, 1);
     }
-    for (int j = 0; j < DQ_NA; ++j) {
+    for (int j = 0; j < NA; ++j) {
       mbar_init(bar_afull + 8 * j, 256);
       mbar_init(bar_aempty + 8 * j, 1);
     }
@@ -208,9 +217,9 @@ __global__ void __launch_bounds__(DQ_THREADS, MINB)
       const uint32_t idesc = idesc_make(0u, 0u, 0u, 0u, DQ_BM, static_cast<uint32_t>(tn));  // f16 x f16, K-major
       bool ok = true;
       for (int i = 0; i < nk && ok; ++i) {
-        const int s = i % stages, j = i % DQ_NA;
+        const int s = i % stages, j = i % NA;
         if (!mbar_wait_bounded(bar_full + 8 * s, static_cast<uint32_t>(i / stages) & 1u, abort_flag) ||
-            !mbar_wait_bounded(bar_afull + 8 * j, static_cast<uint32_t>(i / DQ_NA) & 1u, abort_flag)) {
+            !mbar_wait_bounded(bar_afull + 8 * j, static_cast<uint32_t>(i / NA) & 1u, abort_flag)) {
           ok = false;
           break;
         }
@@ -263,11 +272,11 @@ __global__ void __launch_bounds__(DQ_THREADS, MINB)
     for (int i = 0; i < nk; ++i) {
       const float s0 = ns0, zm0 = nz0, s1 = ns1, zm1 = nz1;
       if (i + 1 < nk) load_sz(kt0 + i + 1, ns0, nz0, ns1, nz1);
-      const int s = i % stages, j = i % DQ_NA;
+      const int s = i % stages, j = i % NA;
       int okw = 1;
       if (lane == 0)
         okw = (mbar_wait_bounded(bar_full + 8 * s, static_cast<uint32_t>(i / stages) & 1u, abort_flag) &&
-               mbar_wait_bounded(bar_aempty + 8 * j, (static_cast<uint32_t>(i / DQ_NA) & 1u) ^ 1u, abort_flag))
+               mbar_wait_bounded(bar_aempty + 8 * j, (static_cast<uint32_t>(i / NA) & 1u) ^ 1u, abort_flag))
                    ? 1
                    : 0;
       okw = __shfl_sync(0xffffffffu, okw, 0);

@@ -1480,7 +1480,7 @@ bool dq_plan(int64_t T, int64_t m, int64_t n, int act_order, DqPlan* p) {
   p->tiles_t = static_cast<int>((T + p->tn - 1) / p->tn);
   p->k_tiles = static_cast<int>(n / DQ_BK);
   const int64_t base = static_cast<int64_t>(p->tiles_m) * p->tiles_t;
-  // fill every SM (two CTAs each when the tile is decode-sized, see dq_minb) with K splits
+  // fill every SM (two CTAs each when the tile is decode-sized, see dq_shape) with K splits
   const int64_t target = kDqPlanSms * (p->tn <= 32 ? 2 : 1);
   int splits = base >= target ? 1 : static_cast<int>(std::min<int64_t>(p->k_tiles, target / base));
   splits = std::max(1, splits);
@@ -1499,7 +1499,7 @@ bool dq_plan(int64_t T, int64_t m, int64_t n, int act_order, DqPlan* p) {
 // Raise a kernel's dynamic shared-memory limit once per device (later calls, which may be
 // recorded into a graph, then make no attribute call).
 std::mutex g_attr_mu;
-int g_attr_smem[kMaxDevicesAttr][12] = {};
+int g_attr_smem[kMaxDevicesAttr][16] = {};
 
 template <typename K>
 cudaError_t ensure_smem_attr(int device, int slot, K kernel, int smem) {
@@ -1587,42 +1587,31 @@ extern "C" gptq_status gptq_dequant_matmul(const void* X, int64_t T, const uint3
   a.scales = scales;
   a.zeros = zeros;
   a.status = status;
-  const int smem = dq_smem_bytes(pl.tn, bits);
+  // decode-sized tiles: two CTAs per SM with two dequantized tiles each, or (GPTQ_DQ_DECODE=4)
+  // one CTA with four
+  const DqShape sh = dq_shape(pl.tn, bits, static_cast<int>(env_int("GPTQ_DQ_DECODE", 2)));
+  const int smem = dq_smem_bytes(pl.tn, bits, sh.minb, sh.na);
   const dim3 grid(pl.tiles_m, pl.tiles_t, pl.splits);
-  const bool two = dq_minb(pl.tn, bits) == 2;
-  switch (bits) {
-    case 2:
-      if (two) {
-        CK(ensure_smem_attr(device, 0, dequant_gemm_kernel<2, 2>, smem));
-        dequant_gemm_kernel<2, 2><<<grid, DQ_THREADS, smem, st>>>(cmap, xmap, a);
-      } else {
-        CK(ensure_smem_attr(device, 8, dequant_gemm_kernel<2, 1>, smem));
-        dequant_gemm_kernel<2, 1><<<grid, DQ_THREADS, smem, st>>>(cmap, xmap, a);
-      }
-      break;
-    case 3:
-      if (two) {
-        CK(ensure_smem_attr(device, 1, dequant_gemm_kernel<3, 2>, smem));
-        dequant_gemm_kernel<3, 2><<<grid, DQ_THREADS, smem, st>>>(cmap, xmap, a);
-      } else {
-        CK(ensure_smem_attr(device, 9, dequant_gemm_kernel<3, 1>, smem));
-        dequant_gemm_kernel<3, 1><<<grid, DQ_THREADS, smem, st>>>(cmap, xmap, a);
-      }
-      break;
-    case 4:
-      if (two) {
-        CK(ensure_smem_attr(device, 2, dequant_gemm_kernel<4, 2>, smem));
-        dequant_gemm_kernel<4, 2><<<grid, DQ_THREADS, smem, st>>>(cmap, xmap, a);
-      } else {
-        CK(ensure_smem_attr(device, 10, dequant_gemm_kernel<4, 1>, smem));
-        dequant_gemm_kernel<4, 1><<<grid, DQ_THREADS, smem, st>>>(cmap, xmap, a);
-      }
-      break;
-    default:
-      CK(ensure_smem_attr(device, 3, dequant_gemm_kernel<8, 1>, smem));
-      dequant_gemm_kernel<8, 1><<<grid, DQ_THREADS, smem, st>>>(cmap, xmap, a);
-      break;
+#define GPTQ_DQ_LAUNCH(B, M, N, SLOT)                                                      \
+  do {                                                                                    \
+    CK(ensure_smem_attr(device, SLOT, dequant_gemm_kernel<B, M, N>, smem));               \
+    dequant_gemm_kernel<B, M, N><<<grid, DQ_THREADS, smem, st>>>(cmap, xmap, a);          \
+  } while (0)
+  const int shape = sh.minb == 2 ? 0 : (sh.na == 4 ? 1 : 2);
+  switch (bits * 4 + shape) {
+    case 2 * 4 + 0: GPTQ_DQ_LAUNCH(2, 2, 2, 0); break;
+    case 2 * 4 + 1: GPTQ_DQ_LAUNCH(2, 1, 4, 1); break;
+    case 2 * 4 + 2: GPTQ_DQ_LAUNCH(2, 1, 2, 2); break;
+    case 3 * 4 + 0: GPTQ_DQ_LAUNCH(3, 2, 2, 3); break;
+    case 3 * 4 + 1: GPTQ_DQ_LAUNCH(3, 1, 4, 5); break;
+    case 3 * 4 + 2: GPTQ_DQ_LAUNCH(3, 1, 2, 6); break;
+    case 4 * 4 + 0: GPTQ_DQ_LAUNCH(4, 2, 2, 7); break;
+    case 4 * 4 + 1: GPTQ_DQ_LAUNCH(4, 1, 4, 8); break;
+    case 4 * 4 + 2: GPTQ_DQ_LAUNCH(4, 1, 2, 9); break;
+    case 8 * 4 + 1: GPTQ_DQ_LAUNCH(8, 1, 4, 10); break;
+    default: GPTQ_DQ_LAUNCH(8, 1, 2, 11); break;
   }
+#undef GPTQ_DQ_LAUNCH
   CKL("dequant_gemm");
   if (pl.splits > 1) {
     splitk_reduce_kernel<<<592, 256, 0, st>>>(a.out, pl.splits, static_cast<size_t>(T) * m, Y);
