@@ -101,7 +101,9 @@ gptq_status gptq_set_hessian(gptq_ctx* ctx, const float* H_in, int64_t n_tok);
 
 /* S2-S4 (synchronizes once): dead-column fix, optional act-order permutation, damping by
  * damp * mean(diag H) (0 <= damp <= 1e6), then U = upper-Cholesky(H_perm^-1) by a blocked
- * reverse Cholesky H_perm = V V^T and U = V^-1.
+ * reverse Cholesky H_perm = V V^T and U = V^-1.  Past 1024 columns only the blocks of U the
+ * sweep reads are formed here (V whole, U inside every aligned 1024-column diagonal block and
+ * inside the recursion's right parts); gptq_get_factor forms the rest when asked.
  *   desc_act : 0 = identity order; 1 = stable descending diag H (after the dead fix).
  *   perm_out : device int32 [n] or NULL; perm_out[k] = original column swept at position k.
  * Returns GPTQ_ERR_NOT_PD when a pivot is not positive (the context stays unprepared).
@@ -109,7 +111,10 @@ gptq_status gptq_set_hessian(gptq_ctx* ctx, const float* H_in, int64_t n_tok);
 gptq_status gptq_prepare(gptq_ctx* ctx, double damp, int desc_act, int32_t* perm_out);
 
 /* Copy the factor U (fp32 [n x n], sweep order, zeros below the diagonal) to the device
- * buffer U_out.  GPTQ_ERR_STATE before gptq_prepare.  Asynchronous. */
+ * buffer U_out.  The first call after a gptq_prepare of a layer wider than 1024 columns first
+ * launches the products that complete U (up to about 40 % of the factorization's work);
+ * later results of gptq_quantize_layer do not change.  GPTQ_ERR_STATE before gptq_prepare.
+ * Asynchronous. */
 gptq_status gptq_get_factor(gptq_ctx* ctx, float* U_out);
 
 /* Copy the dead-column mask of the last gptq_prepare to the device buffer dead_out
@@ -129,6 +134,10 @@ gptq_status gptq_get_dead_columns(gptq_ctx* ctx, uint8_t* dead_out);
  *   zeros_out  : device fp32 [m x G], integer-valued.
  *   g_idx_out  : device int32 [n] or NULL; g_idx[perm[k]] = k / group_size.
  *   W_hat_out  : device fp32 [m x n] or NULL; dequantized weights in ORIGINAL column order.
+ * The columns past each slab of the sweep receive the slab's contribution as (W0 - Q) Vs
+ * with Vs = V blockdiag(U_SS), which the first call after gptq_prepare forms (one product);
+ * group widths that do not fit a power-of-two slab of at most 1024 columns use -E U on the
+ * completed factor instead (the same arithmetic in exact numbers).
  * GPTQ_ERR_STATE before gptq_prepare. */
 gptq_status gptq_quantize_layer(gptq_ctx* ctx, const void* W_fp16, int64_t m, gptq_qparams qp,
                                 uint32_t* codes_out, float* scales_out, float* zeros_out,
