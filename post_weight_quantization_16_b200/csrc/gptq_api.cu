@@ -432,16 +432,18 @@ gptq_status gemm_tc(gptq_ctx* c, int M, int N, int K, TcOperand A, TcOperand B, 
   const CUtensorMap& cm = o.c_map ? *o.c_map : *A.hi;  // unused unless c_reduce
   const dim3 grid(std::min(tc_tiles, c->num_sms));
   tag(c, kGemmTcNames[c->gemm_role], gemm_algo_flops(M, N, K, klo, khi, upper), 0.0);
-  // Dense products (full K range on every tile) with wide tiles and work for at least two waves
-  // of SM pairs run on CTA pairs (256 x 256 tiles, each CTA loading half of B: a third fewer L2
-  // bytes per flop).  Measured on the 8192 x 28672 layer: the updates past a slab 27.5 ms against
-  // 32.8 ms; the factorization's triangular products gained nothing, so they stay on single CTAs.
-  // GPTQ_GEMM_PAIR=0 turns pairs off.
+  // Products with wide tiles and work for at least two waves of SM pairs run on CTA pairs
+  // (256 x 256 tiles, each CTA loading half of B: a third fewer L2 bytes per flop).  Measured on
+  // the 8192 x 28672 layer (same box, alternating runs): the updates past a slab 27.5 ms against
+  // 32.8 ms; with four K stages per TMEM chunk the factorization's V12 18.9 ms against 25.6 ms and
+  // its SYRK 19.7 ms against 22.6 ms.  GPTQ_GEMM_PAIR: 0 off, 1 dense products only, 2 (default)
+  // every eligible product.
   const int pair_tiles = gt_num_tiles(M, N, upper, GP_BN, GP_BM);
   const bool dense = klo == GT_KLO_NONE && khi == GT_KHI_NONE && !upper;
+  const int64_t pair_mode = env_int("GPTQ_GEMM_PAIR", 2);
   const bool pair = bn == GP_BN && klo < GT_KLO_BLK &&
                     (force_bn == 2 * GP_BN ||
-                     (force_bn == 0 && dense && pair_tiles >= c->num_sms && env_int("GPTQ_GEMM_PAIR", 1) != 0));
+                     (force_bn == 0 && pair_tiles >= c->num_sms && (pair_mode == 2 || (pair_mode == 1 && dense))));
   if (pair) {
     const dim3 pgrid(2 * std::min(pair_tiles, c->num_sms / 2));
     CK(launch(c, gemm_tf32x3_pair_kernel, pgrid, dim3(GT_THREADS), GP_SMEM, *A.hi, *A.lo, *B.hi, *B.lo, cm, a));
