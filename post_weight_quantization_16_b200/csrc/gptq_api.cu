@@ -69,7 +69,7 @@ struct gptq_ctx {
   int mirrored = 0;           // H's lower triangle has been filled
   bool u_complete = false;    // U holds every block (the factorization leaves the blocks no step needs)
   int vs_width = 0;           // slab width S of the Vs held in A (0: none since the last prepare)
-  int64_t chunk_tokens = 512;
+  int64_t chunk_tokens = 1024;
   int64_t launches = 0;       // kernels launched by this context (instrumentation)
   int num_sms = 148;
   // tensor maps of whole matrices, encoded once: A-operand maps (128-row boxes) and
@@ -812,7 +812,10 @@ gptq_status gptq_create(gptq_ctx** out, int64_t n, int64_t m_max, int device, vo
   c->stream = static_cast<cudaStream_t>(stream);
   c->n = n;
   c->m_max = m_max;
-  c->chunk_tokens = 512;
+  // tokens summed in tensor memory per round-to-nearest register add of the Hessian: measured on
+  // B200 (4096 features, 65536 tokens) 1024 runs 4 % faster than 512 with the diagonal's max
+  // relative error 2.3e-6 (512: 1.6e-6; 2048: 5.6e-6, the tensor-core sum truncates)
+  c->chunk_tokens = 1024;
   // K stages (32 wide) summed in tensor memory before each round-to-nearest register add, in the
   // factorization's products: 4 (as the updates past a slab), measured on B200: the factor's
   // max-abs relative error against float64 1.1e-6 at n = 3200 (6.6e-7 with 1 stage), the 70B
