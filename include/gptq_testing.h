@@ -65,6 +65,15 @@ gptq_status gptq_test_bounded_wait(gptq_ctx* ctx, uint64_t limit_ns);
  *   triangle, otherwise all of them), and every non-empty K range is aligned and within K; otherwise
  *   the number (1-8) of the first check that failed, or -1 on bad arguments. */
 int gptq_test_pick_tile_n(int M, int N, int K, int k_lo_mode, int k_hi_mode, int upper_only, int sms);
+/* gptq_test_factor_plan (host only, no GPU): the factorization recursion's nodes for a width
+ *   n (multiple of 128, up to 32768) in the order gptq_prepare visits them, as int32 triples
+ *   (offset, width, 1 when the node's whole U is formed by gptq_prepare, else 0) into
+ *   nodes_out[3 * capacity]; leaves are the 128-wide nodes.  spine_out[spine_capacity] (may be
+ *   NULL) receives the widths of the nodes at offset 0 whose U gptq_get_factor completes, in
+ *   the order it completes them; *spine_count their number.  Returns the number of nodes, or -1
+ *   on bad arguments. */
+int gptq_test_factor_plan(int64_t n, int32_t* nodes_out, int capacity, int32_t* spine_out, int spine_capacity,
+                          int* spine_count);
 int gptq_test_tile_schedule(int M, int N, int K, int k_lo_mode, int k_hi_mode, int upper_only, int tile_n, int ctas);
 
 #ifdef __cplusplus

@@ -622,6 +622,21 @@ gptq_status complete_factor(gptq_ctx* c) {
   return GPTQ_OK;
 }
 
+// The recursion's node plan, host side only, mirroring chol_inv's splits: every node as
+// (offset, width, U complete) in the order chol_inv visits them (right part, the node, left
+// part); leaves are the 128-wide nodes.  The test hook below hands it to the host tests.
+void factor_plan(int o, int h, bool need_u, std::vector<int>& out) {
+  if (h <= LF_NB) {
+    out.insert(out.end(), {o, h, 1});
+    return;
+  }
+  if (h <= kSuperBlock) need_u = true;
+  const int h1 = split_left(h, need_u), h2 = h - h1;
+  factor_plan(o + h1, h2, true, out);
+  out.insert(out.end(), {o, h, need_u ? 1 : 0});
+  factor_plan(o, h1, need_u, out);
+}
+
 // Encode the context's whole-matrix tensor maps (once, at create).
 gptq_status encode_maps(gptq_ctx* c) {
   const int64_t n = c->n;
@@ -1325,6 +1340,23 @@ int gptq_test_tile_schedule(int M, int N, int K, int k_lo_mode, int k_hi_mode, i
         if ((mt * GT_BM < (nt + 1) * tile_n) != (cell[static_cast<size_t>(mt) * ntn + nt] == 1)) return 8;
   }
   return 0;
+}
+
+int gptq_test_factor_plan(int64_t n, int32_t* nodes_out, int capacity, int32_t* spine_out, int spine_capacity,
+                          int* spine_count) {
+  if (n < LF_NB || n > kMaxN || n % LF_NB || !nodes_out || capacity < 0 || !spine_count) return -1;
+  std::vector<int> v;
+  factor_plan(0, static_cast<int>(n), false, v);
+  const int count = static_cast<int>(v.size() / 3);
+  for (int i = 0; i < count && i < capacity; ++i)
+    for (int k = 0; k < 3; ++k) nodes_out[3 * i + k] = v[3 * i + k];
+  // the nodes gptq_get_factor completes, in its order (complete_factor)
+  std::vector<int> hs;
+  for (int h = static_cast<int>(n); h > kSuperBlock; h = split_left(h, false)) hs.push_back(h);
+  *spine_count = static_cast<int>(hs.size());
+  for (int i = 0; i < static_cast<int>(hs.size()) && spine_out && i < spine_capacity; ++i)
+    spine_out[i] = hs[hs.size() - 1 - i];
+  return count;
 }
 
 gptq_status gptq_destroy(gptq_ctx* c) {

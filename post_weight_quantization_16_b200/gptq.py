@@ -96,6 +96,8 @@ _SIGS = {
                                         ctypes.POINTER(ctypes.c_float), ctypes.c_int, _P]),
     "gptq_test_pick_tile_n": (ctypes.c_int, [ctypes.c_int] * 7),
     "gptq_test_tile_schedule": (ctypes.c_int, [ctypes.c_int] * 8),
+    "gptq_test_factor_plan": (ctypes.c_int, [ctypes.c_int64, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_int,
+                                             ctypes.POINTER(ctypes.c_int)]),
 }
 
 

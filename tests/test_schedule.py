@@ -1,6 +1,7 @@
 """Host-only checks of the tensor-core GEMM's work split (include/gptq_testing.h): the tile
 schedule of the persistent CTAs covers every tile exactly once for every K-range mode, and the
 tile width choice follows the cost model's intent.  No GPU needed."""
+import ctypes
 import itertools
 
 import pytest
@@ -44,3 +45,40 @@ def test_tile_width_choice():
     for args in [(128, 128, 128, 0, 0, 0, 148), (2048, 2048, 2048, 1, 0, 0, 148), (4096, 128, 128, 0, 0, 0, 148)]:
         assert pick(*args) in (64, 128, 256)
     assert pick(0, 128, 128, 0, 0, 0, 148) == -1
+
+
+def _factor_plan(n):
+    cap = 4 * (n // 128) + 8
+    nodes = (ctypes.c_int32 * (3 * cap))()
+    spine = (ctypes.c_int32 * 64)()
+    ns = ctypes.c_int()
+    cnt = G.lib().gptq_test_factor_plan(n, nodes, cap, spine, 64, ctypes.byref(ns))
+    assert 0 < cnt <= cap
+    return [tuple(nodes[3 * i:3 * i + 3]) for i in range(cnt)], list(spine[:ns.value])
+
+
+@pytest.mark.parametrize("n", [128, 256, 896, 1024, 1152, 2048, 2304, 3200, 4096, 5120, 7168, 11008, 14336, 28672, 32768])
+def test_factor_plan_forms_every_slab_block_of_U(n):
+    """The sweep reads U inside every aligned slab of 128-1024 columns (the update past a slab
+    is D V U[slab, slab]): each such block must lie inside a node whose whole U the
+    factorization forms.  Also: the leaves tile [0, n), every node is split into two parts that
+    the plan holds, and the nodes left incomplete are exactly those gptq_get_factor completes,
+    each after its left part is complete."""
+    nodes, spine = _factor_plan(n)
+    leaves = sorted((o, h) for o, h, _ in nodes if h == 128)
+    assert [o for o, _ in leaves] == list(range(0, n, 128))
+    full = {(o, h) for o, h, u in nodes if u}
+    spans = {(o, h) for o, h, _ in nodes}
+    for o, h, _ in nodes:
+        if h > 128:  # a left part (o, h1) and a right part (o + h1, h - h1), both in the plan
+            assert any((o, h1) in spans and (o + h1, h - h1) in spans for h1 in range(128, h, 128)), (o, h)
+    for S in (128, 256, 512, 1024):
+        for a in range(0, n, S):
+            b = min(n, a + S)
+            assert any(o <= a and b <= o + h for o, h in full), (S, a, b)
+    incomplete = sorted(h for o, h, u in nodes if not u)
+    assert all(o == 0 for o, h, u in nodes if not u)  # only the left edge
+    assert sorted(spine) == incomplete and spine == sorted(spine)  # completed smallest first
+    for h in spine:  # its left part is complete by the time it is completed
+        left = max(hh for oo, hh in spans if oo == 0 and hh < h)
+        assert (0, left) in full or left in spine[:spine.index(h)]
