@@ -170,24 +170,72 @@ def qrange(bits: int, sym: bool):
     return 0, (1 << bits) - 1
 
 
-def group_params(wg, bits: int, sym: bool):
+def percentile_f32(v, p: float):
+    """The p-th percentile (0 <= p <= 100) of each row of float32 values ``v`` [m, k], by
+    linear interpolation between the two order statistics around the position (k - 1) q,
+    q = p / 100 (the default method of the page's np.percentile, [P4] §3.1).  Arithmetic in
+    float32, as numpy does it for float32 data: p rounded to float32 and divided by 100 in
+    float32, h = (k - 1) q, the weight
+    t = h - floor(h); the value a + (b - a) t for t < 1/2 and b - (b - a) (1 - t) otherwise,
+    with a, b the order statistics of ranks floor(h) and floor(h) + 1 (the latter clamped to
+    k - 1)."""
+    v = np.asarray(v, dtype=np.float32)
+    k = v.shape[1]
+    srt = np.sort(v, axis=1)
+    q = np.float32(p) / np.float32(100.0)
+    h = np.float32(k - 1) * q
+    lo = int(np.floor(h))
+    hi = min(lo + 1, k - 1)
+    t = h - np.float32(lo)
+    a, b = srt[:, lo], srt[:, hi]
+    d = b - a
+    if t < np.float32(0.5):
+        return a + d * t
+    return b - d * (np.float32(1.0) - t)
+
+
+def clip_percentiles(clip: float, sym: bool):
+    """The percentiles that bound the clipped range ([P4] §3.1 ``clip_ratio``): the 100 c-th
+    percentile of |w| for symmetric codes; the (1 - c) 50-th and the 100 - (1 - c) 50-th
+    percentiles of w for asymmetric codes.  c is the clip ratio rounded to float32 (the
+    library takes it as a float); the percentiles are formed in float64."""
+    c = float(np.float32(clip))
+    if sym:
+        return (c * 100.0,)
+    return ((1.0 - c) * 50.0, 100.0 - (1.0 - c) * 50.0)
+
+
+def group_params(wg, bits: int, sym: bool, clip: float = 1.0):
     """Scale and zero-point of each row of a group of columns ``wg`` [m, k].
 
+    The range is the group's min / max (|w| max for symmetric codes), or with clip < 1 the
+    percentiles of ``clip_percentiles`` ([P4] §3.1: a clip ratio below 1 replaces the range
+    by percentiles, so that outliers saturate instead of widening the step).
     Returns (s, z, t) in float32: s the scale, z the zero-point of the UNSIGNED code
     (2^(b-1) for symmetric), t the pre-round zero value xmin/s (asymmetric only, else
     NaN), used by the replay check.
     """
     w = np.asarray(wg, dtype=np.float64).astype(np.float32)
     m = w.shape[0]
+    clipped = float(np.float32(clip)) < 1.0
     if sym:
         qpos = np.float32((1 << (bits - 1)) - 1)
-        s = np.maximum(np.max(np.abs(w), axis=1) / qpos, np.float32(1e-8))
+        if clipped:
+            amax = percentile_f32(np.abs(w), clip_percentiles(clip, True)[0])
+        else:
+            amax = np.max(np.abs(w), axis=1)
+        s = np.maximum(amax / qpos, np.float32(1e-8))
         z = np.full(m, np.float32(1 << (bits - 1)), dtype=np.float32)
         t = np.full(m, np.nan, dtype=np.float32)
     else:
         qmax = np.float32((1 << bits) - 1)
-        xmin = np.minimum(np.min(w, axis=1), np.float32(0))
-        xmax = np.maximum(np.max(w, axis=1), np.float32(0))
+        if clipped:
+            p_lo, p_hi = clip_percentiles(clip, False)
+            wlo, whi = percentile_f32(w, p_lo), percentile_f32(w, p_hi)
+        else:
+            wlo, whi = np.min(w, axis=1), np.max(w, axis=1)
+        xmin = np.minimum(wlo, np.float32(0))
+        xmax = np.maximum(whi, np.float32(0))
         s = np.maximum((xmax - xmin) / qmax, np.float32(1e-8))
         t = xmin / s
         z = -np.rint(t)
@@ -322,8 +370,10 @@ def gptq_sweep(Wp, U, bits: int, group_size: int, sym: bool, block: int | None =
     return {"codes": codes, "scales": scales, "zeros": zeros, "what": what, "pre": pre, "err": errs}
 
 
-def rtn(W, bits: int, group_size: int, sym: bool):
-    """Round-to-nearest with the same min-max groups and no compensation ([P5] "naive" 4-bit).
+def rtn(W, bits: int, group_size: int, sym: bool, clip: float = 1.0):
+    """Round-to-nearest with the same min-max groups and no compensation ([P5] "naive" 4-bit);
+    with clip < 1 the groups' ranges are percentiles ([P4] §3.1 LinearQuantizer with
+    ``clip_ratio``; the page's per-channel granularity is group_size -1 here).
 
     Returns dict(codes, scales, zeros, what) in the column order of W.
     """
@@ -336,12 +386,23 @@ def rtn(W, bits: int, group_size: int, sym: bool):
     zeros = np.zeros((m, G), dtype=np.float32)
     what = np.zeros((m, n), dtype=np.float64)
     for k in range(G):
-        s, z, _ = group_params(W[:, k * g:(k + 1) * g], bits, sym)
+        s, z, _ = group_params(W[:, k * g:(k + 1) * g], bits, sym, clip)
         scales[:, k], zeros[:, k] = s, z
         for j in range(k * g, (k + 1) * g):
             u, _, wq = quantize_values(W[:, j], s, z, bits, sym)
             codes[:, j], what[:, j] = u, wq
     return {"codes": codes, "scales": scales, "zeros": zeros, "what": what}
+
+
+def quantization_error(W, What):
+    """The page's two error measures of a quantized tensor ([P4] §3.1 ``quantization_error``):
+    the mean squared error and the cosine similarity of W and its dequantized copy, the latter
+    with 1e-8 added to the product of the norms.  float64."""
+    W = np.asarray(W, dtype=np.float64)
+    What = np.asarray(What, dtype=np.float64)
+    mse = float(np.mean((W - What) ** 2))
+    cos = float(np.sum(W * What) / (np.sqrt(np.sum(W * W)) * np.sqrt(np.sum(What * What)) + 1e-8))
+    return mse, cos
 
 
 # ==================================================================================

@@ -645,3 +645,116 @@ def test_awq_protected_channels_get_a_finer_step(sym):
     step = np.repeat(a["scales"].astype(np.float64), 64, axis=1)
     err = np.abs(W - a["what"])
     assert np.all(err <= 0.5 * step / sc[None, :] * (1 + 1e-5) + 1e-12)
+
+
+# ----------------------------------------------------------------------------------------
+# Percentile clipping of the range ("模型量化实战…" §3.1 LinearQuantizer, clip_ratio) and the
+# page's error measures (same section, quantization_error)
+# ----------------------------------------------------------------------------------------
+def test_percentile_matches_numpy_bit_for_bit():
+    """The page takes the clipped range from np.percentile; the oracle's percentile is written
+    out from its definition and must give numpy's float32 result exactly, on ties, signed zeros
+    and the percentiles that the clip ratios produce."""
+    rng = _rng(71)
+    ps = [0.0, 0.5, 1.0, 25.0, 37.3, 50.0, 63.2, 99.0, 99.5, 100.0]
+    for c in (0.9, 0.95, 0.99, 0.999, 0.5, 0.01):
+        ps += list(O.clip_percentiles(c, True)) + list(O.clip_percentiles(c, False))
+    for k in (2, 3, 32, 128, 1000, 4096):
+        a = rng.standard_normal((40, k)).astype(np.float16).astype(np.float32)   # many ties
+        a[:, : k // 4] = np.where(rng.random((40, k // 4)) < 0.5, -0.0, 0.0)  # signed zeros
+        for p in ps:
+            assert np.array_equal(O.percentile_f32(a, p), np.percentile(a, p, axis=1)), (k, p)
+
+
+def test_percentile_closed_forms():
+    rng = _rng(72)
+    v = rng.permutation(129).astype(np.float32)[None, :]          # the values 0..128
+    for p, want in ((0.0, 0.0), (25.0, 32.0), (50.0, 64.0), (100.0, 128.0)):
+        assert O.percentile_f32(v, p)[0] == want
+    # five values: the 90th percentile sits 0.6 of the way from the 4th to the 5th
+    w = np.array([[5.0, 1.0, 4.0, 2.0, 3.0]], dtype=np.float32)
+    assert abs(float(O.percentile_f32(w, 90.0)[0]) - 4.6) <= 1e-6
+    assert O.clip_percentiles(0.99, True) == (float(np.float32(0.99)) * 100.0,)
+    lo, hi = O.clip_percentiles(0.99, False)
+    assert abs(lo - 0.5) < 1e-6 and abs(hi - 99.5) < 1e-6 and abs(lo + hi - 100.0) < 1e-12
+
+
+@pytest.mark.parametrize("sym", [False, True])
+def test_clip_ratio_one_is_the_min_max_quantizer(sym):
+    rng = _rng(73)
+    W = rng.normal(0, 0.02, (24, 256)).astype(np.float16).astype(np.float64)
+    a, b = O.rtn(W, 4, 64, sym), O.rtn(W, 4, 64, sym, clip=1.0)
+    for key in ("codes", "scales", "zeros", "what"):
+        assert np.array_equal(a[key], b[key])
+
+
+def test_clipped_symmetric_scale_ignores_the_outlier():
+    """One outlier in a group of 128: the 99th percentile of |w| interpolates between the
+    126th and 127th smallest magnitudes, so the outlier (the largest) no longer sets the
+    step, and its code saturates at the top of the range."""
+    rng = _rng(74)
+    base = rng.uniform(-1.0, 1.0, 128).astype(np.float32)
+    rows = []
+    for big in (50.0, 5000.0):
+        r = base.copy()
+        r[5] = big
+        rows.append(r)
+    W = np.stack(rows).astype(np.float64)
+    s, z, _ = O.group_params(W, 8, True, clip=0.99)
+    assert s[0] == s[1]
+    mags = np.sort(np.abs(base[np.arange(128) != 5]))
+    assert mags[-2] / 127 <= s[0] <= mags[-1] / 127 * (1 + 1e-6)
+    r = O.rtn(W, 8, -1, True, clip=0.99)
+    assert np.all(r["codes"][:, 5] == 255)                          # +127 stored as 127 + 128
+    s_mm, _, _ = O.group_params(W, 8, True)
+    assert np.all(s_mm > 10 * s)
+
+
+def test_clipped_asymmetric_range_excludes_the_tails():
+    """Groups of 1000 with clip 0.99: the 0.5th and 99.5th percentiles sit between ranks 4 and
+    5 from either end, so the four smallest and four largest values may move anywhere beyond
+    them without changing the parameters; the clipped range lies inside the min-max range and
+    narrows as the ratio falls."""
+    rng = _rng(75)
+    w = rng.normal(0.1, 1.0, 1000).astype(np.float32)
+    order = np.argsort(w)
+    w2 = w.copy()
+    w2[order[:4]] -= 100.0
+    w2[order[-4:]] += 100.0
+    W = np.stack([w, w2]).astype(np.float64)
+    s, z, _ = O.group_params(W, 4, False, clip=0.99)
+    assert s[0] == s[1] and z[0] == z[1]
+    prev = None
+    for c in (1.0, 0.999, 0.99, 0.9, 0.5):
+        s_c, _, _ = O.group_params(W[:1], 4, False, clip=c)
+        if prev is not None:
+            assert s_c[0] <= prev
+        prev = s_c[0]
+
+
+def test_clipping_lowers_the_error_of_the_bulk_on_an_outlier_layer():
+    """The page's reason for the ratio: clipping the outliers shrinks the step for every other
+    weight.  With one large weight per 128, the bulk's squared error falls well below the
+    min-max quantizer's, while the outliers' rises."""
+    rng = _rng(76)
+    W = rng.normal(0, 0.02, (64, 512))
+    W[:, ::128] = 0.5
+    W = W.astype(np.float16).astype(np.float64)
+    bulk = np.ones(W.shape, bool)
+    bulk[:, ::128] = False
+    a, b = O.rtn(W, 4, 128, True), O.rtn(W, 4, 128, True, clip=0.99)
+    e_mm, e_cl = (W - a["what"]) ** 2, (W - b["what"]) ** 2
+    assert e_cl[bulk].mean() < 0.2 * e_mm[bulk].mean()
+    assert e_cl[~bulk].mean() > e_mm[~bulk].mean()
+
+
+def test_quantization_error_closed_forms():
+    W = np.array([[1.0, 0.0], [0.0, 2.0]])
+    mse, cos = O.quantization_error(W, W)
+    assert mse == 0.0 and abs(cos - 1.0) < 1e-8
+    mse, cos = O.quantization_error(W, 2 * W)
+    assert mse == np.mean(W ** 2) and abs(cos - 1.0) < 1e-8
+    mse, cos = O.quantization_error(np.array([1.0, 0.0]), np.array([0.0, 1.0]))
+    assert mse == 1.0 and cos == 0.0
+    mse, cos = O.quantization_error(np.array([3.0, 4.0]), np.array([-3.0, -4.0]))
+    assert mse == 50.0 and abs(cos + 1.0) < 1e-9
