@@ -239,6 +239,10 @@ def run_reference(args, rank, world):
     """The reference arm: the CPU oracle, timed as it stands, on bounded samples."""
     if rank != 0:
         return
+    if args.config not in synth.WORKLOADS:
+        print(json.dumps({"impl": "reference", "unavailable": f"the oracle arm times the layer solve; {args.config} "
+                                                              "is measured on the GPU arm only"}), flush=True)
+        return
     layer, qs = synth.WORKLOADS[args.config]
     # each step a sample small enough that all warm-up and timed steps end within a few minutes
     n_steps = args.warmup + args.steps
@@ -642,13 +646,161 @@ def run_block(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+AWQ_CONFIG = "awq_q_proj_4096x4096"
+SEQ_CONFIG = "sequential_mlp_4096_11008"
+
+
+def _median_call_ms(fn, stream, dev, steps, warmup, flush):
+    """Median of `steps` single calls of fn, each bracketed by CUDA events on the launching stream
+    after `warmup` untimed calls, with L2 flushed (a 256 MB write) before every call."""
+    import torch
+    ms = []
+    for r in range(warmup + steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        if r >= warmup:
+            ms.append(e0.elapsed_time(e1))
+    return statistics.median(ms)
+
+
+def run_awq(args, rank, world, local_rank):
+    """AWQ channel scaling plus round-to-nearest on the q_proj recipe (W 4096 x 4096, 65536
+    calibration tokens of X, 0.5 GB: larger than L2), 4-bit asymmetric groups of 128; and the
+    round-to-nearest quantizer alone on the same W, with and without the clipped range (the
+    page's INT8 per-channel symmetric quantizer with clip ratio 0.99, and 4-bit groups).  Each
+    call is timed alone after an L2 flush; HBM-bound: algorithmic bytes over the call's time."""
+    import torch
+    from post_weight_quantization_16_b200 import build as B
+    from post_weight_quantization_16_b200 import gptq as G
+    B.build()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    layer0, qs = synth.WORKLOADS["q_proj_4096x4096"]
+    layer = synth.scaled_layer(layer0, n_tok=65536, name=AWQ_CONFIG)
+    peaks, _ = load_peaks()
+    X = torch.from_numpy(synth.make_x_bf16(layer).view(np.int16)).to(dev).view(torch.bfloat16)
+    W = torch.from_numpy(synth.make_w_fp16(layer)).to(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    m, n, N = layer.m, layer.n, layer.n_tok
+    res = {}
+    out = {}
+
+    def awq():
+        out["awq"] = G.awq_quantize(X, W, 2.0, qs.bits, qs.group_size, qs.sym, want_w_hat=False, stream=stream)
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    t_awq = _median_call_ms(awq, stream, dev, args.steps, args.warmup, flush)
+    G_ = n // qs.group_size
+    b_awq = 2 * N * n + 2 * m * n + m * n * qs.bits / 8 + 8 * m * G_ + 4 * n
+    scale = out["awq"]["channel_scale"]
+    for name, bits, g, sym, clip, sc in (("rtn_awq_scaled_4bit_g128_asym", 4, 128, False, 1.0, scale),
+                                         ("rtn_4bit_g128_asym_clip0.99", 4, 128, False, 0.99, None),
+                                         ("rtn_8bit_per_channel_sym_clip0.99", 8, -1, True, 0.99, None),
+                                         ("rtn_8bit_per_channel_sym", 8, -1, True, 1.0, None)):
+        t = _median_call_ms(lambda: G.rtn_quantize(W, bits, g, sym, clip, channel_scale=sc, want_w_hat=False,
+                                                   stream=stream), stream, dev, args.steps, args.warmup, flush)
+        gg = n if g == -1 else g
+        byts = 2 * m * n + m * n * bits / 8 + 8 * m * (n // gg) + (4 * n if sc is not None else 0)
+        ach = byts / (t / 1e3) / 1e9
+        res[name] = {"ms": t, "algorithmic_bytes": byts, "achieved_gbs": ach, "frac_hbm": ach / peaks["hbm_gbs"]}
+    clk = clocks.stop()
+    ach = b_awq / (t_awq / 1e3) / 1e9
+    line = {
+        "metric": "AWQ layer quant (channel scaling + round-to-nearest): Gweights/s, 1xB200",
+        "value": m * n / (t_awq / 1e3) / 1e9, "unit": "Gweights/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t_awq, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": AWQ_CONFIG + ", 65536 tokens", "m": m, "n": n, "n_tok": N, "bits": qs.bits,
+                   "group_size": qs.group_size, "sym": qs.sym, "s_protect": 2.0,
+                   "l2": "flushed before every call (256 MB write)"},
+        "roofline": {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": ach / peaks["hbm_gbs"], "algorithmic_bytes": b_awq, "traffic": None},
+        "rtn": res, "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_sequential(args, rank, world, local_rank):
+    """Sequential quantization of the 7B-shaped MLP pair (up 11008 x 4096, ReLU, down 4096 x 11008)
+    through gptq.quantize_sequential: layer 0 calibrated on 65536 tokens of the block recipe, layer
+    1 on ReLU of layer 0's product with its own quantized weights; 4-bit asymmetric groups of 128,
+    damp 0.01, act-order.  One step = the whole stack through the public call (contexts included).
+    Inputs resident before timing; the intermediate activations (1.4 GB) exceed L2."""
+    import torch
+    from post_weight_quantization_16_b200 import build as B
+    from post_weight_quantization_16_b200 import gptq as G
+    B.build()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    up, _ = synth.WORKLOADS["block7b_up_11008x4096"]
+    down, _ = synth.WORKLOADS["block7b_down_4096x11008"]
+    qs = synth.QuantSetting(4, 128, False, 0.01, True)
+    peaks, _ = load_peaks()
+    X0 = torch.from_numpy(synth.make_x_bf16(up).view(np.int16)).to(dev).view(torch.bfloat16)
+    Ws = [torch.from_numpy(synth.make_w_fp16(L)).to(dev) for L in (up, down)]
+    layers = [dict(W=W, bits=qs.bits, group_size=qs.group_size, sym=qs.sym, damp=qs.damp, desc_act=qs.desc_act)
+              for W in Ws]
+
+    def step():
+        res = G.quantize_sequential(X0, layers, act=1, stream=stream)
+        torch.cuda.synchronize(dev)
+        return res
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    N = up.n_tok
+    # lower bound: every contraction at the bf16 peak (each layer's solve, and layer 0's product)
+    peak = choose_peak(peaks, ms / 1e3 * args.steps, clk)[0]
+    t_roof = 0.0
+    flops = 0.0
+    for L in (up, down):
+        Lr = synth.scaled_layer(L, n_tok=N)
+        t_bf16, _, parts = path_rooflines(Lr, qs, peak, peaks["hbm_gbs"])
+        t_roof += t_bf16
+        flops += parts["hessian"] + parts["factorization"] + parts["trailing"]
+    f_prod = 2.0 * N * up.m * up.n
+    t_roof += f_prod / (peak * 1e12)
+    weights = sum(L.m * L.n for L in (up, down))
+    line = {
+        "metric": "Sequential quantization of an MLP pair: Gweights/s, 1xB200",
+        "value": weights / (ms / 1e3) / 1e9, "unit": "Gweights/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16->f32", "data": "synthetic",
+        "config": {"workload": SEQ_CONFIG + ": up 11008x4096 -> ReLU -> down 4096x11008, 65536 tokens",
+                   "bits": qs.bits, "group_size": qs.group_size, "sym": qs.sym, "damp": qs.damp,
+                   "desc_act": qs.desc_act, "l2": "inputs and activations larger than L2"},
+        "path_roofline": {"t_roof_ms": t_roof * 1e3, "frac": t_roof * 1e3 / ms, "peak_bf16_tflops": peak,
+                          "flops": flops + f_prod},
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--config", default=WORKLOAD, choices=sorted(synth.WORKLOADS) + ["block7b"])
+    ap.add_argument("--config", default=WORKLOAD, choices=sorted(synth.WORKLOADS) + ["block7b", AWQ_CONFIG, SEQ_CONFIG])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the separate host-buffer end-to-end measurement")
     ap.add_argument("--no-w4a16", action="store_true", help="skip the dequantizing product on the layer's output")
@@ -661,6 +813,12 @@ def main():
         return
     if args.config == "block7b":
         run_block(args, rank, world, local_rank)
+        return
+    if args.config == AWQ_CONFIG:
+        run_awq(args, rank, world, local_rank)
+        return
+    if args.config == SEQ_CONFIG:
+        run_sequential(args, rank, world, local_rank)
         return
     run_gpu(args, rank, world, local_rank)
 

@@ -262,6 +262,32 @@ gptq_status gptq_awq_quantize(const void* X_bf16, int64_t n_tok, int64_t ld_x, c
                               size_t workspace_bytes, int device, void* cuda_stream);
 
 /* ---------------------------------------------------------------------------------------
+ * Round-to-nearest with a clipped range
+ * ("模型量化实战：从 INT8 PTQ 到 GPTQ 的精度保持与推理加速全解析" §3.1, LinearQuantizer and its
+ *  clip_ratio: outliers are clipped so that the rest of the weights get a finer step.)
+ *   W'      = fp32(W) * channel_scale[c]   (channel_scale may be NULL: 1; pass the scales of
+ *             gptq_awq_quantize to clip an AWQ-scaled layer)
+ *   range   per row and group of gptq_qparams (ORIGINAL column order):
+ *             clip_ratio = 1: min and max of W' (max |W'| for sym), as gptq_awq_quantize;
+ *             clip_ratio < 1, sym:  the 100 c-th percentile of |W'|;
+ *                             asym: the (1 - c) 50-th and 100 - (1 - c) 50-th percentiles of W'
+ *             A percentile is the linear interpolation between the order statistics of ranks
+ *             floor(h) and floor(h) + 1 at h = (g - 1) q, in fp32 as numpy computes it for fp32
+ *             data: q = fp32(p) / 100, t = h - floor(h), a + (b - a) t for t < 1/2, else
+ *             b - (b - a)(1 - t).
+ *   scale, zero from the range as in gptq_quantize_layer (asym range widened to include 0,
+ *             scales floored at 1e-8); codes clip(round_half_even(W' / s + z)), so the weights
+ *             outside the range saturate; packed LSB-first per row in original column order.
+ *   W_hat   = (code - zero) * group scale / channel_scale[c]   (optional, may be NULL)
+ * W_fp16: device fp16 [m x n] (n % 128 == 0, 128 <= n <= 32768); codes_out: device uint32
+ * [m x n*bits/32]; scales_out, zeros_out: device fp32 [m x n/g]; clip_ratio in (0, 1], else
+ * GPTQ_ERR_ARG.  Every pointer is caller-owned device memory.  Asynchronous on cuda_stream;
+ * arguments checked before any launch. */
+gptq_status gptq_rtn_quantize(const void* W_fp16, int64_t m, int64_t n, gptq_qparams qp, float clip_ratio,
+                              const float* channel_scale, uint32_t* codes_out, float* scales_out, float* zeros_out,
+                              float* W_hat_out, int device, void* cuda_stream);
+
+/* ---------------------------------------------------------------------------------------
  * The packed result's consumer: Y = X W16^T
  * ("模型量化实战：从 INT8 PTQ 到 GPTQ 的精度保持与推理加速全解析" §4.3: INT4 weights are turned
  *  back into FP16 before the matrix product; the low-bit storage saves memory bandwidth.)

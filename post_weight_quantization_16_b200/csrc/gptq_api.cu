@@ -6,6 +6,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cmath>
 #include <chrono>
 #include <cstdio>
 #include <cstdlib>
@@ -1890,6 +1891,51 @@ extern "C" gptq_status gptq_quantize_layers(const gptq_layer_job* jobs, int coun
 // ==========================================================================================
 // AWQ channel scaling and round-to-nearest on the same inputs (awq_kernels.cuh)
 // ==========================================================================================
+namespace {
+// Position of the p-th percentile among k sorted values, in the fp32 steps of numpy's linear
+// method: p rounded to fp32 and divided by 100, h = (k - 1) q, the ranks floor(h) and
+// floor(h) + 1 (clamped to k - 1), the weight t = h - floor(h) and 1 - t.
+struct PctPos {
+  int lo, hi;
+  float t, omt;
+};
+PctPos pct_position(double p, int k) {
+  const float q = static_cast<float>(p) / 100.0f;
+  volatile float h = static_cast<float>(k - 1) * q;  // rounded once, before the floor
+  const float hv = h;
+  const int lo = std::max(0, std::min(static_cast<int>(std::floor(hv)), k - 1));
+  const float t = hv - static_cast<float>(lo);
+  return {lo, std::min(lo + 1, k - 1), t, 1.0f - t};
+}
+
+AwqRtnArgs rtn_args(const void* W, int m, int n, const gptq_qparams& qp, const float* channel_scale, uint32_t* codes,
+                    float* scales, float* zeros, float* W_hat) {
+  AwqRtnArgs a{};
+  a.W = static_cast<const __half*>(W);
+  a.scale = channel_scale;
+  a.m = m;
+  a.n = n;
+  a.bits = qp.bits;
+  a.sym = qp.sym;
+  a.g = (qp.group_size == -1) ? n : qp.group_size;
+  a.G = n / a.g;
+  a.codes = codes;
+  a.scales = scales;
+  a.zeros = zeros;
+  a.W_hat = W_hat;
+  a.clip = 0;
+  return a;
+}
+
+gptq_status launch_rtn(const AwqRtnArgs& a, cudaStream_t st) {
+  const size_t smem = static_cast<size_t>(a.n + 6 * a.G) * 4;  // row, scales, zeros, order statistics
+  CK(cudaFuncSetAttribute(awq_rtn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
+  awq_rtn_kernel<<<a.m, 256, smem, st>>>(a);
+  CKL("awq_rtn");
+  return GPTQ_OK;
+}
+}  // namespace
+
 extern "C" size_t gptq_awq_workspace_bytes(int64_t n) {
   if (n < 128 || n > kMaxN || n % 128) return 0;
   return 256 + static_cast<size_t>(n) * sizeof(double);
@@ -1929,24 +1975,38 @@ extern "C" gptq_status gptq_awq_quantize(const void* X, int64_t n_tok, int64_t l
   CKL("awq_median");
   awq_scale_kernel<<<(ni + 255) / 256, 256, 0, st>>>(sums, ni, n_tok, median, s_protect, channel_scale);
   CKL("awq_scale");
-  AwqRtnArgs a;
-  a.W = static_cast<const __half*>(W);
-  a.scale = channel_scale;
-  a.m = mi;
-  a.n = ni;
-  a.bits = qp.bits;
-  a.sym = qp.sym;
-  a.g = (qp.group_size == -1) ? ni : qp.group_size;
-  a.G = ni / a.g;
-  a.codes = codes;
-  a.scales = scales;
-  a.zeros = zeros;
-  a.W_hat = W_hat;
-  const size_t smem = static_cast<size_t>(ni + 2 * a.G) * 4;
-  CK(cudaFuncSetAttribute(awq_rtn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
-  awq_rtn_kernel<<<mi, 256, smem, st>>>(a);
-  CKL("awq_rtn");
-  return GPTQ_OK;
+  return launch_rtn(rtn_args(W, mi, ni, qp, channel_scale, codes, scales, zeros, W_hat), st);
+}
+
+// Round-to-nearest with an optional percentile range ("模型量化实战…" §3.1 LinearQuantizer)
+extern "C" gptq_status gptq_rtn_quantize(const void* W, int64_t m, int64_t n, gptq_qparams qp, float clip_ratio,
+                                         const float* channel_scale, uint32_t* codes, float* scales, float* zeros,
+                                         float* W_hat, int device, void* cuda_stream) {
+  if (!W || !codes || !scales || !zeros) return GPTQ_ERR_ARG;
+  if (n < 128 || n > kMaxN || n % 128 || m < 1 || m > kMaxM) return GPTQ_ERR_ARG;
+  if (!valid_qparams(qp, n) || !(clip_ratio > 0.0f && clip_ratio <= 1.0f)) return GPTQ_ERR_ARG;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) {
+    cudaGetLastError();
+    return GPTQ_ERR_CUDA;
+  }
+  DeviceGuard dg(device);
+  AwqRtnArgs a = rtn_args(W, static_cast<int>(m), static_cast<int>(n), qp, channel_scale, codes, scales, zeros, W_hat);
+  if (clip_ratio < 1.0f) {
+    const double c = clip_ratio;
+    const PctPos lo = pct_position(qp.sym ? c * 100.0 : (1.0 - c) * 50.0, a.g);
+    const PctPos hi = qp.sym ? lo : pct_position(100.0 - (1.0 - c) * 50.0, a.g);
+    a.clip = 1;
+    a.rank[0] = lo.lo;
+    a.rank[1] = lo.hi;
+    a.rank[2] = hi.lo;
+    a.rank[3] = hi.hi;
+    a.t_lo = lo.t;
+    a.omt_lo = lo.omt;
+    a.t_hi = hi.t;
+    a.omt_hi = hi.omt;
+  }
+  return launch_rtn(a, static_cast<cudaStream_t>(cuda_stream));
 }
 
 // ==========================================================================================

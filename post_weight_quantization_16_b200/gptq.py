@@ -85,6 +85,8 @@ _SIGS = {
     "gptq_awq_quantize": (ctypes.c_int, [_P, ctypes.c_int64, ctypes.c_int64, _P, ctypes.c_int64, ctypes.c_int64,
                                          ctypes.c_float, QParams, _P, _P, _P, _P, _P, _P, ctypes.c_size_t,
                                          ctypes.c_int, _P]),
+    "gptq_rtn_quantize": (ctypes.c_int, [_P, ctypes.c_int64, ctypes.c_int64, QParams, ctypes.c_float, _P, _P, _P, _P,
+                                         _P, ctypes.c_int, _P]),
     "gptq_quantize_layer_noalloc": (ctypes.c_int, [_P, ctypes.c_int64, ctypes.c_int64, _P, _P, _P, QParams,
                                                    _P, _P, _P, _P, _P, ctypes.c_int, _P]),
     "gptq_test_gemm_tf32x3": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P, ctypes.c_int, _P, _P,
@@ -393,6 +395,28 @@ def awq_quantize(X: torch.Tensor | None, W: torch.Tensor, s_protect: float = 2.0
                                    _ptr(out["scales"]), _ptr(out["zeros"]), _ptr(out["channel_scale"]),
                                    _ptr(out["w_hat"]), _ptr(ws), ws.numel(), dev.index,
                                    ctypes.c_void_p(stream.cuda_stream)), "gptq_awq_quantize")
+    return out
+
+
+def rtn_quantize(W: torch.Tensor, bits: int = 8, group_size: int = -1, sym: bool = True, clip_ratio: float = 1.0,
+                 channel_scale: torch.Tensor | None = None, want_w_hat: bool = True,
+                 stream: torch.cuda.Stream | None = None) -> dict:
+    """Round-to-nearest with a clipped range (gptq_rtn_quantize; the page's INT8 LinearQuantizer
+    is bits 8, per-channel, symmetric, clip_ratio 0.99).  W: fp16 [m, n]; channel_scale: fp32 [n]
+    or None.  Returns device tensors codes, scales, zeros and (optionally) w_hat, in original
+    column order."""
+    m, n = W.shape
+    dev = W.device
+    stream = stream if stream is not None else torch.cuda.current_stream(dev)
+    g = n if group_size == -1 else group_size
+    out = {"codes": torch.empty((m, n * bits // 32), dtype=torch.int32, device=dev),
+           "scales": torch.empty((m, n // g), dtype=torch.float32, device=dev),
+           "zeros": torch.empty((m, n // g), dtype=torch.float32, device=dev),
+           "w_hat": torch.empty((m, n), dtype=torch.float32, device=dev) if want_w_hat else None}
+    qp = QParams(int(bits), int(group_size), int(bool(sym)))
+    _check(lib().gptq_rtn_quantize(_ptr(W), m, n, qp, float(clip_ratio), _ptr(channel_scale), _ptr(out["codes"]),
+                                   _ptr(out["scales"]), _ptr(out["zeros"]), _ptr(out["w_hat"]), dev.index,
+                                   ctypes.c_void_p(stream.cuda_stream)), "gptq_rtn_quantize")
     return out
 
 

@@ -93,3 +93,17 @@ def test_dequant_matmul_workspace_is_a_pure_size_function(L):
     assert L.gptq_dequant_matmul_workspace_bytes(0, 4096, 4096, 0) == 0      # no tokens
     assert L.gptq_dequant_matmul(None, 1, None, None, None, None, 1, 128, G.QParams(4, 128, 0), None, None, 0, 0,
                                  None) == G.ERR_ARG
+
+
+def test_rtn_quantize_rejects_bad_arguments_before_any_device_call(L):
+    """Every case below is refused on the host, so no pointer is ever dereferenced."""
+    p = ctypes.c_void_p(1 << 20)
+    qp = G.QParams(8, -1, 1)
+    assert L.gptq_rtn_quantize(None, 16, 512, qp, 0.99, None, p, p, p, None, 0, None) == G.ERR_ARG
+    assert L.gptq_rtn_quantize(p, 16, 512, qp, 0.99, None, None, p, p, None, 0, None) == G.ERR_ARG
+    for clip in (0.0, -0.5, 1.5, float("nan"), float("inf")):
+        assert L.gptq_rtn_quantize(p, 16, 512, qp, clip, None, p, p, p, None, 0, None) == G.ERR_ARG, clip
+    assert L.gptq_rtn_quantize(p, 16, 500, qp, 0.99, None, p, p, p, None, 0, None) == G.ERR_ARG      # n % 128
+    assert L.gptq_rtn_quantize(p, 0, 512, qp, 0.99, None, p, p, p, None, 0, None) == G.ERR_ARG       # no rows
+    assert L.gptq_rtn_quantize(p, 16, 512, G.QParams(5, -1, 1), 0.99, None, p, p, p, None, 0, None) == G.ERR_ARG
+    assert L.gptq_rtn_quantize(p, 16, 512, G.QParams(4, 96, 0), 0.99, None, p, p, p, None, 0, None) == G.ERR_ARG
