@@ -30,23 +30,34 @@ namespace gptq {
 
 constexpr int AWQ_SUM_COLS = 256;  // columns per warp pass (8 bf16 per lane)
 
+// |x| of the 8 bf16 values in v added into acc (fp64).
+__device__ __forceinline__ void add_abs8(double* acc, const uint4& v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    acc[2 * k] += fabs(static_cast<double>(__uint_as_float(w[k] << 16)));
+    acc[2 * k + 1] += fabs(static_cast<double>(__uint_as_float(w[k] & 0xFFFF0000u)));
+  }
+}
+
 // grid (ceil(n / 256), token splits), block (32, 8): lane owns 8 consecutive columns, the 8 warps
-// and the grid's y dimension split the tokens; fp64 partial sums are added atomically.
+// and the grid's y dimension split the tokens; each thread keeps four rows' loads in flight
+// before adding them; fp64 partial sums are added atomically.
 __global__ void __launch_bounds__(256) channel_abs_sum_kernel(const __nv_bfloat16* __restrict__ X, int64_t n_tok,
                                                               int64_t ld, int n, double* __restrict__ sums) {
   const int c0 = blockIdx.x * AWQ_SUM_COLS + threadIdx.x * 8;
   if (c0 >= n) return;
   double acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   const int64_t step = static_cast<int64_t>(blockDim.y) * gridDim.y;
-  for (int64_t t = static_cast<int64_t>(blockIdx.y) * blockDim.y + threadIdx.y; t < n_tok; t += step) {
-    const uint4 v = *reinterpret_cast<const uint4*>(X + t * ld + c0);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  int64_t t = static_cast<int64_t>(blockIdx.y) * blockDim.y + threadIdx.y;
+  for (; t + 3 * step < n_tok; t += 4 * step) {
+    uint4 v[4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      acc[2 * k] += fabs(static_cast<double>(__uint_as_float(w[k] << 16)));
-      acc[2 * k + 1] += fabs(static_cast<double>(__uint_as_float(w[k] & 0xFFFF0000u)));
-    }
+    for (int u = 0; u < 4; ++u) v[u] = *reinterpret_cast<const uint4*>(X + (t + u * step) * ld + c0);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) add_abs8(acc, v[u]);
   }
+  for (; t < n_tok; t += step) add_abs8(acc, *reinterpret_cast<const uint4*>(X + t * ld + c0));
 #pragma unroll
   for (int k = 0; k < 8; ++k)
     if (acc[k] != 0.0) atomicAdd(sums + c0 + k, acc[k]);

@@ -436,8 +436,31 @@ def activation_convert(Y: torch.Tensor, act: int = 1, want_bf16: bool = True, wa
     return xb, xh
 
 
+def _sequential_context(contexts: dict | None, n: int, m: int, dev: torch.device,
+                        stream: torch.cuda.Stream) -> "GPTQContext":
+    """A context of width n for at least m rows on this stream: kept in `contexts` when given."""
+    if contexts is None:
+        return GPTQContext(n, m, dev.index, stream)
+    key = (n, dev.index, stream.cuda_stream)
+    ctx = contexts.get(key)
+    if ctx is not None and ctx.m_max < m:
+        ctx.close()
+        ctx = None
+    if ctx is None:
+        ctx = GPTQContext(n, m, dev.index, stream)
+        contexts[key] = ctx
+    return ctx
+
+
+def close_contexts(contexts: dict) -> None:
+    """Close the contexts that quantize_sequential kept in `contexts`."""
+    for ctx in contexts.values():
+        ctx.close()
+    contexts.clear()
+
+
 def quantize_sequential(X0: torch.Tensor, layers: list, act: int = 1, stream: torch.cuda.Stream | None = None,
-                        keep_hessian: bool = False) -> list:
+                        keep_hessian: bool = False, contexts: dict | None = None) -> list:
     """Sequential quantization of a stack of linear layers ("GPTQ算法原理深度解析" §2.1: the error
     of a layer reaches the next one through its input).  X0: bf16 [N, n0] calibration inputs of
     layer 0; layers: dicts with W (fp16 [m_l, n_l], n_{l+1} = m_l), bits, group_size, sym, damp,
@@ -445,7 +468,10 @@ def quantize_sequential(X0: torch.Tensor, layers: list, act: int = 1, stream: to
     layer l's quantized weights (gptq_dequant_matmul on the fp16 copy of X_l).  Every step runs in
     the library's kernels; this function only sequences the calls.  Returns, per layer, its
     outputs (codes, scales, zeros, g_idx, perm), its calibration inputs X (bf16) and X16 (the
-    fp16 copy its product reads), and with keep_hessian its H (fp32 [n, n])."""
+    fp16 copy its product reads), and with keep_hessian its H (fp32 [n, n]).  contexts: an optional
+    dict in which the contexts (one per layer width and stream) stay between calls, so that repeated
+    calls skip their creation (workspace allocation, the factorization's graph); the caller closes
+    them with close_contexts.  Without it, each layer's context is created and closed here."""
     dev = X0.device
     stream = stream if stream is not None else torch.cuda.current_stream(dev)
     xb = X0
@@ -456,12 +482,17 @@ def quantize_sequential(X0: torch.Tensor, layers: list, act: int = 1, stream: to
         m, n = W.shape
         if xb.shape[1] != n:
             raise ValueError(f"layer {li}: {n} inputs, but the previous layer gives {xb.shape[1]}")
-        with GPTQContext(n, m, dev.index, stream) as ctx:
+        ctx = _sequential_context(contexts, n, m, dev, stream)
+        try:
+            ctx.reset()
             ctx.accumulate_hessian(xb)
             H = ctx.get_hessian()[0] if keep_hessian else None
             perm = ctx.prepare(L["damp"], L["desc_act"])
             out = ctx.quantize_layer(W, L["bits"], L["group_size"], L["sym"], want_w_hat=False)
             ctx.synchronize()
+        finally:
+            if contexts is None:
+                ctx.close()
         out = dict(out, perm=perm, X=xb, X16=xh, H=H)
         res.append(out)
         if li + 1 < len(layers):

@@ -79,3 +79,30 @@ def test_three_layer_relu_stack_stage_by_stage():
             assert np.all(np.abs(nxt_b - relu) <= tol + 2.0 ** -8 * np.abs(relu) + 1e-30), li
             assert np.all(np.abs(nxt_h - relu) <= tol + 2.0 ** -11 * np.abs(relu) + 2.0 ** -24), li
             assert (nxt_b >= 0).all() and (nxt_h >= 0).all()
+
+
+def test_contexts_kept_between_calls_give_the_same_result():
+    """quantize_sequential with a contexts dict: the first call creates the width-256 context, the
+    third layer (384 rows) replaces it with a larger one, and a second call reuses it; every output
+    equals the call that creates and closes its own contexts."""
+    N = 1024
+    dims = [256, 256, 256, 384]
+    lay0 = synth.scaled_layer(synth.WORKLOADS["tiny_256x512"][0], m=dims[1], n=dims[0], n_tok=N)
+    X0 = GH.bf16_to_dev(synth.make_x_bf16(lay0))
+    rng = np.random.default_rng(12)
+    layers = [dict(W=torch.from_numpy((rng.standard_normal((dims[i + 1], dims[i])) / 16).astype(np.float16)).to(GH.DEV),
+                   bits=4, group_size=128, sym=bool(i % 2), damp=0.01, desc_act=True) for i in range(3)]
+    ref = G.quantize_sequential(X0, layers, act=1)
+    torch.cuda.synchronize(GH.DEV)
+    ctxs = {}
+    try:
+        for _ in range(2):
+            res = G.quantize_sequential(X0, layers, act=1, contexts=ctxs)
+            torch.cuda.synchronize(GH.DEV)
+            assert len(ctxs) == 1 and next(iter(ctxs.values())).m_max == 384
+            for a, b in zip(ref, res):
+                for key in ("codes", "scales", "zeros", "perm", "g_idx"):
+                    assert torch.equal(a[key], b[key]), key
+    finally:
+        G.close_contexts(ctxs)
+    assert not ctxs
