@@ -75,6 +75,11 @@ int gptq_test_pick_tile_n(int M, int N, int K, int k_lo_mode, int k_hi_mode, int
 int gptq_test_factor_plan(int64_t n, int32_t* nodes_out, int capacity, int32_t* spine_out, int spine_capacity,
                           int* spine_count);
 int gptq_test_tile_schedule(int M, int N, int K, int k_lo_mode, int k_hi_mode, int upper_only, int tile_n, int ctas);
+/* gptq_test_pct_position (host only, no GPU): where gptq_rtn_quantize takes the p-th percentile
+ *   (0 <= p <= 100) of k >= 1 sorted values: the ranks *lo and *hi of the two order statistics and
+ *   the interpolation weights *t and *omt (= 1 - t), exactly as the call passes them to its kernel.
+ *   Returns 0, or -1 on bad arguments. */
+int gptq_test_pct_position(double p, int k, int* lo, int* hi, float* t, float* omt);
 
 #ifdef __cplusplus
 }

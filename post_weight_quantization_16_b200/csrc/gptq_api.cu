@@ -2009,6 +2009,16 @@ extern "C" gptq_status gptq_rtn_quantize(const void* W, int64_t m, int64_t n, gp
   return launch_rtn(a, static_cast<cudaStream_t>(cuda_stream));
 }
 
+extern "C" int gptq_test_pct_position(double p, int k, int* lo, int* hi, float* t, float* omt) {
+  if (!(p >= 0.0 && p <= 100.0) || k < 1 || !lo || !hi || !t || !omt) return -1;
+  const PctPos q = pct_position(p, k);
+  *lo = q.lo;
+  *hi = q.hi;
+  *t = q.t;
+  *omt = q.omt;
+  return 0;
+}
+
 // ==========================================================================================
 // Sequential quantization: a layer's output, through its activation, as the next layer's inputs
 // ==========================================================================================

@@ -100,6 +100,9 @@ _SIGS = {
     "gptq_test_tile_schedule": (ctypes.c_int, [ctypes.c_int] * 8),
     "gptq_test_factor_plan": (ctypes.c_int, [ctypes.c_int64, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_int,
                                              ctypes.POINTER(ctypes.c_int)]),
+    "gptq_test_pct_position": (ctypes.c_int, [ctypes.c_double, ctypes.c_int, ctypes.POINTER(ctypes.c_int),
+                                              ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_float),
+                                              ctypes.POINTER(ctypes.c_float)]),
 }
 
 
