@@ -107,3 +107,33 @@ def test_rtn_quantize_rejects_bad_arguments_before_any_device_call(L):
     assert L.gptq_rtn_quantize(p, 0, 512, qp, 0.99, None, p, p, p, None, 0, None) == G.ERR_ARG       # no rows
     assert L.gptq_rtn_quantize(p, 16, 512, G.QParams(5, -1, 1), 0.99, None, p, p, p, None, 0, None) == G.ERR_ARG
     assert L.gptq_rtn_quantize(p, 16, 512, G.QParams(4, 96, 0), 0.99, None, p, p, p, None, 0, None) == G.ERR_ARG
+
+
+def test_sequential_keeps_one_context_per_width_and_grows_it(monkeypatch):
+    """The binding's context bookkeeping for quantize_sequential, with a stand-in context class."""
+    import types
+    made = []
+
+    class FakeContext:
+        def __init__(self, n, m_max, device, stream):
+            self.n, self.m_max, self.closed = n, m_max, False
+            made.append(self)
+
+        def close(self):
+            self.closed = True
+
+    monkeypatch.setattr(G, "GPTQContext", FakeContext)
+    dev, st = types.SimpleNamespace(index=0), types.SimpleNamespace(cuda_stream=7)
+    ctxs = {}
+    a = G._sequential_context(ctxs, 256, 100, dev, st)
+    assert G._sequential_context(ctxs, 256, 50, dev, st) is a              # fewer rows: reused
+    b = G._sequential_context(ctxs, 256, 300, dev, st)                     # more rows: replaced
+    assert b is not a and a.closed and b.m_max == 300 and not b.closed
+    c = G._sequential_context(ctxs, 512, 10, dev, st)
+    assert len(ctxs) == 2 and c.n == 512
+    other = G._sequential_context(ctxs, 256, 10, dev, types.SimpleNamespace(cuda_stream=9))
+    assert other is not b and len(ctxs) == 3                                # one per stream
+    loose = G._sequential_context(None, 256, 10, dev, st)
+    assert loose not in ctxs.values() and len(made) == 5
+    G.close_contexts(ctxs)
+    assert not ctxs and b.closed and c.closed and other.closed
