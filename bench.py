@@ -696,6 +696,9 @@ def run_awq(args, rank, world, local_rank):
     clocks = ClockSampler(local_rank)
     clocks.start()
     t_awq = _median_call_ms(awq, stream, dev, args.steps, args.warmup, flush)
+    # the same call without calibration tokens skips only the channel sums: the difference is their time
+    t_awq_no_x = _median_call_ms(lambda: G.awq_quantize(None, W, 2.0, qs.bits, qs.group_size, qs.sym, want_w_hat=False,
+                                                        stream=stream), stream, dev, args.steps, args.warmup, flush)
     G_ = n // qs.group_size
     b_awq = 2 * N * n + 2 * m * n + m * n * qs.bits / 8 + 8 * m * G_ + 4 * n
     scale = out["awq"]["channel_scale"]
@@ -722,6 +725,8 @@ def run_awq(args, rank, world, local_rank):
         "roofline": {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": ach / peaks["hbm_gbs"], "algorithmic_bytes": b_awq, "traffic": None},
         "rtn": res, "clocks": clk,
+        "split": {"ms_without_tokens": t_awq_no_x, "channel_sums_ms": t_awq - t_awq_no_x,
+                  "channel_sums_gbs": 2 * N * n / ((t_awq - t_awq_no_x) / 1e3) / 1e9 if t_awq > t_awq_no_x else None},
     }
     print(json.dumps(line), flush=True)
 
