@@ -48,7 +48,7 @@ typedef enum {
   GPTQ_ERR_OOM = 4,         /* workspace does not fit (checked before allocating) */
   GPTQ_ERR_CUDA = 5,        /* a CUDA runtime/driver call failed (no device, launch error...) */
   GPTQ_ERR_TIMEOUT = 6,     /* a bounded device or host wait ran out */
-  GPTQ_ERR_UNSUPPORTED = 7  /* valid request that this build does not implement */
+  GPTQ_ERR_UNSUPPORTED = 7  /* valid request that this library does not implement */
 } gptq_status;
 
 /* Quantizer settings ("GPTQ算法原理深度解析" §3.3 quantize_config: bits, group_size; sym from
