@@ -758,3 +758,22 @@ def test_quantization_error_closed_forms():
     assert mse == 1.0 and cos == 0.0
     mse, cos = O.quantization_error(np.array([3.0, 4.0]), np.array([-3.0, -4.0]))
     assert mse == 50.0 and abs(cos + 1.0) < 1e-9
+
+
+def test_percentile_equals_numpy_on_arbitrary_data():
+    """Property check over arbitrary finite float32 groups (extreme magnitudes, subnormals, heavy
+    ties) and percentiles: the oracle's written-out percentile is np.percentile's, bit for bit."""
+    hyp = pytest.importorskip("hypothesis")
+    st = pytest.importorskip("hypothesis.strategies")
+    from hypothesis.extra import numpy as hnp
+
+    @hyp.settings(max_examples=300, deadline=None, derandomize=True)
+    @hyp.given(hnp.arrays(np.float32, hnp.array_shapes(min_dims=2, max_dims=2, min_side=1, max_side=70),
+                          elements=st.floats(-float(np.float32(1e30)), float(np.float32(1e30)), width=32)),
+               st.floats(0.0, 100.0, allow_nan=False))
+    def check(a, p):
+        want = np.percentile(a, p, axis=1)
+        got = O.percentile_f32(a, p)
+        assert np.array_equal(got, want, equal_nan=True)
+
+    check()
